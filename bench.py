@@ -1,0 +1,425 @@
+"""Throughput of the HSTU forward stack and of M-FALCON ranking on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward pass of the 8-layer, d=1024 HSTU stack over the
+full-stack workload (128 users, Stochastic-Length-shortened lognormal
+lengths, ~36k tokens), i.e. every step of the layer path: schedule, f1 +
+SiLU, pointwise attention with relative bias, LayerNorm * U, f2 + residual.
+M-FALCON ranking (32 users, 1024 candidates each, 3 layers) is timed the same
+way and reported in the same line under "mfalcon".
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream with a 256 MB L2 flush between steps (outside the
+events); barrier + synchronize around the timed region; max over ranks.
+Under torchrun every rank runs its own replica batch (users are independent;
+no collective on the data path) and `value` sums the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HSTU fwd tokens/s & M-FALCON candidates/s at 1 B200; % of bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------- algorithmic work
+def layer_flops(dims, lengths):
+    d, h, dqk, dv = dims.d_model, dims.n_heads, dims.d_qk, dims.d_v
+    F = 2 * h * (dqk + dv)
+    n = np.asarray(lengths, np.float64)
+    T = float(n.sum())
+    pairs = float((n * (n + 1) / 2).sum())
+    return dict(f1=2.0 * T * d * F, f2=2.0 * T * h * dv * d, attn=h * (2 * dqk + 2 * dv) * pairs)
+
+
+def mfalcon_flops(dims, n_layers, hist_lens, cands):
+    d, h, dqk, dv = dims.d_model, dims.n_heads, dims.d_qk, dims.d_v
+    F = 2 * h * (dqk + dv)
+    lf = layer_flops(dims, hist_lens)
+    T = float(np.sum(hist_lens))
+    hist = (n_layers - 1) * sum(lf.values()) + T * 2 * d * h * (dqk + dv)
+    n = np.asarray(hist_lens, np.float64)
+    m = np.asarray(cands, np.float64)
+    cand = float((m * n_layers * (2 * d * F + 2 * h * dv * d + h * (2 * dqk + 2 * dv) * (n + 1))).sum()
+                 + (2 * d * m).sum())
+    return hist + cand
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- traffic from ncu
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "hstu_sequential_transducer_layer_b200", "csrc"))):
+        with open(os.path.join(ROOT, "hstu_sequential_transducer_layer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if its
+    recorded source hash matches the current kernels (else null)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+def cpu_baseline_stack(w, budget_tokens: int):
+    """Oracle on whole users of the workload (fixed seeded sample), tokens/s."""
+    from oracle import hstu_oracle as O
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    order = np.random.default_rng(123).permutation(w.B)
+    users, tok = [], 0
+    for b in order:
+        users.append(int(b))
+        tok += int(w.lengths[b])
+        if tok >= budget_tokens:
+            break
+    t0 = time.perf_counter()
+    for b in users:
+        s, e = int(w.offsets[b]), int(w.offsets[b + 1])
+        O.stack_user(w.X[s:e], w.timestamps[s:e], w.weights, w.dims)
+    dt = time.perf_counter() - t0
+    return {"value": tok / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(users)} whole users ({tok} tokens) of the {w.name} workload, "
+                      f"all {w.n_layers} layers, numpy float64",
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import hstu_workloads as hw
+    import hstu_sequential_transducer_layer_b200 as H
+    from hstu_sequential_transducer_layer_b200.build import build
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0 or world == 1:
+        build()
+    if world > 1:
+        torch.distributed.barrier()
+    peaks, peak_src = load_peaks()
+
+    # ---------------- inputs (a replica batch per rank)
+    w = hw.full_stack(seed=args.seed + rank)
+    r = H.HSTURunner(hw.dims_dict(w.dims), w.weights, dev)
+    off = r.to_device(w.offsets, "i64")
+    X = r.to_device(w.X, "act")
+    ts = r.to_device(w.timestamps, "i64")
+    out = torch.empty_like(X)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flops = layer_flops(w.dims, w.lengths)
+    T = w.T
+
+    def step():
+        r.stack(off, X, ts, w.max_len, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if r.status() != 0:
+        raise RuntimeError(f"device status {r.status()} after warm-up")
+
+    # ---------------- timed region
+    n_launch0 = H.hstu_launch_count()
+    H.hstu_trace_enable(args.steps * 8 * 6 + 64)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    n_launch = H.hstu_launch_count() - n_launch0
+    trace = H.hstu_trace_read()
+    H.hstu_trace_enable(0)
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = sum(step_ms) / len(step_ms)
+    if r.status() != 0:
+        raise RuntimeError(f"device status {r.status()} after timing")
+
+    # per-kernel device time inside the timed region
+    per_kernel = {}
+    for kid, t in trace:
+        nm = H.hstu_kernel_name(kid)
+        a = per_kernel.setdefault(nm, [0, 0.0])
+        a[0] += 1
+        a[1] += t
+    dominant = max(per_kernel.items(), key=lambda kv: kv[1][1])[0] if per_kernel else None
+    kflops = {"gemm_f1_tc": flops["f1"], "gemm_f2_tc": flops["f2"], "attn_tc": flops["attn"]}
+    roofline = None
+    if dominant in kflops:
+        n, tot = per_kernel[dominant]
+        avg_s = tot / n / 1e3
+        achieved = kflops[dominant] / avg_s / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_source": f"bf16_tflops_sustained ({peak_src})",
+                    "traffic": ncu_traffic(dominant, w.name),
+                    "avg_launch_ms": round(tot / n, 4)}
+    step_flops = args_layers = w.n_layers * sum(flops.values())
+    del args_layers
+
+    # ---------------- end to end through the public API, host buffers
+    Xh = X.cpu().pin_memory()
+    offh = off.cpu().pin_memory()
+    tsh = ts.cpu().pin_memory()
+    Yh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(max(3, args.steps // 2))]
+    Xd, offd, tsd = torch.empty_like(X), torch.empty_like(off), torch.empty_like(ts)
+    for a, b in e_evs:
+        flush.zero_()
+        a.record(stream)
+        Xd.copy_(Xh, non_blocking=True)
+        offd.copy_(offh, non_blocking=True)
+        tsd.copy_(tsh, non_blocking=True)
+        r.stack(offd, Xd, tsd, w.max_len, out=out)
+        Yh.copy_(out, non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e_evs) / len(e_evs)
+    h2d = Xh.numel() * Xh.element_size() + offh.numel() * 8 + tsh.numel() * 8
+    d2h = Yh.numel() * Yh.element_size()
+
+    # ---------------- M-FALCON
+    mf = None
+    if not args.no_mfalcon:
+        wm = hw.mfalcon(seed=args.seed + rank)
+        rm = H.HSTURunner(hw.dims_dict(wm.dims), wm.weights, dev)
+        ins = dict(ho=rm.to_device(wm.offsets, "i64"), hx=rm.to_device(wm.X),
+                   ht=rm.to_device(wm.timestamps, "i64"), co=rm.to_device(wm.cand_offsets, "i64"),
+                   cx=rm.to_device(wm.candidates), hv=rm.to_device(wm.head_vec))
+        scores = torch.empty(wm.candidates.shape[0], dtype=torch.float32, device=dev)
+
+        def mstep():
+            rm.rank(ins["ho"], ins["hx"], ins["ht"], ins["co"], ins["cx"], None, wm.microbatch,
+                    ins["hv"], wm.max_len, wm.max_cands, scores=scores)
+        for _ in range(args.warmup):
+            mstep()
+        torch.cuda.synchronize()
+        m_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for a, b in m_evs:
+            flush.zero_()
+            a.record(stream)
+            mstep()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if rm.status() != 0:
+            raise RuntimeError(f"M-FALCON device status {rm.status()}")
+        m_ms = sum(a.elapsed_time(b) for a, b in m_evs) / len(m_evs)
+        C = wm.candidates.shape[0]
+        mflop = mfalcon_flops(wm.dims, wm.n_layers, wm.lengths, np.diff(wm.cand_offsets))
+        mf = {"value": C / (m_ms / 1e3), "unit": "candidates/s", "ms_per_step": round(m_ms, 4),
+              "tflops": round(mflop / (m_ms / 1e3) / 1e12, 1),
+              "config": {"workload": "mfalcon", "users": wm.B, "candidates_per_user": wm.max_cands,
+                         "microbatch": wm.microbatch, "layers": wm.n_layers, "d_model": 512,
+                         "heads": 4, "head_dim": 128, "history_tokens": wm.T}}
+
+    # ---------------- reduce over ranks
+    tokens = float(T)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+        s = torch.tensor([tokens], dtype=torch.float64, device=dev)
+        dist.all_reduce(s, op=dist.ReduceOp.SUM)
+        tokens = float(s[0])
+        if mf is not None:
+            t = torch.tensor([mf["ms_per_step"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            mf["value"] = wm.candidates.shape[0] * world / (float(t[0]) / 1e3)
+            mf["ms_per_step"] = float(t[0])
+
+    line = None
+    if rank == 0:
+        cpu = None if (world > 1 or args.no_cpu_baseline) else cpu_baseline_stack(w, args.cpu_tokens)
+        line = {
+            "metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights)",
+            "config": {"workload": "full_stack", "layers": w.n_layers, "d_model": w.dims.d_model,
+                       "heads": w.dims.n_heads, "head_dim": w.dims.d_qk, "users_per_gpu": w.B,
+                       "tokens_per_gpu": T, "max_len": w.max_len,
+                       "l2": "256 MB flush between timed steps",
+                       "parallelism": f"replicas x{world} (users independent, no collective)"},
+            "tflops": round(step_flops / (ms / 1e3) / 1e12, 1),
+            "roofline": roofline,
+            "kernels": {k: {"launches": v[0], "ms": round(v[1], 3),
+                            "share": round(v[1] / max(1e-9, sum(x[1] for x in per_kernel.values())), 4)}
+                        for k, v in sorted(per_kernel.items(), key=lambda kv: -kv[1][1])},
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": int(n_launch),
+            "clocks": clk.summary(),
+            "mfalcon": mf,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import hstu_workloads as hw
+    w = hw.full_stack(seed=args.seed)
+    base = cpu_baseline_stack(w, 1)  # warm caches / BLAS threads
+    del base
+    vals = []
+    sample_tokens = args.ref_tokens
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline_stack(w, sample_tokens)
+        if i >= args.warmup:
+            vals.append(cb)
+    v = sum(c["value"] for c in vals) / len(vals)
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded; random-init weights)", "impl": "reference",
+            "config": {"workload": "full_stack", "sample": vals[0]["sample"]},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-mfalcon", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=4000)
+    ap.add_argument("--ref-tokens", type=int, default=600)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

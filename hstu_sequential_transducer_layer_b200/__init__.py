@@ -1,0 +1,13 @@
+"""HSTU layer stack + M-FALCON ranking on one B200 (sm_100a).
+
+The computation lives in ``libhstu.so`` (CUDA kernels behind the C ABI of
+``include/hstu.h``); ``binding`` marshals torch tensors into those calls and
+``runner`` holds device weights and workspaces for repeated calls.
+"""
+from .binding import (  # noqa: F401
+    HstuError, LayerDesc, LayerWeights, make_desc, weights_struct, weights_array,
+    weights_to_device, hstu_workspace_size, hstu_layer_fwd, hstu_stack_fwd, hstu_mfalcon_rank,
+    hstu_read_status, hstu_debug_offsets, hstu_trace_enable, hstu_trace_read, hstu_kernel_name,
+    hstu_launch_count, hstu_status_string, hstu_version, lib, LIB_PATH, EXPORTED,
+)
+from .runner import HSTURunner  # noqa: F401,E402

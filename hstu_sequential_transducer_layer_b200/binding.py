@@ -1,0 +1,237 @@
+"""ctypes binding of libhstu.so (include/hstu.h), argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes torch
+tensors (for device memory) or plain integers.  PyTorch supplies device
+memory and the current CUDA stream; every step of the computation runs in
+the library's CUDA kernels.  If libhstu.so is missing the first call raises
+``HstuError``: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhstu.so")
+
+HSTU_BF16, HSTU_FP32 = 0, 1
+STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED",
+                3: "HSTU_ERR_WORKSPACE", 4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_BAD_OFFSETS",
+                6: "HSTU_ERR_TIMEOUT", 7: "HSTU_ERR_BAD_TIMESTAMPS"}
+
+# Every symbol include/hstu.h declares.
+EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
+            "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
+            "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
+
+
+class HstuError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = int(code)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.code, self.code)}")
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("n_pos_buckets", ctypes.c_int32), ("n_time_buckets", ctypes.c_int32),
+                ("pos_sub_bits", ctypes.c_int32), ("time_sub_bits", ctypes.c_int32),
+                ("ln_eps", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
+                ("b2", ctypes.c_void_p), ("ln_gamma", ctypes.c_void_p),
+                ("ln_beta", ctypes.c_void_p), ("rab_pos", ctypes.c_void_p),
+                ("rab_time", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhstu.so (built in-tree by ``build.py``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise HstuError(4, f"libhstu.so not found at {LIB_PATH}; build it with "
+                           "`python -m hstu_sequential_transducer_layer_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i32, i64, sz, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+    pdesc = ctypes.POINTER(LayerDesc)
+    pw = ctypes.POINTER(LayerWeights)
+    L.hstu_workspace_size.argtypes = [pdesc, i32, i64, i64, i64, i64, i64, i32]
+    L.hstu_workspace_size.restype = sz
+    L.hstu_layer_fwd.argtypes = [pdesc, i64, i64, i64, vp, vp, pw, vp, vp, vp, sz, vp]
+    L.hstu_layer_fwd.restype = i32
+    L.hstu_stack_fwd.argtypes = [pdesc, i32, pw, i64, i64, i64, vp, vp, vp, vp, vp, sz, vp]
+    L.hstu_stack_fwd.restype = i32
+    L.hstu_mfalcon_rank.argtypes = [pdesc, i32, pw, i64, i64, i64, vp, vp, vp, i64, i64, vp, vp,
+                                    vp, i32, vp, vp, vp, sz, vp]
+    L.hstu_mfalcon_rank.restype = i32
+    L.hstu_read_status.argtypes = [vp, sz, vp]
+    L.hstu_read_status.restype = i32
+    L.hstu_debug_offsets.argtypes = [pdesc, i64, i64, i64, ctypes.POINTER(sz),
+                                     ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.hstu_debug_offsets.restype = i32
+    L.hstu_trace_enable.argtypes = [i32]
+    L.hstu_trace_enable.restype = i32
+    L.hstu_trace_read.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float), i32]
+    L.hstu_trace_read.restype = i32
+    L.hstu_kernel_name.argtypes = [i32]
+    L.hstu_kernel_name.restype = ctypes.c_char_p
+    L.hstu_launch_count.argtypes = []
+    L.hstu_launch_count.restype = i64
+    L.hstu_status_string.argtypes = [i32]
+    L.hstu_status_string.restype = ctypes.c_char_p
+    L.hstu_version.argtypes = []
+    L.hstu_version.restype = i32
+    _lib = L
+    return L
+
+
+# ---------------------------------------------------------------- marshalling
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _nbytes(t) -> int:
+    return int(t.numel() * t.element_size())
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise HstuError(code, where)
+
+
+def make_desc(d_model, n_heads, d_qk, d_v, n_pos_buckets, n_time_buckets, pos_sub_bits,
+              time_sub_bits, ln_eps=1e-6, dtype="bf16") -> LayerDesc:
+    dt = HSTU_BF16 if dtype in ("bf16", HSTU_BF16) else HSTU_FP32
+    return LayerDesc(d_model, n_heads, d_qk, d_v, n_pos_buckets, n_time_buckets, pos_sub_bits,
+                     time_sub_bits, float(ln_eps), dt)
+
+
+def weights_struct(w: Dict[str, object]) -> LayerWeights:
+    """LayerWeights from a dict of device tensors (W1, b1, W2, b2, ln_gamma,
+    ln_beta, rab_pos, rab_time)."""
+    return LayerWeights(*[_ptr(w[k]) for k in ("W1", "b1", "W2", "b2", "ln_gamma", "ln_beta",
+                                                "rab_pos", "rab_time")])
+
+
+def weights_array(ws: Sequence[Dict[str, object]]):
+    arr = (LayerWeights * len(ws))()
+    for i, w in enumerate(ws):
+        arr[i] = weights_struct(w)
+    return arr
+
+
+def weights_to_device(weights: Sequence[Dict[str, np.ndarray]], dtype: str, device) -> List[Dict]:
+    """Copy a list of per-layer numpy weight dicts to the device (dense
+    weights in the layer dtype, rab tables fp32)."""
+    import torch
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = []
+    for w in weights:
+        d = {}
+        for k in ("W1", "b1", "W2", "b2", "ln_gamma", "ln_beta"):
+            d[k] = torch.from_numpy(np.ascontiguousarray(w[k], np.float32)).to(device=device, dtype=tdt)
+        for k in ("rab_pos", "rab_time"):
+            d[k] = torch.from_numpy(np.ascontiguousarray(w[k], np.float32)).to(device)
+        out.append(d)
+    return out
+
+
+# ---------------------------------------------------------------- entry points
+def hstu_workspace_size(desc: LayerDesc, n_layers: int, B: int, total_tokens: int, max_len: int,
+                        total_cands: int = 0, max_cands: int = 0, microbatch: int = 0) -> int:
+    n = lib().hstu_workspace_size(ctypes.byref(desc), n_layers, B, total_tokens, max_len,
+                                  total_cands, max_cands, microbatch)
+    if n == 0:
+        raise HstuError(1, "hstu_workspace_size")
+    return int(n)
+
+
+def hstu_layer_fwd(desc, B, total_tokens, max_len, offsets, X, weights, timestamps, out,
+                   workspace, stream=None) -> None:
+    ws = weights if isinstance(weights, LayerWeights) else weights_struct(weights)
+    _check(lib().hstu_layer_fwd(ctypes.byref(desc), B, total_tokens, max_len, _ptr(offsets),
+                                _ptr(X), ctypes.byref(ws), _ptr(timestamps), _ptr(out),
+                                _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "hstu_layer_fwd")
+
+
+def hstu_stack_fwd(desc, n_layers, weights, B, total_tokens, max_len, offsets, X, timestamps,
+                   out, workspace, stream=None) -> None:
+    arr = weights if not isinstance(weights, (list, tuple)) else weights_array(weights)
+    _check(lib().hstu_stack_fwd(ctypes.byref(desc), n_layers, arr, B, total_tokens, max_len,
+                                _ptr(offsets), _ptr(X), _ptr(timestamps), _ptr(out),
+                                _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "hstu_stack_fwd")
+
+
+def hstu_mfalcon_rank(desc, n_layers, weights, B, total_hist, max_len, hist_offsets, history,
+                      hist_timestamps, total_cands, max_cands, cand_offsets, candidates,
+                      request_ts, microbatch, head_vec, scores, workspace, stream=None) -> None:
+    arr = weights if not isinstance(weights, (list, tuple)) else weights_array(weights)
+    _check(lib().hstu_mfalcon_rank(ctypes.byref(desc), n_layers, arr, B, total_hist, max_len,
+                                   _ptr(hist_offsets), _ptr(history), _ptr(hist_timestamps),
+                                   total_cands, max_cands, _ptr(cand_offsets), _ptr(candidates),
+                                   _ptr(request_ts), microbatch, _ptr(head_vec), _ptr(scores),
+                                   _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "hstu_mfalcon_rank")
+
+
+def hstu_read_status(workspace, stream=None) -> int:
+    return int(lib().hstu_read_status(_ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def hstu_debug_offsets(desc, B, total_tokens, max_len):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().hstu_debug_offsets(ctypes.byref(desc), B, total_tokens, max_len,
+                                    ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "hstu_debug_offsets")
+    return int(a.value), int(b.value), int(c.value)
+
+
+def hstu_trace_enable(max_records: int) -> None:
+    _check(lib().hstu_trace_enable(max_records), "hstu_trace_enable")
+
+
+def hstu_trace_read(capacity: int = 1 << 16):
+    ids = (ctypes.c_int32 * capacity)()
+    ms = (ctypes.c_float * capacity)()
+    n = lib().hstu_trace_read(ids, ms, capacity)
+    return [(int(ids[i]), float(ms[i])) for i in range(n)]
+
+
+def hstu_kernel_name(kernel_id: int) -> str:
+    return lib().hstu_kernel_name(kernel_id).decode()
+
+
+def hstu_launch_count() -> int:
+    return int(lib().hstu_launch_count())
+
+
+def hstu_status_string(code: int) -> str:
+    return lib().hstu_status_string(code).decode()
+
+
+def hstu_version() -> int:
+    return int(lib().hstu_version())

@@ -1,0 +1,547 @@
+// attn_tc.cu — pointwise (softmax-free) attention with the relative bias on
+// the tcgen05 tensor cores, over jagged batches.
+//
+// 'HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか',
+// subsection '2. QKᵀで「どの履歴を見るか」を決める': per head,
+//   s_ij = Q_i.K_j + pos_bias(i - j) + time_bias(t_i - t_j), j <= i,
+//   O_i  = (1/n) sum_j SiLU(s_ij) V_j          (no softmax, no running max)
+// and section '長い履歴を現実の計算量へ収める4つの工夫', subsection
+// '4. M-FALCONで候補間の履歴計算を共有する': candidates attend to their user's
+// whole cached history and to themselves only.
+//
+// One work item = (user, 128-row query tile, head).  The host-side schedule
+// lists, for each item, only the KV tiles at or left of the causal diagonal,
+// longest items first, so fully masked tiles are never loaded or multiplied.
+// Because there is no softmax, KV tiles combine by plain accumulation in TMEM.
+//
+// Roles (320 threads): warp 0 TMA producer (Q tile once per item, K/V tiles
+// through a 2-stage ring); warp 1 MMA issuer: S = Q K^T into one of two TMEM
+// buffers, then O += P V into a TMEM accumulator; warps 2-9 ("P warps", two
+// per TMEM lane quarter, each owning 64 of the 128 columns) read S with
+// tcgen05.ld, add the bias, apply SiLU, mask, round to bf16 and write P into
+// shared memory in the 128-byte-swizzled K-major layout the MMA reads.  At
+// the end of an item the P warps read O, scale by 1/n (and, for candidates,
+// add the self term) and store bf16.
+//
+// Bias evaluation per element: the position bias comes from a per-warp
+// window of the 95 distances this warp's 32 x 64 block spans (one shared
+// load); the time bias is held in a register and recomputed only when the
+// gap leaves the current bucket's range (timestamps are usually sorted, so
+// this happens a few times per row and tile).
+#include <cuda_bf16.h>
+
+#include <climits>
+
+#include "ptx.cuh"
+
+namespace hstu {
+
+struct AttnDev {
+  int mode;
+  const AttnItem* items;
+  const int32_t* n_items;
+  const int64_t* q_off;
+  const int64_t* kv_off;
+  int64_t kv_rows;
+  const int32_t* t_rel;
+  const int32_t* t_req_rel;
+  const float* rab_pos;
+  const float* rab_time;
+  int Np, Nt, Sp, St;
+  int q_col, k_col, v_col;
+  const __nv_bfloat16* q_buf;  // for the candidate self term
+  int64_t ld_f1;
+  __nv_bfloat16* O;
+  int64_t ldo;
+  int* status;
+};
+
+template <int D>
+struct AttnCfg {
+  static constexpr int NA = D / 64;                       // 64-column swizzle atoms
+  static constexpr uint32_t TILE = 128u * D * 2;          // Q, K or V tile bytes
+  static constexpr int P_BUFS = (D == 64) ? 2 : 1;
+  static constexpr uint32_t P_BYTES = 128u * 128u * 2;
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t K_OFF = Q_OFF + TILE;
+  static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
+  static constexpr uint32_t P_OFF = V_OFF + 2 * TILE;
+  static constexpr uint32_t WIN_OFF = P_OFF + P_BUFS * P_BYTES;
+  static constexpr uint32_t TJ_OFF = WIN_OFF + 8 * 96 * 4;
+  static constexpr uint32_t BAR_OFF = TJ_OFF + 8 * 64 * 4;
+  static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
+  static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O
+};
+
+enum { MODE_SELF = 0, MODE_CAND = 1 };
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(320, 1)
+    k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+              const AttnDev a) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;    // [2]
+  uint64_t* kv_empty = bars + 4;   // [2]
+  uint64_t* s_full = bars + 6;     // [2]
+  uint64_t* s_free = bars + 8;     // [2]
+  uint64_t* p_full = bars + 10;    // [2]
+  uint64_t* p_free = bars + 12;    // [2]
+  uint64_t* o_full = bars + 14;
+  uint64_t* o_free = bars + 15;
+  uint64_t* drain = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
+  int* s_go = reinterpret_cast<int*>(ab + 1);
+  int* s_nitems = s_go + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    const int st = a.status ? *reinterpret_cast<volatile int*>(a.status) : 0;
+    *s_go = (st == 0);
+    *s_nitems = *a.n_items;
+    ab->flag = 0;
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(kv_full + i, 1);
+      mbar_init(kv_empty + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(s_free + i, 8);
+      mbar_init(p_full + i, 8);
+      mbar_init(p_free + i, 1);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 8);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmKV);
+  }
+  __syncthreads();
+  if (!*s_go) return;
+  const int n_items = *s_nitems;
+
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  uint8_t* sQ = smem + C::Q_OFF;
+  uint8_t* sK = smem + C::K_OFF;
+  uint8_t* sV = smem + C::V_OFF;
+  uint8_t* sP = smem + C::P_OFF;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int kst = 0, litem = 0;
+      uint32_t kph = 0, issued = 0, last_par = 0, q_issued = 0, q_par = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++litem) {
+        const AttnItem w = a.items[it];
+        const int q_row0 = (int)(a.q_off[w.b] + (int64_t)w.qt * 128);
+        const int kv_row0 = (int)a.kv_off[w.b];
+        if (!mbar_wait(q_empty, (litem & 1) ^ 1, ab, a.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(q_full, C::TILE);
+#pragma unroll
+        for (int at = 0; at < C::NA; ++at)
+          tma_load_2d(sQ + at * 16384, &tmQ, a.q_col + w.head * D + at * 64, q_row0, q_full);
+        q_issued = 1;
+        q_par = litem & 1;
+        for (int j = 0; j < w.nkv; ++j) {
+          if (!mbar_wait(kv_empty + kst, kph ^ 1, ab, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full + kst, 2 * C::TILE);
+          const int y = kv_row0 + j * 128;
+#pragma unroll
+          for (int at = 0; at < C::NA; ++at) {
+            tma_load_2d(sK + kst * C::TILE + at * 16384, &tmKV, a.k_col + w.head * D + at * 64, y,
+                        kv_full + kst);
+            tma_load_2d(sV + kst * C::TILE + at * 16384, &tmKV, a.v_col + w.head * D + at * 64, y,
+                        kv_full + kst);
+          }
+          issued |= 1u << kst;
+          last_par = (last_par & ~(1u << kst)) | (kph << kst);
+          if (++kst == 2) {
+            kst = 0;
+            kph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        AbortState tmp{0};
+        for (int s = 0; s < 2; ++s)
+          if ((issued >> s) & 1u) mbar_wait(kv_full + s, (last_par >> s) & 1u, &tmp, nullptr);
+        if (q_issued) mbar_wait(q_full, q_par, &tmp, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);  // V is MN-major
+      int kst = 0, litem = 0;
+      uint32_t kph = 0, scount = 0, pcount = 0;
+      bool ok = true, any = false;
+      const uint32_t q_base = smem_u32(sQ);
+      auto issue_pv = [&](int jj, int st, int nkv) -> bool {
+        const int pb = (int)(pcount % C::P_BUFS);
+        const uint32_t pph = (pcount / C::P_BUFS) & 1;
+        if (!mbar_wait(p_full + pb, pph, ab, a.status)) return false;
+        if (jj == 0 && !mbar_wait(o_free, (litem & 1) ^ 1, ab, a.status)) return false;
+        tc_fence_after();
+        const uint32_t p_base = smem_u32(sP + pb * C::P_BYTES);
+        const uint32_t v_base = smem_u32(sV + st * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_bf16_ss(tmem + C::O_COL,
+                         sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                         sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
+                         (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(p_free + pb);
+        tc_commit(kv_empty + st);
+        if (jj == nkv - 1) tc_commit(o_full);
+        ++pcount;
+        any = true;
+        return true;
+      };
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++litem) {
+        const int nkv = a.items[it].nkv;
+        if (!mbar_wait(q_full, litem & 1, ab, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        int prev = -1;
+        for (int j = 0; j < nkv; ++j) {
+          if (!mbar_wait(kv_full + kst, kph, ab, a.status)) {
+            ok = false;
+            break;
+          }
+          const int sb = scount & 1;
+          if (!mbar_wait(s_free + sb, ((scount >> 1) & 1) ^ 1, ab, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sK + kst * C::TILE);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            tc_mma_bf16_ss(tmem + sb * 128,
+                           sdesc_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                           sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                           IDESC_S, kk > 0 ? 1u : 0u);
+          tc_commit(s_full + sb);
+          ++scount;
+          any = true;
+          if (j > 0 && !issue_pv(j - 1, prev, nkv)) {
+            ok = false;
+            break;
+          }
+          prev = kst;
+          if (++kst == 2) {
+            kst = 0;
+            kph ^= 1;
+          }
+        }
+        if (!ok) break;
+        if (nkv > 0) {
+          if (!issue_pv(nkv - 1, prev, nkv)) {
+            ok = false;
+            break;
+          }
+        } else {
+          tc_commit(o_full);  // nothing to accumulate: O is taken as zero
+        }
+        tc_commit(q_empty);
+      }
+      if (any) {
+        tc_commit(drain);
+        AbortState tmp{0};
+        mbar_wait(drain, 0, &tmp, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ P warps
+    const int pw = warp - 2;         // 0..7
+    const int q = warp & 3;          // TMEM lane quarter
+    const int half = pw >> 2;        // which 64 of the 128 S columns
+    const int r = q * 32 + lane;     // row inside the 128-row tile
+    float* win = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 96;
+    int* tj = reinterpret_cast<int*>(smem + C::TJ_OFF) + pw * 64;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint32_t scount = 0, pcount = 0;
+    int litem = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++litem) {
+      const AttnItem w = a.items[it];
+      const int64_t kv0 = a.kv_off[w.b];
+      const int n_kv = (int)(a.kv_off[w.b + 1] - kv0);           // history / sequence length
+      const int64_t q0 = a.q_off[w.b] + (int64_t)w.qt * 128;
+      const int n_q = (int)(a.q_off[w.b + 1] - a.q_off[w.b]);
+      const int rows_valid = min(128, n_q - w.qt * 128);
+      const bool row_ok = r < rows_valid;
+      const float inv_n = 1.0f / (float)max(n_kv, 1);
+      const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
+      const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
+      int t_i = 0;
+      if (MODE == MODE_SELF) t_i = row_ok ? a.t_rel[kv0 + (int64_t)w.qt * 128 + r] : 0;
+      else t_i = a.t_req_rel[w.b];
+      int lo = 1, hi = 0;   // empty range: the first column computes the bucket
+      float tb = 0.f;
+      bool alive = true;
+      for (int j = 0; j < w.nkv && alive; ++j) {
+        // ---- per-warp bias tables for this tile
+        __syncwarp();
+        if (MODE == MODE_SELF) {
+          const int base = (w.qt - j) * 128 + q * 32 - half * 64 - 63;
+#pragma unroll
+          for (int u = 0; u < 3; ++u) {
+            const int k = lane + 32 * u;
+            if (k < 95) {
+              const int dist = base + k;
+              win[k] = dist >= 0 ? __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int jc = j * 128 + half * 64 + lane + 32 * u;
+            tj[lane + 32 * u] = jc < n_kv ? a.t_rel[kv0 + jc] : 0;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int jc = j * 128 + half * 64 + lane + 32 * u;
+            float bias = 0.f;
+            if (jc < n_kv) {
+              const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
+              bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
+                     __ldg(Rt + log_bucket(gap, a.St, a.Nt));
+            }
+            win[lane + 32 * u] = bias;
+          }
+        }
+        __syncwarp();
+        // ---- S tile from TMEM
+        const int sb = scount & 1;
+        if (!mbar_wait_warp(s_full + sb, (scount >> 1) & 1, ab, a.status)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[64];
+        {
+          uint32_t (&lo32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+          uint32_t (&hi32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+          tmem_ld32(tmem + sb * 128 + half * 64 + lane_base, lo32);
+          tmem_ld32(tmem + sb * 128 + half * 64 + 32 + lane_base, hi32);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + sb);
+        ++scount;
+        // ---- P = SiLU(S + bias), masked, bf16
+        uint32_t pk[32];
+        if (MODE == MODE_SELF) {
+          const bool diag = (j == w.qt);
+          const float* wr = win + lane + 63;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            float x = __uint_as_float(sr[c]) + wr[-c];
+            const int gap = t_i - tj[c];
+            if (gap < lo || gap >= hi) {
+              const int b = log_bucket(max(gap, 0), a.St, a.Nt);
+              lo = b == 0 ? INT_MIN : bucket_lo(b, a.St);
+              hi = b >= a.Nt - 1 ? INT_MAX : bucket_lo(b + 1, a.St);
+              tb = __ldg(Rt + b);
+            }
+            x += tb;
+            float p = silu_fast(x);
+            if (diag && (half * 64 + c > r)) p = 0.f;
+            if (c & 1) pk[c >> 1] = pack_bf16x2(__uint_as_float(pk[c >> 1]), p);
+            else pk[c >> 1] = __float_as_uint(p);
+          }
+        } else {
+          const int limit = n_kv - j * 128 - half * 64;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            float p = silu_fast(__uint_as_float(sr[c]) + win[c]);
+            if (c >= limit) p = 0.f;
+            if (c & 1) pk[c >> 1] = pack_bf16x2(__uint_as_float(pk[c >> 1]), p);
+            else pk[c >> 1] = __float_as_uint(p);
+          }
+        }
+        // ---- write P (K-major, 128-byte swizzle: chunk m of row r at m ^ (r & 7))
+        const int pb = (int)(pcount % C::P_BUFS);
+        if (!mbar_wait_warp(p_free + pb, ((pcount / C::P_BUFS) & 1) ^ 1, ab, a.status)) {
+          alive = false;
+          break;
+        }
+        uint8_t* prow = sP + pb * C::P_BYTES + half * 16384 + r * 128;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          uint4 v;
+          v.x = pk[4 * m + 0];
+          v.y = pk[4 * m + 1];
+          v.z = pk[4 * m + 2];
+          v.w = pk[4 * m + 3];
+          *reinterpret_cast<uint4*>(prow + ((m ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + pb);
+        ++pcount;
+      }
+      if (!alive) break;
+      // ---- O epilogue
+      if (!mbar_wait_warp(o_full, litem & 1, ab, a.status)) break;
+      tc_fence_after();
+      float o[D / 2];
+      if (w.nkv > 0) {
+#pragma unroll
+        for (int c32 = 0; c32 < D / 64; ++c32) {
+          uint32_t orr[32];
+          tmem_ld32(tmem + C::O_COL + half * (D / 2) + c32 * 32 + lane_base, orr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[c32 * 32 + i] = __uint_as_float(orr[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < D / 2; ++i) o[i] = 0.f;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
+      if (row_ok) {
+        if (MODE == MODE_CAND) {
+          // self term: the candidate attends to itself at distance 0, gap 0
+          const __nv_bfloat16* rowp = a.q_buf + (q0 + r) * a.ld_f1;
+          const uint4* qp = reinterpret_cast<const uint4*>(rowp + a.q_col + w.head * D);
+          const uint4* kp = reinterpret_cast<const uint4*>(rowp + a.k_col + w.head * D);
+          float dot = 0.f;
+#pragma unroll 4
+          for (int i = 0; i < D / 8; ++i) {
+            const uint4 qa = qp[i], ka = kp[i];
+            const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              dot += bf16lo(qw[k]) * bf16lo(kw[k]) + bf16hi(qw[k]) * bf16hi(kw[k]);
+          }
+          const float s_self = dot + __ldg(Rp) + __ldg(Rt);
+          const float p_self = __bfloat162float(__float2bfloat16(silu_fast(s_self)));
+          const uint4* vp =
+              reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + half * (D / 2));
+#pragma unroll
+          for (int i = 0; i < D / 16; ++i) {
+            const uint4 va = vp[i];
+            const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              o[i * 8 + 2 * k] += p_self * bf16lo(vw[k]);
+              o[i * 8 + 2 * k + 1] += p_self * bf16hi(vw[k]);
+            }
+          }
+        }
+        uint4* op = reinterpret_cast<uint4*>(a.O + (q0 + r) * a.ldo + w.head * D + half * (D / 2));
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+          uint4 v;
+          v.x = pack_bf16x2(o[8 * i + 0] * inv_n, o[8 * i + 1] * inv_n);
+          v.y = pack_bf16x2(o[8 * i + 2] * inv_n, o[8 * i + 3] * inv_n);
+          v.z = pack_bf16x2(o[8 * i + 4] * inv_n, o[8 * i + 5] * inv_n);
+          v.w = pack_bf16x2(o[8 * i + 6] * inv_n, o[8 * i + 7] * inv_n);
+          op[i] = v;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, int MODE>
+static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tkv,
+                                    const AttnDev& ad, int grid, cudaStream_t s) {
+  using C = AttnCfg<D>;
+  auto kfn = k_attn_tc<D, MODE>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kfn<<<grid, 320, C::SMEM, s>>>(tq, tkv, ad);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
+  if (c.dqk != c.dv || (c.dqk != 64 && c.dqk != 128)) return cudaErrorInvalidValue;
+  if (c.item_cap <= 0 || c.q_rows_cap <= 0) return cudaSuccess;
+  CUtensorMap tq, tkv;
+  const uint64_t F = (uint64_t)c.ld_f1;
+  if (!encode_tmap_2d_bf16(&tq, c.q_buf, (uint64_t)c.q_rows_cap, F, F * 2, 64, 128))
+    return cudaErrorInvalidValue;
+  // With no history rows there is nothing to load from the KV buffer; any
+  // valid map will do (no KV tile is ever requested).
+  if (c.kv_rows_cap > 0) {
+    if (!encode_tmap_2d_bf16(&tkv, c.kv_buf, (uint64_t)c.kv_rows_cap, F, F * 2, 64, 128))
+      return cudaErrorInvalidValue;
+  } else {
+    tkv = tq;
+  }
+  AttnDev ad;
+  ad.mode = c.mode;
+  ad.items = c.items;
+  ad.n_items = c.n_items;
+  ad.q_off = c.q_off;
+  ad.kv_off = c.kv_off;
+  ad.kv_rows = c.kv_rows_cap;
+  ad.t_rel = c.t_rel;
+  ad.t_req_rel = c.t_req_rel;
+  ad.rab_pos = c.rab_pos;
+  ad.rab_time = c.rab_time;
+  ad.Np = c.Np;
+  ad.Nt = c.Nt;
+  ad.Sp = c.Sp;
+  ad.St = c.St;
+  ad.q_col = c.q_col;
+  ad.k_col = c.k_col;
+  ad.v_col = c.v_col;
+  ad.q_buf = static_cast<const __nv_bfloat16*>(c.q_buf);
+  ad.ld_f1 = c.ld_f1;
+  ad.O = static_cast<__nv_bfloat16*>(c.O);
+  ad.ldo = c.ldo;
+  ad.status = c.status;
+  const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());
+  LaunchScope ls(c.mode == MODE_SELF ? K_ATTN : K_ATTN_CAND, s);
+  if (c.mode == MODE_SELF)
+    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF>(tq, tkv, ad, grid, s)
+                     : launch_attn_inst<128, MODE_SELF>(tq, tkv, ad, grid, s);
+  return c.dqk == 64 ? launch_attn_inst<64, MODE_CAND>(tq, tkv, ad, grid, s)
+                   : launch_attn_inst<128, MODE_CAND>(tq, tkv, ad, grid, s);
+}
+
+}  // namespace hstu

@@ -1,0 +1,307 @@
+// gemm_tc.cu — bf16 GEMM on the 5th-generation tensor cores (tcgen05) with
+// fused epilogues, used for both projections of the HSTU layer:
+//   f1:  G = SiLU(X W1^T + b1)         (EPI_SILU; output = [U | V | Q | K])
+//   f2:  Y = X + Z W2^T + b2           (EPI_RESID)
+// ('HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか':
+// one projection f1 followed by SiLU and a split; f2 back to d_model plus
+// the residual connection.)
+//
+// Design (B200, sm_100a): persistent CTAs (one per SM), 128 x BN output tiles
+// walked n-fastest so that a wave of CTAs shares the A rows through L2.
+// Warp 0 streams A and W tiles with TMA (128-byte swizzle) into a STAGES-deep
+// ring; warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
+// accumulators; warps 2-5 drain the other accumulator with tcgen05.ld, apply
+// the epilogue in registers and store bf16 rows.  Every wait is bounded.
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace hstu {
+
+struct GemmDev {
+  int64_t M_cap;
+  const int64_t* M_dev;
+  int N, K, n_off;
+  const __nv_bfloat16* bias;
+  __nv_bfloat16* out;
+  int64_t ldo;
+  const __nv_bfloat16* resid;
+  int64_t ldr;
+  int* status;
+};
+
+template <int BN, int STAGES>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+};
+
+template <int EPI>
+DEVI void gemm_epilogue_store(const GemmDev& g, int64_t row, bool valid, int col,
+                              const uint32_t (&r)[32]) {
+  float v[32];
+  const uint4* bp = reinterpret_cast<const uint4*>(g.bias + col);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 bb = __ldg(bp + i);
+    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[i * 8 + 2 * k] = __uint_as_float(r[i * 8 + 2 * k]) + bf16lo(bw[k]);
+      v[i * 8 + 2 * k + 1] = __uint_as_float(r[i * 8 + 2 * k + 1]) + bf16hi(bw[k]);
+    }
+  }
+  if (!valid) return;
+  if (EPI == EPI_SILU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
+  } else {
+    const uint4* rp = reinterpret_cast<const uint4*>(g.resid + row * g.ldr + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 rr = rp[i];
+      const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[i * 8 + 2 * k] += bf16lo(rw[k]);
+        v[i * 8 + 2 * k + 1] += bf16hi(rw[k]);
+      }
+    }
+  }
+  uint4* op = reinterpret_cast<uint4*>(g.out + row * g.ldo + col);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 o;
+    o.x = pack_bf16x2(v[i * 8 + 0], v[i * 8 + 1]);
+    o.y = pack_bf16x2(v[i * 8 + 2], v[i * 8 + 3]);
+    o.z = pack_bf16x2(v[i * 8 + 4], v[i * 8 + 5]);
+    o.w = pack_bf16x2(v[i * 8 + 6], v[i * 8 + 7]);
+    op[i] = o;
+  }
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const GemmDev g) {
+  using C = GemmCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
+  int* s_go = reinterpret_cast<int*>(ab + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    *s_go = (g.status == nullptr) || (*reinterpret_cast<volatile int*>(g.status) == 0);
+    ab->flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(tfull + 0, 1);
+    mbar_init(tfull + 1, 1);
+    mbar_init(tempty + 0, 4);
+    mbar_init(tempty + 1, 4);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  __syncthreads();
+  if (!*s_go) return;
+
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int64_t Mrows = g.M_cap;
+  if (g.M_dev) {
+    const int64_t m = *g.M_dev;
+    Mrows = m < Mrows ? m : Mrows;
+  }
+  if (Mrows < 0) Mrows = 0;
+  const int n_tiles = g.N / BN;
+  const int m_tiles = (int)((Mrows + 127) / 128);
+  const int tiles = m_tiles * n_tiles;
+  const int KB = (g.K + 63) / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty + stage, ph ^ 1, ab, g.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(full + stage, C::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, kb * 64, mt * 128, full + stage);
+          tma_load_2d(sa + C::A_BYTES, &tmB, kb * 64, g.n_off + nt * BN, full + stage);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (ph << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {  // let every load already in flight land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if ((issued >> s) & 1u) {
+            AbortState tmp{0};
+            mbar_wait(full + s, (last_par >> s) & 1u, &tmp, nullptr);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, 0, 0);
+      int stage = 0, local = 0;
+      uint32_t ph = 0;
+      bool ok = true, issued_any = false;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait(tempty + acc, aph ^ 1, ab, g.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full + stage, ph, ab, g.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_bf16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
+                           sdesc_sw128(b0 + k * 32, 16, 1024), IDESC, (kb | k) != 0);
+          tc_commit(empty + stage);
+          issued_any = true;
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) tc_commit(tfull + acc);
+      }
+      if (issued_any) {
+        tc_commit(drain);  // completes once every MMA issued above has finished
+        AbortState tmp{0};
+        mbar_wait(drain, 0, &tmp, nullptr);
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) break;
+      tc_fence_after();
+      const int64_t row = (int64_t)mt * 128 + q * 32 + lane;
+      const bool valid = row < Mrows;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + acc * BN + c * 32 + ((uint32_t)(q * 32) << 16), r);
+        tmem_ld_wait();
+        gemm_epilogue_store<EPI>(g, row, valid, g.n_off + nt * BN + c * 32, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN, int STAGES, int EPI>
+static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmDev& gd,
+                              int grid, cudaStream_t s) {
+  using C = GemmCfg<BN, STAGES>;
+  auto kfn = k_gemm_tc<BN, STAGES, EPI>;
+  static bool attr_set = false;  // per instantiation; the attribute is per device function
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kfn<<<grid, 192, C::SMEM, s>>>(ta, tb, gd);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
+  if (c.M_cap <= 0 || c.N <= 0) return cudaSuccess;
+  if (c.N % 64 != 0 || c.K % 64 != 0) return cudaErrorInvalidValue;
+  const int sms = num_sms();
+  const int64_t mt = (c.M_cap + 127) / 128;
+  int BN = 64;
+  if (c.N % 256 == 0 && mt * (c.N / 256) >= 2 * sms) BN = 256;
+  else if (c.N % 128 == 0) BN = 128;
+  CUtensorMap ta, tb;
+  if (!encode_tmap_2d_bf16(&ta, c.A, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.lda * 2, 64, 128))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d_bf16(&tb, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K,
+                           (uint64_t)c.ldw * 2, 64, (uint32_t)BN))
+    return cudaErrorInvalidValue;
+  GemmDev gd;
+  gd.M_cap = c.M_cap;
+  gd.M_dev = c.M_dev;
+  gd.N = c.N;
+  gd.K = c.K;
+  gd.n_off = c.n_off;
+  gd.bias = static_cast<const __nv_bfloat16*>(c.bias);
+  gd.out = static_cast<__nv_bfloat16*>(c.out);
+  gd.ldo = c.ldo;
+  gd.resid = static_cast<const __nv_bfloat16*>(c.resid);
+  gd.ldr = c.ldr;
+  gd.status = c.status;
+  const int64_t tiles = mt * (c.N / BN);
+  const int grid = (int)std::min<int64_t>(tiles, sms);
+  LaunchScope ls(kernel_id, s);
+  if (c.epi == EPI_SILU) {
+    if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, gd, grid, s);
+    if (BN == 128) return launch_one<128, 6, EPI_SILU>(ta, tb, gd, grid, s);
+    return launch_one<64, 8, EPI_SILU>(ta, tb, gd, grid, s);
+  }
+  if (BN == 256) return launch_one<256, 4, EPI_RESID>(ta, tb, gd, grid, s);
+  if (BN == 128) return launch_one<128, 6, EPI_RESID>(ta, tb, gd, grid, s);
+  return launch_one<64, 8, EPI_RESID>(ta, tb, gd, grid, s);
+}
+
+}  // namespace hstu

@@ -1,0 +1,145 @@
+// hstu_internal.h — declarations shared by the library's translation units:
+// kernel argument blocks, launchers, tracing ids and the workspace layout.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/hstu.h"
+
+namespace hstu {
+
+// Query-tile height of the attention kernels and of every M tile.
+constexpr int kTile = 128;
+
+// ---------------------------------------------------------------- tracing
+enum KernelId : int32_t {
+  K_SCHEDULE = 0,
+  K_TIME_REL = 1,
+  K_GEMM_F1 = 2,
+  K_ATTN = 3,
+  K_LN_GATE = 4,
+  K_GEMM_F2 = 5,
+  K_MB_PLAN = 6,
+  K_MB_GATHER = 7,
+  K_ATTN_CAND = 8,
+  K_SCORE = 9,
+  K_SIMT_GEMM_F1 = 10,
+  K_SIMT_ATTN = 11,
+  K_SIMT_GEMM_F2 = 12,
+  K_SIMT_ATTN_CAND = 13,
+  K_NUM_KERNELS = 14
+};
+const char* kernel_name(int id);
+
+// Wraps one kernel launch: counts it and, when tracing is on, brackets it
+// with a CUDA event pair on `stream`.
+struct LaunchScope {
+  LaunchScope(int kernel_id, cudaStream_t stream);
+  ~LaunchScope();
+  int id;
+  cudaStream_t s;
+  int slot;
+};
+
+// ---------------------------------------------------------------- device info
+int num_sms();
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).  Returns false if the driver call is unavailable/failed.
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+
+// ---------------------------------------------------------------- workspace
+struct Header {           // first 256 bytes of every workspace
+  int32_t status;         // hstu_status of the device checks
+  int32_t n_items;        // attention work items of the history pass
+  int32_t n_cand_items;   // attention work items of the current microbatch
+  int32_t pad0;
+  int64_t mb_rows;        // rows of the current candidate microbatch
+};
+
+struct Layout {
+  size_t header, items, t_rel, f1, o, z, xtmp;            // layer / stack
+  size_t f1_cache, xh0, xh1;                              // M-FALCON history
+  size_t mb_off, c_items, t_req_rel, hist_n, xc0, xc1, f1c, oc, zc;  // candidates
+  size_t total;
+  int64_t item_cap, cand_item_cap, mb_cap;
+};
+bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, int64_t max_len,
+                 int64_t total_cands, int64_t max_cands, int microbatch, Layout* L);
+
+// ---------------------------------------------------------------- kernels
+struct AttnItem {
+  int32_t b, qt, head, nkv;
+};
+
+// Validate offsets; build the causal work list (user, q-tile, head), longest first.
+void launch_schedule(const int64_t* offsets, int64_t B, int64_t T, int64_t max_len, int n_heads,
+                     AttnItem* items, int64_t item_cap, Header* hdr, cudaStream_t s);
+// Per-row timestamp relative to the user's first one (int32), with checks.
+void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64_t T,
+                     int32_t* t_rel, Header* hdr, cudaStream_t s);
+
+// C[M, N] = A[M, K] * W[n_off + N, K]^T with fused epilogue, bf16 tcgen05.
+enum Epilogue { EPI_SILU = 0, EPI_RESID = 1 };
+struct GemmCall {
+  const void* A;  int64_t lda;   // [M_cap, K] row stride in elements
+  const void* W;  int64_t ldw;   // [N_total, K]
+  int64_t M_cap;                 // rows allocated in A / out
+  const int64_t* M_dev;          // actual rows (device), or null = M_cap
+  int N, K, n_off;
+  const void* bias;              // [N_total]
+  void* out; int64_t ldo;        // written at columns n_off + n
+  const void* resid; int64_t ldr;
+  int epi;
+  int* status;
+};
+cudaError_t launch_gemm_tc(const GemmCall& g, cudaStream_t s, int kernel_id);
+cudaError_t launch_gemm_simt_f32(const GemmCall& g, cudaStream_t s, int kernel_id);
+
+// Pointwise causal attention (SELF) or candidate-vs-history (CAND).
+struct AttnCall {
+  int mode;                        // 0 self, 1 candidate
+  int64_t B;
+  const AttnItem* items; const int32_t* n_items; int64_t item_cap;  // tensor-core path
+  const int64_t* q_off;            // [B+1] query-row offsets (self: = kv_off)
+  const int64_t* kv_off;           // [B+1]
+  const int64_t* q_rows_dev;       // SIMT path: device count of query rows (null = cap)
+  const void* q_buf; int64_t q_rows_cap;   // f1 output holding Q (and self K/V for CAND)
+  const void* kv_buf; int64_t kv_rows_cap; // f1 output holding the history K and V
+  int64_t ld_f1;                   // row stride (elements) of both f1 buffers = F
+  int q_col, k_col, v_col;         // column where head 0 of Q, K, V starts
+  const int32_t* t_rel;            // [T_kv] int32 relative timestamps
+  const int32_t* t_req_rel;        // CAND: [B] request time relative to the user's first
+  const float* rab_pos; const float* rab_time;
+  int Np, Nt, Sp, St, h, dqk, dv;
+  void* O; int64_t ldo;
+  int* status;
+};
+cudaError_t launch_attn_tc(const AttnCall& a, cudaStream_t s);
+cudaError_t launch_attn_simt_f32(const AttnCall& a, cudaStream_t s);
+
+// Z = LayerNorm(O) * gamma + beta, then * U (per row over h*d_v features).
+cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_f1,
+                           const void* gamma, const void* beta, float eps, void* Z, int hdv,
+                           int64_t rows_cap, const int64_t* rows_dev, const int* status,
+                           cudaStream_t s);
+
+// M-FALCON microbatch plumbing.
+void launch_mb_plan(const int64_t* hist_off, const int64_t* cand_off, int64_t B, int64_t max_len,
+                    int64_t max_cands, int k, int microbatch, int n_heads,
+                    const int64_t* hist_ts, const int64_t* request_ts, int64_t* mb_off,
+                    AttnItem* items, int64_t item_cap, int32_t* t_req_rel, Header* hdr,
+                    cudaStream_t s);
+cudaError_t launch_mb_gather(int dtype, const void* cands, int64_t d, const int64_t* cand_off,
+                             const int64_t* mb_off, int64_t B, int k, int microbatch,
+                             void* xc, int64_t rows_cap, const int64_t* rows_dev,
+                             const int* status, cudaStream_t s);
+cudaError_t launch_score(int dtype, const void* xc, int64_t d, const void* head_vec,
+                         const int64_t* cand_off, const int64_t* mb_off, int64_t B, int k,
+                         int microbatch, float* scores, int64_t rows_cap,
+                         const int64_t* rows_dev, const int* status, cudaStream_t s);
+
+}  // namespace hstu

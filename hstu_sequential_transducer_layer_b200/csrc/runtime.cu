@@ -1,0 +1,188 @@
+// runtime.cu — host-side runtime of libhstu: launch counting and tracing,
+// device queries, TMA descriptor encoding, and the workspace layout.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "hstu_internal.h"
+
+namespace hstu {
+
+// ---------------------------------------------------------------- tracing
+namespace {
+std::atomic<int64_t> g_launches{0};
+std::mutex g_trace_mu;
+int g_trace_cap = 0;
+int g_trace_used = 0;
+std::vector<cudaEvent_t> g_ev0, g_ev1;
+std::vector<int> g_ids;
+}  // namespace
+
+const char* kernel_name(int id) {
+  static const char* names[K_NUM_KERNELS] = {
+      "schedule",   "time_rel",   "gemm_f1_tc",      "attn_tc",
+      "ln_gate",    "gemm_f2_tc", "mb_plan",         "mb_gather",
+      "attn_cand_tc", "score",    "gemm_f1_simt_f32", "attn_simt_f32",
+      "gemm_f2_simt_f32", "attn_cand_simt_f32"};
+  return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
+}
+
+LaunchScope::LaunchScope(int kernel_id, cudaStream_t stream) : id(kernel_id), s(stream), slot(-1) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  if (g_trace_used < g_trace_cap) {
+    slot = g_trace_used++;
+    g_ids[slot] = kernel_id;
+    cudaEventRecord(g_ev0[slot], s);
+  }
+}
+LaunchScope::~LaunchScope() {
+  if (slot >= 0) cudaEventRecord(g_ev1[slot], s);
+}
+
+// ---------------------------------------------------------------- device
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- workspace
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, int64_t max_len,
+                 int64_t total_cands, int64_t max_cands, int microbatch, Layout* L) {
+  if (B < 0 || T < 0 || n_layers < 1 || total_cands < 0 || max_cands < 0) return false;
+  const size_t es = d.dtype == HSTU_BF16 ? 2 : 4;
+  const size_t F = 2 * (size_t)d.n_heads * (d.d_v + d.d_qk);
+  const size_t hdv = (size_t)d.n_heads * d.d_v;
+  const size_t dm = (size_t)d.d_model;
+  const bool mf = total_cands > 0 || microbatch > 0;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += up256(bytes);
+    return o;
+  };
+  *L = Layout{};
+  L->item_cap = ((T + kTile - 1) / kTile + B) * (int64_t)d.n_heads;
+  L->header = take(256);
+  L->items = take((size_t)L->item_cap * sizeof(AttnItem));
+  L->t_rel = take((size_t)T * 4);
+  if (!mf) {
+    L->f1 = take((size_t)T * F * es);
+  } else {
+    L->f1_cache = take((size_t)n_layers * T * F * es);
+    L->f1 = L->f1_cache;
+  }
+  L->o = take((size_t)T * hdv * es);
+  L->z = take((size_t)T * hdv * es);
+  L->xtmp = take((size_t)T * dm * es);
+  if (mf) {
+    if (microbatch < 1) return false;
+    L->xh0 = L->xtmp;
+    L->xh1 = take((size_t)T * dm * es);
+    int64_t cap = std::min<int64_t>(total_cands, B * (int64_t)microbatch);
+    L->mb_cap = cap;
+    L->cand_item_cap = ((cap + kTile - 1) / kTile + B) * (int64_t)d.n_heads;
+    L->mb_off = take((size_t)(B + 1) * 8);
+    L->c_items = take((size_t)L->cand_item_cap * sizeof(AttnItem));
+    L->t_req_rel = take((size_t)B * 4);
+    L->hist_n = take((size_t)B * 4);
+    L->xc0 = take((size_t)cap * dm * es);
+    L->xc1 = take((size_t)cap * dm * es);
+    L->f1c = take((size_t)cap * F * es);
+    L->oc = take((size_t)cap * hdv * es);
+    L->zc = take((size_t)cap * hdv * es);
+  }
+  (void)max_len;
+  (void)max_cands;
+  L->total = off;
+  return true;
+}
+
+}  // namespace hstu
+
+// ---------------------------------------------------------------- C ABI
+extern "C" {
+
+hstu_status hstu_trace_enable(int32_t max_records) {
+  using namespace hstu;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  for (auto e : g_ev0) cudaEventDestroy(e);
+  for (auto e : g_ev1) cudaEventDestroy(e);
+  g_ev0.clear();
+  g_ev1.clear();
+  g_ids.clear();
+  g_trace_cap = 0;
+  g_trace_used = 0;
+  if (max_records <= 0) return HSTU_OK;
+  g_ev0.resize(max_records);
+  g_ev1.resize(max_records);
+  g_ids.resize(max_records, -1);
+  for (int i = 0; i < max_records; ++i) {
+    if (cudaEventCreate(&g_ev0[i]) != cudaSuccess || cudaEventCreate(&g_ev1[i]) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+  }
+  g_trace_cap = max_records;
+  return HSTU_OK;
+}
+
+int32_t hstu_trace_read(int32_t* kernel_ids, float* ms, int32_t capacity) {
+  using namespace hstu;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  int n = std::min(g_trace_used, (int)capacity);
+  for (int i = 0; i < n; ++i) {
+    float t = -1.f;
+    if (cudaEventSynchronize(g_ev1[i]) == cudaSuccess) cudaEventElapsedTime(&t, g_ev0[i], g_ev1[i]);
+    if (kernel_ids) kernel_ids[i] = g_ids[i];
+    if (ms) ms[i] = t;
+  }
+  return n;
+}
+
+const char* hstu_kernel_name(int32_t kernel_id) { return hstu::kernel_name(kernel_id); }
+
+int64_t hstu_launch_count(void) { return hstu::g_launches.load(); }
+
+}  // extern "C"

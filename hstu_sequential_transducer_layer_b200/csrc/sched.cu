@@ -1,0 +1,498 @@
+// sched.cu — the jagged tile scheduler and the small memory-bound kernels
+// around the tensor-core ones:
+//   * k_schedule: validates the offsets and lists the attention work items
+//     (user, query tile, head) with the number of KV tiles each needs, longest
+//     first ('HSTUとGenerative Recommenders', section '長い履歴を現実の計算量へ
+//     収める4つの工夫', subsection '1. 長さの異なるsequenceをpaddingせず処理する':
+//     ragged sequences without padding); fully masked causal tiles never appear.
+//   * k_time_rel: per-row timestamp relative to the user's first one (int32).
+//   * k_ln_gate: Z = LayerNorm(O) * gamma + beta, times U (subsection
+//     '3. Uでcontextをgateし、次のlayerへ渡す').
+//   * M-FALCON microbatch plan / gather / score (subsection '4. M-FALCONで
+//     候補間の履歴計算を共有する').
+#include <cuda_bf16.h>
+
+#include <climits>
+
+#include "ptx.cuh"
+
+namespace hstu {
+
+constexpr int kSchedThreads = 1024;
+
+__device__ __forceinline__ void set_status(int* st, int code) { atomicCAS(st, 0, code); }
+
+// ---------------------------------------------------------------- schedule
+__global__ void __launch_bounds__(kSchedThreads)
+    k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t T, int64_t max_len, int h,
+               AttnItem* __restrict__ items, int64_t item_cap, Header* hdr) {
+  __shared__ int s_bad;
+  __shared__ int s_count[1024];
+  __shared__ int s_start[1024];
+  if (threadIdx.x == 0) {
+    hdr->status = HSTU_OK;
+    hdr->n_items = 0;
+    s_bad = 0;
+    if (off[0] != 0 || off[B] != T) s_bad = 1;
+  }
+  __syncthreads();
+  for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t n = off[b + 1] - off[b];
+    if (n < 0 || n > max_len) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0) hdr->status = HSTU_ERR_BAD_OFFSETS;
+    return;
+  }
+  // Work item (b, qt) needs qt + 1 KV tiles.  Level c = qt + 1 holds one item
+  // per user with at least c query tiles.  Levels are emitted longest first,
+  // users in order inside a level, heads innermost.
+  const int levels = (int)((max_len + kTile - 1) / kTile);
+  // Chunks of blockDim levels, highest level first: every thread counts its
+  // level, thread 0 turns the counts into start positions, every thread then
+  // writes its level's items.
+  __shared__ long long s_base;
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  for (int c_hi = levels; c_hi >= 1; c_hi -= blockDim.x) {
+    const int c = c_hi - (int)threadIdx.x;  // this thread's level in the chunk
+    int cnt = 0;
+    if (c >= 1)
+      for (int64_t b = 0; b < B; ++b) {
+        const int64_t nq = (off[b + 1] - off[b] + kTile - 1) / kTile;
+        cnt += nq >= c;
+      }
+    s_count[threadIdx.x] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long acc = s_base;
+      const int m = min((int)blockDim.x, c_hi);
+      for (int i = 0; i < m; ++i) {
+        s_start[i] = (int)acc;
+        acc += s_count[i];
+      }
+      s_base = acc;
+    }
+    __syncthreads();
+    if (c >= 1) {
+      int64_t pos = s_start[threadIdx.x];
+      for (int64_t b = 0; b < B; ++b) {
+        const int64_t nq = (off[b + 1] - off[b] + kTile - 1) / kTile;
+        if (nq >= c) {
+          for (int hh = 0; hh < h; ++hh) {
+            const int64_t idx = pos * h + hh;
+            if (idx < item_cap) items[idx] = AttnItem{(int32_t)b, c - 1, hh, c};
+          }
+          ++pos;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) hdr->n_items = (int32_t)(s_base * h < item_cap ? s_base * h : item_cap);
+}
+
+void launch_schedule(const int64_t* offsets, int64_t B, int64_t T, int64_t max_len, int n_heads,
+                     AttnItem* items, int64_t item_cap, Header* hdr, cudaStream_t s) {
+  LaunchScope ls(K_SCHEDULE, s);
+  k_schedule<<<1, kSchedThreads, 0, s>>>(offsets, B, T, max_len, n_heads, items, item_cap, hdr);
+}
+
+// ---------------------------------------------------------------- timestamps
+__device__ __forceinline__ int64_t find_user(const int64_t* off, int64_t B, int64_t row) {
+  int64_t lo = 0, hi = B;  // off[lo] <= row < off[hi]
+  while (hi - lo > 1) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (off[mid] <= row) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void k_time_rel(const int64_t* __restrict__ off, int64_t B,
+                           const int64_t* __restrict__ ts, int64_t T, int32_t* __restrict__ t_rel,
+                           Header* hdr) {
+  if (hdr->status != HSTU_OK) return;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < T;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t b = find_user(off, B, i);
+    const int64_t d = ts[i] - ts[off[b]];
+    if (d >= (1ll << 30) || d <= -(1ll << 30)) {
+      set_status(&hdr->status, HSTU_ERR_BAD_TIMESTAMPS);
+      t_rel[i] = 0;
+    } else {
+      t_rel[i] = (int32_t)d;
+    }
+  }
+}
+
+void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64_t T,
+                     int32_t* t_rel, Header* hdr, cudaStream_t s) {
+  if (T <= 0) return;
+  LaunchScope ls(K_TIME_REL, s);
+  const int grid = (int)std::min<int64_t>((T + 255) / 256, 4 * num_sms());
+  k_time_rel<<<grid, 256, 0, s>>>(offsets, B, ts, T, t_rel, hdr);
+}
+
+// ---------------------------------------------------------------- LayerNorm * U
+template <typename Tv>
+struct Elem;
+template <>
+struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16(v); }
+};
+template <>
+struct Elem<float> {
+  static __device__ __forceinline__ float ld(const float* p) { return *p; }
+  static __device__ __forceinline__ void st(float* p, float v) { *p = v; }
+};
+
+// One warp per row.  Vectorised path for bf16 rows of a multiple of 256
+// features (8 per lane per 16-byte load, up to 2048 features); otherwise
+// strided scalar loads (up to 2048 features).
+constexpr int kLnMaxPerLane = 64;
+
+template <typename Tv, bool VEC>
+__global__ void __launch_bounds__(256)
+    k_ln_gate(const Tv* __restrict__ O, const Tv* __restrict__ f1, int64_t ld_f1,
+              const Tv* __restrict__ gamma, const Tv* __restrict__ beta, float eps,
+              Tv* __restrict__ Z, int hdv, int64_t rows_cap, const int64_t* rows_dev,
+              const int* status) {
+  if (status && *status != HSTU_OK) return;
+  int64_t rows = rows_cap;
+  if (rows_dev) rows = min(rows, *rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  float x[kLnMaxPerLane];
+  const Tv* orow = O + row * (int64_t)hdv;
+  const Tv* urow = f1 + row * ld_f1;  // U occupies the first h*d_v columns
+  Tv* zrow = Z + row * (int64_t)hdv;
+  float sum = 0.f;
+  if (VEC) {
+    const int nch = hdv / 256;
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane / 8; ++k) {
+      if (k < nch) {
+        const uint4 v = *reinterpret_cast<const uint4*>(orow + (k * 32 + lane) * 8);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[k * 8 + 2 * e] = bf16lo(w[e]);
+          x[k * 8 + 2 * e + 1] = bf16hi(w[e]);
+          sum += x[k * 8 + 2 * e] + x[k * 8 + 2 * e + 1];
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane; ++k) {
+      const int c = k * 32 + lane;
+      x[k] = c < hdv ? Elem<Tv>::ld(orow + c) : 0.f;
+      sum += x[k];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum / (float)hdv;
+  float ss = 0.f;
+  if (VEC) {
+    const int nch = hdv / 256;
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane / 8; ++k)
+      if (k < nch)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float dlt = x[k * 8 + e] - mean;
+          ss += dlt * dlt;
+        }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane; ++k) {
+      const int c = k * 32 + lane;
+      if (c < hdv) {
+        const float dlt = x[k] - mean;
+        ss += dlt * dlt;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rstd = rsqrtf(ss / (float)hdv + eps);
+  if (VEC) {
+    const int nch = hdv / 256;
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane / 8; ++k) {
+      if (k < nch) {
+        const int c0 = (k * 32 + lane) * 8;
+        const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gamma + c0));
+        const uint4 bv = __ldg(reinterpret_cast<const uint4*>(beta + c0));
+        const uint4 uv = *reinterpret_cast<const uint4*>(urow + c0);
+        const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w}, bb[4] = {bv.x, bv.y, bv.z, bv.w},
+                       u[4] = {uv.x, uv.y, uv.z, uv.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float z0 = ((x[k * 8 + 2 * e] - mean) * rstd * bf16lo(g[e]) + bf16lo(bb[e])) * bf16lo(u[e]);
+          const float z1 =
+              ((x[k * 8 + 2 * e + 1] - mean) * rstd * bf16hi(g[e]) + bf16hi(bb[e])) * bf16hi(u[e]);
+          out[e] = pack_bf16x2(z0, z1);
+        }
+        *reinterpret_cast<uint4*>(zrow + c0) = make_uint4(out[0], out[1], out[2], out[3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane; ++k) {
+      const int c = k * 32 + lane;
+      if (c < hdv) {
+        const float z = ((x[k] - mean) * rstd * Elem<Tv>::ld(gamma + c) + Elem<Tv>::ld(beta + c)) *
+                        Elem<Tv>::ld(urow + c);
+        Elem<Tv>::st(zrow + c, z);
+      }
+    }
+  }
+}
+
+cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_f1,
+                           const void* gamma, const void* beta, float eps, void* Z, int hdv,
+                           int64_t rows_cap, const int64_t* rows_dev, const int* status,
+                           cudaStream_t s) {
+  if (rows_cap <= 0) return cudaSuccess;
+  if (hdv > 32 * kLnMaxPerLane) return cudaErrorInvalidValue;
+  LaunchScope ls(K_LN_GATE, s);
+  const int grid = (int)((rows_cap + 7) / 8);
+  if (dtype == HSTU_BF16) {
+    using T = __nv_bfloat16;
+    if (hdv % 256 == 0)
+      k_ln_gate<T, true><<<grid, 256, 0, s>>>((const T*)O, (const T*)f1, ld_f1, (const T*)gamma,
+                                              (const T*)beta, eps, (T*)Z, hdv, rows_cap, rows_dev,
+                                              status);
+    else
+      k_ln_gate<T, false><<<grid, 256, 0, s>>>((const T*)O, (const T*)f1, ld_f1, (const T*)gamma,
+                                               (const T*)beta, eps, (T*)Z, hdv, rows_cap,
+                                               rows_dev, status);
+  } else {
+    using T = float;
+    k_ln_gate<T, false><<<grid, 256, 0, s>>>((const T*)O, (const T*)f1, ld_f1, (const T*)gamma,
+                                             (const T*)beta, eps, (T*)Z, hdv, rows_cap, rows_dev,
+                                             status);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- M-FALCON plan
+// For microbatch k: per user, rows [k*bm, min((k+1)*bm, m_b)) of its
+// candidates; mb_off = prefix of those counts; attention items (b, q-tile,
+// head) needing ceil(n_b/128) history KV tiles, longest first; request time
+// relative to the user's first history timestamp.
+__global__ void __launch_bounds__(kSchedThreads)
+    k_mb_plan(const int64_t* __restrict__ hoff, const int64_t* __restrict__ coff, int64_t B,
+              int64_t max_len, int64_t max_cands, int k, int bm, int h,
+              const int64_t* __restrict__ hts, const int64_t* __restrict__ req_ts,
+              int64_t* __restrict__ mb_off, AttnItem* __restrict__ items, int64_t item_cap,
+              int32_t* __restrict__ t_req_rel, Header* hdr) {
+  __shared__ long long s_part[kSchedThreads];
+  __shared__ long long s_carry;
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) {
+    s_bad = 0;
+    hdr->n_cand_items = 0;
+    hdr->mb_rows = 0;
+  }
+  __syncthreads();
+  if (hdr->status != HSTU_OK) return;
+  if (k == 0) {
+    if (threadIdx.x == 0 && coff[0] != 0) s_bad = 1;
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+      const int64_t m = coff[b + 1] - coff[b];
+      if (m < 0 || m > max_cands) s_bad = 1;
+    }
+    __syncthreads();
+    if (s_bad) {
+      if (threadIdx.x == 0) set_status(&hdr->status, HSTU_ERR_BAD_OFFSETS);
+      return;
+    }
+  }
+  // prefix sum of per-user microbatch counts
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int64_t b0 = 0; b0 <= B; b0 += blockDim.x) {
+    const int64_t b = b0 + threadIdx.x;
+    long long cnt = 0;
+    if (b < B) {
+      const int64_t m = coff[b + 1] - coff[b];
+      { const int64_t rem = m - (int64_t)k * bm; cnt = rem < 0 ? 0 : (rem > bm ? bm : rem); }
+    }
+    s_part[threadIdx.x] = cnt;
+    __syncthreads();
+    for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+      const long long v = threadIdx.x >= (unsigned)o ? s_part[threadIdx.x - o] : 0;
+      __syncthreads();
+      s_part[threadIdx.x] += v;
+      __syncthreads();
+    }
+    if (b <= B) mb_off[b] = s_carry + s_part[threadIdx.x] - cnt;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) s_carry += s_part[threadIdx.x];
+    __syncthreads();
+  }
+  // request time relative to the first history timestamp
+  for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t n = hoff[b + 1] - hoff[b];
+    const int64_t t_last = n > 0 ? hts[hoff[b + 1] - 1] : 0;
+    const int64_t t_req = req_ts ? req_ts[b] : t_last;
+    const int64_t base = n > 0 ? hts[hoff[b]] : t_req;
+    const int64_t d = t_req - base;
+    if (d >= (1ll << 30) || d <= -(1ll << 30)) {
+      set_status(&hdr->status, HSTU_ERR_BAD_TIMESTAMPS);
+      t_req_rel[b] = 0;
+    } else {
+      t_req_rel[b] = (int32_t)d;
+    }
+  }
+  __syncthreads();
+  // items, longest history first: level c = number of KV tiles (0..levels)
+  __shared__ long long s_base;
+  __shared__ int s_cnt[kSchedThreads];
+  __shared__ long long s_start[kSchedThreads];
+  const int levels = (int)((max_len + kTile - 1) / kTile);
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  for (int c_hi = levels; c_hi >= 0; c_hi -= blockDim.x) {
+    const int c = c_hi - (int)threadIdx.x;
+    int cnt = 0;
+    if (c >= 0)
+      for (int64_t b = 0; b < B; ++b) {
+        const int64_t n = hoff[b + 1] - hoff[b];
+        const int nkv = (int)((n + kTile - 1) / kTile);
+        if (nkv == c) {
+          const int64_t rows = mb_off[b + 1] - mb_off[b];
+          cnt += (int)((rows + kTile - 1) / kTile);
+        }
+      }
+    s_cnt[threadIdx.x] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long acc = s_base;
+      const int m = min((int)blockDim.x, c_hi + 1);
+      for (int i = 0; i < m; ++i) {
+        s_start[i] = acc;
+        acc += s_cnt[i];
+      }
+      s_base = acc;
+    }
+    __syncthreads();
+    if (c >= 0) {
+      long long pos = s_start[threadIdx.x];
+      for (int64_t b = 0; b < B; ++b) {
+        const int64_t n = hoff[b + 1] - hoff[b];
+        const int nkv = (int)((n + kTile - 1) / kTile);
+        if (nkv != c) continue;
+        const int64_t rows = mb_off[b + 1] - mb_off[b];
+        const int nq = (int)((rows + kTile - 1) / kTile);
+        for (int qt = 0; qt < nq; ++qt, ++pos)
+          for (int hh = 0; hh < h; ++hh) {
+            const long long idx = pos * h + hh;
+            if (idx < item_cap) items[idx] = AttnItem{(int32_t)b, qt, hh, nkv};
+          }
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    hdr->n_cand_items = (int32_t)(s_base * h < item_cap ? s_base * h : item_cap);
+    hdr->mb_rows = mb_off[B];
+  }
+}
+
+void launch_mb_plan(const int64_t* hist_off, const int64_t* cand_off, int64_t B, int64_t max_len,
+                    int64_t max_cands, int k, int microbatch, int n_heads,
+                    const int64_t* hist_ts, const int64_t* request_ts, int64_t* mb_off,
+                    AttnItem* items, int64_t item_cap, int32_t* t_req_rel, Header* hdr,
+                    cudaStream_t s) {
+  LaunchScope ls(K_MB_PLAN, s);
+  k_mb_plan<<<1, kSchedThreads, 0, s>>>(hist_off, cand_off, B, max_len, max_cands, k, microbatch,
+                                        n_heads, hist_ts, request_ts, mb_off, items, item_cap,
+                                        t_req_rel, hdr);
+}
+
+// ---------------------------------------------------------------- gather / score
+template <typename Tv>
+__global__ void k_mb_gather(const Tv* __restrict__ cands, int64_t d,
+                            const int64_t* __restrict__ coff, const int64_t* __restrict__ mb_off,
+                            int64_t B, int k, int bm, Tv* __restrict__ xc, int64_t rows_cap,
+                            const int64_t* rows_dev, const int* status) {
+  if (*status != HSTU_OK) return;
+  const int64_t rows = min(rows_cap, *rows_dev);
+  const int64_t vec = (int64_t)(16 / sizeof(Tv));
+  const int64_t per_row = d / vec;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < rows * per_row;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / per_row, c = i - r * per_row;
+    const int64_t b = find_user(mb_off, B, r);
+    const int64_t src = coff[b] + (int64_t)k * bm + (r - mb_off[b]);
+    reinterpret_cast<uint4*>(xc + r * d)[c] = reinterpret_cast<const uint4*>(cands + src * d)[c];
+  }
+}
+
+cudaError_t launch_mb_gather(int dtype, const void* cands, int64_t d, const int64_t* cand_off,
+                             const int64_t* mb_off, int64_t B, int k, int microbatch, void* xc,
+                             int64_t rows_cap, const int64_t* rows_dev, const int* status,
+                             cudaStream_t s) {
+  if (rows_cap <= 0) return cudaSuccess;
+  LaunchScope ls(K_MB_GATHER, s);
+  const int grid = 4 * num_sms();
+  if (dtype == HSTU_BF16)
+    k_mb_gather<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)cands, d, cand_off,
+                                                     mb_off, B, k, microbatch,
+                                                     (__nv_bfloat16*)xc, rows_cap, rows_dev,
+                                                     status);
+  else
+    k_mb_gather<float><<<grid, 256, 0, s>>>((const float*)cands, d, cand_off, mb_off, B, k,
+                                            microbatch, (float*)xc, rows_cap, rows_dev, status);
+  return cudaGetLastError();
+}
+
+template <typename Tv>
+__global__ void k_score(const Tv* __restrict__ xc, int64_t d, const Tv* __restrict__ w,
+                        const int64_t* __restrict__ coff, const int64_t* __restrict__ mb_off,
+                        int64_t B, int k, int bm, float* __restrict__ scores, int64_t rows_cap,
+                        const int64_t* rows_dev, const int* status) {
+  if (*status != HSTU_OK) return;
+  const int64_t rows = min(rows_cap, *rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int64_t r = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  float acc = 0.f;
+  for (int64_t c = lane; c < d; c += 32) acc += Elem<Tv>::ld(xc + r * d + c) * Elem<Tv>::ld(w + c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    const int64_t b = find_user(mb_off, B, r);
+    scores[coff[b] + (int64_t)k * bm + (r - mb_off[b])] = acc;
+  }
+}
+
+cudaError_t launch_score(int dtype, const void* xc, int64_t d, const void* head_vec,
+                         const int64_t* cand_off, const int64_t* mb_off, int64_t B, int k,
+                         int microbatch, float* scores, int64_t rows_cap,
+                         const int64_t* rows_dev, const int* status, cudaStream_t s) {
+  if (rows_cap <= 0) return cudaSuccess;
+  LaunchScope ls(K_SCORE, s);
+  const int grid = (int)((rows_cap + 7) / 8);
+  if (dtype == HSTU_BF16)
+    k_score<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)xc, d,
+                                                 (const __nv_bfloat16*)head_vec, cand_off, mb_off,
+                                                 B, k, microbatch, scores, rows_cap, rows_dev,
+                                                 status);
+  else
+    k_score<float><<<grid, 256, 0, s>>>((const float*)xc, d, (const float*)head_vec, cand_off,
+                                        mb_off, B, k, microbatch, scores, rows_cap, rows_dev,
+                                        status);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

@@ -1,0 +1,92 @@
+"""Holds a layer descriptor, device weights and a reusable workspace, and
+calls the C ABI with them.  Allocation (weights, workspace, outputs) goes
+through torch; the computation is the library's."""
+from __future__ import annotations
+
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+from . import binding as _b
+
+
+class HSTURunner:
+    def __init__(self, dims: Dict[str, object], weights: Sequence[Dict[str, np.ndarray]],
+                 device="cuda"):
+        import torch
+        self.torch = torch
+        self.device = torch.device(device)
+        self.dtype = str(dims["dtype"])
+        self.tdtype = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        self.desc = _b.make_desc(int(dims["d_model"]), int(dims["n_heads"]), int(dims["d_qk"]),
+                                 int(dims["d_v"]), int(dims["n_pos_buckets"]),
+                                 int(dims["n_time_buckets"]), int(dims["pos_sub_bits"]),
+                                 int(dims["time_sub_bits"]), float(dims["ln_eps"]), self.dtype)
+        self.weights = _b.weights_to_device(weights, self.dtype, self.device)
+        self.n_layers = len(self.weights)
+        self._warr = _b.weights_array(self.weights)
+        self._ws = None
+
+    # ------------------------------------------------------------ memory
+    def workspace(self, nbytes: int):
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = self.torch.empty(max(nbytes, 256), dtype=self.torch.uint8, device=self.device)
+        return self._ws
+
+    def to_device(self, a: np.ndarray, kind: str = "act"):
+        t = self.torch
+        if kind == "act":
+            return t.from_numpy(np.ascontiguousarray(a, np.float32)).to(self.device, self.tdtype)
+        if kind == "i64":
+            return t.from_numpy(np.ascontiguousarray(a, np.int64)).to(self.device)
+        return t.from_numpy(np.ascontiguousarray(a, np.float32)).to(self.device)
+
+    # ------------------------------------------------------------ calls
+    def stack(self, offsets, X, timestamps, max_len: int, n_layers: Optional[int] = None,
+              out=None, stream=None):
+        """hstu_stack_fwd over device tensors; returns `out`."""
+        L = self.n_layers if n_layers is None else n_layers
+        B = offsets.numel() - 1
+        T = X.shape[0]
+        if out is None:
+            out = self.torch.empty_like(X)
+        nb = _b.hstu_workspace_size(self.desc, L, B, T, max_len)
+        ws = self.workspace(nb)
+        if L == 1:
+            _b.hstu_layer_fwd(self.desc, B, T, max_len, offsets, X, self._warr[0], timestamps, out,
+                              ws, stream)
+        else:
+            _b.hstu_stack_fwd(self.desc, L, self._warr, B, T, max_len, offsets, X, timestamps, out,
+                              ws, stream)
+        return out
+
+    def rank(self, hist_offsets, history, hist_ts, cand_offsets, candidates, request_ts,
+             microbatch: int, head_vec, max_len: int, max_cands: int, scores=None, stream=None):
+        B = hist_offsets.numel() - 1
+        T = history.shape[0]
+        C = candidates.shape[0]
+        if scores is None:
+            scores = self.torch.empty(C, dtype=self.torch.float32, device=self.device)
+        nb = _b.hstu_workspace_size(self.desc, self.n_layers, B, T, max_len, C, max_cands,
+                                    microbatch)
+        ws = self.workspace(nb)
+        _b.hstu_mfalcon_rank(self.desc, self.n_layers, self._warr, B, T, max_len, hist_offsets,
+                             history, hist_ts, C, max_cands, cand_offsets, candidates, request_ts,
+                             microbatch, head_vec, scores, ws, stream)
+        return scores
+
+    def status(self, stream=None) -> int:
+        return _b.hstu_read_status(self._ws, stream)
+
+    def intermediates(self, B: int, T: int, max_len: int):
+        """Views of the f1 output, O and Z the last layer call left in the workspace."""
+        f1o, oo, zo = _b.hstu_debug_offsets(self.desc, B, T, max_len)
+        d = self.desc
+        F = 2 * d.n_heads * (d.d_v + d.d_qk)
+        hdv = d.n_heads * d.d_v
+        es = 2 if self.dtype == "bf16" else 4
+        ws = self._ws
+
+        def view(off, cols):
+            return ws[off:off + T * cols * es].view(self.tdtype).view(T, cols)
+        return view(f1o, F), view(oo, hdv), view(zo, hdv)

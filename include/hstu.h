@@ -1,0 +1,181 @@
+/*
+ * hstu.h — C ABI of libhstu.so: the forward pass of an HSTU layer stack over
+ * jagged (unpadded) user sequences, and M-FALCON candidate ranking, on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Source of the operations: the page 'HSTUとGenerative Recommenders――行動履歴から
+ * 1.5兆parameterの推薦モデルへ' (koktn.github.io, an explainer of Zhai et al.,
+ * "Actions Speak Louder than Words", ICML 2024):
+ *   - section 'HSTUはTransformerと何が違うのか', subsections
+ *     '1. U、V、Q、Kは同じ入力を見る4つの役割' (f1 + SiLU, split U,V,Q,K),
+ *     '2. QKᵀで「どの履歴を見るか」を決める' (score = Q_i.K_j + position bias +
+ *     time bias, causal, pointwise SiLU weights without softmax),
+ *     '3. Uでcontextをgateし、次のlayerへ渡す' (LayerNorm(context) * U, f2,
+ *     residual connection);
+ *   - section '長い履歴を現実の計算量へ収める4つの工夫', subsections
+ *     '1. 長さの異なるsequenceをpaddingせず処理する' (ragged batches without
+ *     padding) and '4. M-FALCONで候補間の履歴計算を共有する' (candidates in
+ *     microbatches appended after the history, mask and relative bias
+ *     adjusted, history K/V cache shared across microbatches).
+ *
+ * Per user b (rows i, j of that user, n_b rows) one layer computes
+ *   G = SiLU(X W1^T + b1) = [U | V | Q | K]   (head-major inside each part)
+ *   s_ij = Q_i.K_j + rab_pos[h][pb(i-j)] + rab_time[h][tb(max(0, t_i - t_j))],  j <= i
+ *   O_i  = (1/n_b) sum_{j<=i} SiLU(s_ij) V_j
+ *   Y_i  = X_i + (LayerNorm(O_i) * U_i) W2^T + b2
+ * where pb/tb are log-linear buckets: x < 2^S -> x; otherwise, with
+ * e = floor(log2 x), (e-S+1)*2^S + (x >> (e-S)) - 2^S; clamped to N-1.
+ * LayerNorm runs over all h*d_v features of a row (biased variance, eps from
+ * the descriptor), then gamma, beta.
+ *
+ * Conventions for every entry point
+ *   Ownership   The caller owns every buffer.  The library never allocates,
+ *               frees or synchronises device memory, except that
+ *               hstu_read_status synchronises the given stream.
+ *   Execution   Asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *               default stream).  Returning HSTU_OK means the work was
+ *               enqueued; device-detected errors are read with hstu_read_status.
+ *   Layout      Row-major.  Activations [rows, d_model]; weights in [out, in]
+ *               layout: W1 [F, d_model] with F = 2*h*d_v + 2*h*d_qk in the
+ *               column order U, V, Q, K; W2 [d_model, h*d_v]; b1 [F]; b2
+ *               [d_model]; ln_gamma, ln_beta [h*d_v]; rab_pos [h, n_pos_buckets]
+ *               and rab_time [h, n_time_buckets] always fp32.  Element type of
+ *               everything else is the descriptor's dtype (bf16 or fp32).
+ *               Every device pointer must be 16-byte aligned.  Inputs and
+ *               outputs must not alias each other or the workspace.
+ *   Offsets     int64 [B+1], offsets[0] = 0, non-decreasing, offsets[B] =
+ *               total rows; every length <= max_len.
+ *   Timestamps  int64 seconds, one per row; within one user every timestamp
+ *               must lie within 2^30 s of that user's first one.
+ *   Errors      Host-detectable argument errors return at once and enqueue
+ *               nothing.  Device-detected errors (bad offsets or timestamps,
+ *               a wait that timed out) set a status word in the workspace; the
+ *               remaining kernels of the call then exit early.  No entry
+ *               point traps or asserts on the device.
+ *   Supported   bf16: d_qk = d_v in {64, 128}; d_model and h*d_v multiples
+ *               of 64; bucket counts in [1, 4096].  fp32: d_qk, d_v <= 128
+ *               and multiples of 4; d_model multiple of 4.
+ */
+#ifndef HSTU_H_
+#define HSTU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,   /* host: null/misaligned pointer, bad size */
+  HSTU_ERR_UNSUPPORTED = 2,   /* host: shape or dtype this build does not run */
+  HSTU_ERR_WORKSPACE = 3,     /* host: workspace smaller than hstu_workspace_size */
+  HSTU_ERR_CUDA = 4,          /* host: a CUDA runtime call failed */
+  HSTU_ERR_BAD_OFFSETS = 5,   /* device: offsets not monotone, wrong total, length > max */
+  HSTU_ERR_TIMEOUT = 6,       /* device: an in-kernel wait gave up */
+  HSTU_ERR_BAD_TIMESTAMPS = 7 /* device: a user's timestamps span 2^30 s or more */
+} hstu_status;
+
+typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1 } hstu_dtype;
+
+/* Shape of one layer (all layers of a stack share it). */
+typedef struct {
+  int32_t d_model;         /* d */
+  int32_t n_heads;         /* h */
+  int32_t d_qk;            /* per-head query/key width */
+  int32_t d_v;             /* per-head value/gate width */
+  int32_t n_pos_buckets;   /* N_p: entries per head in rab_pos */
+  int32_t n_time_buckets;  /* N_t: entries per head in rab_time */
+  int32_t pos_sub_bits;    /* S_p of the position buckets, 0..20 */
+  int32_t time_sub_bits;   /* S_t of the time-gap buckets, 0..20 */
+  float ln_eps;            /* LayerNorm epsilon */
+  int32_t dtype;           /* hstu_dtype of activations and dense weights */
+} hstu_layer_desc;
+
+/* Device pointers to one layer's parameters (layout above). */
+typedef struct {
+  const void* W1;
+  const void* b1;
+  const void* W2;
+  const void* b2;
+  const void* ln_gamma;
+  const void* ln_beta;
+  const float* rab_pos;
+  const float* rab_time;
+} hstu_layer_weights;
+
+/* Bytes of device workspace an entry point needs for these sizes.
+ * For hstu_layer_fwd / hstu_stack_fwd pass total_cands = max_cands = 0 and
+ * microbatch = 0.  Returns 0 if the arguments are invalid. */
+size_t hstu_workspace_size(const hstu_layer_desc* desc, int32_t n_layers, int64_t B,
+                           int64_t total_tokens, int64_t max_len, int64_t total_cands,
+                           int64_t max_cands, int32_t microbatch);
+
+/* One HSTU layer.  offsets: device int64 [B+1]; X: device [T, d]; weights:
+ * host struct of device pointers; timestamps: device int64 [T]; out: device
+ * [T, d] (must not alias X). */
+hstu_status hstu_layer_fwd(const hstu_layer_desc* desc, int64_t B, int64_t total_tokens,
+                           int64_t max_len, const int64_t* offsets, const void* X,
+                           const hstu_layer_weights* weights, const int64_t* timestamps,
+                           void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* n_layers layers, each layer's output the next one's input (section '3. U
+ * でcontextをgateし、次のlayerへ渡す').  weights: host array [n_layers].  The
+ * offsets are validated once and the tile schedule is shared by all layers. */
+hstu_status hstu_stack_fwd(const hstu_layer_desc* desc, int32_t n_layers,
+                           const hstu_layer_weights* weights, int64_t B, int64_t total_tokens,
+                           int64_t max_len, const int64_t* offsets, const void* X,
+                           const int64_t* timestamps, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* M-FALCON ranking (section '4. M-FALCONで候補間の履歴計算を共有する').
+ * The histories run through n_layers layers once, keeping every layer's K/V;
+ * then candidates, in microbatches of `microbatch` per user, run through the
+ * layers attending to their user's whole history and to themselves only.
+ * Every candidate sits at position n_b (distance n_b - j to history row j)
+ * and at time request_ts[b] (NULL: the user's last history timestamp); its
+ * normaliser is max(n_b, 1).  scores[c] = <y_c, head_vec> in fp32, where y_c
+ * is candidate c's output of the last layer.
+ * hist_offsets [B+1], history [T_hist, d], hist_timestamps [T_hist],
+ * cand_offsets [B+1] (device), candidates [C, d], head_vec [d], scores fp32
+ * [C].  Every user has at most max_cands candidates. */
+hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
+                              const hstu_layer_weights* weights, int64_t B, int64_t total_hist,
+                              int64_t max_len, const int64_t* hist_offsets, const void* history,
+                              const int64_t* hist_timestamps, int64_t total_cands,
+                              int64_t max_cands, const int64_t* cand_offsets,
+                              const void* candidates, const int64_t* request_ts,
+                              int32_t microbatch, const void* head_vec, float* scores,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the device status word that the last
+ * call using this workspace left (HSTU_OK if none of its checks failed). */
+hstu_status hstu_read_status(const void* workspace, size_t workspace_bytes, void* stream);
+
+/* Test hook: byte offsets inside the workspace where hstu_layer_fwd (and the
+ * last layer of hstu_stack_fwd) leaves its intermediates: the f1 output
+ * [T, F] (U|V|Q|K after SiLU), the pre-LayerNorm attention output O [T, h*d_v]
+ * (already scaled by 1/n_b) and the gated Z [T, h*d_v]. */
+hstu_status hstu_debug_offsets(const hstu_layer_desc* desc, int64_t B, int64_t total_tokens,
+                               int64_t max_len, size_t* f1_offset, size_t* o_offset,
+                               size_t* z_offset);
+
+/* Tracing.  hstu_trace_enable(n) records a CUDA event pair around each of
+ * the next n kernel launches (n = 0 turns tracing off); hstu_trace_read
+ * synchronises and returns, per traced launch, the kernel id and the device
+ * time in ms.  hstu_kernel_name maps an id to a name.  hstu_launch_count
+ * counts every kernel this library has launched in this process. */
+hstu_status hstu_trace_enable(int32_t max_records);
+int32_t hstu_trace_read(int32_t* kernel_ids, float* ms, int32_t capacity);
+const char* hstu_kernel_name(int32_t kernel_id);
+int64_t hstu_launch_count(void);
+
+const char* hstu_status_string(hstu_status s);
+int32_t hstu_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H_ */

@@ -1,0 +1,61 @@
+"""Helpers shared by the GPU parity tests: error metrics and running a
+workload through the C ABI (via the runner)."""
+import math
+
+import numpy as np
+
+import hstu_workloads as hw
+
+# Tolerances: max |gpu - oracle| / RMS(oracle).
+TOL = {hw.FP32: 1e-4, hw.BF16: 2e-2}
+
+
+def relerr(g, r) -> float:
+    g = np.asarray(g, np.float64)
+    r = np.asarray(r, np.float64)
+    rms = math.sqrt(float(np.mean(r * r))) if r.size else 0.0
+    if rms == 0.0:
+        return float(np.max(np.abs(g - r))) if r.size else 0.0
+    return float(np.max(np.abs(g - r))) / rms
+
+
+def rmserr(g, r) -> float:
+    g = np.asarray(g, np.float64)
+    r = np.asarray(r, np.float64)
+    rms = math.sqrt(float(np.mean(r * r))) or 1.0
+    return math.sqrt(float(np.mean((g - r) ** 2))) / rms
+
+
+def runner_for(w, device="cuda"):
+    from hstu_sequential_transducer_layer_b200 import HSTURunner
+    return HSTURunner(hw.dims_dict(w.dims), w.weights, device)
+
+
+def run_stack(w, n_layers=None, runner=None):
+    """Runs the stack on the GPU.  Returns (Y float64 [T,d], runner, device inputs)."""
+    import torch
+    r = runner or runner_for(w)
+    off = r.to_device(w.offsets, "i64")
+    X = r.to_device(w.X, "act")
+    ts = r.to_device(w.timestamps, "i64")
+    out = r.stack(off, X, ts, w.max_len, n_layers=n_layers)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy(), r, (off, X, ts)
+
+
+def run_rank(w, microbatch=None, runner=None, candidates=None, cand_offsets=None,
+             request_ts="auto"):
+    import torch
+    r = runner or runner_for(w)
+    cands = w.candidates if candidates is None else candidates
+    coff = w.cand_offsets if cand_offsets is None else cand_offsets
+    req = w.request_ts if isinstance(request_ts, str) else request_ts
+    m = np.diff(coff)
+    scores = r.rank(r.to_device(w.offsets, "i64"), r.to_device(w.X, "act"),
+                    r.to_device(w.timestamps, "i64"), r.to_device(coff, "i64"),
+                    r.to_device(cands, "act"),
+                    None if req is None else r.to_device(req, "i64"),
+                    int(microbatch or w.microbatch), r.to_device(w.head_vec, "act"),
+                    w.max_len, int(m.max(initial=0)))
+    torch.cuda.synchronize()
+    return scores.double().cpu().numpy(), r

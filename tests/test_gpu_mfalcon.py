@@ -1,0 +1,104 @@
+"""GPU parity of M-FALCON ranking (through the C ABI) against the float64
+oracle, plus the method's invariants on the GPU: microbatch size and
+candidate order do not change a candidate's score.
+
+Tolerance: max |gpu - oracle| / RMS(oracle scores) <= 2e-2 (bf16) and
+<= 1e-4 (fp32)."""
+import numpy as np
+import pytest
+
+import hstu_workloads as hw
+from oracle import hstu_oracle as O
+from gpu_util import TOL, relerr, run_rank, runner_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from hstu_sequential_transducer_layer_b200.build import build
+    build()
+
+
+def _oracle_scores(w, users=None, microbatch=None):
+    return O.mfalcon_rank(w.X, w.offsets, w.timestamps, w.candidates, w.cand_offsets,
+                          w.request_ts, microbatch or w.microbatch, w.head_vec, w.weights, w.dims,
+                          users=users)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_mfalcon_small_bf16(D):
+    dims = hw.LayerDims(128, 2, D, D, 64, 128, 3, 2, 1e-6, hw.BF16)
+    # users: long history, empty history, history with no candidates, short history
+    w = hw.custom(f"mf{D}", [300, 0, 50, 129], dims, n_layers=2, seed=60 + D,
+                  cands_per_user=[200, 3, 0, 130], microbatch=64)
+    got, _ = run_rank(w)
+    ref = _oracle_scores(w)
+    err = relerr(got, ref)
+    print("mfalcon small", D, err)
+    assert err <= TOL[hw.BF16]
+
+
+def test_mfalcon_fp32():
+    dims = hw.LayerDims(64, 2, 32, 32, 32, 32, 3, 0, 1e-6, hw.FP32)
+    w = hw.custom("mf32", [17, 0, 40], dims, n_layers=2, seed=70, init="normal",
+                  cands_per_user=[5, 2, 9], microbatch=4)
+    got, _ = run_rank(w)
+    ref = _oracle_scores(w)
+    assert relerr(got, ref) <= TOL[hw.FP32]
+
+
+def test_mfalcon_request_time_default_and_explicit():
+    dims = hw.LayerDims(128, 2, 64, 64, 64, 128, 3, 2, 1e-6, hw.BF16)
+    w = hw.custom("mfreq", [100, 33], dims, n_layers=1, seed=71, cands_per_user=[10, 7],
+                  microbatch=8)
+    got_default, r = run_rank(w, request_ts=None)          # NULL: last history timestamp
+    got_last, _ = run_rank(w, runner=r)                    # explicit, equal to the last one
+    assert np.array_equal(got_default, got_last)
+    req = w.request_ts + np.array([86400, 5])
+    got_late, _ = run_rank(w, runner=r, request_ts=req)
+    ref = O.mfalcon_rank(w.X, w.offsets, w.timestamps, w.candidates, w.cand_offsets, req,
+                         w.microbatch, w.head_vec, w.weights, dims)
+    assert relerr(got_late, ref) <= TOL[hw.BF16]
+
+
+def test_mfalcon_microbatch_invariance_bitwise():
+    dims = hw.LayerDims(128, 2, 64, 64, 64, 128, 3, 2, 1e-6, hw.BF16)
+    w = hw.custom("mfmb", [150, 70], dims, n_layers=2, seed=72, cands_per_user=[40, 23],
+                  microbatch=40)
+    ref, r = run_rank(w, microbatch=40)
+    for mb in (1, 7, 16, 1000):
+        got, _ = run_rank(w, microbatch=mb, runner=r)
+        assert np.array_equal(got, ref), mb
+
+
+def test_mfalcon_candidate_permutation_and_drop_bitwise():
+    dims = hw.LayerDims(128, 2, 64, 64, 64, 128, 3, 2, 1e-6, hw.BF16)
+    w = hw.custom("mfperm", [150, 70], dims, n_layers=2, seed=73, cands_per_user=[40, 23],
+                  microbatch=16)
+    ref, r = run_rank(w)
+    perm = np.arange(63)
+    perm[40:] = perm[40:][::-1]
+    perm[:40] = np.random.default_rng(0).permutation(40)
+    got, _ = run_rank(w, runner=r, candidates=w.candidates[perm])
+    assert np.array_equal(got, ref[perm])
+    keep = np.r_[0:5, 40:41]
+    got, _ = run_rank(w, runner=r, candidates=w.candidates[keep],
+                      cand_offsets=np.array([0, 5, 6]))
+    assert np.array_equal(got, ref[keep])
+
+
+def test_mfalcon_workload_sampled_users():
+    """The full M-FALCON workload (32 users, 1024 candidates each, 3 layers,
+    d=512) on the GPU in the bench's launch configuration; the oracle scores
+    every candidate of two users (the longest and the shortest history)."""
+    w = hw.mfalcon(0)
+    got, _ = run_rank(w)
+    lens = w.lengths
+    users = [int(np.argmax(lens)), int(np.argmin(lens))]
+    ref = _oracle_scores(w, users=users)
+    for b in users:
+        cs, ce = int(w.cand_offsets[b]), int(w.cand_offsets[b + 1])
+        err = relerr(got[cs:ce], ref[cs:ce])
+        print("mfalcon user", b, lens[b], err)
+        assert err <= TOL[hw.BF16]
