@@ -86,19 +86,62 @@ cudaError_t gemm(const Ctx& c, const GemmCall& g, int kid_tc, int kid_simt) {
   return c.bf16 ? launch_gemm_tc(g, c.s, kid_tc) : launch_gemm_simt_f32(g, c.s, kid_simt);
 }
 
-// f1 (all columns, or only the V and K columns when kv_only)
-cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const void* X, int64_t rows_cap,
-                   const int64_t* rows_dev, void* f1, bool kv_only) {
+// Operands of one f1 / f2 on the tensor-core path: fp16 copies of the
+// weights live in the workspace (W1 of layers >= 1, every W2); layer 0's f1
+// multiplies the caller's bf16 X by the caller's bf16 W1 directly.
+struct LayerOps {
+  const void* W1;
+  int w1_f16;
+  const void* W2;
+};
+
+LayerOps layer_ops(const Ctx& c, const hstu_layer_weights& w, const Layout& L, void* ws, int l,
+                   int n_layers) {
+  LayerOps o{w.W1, 0, w.W2};
+  if (!c.bf16) return o;
+  const size_t F = c.F, dm = c.d.d_model, hdv = c.hdv;
+  uint8_t* base = at<uint8_t>(ws, L.w16) + (size_t)l * (F * dm + dm * hdv) * 2;
+  if (l > 0) {
+    o.W1 = base;
+    o.w1_f16 = 1;
+  }
+  o.W2 = base + F * dm * 2;
+  (void)n_layers;
+  return o;
+}
+
+// fp16 copies of the weights the call needs (W1 of layers >= 1, every W2).
+cudaError_t convert_weights(const Ctx& c, const hstu_layer_weights* w, int n_layers,
+                            const Layout& L, void* ws) {
+  if (!c.bf16) return cudaSuccess;
+  const int64_t F = c.F, dm = c.d.d_model, hdv = c.hdv;
+  for (int l = 0; l < n_layers; ++l) {
+    LayerOps o = layer_ops(c, w[l], L, ws, l, n_layers);
+    cudaError_t e;
+    if (l > 0 && (e = launch_bf16_to_f16(w[l].W1, const_cast<void*>(o.W1), F * dm, c.s)) != cudaSuccess)
+      return e;
+    if ((e = launch_bf16_to_f16(w[l].W2, const_cast<void*>(o.W2), dm * hdv, c.s)) != cudaSuccess)
+      return e;
+  }
+  return cudaSuccess;
+}
+
+// f1 (all columns, or only the V and K columns when kv_only); the output is
+// fp16 on the tensor-core path.
+cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, const void* X,
+                   int a_f16, int64_t rows_cap, const int64_t* rows_dev, void* f1, bool kv_only) {
   GemmCall g{};
   g.A = X;
   g.lda = c.d.d_model;
-  g.W = w.W1;
+  g.W = ops.W1;
   g.ldw = c.d.d_model;
+  g.ab_f16 = a_f16;
   g.M_cap = rows_cap;
   g.M_dev = rows_dev;
   g.K = c.d.d_model;
   g.bias = w.b1;
   g.out = f1;
+  g.out_f16 = 1;
   g.ldo = c.F;
   g.epi = EPI_SILU;
   g.status = c.status;
@@ -116,25 +159,39 @@ cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const void* X, int
   return gemm(c, g, K_GEMM_F1, K_SIMT_GEMM_F1);
 }
 
-cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const void* Z, const void* X,
-                   int64_t rows_cap, const int64_t* rows_dev, void* out) {
+// f2 + bias + residual.  resid_f32: the residual is the fp32 stream (else the
+// caller's bf16 rows); out16 (fp16 copy, or the caller's bf16 output when
+// out16_bf16) and out32 (fp32 stream) may each be null.  Each output element
+// is read (residual) and written by the same thread, so the fp32 stream is
+// updated in place.
+cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, const void* Z,
+                   const void* resid, bool resid_f32, int64_t rows_cap, const int64_t* rows_dev,
+                   void* out16, bool out16_bf16, float* out32) {
   GemmCall g{};
   g.A = Z;
   g.lda = c.hdv;
-  g.W = w.W2;
+  g.W = ops.W2;
   g.ldw = c.hdv;
+  g.ab_f16 = 1;
   g.M_cap = rows_cap;
   g.M_dev = rows_dev;
   g.N = c.d.d_model;
   g.K = c.hdv;
   g.n_off = 0;
   g.bias = w.b2;
-  g.out = out;
   g.ldo = c.d.d_model;
-  g.resid = X;
+  g.resid = resid;
   g.ldr = c.d.d_model;
   g.epi = EPI_RESID;
   g.status = c.status;
+  if (c.bf16) {
+    g.out = out16;
+    g.out_f16 = out16_bf16 ? 0 : 1;
+    g.out32 = out32;
+    g.resid_f32 = resid_f32 ? 1 : 0;
+  } else {  // fp32 layers: everything is already fp32; `out` is the fp32 destination
+    g.out = out16 ? out16 : out32;
+  }
   return gemm(c, g, K_GEMM_F2, K_SIMT_GEMM_F2);
 }
 
@@ -163,11 +220,13 @@ cudaError_t attn(const Ctx& c, const AttnCall& a) {
   return c.bf16 ? launch_attn_tc(a, c.s) : launch_attn_simt_f32(a, c.s);
 }
 
-// One causal layer over the jagged rows described by `off`.
-cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, int64_t B, int64_t T,
-                      const int64_t* off, const void* X, void* out, void* f1, void* O, void* Z,
+// One causal layer over the jagged rows described by `off`: f1 reads `A`,
+// f2 adds `resid` and writes out16 / out32 (see run_f2).
+cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, int64_t B,
+                      int64_t T, const int64_t* off, const void* A, int a_f16, const void* resid,
+                      bool resid_f32, void* out16, bool out16_bf16, float* out32, void* f1,
                       const Layout& L, void* ws) {
-  cudaError_t e = run_f1(c, w, X, T, nullptr, f1, false);
+  cudaError_t e = run_f1(c, w, ops, A, a_f16, T, nullptr, f1, false);
   if (e != cudaSuccess) return e;
   AttnCall a = attn_common(c, w, B);
   a.mode = 0;
@@ -181,13 +240,14 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, int64_t B, int6
   a.kv_buf = f1;
   a.kv_rows_cap = T;
   a.t_rel = at<int32_t>(ws, L.t_rel);
-  a.O = O;
+  a.O = at<void>(ws, L.o);
   e = attn(c, a);
   if (e != cudaSuccess) return e;
-  e = launch_ln_gate(c.d.dtype, O, f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps, Z, c.hdv, T,
-                     nullptr, c.status, c.s);
+  e = launch_ln_gate(c.d.dtype, at<void>(ws, L.o), f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps,
+                     at<void>(ws, L.z), c.hdv, T, nullptr, c.status, c.s);
   if (e != cudaSuccess) return e;
-  return run_f2(c, w, Z, X, T, nullptr, out);
+  return run_f2(c, w, ops, at<void>(ws, L.z), resid, resid_f32, T, nullptr, out16, out16_bf16,
+                out32);
 }
 
 hstu_status finish(cudaError_t e) {
@@ -217,14 +277,20 @@ hstu_status stack_impl(const hstu_layer_desc* desc, int32_t n_layers,
                   c.hdr, c.s);
   if (T == 0) return finish(cudaSuccess);
   launch_time_rel(offsets, B, timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
-  void* xtmp = at<void>(ws, L.xtmp);
-  const void* in = X;
-  cudaError_t e = cudaSuccess;
+  // Between layers the residual stream stays fp32 (xres, updated in place);
+  // the tensor-core path also keeps an fp16 copy (xh) as the next f1's operand.
+  float* xres = at<float>(ws, L.xres);
+  void* xh = at<void>(ws, L.xh);
+  cudaError_t e = convert_weights(c, weights, n_layers, L, ws);
   for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
-    void* dst = ((n_layers - 1 - l) % 2 == 0) ? out : xtmp;
-    e = run_layer(c, weights[l], B, T, offsets, in, dst, at<void>(ws, L.f1), at<void>(ws, L.o),
-                  at<void>(ws, L.z), L, ws);
-    in = dst;
+    const bool first = l == 0, last = l == n_layers - 1;
+    const LayerOps ops = layer_ops(c, weights[l], L, ws, l, n_layers);
+    const void* A = first ? X : (c.bf16 ? xh : (const void*)xres);
+    const void* resid = first ? X : (const void*)xres;
+    void* o16 = last ? out : (c.bf16 ? xh : nullptr);
+    float* o32 = last ? nullptr : xres;
+    e = run_layer(c, weights[l], ops, B, T, offsets, A, first ? 0 : 1, resid, !first, o16, last,
+                  o32, at<void>(ws, L.f1), L, ws);
   }
   return finish(e);
 }
@@ -302,19 +368,22 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
   // ---- history pass: every layer's f1 output (and so its K/V) is kept
   launch_schedule(hist_offsets, B, T, max_len, desc->n_heads, at<AttnItem>(ws, L.items),
                   L.item_cap, c.hdr, c.s);
-  cudaError_t e = cudaSuccess;
-  if (T > 0) {
+  cudaError_t e = convert_weights(c, weights, n_layers, L, ws);
+  float* xres = at<float>(ws, L.xres);
+  void* xh = at<void>(ws, L.xh);
+  if (T > 0 && e == cudaSuccess) {
     launch_time_rel(hist_offsets, B, hist_timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
-    const void* in = history;
     for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
-      if (l == n_layers - 1) {
-        e = run_f1(c, weights[l], in, T, nullptr, f1_of(l), true);
+      const bool first = l == 0;
+      const LayerOps ops = layer_ops(c, weights[l], L, ws, l, n_layers);
+      const void* A = first ? history : (c.bf16 ? xh : (const void*)xres);
+      if (l == n_layers - 1) {  // the last layer's history rows only serve as K and V
+        e = run_f1(c, weights[l], ops, A, first ? 0 : 1, T, nullptr, f1_of(l), true);
         break;
       }
-      void* dst = at<void>(ws, (l % 2 == 0) ? L.xh0 : L.xh1);
-      e = run_layer(c, weights[l], B, T, hist_offsets, in, dst, f1_of(l), at<void>(ws, L.o),
-                    at<void>(ws, L.z), L, ws);
-      in = dst;
+      e = run_layer(c, weights[l], ops, B, T, hist_offsets, A, first ? 0 : 1,
+                    first ? history : (const void*)xres, !first, c.bf16 ? xh : nullptr, false,
+                    xres, f1_of(l), L, ws);
     }
   }
   if (e != cudaSuccess || total_cands == 0) return finish(e);
@@ -325,7 +394,9 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
   int64_t* mb_off = at<int64_t>(ws, L.mb_off);
   AttnItem* citems = at<AttnItem>(ws, L.c_items);
   int32_t* t_req_rel = at<int32_t>(ws, L.t_req_rel);
-  void* xc[2] = {at<void>(ws, L.xc0), at<void>(ws, L.xc1)};
+  float* xres_c = at<float>(ws, L.xres_c);
+  void* xb_c = at<void>(ws, L.xb_c);   // gathered candidate rows (caller dtype)
+  void* xh_c = at<void>(ws, L.xh_c);   // fp16 copy of the stream (tensor-core path)
   void* f1c = at<void>(ws, L.f1c);
   void* oc = at<void>(ws, L.oc);
   void* zc = at<void>(ws, L.zc);
@@ -335,11 +406,12 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
                    desc->n_heads, hist_timestamps, request_ts, mb_off, citems, L.cand_item_cap,
                    t_req_rel, c.hdr, c.s);
     e = launch_mb_gather(desc->dtype, candidates, desc->d_model, cand_offsets, mb_off, B, k,
-                         microbatch, xc[0], R, rows_dev, c.status, c.s);
+                         microbatch, xb_c, R, rows_dev, c.status, c.s);
     for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
-      void* in = xc[l % 2];
-      void* dst = xc[(l + 1) % 2];
-      e = run_f1(c, weights[l], in, R, rows_dev, f1c, false);
+      const bool first = l == 0, last = l == n_layers - 1;
+      const LayerOps ops = layer_ops(c, weights[l], L, ws, l, n_layers);
+      const void* A = first ? xb_c : (c.bf16 ? xh_c : (const void*)xres_c);
+      e = run_f1(c, weights[l], ops, A, first ? 0 : 1, R, rows_dev, f1c, false);
       if (e != cudaSuccess) break;
       AttnCall a = attn_common(c, weights[l], B);
       a.mode = 1;
@@ -361,11 +433,13 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
       e = launch_ln_gate(desc->dtype, oc, f1c, c.F, weights[l].ln_gamma, weights[l].ln_beta,
                          desc->ln_eps, zc, c.hdv, R, rows_dev, c.status, c.s);
       if (e != cudaSuccess) break;
-      e = run_f2(c, weights[l], zc, in, R, rows_dev, dst);
+      const void* resid = first ? xb_c : (const void*)xres_c;
+      void* o16 = (c.bf16 && !last) ? xh_c : nullptr;
+      e = run_f2(c, weights[l], ops, zc, resid, !first, R, rows_dev, o16, false, xres_c);
     }
     if (e == cudaSuccess)
-      e = launch_score(desc->dtype, xc[n_layers % 2], desc->d_model, head_vec, cand_offsets,
-                       mb_off, B, k, microbatch, scores, R, rows_dev, c.status, c.s);
+      e = launch_score(desc->dtype, xres_c, desc->d_model, head_vec, cand_offsets, mb_off, B, k,
+                       microbatch, scores, R, rows_dev, c.status, c.s);
   }
   return finish(e);
 }

@@ -18,7 +18,7 @@
 // through a 2-stage ring); warp 1 MMA issuer: S = Q K^T into one of two TMEM
 // buffers, then O += P V into a TMEM accumulator; warps 2-9 ("P warps", two
 // per TMEM lane quarter, each owning 64 of the 128 columns) read S with
-// tcgen05.ld, add the bias, apply SiLU, mask, round to bf16 and write P into
+// tcgen05.ld, add the bias, apply SiLU, mask, round to fp16 and write P into
 // shared memory in the 128-byte-swizzled K-major layout the MMA reads.  At
 // the end of an item the P warps read O, scale by 1/n (and, for candidates,
 // add the self term) and store bf16.
@@ -49,9 +49,9 @@ struct AttnDev {
   const float* rab_time;
   int Np, Nt, Sp, St;
   int q_col, k_col, v_col;
-  const __nv_bfloat16* q_buf;  // for the candidate self term
+  const __half* q_buf;         // for the candidate self term (fp16 f1 output)
   int64_t ld_f1;
-  __nv_bfloat16* O;
+  float* O;                    // fp32: LayerNorm's mean subtraction would amplify bf16 rounding
   int64_t ldo;
   int* status;
 };
@@ -195,8 +195,8 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);  // V is MN-major
+      constexpr uint32_t IDESC_S = idesc_f16_f32(128, 128, 0, 0, 1);
+      constexpr uint32_t IDESC_O = idesc_f16_f32(128, D, 0, 1, 1);  // V is MN-major
       int kst = 0, litem = 0;
       uint32_t kph = 0, scount = 0, pcount = 0;
       bool ok = true, any = false;
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t v_base = smem_u32(sV + st * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_bf16_ss(tmem + C::O_COL,
+          tc_mma_f16_ss(tmem + C::O_COL,
                          sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                          sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
                          (jj > 0 || kk > 0) ? 1u : 0u);
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t k_base = smem_u32(sK + kst * C::TILE);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            tc_mma_bf16_ss(tmem + sb * 128,
+            tc_mma_f16_ss(tmem + sb * 128,
                            sdesc_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                            sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                            IDESC_S, kk > 0 ? 1u : 0u);
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free + sb);
         ++scount;
-        // ---- P = SiLU(S + bias), masked, bf16
+        // ---- P = SiLU(S + bias), masked, fp16
         uint32_t pk[32];
         if (MODE == MODE_SELF) {
           const bool diag = (j == w.qt);
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(320, 1)
             x += tb;
             float p = silu_fast(x);
             if (diag && (half * 64 + c > r)) p = 0.f;
-            if (c & 1) pk[c >> 1] = pack_bf16x2(__uint_as_float(pk[c >> 1]), p);
+            if (c & 1) pk[c >> 1] = pack_f16x2_sat(__uint_as_float(pk[c >> 1]), p);
             else pk[c >> 1] = __float_as_uint(p);
           }
         } else {
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int c = 0; c < 64; ++c) {
             float p = silu_fast(__uint_as_float(sr[c]) + win[c]);
             if (c >= limit) p = 0.f;
-            if (c & 1) pk[c >> 1] = pack_bf16x2(__uint_as_float(pk[c >> 1]), p);
+            if (c & 1) pk[c >> 1] = pack_f16x2_sat(__uint_as_float(pk[c >> 1]), p);
             else pk[c >> 1] = __float_as_uint(p);
           }
         }
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(320, 1)
       if (row_ok) {
         if (MODE == MODE_CAND) {
           // self term: the candidate attends to itself at distance 0, gap 0
-          const __nv_bfloat16* rowp = a.q_buf + (q0 + r) * a.ld_f1;
+          const __half* rowp = a.q_buf + (q0 + r) * a.ld_f1;
           const uint4* qp = reinterpret_cast<const uint4*>(rowp + a.q_col + w.head * D);
           const uint4* kp = reinterpret_cast<const uint4*>(rowp + a.k_col + w.head * D);
           float dot = 0.f;
@@ -443,10 +443,10 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              dot += bf16lo(qw[k]) * bf16lo(kw[k]) + bf16hi(qw[k]) * bf16hi(kw[k]);
+              dot += f16lo(qw[k]) * f16lo(kw[k]) + f16hi(qw[k]) * f16hi(kw[k]);
           }
           const float s_self = dot + __ldg(Rp) + __ldg(Rt);
-          const float p_self = __bfloat162float(__float2bfloat16(silu_fast(s_self)));
+          const float p_self = __half2float(__float2half_rn(silu_fast(s_self)));
           const uint4* vp =
               reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + half * (D / 2));
 #pragma unroll
@@ -455,21 +455,16 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              o[i * 8 + 2 * k] += p_self * bf16lo(vw[k]);
-              o[i * 8 + 2 * k + 1] += p_self * bf16hi(vw[k]);
+              o[i * 8 + 2 * k] += p_self * f16lo(vw[k]);
+              o[i * 8 + 2 * k + 1] += p_self * f16hi(vw[k]);
             }
           }
         }
-        uint4* op = reinterpret_cast<uint4*>(a.O + (q0 + r) * a.ldo + w.head * D + half * (D / 2));
+        float4* op = reinterpret_cast<float4*>(a.O + (q0 + r) * a.ldo + w.head * D + half * (D / 2));
 #pragma unroll
-        for (int i = 0; i < D / 16; ++i) {
-          uint4 v;
-          v.x = pack_bf16x2(o[8 * i + 0] * inv_n, o[8 * i + 1] * inv_n);
-          v.y = pack_bf16x2(o[8 * i + 2] * inv_n, o[8 * i + 3] * inv_n);
-          v.z = pack_bf16x2(o[8 * i + 4] * inv_n, o[8 * i + 5] * inv_n);
-          v.w = pack_bf16x2(o[8 * i + 6] * inv_n, o[8 * i + 7] * inv_n);
-          op[i] = v;
-        }
+        for (int i = 0; i < D / 8; ++i)
+          op[i] = make_float4(o[4 * i + 0] * inv_n, o[4 * i + 1] * inv_n, o[4 * i + 2] * inv_n,
+                              o[4 * i + 3] * inv_n);
       }
     }
   }
@@ -502,12 +497,12 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   if (c.item_cap <= 0 || c.q_rows_cap <= 0) return cudaSuccess;
   CUtensorMap tq, tkv;
   const uint64_t F = (uint64_t)c.ld_f1;
-  if (!encode_tmap_2d_bf16(&tq, c.q_buf, (uint64_t)c.q_rows_cap, F, F * 2, 64, 128))
+  if (!encode_tmap_2d(&tq, c.q_buf, (uint64_t)c.q_rows_cap, F, F * 2, 64, 128, true))
     return cudaErrorInvalidValue;
   // With no history rows there is nothing to load from the KV buffer; any
   // valid map will do (no KV tile is ever requested).
   if (c.kv_rows_cap > 0) {
-    if (!encode_tmap_2d_bf16(&tkv, c.kv_buf, (uint64_t)c.kv_rows_cap, F, F * 2, 64, 128))
+    if (!encode_tmap_2d(&tkv, c.kv_buf, (uint64_t)c.kv_rows_cap, F, F * 2, 64, 128, true))
       return cudaErrorInvalidValue;
   } else {
     tkv = tq;
@@ -530,9 +525,9 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   ad.q_col = c.q_col;
   ad.k_col = c.k_col;
   ad.v_col = c.v_col;
-  ad.q_buf = static_cast<const __nv_bfloat16*>(c.q_buf);
+  ad.q_buf = static_cast<const __half*>(c.q_buf);
   ad.ld_f1 = c.ld_f1;
-  ad.O = static_cast<__nv_bfloat16*>(c.O);
+  ad.O = static_cast<float*>(c.O);
   ad.ldo = c.ldo;
   ad.status = c.status;
   const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());

@@ -22,11 +22,15 @@ struct GemmDev {
   int64_t M_cap;
   const int64_t* M_dev;
   int N, K, n_off;
+  int ab_f16;                  // operand format: fp16 (1) or bf16 (0)
   const __nv_bfloat16* bias;
-  __nv_bfloat16* out;
+  void* out;                   // 16-bit output (fp16 if out_f16, else bf16); may be null
+  int out_f16;
   int64_t ldo;
-  const __nv_bfloat16* resid;
+  float* out32;                // EPI_RESID: optional fp32 copy of the output (same ldo)
+  const void* resid;           // EPI_RESID: residual, bf16 or fp32 (resid_f32)
   int64_t ldr;
+  int resid_f32;
   int* status;
 };
 
@@ -60,8 +64,20 @@ DEVI void gemm_epilogue_store(const GemmDev& g, int64_t row, bool valid, int col
   if (EPI == EPI_SILU) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
+  } else if (g.resid_f32) {
+    const float4* rp = reinterpret_cast<const float4*>(
+        static_cast<const float*>(g.resid) + row * g.ldr + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 rr = rp[i];
+      v[4 * i + 0] += rr.x;
+      v[4 * i + 1] += rr.y;
+      v[4 * i + 2] += rr.z;
+      v[4 * i + 3] += rr.w;
+    }
   } else {
-    const uint4* rp = reinterpret_cast<const uint4*>(g.resid + row * g.ldr + col);
+    const uint4* rp = reinterpret_cast<const uint4*>(
+        static_cast<const __nv_bfloat16*>(g.resid) + row * g.ldr + col);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint4 rr = rp[i];
@@ -73,15 +89,23 @@ DEVI void gemm_epilogue_store(const GemmDev& g, int64_t row, bool valid, int col
       }
     }
   }
-  uint4* op = reinterpret_cast<uint4*>(g.out + row * g.ldo + col);
+  if (EPI == EPI_RESID && g.out32) {
+    float4* op = reinterpret_cast<float4*>(g.out32 + row * g.ldo + col);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 o;
-    o.x = pack_bf16x2(v[i * 8 + 0], v[i * 8 + 1]);
-    o.y = pack_bf16x2(v[i * 8 + 2], v[i * 8 + 3]);
-    o.z = pack_bf16x2(v[i * 8 + 4], v[i * 8 + 5]);
-    o.w = pack_bf16x2(v[i * 8 + 6], v[i * 8 + 7]);
-    op[i] = o;
+    for (int i = 0; i < 8; ++i) op[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  if (g.out) {
+    uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) + row * g.ldo + col);
+    const int f16 = g.out_f16;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 o;
+      o.x = pack16(f16, v[i * 8 + 0], v[i * 8 + 1]);
+      o.y = pack16(f16, v[i * 8 + 2], v[i * 8 + 3]);
+      o.z = pack16(f16, v[i * 8 + 4], v[i * 8 + 5]);
+      o.w = pack16(f16, v[i * 8 + 6], v[i * 8 + 7]);
+      op[i] = o;
+    }
   }
 }
 
@@ -178,7 +202,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(128, BN, 0, 0);
+      const uint32_t IDESC = idesc_f16_f32(128, BN, 0, 0, g.ab_f16);
       int stage = 0, local = 0;
       uint32_t ph = 0;
       bool ok = true, issued_any = false;
@@ -201,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t b0 = a0 + C::A_BYTES;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma_bf16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
+            tc_mma_f16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
                            sdesc_sw128(b0 + k * 32, 16, 1024), IDESC, (kb | k) != 0);
           tc_commit(empty + stage);
           issued_any = true;
@@ -274,10 +298,11 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   if (c.N % 256 == 0 && mt * (c.N / 256) >= 2 * sms) BN = 256;
   else if (c.N % 128 == 0) BN = 128;
   CUtensorMap ta, tb;
-  if (!encode_tmap_2d_bf16(&ta, c.A, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.lda * 2, 64, 128))
+  const bool f16 = c.ab_f16 != 0;
+  if (!encode_tmap_2d(&ta, c.A, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.lda * 2, 64, 128, f16))
     return cudaErrorInvalidValue;
-  if (!encode_tmap_2d_bf16(&tb, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K,
-                           (uint64_t)c.ldw * 2, 64, (uint32_t)BN))
+  if (!encode_tmap_2d(&tb, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K, (uint64_t)c.ldw * 2, 64,
+                      (uint32_t)BN, f16))
     return cudaErrorInvalidValue;
   GemmDev gd;
   gd.M_cap = c.M_cap;
@@ -285,11 +310,15 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   gd.N = c.N;
   gd.K = c.K;
   gd.n_off = c.n_off;
+  gd.ab_f16 = c.ab_f16;
   gd.bias = static_cast<const __nv_bfloat16*>(c.bias);
-  gd.out = static_cast<__nv_bfloat16*>(c.out);
+  gd.out = c.out;
+  gd.out_f16 = c.out_f16;
   gd.ldo = c.ldo;
-  gd.resid = static_cast<const __nv_bfloat16*>(c.resid);
+  gd.out32 = static_cast<float*>(c.out32);
+  gd.resid = c.resid;
   gd.ldr = c.ldr;
+  gd.resid_f32 = c.resid_f32;
   gd.status = c.status;
   const int64_t tiles = mt * (c.N / BN);
   const int grid = (int)std::min<int64_t>(tiles, sms);

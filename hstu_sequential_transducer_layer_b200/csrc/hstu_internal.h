@@ -30,7 +30,8 @@ enum KernelId : int32_t {
   K_SIMT_ATTN = 11,
   K_SIMT_GEMM_F2 = 12,
   K_SIMT_ATTN_CAND = 13,
-  K_NUM_KERNELS = 14
+  K_CONVERT = 14,
+  K_NUM_KERNELS = 15
 };
 const char* kernel_name(int id);
 
@@ -48,8 +49,9 @@ struct LaunchScope {
 int num_sms();
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).  Returns false if the driver call is unavailable/failed.
-bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                         uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+// 2-D map of a row-major 16-bit matrix (bf16, or fp16 if f16), 128-byte swizzle.
+bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool f16);
 
 // ---------------------------------------------------------------- workspace
 struct Header {           // first 256 bytes of every workspace
@@ -61,9 +63,11 @@ struct Header {           // first 256 bytes of every workspace
 };
 
 struct Layout {
-  size_t header, items, t_rel, f1, o, z, xtmp;            // layer / stack
-  size_t f1_cache, xh0, xh1;                              // M-FALCON history
-  size_t mb_off, c_items, t_req_rel, hist_n, xc0, xc1, f1c, oc, zc;  // candidates
+  size_t header, items, t_rel, f1, o, z;
+  size_t xres, xh;          // fp32 residual stream; fp16 copy feeding the next f1 (tensor-core path)
+  size_t w16;               // tensor-core path: fp16 copies of W1 (layers >= 1) and W2, per layer
+  size_t f1_cache;          // M-FALCON: every layer's f1 output (its K/V) for the history
+  size_t mb_off, c_items, t_req_rel, xres_c, xb_c, xh_c, f1c, oc, zc;  // candidate microbatch
   size_t total;
   int64_t item_cap, cand_item_cap, mb_cap;
 };
@@ -87,12 +91,16 @@ enum Epilogue { EPI_SILU = 0, EPI_RESID = 1 };
 struct GemmCall {
   const void* A;  int64_t lda;   // [M_cap, K] row stride in elements
   const void* W;  int64_t ldw;   // [N_total, K]
+  int ab_f16;                    // tensor-core path: A and W are fp16 (else bf16)
   int64_t M_cap;                 // rows allocated in A / out
   const int64_t* M_dev;          // actual rows (device), or null = M_cap
   int N, K, n_off;
-  const void* bias;              // [N_total]
-  void* out; int64_t ldo;        // written at columns n_off + n
+  const void* bias;              // [N_total] (bf16 on the tensor-core path)
+  void* out; int64_t ldo;        // written at columns n_off + n; may be null for EPI_RESID
+  int out_f16;                   // tensor-core path: `out` is fp16 (else bf16)
+  void* out32;                   // tensor-core EPI_RESID: optional fp32 copy of the output
   const void* resid; int64_t ldr;
+  int resid_f32;                 // tensor-core EPI_RESID: residual stored as fp32 (else bf16)
   int epi;
   int* status;
 };
@@ -127,6 +135,9 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
                            int64_t rows_cap, const int64_t* rows_dev, const int* status,
                            cudaStream_t s);
 
+// bf16 -> fp16 (round to nearest, saturating at +-65504), n elements.
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, cudaStream_t s);
+
 // M-FALCON microbatch plumbing.
 void launch_mb_plan(const int64_t* hist_off, const int64_t* cand_off, int64_t B, int64_t max_len,
                     int64_t max_cands, int k, int microbatch, int n_heads,
@@ -137,7 +148,7 @@ cudaError_t launch_mb_gather(int dtype, const void* cands, int64_t d, const int6
                              const int64_t* mb_off, int64_t B, int k, int microbatch,
                              void* xc, int64_t rows_cap, const int64_t* rows_dev,
                              const int* status, cudaStream_t s);
-cudaError_t launch_score(int dtype, const void* xc, int64_t d, const void* head_vec,
+cudaError_t launch_score(int dtype, const float* xc, int64_t d, const void* head_vec,
                          const int64_t* cand_off, const int64_t* mb_off, int64_t B, int k,
                          int microbatch, float* scores, int64_t rows_cap,
                          const int64_t* rows_dev, const int* status, cudaStream_t s);

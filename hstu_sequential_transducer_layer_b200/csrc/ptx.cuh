@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -152,8 +153,9 @@ DEVI void tc_commit(uint64_t* bar) {
       : "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulator.
-DEVI void tc_mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+// D[tmem] (+)= A[smem desc] * B[smem desc]; fp16 or bf16 inputs (per the
+// instruction descriptor), fp32 accumulator.
+DEVI void tc_mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -163,16 +165,17 @@ DEVI void tc_mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32
       : "memory");
 }
 
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, M x N tile.
-// a_mn / b_mn select MN-major (transposed) operands.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4)                       // D format: f32
-         | (1u << 7)                     // A format: bf16
-         | (1u << 10)                    // B format: bf16
-         | ((uint32_t)a_mn << 15)        // A major
-         | ((uint32_t)b_mn << 16)        // B major
-         | ((uint32_t)(N >> 3) << 17)    // N / 8
-         | ((uint32_t)(M >> 4) << 24);   // M / 16
+// Instruction descriptor of kind::f16: A and B both fp16 (f16 = 1) or both
+// bf16 (f16 = 0), fp32 D, M x N tile.  a_mn / b_mn select MN-major
+// (transposed) operands.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn, int f16) {
+  return (1u << 4)                            // D format: f32
+         | ((f16 ? 0u : 1u) << 7)             // A format: 0 f16, 1 bf16
+         | ((f16 ? 0u : 1u) << 10)            // B format
+         | ((uint32_t)a_mn << 15)             // A major
+         | ((uint32_t)b_mn << 16)             // B major
+         | ((uint32_t)(N >> 3) << 17)         // N / 8
+         | ((uint32_t)(M >> 4) << 24);        // M / 16
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle.  saddr: shared-window
@@ -223,8 +226,22 @@ DEVI uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// fp16 pair with saturation to +-65504 (no infinities from in-range math).
+DEVI uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+DEVI float f16lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu))); }
+DEVI float f16hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
 DEVI float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 DEVI float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+// A packed pair in either 16-bit format of the tensor-core path (f16 != 0: fp16).
+DEVI uint32_t pack16(int f16, float lo, float hi) {
+  return f16 ? pack_f16x2_sat(lo, hi) : pack_bf16x2(lo, hi);
+}
+DEVI float lo16(int f16, uint32_t v) { return f16 ? f16lo(v) : bf16lo(v); }
+DEVI float hi16(int f16, uint32_t v) { return f16 ? f16hi(v) : bf16hi(v); }
 
 // Log-linear bucket of a non-negative distance (see hstu.h).
 DEVI int log_bucket(int x, int S, int N) {

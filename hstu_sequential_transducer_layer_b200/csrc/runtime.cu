@@ -23,7 +23,7 @@ const char* kernel_name(int id) {
       "schedule",   "time_rel",   "gemm_f1_tc",      "attn_tc",
       "ln_gate",    "gemm_f2_tc", "mb_plan",         "mb_gather",
       "attn_cand_tc", "score",    "gemm_f1_simt_f32", "attn_simt_f32",
-      "gemm_f2_simt_f32", "attn_cand_simt_f32"};
+      "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 
@@ -73,15 +73,15 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                         uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool f16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows == 0 || cols == 0) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -93,7 +93,8 @@ static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, int64_t max_len,
                  int64_t total_cands, int64_t max_cands, int microbatch, Layout* L) {
   if (B < 0 || T < 0 || n_layers < 1 || total_cands < 0 || max_cands < 0) return false;
-  const size_t es = d.dtype == HSTU_BF16 ? 2 : 4;
+  const bool bf16 = d.dtype == HSTU_BF16;
+  const size_t es = bf16 ? 2 : 4;
   const size_t F = 2 * (size_t)d.n_heads * (d.d_v + d.d_qk);
   const size_t hdv = (size_t)d.n_heads * d.d_v;
   const size_t dm = (size_t)d.d_model;
@@ -115,24 +116,24 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
     L->f1_cache = take((size_t)n_layers * T * F * es);
     L->f1 = L->f1_cache;
   }
-  L->o = take((size_t)T * hdv * es);
+  L->o = take((size_t)T * hdv * 4);
   L->z = take((size_t)T * hdv * es);
-  L->xtmp = take((size_t)T * dm * es);
+  L->xres = take((size_t)T * dm * 4);
+  L->xh = bf16 ? take((size_t)T * dm * 2) : L->xres;
+  L->w16 = bf16 ? take((size_t)n_layers * (F * dm + dm * hdv) * 2) : 0;
   if (mf) {
     if (microbatch < 1) return false;
-    L->xh0 = L->xtmp;
-    L->xh1 = take((size_t)T * dm * es);
     int64_t cap = std::min<int64_t>(total_cands, B * (int64_t)microbatch);
     L->mb_cap = cap;
     L->cand_item_cap = ((cap + kTile - 1) / kTile + B) * (int64_t)d.n_heads;
     L->mb_off = take((size_t)(B + 1) * 8);
     L->c_items = take((size_t)L->cand_item_cap * sizeof(AttnItem));
     L->t_req_rel = take((size_t)B * 4);
-    L->hist_n = take((size_t)B * 4);
-    L->xc0 = take((size_t)cap * dm * es);
-    L->xc1 = take((size_t)cap * dm * es);
+    L->xres_c = take((size_t)cap * dm * 4);
+    L->xb_c = bf16 ? take((size_t)cap * dm * 2) : L->xres_c;
+    L->xh_c = bf16 ? take((size_t)cap * dm * 2) : L->xres_c;
     L->f1c = take((size_t)cap * F * es);
-    L->oc = take((size_t)cap * hdv * es);
+    L->oc = take((size_t)cap * hdv * 4);
     L->zc = take((size_t)cap * hdv * es);
   }
   (void)max_len;

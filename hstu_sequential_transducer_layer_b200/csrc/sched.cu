@@ -11,6 +11,7 @@
 //   * M-FALCON microbatch plan / gather / score (subsection '4. M-FALCONで
 //     候補間の履歴計算を共有する').
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <climits>
 
@@ -144,21 +145,28 @@ struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16(v); }
 };
 template <>
+struct Elem<__half> {
+  static __device__ __forceinline__ float ld(const __half* p) { return __half2float(*p); }
+  static __device__ __forceinline__ void st(__half* p, float v) {
+    *p = __float2half_rn(fminf(fmaxf(v, -65504.f), 65504.f));
+  }
+};
+template <>
 struct Elem<float> {
   static __device__ __forceinline__ float ld(const float* p) { return *p; }
   static __device__ __forceinline__ void st(float* p, float v) { *p = v; }
 };
 
-// One warp per row.  Vectorised path for bf16 rows of a multiple of 256
-// features (8 per lane per 16-byte load, up to 2048 features); otherwise
-// strided scalar loads (up to 2048 features).
+// One warp per row; O is fp32, U / gamma / beta / Z are the layer dtype.
+// Vectorised path for bf16 rows of a multiple of 256 features (8 per lane per
+// step, up to 2048 features); otherwise strided scalar accesses.
 constexpr int kLnMaxPerLane = 64;
 
-template <typename Tv, bool VEC>
+template <typename Tu, typename Tg, bool VEC>
 __global__ void __launch_bounds__(256)
-    k_ln_gate(const Tv* __restrict__ O, const Tv* __restrict__ f1, int64_t ld_f1,
-              const Tv* __restrict__ gamma, const Tv* __restrict__ beta, float eps,
-              Tv* __restrict__ Z, int hdv, int64_t rows_cap, const int64_t* rows_dev,
+    k_ln_gate(const float* __restrict__ O, const Tu* __restrict__ f1, int64_t ld_f1,
+              const Tg* __restrict__ gamma, const Tg* __restrict__ beta, float eps,
+              Tu* __restrict__ Z, int hdv, int64_t rows_cap, const int64_t* rows_dev,
               const int* status) {
   if (status && *status != HSTU_OK) return;
   int64_t rows = rows_cap;
@@ -167,30 +175,28 @@ __global__ void __launch_bounds__(256)
   const int64_t row = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5);
   if (row >= rows) return;
   float x[kLnMaxPerLane];
-  const Tv* orow = O + row * (int64_t)hdv;
-  const Tv* urow = f1 + row * ld_f1;  // U occupies the first h*d_v columns
-  Tv* zrow = Z + row * (int64_t)hdv;
+  const float* orow = O + row * (int64_t)hdv;
+  const Tu* urow = f1 + row * ld_f1;  // U occupies the first h*d_v columns
+  Tu* zrow = Z + row * (int64_t)hdv;
+  const int nch = hdv / 256;
   float sum = 0.f;
   if (VEC) {
-    const int nch = hdv / 256;
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane / 8; ++k) {
       if (k < nch) {
-        const uint4 v = *reinterpret_cast<const uint4*>(orow + (k * 32 + lane) * 8);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const float4* p = reinterpret_cast<const float4*>(orow + (k * 32 + lane) * 8);
+        const float4 a = p[0], b = p[1];
+        x[k * 8 + 0] = a.x; x[k * 8 + 1] = a.y; x[k * 8 + 2] = a.z; x[k * 8 + 3] = a.w;
+        x[k * 8 + 4] = b.x; x[k * 8 + 5] = b.y; x[k * 8 + 6] = b.z; x[k * 8 + 7] = b.w;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[k * 8 + 2 * e] = bf16lo(w[e]);
-          x[k * 8 + 2 * e + 1] = bf16hi(w[e]);
-          sum += x[k * 8 + 2 * e] + x[k * 8 + 2 * e + 1];
-        }
+        for (int e = 0; e < 8; ++e) sum += x[k * 8 + e];
       }
     }
   } else {
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane; ++k) {
       const int c = k * 32 + lane;
-      x[k] = c < hdv ? Elem<Tv>::ld(orow + c) : 0.f;
+      x[k] = c < hdv ? orow[c] : 0.f;
       sum += x[k];
     }
   }
@@ -199,7 +205,6 @@ __global__ void __launch_bounds__(256)
   const float mean = sum / (float)hdv;
   float ss = 0.f;
   if (VEC) {
-    const int nch = hdv / 256;
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane / 8; ++k)
       if (k < nch)
@@ -222,7 +227,6 @@ __global__ void __launch_bounds__(256)
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float rstd = rsqrtf(ss / (float)hdv + eps);
   if (VEC) {
-    const int nch = hdv / 256;
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane / 8; ++k) {
       if (k < nch) {
@@ -235,10 +239,11 @@ __global__ void __launch_bounds__(256)
         uint32_t out[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float z0 = ((x[k * 8 + 2 * e] - mean) * rstd * bf16lo(g[e]) + bf16lo(bb[e])) * bf16lo(u[e]);
+          const float z0 =
+              ((x[k * 8 + 2 * e] - mean) * rstd * bf16lo(g[e]) + bf16lo(bb[e])) * f16lo(u[e]);
           const float z1 =
-              ((x[k * 8 + 2 * e + 1] - mean) * rstd * bf16hi(g[e]) + bf16hi(bb[e])) * bf16hi(u[e]);
-          out[e] = pack_bf16x2(z0, z1);
+              ((x[k * 8 + 2 * e + 1] - mean) * rstd * bf16hi(g[e]) + bf16hi(bb[e])) * f16hi(u[e]);
+          out[e] = pack_f16x2_sat(z0, z1);
         }
         *reinterpret_cast<uint4*>(zrow + c0) = make_uint4(out[0], out[1], out[2], out[3]);
       }
@@ -248,9 +253,9 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < kLnMaxPerLane; ++k) {
       const int c = k * 32 + lane;
       if (c < hdv) {
-        const float z = ((x[k] - mean) * rstd * Elem<Tv>::ld(gamma + c) + Elem<Tv>::ld(beta + c)) *
-                        Elem<Tv>::ld(urow + c);
-        Elem<Tv>::st(zrow + c, z);
+        const float z = ((x[k] - mean) * rstd * Elem<Tg>::ld(gamma + c) + Elem<Tg>::ld(beta + c)) *
+                        Elem<Tu>::ld(urow + c);
+        Elem<Tu>::st(zrow + c, z);
       }
     }
   }
@@ -264,22 +269,48 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
   if (hdv > 32 * kLnMaxPerLane) return cudaErrorInvalidValue;
   LaunchScope ls(K_LN_GATE, s);
   const int grid = (int)((rows_cap + 7) / 8);
-  if (dtype == HSTU_BF16) {
-    using T = __nv_bfloat16;
+  const float* Of = static_cast<const float*>(O);
+  if (dtype == HSTU_BF16) {  // tensor-core path: U and Z fp16, gamma / beta bf16
+    using U = __half;
+    using G = __nv_bfloat16;
     if (hdv % 256 == 0)
-      k_ln_gate<T, true><<<grid, 256, 0, s>>>((const T*)O, (const T*)f1, ld_f1, (const T*)gamma,
-                                              (const T*)beta, eps, (T*)Z, hdv, rows_cap, rows_dev,
-                                              status);
+      k_ln_gate<U, G, true><<<grid, 256, 0, s>>>(Of, (const U*)f1, ld_f1, (const G*)gamma,
+                                                 (const G*)beta, eps, (U*)Z, hdv, rows_cap,
+                                                 rows_dev, status);
     else
-      k_ln_gate<T, false><<<grid, 256, 0, s>>>((const T*)O, (const T*)f1, ld_f1, (const T*)gamma,
-                                               (const T*)beta, eps, (T*)Z, hdv, rows_cap,
-                                               rows_dev, status);
+      k_ln_gate<U, G, false><<<grid, 256, 0, s>>>(Of, (const U*)f1, ld_f1, (const G*)gamma,
+                                                  (const G*)beta, eps, (U*)Z, hdv, rows_cap,
+                                                  rows_dev, status);
   } else {
     using T = float;
-    k_ln_gate<T, false><<<grid, 256, 0, s>>>((const T*)O, (const T*)f1, ld_f1, (const T*)gamma,
-                                             (const T*)beta, eps, (T*)Z, hdv, rows_cap, rows_dev,
-                                             status);
+    k_ln_gate<T, T, false><<<grid, 256, 0, s>>>(Of, (const T*)f1, ld_f1, (const T*)gamma,
+                                                (const T*)beta, eps, (T*)Z, hdv, rows_cap,
+                                                rows_dev, status);
   }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- bf16 -> fp16
+__global__ void k_bf16_to_f16(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n8) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = src[i];
+    uint4 o;
+    o.x = pack_f16x2_sat(bf16lo(v.x), bf16hi(v.x));
+    o.y = pack_f16x2_sat(bf16lo(v.y), bf16hi(v.y));
+    o.z = pack_f16x2_sat(bf16lo(v.z), bf16hi(v.z));
+    o.w = pack_f16x2_sat(bf16lo(v.w), bf16hi(v.w));
+    dst[i] = o;
+  }
+}
+
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  if (n % 8 != 0) return cudaErrorInvalidValue;
+  LaunchScope ls(K_CONVERT, s);
+  const int64_t n8 = n / 8;
+  const int grid = (int)std::min<int64_t>((n8 + 255) / 256, 8 * num_sms());
+  k_bf16_to_f16<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n8);
   return cudaGetLastError();
 }
 
@@ -457,7 +488,7 @@ cudaError_t launch_mb_gather(int dtype, const void* cands, int64_t d, const int6
 }
 
 template <typename Tv>
-__global__ void k_score(const Tv* __restrict__ xc, int64_t d, const Tv* __restrict__ w,
+__global__ void k_score(const float* __restrict__ xc, int64_t d, const Tv* __restrict__ w,
                         const int64_t* __restrict__ coff, const int64_t* __restrict__ mb_off,
                         int64_t B, int k, int bm, float* __restrict__ scores, int64_t rows_cap,
                         const int64_t* rows_dev, const int* status) {
@@ -467,7 +498,7 @@ __global__ void k_score(const Tv* __restrict__ xc, int64_t d, const Tv* __restri
   const int64_t r = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5);
   if (r >= rows) return;
   float acc = 0.f;
-  for (int64_t c = lane; c < d; c += 32) acc += Elem<Tv>::ld(xc + r * d + c) * Elem<Tv>::ld(w + c);
+  for (int64_t c = lane; c < d; c += 32) acc += xc[r * d + c] * Elem<Tv>::ld(w + c);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) {
@@ -476,7 +507,7 @@ __global__ void k_score(const Tv* __restrict__ xc, int64_t d, const Tv* __restri
   }
 }
 
-cudaError_t launch_score(int dtype, const void* xc, int64_t d, const void* head_vec,
+cudaError_t launch_score(int dtype, const float* xc, int64_t d, const void* head_vec,
                          const int64_t* cand_off, const int64_t* mb_off, int64_t B, int k,
                          int microbatch, float* scores, int64_t rows_cap,
                          const int64_t* rows_dev, const int* status, cudaStream_t s) {
@@ -484,14 +515,12 @@ cudaError_t launch_score(int dtype, const void* xc, int64_t d, const void* head_
   LaunchScope ls(K_SCORE, s);
   const int grid = (int)((rows_cap + 7) / 8);
   if (dtype == HSTU_BF16)
-    k_score<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)xc, d,
-                                                 (const __nv_bfloat16*)head_vec, cand_off, mb_off,
-                                                 B, k, microbatch, scores, rows_cap, rows_dev,
-                                                 status);
+    k_score<__nv_bfloat16><<<grid, 256, 0, s>>>(xc, d, (const __nv_bfloat16*)head_vec, cand_off,
+                                                 mb_off, B, k, microbatch, scores, rows_cap,
+                                                 rows_dev, status);
   else
-    k_score<float><<<grid, 256, 0, s>>>((const float*)xc, d, (const float*)head_vec, cand_off,
-                                        mb_off, B, k, microbatch, scores, rows_cap, rows_dev,
-                                        status);
+    k_score<float><<<grid, 256, 0, s>>>(xc, d, (const float*)head_vec, cand_off, mb_off, B, k,
+                                        microbatch, scores, rows_cap, rows_dev, status);
   return cudaGetLastError();
 }
 

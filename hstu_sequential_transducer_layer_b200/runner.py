@@ -79,14 +79,17 @@ class HSTURunner:
         return _b.hstu_read_status(self._ws, stream)
 
     def intermediates(self, B: int, T: int, max_len: int):
-        """Views of the f1 output, O and Z the last layer call left in the workspace."""
+        """Views of the f1 output, O (fp32) and Z that the last layer call left
+        in the workspace.  On the tensor-core (bf16) path the f1 output and Z
+        are stored in fp16; on the fp32 path in fp32."""
         f1o, oo, zo = _b.hstu_debug_offsets(self.desc, B, T, max_len)
         d = self.desc
         F = 2 * d.n_heads * (d.d_v + d.d_qk)
         hdv = d.n_heads * d.d_v
-        es = 2 if self.dtype == "bf16" else 4
+        t = self.torch
+        idt, es = (t.float16, 2) if self.dtype == "bf16" else (t.float32, 4)
         ws = self._ws
 
-        def view(off, cols):
-            return ws[off:off + T * cols * es].view(self.tdtype).view(T, cols)
-        return view(f1o, F), view(oo, hdv), view(zo, hdv)
+        def view(off, cols, dt, size):
+            return ws[off:off + T * cols * size].view(dt).view(T, cols)
+        return view(f1o, F, idt, es), view(oo, hdv, t.float32, 4), view(zo, hdv, idt, es)

@@ -19,6 +19,27 @@ def relerr(g, r) -> float:
     return float(np.max(np.abs(g - r))) / rms
 
 
+def ulp16(r, mant_bits=10):
+    """Unit in the last place of |r| for a 16-bit float with `mant_bits`
+    stored mantissa bits (fp16: 10, bf16: 7)."""
+    a = np.abs(np.asarray(r, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 1e-38)))
+    return np.exp2(e - mant_bits)
+
+
+def ulperr(g, r, mant_bits=10, abs_rel=1e-4) -> float:
+    """max |g - r| / (ulp(r) + abs_rel * RMS(r)): a stored 16-bit value within
+    one ulp of the exact result, plus an absolute floor for values near zero,
+    where the fp32 accumulation of the producing GEMM (error ~1e-6 of the
+    summed magnitudes) exceeds any ulp of the result."""
+    g = np.asarray(g, np.float64)
+    r = np.asarray(r, np.float64)
+    if not r.size:
+        return 0.0
+    rms = math.sqrt(float(np.mean(r * r)))
+    return float(np.max(np.abs(g - r) / (ulp16(r, mant_bits) + abs_rel * rms)))
+
+
 def rmserr(g, r) -> float:
     g = np.asarray(g, np.float64)
     r = np.asarray(r, np.float64)
