@@ -29,6 +29,7 @@ hstu_status check_desc(const hstu_layer_desc* d) {
   if (d->dtype == HSTU_BF16) {
     if (d->d_qk != d->d_v || (d->d_qk != 64 && d->d_qk != 128)) return HSTU_ERR_UNSUPPORTED;
     if (d->d_model % 64 != 0 || hdv % 64 != 0) return HSTU_ERR_UNSUPPORTED;
+    if (d->n_time_buckets > 256) return HSTU_ERR_UNSUPPORTED;  // one byte per time bucket
   } else {
     if (d->d_qk > 128 || d->d_v > 128 || d->d_qk % 4 || d->d_v % 4 || d->d_model % 4)
       return HSTU_ERR_UNSUPPORTED;
@@ -212,6 +213,8 @@ AttnCall attn_common(const Ctx& c, const hstu_layer_weights& w, int64_t B) {
   a.dqk = c.d.d_qk;
   a.dv = c.d.d_v;
   a.ldo = c.hdv;
+  a.work_next = &c.hdr->work_next;
+  a.work_done = &c.hdr->work_done;
   a.status = c.status;
   return a;
 }
@@ -240,6 +243,7 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
   a.kv_buf = f1;
   a.kv_rows_cap = T;
   a.t_rel = at<int32_t>(ws, L.t_rel);
+  a.tbuckets = at<uint32_t>(ws, L.tbuckets);
   a.O = at<void>(ws, L.o);
   e = attn(c, a);
   if (e != cudaSuccess) return e;
@@ -274,9 +278,13 @@ hstu_status stack_impl(const hstu_layer_desc* desc, int32_t n_layers,
   if (ws_bytes < L.total) return HSTU_ERR_WORKSPACE;
   Ctx c = make_ctx(*desc, ws, stream);
   launch_schedule(offsets, B, T, max_len, desc->n_heads, at<AttnItem>(ws, L.items), L.item_cap,
-                  c.hdr, c.s);
+                  at<int64_t>(ws, L.ubase), L.tile_cap, c.hdr, c.s);
   if (T == 0) return finish(cudaSuccess);
   launch_time_rel(offsets, B, timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
+  if (c.bf16)  // time buckets: computed once, shared by every head and layer
+    launch_time_buckets(offsets, B, at<int32_t>(ws, L.t_rel), at<int64_t>(ws, L.ubase),
+                        L.tile_cap, desc->time_sub_bits, desc->n_time_buckets,
+                        at<uint32_t>(ws, L.tbuckets), c.hdr, c.s);
   // Between layers the residual stream stays fp32 (xres, updated in place);
   // the tensor-core path also keeps an fp16 copy (xh) as the next f1's operand.
   float* xres = at<float>(ws, L.xres);
@@ -367,12 +375,16 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
 
   // ---- history pass: every layer's f1 output (and so its K/V) is kept
   launch_schedule(hist_offsets, B, T, max_len, desc->n_heads, at<AttnItem>(ws, L.items),
-                  L.item_cap, c.hdr, c.s);
+                  L.item_cap, at<int64_t>(ws, L.ubase), L.tile_cap, c.hdr, c.s);
   cudaError_t e = convert_weights(c, weights, n_layers, L, ws);
   float* xres = at<float>(ws, L.xres);
   void* xh = at<void>(ws, L.xh);
   if (T > 0 && e == cudaSuccess) {
     launch_time_rel(hist_offsets, B, hist_timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
+    if (c.bf16 && n_layers > 1)
+      launch_time_buckets(hist_offsets, B, at<int32_t>(ws, L.t_rel), at<int64_t>(ws, L.ubase),
+                          L.tile_cap, desc->time_sub_bits, desc->n_time_buckets,
+                          at<uint32_t>(ws, L.tbuckets), c.hdr, c.s);
     for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {
       const bool first = l == 0;
       const LayerOps ops = layer_ops(c, weights[l], L, ws, l, n_layers);

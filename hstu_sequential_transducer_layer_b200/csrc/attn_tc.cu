@@ -9,26 +9,32 @@
 // '4. M-FALCONで候補間の履歴計算を共有する': candidates attend to their user's
 // whole cached history and to themselves only.
 //
-// One work item = (user, 128-row query tile, head).  The host-side schedule
-// lists, for each item, only the KV tiles at or left of the causal diagonal,
-// longest items first, so fully masked tiles are never loaded or multiplied.
-// Because there is no softmax, KV tiles combine by plain accumulation in TMEM.
+// One work item = (user, 128-row query tile, head).  The schedule lists, for
+// each item, only the KV tiles at or left of the causal diagonal, so fully
+// masked tiles are never loaded or multiplied.  Items are taken dynamically
+// (one atomic counter per launch) in an order that keeps the q-tiles of one
+// (user, head) adjacent, so CTAs running at the same time read the same K/V
+// tiles from L2.  Because there is no softmax, KV tiles combine by plain
+// accumulation in TMEM.
 //
-// Roles (320 threads): warp 0 TMA producer (Q tile once per item, K/V tiles
-// through a 2-stage ring); warp 1 MMA issuer: S = Q K^T into one of two TMEM
-// buffers, then O += P V into a TMEM accumulator; warps 2-9 ("P warps", two
-// per TMEM lane quarter, each owning 64 of the 128 columns) read S with
-// tcgen05.ld, add the bias, apply SiLU, mask, round to fp16 and write P into
-// shared memory in the 128-byte-swizzled K-major layout the MMA reads.  At
-// the end of an item the P warps read O, scale by 1/n (and, for candidates,
-// add the self term) and store bf16.
+// Roles (320 threads): warp 0 fetches items and issues TMA loads (Q once per
+// item; K, V through a 2-stage ring); warp 1 issues the MMAs: S = Q K^T into
+// one of two TMEM buffers, then O += P V into a TMEM accumulator; warps 2-9
+// ("P warps", two per TMEM lane quarter, 64 of the 128 columns each) read S
+// with tcgen05.ld, add the bias, apply SiLU, mask, round to fp16 and write P
+// into shared memory in the 128-byte-swizzled K-major layout the MMA reads.
+// At the end of an item the P warps read O, scale by 1/n (and, for
+// candidates, add the self term) and store fp32.
 //
-// Bias evaluation per element: the position bias comes from a per-warp
-// window of the 95 distances this warp's 32 x 64 block spans (one shared
-// load); the time bias is held in a register and recomputed only when the
-// gap leaves the current bucket's range (timestamps are usually sorted, so
-// this happens a few times per row and tile).
+// Bias per element (causal self-attention): the position bias comes from a
+// per-warp window of the 95 distances its 32 x 64 block spans; the time
+// bucket comes precomputed (one byte per element, shared by all heads and
+// layers of a call) and indexes a per-warp copy of the head's table.  Both
+// tables hold half the bias so that y = s/2 + bias/2 feeds
+// SiLU(x) = y + y tanh(y) (x = 2y) directly.  For candidates the bias depends
+// only on the history column: one shared-memory broadcast per element.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <climits>
 
@@ -37,22 +43,23 @@
 namespace hstu {
 
 struct AttnDev {
-  int mode;
   const AttnItem* items;
   const int32_t* n_items;
   const int64_t* q_off;
   const int64_t* kv_off;
-  int64_t kv_rows;
   const int32_t* t_rel;
   const int32_t* t_req_rel;
+  const uint32_t* tbuckets;
   const float* rab_pos;
   const float* rab_time;
   int Np, Nt, Sp, St;
   int q_col, k_col, v_col;
   const __half* q_buf;         // for the candidate self term (fp16 f1 output)
   int64_t ld_f1;
-  float* O;                    // fp32: LayerNorm's mean subtraction would amplify bf16 rounding
+  float* O;                    // fp32: LayerNorm's mean subtraction would amplify rounding
   int64_t ldo;
+  int32_t* work_next;
+  int32_t* work_done;
   int* status;
 };
 
@@ -66,14 +73,17 @@ struct AttnCfg {
   static constexpr uint32_t K_OFF = Q_OFF + TILE;
   static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
   static constexpr uint32_t P_OFF = V_OFF + 2 * TILE;
-  static constexpr uint32_t WIN_OFF = P_OFF + P_BUFS * P_BYTES;
-  static constexpr uint32_t TJ_OFF = WIN_OFF + 8 * 96 * 4;
-  static constexpr uint32_t BAR_OFF = TJ_OFF + 8 * 64 * 4;
+  static constexpr uint32_t WIN_OFF = P_OFF + P_BUFS * P_BYTES;   // 8 warps x 96 floats
+  static constexpr uint32_t RT_OFF = WIN_OFF + 8 * 96 * 4;        // 8 warps x 256 floats
+  static constexpr uint32_t BAR_OFF = RT_OFF + 8 * 256 * 4;
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O
 };
 
 enum { MODE_SELF = 0, MODE_CAND = 1 };
+
+// y = x / 2 (score plus bias, halved); returns SiLU(x) = y + y tanh(y).
+DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(320, 1)
@@ -86,16 +96,19 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;    // [2]
-  uint64_t* kv_empty = bars + 4;   // [2]
-  uint64_t* s_full = bars + 6;     // [2]
-  uint64_t* s_free = bars + 8;     // [2]
-  uint64_t* p_full = bars + 10;    // [2]
-  uint64_t* p_free = bars + 12;    // [2]
+  uint64_t* kv_full = bars + 2;     // [2]
+  uint64_t* kv_empty = bars + 4;    // [2]
+  uint64_t* s_full = bars + 6;      // [2]
+  uint64_t* s_free = bars + 8;      // [2]
+  uint64_t* p_full = bars + 10;     // [2]
+  uint64_t* p_free = bars + 12;     // [2]
   uint64_t* o_full = bars + 14;
   uint64_t* o_free = bars + 15;
   uint64_t* drain = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* it_full = bars + 17;    // [2] item ring
+  uint64_t* it_empty = bars + 19;   // [2]
+  AttnItem* ring = reinterpret_cast<AttnItem*>(bars + 21);   // [2], 16 B each
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + 2);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
   int* s_nitems = s_go + 1;
@@ -115,6 +128,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(s_free + i, 8);
       mbar_init(p_full + i, 8);
       mbar_init(p_free + i, 1);
+      mbar_init(it_full + i, 1);
+      mbar_init(it_empty + i, 9);  // the MMA thread + 8 P warps
     }
     mbar_init(o_full, 1);
     mbar_init(o_free, 8);
@@ -144,13 +159,25 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sP = smem + C::P_OFF;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------ item fetch + TMA producer
     if (lane == 0) {
       int kst = 0, litem = 0;
-      uint32_t kph = 0, issued = 0, last_par = 0, q_issued = 0, q_par = 0;
+      uint32_t kph = 0, issued = 0, last_par = 0, q_issued = 0, q_par = 0, npub = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++litem) {
-        const AttnItem w = a.items[it];
+      for (;;) {
+        const int idx = atomicAdd(a.work_next, 1);
+        AttnItem w;
+        if (idx < n_items) w = a.items[idx];
+        else w = AttnItem{-1, 0, 0, 0, 0};
+        const int slot = npub & 1;
+        if (!mbar_wait(it_empty + slot, ((npub >> 1) & 1) ^ 1, ab, a.status)) {
+          ok = false;
+          break;
+        }
+        ring[slot] = w;
+        mbar_arrive(it_full + slot);  // release: the ring entry is visible to waiters
+        ++npub;
+        if (w.b < 0) break;
         const int q_row0 = (int)(a.q_off[w.b] + (int64_t)w.qt * 128);
         const int kv_row0 = (int)a.kv_off[w.b];
         if (!mbar_wait(q_empty, (litem & 1) ^ 1, ab, a.status)) {
@@ -184,8 +211,10 @@ __global__ void __launch_bounds__(320, 1)
             kph ^= 1;
           }
         }
+        if (!ok) break;
+        ++litem;
       }
-      if (!ok) {
+      if (!ok) {  // let every load already in flight land before the CTA exits
         AbortState tmp{0};
         for (int s = 0; s < 2; ++s)
           if ((issued >> s) & 1u) mbar_wait(kv_full + s, (last_par >> s) & 1u, &tmp, nullptr);
@@ -193,12 +222,12 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_f16_f32(128, 128, 0, 0, 1);
       constexpr uint32_t IDESC_O = idesc_f16_f32(128, D, 0, 1, 1);  // V is MN-major
       int kst = 0, litem = 0;
-      uint32_t kph = 0, scount = 0, pcount = 0;
+      uint32_t kph = 0, scount = 0, pcount = 0, ncon = 0;
       bool ok = true, any = false;
       const uint32_t q_base = smem_u32(sQ);
       auto issue_pv = [&](int jj, int st, int nkv) -> bool {
@@ -212,9 +241,9 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_f16_ss(tmem + C::O_COL,
-                         sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                         sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
-                         (jj > 0 || kk > 0) ? 1u : 0u);
+                        sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
         tc_commit(p_free + pb);
         tc_commit(kv_empty + st);
         if (jj == nkv - 1) tc_commit(o_full);
@@ -222,8 +251,14 @@ __global__ void __launch_bounds__(320, 1)
         any = true;
         return true;
       };
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++litem) {
-        const int nkv = a.items[it].nkv;
+      for (;;) {
+        const int slot = ncon & 1;
+        if (!mbar_wait(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
+        const AttnItem w = ring[slot];
+        mbar_arrive(it_empty + slot);
+        ++ncon;
+        if (w.b < 0) break;
+        const int nkv = w.nkv;
         if (!mbar_wait(q_full, litem & 1, ab, a.status)) {
           ok = false;
           break;
@@ -245,9 +280,9 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             tc_mma_f16_ss(tmem + sb * 128,
-                           sdesc_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                           sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                           IDESC_S, kk > 0 ? 1u : 0u);
+                          sdesc_sw128(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                          sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                          IDESC_S, kk > 0 ? 1u : 0u);
           tc_commit(s_full + sb);
           ++scount;
           any = true;
@@ -263,14 +298,12 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!ok) break;
         if (nkv > 0) {
-          if (!issue_pv(nkv - 1, prev, nkv)) {
-            ok = false;
-            break;
-          }
+          if (!issue_pv(nkv - 1, prev, nkv)) break;
         } else {
           tc_commit(o_full);  // nothing to accumulate: O is taken as zero
         }
         tc_commit(q_empty);
+        ++litem;
       }
       if (any) {
         tc_commit(drain);
@@ -279,50 +312,59 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ P warps
+    // ------------------------------------------------ P warps
     const int pw = warp - 2;         // 0..7
     const int q = warp & 3;          // TMEM lane quarter
     const int half = pw >> 2;        // which 64 of the 128 S columns
     const int r = q * 32 + lane;     // row inside the 128-row tile
     float* win = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 96;
-    int* tj = reinterpret_cast<int*>(smem + C::TJ_OFF) + pw * 64;
+    float* rt = reinterpret_cast<float*>(smem + C::RT_OFF) + pw * 256;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    uint32_t scount = 0, pcount = 0;
+    uint32_t scount = 0, pcount = 0, ncon = 0;
     int litem = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++litem) {
-      const AttnItem w = a.items[it];
+    for (;;) {
+      const int slot = ncon & 1;
+      if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
+      const AttnItem w = ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(it_empty + slot);
+      ++ncon;
+      if (w.b < 0) break;
       const int64_t kv0 = a.kv_off[w.b];
       const int n_kv = (int)(a.kv_off[w.b + 1] - kv0);           // history / sequence length
       const int64_t q0 = a.q_off[w.b] + (int64_t)w.qt * 128;
       const int n_q = (int)(a.q_off[w.b + 1] - a.q_off[w.b]);
-      const int rows_valid = min(128, n_q - w.qt * 128);
+      const int rows_valid = min(128, n_q - (int)w.qt * 128);
       const bool row_ok = r < rows_valid;
       const float inv_n = 1.0f / (float)max(n_kv, 1);
       const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
       const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
       int t_i = 0;
-      if (MODE == MODE_SELF) t_i = row_ok ? a.t_rel[kv0 + (int64_t)w.qt * 128 + r] : 0;
-      else t_i = a.t_req_rel[w.b];
-      int lo = 1, hi = 0;   // empty range: the first column computes the bucket
-      float tb = 0.f;
-      bool alive = true;
-      for (int j = 0; j < w.nkv && alive; ++j) {
-        // ---- per-warp bias tables for this tile
+      if (MODE == MODE_SELF) {
+        // this head's time-bias table, halved, in the warp's own slice
         __syncwarp();
+        for (int k = lane; k < a.Nt; k += 32) rt[k] = 0.5f * __ldg(Rt + k);
+      } else {
+        t_i = a.t_req_rel[w.b];
+      }
+      bool alive = true;
+      for (int j = 0; j < w.nkv; ++j) {
+        // ---- per-warp bias inputs for this tile
+        __syncwarp();
+        uint32_t bw[16];
         if (MODE == MODE_SELF) {
+          const uint32_t* tbw = a.tbuckets + (size_t)(w.tile0 + j) * kBucketTileWords +
+                                (half * 16) * 128 + r;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) bw[m] = __ldg(tbw + m * 128);
           const int base = (w.qt - j) * 128 + q * 32 - half * 64 - 63;
 #pragma unroll
           for (int u = 0; u < 3; ++u) {
             const int k = lane + 32 * u;
             if (k < 95) {
               const int dist = base + k;
-              win[k] = dist >= 0 ? __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
+              win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
             }
-          }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int jc = j * 128 + half * 64 + lane + 32 * u;
-            tj[lane + 32 * u] = jc < n_kv ? a.t_rel[kv0 + jc] : 0;
           }
         } else {
 #pragma unroll
@@ -334,7 +376,7 @@ __global__ void __launch_bounds__(320, 1)
               bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
                      __ldg(Rt + log_bucket(gap, a.St, a.Nt));
             }
-            win[lane + 32 * u] = bias;
+            win[lane + 32 * u] = 0.5f * bias;
           }
         }
         __syncwarp();
@@ -360,32 +402,38 @@ __global__ void __launch_bounds__(320, 1)
         // ---- P = SiLU(S + bias), masked, fp16
         uint32_t pk[32];
         if (MODE == MODE_SELF) {
-          const bool diag = (j == w.qt);
           const float* wr = win + lane + 63;
+          if (j == w.qt) {  // diagonal tile: causal mask j > i
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            float x = __uint_as_float(sr[c]) + wr[-c];
-            const int gap = t_i - tj[c];
-            if (gap < lo || gap >= hi) {
-              const int b = log_bucket(max(gap, 0), a.St, a.Nt);
-              lo = b == 0 ? INT_MIN : bucket_lo(b, a.St);
-              hi = b >= a.Nt - 1 ? INT_MAX : bucket_lo(b + 1, a.St);
-              tb = __ldg(Rt + b);
+            for (int c = 0; c < 64; c += 2) {
+              const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
+              const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
+              float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, wr[-c]) + rt[b0]);
+              float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, wr[-c - 1]) + rt[b1]);
+              if (half * 64 + c > r) p0 = 0.f;
+              if (half * 64 + c + 1 > r) p1 = 0.f;
+              pk[c >> 1] = pack_f16x2_sat(p0, p1);
             }
-            x += tb;
-            float p = silu_fast(x);
-            if (diag && (half * 64 + c > r)) p = 0.f;
-            if (c & 1) pk[c >> 1] = pack_f16x2_sat(__uint_as_float(pk[c >> 1]), p);
-            else pk[c >> 1] = __float_as_uint(p);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
+              const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
+              const float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, wr[-c]) + rt[b0]);
+              const float p1 =
+                  silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, wr[-c - 1]) + rt[b1]);
+              pk[c >> 1] = pack_f16x2_sat(p0, p1);
+            }
           }
         } else {
           const int limit = n_kv - j * 128 - half * 64;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            float p = silu_fast(__uint_as_float(sr[c]) + win[c]);
-            if (c >= limit) p = 0.f;
-            if (c & 1) pk[c >> 1] = pack_f16x2_sat(__uint_as_float(pk[c >> 1]), p);
-            else pk[c >> 1] = __float_as_uint(p);
+          for (int c = 0; c < 64; c += 2) {
+            float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, win[c]));
+            float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, win[c + 1]));
+            if (c >= limit) p0 = 0.f;
+            if (c + 1 >= limit) p1 = 0.f;
+            pk[c >> 1] = pack_f16x2_sat(p0, p1);
           }
         }
         // ---- write P (K-major, 128-byte swizzle: chunk m of row r at m ^ (r & 7))
@@ -466,6 +514,7 @@ __global__ void __launch_bounds__(320, 1)
           op[i] = make_float4(o[4 * i + 0] * inv_n, o[4 * i + 1] * inv_n, o[4 * i + 2] * inv_n,
                               o[4 * i + 3] * inv_n);
       }
+      ++litem;
     }
   }
   tc_fence_before();
@@ -474,6 +523,16 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0) {
+    // The last CTA to finish re-arms the work counter for the next launch
+    // (launches on one stream never overlap).
+    __threadfence();
+    if (atomicAdd(a.work_done, 1) == (int)gridDim.x - 1) {
+      atomicExch(a.work_next, 0);
+      atomicExch(a.work_done, 0);
+      __threadfence();
+    }
   }
 }
 
@@ -494,6 +553,7 @@ static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tk
 
 cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   if (c.dqk != c.dv || (c.dqk != 64 && c.dqk != 128)) return cudaErrorInvalidValue;
+  if (c.mode == MODE_SELF && c.Nt > 256) return cudaErrorInvalidValue;
   if (c.item_cap <= 0 || c.q_rows_cap <= 0) return cudaSuccess;
   CUtensorMap tq, tkv;
   const uint64_t F = (uint64_t)c.ld_f1;
@@ -508,14 +568,13 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
     tkv = tq;
   }
   AttnDev ad;
-  ad.mode = c.mode;
   ad.items = c.items;
   ad.n_items = c.n_items;
   ad.q_off = c.q_off;
   ad.kv_off = c.kv_off;
-  ad.kv_rows = c.kv_rows_cap;
   ad.t_rel = c.t_rel;
   ad.t_req_rel = c.t_req_rel;
+  ad.tbuckets = c.tbuckets;
   ad.rab_pos = c.rab_pos;
   ad.rab_time = c.rab_time;
   ad.Np = c.Np;
@@ -529,14 +588,16 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   ad.ld_f1 = c.ld_f1;
   ad.O = static_cast<float*>(c.O);
   ad.ldo = c.ldo;
+  ad.work_next = c.work_next;
+  ad.work_done = c.work_done;
   ad.status = c.status;
   const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());
   LaunchScope ls(c.mode == MODE_SELF ? K_ATTN : K_ATTN_CAND, s);
   if (c.mode == MODE_SELF)
     return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF>(tq, tkv, ad, grid, s)
-                     : launch_attn_inst<128, MODE_SELF>(tq, tkv, ad, grid, s);
+                       : launch_attn_inst<128, MODE_SELF>(tq, tkv, ad, grid, s);
   return c.dqk == 64 ? launch_attn_inst<64, MODE_CAND>(tq, tkv, ad, grid, s)
-                   : launch_attn_inst<128, MODE_CAND>(tq, tkv, ad, grid, s);
+                     : launch_attn_inst<128, MODE_CAND>(tq, tkv, ad, grid, s);
 }
 
 }  // namespace hstu

@@ -31,7 +31,8 @@ enum KernelId : int32_t {
   K_SIMT_GEMM_F2 = 12,
   K_SIMT_ATTN_CAND = 13,
   K_CONVERT = 14,
-  K_NUM_KERNELS = 15
+  K_TIME_BUCKETS = 15,
+  K_NUM_KERNELS = 16
 };
 const char* kernel_name(int id);
 
@@ -58,30 +59,50 @@ struct Header {           // first 256 bytes of every workspace
   int32_t status;         // hstu_status of the device checks
   int32_t n_items;        // attention work items of the history pass
   int32_t n_cand_items;   // attention work items of the current microbatch
-  int32_t pad0;
+  int32_t n_tiles;        // time-bucket tiles of the history pass
   int64_t mb_rows;        // rows of the current candidate microbatch
+  int32_t work_next;      // dynamic work counter of the running attention launch
+  int32_t work_done;      // CTAs of that launch that have finished
 };
 
 struct Layout {
-  size_t header, items, t_rel, f1, o, z;
+  size_t header, items, t_rel, ubase, tbuckets, f1, o, z;
   size_t xres, xh;          // fp32 residual stream; fp16 copy feeding the next f1 (tensor-core path)
   size_t w16;               // tensor-core path: fp16 copies of W1 (layers >= 1) and W2, per layer
   size_t f1_cache;          // M-FALCON: every layer's f1 output (its K/V) for the history
   size_t mb_off, c_items, t_req_rel, xres_c, xb_c, xh_c, f1c, oc, zc;  // candidate microbatch
   size_t total;
-  int64_t item_cap, cand_item_cap, mb_cap;
+  int64_t item_cap, cand_item_cap, mb_cap, tile_cap;
 };
 bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, int64_t max_len,
                  int64_t total_cands, int64_t max_cands, int microbatch, Layout* L);
 
 // ---------------------------------------------------------------- kernels
+// One attention work item: (user, 128-row query tile, head), the number of
+// 128-row KV tiles it reads, and (causal self-attention) the index of the
+// time-bucket tile of (user, query tile, KV tile 0).
 struct AttnItem {
-  int32_t b, qt, head, nkv;
+  int32_t b;
+  int16_t qt, head;
+  int32_t nkv;
+  int32_t tile0;
 };
+// A time-bucket tile: the bucket of t_i - t_j for 128 query rows x 128 KV
+// columns, one byte each, 4 consecutive columns per 32-bit word, stored
+// word-column-major ([32][128] words) so that a warp's 32 rows read 128
+// contiguous bytes.
+constexpr int kBucketTileWords = 32 * 128;
 
-// Validate offsets; build the causal work list (user, q-tile, head), longest first.
+// Validate offsets; build the causal work list (user, q-tile, head) grouped
+// by (user, head), longest users first, q-tiles longest first inside a group;
+// ubase[b] = first time-bucket tile of user b.
 void launch_schedule(const int64_t* offsets, int64_t B, int64_t T, int64_t max_len, int n_heads,
-                     AttnItem* items, int64_t item_cap, Header* hdr, cudaStream_t s);
+                     AttnItem* items, int64_t item_cap, int64_t* ubase, int64_t tile_cap,
+                     Header* hdr, cudaStream_t s);
+// Time-bucket tiles of every causal (q-tile, kv-tile) pair of the batch.
+void launch_time_buckets(const int64_t* offsets, int64_t B, const int32_t* t_rel,
+                         const int64_t* ubase, int64_t tile_cap, int St, int Nt,
+                         uint32_t* tbuckets, Header* hdr, cudaStream_t s);
 // Per-row timestamp relative to the user's first one (int32), with checks.
 void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64_t T,
                      int32_t* t_rel, Header* hdr, cudaStream_t s);
@@ -121,6 +142,8 @@ struct AttnCall {
   int q_col, k_col, v_col;         // column where head 0 of Q, K, V starts
   const int32_t* t_rel;            // [T_kv] int32 relative timestamps
   const int32_t* t_req_rel;        // CAND: [B] request time relative to the user's first
+  const uint32_t* tbuckets;        // SELF: time-bucket tiles
+  int32_t* work_next; int32_t* work_done;  // dynamic scheduling counters (header)
   const float* rab_pos; const float* rab_time;
   int Np, Nt, Sp, St, h, dqk, dv;
   void* O; int64_t ldo;

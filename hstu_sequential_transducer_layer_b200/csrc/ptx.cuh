@@ -220,7 +220,9 @@ DEVI float silu_fast(float x) {
   const float hx = 0.5f * x;
   return fmaf(hx, tanh_approx(hx), hx);
 }
-DEVI float silu_accurate(float x) { return x / (1.0f + __expf(-x)); }
+// x / (1 + e^-x) with the fast exponential and reciprocal (relative error of
+// a few fp32 ulps); saturates to -0 for x below about -88.
+DEVI float silu_accurate(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 DEVI uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -23,7 +23,7 @@ const char* kernel_name(int id) {
       "schedule",   "time_rel",   "gemm_f1_tc",      "attn_tc",
       "ln_gate",    "gemm_f2_tc", "mb_plan",         "mb_gather",
       "attn_cand_tc", "score",    "gemm_f1_simt_f32", "attn_simt_f32",
-      "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16"};
+      "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16", "time_buckets"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 
@@ -110,6 +110,11 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
   L->header = take(256);
   L->items = take((size_t)L->item_cap * sizeof(AttnItem));
   L->t_rel = take((size_t)T * 4);
+  // time-bucket tiles: sum over users of nq(nq+1)/2 <= (sum nq) * (max_q + 1) / 2
+  const int64_t max_q = (max_len + kTile - 1) / kTile;
+  L->tile_cap = bf16 ? ((T + kTile - 1) / kTile + B) * (max_q + 1) / 2 + 1 : 0;
+  L->ubase = take((size_t)(B + 1) * 8);
+  L->tbuckets = take((size_t)L->tile_cap * kBucketTileWords * 4);
   if (!mf) {
     L->f1 = take((size_t)T * F * es);
   } else {

@@ -24,15 +24,48 @@ constexpr int kSchedThreads = 1024;
 __device__ __forceinline__ void set_status(int* st, int code) { atomicCAS(st, 0, code); }
 
 // ---------------------------------------------------------------- schedule
+// Block-wide exclusive scan over users of v(b); writes out[0..B] (out[B] =
+// total) and returns the total.  All threads of the block must call it.
+template <typename F>
+__device__ long long block_scan_users(int64_t B, F v, int64_t* out, long long* s_part,
+                                      long long* s_carry) {
+  if (threadIdx.x == 0) *s_carry = 0;
+  __syncthreads();
+  for (int64_t b0 = 0; b0 <= B; b0 += blockDim.x) {
+    const int64_t b = b0 + threadIdx.x;
+    const long long x = b < B ? v(b) : 0;
+    s_part[threadIdx.x] = x;
+    __syncthreads();
+    for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+      const long long y = threadIdx.x >= (unsigned)o ? s_part[threadIdx.x - o] : 0;
+      __syncthreads();
+      s_part[threadIdx.x] += y;
+      __syncthreads();
+    }
+    if (b <= B) out[b] = *s_carry + s_part[threadIdx.x] - x;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) *s_carry += s_part[threadIdx.x];
+    __syncthreads();
+  }
+  return *s_carry;
+}
+
 __global__ void __launch_bounds__(kSchedThreads)
     k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t T, int64_t max_len, int h,
-               AttnItem* __restrict__ items, int64_t item_cap, Header* hdr) {
+               AttnItem* __restrict__ items, int64_t item_cap, int64_t* __restrict__ ubase,
+               int64_t tile_cap, Header* hdr) {
   __shared__ int s_bad;
-  __shared__ int s_count[1024];
-  __shared__ int s_start[1024];
+  __shared__ long long s_part[kSchedThreads];
+  __shared__ long long s_carry;
+  __shared__ long long s_cnt[kSchedThreads];
+  __shared__ long long s_start[kSchedThreads];
+  __shared__ long long s_base;
   if (threadIdx.x == 0) {
     hdr->status = HSTU_OK;
     hdr->n_items = 0;
+    hdr->n_tiles = 0;
+    hdr->work_next = 0;
+    hdr->work_done = 0;
     s_bad = 0;
     if (off[0] != 0 || off[B] != T) s_bad = 1;
   }
@@ -46,58 +79,59 @@ __global__ void __launch_bounds__(kSchedThreads)
     if (threadIdx.x == 0) hdr->status = HSTU_ERR_BAD_OFFSETS;
     return;
   }
-  // Work item (b, qt) needs qt + 1 KV tiles.  Level c = qt + 1 holds one item
-  // per user with at least c query tiles.  Levels are emitted longest first,
-  // users in order inside a level, heads innermost.
+  auto nq_of = [&](int64_t b) { return (off[b + 1] - off[b] + kTile - 1) / kTile; };
+  // first time-bucket tile of every user: prefix of nq (nq + 1) / 2
+  const long long tiles = block_scan_users(
+      B, [&](int64_t b) { const long long q = nq_of(b); return q * (q + 1) / 2; }, ubase, s_part,
+      &s_carry);
+  // Items grouped by (user, head): users with more q-tiles first (level c =
+  // nq, highest first), users in order inside a level, then heads, then
+  // q-tiles longest first.  Neighbouring items read the same K/V.
   const int levels = (int)((max_len + kTile - 1) / kTile);
-  // Chunks of blockDim levels, highest level first: every thread counts its
-  // level, thread 0 turns the counts into start positions, every thread then
-  // writes its level's items.
-  __shared__ long long s_base;
   if (threadIdx.x == 0) s_base = 0;
   __syncthreads();
   for (int c_hi = levels; c_hi >= 1; c_hi -= blockDim.x) {
-    const int c = c_hi - (int)threadIdx.x;  // this thread's level in the chunk
-    int cnt = 0;
+    const int c = c_hi - (int)threadIdx.x;
+    long long cnt = 0;
     if (c >= 1)
-      for (int64_t b = 0; b < B; ++b) {
-        const int64_t nq = (off[b + 1] - off[b] + kTile - 1) / kTile;
-        cnt += nq >= c;
-      }
-    s_count[threadIdx.x] = cnt;
+      for (int64_t b = 0; b < B; ++b) cnt += nq_of(b) == c;
+    s_cnt[threadIdx.x] = cnt * c * h;
     __syncthreads();
     if (threadIdx.x == 0) {
       long long acc = s_base;
       const int m = min((int)blockDim.x, c_hi);
       for (int i = 0; i < m; ++i) {
-        s_start[i] = (int)acc;
-        acc += s_count[i];
+        s_start[i] = acc;
+        acc += s_cnt[i];
       }
       s_base = acc;
     }
     __syncthreads();
     if (c >= 1) {
-      int64_t pos = s_start[threadIdx.x];
+      long long pos = s_start[threadIdx.x];
       for (int64_t b = 0; b < B; ++b) {
-        const int64_t nq = (off[b + 1] - off[b] + kTile - 1) / kTile;
-        if (nq >= c) {
-          for (int hh = 0; hh < h; ++hh) {
-            const int64_t idx = pos * h + hh;
-            if (idx < item_cap) items[idx] = AttnItem{(int32_t)b, c - 1, hh, c};
-          }
-          ++pos;
-        }
+        if (nq_of(b) != c) continue;
+        for (int hh = 0; hh < h; ++hh)
+          for (int qt = c - 1; qt >= 0; --qt, ++pos)
+            if (pos < item_cap)
+              items[pos] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, qt + 1,
+                                    (int32_t)(ubase[b] + (long long)qt * (qt + 1) / 2)};
       }
     }
     __syncthreads();
   }
-  if (threadIdx.x == 0) hdr->n_items = (int32_t)(s_base * h < item_cap ? s_base * h : item_cap);
+  if (threadIdx.x == 0) {
+    hdr->n_items = (int32_t)(s_base < item_cap ? s_base : item_cap);
+    hdr->n_tiles = (int32_t)(tiles < tile_cap ? tiles : tile_cap);
+  }
 }
 
 void launch_schedule(const int64_t* offsets, int64_t B, int64_t T, int64_t max_len, int n_heads,
-                     AttnItem* items, int64_t item_cap, Header* hdr, cudaStream_t s) {
+                     AttnItem* items, int64_t item_cap, int64_t* ubase, int64_t tile_cap,
+                     Header* hdr, cudaStream_t s) {
   LaunchScope ls(K_SCHEDULE, s);
-  k_schedule<<<1, kSchedThreads, 0, s>>>(offsets, B, T, max_len, n_heads, items, item_cap, hdr);
+  k_schedule<<<1, kSchedThreads, 0, s>>>(offsets, B, T, max_len, n_heads, items, item_cap, ubase,
+                                         tile_cap, hdr);
 }
 
 // ---------------------------------------------------------------- timestamps
@@ -134,6 +168,56 @@ void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64
   LaunchScope ls(K_TIME_REL, s);
   const int grid = (int)std::min<int64_t>((T + 255) / 256, 4 * num_sms());
   k_time_rel<<<grid, 256, 0, s>>>(offsets, B, ts, T, t_rel, hdr);
+}
+
+// ---------------------------------------------------------------- time buckets
+// One block per tile (grid-stride): tile t of user b is local index
+// qt (qt + 1) / 2 + j (j <= qt).  Word (c4, r) packs the buckets of row
+// qt*128 + r against columns j*128 + 4*c4 .. +3; entries outside the causal
+// triangle or the sequence are 0 (they are masked or unused).
+__global__ void __launch_bounds__(256)
+    k_time_buckets(const int64_t* __restrict__ off, int64_t B, const int32_t* __restrict__ t_rel,
+                   const int64_t* __restrict__ ubase, int St, int Nt,
+                   uint32_t* __restrict__ tb, const Header* hdr) {
+  if (hdr->status != HSTU_OK) return;
+  const int n_tiles = hdr->n_tiles;
+  for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int64_t b = find_user(ubase, B, t);  // ubase[b] <= t < ubase[b+1]
+    const int64_t local = t - ubase[b];
+    int qt = (int)((sqrt(8.0 * (double)local + 1.0) - 1.0) * 0.5);
+    while ((int64_t)qt * (qt + 1) / 2 > local) --qt;
+    while ((int64_t)(qt + 1) * (qt + 2) / 2 <= local) ++qt;
+    const int j = (int)(local - (int64_t)qt * (qt + 1) / 2);
+    const int64_t kv0 = off[b];
+    const int n = (int)(off[b + 1] - kv0);
+    const int r = threadIdx.x & 127;
+    const int i = qt * kTile + r;
+    const bool row_ok = i < n;
+    const int ti = row_ok ? t_rel[kv0 + i] : 0;
+    uint32_t* dst = tb + (size_t)t * kBucketTileWords;
+#pragma unroll 4
+    for (int u = 0; u < 16; ++u) {
+      const int c4 = (threadIdx.x >> 7) + 2 * u;
+      uint32_t word = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int jj = j * kTile + 4 * c4 + k;
+        uint32_t bk = 0;
+        if (row_ok && jj <= i) bk = (uint32_t)log_bucket(max(ti - t_rel[kv0 + jj], 0), St, Nt);
+        word |= bk << (8 * k);
+      }
+      dst[c4 * 128 + r] = word;
+    }
+  }
+}
+
+void launch_time_buckets(const int64_t* offsets, int64_t B, const int32_t* t_rel,
+                         const int64_t* ubase, int64_t tile_cap, int St, int Nt,
+                         uint32_t* tbuckets, Header* hdr, cudaStream_t s) {
+  if (tile_cap <= 0) return;
+  LaunchScope ls(K_TIME_BUCKETS, s);
+  const int grid = (int)std::min<int64_t>(tile_cap, 8 * num_sms());
+  k_time_buckets<<<grid, 256, 0, s>>>(offsets, B, t_rel, ubase, St, Nt, tbuckets, hdr);
 }
 
 // ---------------------------------------------------------------- LayerNorm * U
@@ -424,11 +508,13 @@ __global__ void __launch_bounds__(kSchedThreads)
         if (nkv != c) continue;
         const int64_t rows = mb_off[b + 1] - mb_off[b];
         const int nq = (int)((rows + kTile - 1) / kTile);
-        for (int qt = 0; qt < nq; ++qt, ++pos)
-          for (int hh = 0; hh < h; ++hh) {
-            const long long idx = pos * h + hh;
-            if (idx < item_cap) items[idx] = AttnItem{(int32_t)b, qt, hh, nkv};
+        // items of one (user, head) are adjacent: they read the same history K/V
+        for (int hh = 0; hh < h; ++hh)
+          for (int qt = 0; qt < nq; ++qt) {
+            const long long idx = pos * h + (long long)hh * nq + qt;
+            if (idx < item_cap) items[idx] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, nkv, 0};
           }
+        pos += nq;
       }
     }
     __syncthreads();
