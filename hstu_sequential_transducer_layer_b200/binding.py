@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 
 # Every symbol include/hstu.h declares.
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
+            "hstu_layer_fwd_noalloc",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_mfalcon_rank.argtypes = [pdesc, i32, pw, i64, i64, i64, vp, vp, vp, i64, i64, vp, vp,
                                     vp, i32, vp, vp, vp, sz, vp]
     L.hstu_mfalcon_rank.restype = i32
+    L.hstu_layer_fwd_noalloc.argtypes = [pdesc, i64, i64, i64, vp, vp, pw, vp, vp, vp]
+    L.hstu_layer_fwd_noalloc.restype = i32
     L.hstu_read_status.argtypes = [vp, sz, vp]
     L.hstu_read_status.restype = i32
     L.hstu_debug_offsets.argtypes = [pdesc, i64, i64, i64, ctypes.POINTER(sz),
@@ -175,6 +178,19 @@ def hstu_layer_fwd(desc, B, total_tokens, max_len, offsets, X, weights, timestam
                                 _ptr(X), ctypes.byref(ws), _ptr(timestamps), _ptr(out),
                                 _ptr(workspace), _nbytes(workspace), _stream(stream)),
            "hstu_layer_fwd")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # HSTU_NOALLOC_SCRATCH_BYTES
+
+
+def hstu_layer_fwd_noalloc(desc, B, total_tokens, max_len, offsets, X, weights, timestamps, out,
+                           stream=None) -> None:
+    """One layer in the library's fixed device scratch (no workspace argument)."""
+    ws = weights if isinstance(weights, LayerWeights) else weights_struct(weights)
+    _check(lib().hstu_layer_fwd_noalloc(ctypes.byref(desc), B, total_tokens, max_len,
+                                        _ptr(offsets), _ptr(X), ctypes.byref(ws),
+                                        _ptr(timestamps), _ptr(out), _stream(stream)),
+           "hstu_layer_fwd_noalloc")
 
 
 def hstu_stack_fwd(desc, n_layers, weights, B, total_tokens, max_len, offsets, X, timestamps,

@@ -24,7 +24,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libhstu.so")
 
-SOURCES = ["runtime.cu", "api.cu", "sched.cu", "gemm_tc.cu", "attn_tc.cu", "simt_f32.cu"]
+SOURCES = ["runtime.cu", "api.cu", "sched.cu", "gemm_tc.cu", "attn_tc.cu", "simt_f32.cu",
+           "noalloc.cu"]
 HEADERS = [os.path.join(CSRC, "ptx.cuh"), os.path.join(CSRC, "hstu_internal.h"),
            os.path.join(INCLUDE, "hstu.h")]
 

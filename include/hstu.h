@@ -159,6 +159,34 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
                               int32_t microbatch, const void* head_vec, float* scores,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of the fixed device scratch used by hstu_layer_fwd_noalloc. */
+#define HSTU_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* hstu_layer_fwd without a workspace argument, for callers that cannot
+ * allocate device memory (an allocator owned by another runtime, no
+ * cudaMalloc allowed after start-up, a memory-capped sandbox).  It has no
+ * counterpart on the pages: it is the same layer as hstu_layer_fwd, run in a
+ * file-scope device array of HSTU_NOALLOC_SCRATCH_BYTES (64 MiB) that every
+ * device loading this library holds until the process exits.  It allocates
+ * nothing itself: no cudaMalloc, no cudaFree, no allocating library call.
+ * The caller still passes the inputs and the output (as for hstu_layer_fwd).
+ *   - Sizes whose workspace (hstu_workspace_size with n_layers = 1) exceeds
+ *     HSTU_NOALLOC_SCRATCH_BYTES return HSTU_ERR_WORKSPACE and launch nothing;
+ *     other argument errors are those of hstu_layer_fwd.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; each
+ *     call resets what must start at zero (the status word and counters).
+ *     Calls whose execution overlaps on the GPU (other streams, other host
+ *     threads) race on the array: serialise them.
+ *   - The device status word lives in the array, so hstu_read_status cannot
+ *     read it; check the output or use hstu_layer_fwd to diagnose. */
+hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64_t total_tokens,
+                                   int64_t max_len, const int64_t* offsets, const void* X,
+                                   const hstu_layer_weights* weights, const int64_t* timestamps,
+                                   void* out, void* stream);
+
 /* Synchronises `stream`, then returns the device status word that the last
  * call using this workspace left (HSTU_OK if none of its checks failed). */
 hstu_status hstu_read_status(const void* workspace, size_t workspace_bytes, void* stream);
