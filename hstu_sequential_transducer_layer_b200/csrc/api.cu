@@ -111,18 +111,22 @@ LayerOps layer_ops(const Ctx& c, const hstu_layer_weights& w, const Layout& L, v
   return o;
 }
 
-// fp16 copies of the weights the call needs (W1 of layers >= 1, every W2).
+// fp16 copies of the weights the call needs (W1 of layers >= 1, every W2),
+// batched kMaxConvSegs segments per launch.
 cudaError_t convert_weights(const Ctx& c, const hstu_layer_weights* w, int n_layers,
                             const Layout& L, void* ws) {
   if (!c.bf16) return cudaSuccess;
   const int64_t F = c.F, dm = c.d.d_model, hdv = c.hdv;
+  ConvBatch cb{};
   for (int l = 0; l < n_layers; ++l) {
     LayerOps o = layer_ops(c, w[l], L, ws, l, n_layers);
-    cudaError_t e;
-    if (l > 0 && (e = launch_bf16_to_f16(w[l].W1, const_cast<void*>(o.W1), F * dm, c.s)) != cudaSuccess)
-      return e;
-    if ((e = launch_bf16_to_f16(w[l].W2, const_cast<void*>(o.W2), dm * hdv, c.s)) != cudaSuccess)
-      return e;
+    if (l > 0) cb.seg[cb.n++] = ConvSeg{w[l].W1, const_cast<void*>(o.W1), F * dm};
+    cb.seg[cb.n++] = ConvSeg{w[l].W2, const_cast<void*>(o.W2), dm * hdv};
+    if (cb.n > kMaxConvSegs - 2 || l == n_layers - 1) {
+      cudaError_t e = launch_bf16_to_f16(cb, c.s);
+      if (e != cudaSuccess) return e;
+      cb.n = 0;
+    }
   }
   return cudaSuccess;
 }

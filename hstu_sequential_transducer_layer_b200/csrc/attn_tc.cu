@@ -29,10 +29,12 @@
 // Bias per element (causal self-attention): the position bias comes from a
 // per-warp window of the 95 distances its 32 x 64 block spans; the time
 // bucket comes precomputed (one byte per element, shared by all heads and
-// layers of a call) and indexes a per-warp copy of the head's table.  Both
-// tables hold half the bias so that y = s/2 + bias/2 feeds
-// SiLU(x) = y + y tanh(y) (x = 2y) directly.  For candidates the bias depends
-// only on the history column: one shared-memory broadcast per element.
+// layers of a call) and indexes the head's table, which the producer warp
+// stores next to the item in the ring.  Both tables hold half the bias so that
+// y = s/2 + bias/2 feeds SiLU(x) = y + y tanh(y) (x = 2y) directly.  The P
+// warps fetch the next tile's bucket words and window while computing the
+// current tile.  For candidates the bias depends only on the history column:
+// one shared-memory broadcast per element.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -73,14 +75,17 @@ struct AttnCfg {
   static constexpr uint32_t K_OFF = Q_OFF + TILE;
   static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
   static constexpr uint32_t P_OFF = V_OFF + 2 * TILE;
-  static constexpr uint32_t WIN_OFF = P_OFF + P_BUFS * P_BYTES;   // 8 warps x 96 floats
-  static constexpr uint32_t RT_OFF = WIN_OFF + 8 * 96 * 4;        // 8 warps x 256 floats
-  static constexpr uint32_t BAR_OFF = RT_OFF + 8 * 256 * 4;
+  static constexpr uint32_t WIN_OFF = P_OFF + P_BUFS * P_BYTES;   // 8 warps x 2 x 96 floats
+  static constexpr uint32_t RT_OFF = WIN_OFF + 8 * 2 * 96 * 4;    // 2 ring slots x 256 floats
+  static constexpr uint32_t BAR_OFF = RT_OFF + 2 * 256 * 4;
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O
 };
 
 enum { MODE_SELF = 0, MODE_CAND = 1 };
+
+// Item ring entry (the item carries its row offsets).
+typedef AttnItem RingItem;
 
 // y = x / 2 (score plus bias, halved); returns SiLU(x) = y + y tanh(y).
 DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
@@ -107,7 +112,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* drain = bars + 16;
   uint64_t* it_full = bars + 17;    // [2] item ring
   uint64_t* it_empty = bars + 19;   // [2]
-  AttnItem* ring = reinterpret_cast<AttnItem*>(bars + 21);   // [2], 16 B each
+  RingItem* ring = reinterpret_cast<RingItem*>(bars + 21);   // [2], 32 B each
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + 2);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
@@ -160,66 +165,98 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ item fetch + TMA producer
-    if (lane == 0) {
-      int kst = 0, litem = 0;
-      uint32_t kph = 0, issued = 0, last_par = 0, q_issued = 0, q_par = 0, npub = 0;
-      bool ok = true;
-      for (;;) {
-        const int idx = atomicAdd(a.work_next, 1);
-        AttnItem w;
-        if (idx < n_items) w = a.items[idx];
-        else w = AttnItem{-1, 0, 0, 0, 0};
-        const int slot = npub & 1;
-        if (!mbar_wait(it_empty + slot, ((npub >> 1) & 1) ^ 1, ab, a.status)) {
-          ok = false;
-          break;
-        }
-        ring[slot] = w;
-        mbar_arrive(it_full + slot);  // release: the ring entry is visible to waiters
-        ++npub;
-        if (w.b < 0) break;
-        const int q_row0 = (int)(a.q_off[w.b] + (int64_t)w.qt * 128);
-        const int kv_row0 = (int)a.kv_off[w.b];
+    // Lane 0 fetches items and issues every TMA load; the whole warp fills the
+    // ring slot's halved time-bias table.
+    float* rt_ring = reinterpret_cast<float*>(smem + C::RT_OFF);
+    int kst = 0, litem = 0;
+    uint32_t kph = 0, issued = 0, last_par = 0, q_issued = 0, q_par = 0, npub = 0;
+    bool ok = true;
+    // Work indices are claimed two items ahead and the next item's entry is
+    // read one item ahead, so neither latency sits between two items.
+    auto claim = [&]() {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(a.work_next, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    auto entry = [&](int idx) {
+      RingItem x;
+      if (idx < n_items) x = a.items[idx];
+      else x = AttnItem{-1, 0, 0, 0, 0, 0, 0, 0, 0};
+      return x;
+    };
+    int idx_next = claim();
+    int idx_after = claim();
+    RingItem nxt = entry(idx_next);
+    for (;;) {
+      const RingItem x = nxt;
+      if (x.b >= 0) {
+        idx_next = idx_after;
+        idx_after = claim();
+        nxt = entry(idx_next);
+      }
+      const int slot = npub & 1;
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(it_empty + slot, ((npub >> 1) & 1) ^ 1, ab, a.status);
+      if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) {
+        ok = false;
+        break;
+      }
+      if (MODE == MODE_SELF && x.b >= 0) {
+        const float* Rt = a.rab_time + (size_t)x.head * a.Nt;
+        for (int k = lane; k < a.Nt; k += 32) rt_ring[slot * 256 + k] = 0.5f * __ldg(Rt + k);
+      }
+      if (lane == 0) ring[slot] = x;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(it_full + slot);  // release: slot contents visible to waiters
+      ++npub;
+      if (x.b < 0) break;
+      if (lane == 0) {
+        const AttnItem w = x;
+        const int q_row0 = x.q_row0;
+        const int kv_row0 = x.kv_row0;
         if (!mbar_wait(q_empty, (litem & 1) ^ 1, ab, a.status)) {
           ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(q_full, C::TILE);
+        } else {
+          mbar_arrive_expect_tx(q_full, C::TILE);
 #pragma unroll
-        for (int at = 0; at < C::NA; ++at)
-          tma_load_2d(sQ + at * 16384, &tmQ, a.q_col + w.head * D + at * 64, q_row0, q_full);
-        q_issued = 1;
-        q_par = litem & 1;
-        for (int j = 0; j < w.nkv; ++j) {
-          if (!mbar_wait(kv_empty + kst, kph ^ 1, ab, a.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(kv_full + kst, 2 * C::TILE);
-          const int y = kv_row0 + j * 128;
+          for (int at = 0; at < C::NA; ++at)
+            tma_load_2d(sQ + at * 16384, &tmQ, a.q_col + w.head * D + at * 64, q_row0, q_full);
+          q_issued = 1;
+          q_par = litem & 1;
+          for (int j = 0; j < w.nkv; ++j) {
+            if (!mbar_wait(kv_empty + kst, kph ^ 1, ab, a.status)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(kv_full + kst, 2 * C::TILE);
+            const int y = kv_row0 + j * 128;
 #pragma unroll
-          for (int at = 0; at < C::NA; ++at) {
-            tma_load_2d(sK + kst * C::TILE + at * 16384, &tmKV, a.k_col + w.head * D + at * 64, y,
-                        kv_full + kst);
-            tma_load_2d(sV + kst * C::TILE + at * 16384, &tmKV, a.v_col + w.head * D + at * 64, y,
-                        kv_full + kst);
-          }
-          issued |= 1u << kst;
-          last_par = (last_par & ~(1u << kst)) | (kph << kst);
-          if (++kst == 2) {
-            kst = 0;
-            kph ^= 1;
+            for (int at = 0; at < C::NA; ++at) {
+              tma_load_2d(sK + kst * C::TILE + at * 16384, &tmKV, a.k_col + w.head * D + at * 64,
+                          y, kv_full + kst);
+              tma_load_2d(sV + kst * C::TILE + at * 16384, &tmKV, a.v_col + w.head * D + at * 64,
+                          y, kv_full + kst);
+            }
+            issued |= 1u << kst;
+            last_par = (last_par & ~(1u << kst)) | (kph << kst);
+            if (++kst == 2) {
+              kst = 0;
+              kph ^= 1;
+            }
           }
         }
-        if (!ok) break;
-        ++litem;
       }
-      if (!ok) {  // let every load already in flight land before the CTA exits
-        AbortState tmp{0};
-        for (int s = 0; s < 2; ++s)
-          if ((issued >> s) & 1u) mbar_wait(kv_full + s, (last_par >> s) & 1u, &tmp, nullptr);
-        if (q_issued) mbar_wait(q_full, q_par, &tmp, nullptr);
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+        ok = false;
+        break;
       }
+      ++litem;
+    }
+    if (!ok && lane == 0) {  // let every load already in flight land before the CTA exits
+      AbortState tmp{0};
+      for (int s2 = 0; s2 < 2; ++s2)
+        if ((issued >> s2) & 1u) mbar_wait(kv_full + s2, (last_par >> s2) & 1u, &tmp, nullptr);
+      if (q_issued) mbar_wait(q_full, q_par, &tmp, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -284,6 +321,7 @@ __global__ void __launch_bounds__(320, 1)
                           sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                           IDESC_S, kk > 0 ? 1u : 0u);
           tc_commit(s_full + sb);
+          if (j == nkv - 1) tc_commit(q_empty);  // P.V does not read Q: free it early
           ++scount;
           any = true;
           if (j > 0 && !issue_pv(j - 1, prev, nkv)) {
@@ -301,8 +339,8 @@ __global__ void __launch_bounds__(320, 1)
           if (!issue_pv(nkv - 1, prev, nkv)) break;
         } else {
           tc_commit(o_full);  // nothing to accumulate: O is taken as zero
+          tc_commit(q_empty);
         }
-        tc_commit(q_empty);
         ++litem;
       }
       if (any) {
@@ -317,8 +355,8 @@ __global__ void __launch_bounds__(320, 1)
     const int q = warp & 3;          // TMEM lane quarter
     const int half = pw >> 2;        // which 64 of the 128 S columns
     const int r = q * 32 + lane;     // row inside the 128-row tile
-    float* win = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 96;
-    float* rt = reinterpret_cast<float*>(smem + C::RT_OFF) + pw * 256;
+    float* win2 = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 2 * 96;  // 2 buffers
+    const float* rt_ring = reinterpret_cast<const float*>(smem + C::RT_OFF);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t scount = 0, pcount = 0, ncon = 0;
     int litem = 0;
@@ -326,38 +364,32 @@ __global__ void __launch_bounds__(320, 1)
       const int slot = ncon & 1;
       if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
       const AttnItem w = ring[slot];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(it_empty + slot);
+      const float* rt = rt_ring + slot * 256;   // valid while this item holds the slot
       ++ncon;
-      if (w.b < 0) break;
-      const int64_t kv0 = a.kv_off[w.b];
-      const int n_kv = (int)(a.kv_off[w.b + 1] - kv0);           // history / sequence length
-      const int64_t q0 = a.q_off[w.b] + (int64_t)w.qt * 128;
-      const int n_q = (int)(a.q_off[w.b + 1] - a.q_off[w.b]);
-      const int rows_valid = min(128, n_q - (int)w.qt * 128);
+      if (w.b < 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(it_empty + slot);
+        break;
+      }
+      const int64_t kv0 = w.kv_row0;
+      const int n_kv = w.n_kv;                   // history / sequence length
+      const int64_t q0 = w.q_row0;
+      const int rows_valid = min(128, w.n_q - (int)w.qt * 128);
       const bool row_ok = r < rows_valid;
       const float inv_n = 1.0f / (float)max(n_kv, 1);
       const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
       const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
-      int t_i = 0;
-      if (MODE == MODE_SELF) {
-        // this head's time-bias table, halved, in the warp's own slice
-        __syncwarp();
-        for (int k = lane; k < a.Nt; k += 32) rt[k] = 0.5f * __ldg(Rt + k);
-      } else {
-        t_i = a.t_req_rel[w.b];
-      }
-      bool alive = true;
-      for (int j = 0; j < w.nkv; ++j) {
-        // ---- per-warp bias inputs for this tile
-        __syncwarp();
-        uint32_t bw[16];
+      const int t_i = (MODE == MODE_SELF) ? 0 : a.t_req_rel[w.b];
+      // Bias inputs of KV tile jt into window buffer `buf` (and, causal mode,
+      // the tile's time-bucket words into bwn).
+      auto prep = [&](int jt, int buf, uint32_t (&bwn)[16]) {
+        float* win = win2 + buf * 96;
         if (MODE == MODE_SELF) {
-          const uint32_t* tbw = a.tbuckets + (size_t)(w.tile0 + j) * kBucketTileWords +
+          const uint32_t* tbw = a.tbuckets + (size_t)(w.tile0 + jt) * kBucketTileWords +
                                 (half * 16) * 128 + r;
 #pragma unroll
-          for (int m = 0; m < 16; ++m) bw[m] = __ldg(tbw + m * 128);
-          const int base = (w.qt - j) * 128 + q * 32 - half * 64 - 63;
+          for (int m = 0; m < 16; ++m) bwn[m] = __ldg(tbw + m * 128);
+          const int base = (w.qt - jt) * 128 + q * 32 - half * 64 - 63;
 #pragma unroll
           for (int u = 0; u < 3; ++u) {
             const int k = lane + 32 * u;
@@ -369,7 +401,7 @@ __global__ void __launch_bounds__(320, 1)
         } else {
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int jc = j * 128 + half * 64 + lane + 32 * u;
+            const int jc = jt * 128 + half * 64 + lane + 32 * u;
             float bias = 0.f;
             if (jc < n_kv) {
               const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
@@ -379,7 +411,13 @@ __global__ void __launch_bounds__(320, 1)
             win[lane + 32 * u] = 0.5f * bias;
           }
         }
-        __syncwarp();
+      };
+      uint32_t bw[16], bwn[16];
+      if (w.nkv > 0) prep(0, 0, bw);
+      bool alive = true;
+      for (int j = 0; j < w.nkv; ++j) {
+        __syncwarp();  // this tile's window is written; the one before it is free
+        const float* win = win2 + (j & 1) * 96;
         // ---- S tile from TMEM
         const int sb = scount & 1;
         if (!mbar_wait_warp(s_full + sb, (scount >> 1) & 1, ab, a.status)) {
@@ -394,6 +432,8 @@ __global__ void __launch_bounds__(320, 1)
           tmem_ld32(tmem + sb * 128 + half * 64 + lane_base, lo32);
           tmem_ld32(tmem + sb * 128 + half * 64 + 32 + lane_base, hi32);
         }
+        // prefetch the next tile's bias inputs while this tile computes
+        if (j + 1 < w.nkv) prep(j + 1, (j + 1) & 1, bwn);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -436,6 +476,8 @@ __global__ void __launch_bounds__(320, 1)
             pk[c >> 1] = pack_f16x2_sat(p0, p1);
           }
         }
+#pragma unroll
+        for (int m = 0; m < 16; ++m) bw[m] = bwn[m];
         // ---- write P (K-major, 128-byte swizzle: chunk m of row r at m ^ (r & 7))
         const int pb = (int)(pcount % C::P_BUFS);
         if (!mbar_wait_warp(p_free + pb, ((pcount / C::P_BUFS) & 1) ^ 1, ab, a.status)) {
@@ -457,6 +499,9 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) mbar_arrive(p_full + pb);
         ++pcount;
       }
+      // the ring slot (and its time table) may be refilled from here on
+      __syncwarp();
+      if (lane == 0) mbar_arrive(it_empty + slot);
       if (!alive) break;
       // ---- O epilogue
       if (!mbar_wait_warp(o_full, litem & 1, ab, a.status)) break;

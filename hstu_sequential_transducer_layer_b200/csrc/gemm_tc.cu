@@ -10,8 +10,10 @@
 // walked n-fastest so that a wave of CTAs shares the A rows through L2.
 // Warp 0 streams A and W tiles with TMA (128-byte swizzle) into a STAGES-deep
 // ring; warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
-// accumulators; warps 2-5 drain the other accumulator with tcgen05.ld, apply
-// the epilogue in registers and store bf16 rows.  Every wait is bounded.
+// accumulators; warps 2-9 (two per TMEM lane quarter, half of the columns
+// each) drain the other accumulator with tcgen05.ld, loading the next 32
+// columns while they apply the epilogue to the current ones.  The bias is
+// staged once per CTA in shared memory as fp32.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
@@ -34,6 +36,9 @@ struct GemmDev {
   int* status;
 };
 
+constexpr int kMaxBiasN = 8192;       // output columns whose bias fits in shared memory
+constexpr int kEpiThreads = 256;      // 8 epilogue warps
+
 template <int BN, int STAGES>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
@@ -41,24 +46,23 @@ struct GemmCfg {
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
+  static constexpr uint32_t BIAS_OFF = BAR_OFF + 512;          // fp32 bias, up to kMaxBiasN
+  static constexpr uint32_t SMEM = BIAS_OFF + kMaxBiasN * 4 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
 
 template <int EPI>
 DEVI void gemm_epilogue_store(const GemmDev& g, int64_t row, bool valid, int col,
-                              const uint32_t (&r)[32]) {
+                              const float* sbias, const uint32_t (&r)[32]) {
   float v[32];
-  const uint4* bp = reinterpret_cast<const uint4*>(g.bias + col);
+  const float4* bp = reinterpret_cast<const float4*>(sbias + col - g.n_off);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 bb = __ldg(bp + i);
-    const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[i * 8 + 2 * k] = __uint_as_float(r[i * 8 + 2 * k]) + bf16lo(bw[k]);
-      v[i * 8 + 2 * k + 1] = __uint_as_float(r[i * 8 + 2 * k + 1]) + bf16hi(bw[k]);
-    }
+  for (int i = 0; i < 8; ++i) {
+    const float4 bb = bp[i];  // shared-memory broadcast
+    v[4 * i + 0] = __uint_as_float(r[4 * i + 0]) + bb.x;
+    v[4 * i + 1] = __uint_as_float(r[4 * i + 1]) + bb.y;
+    v[4 * i + 2] = __uint_as_float(r[4 * i + 2]) + bb.z;
+    v[4 * i + 3] = __uint_as_float(r[4 * i + 3]) + bb.w;
   }
   if (!valid) return;
   if (EPI == EPI_SILU) {
@@ -110,7 +114,7 @@ DEVI void gemm_epilogue_store(const GemmDev& g, int64_t row, bool valid, int col
 }
 
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + kEpiThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const GemmDev g) {
   using C = GemmCfg<BN, STAGES>;
@@ -136,8 +140,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(tfull + 0, 1);
     mbar_init(tfull + 1, 1);
-    mbar_init(tempty + 0, 4);
-    mbar_init(tempty + 1, 4);
+    mbar_init(tempty + 0, kEpiThreads / 32);
+    mbar_init(tempty + 1, kEpiThreads / 32);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -145,6 +149,10 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
+  // the bias of this call's output columns, fp32, once per CTA
+  float* sbias = reinterpret_cast<float*>(smem + C::BIAS_OFF);
+  for (int i = threadIdx.x; i < g.N; i += blockDim.x)
+    sbias[i] = __bfloat162float(g.bias[g.n_off + i]);
   __syncthreads();
   if (!*s_go) return;
 
@@ -243,7 +251,9 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int q = warp & 3;              // TMEM lane quarter this warp may read
+    const int part = (warp - 2) >> 2;    // which half of the BN columns
+    constexpr int CH = BN / 64;          // 32-column chunks per warp
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
@@ -253,12 +263,21 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int64_t row = (int64_t)mt * 128 + q * 32 + lane;
       const bool valid = row < Mrows;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + acc * BN + c * 32 + ((uint32_t)(q * 32) << 16), r);
-        tmem_ld_wait();
-        gemm_epilogue_store<EPI>(g, row, valid, g.n_off + nt * BN + c * 32, r);
+      const uint32_t tbase = tmem + acc * BN + part * (BN / 2) + ((uint32_t)(q * 32) << 16);
+      const int col0 = g.n_off + nt * BN + part * (BN / 2);
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tbase, ra);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        // the next chunk's TMEM load runs while this chunk is processed
+        if (c + 1 < CH) {
+          if (c & 1) tmem_ld32(tbase + (c + 1) * 32, ra);
+          else tmem_ld32(tbase + (c + 1) * 32, rb);
+        }
+        if (c & 1) gemm_epilogue_store<EPI>(g, row, valid, col0 + c * 32, sbias, rb);
+        else gemm_epilogue_store<EPI>(g, row, valid, col0 + c * 32, sbias, ra);
+        if (c + 1 < CH) tmem_ld_wait();
       }
       tc_fence_before();
       __syncwarp();
@@ -285,13 +304,13 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kfn<<<grid, 192, C::SMEM, s>>>(ta, tb, gd);
+  kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, gd);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   if (c.M_cap <= 0 || c.N <= 0) return cudaSuccess;
-  if (c.N % 64 != 0 || c.K % 64 != 0) return cudaErrorInvalidValue;
+  if (c.N % 64 != 0 || c.K % 64 != 0 || c.N > kMaxBiasN) return cudaErrorInvalidValue;
   const int sms = num_sms();
   const int64_t mt = (c.M_cap + 127) / 128;
   int BN = 64;

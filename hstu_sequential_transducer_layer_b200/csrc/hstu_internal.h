@@ -79,13 +79,18 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
 
 // ---------------------------------------------------------------- kernels
 // One attention work item: (user, 128-row query tile, head), the number of
-// 128-row KV tiles it reads, and (causal self-attention) the index of the
-// time-bucket tile of (user, query tile, KV tile 0).
+// 128-row KV tiles it reads, (causal self-attention) the index of the
+// time-bucket tile of (user, query tile, KV tile 0), and the row offsets the
+// kernel needs, so that starting an item takes no dependent loads.
 struct AttnItem {
   int32_t b;
   int16_t qt, head;
   int32_t nkv;
   int32_t tile0;
+  int32_t q_row0;   // first query row of the tile
+  int32_t kv_row0;  // first KV row of the user
+  int32_t n_q;      // query rows of the user
+  int32_t n_kv;     // KV rows of the user (history length for candidates)
 };
 // A time-bucket tile: the bucket of t_i - t_j for 128 query rows x 128 KV
 // columns, one byte each, 4 consecutive columns per 32-bit word, stored
@@ -158,8 +163,19 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
                            int64_t rows_cap, const int64_t* rows_dev, const int* status,
                            cudaStream_t s);
 
-// bf16 -> fp16 (round to nearest, saturating at +-65504), n elements.
-cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, cudaStream_t s);
+// bf16 -> fp16 (round to nearest, saturating at +-65504) of up to
+// kMaxConvSegs segments in one launch; n elements each, multiples of 8.
+constexpr int kMaxConvSegs = 32;
+struct ConvSeg {
+  const void* src;
+  void* dst;
+  int64_t n;
+};
+struct ConvBatch {
+  ConvSeg seg[kMaxConvSegs];
+  int n;
+};
+cudaError_t launch_bf16_to_f16(const ConvBatch& cb, cudaStream_t s);
 
 // M-FALCON microbatch plumbing.
 void launch_mb_plan(const int64_t* hist_off, const int64_t* cand_off, int64_t B, int64_t max_len,

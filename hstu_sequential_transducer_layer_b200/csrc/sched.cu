@@ -50,16 +50,17 @@ __device__ long long block_scan_users(int64_t B, F v, int64_t* out, long long* s
   return *s_carry;
 }
 
+constexpr int kMaxLevels = 4096;  // q-tiles per user handled by the parallel path
+
 __global__ void __launch_bounds__(kSchedThreads)
     k_schedule(const int64_t* __restrict__ off, int64_t B, int64_t T, int64_t max_len, int h,
                AttnItem* __restrict__ items, int64_t item_cap, int64_t* __restrict__ ubase,
                int64_t tile_cap, Header* hdr) {
-  __shared__ int s_bad;
+  __shared__ int s_bad, s_nqmax;
   __shared__ long long s_part[kSchedThreads];
   __shared__ long long s_carry;
-  __shared__ long long s_cnt[kSchedThreads];
-  __shared__ long long s_start[kSchedThreads];
-  __shared__ long long s_base;
+  __shared__ int s_hist[kMaxLevels + 1];     // users per q-tile count
+  __shared__ int s_cursor[kMaxLevels + 1];   // next item position per q-tile count
   if (threadIdx.x == 0) {
     hdr->status = HSTU_OK;
     hdr->n_items = 0;
@@ -67,61 +68,78 @@ __global__ void __launch_bounds__(kSchedThreads)
     hdr->work_next = 0;
     hdr->work_done = 0;
     s_bad = 0;
+    s_nqmax = 0;
     if (off[0] != 0 || off[B] != T) s_bad = 1;
   }
+  for (int i = threadIdx.x; i <= kMaxLevels; i += blockDim.x) s_hist[i] = 0;
   __syncthreads();
   for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
     const int64_t n = off[b + 1] - off[b];
     if (n < 0 || n > max_len) s_bad = 1;
+    else atomicMax(&s_nqmax, (int)((n + kTile - 1) / kTile));
   }
   __syncthreads();
   if (s_bad) {
     if (threadIdx.x == 0) hdr->status = HSTU_ERR_BAD_OFFSETS;
     return;
   }
-  auto nq_of = [&](int64_t b) { return (off[b + 1] - off[b] + kTile - 1) / kTile; };
+  auto nq_of = [&](int64_t b) { return (int)((off[b + 1] - off[b] + kTile - 1) / kTile); };
   // first time-bucket tile of every user: prefix of nq (nq + 1) / 2
   const long long tiles = block_scan_users(
       B, [&](int64_t b) { const long long q = nq_of(b); return q * (q + 1) / 2; }, ubase, s_part,
       &s_carry);
-  // Items grouped by (user, head): users with more q-tiles first (level c =
-  // nq, highest first), users in order inside a level, then heads, then
-  // q-tiles longest first.  Neighbouring items read the same K/V.
-  const int levels = (int)((max_len + kTile - 1) / kTile);
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
-  for (int c_hi = levels; c_hi >= 1; c_hi -= blockDim.x) {
-    const int c = c_hi - (int)threadIdx.x;
-    long long cnt = 0;
-    if (c >= 1)
-      for (int64_t b = 0; b < B; ++b) cnt += nq_of(b) == c;
-    s_cnt[threadIdx.x] = cnt * c * h;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      long long acc = s_base;
-      const int m = min((int)blockDim.x, c_hi);
-      for (int i = 0; i < m; ++i) {
-        s_start[i] = acc;
-        acc += s_cnt[i];
-      }
-      s_base = acc;
+  // Items grouped by (user, head): users with more q-tiles first, then heads,
+  // then q-tiles longest first; neighbouring items read the same K/V.  The
+  // order of users with equal q-tile counts is immaterial (each item writes
+  // only its own rows).
+  const int nqmax = s_nqmax;
+  long long total = 0;
+  if (nqmax <= kMaxLevels) {
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+      const int c = nq_of(b);
+      if (c > 0) atomicAdd(&s_hist[c], 1);
     }
     __syncthreads();
-    if (c >= 1) {
-      long long pos = s_start[threadIdx.x];
+    if (threadIdx.x == 0) {
+      long long acc = 0;
+      for (int c = nqmax; c >= 1; --c) {
+        s_cursor[c] = (int)(acc < (1ll << 30) ? acc : (1ll << 30));
+        acc += (long long)s_hist[c] * c * h;
+      }
+      s_carry = acc;
+    }
+    __syncthreads();
+    total = s_carry;
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+      const int c = nq_of(b);
+      if (c == 0) continue;
+      long long pos = atomicAdd(&s_cursor[c], c * h);
+      for (int hh = 0; hh < h; ++hh)
+        for (int qt = c - 1; qt >= 0; --qt, ++pos)
+          if (pos < item_cap)
+            items[pos] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, qt + 1,
+                                  (int32_t)(ubase[b] + (long long)qt * (qt + 1) / 2),
+                                  (int32_t)(off[b] + (int64_t)qt * kTile), (int32_t)off[b],
+                                  (int32_t)(off[b + 1] - off[b]), (int32_t)(off[b + 1] - off[b])};
+    }
+  } else if (threadIdx.x == 0) {  // users over kMaxLevels * 128 tokens: one thread walks them
+    long long pos = 0;
+    for (int c = nqmax; c >= 1; --c)
       for (int64_t b = 0; b < B; ++b) {
         if (nq_of(b) != c) continue;
         for (int hh = 0; hh < h; ++hh)
           for (int qt = c - 1; qt >= 0; --qt, ++pos)
             if (pos < item_cap)
               items[pos] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, qt + 1,
-                                    (int32_t)(ubase[b] + (long long)qt * (qt + 1) / 2)};
+                                    (int32_t)(ubase[b] + (long long)qt * (qt + 1) / 2),
+                                    (int32_t)(off[b] + (int64_t)qt * kTile), (int32_t)off[b],
+                                    (int32_t)(off[b + 1] - off[b]),
+                                    (int32_t)(off[b + 1] - off[b])};
       }
-    }
-    __syncthreads();
+    total = pos;
   }
   if (threadIdx.x == 0) {
-    hdr->n_items = (int32_t)(s_base < item_cap ? s_base : item_cap);
+    hdr->n_items = (int32_t)(total < item_cap ? total : item_cap);
     hdr->n_tiles = (int32_t)(tiles < tile_cap ? tiles : tile_cap);
   }
 }
@@ -264,7 +282,11 @@ __global__ void __launch_bounds__(256)
   Tu* zrow = Z + row * (int64_t)hdv;
   const int nch = hdv / 256;
   float sum = 0.f;
+  uint4 uvec[kLnMaxPerLane / 8];  // U is loaded together with O (more bytes in flight)
   if (VEC) {
+#pragma unroll
+    for (int k = 0; k < kLnMaxPerLane / 8; ++k)
+      if (k < nch) uvec[k] = *reinterpret_cast<const uint4*>(urow + (k * 32 + lane) * 8);
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane / 8; ++k) {
       if (k < nch) {
@@ -317,7 +339,7 @@ __global__ void __launch_bounds__(256)
         const int c0 = (k * 32 + lane) * 8;
         const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gamma + c0));
         const uint4 bv = __ldg(reinterpret_cast<const uint4*>(beta + c0));
-        const uint4 uv = *reinterpret_cast<const uint4*>(urow + c0);
+        const uint4 uv = uvec[k];
         const uint32_t g[4] = {gv.x, gv.y, gv.z, gv.w}, bb[4] = {bv.x, bv.y, bv.z, bv.w},
                        u[4] = {uv.x, uv.y, uv.z, uv.w};
         uint32_t out[4];
@@ -375,7 +397,12 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
 }
 
 // ---------------------------------------------------------------- bf16 -> fp16
-__global__ void k_bf16_to_f16(const uint4* __restrict__ src, uint4* __restrict__ dst, int64_t n8) {
+// One launch converts up to kMaxConvSegs segments (blockIdx.y = segment).
+__global__ void k_bf16_to_f16(ConvBatch cb) {
+  const ConvSeg sg = cb.seg[blockIdx.y];
+  const uint4* src = static_cast<const uint4*>(sg.src);
+  uint4* dst = static_cast<uint4*>(sg.dst);
+  const int64_t n8 = sg.n / 8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
        i += (int64_t)gridDim.x * blockDim.x) {
     const uint4 v = src[i];
@@ -388,13 +415,16 @@ __global__ void k_bf16_to_f16(const uint4* __restrict__ src, uint4* __restrict__
   }
 }
 
-cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, cudaStream_t s) {
-  if (n <= 0) return cudaSuccess;
-  if (n % 8 != 0) return cudaErrorInvalidValue;
+cudaError_t launch_bf16_to_f16(const ConvBatch& cb, cudaStream_t s) {
+  if (cb.n <= 0) return cudaSuccess;
+  int64_t mx = 0;
+  for (int i = 0; i < cb.n; ++i) {
+    if (cb.seg[i].n % 8 != 0) return cudaErrorInvalidValue;
+    mx = std::max<int64_t>(mx, cb.seg[i].n);
+  }
   LaunchScope ls(K_CONVERT, s);
-  const int64_t n8 = n / 8;
-  const int grid = (int)std::min<int64_t>((n8 + 255) / 256, 8 * num_sms());
-  k_bf16_to_f16<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n8);
+  const int gx = (int)std::max<int64_t>(1, std::min<int64_t>((mx / 8 + 255) / 256, 2 * num_sms()));
+  k_bf16_to_f16<<<dim3(gx, cb.n), 256, 0, s>>>(cb);
   return cudaGetLastError();
 }
 
@@ -512,7 +542,10 @@ __global__ void __launch_bounds__(kSchedThreads)
         for (int hh = 0; hh < h; ++hh)
           for (int qt = 0; qt < nq; ++qt) {
             const long long idx = pos * h + (long long)hh * nq + qt;
-            if (idx < item_cap) items[idx] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, nkv, 0};
+            if (idx < item_cap)
+              items[idx] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, nkv, 0,
+                                    (int32_t)(mb_off[b] + (int64_t)qt * kTile), (int32_t)hoff[b],
+                                    (int32_t)rows, (int32_t)n};
           }
         pos += nq;
       }
