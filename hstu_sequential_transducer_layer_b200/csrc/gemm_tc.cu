@@ -1,5 +1,5 @@
-// gemm_tc.cu — bf16 GEMM on the 5th-generation tensor cores (tcgen05) with
-// fused epilogues, used for both projections of the HSTU layer:
+// gemm_tc.cu — GEMM on the 5th-generation tensor cores (tcgen05) with fused
+// epilogues, used for both projections of the HSTU layer:
 //   f1:  G = SiLU(X W1^T + b1)         (EPI_SILU; output = [U | V | Q | K])
 //   f2:  Y = X + Z W2^T + b2           (EPI_RESID)
 // ('HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか':
@@ -11,9 +11,10 @@
 // Warp 0 streams A and W tiles with TMA (128-byte swizzle) into a STAGES-deep
 // ring; warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM
 // accumulators; warps 2-9 (two per TMEM lane quarter, half of the columns
-// each) drain the other accumulator with tcgen05.ld, loading the next 32
-// columns while they apply the epilogue to the current ones.  The bias is
-// staged once per CTA in shared memory as fp32.  Every wait is bounded.
+// each) drain the other accumulator 32 columns at a time, loading the next
+// chunk (accumulator and bias) while they finish the current one, and write
+// each 32 x 32 result through a swizzled shared-memory buffer with TMA bulk
+// tensor stores (whole lines, asynchronous).  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
@@ -26,18 +27,17 @@ struct GemmDev {
   int N, K, n_off;
   int ab_f16;                  // operand format: fp16 (1) or bf16 (0)
   const __nv_bfloat16* bias;
-  void* out;                   // 16-bit output (fp16 if out_f16, else bf16); may be null
+  int has_out16;               // 16-bit output (fp16 if out_f16, else bf16)
   int out_f16;
-  int64_t ldo;
-  float* out32;                // EPI_RESID: optional fp32 copy of the output (same ldo)
+  int has_out32;               // EPI_RESID: fp32 copy of the output
   const void* resid;           // EPI_RESID: residual, bf16 or fp32 (resid_f32)
   int64_t ldr;
   int resid_f32;
   int* status;
 };
 
-constexpr int kMaxBiasN = 8192;       // output columns whose bias fits in shared memory
 constexpr int kEpiThreads = 256;      // 8 epilogue warps
+constexpr uint32_t kStageBuf = 4096;  // per-warp output staging bytes (32 x 32 fp32)
 
 template <int BN, int STAGES>
 struct GemmCfg {
@@ -45,78 +45,113 @@ struct GemmCfg {
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr uint32_t BIAS_OFF = BAR_OFF + 512;          // fp32 bias, up to kMaxBiasN
-  static constexpr uint32_t SMEM = BIAS_OFF + kMaxBiasN * 4 + 1024;
+  static constexpr uint32_t OUT_OFF = STAGES * STAGE_BYTES;             // 8 x 4 KB staging
+  static constexpr uint32_t BAR_OFF = OUT_OFF + (kEpiThreads / 32) * kStageBuf;
+  static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
 
+// Applies the epilogue to one 32-column chunk of this thread's row and stores
+// the warp's 32 x 32 tile: the fp32 copy through a 128-byte-swizzled buffer
+// and/or the 16-bit output through a 64-byte-swizzled one, each with one TMA
+// store issued by lane 0.  `stage` is the warp's 4 KB buffer; `parity` picks
+// the 2 KB half of a 16-bit-only output (double buffering).  Returns whether
+// the warp stored anything (not when all its 32 rows are past the end).
 template <int EPI>
-DEVI void gemm_epilogue_store(const GemmDev& g, int64_t row, bool valid, int col,
-                              const float* sbias, const uint32_t (&r)[32]) {
+DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorMap* tmO32,
+                     int64_t row, bool valid, int col, int y0, const uint32_t (&r)[32],
+                     const uint4 (&bias)[4], uint8_t* stage, int parity) {
+  const int lane = threadIdx.x & 31;
   float v[32];
-  const float4* bp = reinterpret_cast<const float4*>(sbias + col - g.n_off);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 bb = bp[i];  // shared-memory broadcast
-    v[4 * i + 0] = __uint_as_float(r[4 * i + 0]) + bb.x;
-    v[4 * i + 1] = __uint_as_float(r[4 * i + 1]) + bb.y;
-    v[4 * i + 2] = __uint_as_float(r[4 * i + 2]) + bb.z;
-    v[4 * i + 3] = __uint_as_float(r[4 * i + 3]) + bb.w;
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t bw[4] = {bias[i].x, bias[i].y, bias[i].z, bias[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[i * 8 + 2 * k] = __uint_as_float(r[i * 8 + 2 * k]) + bf16lo(bw[k]);
+      v[i * 8 + 2 * k + 1] = __uint_as_float(r[i * 8 + 2 * k + 1]) + bf16hi(bw[k]);
+    }
   }
-  if (!valid) return;
   if (EPI == EPI_SILU) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
-  } else if (g.resid_f32) {
-    const float4* rp = reinterpret_cast<const float4*>(
-        static_cast<const float*>(g.resid) + row * g.ldr + col);
+  } else if (valid) {
+    if (g.resid_f32) {
+      const float4* rp = reinterpret_cast<const float4*>(
+          static_cast<const float*>(g.resid) + row * g.ldr + col);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 rr = rp[i];
-      v[4 * i + 0] += rr.x;
-      v[4 * i + 1] += rr.y;
-      v[4 * i + 2] += rr.z;
-      v[4 * i + 3] += rr.w;
-    }
-  } else {
-    const uint4* rp = reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(g.resid) + row * g.ldr + col);
+      for (int i = 0; i < 8; ++i) {
+        const float4 rr = rp[i];
+        v[4 * i + 0] += rr.x;
+        v[4 * i + 1] += rr.y;
+        v[4 * i + 2] += rr.z;
+        v[4 * i + 3] += rr.w;
+      }
+    } else {
+      const uint4* rp = reinterpret_cast<const uint4*>(
+          static_cast<const __nv_bfloat16*>(g.resid) + row * g.ldr + col);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 rr = rp[i];
-      const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+      for (int i = 0; i < 4; ++i) {
+        const uint4 rr = rp[i];
+        const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[i * 8 + 2 * k] += bf16lo(rw[k]);
-        v[i * 8 + 2 * k + 1] += bf16hi(rw[k]);
+        for (int k = 0; k < 4; ++k) {
+          v[i * 8 + 2 * k] += bf16lo(rw[k]);
+          v[i * 8 + 2 * k + 1] += bf16hi(rw[k]);
+        }
       }
     }
   }
-  if (EPI == EPI_RESID && g.out32) {
-    float4* op = reinterpret_cast<float4*>(g.out32 + row * g.ldo + col);
+  if (__shfl_sync(0xffffffffu, valid ? 1 : 0, 0) == 0) return false;  // rows y0.. all invalid
+  const bool both = (EPI == EPI_RESID) && g.has_out32;
+  if (both) {
+    if (lane == 0) bulk_wait_read<0>();  // the warp's earlier stores have read the buffer
+    __syncwarp();
+    uint8_t* rowp = stage + lane * 128;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) op[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-  }
-  if (g.out) {
-    uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) + row * g.ldo + col);
-    const int f16 = g.out_f16;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint4 o;
-      o.x = pack16(f16, v[i * 8 + 0], v[i * 8 + 1]);
-      o.y = pack16(f16, v[i * 8 + 2], v[i * 8 + 3]);
-      o.z = pack16(f16, v[i * 8 + 4], v[i * 8 + 5]);
-      o.w = pack16(f16, v[i * 8 + 6], v[i * 8 + 7]);
-      op[i] = o;
+    for (int k = 0; k < 8; ++k)
+      *reinterpret_cast<float4*>(rowp + ((k ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmO32, col, y0, stage);
+      bulk_commit();
     }
   }
+  if (g.has_out16) {
+    uint8_t* buf = stage + (both ? 0 : parity * 2048);
+    if (lane == 0) {
+      if (both) bulk_wait_read<0>();
+      else bulk_wait_read<1>();
+    }
+    __syncwarp();
+    uint8_t* rowp = buf + lane * 64;
+    const int f16 = g.out_f16;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint4 o;
+      o.x = pack16(f16, v[k * 8 + 0], v[k * 8 + 1]);
+      o.y = pack16(f16, v[k * 8 + 2], v[k * 8 + 3]);
+      o.z = pack16(f16, v[k * 8 + 4], v[k * 8 + 5]);
+      o.w = pack16(f16, v[k * 8 + 6], v[k * 8 + 7]);
+      *reinterpret_cast<uint4*>(rowp + ((k ^ ((lane >> 1) & 3)) << 4)) = o;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmO16, col, y0, buf);
+      bulk_commit();
+    }
+  }
+  return true;
 }
 
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const GemmDev g) {
+              const __grid_constant__ CUtensorMap tmO16,
+              const __grid_constant__ CUtensorMap tmO32, const GemmDev g) {
   using C = GemmCfg<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -149,10 +184,6 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  // the bias of this call's output columns, fp32, once per CTA
-  float* sbias = reinterpret_cast<float*>(smem + C::BIAS_OFF);
-  for (int i = threadIdx.x; i < g.N; i += blockDim.x)
-    sbias[i] = __bfloat162float(g.bias[g.n_off + i]);
   __syncthreads();
   if (!*s_go) return;
 
@@ -234,7 +265,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc_mma_f16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
-                           sdesc_sw128(b0 + k * 32, 16, 1024), IDESC, (kb | k) != 0);
+                          sdesc_sw128(b0 + k * 32, 16, 1024), IDESC, (kb | k) != 0);
           tc_commit(empty + stage);
           issued_any = true;
           if (++stage == STAGES) {
@@ -254,35 +285,54 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     const int q = warp & 3;              // TMEM lane quarter this warp may read
     const int part = (warp - 2) >> 2;    // which half of the BN columns
     constexpr int CH = BN / 64;          // 32-column chunks per warp
-    int local = 0;
+    uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * kStageBuf;
+    int local = 0, nchunk = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
+      const int col0 = g.n_off + nt * BN + part * (BN / 2);
+      const uint4* bptr = reinterpret_cast<const uint4*>(g.bias + col0);
+      uint4 ba[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ba[i] = __ldg(bptr + i);
       if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) break;
       tc_fence_after();
-      const int64_t row = (int64_t)mt * 128 + q * 32 + lane;
+      const int y0 = mt * 128 + q * 32;
+      const int64_t row = (int64_t)y0 + lane;
       const bool valid = row < Mrows;
       const uint32_t tbase = tmem + acc * BN + part * (BN / 2) + ((uint32_t)(q * 32) << 16);
-      const int col0 = g.n_off + nt * BN + part * (BN / 2);
       uint32_t ra[32], rb[32];
       tmem_ld32(tbase, ra);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
-        // the next chunk's TMEM load runs while this chunk is processed
+        // the next chunk's accumulator and bias load while this chunk is stored
         if (c + 1 < CH) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (c & 1) ba[i] = __ldg(bptr + (c + 1) * 4 + i);
+            else bb[i] = __ldg(bptr + (c + 1) * 4 + i);
+          }
           if (c & 1) tmem_ld32(tbase + (c + 1) * 32, ra);
           else tmem_ld32(tbase + (c + 1) * 32, rb);
         }
-        if (c & 1) gemm_epilogue_store<EPI>(g, row, valid, col0 + c * 32, sbias, rb);
-        else gemm_epilogue_store<EPI>(g, row, valid, col0 + c * 32, sbias, ra);
+        bool stored;
+        if (c & 1)
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb, bb,
+                                   stage, nchunk & 1);
+        else
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba,
+                                   stage, nchunk & 1);
+        nchunk += stored ? 1 : 0;
         if (c + 1 < CH) tmem_ld_wait();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
     }
+    if (lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -294,7 +344,8 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 }
 
 template <int BN, int STAGES, int EPI>
-static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, const GemmDev& gd,
+static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
+                              const CUtensorMap& to16, const CUtensorMap& to32, const GemmDev& gd,
                               int grid, cudaStream_t s) {
   using C = GemmCfg<BN, STAGES>;
   auto kfn = k_gemm_tc<BN, STAGES, EPI>;
@@ -304,24 +355,38 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb, cons
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, gd);
+  kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, to16, to32, gd);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   if (c.M_cap <= 0 || c.N <= 0) return cudaSuccess;
-  if (c.N % 64 != 0 || c.K % 64 != 0 || c.N > kMaxBiasN) return cudaErrorInvalidValue;
+  if (c.N % 64 != 0 || c.K % 64 != 0) return cudaErrorInvalidValue;
+  if (c.M_cap > (1ll << 31) - 256) return cudaErrorInvalidValue;
   const int sms = num_sms();
   const int64_t mt = (c.M_cap + 127) / 128;
   int BN = 64;
   if (c.N % 256 == 0 && mt * (c.N / 256) >= 2 * sms) BN = 256;
   else if (c.N % 128 == 0) BN = 128;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to16, to32;
   const bool f16 = c.ab_f16 != 0;
   if (!encode_tmap_2d(&ta, c.A, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.lda * 2, 64, 128, f16))
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d(&tb, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K, (uint64_t)c.ldw * 2, 64,
                       (uint32_t)BN, f16))
+    return cudaErrorInvalidValue;
+  // output maps over the whole [M_cap, ldo] matrix, 32 x 32 boxes; an unused
+  // map is a copy of a valid one (never dereferenced)
+  to16 = ta;
+  to32 = ta;
+  const CUtensorMapDataType t16 =
+      c.out_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (c.out && !encode_tmap_2d_ex(&to16, c.out, (uint64_t)c.M_cap, (uint64_t)c.ldo,
+                                  (uint64_t)c.ldo * 2, 32, 32, t16, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (c.out32 && !encode_tmap_2d_ex(&to32, c.out32, (uint64_t)c.M_cap, (uint64_t)c.ldo,
+                                    (uint64_t)c.ldo * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   GemmDev gd;
   gd.M_cap = c.M_cap;
@@ -331,10 +396,9 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   gd.n_off = c.n_off;
   gd.ab_f16 = c.ab_f16;
   gd.bias = static_cast<const __nv_bfloat16*>(c.bias);
-  gd.out = c.out;
+  gd.has_out16 = c.out != nullptr;
   gd.out_f16 = c.out_f16;
-  gd.ldo = c.ldo;
-  gd.out32 = static_cast<float*>(c.out32);
+  gd.has_out32 = (c.epi == EPI_RESID && c.out32 != nullptr);
   gd.resid = c.resid;
   gd.ldr = c.ldr;
   gd.resid_f32 = c.resid_f32;
@@ -343,13 +407,13 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   const int grid = (int)std::min<int64_t>(tiles, sms);
   LaunchScope ls(kernel_id, s);
   if (c.epi == EPI_SILU) {
-    if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, gd, grid, s);
-    if (BN == 128) return launch_one<128, 6, EPI_SILU>(ta, tb, gd, grid, s);
-    return launch_one<64, 8, EPI_SILU>(ta, tb, gd, grid, s);
+    if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, to16, to32, gd, grid, s);
+    if (BN == 128) return launch_one<128, 6, EPI_SILU>(ta, tb, to16, to32, gd, grid, s);
+    return launch_one<64, 8, EPI_SILU>(ta, tb, to16, to32, gd, grid, s);
   }
-  if (BN == 256) return launch_one<256, 4, EPI_RESID>(ta, tb, gd, grid, s);
-  if (BN == 128) return launch_one<128, 6, EPI_RESID>(ta, tb, gd, grid, s);
-  return launch_one<64, 8, EPI_RESID>(ta, tb, gd, grid, s);
+  if (BN == 256) return launch_one<256, 4, EPI_RESID>(ta, tb, to16, to32, gd, grid, s);
+  if (BN == 128) return launch_one<128, 6, EPI_RESID>(ta, tb, to16, to32, gd, grid, s);
+  return launch_one<64, 8, EPI_RESID>(ta, tb, to16, to32, gd, grid, s);
 }
 
 }  // namespace hstu

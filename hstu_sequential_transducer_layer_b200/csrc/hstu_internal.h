@@ -50,6 +50,10 @@ struct LaunchScope {
 int num_sms();
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).  Returns false if the driver call is unavailable/failed.
+// 2-D map of a row-major matrix with an explicit element type and swizzle.
+bool encode_tmap_2d_ex(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
+                       CUtensorMapDataType dtype, CUtensorMapSwizzle swizzle);
 // 2-D map of a row-major 16-bit matrix (bf16, or fp16 if f16), 128-byte swizzle.
 bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool f16);
