@@ -19,10 +19,10 @@
 //
 // Roles (320 threads): warp 0 fetches items and issues TMA loads (Q once per
 // item; K, V through a 2-stage ring); warp 1 issues the MMAs: S = Q K^T into
-// one of two TMEM buffers, then O += P V into a TMEM accumulator; warps 2-9
+// one of two TMEM buffers, then O += P V (P from TMEM) into a TMEM accumulator; warps 2-9
 // ("P warps", two per TMEM lane quarter, 64 of the 128 columns each) read S
 // with tcgen05.ld, add the bias, apply SiLU, mask, round to fp16 and write P
-// into shared memory in the 128-byte-swizzled K-major layout the MMA reads.
+// back into TMEM (two buffers), from where the P.V MMA reads its A operand.
 // At the end of an item the P warps read O, scale by 1/n (and, for
 // candidates, add the self term) and store fp32.
 //
@@ -69,17 +69,17 @@ template <int D>
 struct AttnCfg {
   static constexpr int NA = D / 64;                       // 64-column swizzle atoms
   static constexpr uint32_t TILE = 128u * D * 2;          // Q, K or V tile bytes
-  static constexpr int P_BUFS = (D == 64) ? 2 : 1;
-  static constexpr uint32_t P_BYTES = 128u * 128u * 2;
+  static constexpr int P_BUFS = 2;                        // P lives in TMEM
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = Q_OFF + TILE;
   static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
-  static constexpr uint32_t P_OFF = V_OFF + 2 * TILE;
-  static constexpr uint32_t WIN_OFF = P_OFF + P_BUFS * P_BYTES;   // 8 warps x 2 x 96 floats
+  static constexpr uint32_t WIN_OFF = V_OFF + 2 * TILE;           // 8 warps x 2 x 96 floats
   static constexpr uint32_t RT_OFF = WIN_OFF + 8 * 2 * 96 * 4;    // 2 ring slots x 256 floats
   static constexpr uint32_t BAR_OFF = RT_OFF + 2 * 256 * 4;
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
-  static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O
+  static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O,
+  static constexpr uint32_t P_COL = O_COL + D;            // then P0, P1 (64 columns each:
+                                                          // 128 fp16 per row, packed in pairs)
 };
 
 enum { MODE_SELF = 0, MODE_CAND = 1 };
@@ -161,7 +161,6 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sQ = smem + C::Q_OFF;
   uint8_t* sK = smem + C::K_OFF;
   uint8_t* sV = smem + C::V_OFF;
-  uint8_t* sP = smem + C::P_OFF;
 
   if (warp == 0) {
     // ------------------------------------------------ item fetch + TMA producer
@@ -273,12 +272,11 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(p_full + pb, pph, ab, a.status)) return false;
         if (jj == 0 && !mbar_wait(o_free, (litem & 1) ^ 1, ab, a.status)) return false;
         tc_fence_after();
-        const uint32_t p_base = smem_u32(sP + pb * C::P_BYTES);
+        const uint32_t p_tmem = tmem + C::P_COL + pb * 64;
         const uint32_t v_base = smem_u32(sV + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_f16_ss(tmem + C::O_COL,
-                        sdesc_sw128(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+        for (int kk = 0; kk < 8; ++kk)  // 16 KV rows per MMA = 8 packed P columns
+          tc_mma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8,
                         sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
                         (jj > 0 || kk > 0) ? 1u : 0u);
         tc_commit(p_free + pb);
@@ -478,23 +476,16 @@ __global__ void __launch_bounds__(320, 1)
         }
 #pragma unroll
         for (int m = 0; m < 16; ++m) bw[m] = bwn[m];
-        // ---- write P (K-major, 128-byte swizzle: chunk m of row r at m ^ (r & 7))
+        // ---- write P into TMEM: this warp's 32 rows, 64 fp16 (32 packed columns)
         const int pb = (int)(pcount % C::P_BUFS);
         if (!mbar_wait_warp(p_free + pb, ((pcount / C::P_BUFS) & 1) ^ 1, ab, a.status)) {
           alive = false;
           break;
         }
-        uint8_t* prow = sP + pb * C::P_BYTES + half * 16384 + r * 128;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          uint4 v;
-          v.x = pk[4 * m + 0];
-          v.y = pk[4 * m + 1];
-          v.z = pk[4 * m + 2];
-          v.w = pk[4 * m + 3];
-          *reinterpret_cast<uint4*>(prow + ((m ^ (r & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();
+        tc_fence_after();
+        tmem_st32(tmem + C::P_COL + pb * 64 + half * 32 + lane_base, pk);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full + pb);
         ++pcount;
