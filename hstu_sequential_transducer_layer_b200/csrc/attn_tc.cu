@@ -17,17 +17,19 @@
 // tiles from L2.  Because there is no softmax, KV tiles combine by plain
 // accumulation in TMEM.
 //
-// Roles (320 threads): warp 0 fetches items and issues TMA loads (Q once per
+// Roles (576 threads): warp 0 fetches items and issues TMA loads (Q once per
 // item; K, V through a 2-stage ring); warp 1 issues the MMAs: S = Q K^T into
-// one of two TMEM buffers, then O += P V (P from TMEM) into a TMEM accumulator; warps 2-9
-// ("P warps", two per TMEM lane quarter, 64 of the 128 columns each) read S
-// with tcgen05.ld, add the bias, apply SiLU, mask, round to fp16 and write P
-// back into TMEM (two buffers), from where the P.V MMA reads its A operand.
+// one of two TMEM buffers, then O += P V (P from TMEM) into a TMEM
+// accumulator; warps 2-17 ("P warps", four per TMEM lane quarter, 32 of the
+// 128 columns each) read S with tcgen05.ld, add the bias, apply SiLU, mask,
+// round to fp16 and write P back into TMEM (two buffers), from where the P.V
+// MMA reads its A operand.  Sixteen P warps with little state each hide the
+// latency of the bias look-ups better than fewer warps with more registers.
 // At the end of an item the P warps read O, scale by 1/n (and, for
-// candidates, add the self term) and store fp32.
+// candidates, add the self term) and store fp32 through TMA bulk stores.
 //
 // Bias per element (causal self-attention): the position bias comes from a
-// per-warp window of the 95 distances its 32 x 64 block spans; the time
+// per-warp window of the 63 distances its 32 x 32 block spans; the time
 // bucket comes precomputed (one byte per element, shared by all heads and
 // layers of a call) and indexes the head's table, which the producer warp
 // stores next to the item in the ring.  Both tables hold half the bias so that
@@ -73,9 +75,11 @@ struct AttnCfg {
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = Q_OFF + TILE;
   static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
-  static constexpr uint32_t WIN_OFF = V_OFF + 2 * TILE;           // 8 warps x 2 x 96 floats
-  static constexpr uint32_t RT_OFF = WIN_OFF + 8 * 2 * 96 * 4;    // 2 ring slots x 256 floats
-  static constexpr uint32_t BAR_OFF = RT_OFF + 2 * 256 * 4;
+  static constexpr int PW = 16;                           // P warps, 4 per TMEM lane quarter
+  static constexpr uint32_t WIN_OFF = V_OFF + 2 * TILE;           // PW warps x 2 x 64 floats
+  static constexpr uint32_t RT_OFF = WIN_OFF + PW * 2 * 64 * 4;   // 2 ring slots x 256 floats
+  static constexpr uint32_t STG_OFF = RT_OFF + 2 * 256 * 4;       // PW warps x 32 x 16 floats
+  static constexpr uint32_t BAR_OFF = STG_OFF + PW * 2048;
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O,
   static constexpr uint32_t P_COL = O_COL + D;            // then P0, P1 (64 columns each:
@@ -91,9 +95,9 @@ typedef AttnItem RingItem;
 DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
-              const AttnDev a) {
+              const __grid_constant__ CUtensorMap tmO, const AttnDev a) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -130,20 +134,21 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
       mbar_init(s_full + i, 1);
-      mbar_init(s_free + i, 8);
-      mbar_init(p_full + i, 8);
+      mbar_init(s_free + i, C::PW);
+      mbar_init(p_full + i, C::PW);
       mbar_init(p_free + i, 1);
       mbar_init(it_full + i, 1);
-      mbar_init(it_empty + i, 9);  // the MMA thread + 8 P warps
+      mbar_init(it_empty + i, 1 + C::PW);  // the MMA thread + the P warps
     }
     mbar_init(o_full, 1);
-    mbar_init(o_free, 8);
+    mbar_init(o_free, C::PW);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmKV);
+    tma_prefetch_desc(&tmO);
   }
   __syncthreads();
   if (!*s_go) return;
@@ -209,6 +214,20 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive(it_full + slot);  // release: slot contents visible to waiters
       ++npub;
       if (x.b < 0) break;
+      if (lane == 0 && nxt.b >= 0) {
+        // warm L2 with the following item's tiles so that its first S does
+        // not wait for HBM
+#pragma unroll
+        for (int at = 0; at < C::NA; ++at)
+          tma_prefetch_l2_2d(&tmQ, a.q_col + nxt.head * D + at * 64, nxt.q_row0);
+        for (int j = 0; j < nxt.nkv; ++j) {
+#pragma unroll
+          for (int at = 0; at < C::NA; ++at) {
+            tma_prefetch_l2_2d(&tmKV, a.k_col + nxt.head * D + at * 64, nxt.kv_row0 + j * 128);
+            tma_prefetch_l2_2d(&tmKV, a.v_col + nxt.head * D + at * 64, nxt.kv_row0 + j * 128);
+          }
+        }
+      }
       if (lane == 0) {
         const AttnItem w = x;
         const int q_row0 = x.q_row0;
@@ -349,11 +368,11 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------ P warps
-    const int pw = warp - 2;         // 0..7
+    const int pw = warp - 2;         // 0..15
     const int q = warp & 3;          // TMEM lane quarter
-    const int half = pw >> 2;        // which 64 of the 128 S columns
+    const int g = pw >> 2;           // which 32 of the 128 S columns
     const int r = q * 32 + lane;     // row inside the 128-row tile
-    float* win2 = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 2 * 96;  // 2 buffers
+    float* win2 = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 2 * 64;  // 2 buffers
     const float* rt_ring = reinterpret_cast<const float*>(smem + C::RT_OFF);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t scount = 0, pcount = 0, ncon = 0;
@@ -379,58 +398,51 @@ __global__ void __launch_bounds__(320, 1)
       const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
       const int t_i = (MODE == MODE_SELF) ? 0 : a.t_req_rel[w.b];
       // Bias inputs of KV tile jt into window buffer `buf` (and, causal mode,
-      // the tile's time-bucket words into bwn).
-      auto prep = [&](int jt, int buf, uint32_t (&bwn)[16]) {
-        float* win = win2 + buf * 96;
+      // the tile's time-bucket words into bwn).  Causal mode: the warp's
+      // 32 x 32 block spans the 63 distances base .. base + 62.
+      auto prep = [&](int jt, int buf, uint32_t (&bwn)[8]) {
+        float* win = win2 + buf * 64;
         if (MODE == MODE_SELF) {
           const uint32_t* tbw = a.tbuckets + (size_t)(w.tile0 + jt) * kBucketTileWords +
-                                (half * 16) * 128 + r;
+                                (g * 8) * 128 + r;
 #pragma unroll
-          for (int m = 0; m < 16; ++m) bwn[m] = __ldg(tbw + m * 128);
-          const int base = (w.qt - jt) * 128 + q * 32 - half * 64 - 63;
+          for (int m = 0; m < 8; ++m) bwn[m] = __ldg(tbw + m * 128);
+          const int base = (w.qt - jt) * 128 + q * 32 - g * 32 - 31;
 #pragma unroll
-          for (int u = 0; u < 3; ++u) {
+          for (int u = 0; u < 2; ++u) {
             const int k = lane + 32 * u;
-            if (k < 95) {
+            if (k < 63) {
               const int dist = base + k;
               win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
             }
           }
         } else {
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int jc = jt * 128 + half * 64 + lane + 32 * u;
-            float bias = 0.f;
-            if (jc < n_kv) {
-              const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
-              bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
-                     __ldg(Rt + log_bucket(gap, a.St, a.Nt));
-            }
-            win[lane + 32 * u] = 0.5f * bias;
+          const int jc = jt * 128 + g * 32 + lane;
+          float bias = 0.f;
+          if (jc < n_kv) {
+            const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
+            bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
+                   __ldg(Rt + log_bucket(gap, a.St, a.Nt));
           }
+          win[lane] = 0.5f * bias;
         }
       };
-      uint32_t bw[16], bwn[16];
+      uint32_t bw[8], bwn[8];
       if (w.nkv > 0) prep(0, 0, bw);
       bool alive = true;
       for (int j = 0; j < w.nkv; ++j) {
         __syncwarp();  // this tile's window is written; the one before it is free
-        const float* win = win2 + (j & 1) * 96;
-        // ---- S tile from TMEM
+        const float* win = win2 + (j & 1) * 64;
+        // ---- S tile from TMEM: this warp's 32 rows x 32 columns
         const int sb = scount & 1;
         if (!mbar_wait_warp(s_full + sb, (scount >> 1) & 1, ab, a.status)) {
           alive = false;
           break;
         }
         tc_fence_after();
-        uint32_t sr[64];
-        {
-          uint32_t (&lo32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-          uint32_t (&hi32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-          tmem_ld32(tmem + sb * 128 + half * 64 + lane_base, lo32);
-          tmem_ld32(tmem + sb * 128 + half * 64 + 32 + lane_base, hi32);
-        }
-        // prefetch the next tile's bias inputs while this tile computes
+        uint32_t sr[32];
+        tmem_ld32(tmem + sb * 128 + g * 32 + lane_base, sr);
+        // fetch the next tile's bias inputs while this tile computes
         if (j + 1 < w.nkv) prep(j + 1, (j + 1) & 1, bwn);
         tmem_ld_wait();
         tc_fence_before();
@@ -438,23 +450,23 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) mbar_arrive(s_free + sb);
         ++scount;
         // ---- P = SiLU(S + bias), masked, fp16
-        uint32_t pk[32];
+        uint32_t pk[16];
         if (MODE == MODE_SELF) {
-          const float* wr = win + lane + 63;
+          const float* wr = win + lane + 31;
           if (j == w.qt) {  // diagonal tile: causal mask j > i
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
+            for (int c = 0; c < 32; c += 2) {
               const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
               const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
               float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, wr[-c]) + rt[b0]);
               float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, wr[-c - 1]) + rt[b1]);
-              if (half * 64 + c > r) p0 = 0.f;
-              if (half * 64 + c + 1 > r) p1 = 0.f;
+              if (g * 32 + c > r) p0 = 0.f;
+              if (g * 32 + c + 1 > r) p1 = 0.f;
               pk[c >> 1] = pack_f16x2_sat(p0, p1);
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
+            for (int c = 0; c < 32; c += 2) {
               const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
               const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
               const float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, wr[-c]) + rt[b0]);
@@ -464,9 +476,9 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         } else {
-          const int limit = n_kv - j * 128 - half * 64;
+          const int limit = n_kv - j * 128 - g * 32;
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
+          for (int c = 0; c < 32; c += 2) {
             float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, win[c]));
             float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, win[c + 1]));
             if (c >= limit) p0 = 0.f;
@@ -475,15 +487,15 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
 #pragma unroll
-        for (int m = 0; m < 16; ++m) bw[m] = bwn[m];
-        // ---- write P into TMEM: this warp's 32 rows, 64 fp16 (32 packed columns)
+        for (int m = 0; m < 8; ++m) bw[m] = bwn[m];
+        // ---- write P into TMEM: this warp's 32 rows, 32 fp16 (16 packed columns)
         const int pb = (int)(pcount % C::P_BUFS);
         if (!mbar_wait_warp(p_free + pb, ((pcount / C::P_BUFS) & 1) ^ 1, ab, a.status)) {
           alive = false;
           break;
         }
         tc_fence_after();
-        tmem_st32(tmem + C::P_COL + pb * 64 + half * 32 + lane_base, pk);
+        tmem_st16(tmem + C::P_COL + pb * 64 + g * 16 + lane_base, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -494,22 +506,23 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(it_empty + slot);
       if (!alive) break;
-      // ---- O epilogue
+      // ---- O epilogue: this warp's 32 rows x OC columns of the head
+      constexpr int OC = D / 4;
       if (!mbar_wait_warp(o_full, litem & 1, ab, a.status)) break;
       tc_fence_after();
-      float o[D / 2];
+      float o[OC];
       if (w.nkv > 0) {
 #pragma unroll
-        for (int c32 = 0; c32 < D / 64; ++c32) {
-          uint32_t orr[32];
-          tmem_ld32(tmem + C::O_COL + half * (D / 2) + c32 * 32 + lane_base, orr);
+        for (int c16 = 0; c16 < OC / 16; ++c16) {
+          uint32_t orr[16];
+          tmem_ld16(tmem + C::O_COL + g * OC + c16 * 16 + lane_base, orr);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[c32 * 32 + i] = __uint_as_float(orr[i]);
+          for (int i = 0; i < 16; ++i) o[c16 * 16 + i] = __uint_as_float(orr[i]);
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < D / 2; ++i) o[i] = 0.f;
+        for (int i = 0; i < OC; ++i) o[i] = 0.f;
       }
       tc_fence_before();
       __syncwarp();
@@ -531,10 +544,9 @@ __global__ void __launch_bounds__(320, 1)
           }
           const float s_self = dot + __ldg(Rp) + __ldg(Rt);
           const float p_self = __half2float(__float2half_rn(silu_fast(s_self)));
-          const uint4* vp =
-              reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + half * (D / 2));
+          const uint4* vp = reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + g * OC);
 #pragma unroll
-          for (int i = 0; i < D / 16; ++i) {
+          for (int i = 0; i < OC / 8; ++i) {
             const uint4 va = vp[i];
             const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
@@ -544,15 +556,41 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        float4* op = reinterpret_cast<float4*>(a.O + (q0 + r) * a.ldo + w.head * D + half * (D / 2));
+      }
+      // ---- store O.  A warp whose 32 rows all belong to the user writes each
+      // 32 x 16 block into its staging buffer (64-byte swizzle) and lets one
+      // TMA bulk store carry it out, so the warp moves on while the data
+      // drains; a warp at the user's ragged end stores its valid rows itself
+      // (the rows after them belong to the next user).
+      if (q * 32 + 32 <= rows_valid) {
+        uint8_t* stg = smem + C::STG_OFF + pw * 2048;
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i)
+        for (int c16 = 0; c16 < OC / 16; ++c16) {
+          if (lane == 0) bulk_wait_read<0>();  // the previous store has read the buffer
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4*>(stg + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_float4(o[c16 * 16 + 4 * k] * inv_n, o[c16 * 16 + 4 * k + 1] * inv_n,
+                            o[c16 * 16 + 4 * k + 2] * inv_n, o[c16 * 16 + 4 * k + 3] * inv_n);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmO, w.head * D + g * OC + c16 * 16, (int)(q0 + q * 32), stg);
+            bulk_commit();
+          }
+        }
+      } else if (row_ok) {
+        float4* op = reinterpret_cast<float4*>(a.O + (q0 + r) * a.ldo + w.head * D + g * OC);
+#pragma unroll
+        for (int i = 0; i < OC / 4; ++i)
           op[i] = make_float4(o[4 * i + 0] * inv_n, o[4 * i + 1] * inv_n, o[4 * i + 2] * inv_n,
                               o[4 * i + 3] * inv_n);
       }
       ++litem;
     }
   }
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // O stores complete before the CTA exits
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -574,7 +612,8 @@ __global__ void __launch_bounds__(320, 1)
 
 template <int D, int MODE>
 static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tkv,
-                                    const AttnDev& ad, int grid, cudaStream_t s) {
+                                    const CUtensorMap& to, const AttnDev& ad, int grid,
+                                    cudaStream_t s) {
   using C = AttnCfg<D>;
   auto kfn = k_attn_tc<D, MODE>;
   static bool attr_set = false;
@@ -583,7 +622,7 @@ static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tk
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kfn<<<grid, 320, C::SMEM, s>>>(tq, tkv, ad);
+  kfn<<<grid, 64 + 32 * C::PW, C::SMEM, s>>>(tq, tkv, to, ad);
   return cudaGetLastError();
 }
 
@@ -603,6 +642,13 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   } else {
     tkv = tq;
   }
+  // O: fp32 [q_rows_cap, h * d_v] with row stride ldo; 16-column x 32-row
+  // boxes (64-byte rows) for the epilogue's bulk stores.
+  CUtensorMap to;
+  if (!encode_tmap_2d_ex(&to, c.O, (uint64_t)c.q_rows_cap, (uint64_t)c.h * c.dv,
+                         (uint64_t)c.ldo * 4, 16, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                         CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
   AttnDev ad;
   ad.items = c.items;
   ad.n_items = c.n_items;
@@ -630,10 +676,10 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());
   LaunchScope ls(c.mode == MODE_SELF ? K_ATTN : K_ATTN_CAND, s);
   if (c.mode == MODE_SELF)
-    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF>(tq, tkv, ad, grid, s)
-                       : launch_attn_inst<128, MODE_SELF>(tq, tkv, ad, grid, s);
-  return c.dqk == 64 ? launch_attn_inst<64, MODE_CAND>(tq, tkv, ad, grid, s)
-                     : launch_attn_inst<128, MODE_CAND>(tq, tkv, ad, grid, s);
+    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF>(tq, tkv, to, ad, grid, s)
+                       : launch_attn_inst<128, MODE_SELF>(tq, tkv, to, ad, grid, s);
+  return c.dqk == 64 ? launch_attn_inst<64, MODE_CAND>(tq, tkv, to, ad, grid, s)
+                     : launch_attn_inst<128, MODE_CAND>(tq, tkv, to, ad, grid, s);
 }
 
 }  // namespace hstu
