@@ -17,8 +17,9 @@
 // tiles from L2.  Because there is no softmax, KV tiles combine by plain
 // accumulation in TMEM.
 //
-// Roles (576 threads): warp 0 fetches items and issues TMA loads (Q once per
-// item; K, V through a 2-stage ring); warp 1 issues the MMAs: S = Q K^T into
+// Roles (608 threads): warp 18 claims items and publishes them into a 2-slot
+// ring; warp 0 issues the TMA loads (lane 0: Q once per item and the K tiles,
+// lane 1: the V tiles, each through a 2-stage ring); warp 1 issues the MMAs: S = Q K^T into
 // one of two TMEM buffers, then O += P V (P from TMEM) into a TMEM
 // accumulator; warps 2-17 ("P warps", four per TMEM lane quarter, 32 of the
 // 128 columns each) read S with tcgen05.ld, add the bias, apply SiLU, mask,
@@ -95,7 +96,7 @@ typedef AttnItem RingItem;
 DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
+__global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
               const __grid_constant__ CUtensorMap tmO, const AttnDev a) {
   using C = AttnCfg<D>;
@@ -105,8 +106,8 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;     // [2]
-  uint64_t* kv_empty = bars + 4;    // [2]
+  uint64_t* k_full = bars + 2;      // [2]
+  uint64_t* k_empty = bars + 4;     // [2]
   uint64_t* s_full = bars + 6;      // [2]
   uint64_t* s_free = bars + 8;      // [2]
   uint64_t* p_full = bars + 10;     // [2]
@@ -116,7 +117,9 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
   uint64_t* drain = bars + 16;
   uint64_t* it_full = bars + 17;    // [2] item ring
   uint64_t* it_empty = bars + 19;   // [2]
-  RingItem* ring = reinterpret_cast<RingItem*>(bars + 21);   // [2], 32 B each
+  uint64_t* v_full = bars + 21;     // [2]
+  uint64_t* v_empty = bars + 23;    // [2]
+  RingItem* ring = reinterpret_cast<RingItem*>(bars + 25);   // [2], 32 B each
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + 2);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
@@ -131,14 +134,16 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(kv_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+      mbar_init(v_full + i, 1);
+      mbar_init(v_empty + i, 1);
       mbar_init(s_full + i, 1);
       mbar_init(s_free + i, C::PW);
       mbar_init(p_full + i, C::PW);
       mbar_init(p_free + i, 1);
       mbar_init(it_full + i, 1);
-      mbar_init(it_empty + i, 1 + C::PW);  // the MMA thread + the P warps
+      mbar_init(it_empty + i, 3 + C::PW);  // 2 loader lanes + the MMA thread + the P warps
     }
     mbar_init(o_full, 1);
     mbar_init(o_free, C::PW);
@@ -168,139 +173,98 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
   uint8_t* sV = smem + C::V_OFF;
 
   if (warp == 0) {
-    // ------------------------------------------------ item fetch + TMA producer
-    // Lane 0 fetches items and issues every TMA load; the whole warp fills the
-    // ring slot's halved time-bias table.
-    float* rt_ring = reinterpret_cast<float*>(smem + C::RT_OFF);
-    int kst = 0, litem = 0;
-    uint32_t kph = 0, issued = 0, last_par = 0, q_issued = 0, q_par = 0, npub = 0;
-    bool ok = true;
-    // Work indices are claimed two items ahead and the next item's entry is
-    // read one item ahead, so neither latency sits between two items.
-    auto claim = [&]() {
-      int v = 0;
-      if (lane == 0) v = atomicAdd(a.work_next, 1);
-      return __shfl_sync(0xffffffffu, v, 0);
-    };
-    auto entry = [&](int idx) {
-      RingItem x;
-      if (idx < n_items) x = a.items[idx];
-      else x = AttnItem{-1, 0, 0, 0, 0, 0, 0, 0, 0};
-      return x;
-    };
-    int idx_next = claim();
-    int idx_after = claim();
-    RingItem nxt = entry(idx_next);
-    for (;;) {
-      const RingItem x = nxt;
-      if (x.b >= 0) {
-        idx_next = idx_after;
-        idx_after = claim();
-        nxt = entry(idx_next);
-      }
-      const int slot = npub & 1;
-      bool okw = true;
-      if (lane == 0) okw = mbar_wait(it_empty + slot, ((npub >> 1) & 1) ^ 1, ab, a.status);
-      if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) {
-        ok = false;
-        break;
-      }
-      if (MODE == MODE_SELF && x.b >= 0) {
-        const float* Rt = a.rab_time + (size_t)x.head * a.Nt;
-        for (int k = lane; k < a.Nt; k += 32) rt_ring[slot * 256 + k] = 0.5f * __ldg(Rt + k);
-      }
-      if (lane == 0) ring[slot] = x;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(it_full + slot);  // release: slot contents visible to waiters
-      ++npub;
-      if (x.b < 0) break;
-      if (lane == 0 && nxt.b >= 0) {
-        // warm L2 with the following item's tiles so that its first S does
-        // not wait for HBM
-#pragma unroll
-        for (int at = 0; at < C::NA; ++at)
-          tma_prefetch_l2_2d(&tmQ, a.q_col + nxt.head * D + at * 64, nxt.q_row0);
-        for (int j = 0; j < nxt.nkv; ++j) {
-#pragma unroll
-          for (int at = 0; at < C::NA; ++at) {
-            tma_prefetch_l2_2d(&tmKV, a.k_col + nxt.head * D + at * 64, nxt.kv_row0 + j * 128);
-            tma_prefetch_l2_2d(&tmKV, a.v_col + nxt.head * D + at * 64, nxt.kv_row0 + j * 128);
-          }
-        }
-      }
-      if (lane == 0) {
-        const AttnItem w = x;
-        const int q_row0 = x.q_row0;
-        const int kv_row0 = x.kv_row0;
-        if (!mbar_wait(q_empty, (litem & 1) ^ 1, ab, a.status)) {
+    // ------------------------------------------------ TMA loaders
+    // Lane 0 loads Q (once per item) and the K tiles, lane 1 the V tiles, each
+    // through its own 2-stage ring: a K stage is free again as soon as its
+    // S = Q K^T has run, so K runs ahead of V by the length of the P stage.
+    if (lane < 2) {
+      const bool kq = (lane == 0);
+      uint64_t* full = kq ? k_full : v_full;
+      uint64_t* empty = kq ? k_empty : v_empty;
+      uint8_t* buf = kq ? sK : sV;
+      const int col = kq ? a.k_col : a.v_col;
+      uint32_t ncon = 0, st = 0, ph = 0, issued = 0, last_par = 0, q_par = 0;
+      int litem = 0;
+      bool ok = true, q_issued = false;
+      for (;;) {
+        const int slot = ncon & 1;
+        if (!mbar_wait(it_full + slot, (ncon >> 1) & 1, ab, a.status)) {
           ok = false;
-        } else {
+          break;
+        }
+        const AttnItem w = ring[slot];
+        mbar_arrive(it_empty + slot);
+        ++ncon;
+        if (w.b < 0) break;
+        if (kq) {
+          if (!mbar_wait(q_empty, (litem & 1) ^ 1, ab, a.status)) {
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(q_full, C::TILE);
 #pragma unroll
           for (int at = 0; at < C::NA; ++at)
-            tma_load_2d(sQ + at * 16384, &tmQ, a.q_col + w.head * D + at * 64, q_row0, q_full);
-          q_issued = 1;
+            tma_load_2d(sQ + at * 16384, &tmQ, a.q_col + w.head * D + at * 64, w.q_row0, q_full);
+          q_issued = true;
           q_par = litem & 1;
-          for (int j = 0; j < w.nkv; ++j) {
-            if (!mbar_wait(kv_empty + kst, kph ^ 1, ab, a.status)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(kv_full + kst, 2 * C::TILE);
-            const int y = kv_row0 + j * 128;
+        }
+        for (int j = 0; j < w.nkv; ++j) {
+          if (!mbar_wait(empty + st, ph ^ 1, ab, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full + st, C::TILE);
 #pragma unroll
-            for (int at = 0; at < C::NA; ++at) {
-              tma_load_2d(sK + kst * C::TILE + at * 16384, &tmKV, a.k_col + w.head * D + at * 64,
-                          y, kv_full + kst);
-              tma_load_2d(sV + kst * C::TILE + at * 16384, &tmKV, a.v_col + w.head * D + at * 64,
-                          y, kv_full + kst);
-            }
-            issued |= 1u << kst;
-            last_par = (last_par & ~(1u << kst)) | (kph << kst);
-            if (++kst == 2) {
-              kst = 0;
-              kph ^= 1;
-            }
+          for (int at = 0; at < C::NA; ++at)
+            tma_load_2d(buf + st * C::TILE + at * 16384, &tmKV, col + w.head * D + at * 64,
+                        w.kv_row0 + j * 128, full + st);
+          issued |= 1u << st;
+          last_par = (last_par & ~(1u << st)) | (ph << st);
+          if (++st == 2) {
+            st = 0;
+            ph ^= 1;
           }
         }
+        if (!ok) break;
+        ++litem;
       }
-      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-        ok = false;
-        break;
+      if (!ok) {  // let every load already in flight land before the CTA exits
+        AbortState tmp{0};
+        for (int s2 = 0; s2 < 2; ++s2)
+          if ((issued >> s2) & 1u) mbar_wait(full + s2, (last_par >> s2) & 1u, &tmp, nullptr);
+        if (q_issued) mbar_wait(q_full, q_par, &tmp, nullptr);
       }
-      ++litem;
-    }
-    if (!ok && lane == 0) {  // let every load already in flight land before the CTA exits
-      AbortState tmp{0};
-      for (int s2 = 0; s2 < 2; ++s2)
-        if ((issued >> s2) & 1u) mbar_wait(kv_full + s2, (last_par >> s2) & 1u, &tmp, nullptr);
-      if (q_issued) mbar_wait(q_full, q_par, &tmp, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_f16_f32(128, 128, 0, 0, 1);
       constexpr uint32_t IDESC_O = idesc_f16_f32(128, D, 0, 1, 1);  // V is MN-major
-      int kst = 0, litem = 0;
-      uint32_t kph = 0, scount = 0, pcount = 0, ncon = 0;
+      int litem = 0;
+      uint32_t kst = 0, kph = 0, vst = 0, vph = 0, scount = 0, pcount = 0, ncon = 0;
       bool ok = true, any = false;
       const uint32_t q_base = smem_u32(sQ);
-      auto issue_pv = [&](int jj, int st, int nkv) -> bool {
+      auto issue_pv = [&](int jj, int nkv) -> bool {
         const int pb = (int)(pcount % C::P_BUFS);
         const uint32_t pph = (pcount / C::P_BUFS) & 1;
         if (!mbar_wait(p_full + pb, pph, ab, a.status)) return false;
         if (jj == 0 && !mbar_wait(o_free, (litem & 1) ^ 1, ab, a.status)) return false;
+        if (!mbar_wait(v_full + vst, vph, ab, a.status)) return false;
         tc_fence_after();
         const uint32_t p_tmem = tmem + C::P_COL + pb * 64;
-        const uint32_t v_base = smem_u32(sV + st * C::TILE);
+        const uint32_t v_base = smem_u32(sV + vst * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // 16 KV rows per MMA = 8 packed P columns
           tc_mma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8,
                         sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
                         (jj > 0 || kk > 0) ? 1u : 0u);
         tc_commit(p_free + pb);
-        tc_commit(kv_empty + st);
+        tc_commit(v_empty + vst);
         if (jj == nkv - 1) tc_commit(o_full);
+        if (++vst == 2) {
+          vst = 0;
+          vph ^= 1;
+        }
         ++pcount;
         any = true;
         return true;
@@ -318,9 +282,8 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
           break;
         }
         tc_fence_after();
-        int prev = -1;
         for (int j = 0; j < nkv; ++j) {
-          if (!mbar_wait(kv_full + kst, kph, ab, a.status)) {
+          if (!mbar_wait(k_full + kst, kph, ab, a.status)) {
             ok = false;
             break;
           }
@@ -338,22 +301,22 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
                           sdesc_sw128(k_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                           IDESC_S, kk > 0 ? 1u : 0u);
           tc_commit(s_full + sb);
+          tc_commit(k_empty + kst);
           if (j == nkv - 1) tc_commit(q_empty);  // P.V does not read Q: free it early
-          ++scount;
-          any = true;
-          if (j > 0 && !issue_pv(j - 1, prev, nkv)) {
-            ok = false;
-            break;
-          }
-          prev = kst;
           if (++kst == 2) {
             kst = 0;
             kph ^= 1;
           }
+          ++scount;
+          any = true;
+          if (j > 0 && !issue_pv(j - 1, nkv)) {
+            ok = false;
+            break;
+          }
         }
         if (!ok) break;
         if (nkv > 0) {
-          if (!issue_pv(nkv - 1, prev, nkv)) break;
+          if (!issue_pv(nkv - 1, nkv)) break;
         } else {
           tc_commit(o_full);  // nothing to accumulate: O is taken as zero
           tc_commit(q_empty);
@@ -366,7 +329,7 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
         mbar_wait(drain, 0, &tmp, nullptr);
       }
     }
-  } else {
+  } else if (warp < 2 + C::PW) {
     // ------------------------------------------------ P warps
     const int pw = warp - 2;         // 0..15
     const int q = warp & 3;          // TMEM lane quarter
@@ -589,8 +552,57 @@ __global__ void __launch_bounds__(64 + 32 * AttnCfg<D>::PW, 1)
       }
       ++litem;
     }
+  } else if (warp == 2 + C::PW) {
+    // ------------------------------------------------ item fetcher
+    // Claims work items (dynamic, one atomic per item), publishes each into
+    // the 2-slot ring with its head's halved time-bias table (causal mode),
+    // and warms L2 with the item's Q/K/V tiles, two items ahead of the P warps.
+    float* rt_ring = reinterpret_cast<float*>(smem + C::RT_OFF);
+    auto claim = [&]() {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(a.work_next, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    // An item is claimed only once a ring slot is free, so a CTA never holds
+    // more than two unstarted items (a short tail at the end of the launch).
+    uint32_t npub = 0;
+    for (;;) {
+      const int slot = npub & 1;
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(it_empty + slot, ((npub >> 1) & 1) ^ 1, ab, a.status);
+      if (!__shfl_sync(0xffffffffu, okw ? 1 : 0, 0)) break;
+      const int idx = claim();
+      RingItem x;
+      if (idx < n_items) x = a.items[idx];
+      else x = AttnItem{-1, 0, 0, 0, 0, 0, 0, 0, 0};
+      if (MODE == MODE_SELF && x.b >= 0) {
+        const float* Rt = a.rab_time + (size_t)x.head * a.Nt;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int k = lane + 32 * u;
+          if (k < a.Nt) rt_ring[slot * 256 + k] = 0.5f * __ldg(Rt + k);
+        }
+      }
+      if (lane == 0) ring[slot] = x;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(it_full + slot);  // release: slot contents visible to waiters
+      ++npub;
+      if (x.b < 0) break;
+      if (lane == 0) {
+#pragma unroll
+        for (int at = 0; at < C::NA; ++at)
+          tma_prefetch_l2_2d(&tmQ, a.q_col + x.head * D + at * 64, x.q_row0);
+        for (int j = 0; j < x.nkv; ++j) {
+#pragma unroll
+          for (int at = 0; at < C::NA; ++at) {
+            tma_prefetch_l2_2d(&tmKV, a.k_col + x.head * D + at * 64, x.kv_row0 + j * 128);
+            tma_prefetch_l2_2d(&tmKV, a.v_col + x.head * D + at * 64, x.kv_row0 + j * 128);
+          }
+        }
+      }
+    }
   }
-  if (warp >= 2 && lane == 0) bulk_wait_all();  // O stores complete before the CTA exits
+  if (warp >= 2 && warp < 2 + C::PW && lane == 0) bulk_wait_all();  // O stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -622,7 +634,7 @@ static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tk
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kfn<<<grid, 64 + 32 * C::PW, C::SMEM, s>>>(tq, tkv, to, ad);
+  kfn<<<grid, 96 + 32 * C::PW, C::SMEM, s>>>(tq, tkv, to, ad);
   return cudaGetLastError();
 }
 
