@@ -77,13 +77,58 @@ def mfalcon_flops(dims, n_layers, hist_lens, cands):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons sampled every ~2 ms while the timed
+    region runs (NVML from a thread; nvidia-smi at 100 ms if NVML is absent).
+    Samples also go to gpurun_out/clocks_rank<i>.csv."""
+
+    NAMES = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+             "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+             "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+             "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+             "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.thread = None
+        self.samples = []           # (sm_mhz, max_mhz, reason bitmask)
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:  # the CUDA device's own GPU, whatever CUDA_VISIBLE_DEVICES maps it to
+            uid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            if not uid.startswith("GPU-"):
+                uid = "GPU-" + uid
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, nv, hdl):
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = nv.nvmlDeviceGetMaxClockInfo(hdl, nv.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(hdl, nv.NVML_CLOCK_SM), mx, get_r(hdl)))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
     def __enter__(self):
+        import threading
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        self.stop = False
+        try:
+            nv, hdl = self._nvml_handle()
+            self.nv = nv
+            self.thread = threading.Thread(target=self._poll, args=(nv, hdl), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -97,6 +142,13 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
+            with open(self.path, "w") as f:
+                f.write("sm_mhz,max_sm_mhz,reasons_mask\n")
+                for sm, mx, r in self.samples:
+                    f.write(f"{sm},{mx},{r:#x}\n")
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -106,6 +158,18 @@ class ClockSampler:
             self.f.close()
 
     def summary(self):
+        if self.thread is not None:
+            if not self.samples:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            reasons = set()
+            for _, _, r in self.samples:
+                for nm, attr in self.NAMES.items():
+                    bit = getattr(self.nv, attr, 0)
+                    if bit and (r & bit):
+                        reasons.add(nm)
+            return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                    "sm_max_mhz": max(s[1] for s in self.samples),
+                    "samples": len(self.samples), "source": "nvml", "reasons": sorted(reasons)}
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons = [], [], set()
@@ -125,7 +189,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "source": "nvidia-smi", "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------- traffic from ncu

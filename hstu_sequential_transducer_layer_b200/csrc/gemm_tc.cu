@@ -39,14 +39,17 @@ struct GemmDev {
 constexpr int kEpiThreads = 256;      // 8 epilogue warps
 constexpr uint32_t kStageBuf = 4096;  // per-warp output staging bytes (32 x 32 fp32)
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int EPI>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t OUT_OFF = STAGES * STAGE_BYTES;             // 8 x 4 KB staging
-  static constexpr uint32_t BAR_OFF = OUT_OFF + (kEpiThreads / 32) * kStageBuf;
+  // EPI_RESID: 8 x 4 KB buffers that TMA fills with the next fp32 residual chunk
+  static constexpr uint32_t RES_OFF = OUT_OFF + (kEpiThreads / 32) * kStageBuf;
+  static constexpr uint32_t BAR_OFF =
+      RES_OFF + (EPI == EPI_RESID ? (kEpiThreads / 32) * kStageBuf : 0);
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
@@ -60,7 +63,7 @@ struct GemmCfg {
 template <int EPI>
 DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorMap* tmO32,
                      int64_t row, bool valid, int col, int y0, const uint32_t (&r)[32],
-                     const uint4 (&bias)[4], uint8_t* stage, int parity) {
+                     const uint4 (&bias)[4], uint8_t* stage, int parity, const uint8_t* rsm) {
   const int lane = threadIdx.x & 31;
   float v[32];
 #pragma unroll
@@ -75,6 +78,15 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   if (EPI == EPI_SILU) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
+  } else if (rsm != nullptr) {  // fp32 residual chunk staged by TMA (128-byte swizzle)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 rr = *reinterpret_cast<const float4*>(rsm + lane * 128 + ((k ^ (lane & 7)) << 4));
+      v[4 * k + 0] += rr.x;
+      v[4 * k + 1] += rr.y;
+      v[4 * k + 2] += rr.z;
+      v[4 * k + 3] += rr.w;
+    }
   } else if (valid) {
     if (g.resid_f32) {
       const float4* rp = reinterpret_cast<const float4*>(
@@ -151,8 +163,9 @@ template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmO16,
-              const __grid_constant__ CUtensorMap tmO32, const GemmDev g) {
-  using C = GemmCfg<BN, STAGES>;
+              const __grid_constant__ CUtensorMap tmO32, const __grid_constant__ CUtensorMap tmR,
+              const GemmDev g) {
+  using C = GemmCfg<BN, STAGES, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -161,7 +174,8 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* rbar = drain + 1;  // [8] residual chunk landed (per epilogue warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 8);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
 
@@ -178,6 +192,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     mbar_init(tempty + 0, kEpiThreads / 32);
     mbar_init(tempty + 1, kEpiThreads / 32);
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(rbar + i, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -287,7 +302,24 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     constexpr int CH = BN / 64;          // 32-column chunks per warp
     uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * kStageBuf;
     int local = 0, nchunk = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+    // fp32 residual: lane 0 has TMA bring the next 32 x 32 chunk into the
+    // warp's buffer while the current one is computed and stored
+    const bool rtma = (EPI == EPI_RESID) && g.resid_f32;
+    uint8_t* rbuf = smem + C::RES_OFF + (warp - 2) * kStageBuf;
+    uint64_t* rb = rbar + (warp - 2);
+    uint32_t rpar = 0;
+    bool r_pending = false, alive = true;
+    auto r_issue = [&](int t_, int c_) {
+      const int mt_ = t_ / n_tiles, nt_ = t_ - (t_ / n_tiles) * n_tiles;
+      mbar_arrive_expect_tx(rb, kStageBuf);
+      tma_load_2d(rbuf, &tmR, g.n_off + nt_ * BN + part * (BN / 2) + c_ * 32, mt_ * 128 + q * 32,
+                  rb);
+    };
+    if (rtma && lane == 0 && (int)blockIdx.x < tiles) {
+      r_issue(blockIdx.x, 0);
+      r_pending = true;
+    }
+    for (int t = blockIdx.x; t < tiles && alive; t += gridDim.x, ++local) {
       const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
@@ -302,7 +334,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       const int64_t row = (int64_t)y0 + lane;
       const bool valid = row < Mrows;
       const uint32_t tbase = tmem + acc * BN + part * (BN / 2) + ((uint32_t)(q * 32) << 16);
-      uint32_t ra[32], rb[32];
+      uint32_t ra[32], rb_acc[32];
       tmem_ld32(tbase, ra);
       tmem_ld_wait();
 #pragma unroll
@@ -315,21 +347,51 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
             else bb[i] = __ldg(bptr + (c + 1) * 4 + i);
           }
           if (c & 1) tmem_ld32(tbase + (c + 1) * 32, ra);
-          else tmem_ld32(tbase + (c + 1) * 32, rb);
+          else tmem_ld32(tbase + (c + 1) * 32, rb_acc);
+        }
+        const uint8_t* rsm = nullptr;
+        if (rtma) {
+          if (!mbar_wait_warp(rb, rpar, ab, g.status)) {
+            alive = false;
+            break;
+          }
+          rpar ^= 1;
+          rsm = rbuf;
         }
         bool stored;
         if (c & 1)
-          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb, bb,
-                                   stage, nchunk & 1);
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb_acc, bb,
+                                   stage, nchunk & 1, rsm);
         else
           stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba,
-                                   stage, nchunk & 1);
+                                   stage, nchunk & 1, rsm);
         nchunk += stored ? 1 : 0;
+        if (rtma) {
+          __syncwarp();  // every lane has read the residual chunk
+          if (lane == 0) {
+            r_pending = false;
+            int tn = t, cn = c + 1;
+            if (cn == CH) {
+              tn = t + (int)gridDim.x;
+              cn = 0;
+            }
+            if (tn < tiles) {
+              fence_proxy_async_smem();
+              r_issue(tn, cn);
+              r_pending = true;
+            }
+          }
+        }
         if (c + 1 < CH) tmem_ld_wait();
       }
+      if (!alive) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
+    }
+    if (lane == 0 && r_pending) {  // a residual load still in flight must land first
+      AbortState tmp{0};
+      mbar_wait(rb, rpar, &tmp, nullptr);
     }
     if (lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
     __syncwarp();
@@ -345,9 +407,9 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 
 template <int BN, int STAGES, int EPI>
 static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
-                              const CUtensorMap& to16, const CUtensorMap& to32, const GemmDev& gd,
-                              int grid, cudaStream_t s) {
-  using C = GemmCfg<BN, STAGES>;
+                              const CUtensorMap& to16, const CUtensorMap& to32,
+                              const CUtensorMap& tr, const GemmDev& gd, int grid, cudaStream_t s) {
+  using C = GemmCfg<BN, STAGES, EPI>;
   auto kfn = k_gemm_tc<BN, STAGES, EPI>;
   static bool attr_set = false;  // per instantiation; the attribute is per device function
   if (!attr_set) {
@@ -355,7 +417,7 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, to16, to32, gd);
+  kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, to16, to32, tr, gd);
   return cudaGetLastError();
 }
 
@@ -368,7 +430,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   int BN = 64;
   if (c.N % 256 == 0 && mt * (c.N / 256) >= 2 * sms) BN = 256;
   else if (c.N % 128 == 0) BN = 128;
-  CUtensorMap ta, tb, to16, to32;
+  CUtensorMap ta, tb, to16, to32, tr;
   const bool f16 = c.ab_f16 != 0;
   if (!encode_tmap_2d(&ta, c.A, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.lda * 2, 64, 128, f16))
     return cudaErrorInvalidValue;
@@ -387,6 +449,13 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   if (c.out32 && !encode_tmap_2d_ex(&to32, c.out32, (uint64_t)c.M_cap, (uint64_t)c.ldo,
                                     (uint64_t)c.ldo * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  // fp32 residual: [M_cap, n_off + N] with row stride ldr, 32 x 32 boxes
+  tr = ta;
+  if (c.epi == EPI_RESID && c.resid_f32 &&
+      !encode_tmap_2d_ex(&tr, c.resid, (uint64_t)c.M_cap, (uint64_t)(c.n_off + c.N),
+                         (uint64_t)c.ldr * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   GemmDev gd;
   gd.M_cap = c.M_cap;
@@ -407,13 +476,14 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   const int grid = (int)std::min<int64_t>(tiles, sms);
   LaunchScope ls(kernel_id, s);
   if (c.epi == EPI_SILU) {
-    if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, to16, to32, gd, grid, s);
-    if (BN == 128) return launch_one<128, 6, EPI_SILU>(ta, tb, to16, to32, gd, grid, s);
-    return launch_one<64, 8, EPI_SILU>(ta, tb, to16, to32, gd, grid, s);
+    if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
+    if (BN == 128) return launch_one<128, 6, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
+    return launch_one<64, 8, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
   }
-  if (BN == 256) return launch_one<256, 4, EPI_RESID>(ta, tb, to16, to32, gd, grid, s);
-  if (BN == 128) return launch_one<128, 6, EPI_RESID>(ta, tb, to16, to32, gd, grid, s);
-  return launch_one<64, 8, EPI_RESID>(ta, tb, to16, to32, gd, grid, s);
+  // the residual buffers take one A/B stage's worth of shared memory
+  if (BN == 256) return launch_one<256, 3, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
+  if (BN == 128) return launch_one<128, 4, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
+  return launch_one<64, 6, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
 }
 
 }  // namespace hstu
