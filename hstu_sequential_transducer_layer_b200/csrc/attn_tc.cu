@@ -17,18 +17,19 @@
 // tiles from L2.  Because there is no softmax, KV tiles combine by plain
 // accumulation in TMEM.
 //
-// Roles (608 threads): warp 18 claims items and publishes them into a 2-slot
-// ring; warp 0 issues the TMA loads (lane 0: Q once per item and the K tiles,
-// lane 1: the V tiles, each through a 2-stage ring); warp 1 issues the MMAs: S = Q K^T into
-// one of two TMEM buffers, then O += P V (P from TMEM) into a TMEM
-// accumulator; warps 2-17 ("P warps", four per TMEM lane quarter, 32 of the
-// 128 columns each) read S with tcgen05.ld, add the bias, apply SiLU, mask,
-// round to fp16 and write P back into TMEM (two buffers), from where the P.V
-// MMA reads its A operand.  Sixteen P warps with little state each hide the
-// latency of the bias look-ups better than fewer warps with more registers.
-// At the end of an item the P warps read O, scale by 1/n (and, for
-// candidates, add the self term) and store fp32 through TMA bulk stores.
-//
+// Roles (768 threads, six warpgroups): warp 2 claims items and publishes them
+// into a 2-slot ring; warp 0 issues the TMA loads (lane 0: Q once per item and
+// the K tiles, lane 1: the V tiles, each through a 2-stage ring); warp 1
+// issues the MMAs: S = Q K^T into one of two TMEM buffers, then O += P V (P
+// from TMEM) into a TMEM accumulator; warps 4-19 ("P warps", four per TMEM
+// lane quarter, 32 of the 128 columns each) read S with tcgen05.ld, add the
+// bias, apply SiLU, mask, round to fp16 and write P back into TMEM (two
+// buffers), from where the P.V MMA reads its A operand; warps 20-23 (one per
+// lane quarter) read O at the end of an item, scale by 1/n (and, for
+// candidates, add the self term) and store fp32 through TMA bulk stores while
+// the P warps already work on the next item.  Sixteen P warps with little
+// state each hide the latency of the bias look-ups better than fewer warps
+// with more registers; every role fits in 80 registers.
 // Bias per element (causal self-attention): the position bias comes from a
 // per-warp window of the 63 distances its 32 x 32 block spans; the time
 // bucket comes precomputed (one byte per element, shared by all heads and
@@ -74,14 +75,22 @@ struct AttnCfg {
   static constexpr uint32_t TILE = 128u * D * 2;          // Q, K or V tile bytes
   static constexpr int P_BUFS = 2;                        // P lives in TMEM
   static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t K_OFF = Q_OFF + TILE;
-  static constexpr uint32_t V_OFF = K_OFF + 2 * TILE;
-  static constexpr int PW = 16;                           // P warps, 4 per TMEM lane quarter
-  static constexpr uint32_t WIN_OFF = V_OFF + 2 * TILE;           // PW warps x 2 x 64 floats
+  static constexpr int QS = 2, KS = 2, VS = 2;            // Q, K and V ring stages
+  static constexpr uint32_t K_OFF = Q_OFF + QS * TILE;
+  static constexpr uint32_t V_OFF = K_OFF + KS * TILE;
+  // Warp roles: 0 loaders, 1 MMA, 2 item fetcher, 3 idle (warpgroup 0);
+  // 4..19 P warps, four per TMEM lane quarter (warpgroups 1-4); 20..23 O
+  // epilogue, one per lane quarter (warpgroup 5).
+  static constexpr int PW = 16, EW = 4;
+  static constexpr int FETCH_WARP = 2, P_WARP0 = 4, EPI_WARP0 = P_WARP0 + PW;
+  static constexpr int THREADS = 32 * (EPI_WARP0 + EW);
+  static constexpr uint32_t WIN_OFF = V_OFF + VS * TILE;          // PW warps x 2 x 64 floats
   static constexpr uint32_t RT_OFF = WIN_OFF + PW * 2 * 64 * 4;   // 2 ring slots x 256 floats
-  static constexpr uint32_t STG_OFF = RT_OFF + 2 * 256 * 4;       // PW warps x 32 x 16 floats
-  static constexpr uint32_t BAR_OFF = STG_OFF + PW * 2048;
+  static constexpr uint32_t STG_OFF = RT_OFF + 2 * 256 * 4;       // EW warps x 2 x 32 x 16 floats
+  static constexpr uint32_t BAR_OFF = STG_OFF + EW * 4096;
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
+  static_assert(QS == 2 && KS <= 4 && VS <= 4, "barrier slots");
+  static_assert(SMEM <= 232448, "shared memory per CTA");
   static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O,
   static constexpr uint32_t P_COL = O_COL + D;            // then P0, P1 (64 columns each:
                                                           // 128 fp16 per row, packed in pairs)
@@ -96,7 +105,7 @@ typedef AttnItem RingItem;
 DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
+__global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
               const __grid_constant__ CUtensorMap tmO, const AttnDev a) {
   using C = AttnCfg<D>;
@@ -104,10 +113,10 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;      // [2]
-  uint64_t* k_empty = bars + 4;     // [2]
+  uint64_t* q_full = bars + 0;      // [QS]
+  uint64_t* q_empty = bars + 2;     // [QS]
+  uint64_t* k_full = bars + 25;     // [KS]
+  uint64_t* k_empty = bars + 29;    // [KS]
   uint64_t* s_full = bars + 6;      // [2]
   uint64_t* s_free = bars + 8;      // [2]
   uint64_t* p_full = bars + 10;     // [2]
@@ -117,9 +126,9 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
   uint64_t* drain = bars + 16;
   uint64_t* it_full = bars + 17;    // [2] item ring
   uint64_t* it_empty = bars + 19;   // [2]
-  uint64_t* v_full = bars + 21;     // [2]
-  uint64_t* v_empty = bars + 23;    // [2]
-  RingItem* ring = reinterpret_cast<RingItem*>(bars + 25);   // [2], 32 B each
+  uint64_t* v_full = bars + 33;     // [VS]
+  uint64_t* v_empty = bars + 37;    // [VS]
+  RingItem* ring = reinterpret_cast<RingItem*>(bars + 41);   // [2], 32 B each
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring + 2);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
@@ -131,22 +140,28 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
     *s_go = (st == 0);
     *s_nitems = *a.n_items;
     ab->flag = 0;
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::QS; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+    }
+    for (int i = 0; i < C::KS; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < C::VS; ++i) {
       mbar_init(v_full + i, 1);
       mbar_init(v_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(s_free + i, C::PW);
       mbar_init(p_full + i, C::PW);
       mbar_init(p_free + i, 1);
       mbar_init(it_full + i, 1);
-      mbar_init(it_empty + i, 3 + C::PW);  // 2 loader lanes + the MMA thread + the P warps
+      mbar_init(it_empty + i, 3 + C::PW + C::EW);  // loader lanes, MMA thread, P and O warps
     }
     mbar_init(o_full, 1);
-    mbar_init(o_free, C::PW);
+    mbar_init(o_free, C::EW);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -183,9 +198,10 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
       uint64_t* empty = kq ? k_empty : v_empty;
       uint8_t* buf = kq ? sK : sV;
       const int col = kq ? a.k_col : a.v_col;
-      uint32_t ncon = 0, st = 0, ph = 0, issued = 0, last_par = 0, q_par = 0;
+      const uint32_t nst = kq ? C::KS : C::VS;
+      uint32_t ncon = 0, st = 0, ph = 0, issued = 0, last_par = 0, q_issued = 0, q_last = 0;
       int litem = 0;
-      bool ok = true, q_issued = false;
+      bool ok = true;
       for (;;) {
         const int slot = ncon & 1;
         if (!mbar_wait(it_full + slot, (ncon >> 1) & 1, ab, a.status)) {
@@ -197,16 +213,18 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
         ++ncon;
         if (w.b < 0) break;
         if (kq) {
-          if (!mbar_wait(q_empty, (litem & 1) ^ 1, ab, a.status)) {
+          const int qs = litem & 1;  // Q stage of this item
+          if (!mbar_wait(q_empty + qs, ((litem >> 1) & 1) ^ 1, ab, a.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(q_full, C::TILE);
+          mbar_arrive_expect_tx(q_full + qs, C::TILE);
 #pragma unroll
           for (int at = 0; at < C::NA; ++at)
-            tma_load_2d(sQ + at * 16384, &tmQ, a.q_col + w.head * D + at * 64, w.q_row0, q_full);
-          q_issued = true;
-          q_par = litem & 1;
+            tma_load_2d(sQ + qs * C::TILE + at * 16384, &tmQ, a.q_col + w.head * D + at * 64,
+                        w.q_row0, q_full + qs);
+          q_issued |= 1u << qs;
+          q_last = (q_last & ~(1u << qs)) | ((uint32_t)((litem >> 1) & 1) << qs);
         }
         for (int j = 0; j < w.nkv; ++j) {
           if (!mbar_wait(empty + st, ph ^ 1, ab, a.status)) {
@@ -220,7 +238,7 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
                         w.kv_row0 + j * 128, full + st);
           issued |= 1u << st;
           last_par = (last_par & ~(1u << st)) | (ph << st);
-          if (++st == 2) {
+          if (++st == nst) {
             st = 0;
             ph ^= 1;
           }
@@ -230,9 +248,10 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
       }
       if (!ok) {  // let every load already in flight land before the CTA exits
         AbortState tmp{0};
-        for (int s2 = 0; s2 < 2; ++s2)
+        for (uint32_t s2 = 0; s2 < nst; ++s2)
           if ((issued >> s2) & 1u) mbar_wait(full + s2, (last_par >> s2) & 1u, &tmp, nullptr);
-        if (q_issued) mbar_wait(q_full, q_par, &tmp, nullptr);
+        for (int s2 = 0; s2 < C::QS; ++s2)
+          if ((q_issued >> s2) & 1u) mbar_wait(q_full + s2, (q_last >> s2) & 1u, &tmp, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -243,12 +262,14 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
       int litem = 0;
       uint32_t kst = 0, kph = 0, vst = 0, vph = 0, scount = 0, pcount = 0, ncon = 0;
       bool ok = true, any = false;
-      const uint32_t q_base = smem_u32(sQ);
-      auto issue_pv = [&](int jj, int nkv) -> bool {
+      const uint32_t q_base0 = smem_u32(sQ);
+      // P.V of tile jj of an item with nkv tiles; `li` is that item's index
+      // on this CTA (the O accumulator's phase).
+      auto issue_pv = [&](int jj, int nkv, int li) -> bool {
         const int pb = (int)(pcount % C::P_BUFS);
         const uint32_t pph = (pcount / C::P_BUFS) & 1;
         if (!mbar_wait(p_full + pb, pph, ab, a.status)) return false;
-        if (jj == 0 && !mbar_wait(o_free, (litem & 1) ^ 1, ab, a.status)) return false;
+        if (jj == 0 && !mbar_wait(o_free, (li & 1) ^ 1, ab, a.status)) return false;
         if (!mbar_wait(v_full + vst, vph, ab, a.status)) return false;
         tc_fence_after();
         const uint32_t p_tmem = tmem + C::P_COL + pb * 64;
@@ -261,7 +282,7 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
         tc_commit(p_free + pb);
         tc_commit(v_empty + vst);
         if (jj == nkv - 1) tc_commit(o_full);
-        if (++vst == 2) {
+        if (++vst == C::VS) {
           vst = 0;
           vph ^= 1;
         }
@@ -269,15 +290,30 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
         any = true;
         return true;
       };
+      // The P.V of each tile is issued after the next S, across item
+      // boundaries too, so the first S of an item overlaps the last P of the
+      // one before it.
+      int pend_j = -1, pend_n = 0, pend_li = 0;
+      auto flush = [&]() -> bool {
+        if (pend_j < 0) return true;
+        const bool r = issue_pv(pend_j, pend_n, pend_li);
+        pend_j = -1;
+        return r;
+      };
       for (;;) {
         const int slot = ncon & 1;
-        if (!mbar_wait(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
+        if (!mbar_wait(it_full + slot, (ncon >> 1) & 1, ab, a.status)) {
+          ok = false;
+          break;
+        }
         const AttnItem w = ring[slot];
         mbar_arrive(it_empty + slot);
         ++ncon;
         if (w.b < 0) break;
         const int nkv = w.nkv;
-        if (!mbar_wait(q_full, litem & 1, ab, a.status)) {
+        const int qs = litem & 1;
+        const uint32_t q_base = q_base0 + qs * C::TILE;
+        if (!mbar_wait(q_full + qs, (litem >> 1) & 1, ab, a.status)) {
           ok = false;
           break;
         }
@@ -302,36 +338,44 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
                           IDESC_S, kk > 0 ? 1u : 0u);
           tc_commit(s_full + sb);
           tc_commit(k_empty + kst);
-          if (j == nkv - 1) tc_commit(q_empty);  // P.V does not read Q: free it early
-          if (++kst == 2) {
+          if (j == nkv - 1) tc_commit(q_empty + qs);  // P.V does not read Q: free it early
+          if (++kst == C::KS) {
             kst = 0;
             kph ^= 1;
           }
           ++scount;
           any = true;
-          if (j > 0 && !issue_pv(j - 1, nkv)) {
+          if (!flush()) {
             ok = false;
             break;
           }
+          pend_j = j;
+          pend_n = nkv;
+          pend_li = litem;
         }
         if (!ok) break;
-        if (nkv > 0) {
-          if (!issue_pv(nkv - 1, nkv)) break;
-        } else {
-          tc_commit(o_full);  // nothing to accumulate: O is taken as zero
-          tc_commit(q_empty);
+        if (nkv == 0) {
+          // nothing to accumulate: O is taken as zero; the previous item's
+          // last P.V goes first so that O's phases stay in item order
+          if (!flush()) {
+            ok = false;
+            break;
+          }
+          tc_commit(o_full);
+          tc_commit(q_empty + qs);
         }
         ++litem;
       }
+      if (ok) flush();
       if (any) {
         tc_commit(drain);
         AbortState tmp{0};
         mbar_wait(drain, 0, &tmp, nullptr);
       }
     }
-  } else if (warp < 2 + C::PW) {
+  } else if (warp >= C::P_WARP0 && warp < C::EPI_WARP0) {
     // ------------------------------------------------ P warps
-    const int pw = warp - 2;         // 0..15
+    const int pw = warp - C::P_WARP0;  // 0..15
     const int q = warp & 3;          // TMEM lane quarter
     const int g = pw >> 2;           // which 32 of the 128 S columns
     const int r = q * 32 + lane;     // row inside the 128-row tile
@@ -339,7 +383,6 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
     const float* rt_ring = reinterpret_cast<const float*>(smem + C::RT_OFF);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t scount = 0, pcount = 0, ncon = 0;
-    int litem = 0;
     for (;;) {
       const int slot = ncon & 1;
       if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
@@ -353,10 +396,6 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
       }
       const int64_t kv0 = w.kv_row0;
       const int n_kv = w.n_kv;                   // history / sequence length
-      const int64_t q0 = w.q_row0;
-      const int rows_valid = min(128, w.n_q - (int)w.qt * 128);
-      const bool row_ok = r < rows_valid;
-      const float inv_n = 1.0f / (float)max(n_kv, 1);
       const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
       const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
       const int t_i = (MODE == MODE_SELF) ? 0 : a.t_req_rel[w.b];
@@ -469,90 +508,8 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(it_empty + slot);
       if (!alive) break;
-      // ---- O epilogue: this warp's 32 rows x OC columns of the head
-      constexpr int OC = D / 4;
-      if (!mbar_wait_warp(o_full, litem & 1, ab, a.status)) break;
-      tc_fence_after();
-      float o[OC];
-      if (w.nkv > 0) {
-#pragma unroll
-        for (int c16 = 0; c16 < OC / 16; ++c16) {
-          uint32_t orr[16];
-          tmem_ld16(tmem + C::O_COL + g * OC + c16 * 16 + lane_base, orr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[c16 * 16 + i] = __uint_as_float(orr[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < OC; ++i) o[i] = 0.f;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
-      if (row_ok) {
-        if (MODE == MODE_CAND) {
-          // self term: the candidate attends to itself at distance 0, gap 0
-          const __half* rowp = a.q_buf + (q0 + r) * a.ld_f1;
-          const uint4* qp = reinterpret_cast<const uint4*>(rowp + a.q_col + w.head * D);
-          const uint4* kp = reinterpret_cast<const uint4*>(rowp + a.k_col + w.head * D);
-          float dot = 0.f;
-#pragma unroll 4
-          for (int i = 0; i < D / 8; ++i) {
-            const uint4 qa = qp[i], ka = kp[i];
-            const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              dot += f16lo(qw[k]) * f16lo(kw[k]) + f16hi(qw[k]) * f16hi(kw[k]);
-          }
-          const float s_self = dot + __ldg(Rp) + __ldg(Rt);
-          const float p_self = __half2float(__float2half_rn(silu_fast(s_self)));
-          const uint4* vp = reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + g * OC);
-#pragma unroll
-          for (int i = 0; i < OC / 8; ++i) {
-            const uint4 va = vp[i];
-            const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              o[i * 8 + 2 * k] += p_self * f16lo(vw[k]);
-              o[i * 8 + 2 * k + 1] += p_self * f16hi(vw[k]);
-            }
-          }
-        }
-      }
-      // ---- store O.  A warp whose 32 rows all belong to the user writes each
-      // 32 x 16 block into its staging buffer (64-byte swizzle) and lets one
-      // TMA bulk store carry it out, so the warp moves on while the data
-      // drains; a warp at the user's ragged end stores its valid rows itself
-      // (the rows after them belong to the next user).
-      if (q * 32 + 32 <= rows_valid) {
-        uint8_t* stg = smem + C::STG_OFF + pw * 2048;
-#pragma unroll
-        for (int c16 = 0; c16 < OC / 16; ++c16) {
-          if (lane == 0) bulk_wait_read<0>();  // the previous store has read the buffer
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<float4*>(stg + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
-                make_float4(o[c16 * 16 + 4 * k] * inv_n, o[c16 * 16 + 4 * k + 1] * inv_n,
-                            o[c16 * 16 + 4 * k + 2] * inv_n, o[c16 * 16 + 4 * k + 3] * inv_n);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmO, w.head * D + g * OC + c16 * 16, (int)(q0 + q * 32), stg);
-            bulk_commit();
-          }
-        }
-      } else if (row_ok) {
-        float4* op = reinterpret_cast<float4*>(a.O + (q0 + r) * a.ldo + w.head * D + g * OC);
-#pragma unroll
-        for (int i = 0; i < OC / 4; ++i)
-          op[i] = make_float4(o[4 * i + 0] * inv_n, o[4 * i + 1] * inv_n, o[4 * i + 2] * inv_n,
-                              o[4 * i + 3] * inv_n);
-      }
-      ++litem;
     }
-  } else if (warp == 2 + C::PW) {
+  } else if (warp == C::FETCH_WARP) {
     // ------------------------------------------------ item fetcher
     // Claims work items (dynamic, one atomic per item), publishes each into
     // the 2-slot ring with its head's halved time-bias table (causal mode),
@@ -601,8 +558,114 @@ __global__ void __launch_bounds__(96 + 32 * AttnCfg<D>::PW, 1)
         }
       }
     }
+  } else if (warp >= C::EPI_WARP0) {
+    // ------------------------------------------------ epilogue warps
+    // One per TMEM lane quarter: 32 rows x D columns of O each, streamed out of
+    // TMEM 16 columns at a time, scaled by 1/n (candidates: plus the self
+    // term) and stored fp32 -- a full 32-row block through swizzled staging and
+    // a TMA bulk store, a block at the user's ragged end row by row (the rows
+    // after it belong to the next user).  The P warps meanwhile go on with the
+    // next item.
+    const int ew = warp - C::EPI_WARP0;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint8_t* stg = smem + C::STG_OFF + ew * 4096;  // two 2 KB buffers
+    uint32_t ncon = 0, nbuf = 0;
+    int litem = 0;
+    for (;;) {
+      const int slot = ncon & 1;
+      if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
+      const AttnItem w = ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(it_empty + slot);
+      ++ncon;
+      if (w.b < 0) break;
+      const int64_t q0 = w.q_row0;
+      const int rows_valid = min(128, w.n_q - (int)w.qt * 128);
+      const bool row_ok = r < rows_valid;
+      const bool full_rows = q * 32 + 32 <= rows_valid;
+      const float inv_n = 1.0f / (float)max(w.n_kv, 1);
+      float p_self = 0.f;
+      const __half* rowp = a.q_buf + (q0 + (row_ok ? r : 0)) * a.ld_f1;
+      if (MODE == MODE_CAND && row_ok) {
+        // self term: the candidate attends to itself at distance 0, gap 0
+        const uint4* qp = reinterpret_cast<const uint4*>(rowp + a.q_col + w.head * D);
+        const uint4* kp = reinterpret_cast<const uint4*>(rowp + a.k_col + w.head * D);
+        float dot = 0.f;
+#pragma unroll 2
+        for (int i = 0; i < D / 8; ++i) {
+          const uint4 qa = qp[i], ka = kp[i];
+          const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dot += f16lo(qw[k]) * f16lo(kw[k]) + f16hi(qw[k]) * f16hi(kw[k]);
+        }
+        const float s_self = dot + __ldg(a.rab_pos + (size_t)w.head * a.Np) +
+                             __ldg(a.rab_time + (size_t)w.head * a.Nt);
+        p_self = __half2float(__float2half_rn(silu_fast(s_self)));
+      }
+      if (!mbar_wait_warp(o_full, litem & 1, ab, a.status)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c16 = 0; c16 < D / 16; ++c16) {
+        float o[16];
+        if (w.nkv > 0) {
+          uint32_t orr[16];
+          tmem_ld16(tmem + C::O_COL + c16 * 16 + lane_base, orr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(orr[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = 0.f;
+        }
+        if (c16 == D / 16 - 1) {  // O is fully read: the next item may accumulate
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
+        if (MODE == MODE_CAND && row_ok) {
+          const uint4* vp = reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + c16 * 16);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint4 va = vp[i];
+            const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              o[i * 8 + 2 * k] += p_self * f16lo(vw[k]);
+              o[i * 8 + 2 * k + 1] += p_self * f16hi(vw[k]);
+            }
+          }
+        }
+        if (full_rows) {
+          uint8_t* buf = stg + (nbuf & 1) * 2048;
+          if (lane == 0) bulk_wait_read<1>();  // the store two blocks back has read `buf`
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<float4*>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_float4(o[4 * k] * inv_n, o[4 * k + 1] * inv_n, o[4 * k + 2] * inv_n,
+                            o[4 * k + 3] * inv_n);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmO, w.head * D + c16 * 16, (int)(q0 + q * 32), buf);
+            bulk_commit();
+          }
+          ++nbuf;
+        } else if (row_ok) {
+          float4* op = reinterpret_cast<float4*>(a.O + (q0 + r) * a.ldo + w.head * D + c16 * 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            op[i] = make_float4(o[4 * i] * inv_n, o[4 * i + 1] * inv_n, o[4 * i + 2] * inv_n,
+                                o[4 * i + 3] * inv_n);
+        }
+      }
+      ++litem;
+    }
+    if (lane == 0) bulk_wait_all();  // O stores complete before the CTA exits
   }
-  if (warp >= 2 && warp < 2 + C::PW && lane == 0) bulk_wait_all();  // O stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -634,7 +697,7 @@ static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tk
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kfn<<<grid, 96 + 32 * C::PW, C::SMEM, s>>>(tq, tkv, to, ad);
+  kfn<<<grid, C::THREADS, C::SMEM, s>>>(tq, tkv, to, ad);
   return cudaGetLastError();
 }
 
