@@ -73,7 +73,6 @@ template <int D>
 struct AttnCfg {
   static constexpr int NA = D / 64;                       // 64-column swizzle atoms
   static constexpr uint32_t TILE = 128u * D * 2;          // Q, K or V tile bytes
-  static constexpr int P_BUFS = 2;                        // P lives in TMEM
   static constexpr uint32_t Q_OFF = 0;
   static constexpr int QS = 2, KS = 2, VS = 2;            // Q, K and V ring stages
   static constexpr uint32_t K_OFF = Q_OFF + QS * TILE;
@@ -91,9 +90,9 @@ struct AttnCfg {
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static_assert(QS == 2 && KS <= 4 && VS <= 4, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory per CTA");
-  static constexpr uint32_t O_COL = 256;                  // TMEM columns: S0, S1, O,
-  static constexpr uint32_t P_COL = O_COL + D;            // then P0, P1 (64 columns each:
-                                                          // 128 fp16 per row, packed in pairs)
+  // TMEM columns: S0 | S1 (128 each; P_j, 128 fp16 per row packed in pairs,
+  // overwrites the first 64 columns of S_j once S_j is read), then O0 | O1.
+  static constexpr uint32_t O_COL = 256;
 };
 
 enum { MODE_SELF = 0, MODE_CAND = 1 };
@@ -118,11 +117,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint64_t* k_full = bars + 25;     // [KS]
   uint64_t* k_empty = bars + 29;    // [KS]
   uint64_t* s_full = bars + 6;      // [2]
-  uint64_t* s_free = bars + 8;      // [2]
   uint64_t* p_full = bars + 10;     // [2]
-  uint64_t* p_free = bars + 12;     // [2]
-  uint64_t* o_full = bars + 14;
-  uint64_t* o_free = bars + 15;
+  uint64_t* o_full = bars + 12;     // [2]
+  uint64_t* o_free = bars + 14;     // [2]
+  uint64_t* rd = bars + 21;         // [4] per lane quarter: its P warps have read S
   uint64_t* drain = bars + 16;
   uint64_t* it_full = bars + 17;    // [2] item ring
   uint64_t* it_empty = bars + 19;   // [2]
@@ -154,14 +152,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(s_free + i, C::PW);
       mbar_init(p_full + i, C::PW);
-      mbar_init(p_free + i, 1);
+      mbar_init(o_full + i, 1);
+      mbar_init(o_free + i, C::EW);
       mbar_init(it_full + i, 1);
       mbar_init(it_empty + i, 3 + C::PW + C::EW);  // loader lanes, MMA thread, P and O warps
     }
-    mbar_init(o_full, 1);
-    mbar_init(o_free, C::EW);
+    for (int i = 0; i < 4; ++i) mbar_init(rd + i, C::PW / 4);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -266,22 +263,22 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       // P.V of tile jj of an item with nkv tiles; `li` is that item's index
       // on this CTA (the O accumulator's phase).
       auto issue_pv = [&](int jj, int nkv, int li) -> bool {
-        const int pb = (int)(pcount % C::P_BUFS);
-        const uint32_t pph = (pcount / C::P_BUFS) & 1;
+        const int pb = (int)(pcount & 1);  // P_j sits in S_j's buffer
+        const uint32_t pph = (pcount >> 1) & 1;
+        const int ob = li & 1;             // O buffer of this item
         if (!mbar_wait(p_full + pb, pph, ab, a.status)) return false;
-        if (jj == 0 && !mbar_wait(o_free, (li & 1) ^ 1, ab, a.status)) return false;
+        if (jj == 0 && !mbar_wait(o_free + ob, ((li >> 1) & 1) ^ 1, ab, a.status)) return false;
         if (!mbar_wait(v_full + vst, vph, ab, a.status)) return false;
         tc_fence_after();
-        const uint32_t p_tmem = tmem + C::P_COL + pb * 64;
+        const uint32_t p_tmem = tmem + pb * 128;
         const uint32_t v_base = smem_u32(sV + vst * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // 16 KV rows per MMA = 8 packed P columns
-          tc_mma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8,
+          tc_mma_f16_ts(tmem + C::O_COL + ob * D, p_tmem + kk * 8,
                         sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
                         (jj > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(p_free + pb);
         tc_commit(v_empty + vst);
-        if (jj == nkv - 1) tc_commit(o_full);
+        if (jj == nkv - 1) tc_commit(o_full + ob);
         if (++vst == C::VS) {
           vst = 0;
           vph ^= 1;
@@ -323,11 +320,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             ok = false;
             break;
           }
+          // S_j reuses the buffer of S_{j-2}; P_{j-2}, written there, was read
+          // by a P.V issued before this MMA, and MMAs run in issue order.
           const int sb = scount & 1;
-          if (!mbar_wait(s_free + sb, ((scount >> 1) & 1) ^ 1, ab, a.status)) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
           const uint32_t k_base = smem_u32(sK + kst * C::TILE);
 #pragma unroll
@@ -361,7 +356,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             ok = false;
             break;
           }
-          tc_commit(o_full);
+          const int ob = litem & 1;  // O's phases stay in item order per buffer
+          if (!mbar_wait(o_free + ob, ((litem >> 1) & 1) ^ 1, ab, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_commit(o_full + ob);
           tc_commit(q_empty + qs);
         }
         ++litem;
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     float* win2 = reinterpret_cast<float*>(smem + C::WIN_OFF) + pw * 2 * 64;  // 2 buffers
     const float* rt_ring = reinterpret_cast<const float*>(smem + C::RT_OFF);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    uint32_t scount = 0, pcount = 0, ncon = 0;
+    uint32_t scount = 0, ncon = 0;
     for (;;) {
       const int slot = ncon & 1;
       if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
@@ -449,8 +449,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + sb);
-        ++scount;
+        if (lane == 0) mbar_arrive(rd + q);  // this warp's part of S_j is in registers
+        const uint32_t tile = scount++;
         // ---- P = SiLU(S + bias), masked, fp16
         uint32_t pk[16];
         if (MODE == MODE_SELF) {
@@ -490,19 +490,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
 #pragma unroll
         for (int m = 0; m < 8; ++m) bw[m] = bwn[m];
-        // ---- write P into TMEM: this warp's 32 rows, 32 fp16 (16 packed columns)
-        const int pb = (int)(pcount % C::P_BUFS);
-        if (!mbar_wait_warp(p_free + pb, ((pcount / C::P_BUFS) & 1) ^ 1, ab, a.status)) {
+        // ---- write P over S_j: this warp's 32 rows, 32 fp16 (16 packed columns),
+        // once all four P warps of the lane quarter have read their part of S_j
+        if (!mbar_wait_warp(rd + q, tile & 1, ab, a.status)) {
           alive = false;
           break;
         }
         tc_fence_after();
-        tmem_st16(tmem + C::P_COL + pb * 64 + g * 16 + lane_base, pk);
+        tmem_st16(tmem + sb * 128 + g * 16 + lane_base, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + pb);
-        ++pcount;
+        if (lane == 0) mbar_arrive(p_full + sb);
       }
       // the ring slot (and its time table) may be refilled from here on
       __syncwarp();
@@ -605,14 +604,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                              __ldg(a.rab_time + (size_t)w.head * a.Nt);
         p_self = __half2float(__float2half_rn(silu_fast(s_self)));
       }
-      if (!mbar_wait_warp(o_full, litem & 1, ab, a.status)) break;
+      const int ob = litem & 1;
+      if (!mbar_wait_warp(o_full + ob, (litem >> 1) & 1, ab, a.status)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int c16 = 0; c16 < D / 16; ++c16) {
         float o[16];
         if (w.nkv > 0) {
           uint32_t orr[16];
-          tmem_ld16(tmem + C::O_COL + c16 * 16 + lane_base, orr);
+          tmem_ld16(tmem + C::O_COL + ob * D + c16 * 16 + lane_base, orr);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(orr[i]);
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         if (c16 == D / 16 - 1) {  // O is fully read: the next item may accumulate
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);
+          if (lane == 0) mbar_arrive(o_free + ob);
         }
         if (MODE == MODE_CAND && row_ok) {
           const uint4* vp = reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + c16 * 16);
