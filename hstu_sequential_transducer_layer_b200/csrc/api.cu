@@ -164,13 +164,13 @@ cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const LayerOps& op
   return gemm(c, g, K_GEMM_F1, K_SIMT_GEMM_F1);
 }
 
-// f2 + bias + residual.  resid_f32: the residual is the fp32 stream (else the
-// caller's bf16 rows); out16 (fp16 copy, or the caller's bf16 output when
-// out16_bf16) and out32 (fp32 stream) may each be null.  Each output element
-// is read (residual) and written by the same thread, so the fp32 stream is
-// updated in place.
+// f2 + bias + residual.  resid_kind (tensor-core path): the residual is the
+// caller's bf16 rows, an fp32 stream or an fp16 stream; out16 (fp16 stream, or
+// the caller's bf16 output when out16_bf16) and out32 (fp32 stream) may each
+// be null.  Each output element is read (residual) before it is written, by
+// the same warp, so a stream may be updated in place.
 cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, const void* Z,
-                   const void* resid, bool resid_f32, int64_t rows_cap, const int64_t* rows_dev,
+                   const void* resid, int resid_kind, int64_t rows_cap, const int64_t* rows_dev,
                    void* out16, bool out16_bf16, float* out32) {
   GemmCall g{};
   g.A = Z;
@@ -193,7 +193,7 @@ cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& op
     g.out = out16;
     g.out_f16 = out16_bf16 ? 0 : 1;
     g.out32 = out32;
-    g.resid_f32 = resid_f32 ? 1 : 0;
+    g.resid_kind = resid_kind;
   } else {  // fp32 layers: everything is already fp32; `out` is the fp32 destination
     g.out = out16 ? out16 : out32;
   }
@@ -231,7 +231,7 @@ cudaError_t attn(const Ctx& c, const AttnCall& a) {
 // f2 adds `resid` and writes out16 / out32 (see run_f2).
 cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, int64_t B,
                       int64_t T, const int64_t* off, const void* A, int a_f16, const void* resid,
-                      bool resid_f32, void* out16, bool out16_bf16, float* out32, void* f1,
+                      int resid_kind, void* out16, bool out16_bf16, float* out32, void* f1,
                       const Layout& L, void* ws) {
   cudaError_t e = run_f1(c, w, ops, A, a_f16, T, nullptr, f1, false);
   if (e != cudaSuccess) return e;
@@ -254,7 +254,7 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
   e = launch_ln_gate(c.d.dtype, at<void>(ws, L.o), f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps,
                      at<void>(ws, L.z), c.hdv, T, nullptr, c.status, c.s);
   if (e != cudaSuccess) return e;
-  return run_f2(c, w, ops, at<void>(ws, L.z), resid, resid_f32, T, nullptr, out16, out16_bf16,
+  return run_f2(c, w, ops, at<void>(ws, L.z), resid, resid_kind, T, nullptr, out16, out16_bf16,
                 out32);
 }
 
@@ -289,8 +289,8 @@ hstu_status stack_impl(const hstu_layer_desc* desc, int32_t n_layers,
     launch_time_buckets(offsets, B, at<int32_t>(ws, L.t_rel), at<int64_t>(ws, L.ubase),
                         L.tile_cap, desc->time_sub_bits, desc->n_time_buckets,
                         at<uint32_t>(ws, L.tbuckets), c.hdr, c.s);
-  // Between layers the residual stream stays fp32 (xres, updated in place);
-  // the tensor-core path also keeps an fp16 copy (xh) as the next f1's operand.
+  // Between layers the residual stream is fp16 on the tensor-core path (xh: the
+  // next f1's operand, updated in place by f2) and fp32 on the fp32 path.
   float* xres = at<float>(ws, L.xres);
   void* xh = at<void>(ws, L.xh);
   cudaError_t e = convert_weights(c, weights, n_layers, L, ws);
@@ -298,11 +298,11 @@ hstu_status stack_impl(const hstu_layer_desc* desc, int32_t n_layers,
     const bool first = l == 0, last = l == n_layers - 1;
     const LayerOps ops = layer_ops(c, weights[l], L, ws, l, n_layers);
     const void* A = first ? X : (c.bf16 ? xh : (const void*)xres);
-    const void* resid = first ? X : (const void*)xres;
+    const void* resid = first ? X : (c.bf16 ? xh : (const void*)xres);
     void* o16 = last ? out : (c.bf16 ? xh : nullptr);
-    float* o32 = last ? nullptr : xres;
-    e = run_layer(c, weights[l], ops, B, T, offsets, A, first ? 0 : 1, resid, !first, o16, last,
-                  o32, at<void>(ws, L.f1), L, ws);
+    float* o32 = (last || c.bf16) ? nullptr : xres;
+    e = run_layer(c, weights[l], ops, B, T, offsets, A, first ? 0 : 1, resid,
+                  first ? RESID_BF16 : RESID_F16, o16, last, o32, at<void>(ws, L.f1), L, ws);
   }
   return finish(e);
 }
@@ -398,8 +398,9 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
         break;
       }
       e = run_layer(c, weights[l], ops, B, T, hist_offsets, A, first ? 0 : 1,
-                    first ? history : (const void*)xres, !first, c.bf16 ? xh : nullptr, false,
-                    xres, f1_of(l), L, ws);
+                    first ? history : (c.bf16 ? xh : (const void*)xres),
+                    first ? RESID_BF16 : RESID_F16, c.bf16 ? xh : nullptr, false,
+                    c.bf16 ? nullptr : xres, f1_of(l), L, ws);
     }
   }
   if (e != cudaSuccess || total_cands == 0) return finish(e);
@@ -451,7 +452,8 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
       if (e != cudaSuccess) break;
       const void* resid = first ? xb_c : (const void*)xres_c;
       void* o16 = (c.bf16 && !last) ? xh_c : nullptr;
-      e = run_f2(c, weights[l], ops, zc, resid, !first, R, rows_dev, o16, false, xres_c);
+      e = run_f2(c, weights[l], ops, zc, resid, first ? RESID_BF16 : RESID_F32, R, rows_dev, o16,
+                 false, xres_c);
     }
     if (e == cudaSuccess)
       e = launch_score(desc->dtype, xres_c, desc->d_model, head_vec, cand_offsets, mb_off, B, k,

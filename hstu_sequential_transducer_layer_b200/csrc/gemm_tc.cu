@@ -30,9 +30,9 @@ struct GemmDev {
   int has_out16;               // 16-bit output (fp16 if out_f16, else bf16)
   int out_f16;
   int has_out32;               // EPI_RESID: fp32 copy of the output
-  const void* resid;           // EPI_RESID: residual, bf16 or fp32 (resid_f32)
+  const void* resid;           // EPI_RESID: residual (resid_kind: bf16, fp32 or fp16)
   int64_t ldr;
-  int resid_f32;
+  int resid_kind;
   int* status;
 };
 
@@ -78,7 +78,7 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   if (EPI == EPI_SILU) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
-  } else if (rsm != nullptr) {  // fp32 residual chunk staged by TMA (128-byte swizzle)
+  } else if (g.resid_kind == RESID_F32) {  // residual chunk staged by TMA, 128-byte swizzle
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float4 rr = *reinterpret_cast<const float4*>(rsm + lane * 128 + ((k ^ (lane & 7)) << 4));
@@ -87,30 +87,17 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
       v[4 * k + 2] += rr.z;
       v[4 * k + 3] += rr.w;
     }
-  } else if (valid) {
-    if (g.resid_f32) {
-      const float4* rp = reinterpret_cast<const float4*>(
-          static_cast<const float*>(g.resid) + row * g.ldr + col);
+  } else {  // 16-bit residual chunk staged by TMA, 64-byte swizzle
+    const int f16 = g.resid_kind == RESID_F16;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 rr = rp[i];
-        v[4 * i + 0] += rr.x;
-        v[4 * i + 1] += rr.y;
-        v[4 * i + 2] += rr.z;
-        v[4 * i + 3] += rr.w;
-      }
-    } else {
-      const uint4* rp = reinterpret_cast<const uint4*>(
-          static_cast<const __nv_bfloat16*>(g.resid) + row * g.ldr + col);
+    for (int k = 0; k < 4; ++k) {
+      const uint4 rr =
+          *reinterpret_cast<const uint4*>(rsm + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4));
+      const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 rr = rp[i];
-        const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          v[i * 8 + 2 * k] += bf16lo(rw[k]);
-          v[i * 8 + 2 * k + 1] += bf16hi(rw[k]);
-        }
+      for (int m = 0; m < 4; ++m) {
+        v[k * 8 + 2 * m] += lo16(f16, rw[m]);
+        v[k * 8 + 2 * m + 1] += hi16(f16, rw[m]);
       }
     }
   }
@@ -302,16 +289,17 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     constexpr int CH = BN / 64;          // 32-column chunks per warp
     uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * kStageBuf;
     int local = 0, nchunk = 0;
-    // fp32 residual: lane 0 has TMA bring the next 32 x 32 chunk into the
-    // warp's buffer while the current one is computed and stored
-    const bool rtma = (EPI == EPI_RESID) && g.resid_f32;
+    // residual: lane 0 has TMA bring the next 32 x 32 chunk into the warp's
+    // buffer while the current one is computed and stored
+    const bool rtma = (EPI == EPI_RESID);
+    const uint32_t rbytes = g.resid_kind == RESID_F32 ? 4096u : 2048u;
     uint8_t* rbuf = smem + C::RES_OFF + (warp - 2) * kStageBuf;
     uint64_t* rb = rbar + (warp - 2);
     uint32_t rpar = 0;
     bool r_pending = false, alive = true;
     auto r_issue = [&](int t_, int c_) {
       const int mt_ = t_ / n_tiles, nt_ = t_ - (t_ / n_tiles) * n_tiles;
-      mbar_arrive_expect_tx(rb, kStageBuf);
+      mbar_arrive_expect_tx(rb, rbytes);
       tma_load_2d(rbuf, &tmR, g.n_off + nt_ * BN + part * (BN / 2) + c_ * 32, mt_ * 128 + q * 32,
                   rb);
     };
@@ -450,13 +438,20 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
                                     (uint64_t)c.ldo * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                                     CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  // fp32 residual: [M_cap, n_off + N] with row stride ldr, 32 x 32 boxes
+  // residual: [M_cap, n_off + N] with row stride ldr, 32 x 32 boxes (fp32 with
+  // 128-byte swizzle, 16-bit with 64-byte swizzle)
   tr = ta;
-  if (c.epi == EPI_RESID && c.resid_f32 &&
-      !encode_tmap_2d_ex(&tr, c.resid, (uint64_t)c.M_cap, (uint64_t)(c.n_off + c.N),
-                         (uint64_t)c.ldr * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+  if (c.epi == EPI_RESID) {
+    const bool r32 = c.resid_kind == RESID_F32;
+    const CUtensorMapDataType rt = r32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : (c.resid_kind == RESID_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    if (!c.resid ||
+        !encode_tmap_2d_ex(&tr, c.resid, (uint64_t)c.M_cap, (uint64_t)(c.n_off + c.N),
+                           (uint64_t)c.ldr * (r32 ? 4 : 2), 32, 32, rt,
+                           r32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
   GemmDev gd;
   gd.M_cap = c.M_cap;
   gd.M_dev = c.M_dev;
@@ -470,7 +465,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   gd.has_out32 = (c.epi == EPI_RESID && c.out32 != nullptr);
   gd.resid = c.resid;
   gd.ldr = c.ldr;
-  gd.resid_f32 = c.resid_f32;
+  gd.resid_kind = c.resid_kind;
   gd.status = c.status;
   const int64_t tiles = mt * (c.N / BN);
   const int grid = (int)std::min<int64_t>(tiles, sms);

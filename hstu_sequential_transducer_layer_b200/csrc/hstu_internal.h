@@ -71,7 +71,7 @@ struct Header {           // first 256 bytes of every workspace
 
 struct Layout {
   size_t header, items, t_rel, ubase, tbuckets, f1, o, z;
-  size_t xres, xh;          // fp32 residual stream; fp16 copy feeding the next f1 (tensor-core path)
+  size_t xres, xh;          // residual stream: fp32 (fp32 path) / fp16, also the next f1's operand
   size_t w16;               // tensor-core path: fp16 copies of W1 (layers >= 1) and W2, per layer
   size_t f1_cache;          // M-FALCON: every layer's f1 output (its K/V) for the history
   size_t mb_off, c_items, t_req_rel, xres_c, xb_c, xh_c, f1c, oc, zc;  // candidate microbatch
@@ -118,6 +118,7 @@ void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64
 
 // C[M, N] = A[M, K] * W[n_off + N, K]^T with fused epilogue, bf16 tcgen05.
 enum Epilogue { EPI_SILU = 0, EPI_RESID = 1 };
+enum ResidKind { RESID_BF16 = 0, RESID_F32 = 1, RESID_F16 = 2 };
 struct GemmCall {
   const void* A;  int64_t lda;   // [M_cap, K] row stride in elements
   const void* W;  int64_t ldw;   // [N_total, K]
@@ -130,7 +131,7 @@ struct GemmCall {
   int out_f16;                   // tensor-core path: `out` is fp16 (else bf16)
   void* out32;                   // tensor-core EPI_RESID: optional fp32 copy of the output
   const void* resid; int64_t ldr;
-  int resid_f32;                 // tensor-core EPI_RESID: residual stored as fp32 (else bf16)
+  int resid_kind;                // tensor-core EPI_RESID residual: RESID_BF16, RESID_F32, RESID_F16
   int epi;
   int* status;
 };

@@ -138,7 +138,8 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
   }
   L->o = take((size_t)T * hdv * 4);
   L->z = take((size_t)T * hdv * es);
-  L->xres = take((size_t)T * dm * 4);
+  // residual stream between layers: fp16 on the tensor-core path, fp32 otherwise
+  L->xres = bf16 ? 0 : take((size_t)T * dm * 4);
   L->xh = bf16 ? take((size_t)T * dm * 2) : L->xres;
   L->w16 = bf16 ? take((size_t)n_layers * (F * dm + dm * hdv) * 2) : 0;
   if (mf) {
