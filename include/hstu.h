@@ -55,12 +55,13 @@
  *   Precision   dtype HSTU_BF16 (inputs, weights, outputs bf16): the tensor
  *               cores take fp16 operands with fp32 accumulation.  bf16 values
  *               within [2^-14, 65504] in magnitude convert to fp16 exactly;
- *               the f1 output, P and Z are stored in fp16 (saturating at
- *               +-65504), the attention output O, LayerNorm statistics and the
- *               residual stream between layers stay fp32, and only the final
+ *               the f1 output, P, Z and the residual stream between layers
+ *               are stored in fp16 (saturating at +-65504), the attention
+ *               output O and the LayerNorm statistics stay fp32 (M-FALCON's
+ *               candidate rows also keep an fp32 residual), and only the final
  *               output is rounded to bf16.  fp16 keeps 3 more mantissa bits than
- *               bf16 at the same tensor-core rate; inputs and weights must lie
- *               within fp16 range.  dtype HSTU_FP32: fp32 throughout (CUDA-core
+ *               bf16 at the same tensor-core rate; inputs, weights and layer
+ *               outputs must lie within fp16 range.  dtype HSTU_FP32: fp32 throughout (CUDA-core
  *               FMA).
  *   Supported   bf16: d_qk = d_v in {64, 128}; d_model and h*d_v multiples
  *               of 64; bucket counts in [1, 4096].  fp32: d_qk, d_v <= 128
