@@ -39,17 +39,19 @@ struct GemmDev {
 constexpr int kEpiThreads = 256;      // 8 epilogue warps
 constexpr uint32_t kStageBuf = 4096;  // per-warp output staging bytes (32 x 32 fp32)
 
-template <int BN, int STAGES, int EPI>
+// COMPACT (EPI_RESID with 16-bit residual and output only): 2 KB output and
+// 2 KB residual buffers per epilogue warp, leaving room for one more A/B stage.
+template <int BN, int STAGES, int EPI, int COMPACT>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t OUT_OFF = STAGES * STAGE_BYTES;             // 8 x 4 KB staging
-  // EPI_RESID: 8 x 4 KB buffers that TMA fills with the next fp32 residual chunk
-  static constexpr uint32_t RES_OFF = OUT_OFF + (kEpiThreads / 32) * kStageBuf;
-  static constexpr uint32_t BAR_OFF =
-      RES_OFF + (EPI == EPI_RESID ? (kEpiThreads / 32) * kStageBuf : 0);
+  static constexpr uint32_t BUF = COMPACT ? 2048 : kStageBuf;         // per-warp buffers
+  static constexpr uint32_t OUT_OFF = STAGES * STAGE_BYTES;             // 8 output staging buffers
+  // EPI_RESID: 8 buffers that TMA fills with the next residual chunk
+  static constexpr uint32_t RES_OFF = OUT_OFF + (kEpiThreads / 32) * BUF;
+  static constexpr uint32_t BAR_OFF = RES_OFF + (EPI == EPI_RESID ? (kEpiThreads / 32) * BUF : 0);
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
 };
@@ -119,9 +121,10 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
     }
   }
   if (g.has_out16) {
-    uint8_t* buf = stage + (both ? 0 : parity * 2048);
+    // parity < 0: one 2 KB buffer (wait for the previous store to read it)
+    uint8_t* buf = stage + ((both || parity < 0) ? 0 : parity * 2048);
     if (lane == 0) {
-      if (both) bulk_wait_read<0>();
+      if (both || parity < 0) bulk_wait_read<0>();
       else bulk_wait_read<1>();
     }
     __syncwarp();
@@ -146,13 +149,13 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   return true;
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int COMPACT>
 __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmO16,
               const __grid_constant__ CUtensorMap tmO32, const __grid_constant__ CUtensorMap tmR,
               const GemmDev g) {
-  using C = GemmCfg<BN, STAGES, EPI>;
+  using C = GemmCfg<BN, STAGES, EPI, COMPACT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -287,13 +290,13 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     const int q = warp & 3;              // TMEM lane quarter this warp may read
     const int part = (warp - 2) >> 2;    // which half of the BN columns
     constexpr int CH = BN / 64;          // 32-column chunks per warp
-    uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * kStageBuf;
+    uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * C::BUF;
     int local = 0, nchunk = 0;
     // residual: lane 0 has TMA bring the next 32 x 32 chunk into the warp's
     // buffer while the current one is computed and stored
     const bool rtma = (EPI == EPI_RESID);
     const uint32_t rbytes = g.resid_kind == RESID_F32 ? 4096u : 2048u;
-    uint8_t* rbuf = smem + C::RES_OFF + (warp - 2) * kStageBuf;
+    uint8_t* rbuf = smem + C::RES_OFF + (warp - 2) * C::BUF;
     uint64_t* rb = rbar + (warp - 2);
     uint32_t rpar = 0;
     bool r_pending = false, alive = true;
@@ -349,10 +352,10 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
         bool stored;
         if (c & 1)
           stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb_acc, bb,
-                                   stage, nchunk & 1, rsm);
+                                   stage, COMPACT ? -1 : (nchunk & 1), rsm);
         else
           stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba,
-                                   stage, nchunk & 1, rsm);
+                                   stage, COMPACT ? -1 : (nchunk & 1), rsm);
         nchunk += stored ? 1 : 0;
         if (rtma) {
           __syncwarp();  // every lane has read the residual chunk
@@ -393,12 +396,13 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
   }
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int COMPACT = 0>
 static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
                               const CUtensorMap& to16, const CUtensorMap& to32,
                               const CUtensorMap& tr, const GemmDev& gd, int grid, cudaStream_t s) {
-  using C = GemmCfg<BN, STAGES, EPI>;
-  auto kfn = k_gemm_tc<BN, STAGES, EPI>;
+  using C = GemmCfg<BN, STAGES, EPI, COMPACT>;
+  static_assert(C::SMEM <= 232448, "shared memory per CTA");
+  auto kfn = k_gemm_tc<BN, STAGES, EPI, COMPACT>;
   static bool attr_set = false;  // per instantiation; the attribute is per device function
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -476,7 +480,11 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
     return launch_one<64, 8, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
   }
   // the residual buffers take one A/B stage's worth of shared memory
-  if (BN == 256) return launch_one<256, 3, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
+  if (BN == 256) {
+    if (c.resid_kind != RESID_F32 && c.out32 == nullptr)
+      return launch_one<256, 4, EPI_RESID, 1>(ta, tb, to16, to32, tr, gd, grid, s);
+    return launch_one<256, 3, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
+  }
   if (BN == 128) return launch_one<128, 4, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
   return launch_one<64, 6, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
 }
