@@ -284,9 +284,10 @@ def run_ours(args):
     if r.status() != 0:
         raise RuntimeError(f"device status {r.status()} after warm-up")
 
-    # ---------------- timed region (step events only: events between the
-    # library's launches would keep consecutive kernels from overlapping)
+    # ---------------- timed region (an event pair around every launch of the
+    # library gives the per-kernel device times for the roofline)
     n_launch0 = H.hstu_launch_count()
+    H.hstu_trace_enable(args.steps * 8 * 6 + 64)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     if world > 1:
@@ -302,24 +303,12 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     n_launch = H.hstu_launch_count() - n_launch0
+    trace = H.hstu_trace_read()
+    H.hstu_trace_enable(0)
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = sum(step_ms) / len(step_ms)
     if r.status() != 0:
         raise RuntimeError(f"device status {r.status()} after timing")
-
-    # ---------------- up to 5 of the same steps again with an event pair
-    # around every launch: per-kernel device times for the roofline and the
-    # breakdown (clocks sampled here too)
-    k_steps = min(args.steps, 5)
-    H.hstu_trace_enable(k_steps * 8 * 6 + 64)
-    torch.cuda.synchronize()
-    with ClockSampler(local, "_kernels") as clk_k:
-        for i in range(k_steps):
-            flush.zero_()
-            step()
-        torch.cuda.synchronize()
-    trace = H.hstu_trace_read()
-    H.hstu_trace_enable(0)
 
     # per-kernel device time inside the timed region
     per_kernel = {}
@@ -340,7 +329,6 @@ def run_ours(args):
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "peak_source": f"bf16_tflops_sustained ({peak_src})",
                     "traffic": ncu_traffic(dominant, w.name),
-                    "timed_steps": k_steps, "clocks": clk_k.summary(),
                     "avg_launch_ms": round(tot / n, 4)}
     step_flops = args_layers = w.n_layers * sum(flops.values())
     del args_layers
