@@ -328,6 +328,15 @@ DEVI int log_bucket(int x, int S, int N) {
   }
   return min(b, N - 1);
 }
+// log_bucket without branches (the same values; x >= 0): lanes of a warp
+// whose distances fall on both sides of 2^S do not diverge.
+DEVI uint32_t log_bucket_nb(int x, int S, int N) {
+  const int e = 31 - __clz(x | 1);
+  const int sh = max(e - S, 0);
+  const int big = ((e - S + 1) << S) + ((x >> sh) - (1 << S));
+  const int b = x < (1 << S) ? x : big;
+  return (uint32_t)min(b, N - 1);
+}
 // Smallest distance that falls in bucket b (b < N), saturated to int32.
 DEVI int bucket_lo(int b, int S) {
   if (b < (1 << S)) return b;

@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(256)
     k_time_buckets(const int64_t* __restrict__ off, int64_t B, const int32_t* __restrict__ t_rel,
                    const int64_t* __restrict__ ubase, int St, int Nt,
                    uint32_t* __restrict__ tb, const Header* hdr) {
+  __shared__ __align__(16) int s_tj[kTile];
   if (hdr->status != HSTU_OK) return;
   const int n_tiles = hdr->n_tiles;
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
@@ -212,17 +213,25 @@ __global__ void __launch_bounds__(256)
     const int i = qt * kTile + r;
     const bool row_ok = i < n;
     const int ti = row_ok ? t_rel[kv0 + i] : 0;
+    // the tile's 128 column timestamps, read once into shared memory
+    __syncthreads();  // the previous tile's columns are no longer read
+    if (threadIdx.x < kTile) {
+      const int jj = j * kTile + threadIdx.x;
+      s_tj[threadIdx.x] = jj < n ? t_rel[kv0 + jj] : 0;
+    }
+    __syncthreads();
     uint32_t* dst = tb + (size_t)t * kBucketTileWords;
 #pragma unroll 4
     for (int u = 0; u < 16; ++u) {
       const int c4 = (threadIdx.x >> 7) + 2 * u;
+      const int4 tj = *reinterpret_cast<const int4*>(s_tj + 4 * c4);
+      const int tjk[4] = {tj.x, tj.y, tj.z, tj.w};
       uint32_t word = 0;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int jj = j * kTile + 4 * c4 + k;
-        uint32_t bk = 0;
-        if (row_ok && jj <= i) bk = (uint32_t)log_bucket(max(ti - t_rel[kv0 + jj], 0), St, Nt);
-        word |= bk << (8 * k);
+        const uint32_t bk = log_bucket_nb(max(ti - tjk[k], 0), St, Nt);
+        word |= (row_ok && jj <= i ? bk : 0u) << (8 * k);
       }
       dst[c4 * 128 + r] = word;
     }
@@ -499,59 +508,63 @@ __global__ void __launch_bounds__(kSchedThreads)
     }
   }
   __syncthreads();
-  // items, longest history first: level c = number of KV tiles (0..levels)
+  // items, longest history first: level c = number of KV tiles (0..levels);
+  // the items of one (user, head) are adjacent (they read the same history
+  // K/V); users of one level are placed in any order (each item writes only
+  // its own rows)
+  __shared__ int s_hist[kMaxLevels + 1];    // candidate q-tiles per level
+  __shared__ int s_cursor[kMaxLevels + 1];  // next q-tile position per level
   __shared__ long long s_base;
-  __shared__ int s_cnt[kSchedThreads];
-  __shared__ long long s_start[kSchedThreads];
   const int levels = (int)((max_len + kTile - 1) / kTile);
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
-  for (int c_hi = levels; c_hi >= 0; c_hi -= blockDim.x) {
-    const int c = c_hi - (int)threadIdx.x;
-    int cnt = 0;
-    if (c >= 0)
-      for (int64_t b = 0; b < B; ++b) {
-        const int64_t n = hoff[b + 1] - hoff[b];
-        const int nkv = (int)((n + kTile - 1) / kTile);
-        if (nkv == c) {
-          const int64_t rows = mb_off[b + 1] - mb_off[b];
-          cnt += (int)((rows + kTile - 1) / kTile);
-        }
+  auto emit = [&](int64_t b, long long pos, int nkv) {
+    const int64_t n = hoff[b + 1] - hoff[b];
+    const int64_t rows = mb_off[b + 1] - mb_off[b];
+    const int nq = (int)((rows + kTile - 1) / kTile);
+    for (int hh = 0; hh < h; ++hh)
+      for (int qt = 0; qt < nq; ++qt) {
+        const long long idx = pos * h + (long long)hh * nq + qt;
+        if (idx < item_cap)
+          items[idx] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, nkv, 0,
+                                (int32_t)(mb_off[b] + (int64_t)qt * kTile), (int32_t)hoff[b],
+                                (int32_t)rows, (int32_t)n};
       }
-    s_cnt[threadIdx.x] = cnt;
+  };
+  auto nkv_of = [&](int64_t b) { return (int)((hoff[b + 1] - hoff[b] + kTile - 1) / kTile); };
+  auto nq_of = [&](int64_t b) { return (int)((mb_off[b + 1] - mb_off[b] + kTile - 1) / kTile); };
+  if (levels <= kMaxLevels) {
+    for (int i = threadIdx.x; i <= kMaxLevels; i += blockDim.x) s_hist[i] = 0;
+    __syncthreads();
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+      const int nq = nq_of(b);
+      if (nq > 0) atomicAdd(&s_hist[min(nkv_of(b), levels)], nq);
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
-      long long acc = s_base;
-      const int m = min((int)blockDim.x, c_hi + 1);
-      for (int i = 0; i < m; ++i) {
-        s_start[i] = acc;
-        acc += s_cnt[i];
+      long long acc = 0;
+      for (int c = levels; c >= 0; --c) {
+        s_cursor[c] = (int)(acc < (1ll << 30) ? acc : (1ll << 30));
+        acc += s_hist[c];
       }
       s_base = acc;
     }
     __syncthreads();
-    if (c >= 0) {
-      long long pos = s_start[threadIdx.x];
-      for (int64_t b = 0; b < B; ++b) {
-        const int64_t n = hoff[b + 1] - hoff[b];
-        const int nkv = (int)((n + kTile - 1) / kTile);
-        if (nkv != c) continue;
-        const int64_t rows = mb_off[b + 1] - mb_off[b];
-        const int nq = (int)((rows + kTile - 1) / kTile);
-        // items of one (user, head) are adjacent: they read the same history K/V
-        for (int hh = 0; hh < h; ++hh)
-          for (int qt = 0; qt < nq; ++qt) {
-            const long long idx = pos * h + (long long)hh * nq + qt;
-            if (idx < item_cap)
-              items[idx] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, nkv, 0,
-                                    (int32_t)(mb_off[b] + (int64_t)qt * kTile), (int32_t)hoff[b],
-                                    (int32_t)rows, (int32_t)n};
-          }
-        pos += nq;
-      }
+    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+      const int nq = nq_of(b);
+      if (nq == 0) continue;
+      const int c = min(nkv_of(b), levels);
+      emit(b, atomicAdd(&s_cursor[c], nq), c);
     }
-    __syncthreads();
+  } else if (threadIdx.x == 0) {  // histories over kMaxLevels * 128 rows: one thread walks them
+    long long pos = 0;
+    for (int c = levels; c >= 0; --c)
+      for (int64_t b = 0; b < B; ++b) {
+        if (nkv_of(b) != c || nq_of(b) == 0) continue;
+        emit(b, pos, c);
+        pos += nq_of(b);
+      }
+    s_base = pos;
   }
+  __syncthreads();
   if (threadIdx.x == 0) {
     hdr->n_cand_items = (int32_t)(s_base * h < item_cap ? s_base * h : item_cap);
     hdr->mb_rows = mb_off[B];
