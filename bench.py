@@ -45,6 +45,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def tensor_frac(tflops: float, peaks) -> dict:
+    """Whole-step algorithmic TFLOP/s as a fraction of the measured bf16 GEMM
+    rates (burst, sustained) and of the part's nominal dense bf16 rate."""
+    return {"of_burst": round(tflops / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 4),
+            "of_sustained": round(tflops / float(peaks.get("bf16_tflops_sustained",
+                                                           FALLBACK_PEAKS["bf16_tflops_sustained"])), 4),
+            "of_nominal": round(tflops / 2250.0, 4)}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -329,7 +338,12 @@ def run_ours(args):
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "peak_source": f"bf16_tflops_sustained ({peak_src})",
                     "traffic": ncu_traffic(dominant, w.name),
-                    "avg_launch_ms": round(tot / n, 4)}
+                    "avg_launch_ms": round(tot / n, 4),
+                    # the same achieved rate against the burst figure and the
+                    # nominal dense bf16 rate of the part (2.25 PFLOP/s)
+                    "frac_burst": round(achieved / float(peaks.get(
+                        "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 4),
+                    "frac_nominal": round(achieved / 2250.0, 4)}
     step_flops = args_layers = w.n_layers * sum(flops.values())
     del args_layers
 
@@ -386,6 +400,7 @@ def run_ours(args):
         mflop = mfalcon_flops(wm.dims, wm.n_layers, wm.lengths, np.diff(wm.cand_offsets))
         mf = {"value": C / (m_ms / 1e3), "unit": "candidates/s", "ms_per_step": round(m_ms, 4),
               "tflops": round(mflop / (m_ms / 1e3) / 1e12, 1),
+              "tensor_frac": tensor_frac(mflop / (m_ms / 1e3) / 1e12, peaks),
               "config": {"workload": "mfalcon", "users": wm.B, "candidates_per_user": wm.max_cands,
                          "microbatch": wm.microbatch, "layers": wm.n_layers, "d_model": 512,
                          "heads": 4, "head_dim": 128, "history_tokens": wm.T}}
@@ -420,6 +435,7 @@ def run_ours(args):
                        "l2": "256 MB flush between timed steps",
                        "parallelism": f"replicas x{world} (users independent, no collective)"},
             "tflops": round(step_flops / (ms / 1e3) / 1e12, 1),
+            "tensor_frac": tensor_frac(step_flops / (ms / 1e3) / 1e12, peaks),
             "roofline": roofline,
             "kernels": {k: {"launches": v[0], "ms": round(v[1], 3),
                             "share": round(v[1] / max(1e-9, sum(x[1] for x in per_kernel.values())), 4)}
