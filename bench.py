@@ -7,7 +7,9 @@ full-stack workload (128 users, Stochastic-Length-shortened lognormal
 lengths, ~36k tokens), i.e. every step of the layer path: schedule, f1 +
 SiLU, pointwise attention with relative bias, LayerNorm * U, f2 + residual.
 M-FALCON ranking (32 users, 1024 candidates each, 3 layers) is timed the same
-way and reported in the same line under "mfalcon".
+way and reported in the same line under "mfalcon"; Stochastic Length sampling
++ token embedding of the raw streams of a 128-user batch (1M-row content
+table) under "stochastic_length".
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream with a 256 MB L2 flush between steps (outside the
@@ -405,6 +407,53 @@ def run_ours(args):
                          "microbatch": wm.microbatch, "layers": wm.n_layers, "d_model": 512,
                          "heads": 4, "head_dim": 128, "history_tokens": wm.T}}
 
+    # ---------------- Stochastic Length + token embedding (raw streams of the
+    # same 128-user batch, 1M-row content table on the device)
+    sl = None
+    if not args.no_sl:
+        rs = hw.full_stack_raw(args.seed + rank)
+        ctab = hw.device_embedding_table(args.seed + rank, 0, rs.n_content, rs.d_model, dev)
+        atab = hw.device_embedding_table(args.seed + rank, 1, rs.n_actions, rs.d_model, dev)
+        s_in = [torch.from_numpy(a).to(dev) for a in (rs.raw_offsets, rs.raw_ids, rs.raw_timestamps)]
+        s_off = torch.empty(rs.B + 1, dtype=torch.int64, device=dev)
+        s_X = torch.empty(rs.R, rs.d_model, dtype=torch.bfloat16, device=dev)
+        s_ts = torch.empty(rs.R, dtype=torch.int64, device=dev)
+        s_ws = torch.empty(H.hstu_sl_embed_workspace_size(), dtype=torch.uint8, device=dev)
+
+        def sstep():
+            H.hstu_sl_embed(rs.B, rs.R, rs.max_raw_len, *s_in, rs.sl_seed, ctab, atab, s_off, s_X,
+                            s_ts, s_ws)
+        for _ in range(args.warmup):
+            sstep()
+        s_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for a, b in s_evs:
+            flush.zero_()
+            a.record(stream)
+            sstep()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if H.hstu_read_status(s_ws) != 0:
+            raise RuntimeError(f"Stochastic Length device status {H.hstu_read_status(s_ws)}")
+        s_ms = sum(a.elapsed_time(b) for a, b in s_evs) / len(s_evs)
+        kept = int(s_off[-1])
+        # algorithmic bytes: raw offsets in, kept offsets out, and per kept
+        # token its id and timestamp in, its timestamp and embedding row out
+        # plus the row read from the table (keys are computed, not read)
+        s_bytes = 16 * (rs.B + 1) + kept * (24 + 4 * rs.d_model)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        s_gbs = s_bytes / (s_ms / 1e3) / 1e9
+        sl = {"value": rs.R / (s_ms / 1e3), "unit": "raw tokens/s",
+              "kept_tokens_per_s": kept / (s_ms / 1e3), "ms_per_step": round(s_ms, 4),
+              "roofline": {"bound": "hbm", "kernels": "sl_offsets + sl_select",
+                           "achieved": round(s_gbs, 1), "peak": hbm, "unit": "GB/s",
+                           "frac": round(s_gbs / hbm, 4), "peak_source": f"hbm_gbs ({peak_src})",
+                           "bytes_per_step": int(s_bytes),
+                           "traffic": ncu_traffic("sl_select", rs.name)},
+              "config": {"workload": rs.name, "users": rs.B, "raw_tokens": rs.R,
+                         "kept_tokens": kept, "d_model": rs.d_model,
+                         "content_rows": rs.n_content, "action_rows": rs.n_actions}}
+
     # ---------------- reduce over ranks
     tokens = float(T)
     if world > 1:
@@ -420,6 +469,14 @@ def run_ours(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             mf["value"] = wm.candidates.shape[0] * world / (float(t[0]) / 1e3)
             mf["ms_per_step"] = float(t[0])
+        if sl is not None:
+            t = torch.tensor([sl["ms_per_step"], rs.R, sl["config"]["kept_tokens"]],
+                             dtype=torch.float64, device=dev)
+            dist.all_reduce(t[:1], op=dist.ReduceOp.MAX)
+            dist.all_reduce(t[1:], op=dist.ReduceOp.SUM)
+            sl["ms_per_step"] = float(t[0])
+            sl["value"] = float(t[1]) / (float(t[0]) / 1e3)
+            sl["kept_tokens_per_s"] = float(t[2]) / (float(t[0]) / 1e3)
 
     line = None
     if rank == 0:
@@ -447,6 +504,7 @@ def run_ours(args):
             "gpu_launches": int(n_launch),
             "clocks": clk.summary(),
             "mfalcon": mf,
+            "stochastic_length": sl,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -492,6 +550,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-mfalcon", action="store_true")
+    ap.add_argument("--no-sl", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)

@@ -20,11 +20,11 @@ LIB_PATH = os.path.join(_HERE, "libhstu.so")
 HSTU_BF16, HSTU_FP32 = 0, 1
 STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED",
                 3: "HSTU_ERR_WORKSPACE", 4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_BAD_OFFSETS",
-                6: "HSTU_ERR_TIMEOUT", 7: "HSTU_ERR_BAD_TIMESTAMPS"}
+                6: "HSTU_ERR_TIMEOUT", 7: "HSTU_ERR_BAD_TIMESTAMPS", 8: "HSTU_ERR_BAD_IDS"}
 
 # Every symbol include/hstu.h declares.
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
-            "hstu_layer_fwd_noalloc",
+            "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
@@ -76,6 +76,11 @@ def lib() -> ctypes.CDLL:
     L.hstu_mfalcon_rank.restype = i32
     L.hstu_layer_fwd_noalloc.argtypes = [pdesc, i64, i64, i64, vp, vp, pw, vp, vp, vp]
     L.hstu_layer_fwd_noalloc.restype = i32
+    L.hstu_sl_embed_workspace_size.argtypes = []
+    L.hstu_sl_embed_workspace_size.restype = sz
+    L.hstu_sl_embed.argtypes = [i64, i64, i64, vp, vp, vp, ctypes.c_uint64, vp, i64, vp, i64, i32,
+                                vp, vp, vp, vp, sz, vp]
+    L.hstu_sl_embed.restype = i32
     L.hstu_read_status.argtypes = [vp, sz, vp]
     L.hstu_read_status.restype = i32
     L.hstu_debug_offsets.argtypes = [pdesc, i64, i64, i64, ctypes.POINTER(sz),
@@ -191,6 +196,25 @@ def hstu_layer_fwd_noalloc(desc, B, total_tokens, max_len, offsets, X, weights, 
                                         _ptr(offsets), _ptr(X), ctypes.byref(ws),
                                         _ptr(timestamps), _ptr(out), _stream(stream)),
            "hstu_layer_fwd_noalloc")
+
+
+def hstu_sl_embed_workspace_size() -> int:
+    return int(lib().hstu_sl_embed_workspace_size())
+
+
+def hstu_sl_embed(B, raw_total, max_raw_len, raw_offsets, raw_ids, raw_timestamps, seed,
+                  content_table, action_table, out_offsets, out_X, out_timestamps, workspace,
+                  stream=None) -> None:
+    """Stochastic Length + token embedding on the device (see include/hstu.h);
+    the tables are bf16 [rows, d] device tensors."""
+    _check(lib().hstu_sl_embed(B, raw_total, max_raw_len, _ptr(raw_offsets), _ptr(raw_ids),
+                               _ptr(raw_timestamps), int(seed) & ((1 << 64) - 1),
+                               _ptr(content_table), int(content_table.shape[0]),
+                               _ptr(action_table), int(action_table.shape[0]),
+                               int(content_table.shape[1]), _ptr(out_offsets), _ptr(out_X),
+                               _ptr(out_timestamps), _ptr(workspace), _nbytes(workspace),
+                               _stream(stream)),
+           "hstu_sl_embed")
 
 
 def hstu_stack_fwd(desc, n_layers, weights, B, total_tokens, max_len, offsets, X, timestamps,

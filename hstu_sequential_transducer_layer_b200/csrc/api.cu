@@ -496,6 +496,7 @@ const char* hstu_status_string(hstu_status s) {
     case HSTU_ERR_BAD_OFFSETS: return "bad offsets (device check)";
     case HSTU_ERR_TIMEOUT: return "in-kernel wait timed out (device check)";
     case HSTU_ERR_BAD_TIMESTAMPS: return "timestamps span 2^30 s or more within a user (device check)";
+    case HSTU_ERR_BAD_IDS: return "a token id outside its embedding table (device check)";
   }
   return "unknown status";
 }

@@ -32,7 +32,9 @@ enum KernelId : int32_t {
   K_SIMT_ATTN_CAND = 13,
   K_CONVERT = 14,
   K_TIME_BUCKETS = 15,
-  K_NUM_KERNELS = 16
+  K_SL_OFFSETS = 16,
+  K_SL_SELECT = 17,
+  K_NUM_KERNELS = 18
 };
 const char* kernel_name(int id);
 

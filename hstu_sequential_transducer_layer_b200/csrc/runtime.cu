@@ -23,7 +23,8 @@ const char* kernel_name(int id) {
       "schedule",   "time_rel",   "gemm_f1_tc",      "attn_tc",
       "ln_gate",    "gemm_f2_tc", "mb_plan",         "mb_gather",
       "attn_cand_tc", "score",    "gemm_f1_simt_f32", "attn_simt_f32",
-      "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16", "time_buckets"};
+      "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16", "time_buckets",
+      "sl_offsets", "sl_select"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 

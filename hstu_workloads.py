@@ -362,6 +362,83 @@ def full_stack(seed: int = 0, n_users: int = 128) -> Workload:
     return _finish(w)
 
 
+@dataclass
+class RawStream:
+    """Raw (not yet shortened) token streams of a batch of users: the input of
+    Stochastic Length + token embedding.  Content and action tokens alternate
+    by position (content at even positions); ids index the content table
+    (n_content rows) or the action table (n_actions rows)."""
+    name: str
+    raw_offsets: np.ndarray        # int64 [B+1]
+    raw_ids: np.ndarray            # int64 [R]
+    raw_timestamps: np.ndarray     # int64 [R]
+    n_content: int
+    n_actions: int
+    d_model: int
+    sl_seed: int                   # 64-bit Stochastic Length seed
+    max_raw_len: int
+
+    @property
+    def B(self) -> int:
+        return len(self.raw_offsets) - 1
+
+    @property
+    def R(self) -> int:
+        return int(self.raw_offsets[-1])
+
+
+def _raw_stream(rng, name, lengths, d_model, n_content, n_actions, zipf_s, max_raw_len):
+    lengths = np.asarray(lengths, np.int64)
+    cdf = _zipf_cdf(n_content, zipf_s)
+    perm = rng.permutation(n_content)
+    ts, ids = [np.zeros(0, np.int64)], [np.zeros(0, np.int64)]
+    for n in lengths:
+        n = int(n)
+        ts.append(_timestamps(rng, n) + int(rng.integers(0, 1 << 31)))
+        u = rng.random(n)
+        rank = np.minimum(np.searchsorted(cdf, u, side="left"), n_content - 1)
+        act = rng.integers(0, n_actions, size=n)
+        ids.append(np.where(np.arange(n) % 2 == 0, perm[rank], act).astype(np.int64))
+    seed = int(rng.integers(0, 1 << 63)) * 2 + int(rng.integers(0, 2))
+    return RawStream(name, _offsets(lengths), np.concatenate(ids), np.concatenate(ts),
+                     n_content, n_actions, d_model, seed,
+                     int(max_raw_len if max_raw_len is not None else max(lengths.max(initial=0), 1)))
+
+
+def raw_stream(name: str, lengths, d_model: int, n_content: int, n_actions: int = 8,
+               seed: int = 0, zipf_s: float = 1.1, max_raw_len: Optional[int] = None) -> RawStream:
+    """Raw streams of the given lengths: per user Exp(60 s) gaps from a random
+    31-bit epoch, content ids Zipf(zipf_s) over n_content (fixed random id
+    permutation), actions uniform over n_actions, and a random 64-bit seed."""
+    return _raw_stream(np.random.default_rng(seed), name, lengths, d_model, n_content, n_actions,
+                       zipf_s, max_raw_len)
+
+
+def full_stack_raw(seed: int = 0, n_users: int = 128) -> RawStream:
+    """The raw input of the 8-layer stack workload: B=128 users, raw lengths
+    lognormal(median 1000, sigma 1) clipped to [2, 4096], d=1024, content ids
+    Zipf(1.1) over 1M ids, 8 action types."""
+    rng = np.random.default_rng([seed, 4096])
+    raw = _lognormal_lengths(rng, n_users, 1000, 1.0, 2, 4096)
+    return _raw_stream(rng, "full_stack_raw", raw, 1024, 1_000_000, 8, 1.1, 4096)
+
+
+def embedding_table_bits(seed: int, table: int, rows: int, d: int) -> np.ndarray:
+    """An N(0,1) embedding table rounded to bf16, as uint16 bit patterns [rows, d]."""
+    a = np.random.default_rng([seed, 7919, table]).standard_normal((rows, d), dtype=np.float32)
+    return bf16_bits(round_to_bf16(a))
+
+
+def device_embedding_table(seed: int, table: int, rows: int, d: int, device):
+    """An N(0,1) bf16 embedding table [rows, d] drawn by torch's generator on
+    `device` (for tables too large to draw on the host; copy it back to feed
+    the oracle)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed((seed * 1_000_003 + 7919 * (table + 1)) & ((1 << 63) - 1))
+    return torch.randn(rows, d, generator=g, device=device, dtype=torch.bfloat16)
+
+
 WORKLOADS = {
     "tiny_fp32": tiny_fp32,
     "single_layer": single_layer,

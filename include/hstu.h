@@ -85,7 +85,8 @@ typedef enum {
   HSTU_ERR_CUDA = 4,          /* host: a CUDA runtime call failed */
   HSTU_ERR_BAD_OFFSETS = 5,   /* device: offsets not monotone, wrong total, length > max */
   HSTU_ERR_TIMEOUT = 6,       /* device: an in-kernel wait gave up */
-  HSTU_ERR_BAD_TIMESTAMPS = 7 /* device: a user's timestamps span 2^30 s or more */
+  HSTU_ERR_BAD_TIMESTAMPS = 7, /* device: a user's timestamps span 2^30 s or more */
+  HSTU_ERR_BAD_IDS = 8         /* device: a token id outside its embedding table */
 } hstu_status;
 
 typedef enum { HSTU_BF16 = 0, HSTU_FP32 = 1 } hstu_dtype;
@@ -187,6 +188,40 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
                                    int64_t max_len, const int64_t* offsets, const void* X,
                                    const hstu_layer_weights* weights, const int64_t* timestamps,
                                    void* out, void* stream);
+
+/* Stochastic Length sampling and token embedding ('HSTUとGenerative
+ * Recommenders', section '2. Stochastic Lengthで学習時の履歴を間引く': a long
+ * history is shortened to a random subset of its positions; 4096 tokens keep
+ * 776).  For each user b with a raw sequence of n_b tokens, keeps
+ * k_b = min(n_b, floor(n_b^0.8)) (at least 1) positions: those whose keys are
+ * smallest, the key of position p being output number b * 2^32 + p + 1 of the
+ * SplitMix64 generator started from state `seed`, ties by position; the kept
+ * tokens stay in their original order.  A kept token at an even original
+ * position is a content item (row raw_ids[.] of content_table), at an odd
+ * position an action (row of action_table).
+ *   raw_offsets     device int64 [B+1], raw_offsets[0] = 0, [B] = raw_total,
+ *                   each length at most max_raw_len (<= 32767)
+ *   raw_ids         device int64 [raw_total] (row indices into the tables)
+ *   raw_timestamps  device int64 [raw_total]
+ *   content_table   device bf16 [n_content, d_model], 16-byte aligned
+ *   action_table    device bf16 [n_action, d_model], 16-byte aligned
+ *   out_offsets     device int64 [B+1]: the kept sequences' offsets
+ *   out_X           device bf16 [sum k_b, d_model] (at most raw_total rows)
+ *   out_timestamps  device int64 [sum k_b]
+ *   workspace       hstu_sl_embed_workspace_size() bytes, 256-byte aligned
+ *                   (holds the device status word)
+ * d_model must be a multiple of 8.  Host-detectable errors return at once;
+ * bad offsets or an id outside its table set the status word
+ * (HSTU_ERR_BAD_OFFSETS: all out_offsets are 0; HSTU_ERR_BAD_IDS: that row is
+ * zero), read back with hstu_read_status.  Asynchronous on `stream`. */
+size_t hstu_sl_embed_workspace_size(void);
+hstu_status hstu_sl_embed(int64_t B, int64_t raw_total, int64_t max_raw_len,
+                          const int64_t* raw_offsets, const int64_t* raw_ids,
+                          const int64_t* raw_timestamps, uint64_t seed,
+                          const void* content_table, int64_t n_content,
+                          const void* action_table, int64_t n_action, int32_t d_model,
+                          int64_t* out_offsets, void* out_X, int64_t* out_timestamps,
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then returns the device status word that the last
  * call using this workspace left (HSTU_OK if none of its checks failed). */
