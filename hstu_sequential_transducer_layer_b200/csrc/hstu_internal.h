@@ -34,7 +34,8 @@ enum KernelId : int32_t {
   K_TIME_BUCKETS = 15,
   K_SL_OFFSETS = 16,
   K_SL_SELECT = 17,
-  K_NUM_KERNELS = 18
+  K_SL_GATHER = 18,
+  K_NUM_KERNELS = 19
 };
 const char* kernel_name(int id);
 
