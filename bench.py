@@ -9,7 +9,8 @@ SiLU, pointwise attention with relative bias, LayerNorm * U, f2 + residual.
 M-FALCON ranking (32 users, 1024 candidates each, 3 layers) is timed the same
 way and reported in the same line under "mfalcon"; Stochastic Length sampling
 + token embedding of the raw streams of a 128-user batch (1M-row content
-table) under "stochastic_length".
+table) under "stochastic_length", and those raw streams through Stochastic
+Length, embedding and the 8-layer stack under "full_pipeline".
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream with a 256 MB L2 flush between steps (outside the
@@ -433,6 +434,20 @@ def run_ours(args):
             sstep()
             b.record(stream)
         torch.cuda.synchronize()
+        # per-kernel times from a second, traced pass (an event pair around
+        # each of three short kernels would inflate the step timed above)
+        H.hstu_trace_enable(args.steps * 3 + 8)
+        for _ in range(args.steps):
+            flush.zero_()
+            sstep()
+        torch.cuda.synchronize()
+        s_trace = H.hstu_trace_read()
+        H.hstu_trace_enable(0)
+        s_kern = {}
+        for kid, t in s_trace:
+            e = s_kern.setdefault(H.hstu_kernel_name(kid), [0, 0.0])
+            e[0] += 1
+            e[1] += t
         if H.hstu_read_status(s_ws) != 0:
             raise RuntimeError(f"Stochastic Length device status {H.hstu_read_status(s_ws)}")
         s_ms = sum(a.elapsed_time(b) for a, b in s_evs) / len(s_evs)
@@ -443,16 +458,81 @@ def run_ours(args):
         s_bytes = 16 * (rs.B + 1) + kept * (24 + 4 * rs.d_model)
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         s_gbs = s_bytes / (s_ms / 1e3) / 1e9
+        # the gather kernel moves all of those bytes except the offsets
+        g_n, g_ms = s_kern.get("sl_gather", [1, float("nan")])
+        g_bytes = kept * (24 + 4 * rs.d_model)
+        g_gbs = g_bytes / (g_ms / g_n / 1e3) / 1e9
         sl = {"value": rs.R / (s_ms / 1e3), "unit": "raw tokens/s",
               "kept_tokens_per_s": kept / (s_ms / 1e3), "ms_per_step": round(s_ms, 4),
-              "roofline": {"bound": "hbm", "kernels": "sl_offsets + sl_select",
-                           "achieved": round(s_gbs, 1), "peak": hbm, "unit": "GB/s",
-                           "frac": round(s_gbs / hbm, 4), "peak_source": f"hbm_gbs ({peak_src})",
-                           "bytes_per_step": int(s_bytes),
-                           "traffic": ncu_traffic("sl_select", rs.name)},
+              "step_hbm": {"achieved": round(s_gbs, 1), "frac": round(s_gbs / hbm, 4),
+                           "bytes_per_step": int(s_bytes)},
+              "roofline": {"bound": "hbm", "kernel": "sl_gather", "achieved": round(g_gbs, 1),
+                           "peak": hbm, "unit": "GB/s", "frac": round(g_gbs / hbm, 4),
+                           "peak_source": f"hbm_gbs ({peak_src})", "bytes_per_launch": int(g_bytes),
+                           "avg_launch_ms": round(g_ms / g_n, 4),
+                           "traffic": ncu_traffic("sl_gather", rs.name)},
+              "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / v[0], 4)}
+                          for k, v in s_kern.items()},
               "config": {"workload": rs.name, "users": rs.B, "raw_tokens": rs.R,
                          "kept_tokens": kept, "d_model": rs.d_model,
                          "content_rows": rs.n_content, "action_rows": rs.n_actions}}
+
+    # ---------------- the whole path from raw streams: Stochastic Length +
+    # embedding, then the 8-layer stack (same weights as the main step)
+    pipe = None
+    if sl is not None:
+        raw_len = np.diff(rs.raw_offsets)
+        kept_sz = r.kept_sizes(raw_len)
+        p_T = kept_sz[0]
+        p_out = torch.empty(p_T, rs.d_model, dtype=torch.bfloat16, device=dev)
+
+        def pstep(ins):
+            r.stack_raw(raw_len, *ins, rs.sl_seed, ctab, atab, rs.max_raw_len, out=p_out,
+                        kept=kept_sz)
+        for _ in range(args.warmup):
+            pstep(s_in)
+        p_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for a, b in p_evs:
+            flush.zero_()
+            a.record(stream)
+            pstep(s_in)
+            b.record(stream)
+        torch.cuda.synchronize()
+        if r.sl_status() != 0 or r.status() != 0:
+            raise RuntimeError(f"pipeline device status {r.sl_status()} / {r.status()}")
+        p_ms = sum(a.elapsed_time(b) for a, b in p_evs) / len(p_evs)
+        # end to end: the raw streams come from pinned host memory every step
+        # (embedding tables and weights stay resident) and Y goes back
+        h_in = [torch.from_numpy(a).pin_memory() for a in (rs.raw_offsets, rs.raw_ids,
+                                                          rs.raw_timestamps)]
+        d_in = [torch.empty_like(x, device=dev) for x in h_in]
+        p_Yh = torch.empty(p_out.shape, dtype=p_out.dtype).pin_memory()
+        pe_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(max(3, args.steps // 2))]
+        for a, b in pe_evs:
+            flush.zero_()
+            a.record(stream)
+            for x, y in zip(d_in, h_in):
+                x.copy_(y, non_blocking=True)
+            pstep(d_in)
+            p_Yh.copy_(p_out, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        pe_ms = sum(a.elapsed_time(b) for a, b in pe_evs) / len(pe_evs)
+        kept_len = np.array([H.hstu_sl_keep_count(int(n)) for n in raw_len])
+        pf = layer_flops(w.dims, kept_len)
+        p_flops = w.n_layers * sum(pf.values())
+        pipe = {"value": p_T / (p_ms / 1e3), "unit": "tokens/s", "ms_per_step": round(p_ms, 4),
+                "tflops": round(p_flops / (p_ms / 1e3) / 1e12, 1),
+                "tensor_frac": tensor_frac(p_flops / (p_ms / 1e3) / 1e12, peaks),
+                "e2e": {"value": p_T / (pe_ms / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": int(sum(x.numel() * 8 for x in h_in)),
+                        "d2h_bytes_per_step": int(p_Yh.numel() * p_Yh.element_size()),
+                        "ms_per_step": round(pe_ms, 4)},
+                "config": {"workload": "full_stack_raw -> Stochastic Length -> 8-layer stack",
+                           "users": rs.B, "raw_tokens": rs.R, "tokens": p_T,
+                           "max_len": kept_sz[1]}}
 
     # ---------------- reduce over ranks
     tokens = float(T)
@@ -469,6 +549,15 @@ def run_ours(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             mf["value"] = wm.candidates.shape[0] * world / (float(t[0]) / 1e3)
             mf["ms_per_step"] = float(t[0])
+        if pipe is not None:
+            t = torch.tensor([pipe["ms_per_step"], pipe["e2e"]["ms_per_step"]],
+                             dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            s = torch.tensor([p_T], dtype=torch.float64, device=dev)
+            dist.all_reduce(s, op=dist.ReduceOp.SUM)
+            pipe["ms_per_step"], pipe["e2e"]["ms_per_step"] = float(t[0]), float(t[1])
+            pipe["value"] = float(s[0]) / (float(t[0]) / 1e3)
+            pipe["e2e"]["value"] = float(s[0]) / (float(t[1]) / 1e3)
         if sl is not None:
             t = torch.tensor([sl["ms_per_step"], rs.R, sl["config"]["kept_tokens"]],
                              dtype=torch.float64, device=dev)
@@ -505,6 +594,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "mfalcon": mf,
             "stochastic_length": sl,
+            "full_pipeline": pipe,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -25,6 +25,7 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 # Every symbol include/hstu.h declares.
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
             "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
+            "hstu_sl_keep_count",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_layer_fwd_noalloc.restype = i32
     L.hstu_sl_embed_workspace_size.argtypes = []
     L.hstu_sl_embed_workspace_size.restype = sz
+    L.hstu_sl_keep_count.argtypes = [i64]
+    L.hstu_sl_keep_count.restype = i64
     L.hstu_sl_embed.argtypes = [i64, i64, i64, vp, vp, vp, ctypes.c_uint64, vp, i64, vp, i64, i32,
                                 vp, vp, vp, vp, sz, vp]
     L.hstu_sl_embed.restype = i32
@@ -200,6 +203,10 @@ def hstu_layer_fwd_noalloc(desc, B, total_tokens, max_len, offsets, X, weights, 
 
 def hstu_sl_embed_workspace_size() -> int:
     return int(lib().hstu_sl_embed_workspace_size())
+
+
+def hstu_sl_keep_count(n: int) -> int:
+    return int(lib().hstu_sl_keep_count(int(n)))
 
 
 def hstu_sl_embed(B, raw_total, max_raw_len, raw_offsets, raw_ids, raw_timestamps, seed,

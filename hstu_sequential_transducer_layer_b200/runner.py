@@ -60,6 +60,46 @@ class HSTURunner:
                               ws, stream)
         return out
 
+    def kept_sizes(self, raw_lengths) -> tuple:
+        """(total, max) of the Stochastic Length keep counts of raw streams of
+        the given lengths, from the library's host keep count."""
+        k = [_b.hstu_sl_keep_count(int(n)) for n in raw_lengths]
+        if any(x < 0 for x in k):
+            raise _b.HstuError(2, "hstu_sl_keep_count")
+        return int(sum(k)), int(max(k, default=0))
+
+    def stack_raw(self, raw_lengths, raw_offsets, raw_ids, raw_ts, seed: int, content_table,
+                  action_table, max_raw_len: int, out=None, stream=None, kept=None):
+        """Raw token streams -> Stochastic Length + token embedding
+        (hstu_sl_embed) -> the layer stack (hstu_stack_fwd), all on `stream`
+        with no host synchronisation.  `raw_lengths` (host) sizes the kept
+        batch (or `kept` = kept_sizes(raw_lengths), computed once by the
+        caller); the device tensors carry the data.  Returns (out, kept
+        offsets, kept timestamps)."""
+        t = self.torch
+        B = raw_offsets.numel() - 1
+        R = raw_ids.numel()
+        T, max_len = kept if kept is not None else self.kept_sizes(raw_lengths)
+        d = int(content_table.shape[1])
+        key = (B, T, d)
+        if getattr(self, "_sl_key", None) != key:
+            self._sl_key = key
+            self._sl_off = t.empty(B + 1, dtype=t.int64, device=self.device)
+            self._sl_X = t.empty(max(T, 1), d, dtype=t.bfloat16, device=self.device)
+            self._sl_ts = t.empty(max(T, 1), dtype=t.int64, device=self.device)
+            self._sl_ws = t.empty(_b.hstu_sl_embed_workspace_size(), dtype=t.uint8,
+                                  device=self.device)
+        _b.hstu_sl_embed(B, R, max_raw_len, raw_offsets, raw_ids, raw_ts, seed, content_table,
+                         action_table, self._sl_off, self._sl_X, self._sl_ts, self._sl_ws, stream)
+        X = self._sl_X[:T]
+        if out is None:
+            out = t.empty_like(X)
+        self.stack(self._sl_off, X, self._sl_ts[:T], max_len, out=out, stream=stream)
+        return out, self._sl_off, self._sl_ts[:T]
+
+    def sl_status(self, stream=None) -> int:
+        return _b.hstu_read_status(self._sl_ws, stream)
+
     def rank(self, hist_offsets, history, hist_ts, cand_offsets, candidates, request_ts,
              microbatch: int, head_vec, max_len: int, max_cands: int, scores=None, stream=None):
         B = hist_offsets.numel() - 1

@@ -215,6 +215,12 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
  * (HSTU_ERR_BAD_OFFSETS: all out_offsets are 0; HSTU_ERR_BAD_IDS: that row is
  * zero), read back with hstu_read_status.  Asynchronous on `stream`. */
 size_t hstu_sl_embed_workspace_size(void);
+/* The keep count k(n) = min(n, floor(n^0.8)) (at least 1 for n >= 1) that
+ * hstu_sl_embed applies to a raw stream of n tokens, computed on the host
+ * with the same integer definition (the largest k with k^5 <= n^4), so a
+ * caller can size the kept batch (sum and max of k) without reading the
+ * device.  Returns -1 for n < 0 or n > 32767. */
+int64_t hstu_sl_keep_count(int64_t n);
 hstu_status hstu_sl_embed(int64_t B, int64_t raw_total, int64_t max_raw_len,
                           const int64_t* raw_offsets, const int64_t* raw_ids,
                           const int64_t* raw_timestamps, uint64_t seed,

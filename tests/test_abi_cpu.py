@@ -118,3 +118,12 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(B.HstuError):
         B.lib()
+
+
+def test_host_keep_count_matches_oracle():
+    """The library's host keep count (used to size the kept batch) equals the
+    oracle's for every supported raw length, and refuses the rest."""
+    from oracle import stochastic_length as SL
+    got = [B.hstu_sl_keep_count(n) for n in range(0, 32768)]
+    assert got == [SL.keep_count(n) for n in range(0, 32768)]
+    assert B.hstu_sl_keep_count(-1) == -1 and B.hstu_sl_keep_count(32768) == -1

@@ -100,6 +100,14 @@ def test_many_users_more_than_one_wave():
     _check(rs, c, a)
 
 
+def test_more_users_than_one_block_can_offset():
+    # beyond 2048 users the kept offsets come from their own kernel
+    rng = np.random.default_rng(12)
+    lengths = rng.integers(0, 60, size=2500)
+    rs, c, a = _small(lengths, d=8, n_content=500, seed=12)
+    _check(rs, c, a)
+
+
 def test_empty_batch_and_all_empty_users():
     for lengths in ([], [0, 0, 0]):
         rs, c, a = _small(lengths, d=64, seed=3)
@@ -145,6 +153,16 @@ def test_bad_offsets_set_status():
         st, o, _, _ = _run(rs, ct, at, raw_offsets=off)
         assert st == HSTU_ERR_BAD_OFFSETS, (off, st)
         np.testing.assert_array_equal(o, np.zeros(4, np.int64))
+    # no users but a nonzero raw total
+    st, o, _, _ = _run(rs, ct, at, raw_offsets=np.array([0]))
+    assert st == HSTU_ERR_BAD_OFFSETS and o.tolist() == [0]
+    # a batch larger than the single-block offsets path, one length negative
+    rs_big, cb, ab = _small(np.full(2100, 3), d=16, seed=4)
+    off = rs_big.raw_offsets.copy()
+    off[1000] = off[1002]
+    st, o, _, _ = _run(rs_big, _bits_to_device(cb), _bits_to_device(ab), raw_offsets=off)
+    assert st == HSTU_ERR_BAD_OFFSETS
+    np.testing.assert_array_equal(o, np.zeros(2101, np.int64))
     # a user longer than max_raw_len
     rs.max_raw_len = 25
     st, o, _, _ = _run(rs, ct, at)
@@ -173,3 +191,34 @@ def test_bad_id_sets_status_and_zeroes_its_row():
     assert not xb[bad_row].any()
     keep = np.arange(len(ref_x)) != bad_row
     np.testing.assert_array_equal(xb[keep].astype(np.float64), ref_x[keep])
+
+
+def _bits_to_f32(bits):
+    return (np.asarray(bits, np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def test_pipeline_raw_streams_to_stack_matches_oracle():
+    """Raw streams -> Stochastic Length + embedding -> 2-layer stack on the
+    GPU (HSTURunner.stack_raw, no host synchronisation in between) against
+    the oracle's sl_embed followed by its stack."""
+    import torch
+    from oracle import hstu_oracle as O
+    from gpu_util import TOL, relerr, rmserr, runner_for
+    dims = hw.LayerDims(256, 2, 128, 128, 128, 128, 4, 2, 1e-6, hw.BF16)
+    w = hw.custom("pipe", [1], dims, n_layers=2, seed=50)
+    rs, c, a = _small([2000, 1, 700, 0, 129, 4096], d=256, n_content=3000, seed=50)
+    ref_o, ref_x, ref_ts = SL.sl_embed(rs.raw_offsets, rs.raw_ids, rs.raw_timestamps, rs.sl_seed,
+                                       _bits_to_f32(c), _bits_to_f32(a))
+    ref = O.stack_fwd(ref_x, ref_o, ref_ts, w.weights, dims)
+    r = runner_for(w)
+    dev = [torch.from_numpy(x).cuda() for x in (rs.raw_offsets, rs.raw_ids, rs.raw_timestamps)]
+    out, off, ts = r.stack_raw(np.diff(rs.raw_offsets), *dev, rs.sl_seed, _bits_to_device(c),
+                               _bits_to_device(a), rs.max_raw_len)
+    torch.cuda.synchronize()
+    assert r.sl_status() == HSTU_OK and r.status() == HSTU_OK
+    np.testing.assert_array_equal(off.cpu().numpy(), ref_o)
+    np.testing.assert_array_equal(ts.cpu().numpy(), ref_ts)
+    Y = out.double().cpu().numpy()
+    e, ed = relerr(Y, ref), rmserr(Y - ref_x, ref - ref_x)
+    print("pipeline", e, ed)
+    assert e <= TOL[hw.BF16] and ed <= TOL[hw.BF16]
