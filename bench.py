@@ -205,23 +205,32 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- traffic from ncu
-def kernel_source_hash():
+# the source files each profiled kernel is built from (its own translation
+# unit plus the shared device helpers and declarations)
+KERNEL_SOURCES = {
+    "gemm_f1_tc": ["gemm_tc.cu"], "gemm_f2_tc": ["gemm_tc.cu"], "attn_tc": ["attn_tc.cu"],
+    "ln_gate": ["sched.cu"], "sl_select": ["sl.cu"], "sl_gather": ["sl.cu"],
+}
+
+
+def kernel_source_hash(kernel: str):
+    csrc = os.path.join(ROOT, "hstu_sequential_transducer_layer_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "hstu_sequential_transducer_layer_b200", "csrc"))):
-        with open(os.path.join(ROOT, "hstu_sequential_transducer_layer_b200", "csrc", f), "rb") as fh:
+    for f in KERNEL_SOURCES.get(kernel, []) + ["ptx.cuh", "hstu_internal.h"]:
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str, workload: str):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if its
-    recorded source hash matches the current kernels (else null)."""
+    recorded source hash matches the kernel's current sources (else null)."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+    if d.get("source_hash") != kernel_source_hash(kernel):
         return None
     return d.get("dram_bytes_per_launch")
 

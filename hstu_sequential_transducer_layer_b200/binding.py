@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 # Every symbol include/hstu.h declares.
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
             "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
-            "hstu_sl_keep_count",
+            "hstu_sl_keep_count", "hstu_bf16_to_f16",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
@@ -48,7 +48,8 @@ class LayerWeights(ctypes.Structure):
     _fields_ = [("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
                 ("b2", ctypes.c_void_p), ("ln_gamma", ctypes.c_void_p),
                 ("ln_beta", ctypes.c_void_p), ("rab_pos", ctypes.c_void_p),
-                ("rab_time", ctypes.c_void_p)]
+                ("rab_time", ctypes.c_void_p), ("W1_f16", ctypes.c_void_p),
+                ("W2_f16", ctypes.c_void_p)]
 
 
 _lib = None
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_sl_embed_workspace_size.restype = sz
     L.hstu_sl_keep_count.argtypes = [i64]
     L.hstu_sl_keep_count.restype = i64
+    L.hstu_bf16_to_f16.argtypes = [vp, vp, i64, vp]
+    L.hstu_bf16_to_f16.restype = i32
     L.hstu_sl_embed.argtypes = [i64, i64, i64, vp, vp, vp, ctypes.c_uint64, vp, i64, vp, i64, i32,
                                 vp, vp, vp, vp, sz, vp]
     L.hstu_sl_embed.restype = i32
@@ -143,7 +146,9 @@ def weights_struct(w: Dict[str, object]) -> LayerWeights:
     """LayerWeights from a dict of device tensors (W1, b1, W2, b2, ln_gamma,
     ln_beta, rab_pos, rab_time)."""
     return LayerWeights(*[_ptr(w[k]) for k in ("W1", "b1", "W2", "b2", "ln_gamma", "ln_beta",
-                                                "rab_pos", "rab_time")])
+                                                "rab_pos", "rab_time")],
+                        *[_ptr(w[k]) if w.get(k) is not None else None
+                          for k in ("W1_f16", "W2_f16")])
 
 
 def weights_array(ws: Sequence[Dict[str, object]]):
@@ -203,6 +208,12 @@ def hstu_layer_fwd_noalloc(desc, B, total_tokens, max_len, offsets, X, weights, 
 
 def hstu_sl_embed_workspace_size() -> int:
     return int(lib().hstu_sl_embed_workspace_size())
+
+
+def hstu_bf16_to_f16(src, dst, stream=None) -> None:
+    """fp16 copy of a bf16 device tensor (same shape) through the library."""
+    _check(lib().hstu_bf16_to_f16(_ptr(src), _ptr(dst), int(src.numel()), _stream(stream)),
+           "hstu_bf16_to_f16")
 
 
 def hstu_sl_keep_count(n: int) -> int:

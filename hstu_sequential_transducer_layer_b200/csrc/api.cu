@@ -42,6 +42,8 @@ hstu_status check_weights(const hstu_layer_weights* w) {
   const void* p[8] = {w->W1, w->b1, w->W2, w->b2, w->ln_gamma, w->ln_beta, w->rab_pos, w->rab_time};
   for (const void* q : p)
     if (!q || !al16(q)) return HSTU_ERR_INVALID_ARG;
+  if ((w->W1_f16 && !al16(w->W1_f16)) || (w->W2_f16 && !al16(w->W2_f16)))
+    return HSTU_ERR_INVALID_ARG;
   return HSTU_OK;
 }
 
@@ -103,10 +105,10 @@ LayerOps layer_ops(const Ctx& c, const hstu_layer_weights& w, const Layout& L, v
   const size_t F = c.F, dm = c.d.d_model, hdv = c.hdv;
   uint8_t* base = at<uint8_t>(ws, L.w16) + (size_t)l * (F * dm + dm * hdv) * 2;
   if (l > 0) {
-    o.W1 = base;
+    o.W1 = w.W1_f16 ? w.W1_f16 : base;
     o.w1_f16 = 1;
   }
-  o.W2 = base + F * dm * 2;
+  o.W2 = w.W2_f16 ? w.W2_f16 : base + F * dm * 2;
   (void)n_layers;
   return o;
 }
@@ -120,8 +122,8 @@ cudaError_t convert_weights(const Ctx& c, const hstu_layer_weights* w, int n_lay
   ConvBatch cb{};
   for (int l = 0; l < n_layers; ++l) {
     LayerOps o = layer_ops(c, w[l], L, ws, l, n_layers);
-    if (l > 0) cb.seg[cb.n++] = ConvSeg{w[l].W1, const_cast<void*>(o.W1), F * dm};
-    cb.seg[cb.n++] = ConvSeg{w[l].W2, const_cast<void*>(o.W2), dm * hdv};
+    if (l > 0 && !w[l].W1_f16) cb.seg[cb.n++] = ConvSeg{w[l].W1, const_cast<void*>(o.W1), F * dm};
+    if (!w[l].W2_f16) cb.seg[cb.n++] = ConvSeg{w[l].W2, const_cast<void*>(o.W2), dm * hdv};
     if (cb.n > kMaxConvSegs - 2 || l == n_layers - 1) {
       cudaError_t e = launch_bf16_to_f16(cb, c.s);
       if (e != cudaSuccess) return e;
@@ -460,6 +462,16 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
                        microbatch, scores, R, rows_dev, c.status, c.s);
   }
   return finish(e);
+}
+
+hstu_status hstu_bf16_to_f16(const void* src, void* dst, int64_t n, void* stream) {
+  if (n < 0 || n % 8 != 0) return HSTU_ERR_INVALID_ARG;
+  if (n == 0) return HSTU_OK;
+  if (!src || !dst || !al16(src) || !al16(dst)) return HSTU_ERR_INVALID_ARG;
+  ConvBatch cb{};
+  cb.seg[cb.n++] = ConvSeg{src, dst, n};
+  return launch_bf16_to_f16(cb, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HSTU_OK
+                                                                                  : HSTU_ERR_CUDA;
 }
 
 hstu_status hstu_read_status(const void* workspace, size_t workspace_bytes, void* stream) {

@@ -12,7 +12,10 @@ from . import binding as _b
 
 class HSTURunner:
     def __init__(self, dims: Dict[str, object], weights: Sequence[Dict[str, np.ndarray]],
-                 device="cuda"):
+                 device="cuda", f16_weights: bool = True):
+        """`f16_weights` (bf16 layers): make the fp16 copies of W1 (layers
+        >= 1) and W2 that the tensor-core path multiplies once, here, instead
+        of in every call."""
         import torch
         self.torch = torch
         self.device = torch.device(device)
@@ -24,6 +27,12 @@ class HSTURunner:
                                  int(dims["time_sub_bits"]), float(dims["ln_eps"]), self.dtype)
         self.weights = _b.weights_to_device(weights, self.dtype, self.device)
         self.n_layers = len(self.weights)
+        if f16_weights and self.dtype == "bf16":
+            for l, w in enumerate(self.weights):
+                for k in (("W1", "W2") if l > 0 else ("W2",)):
+                    w[k + "_f16"] = torch.empty(w[k].shape, dtype=torch.float16,
+                                                device=self.device)
+                    _b.hstu_bf16_to_f16(w[k], w[k + "_f16"])
         self._warr = _b.weights_array(self.weights)
         self._ws = None
 

@@ -115,6 +115,13 @@ typedef struct {
   const void* ln_beta;
   const float* rab_pos;
   const float* rab_time;
+  /* Optional, bf16 layers only: fp16 copies of W1 and W2 (same layout),
+   * e.g. made once with hstu_bf16_to_f16.  The tensor-core path multiplies
+   * the fp16 residual stream and the fp16 gated Z by fp16 weights; when these
+   * are null every call converts W1 (layers >= 1) and W2 into its workspace
+   * first.  Must be 16-byte aligned when set; ignored for fp32 layers. */
+  const void* W1_f16;
+  const void* W2_f16;
 } hstu_layer_weights;
 
 /* Bytes of device workspace an entry point needs for these sizes.
@@ -215,6 +222,11 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
  * (HSTU_ERR_BAD_OFFSETS: all out_offsets are 0; HSTU_ERR_BAD_IDS: that row is
  * zero), read back with hstu_read_status.  Asynchronous on `stream`. */
 size_t hstu_sl_embed_workspace_size(void);
+/* Round-to-nearest conversion of n bf16 values to fp16 (device to device,
+ * asynchronous on `stream`), for the optional W1_f16 / W2_f16 weight copies.
+ * n must be a multiple of 8 and both pointers 16-byte aligned. */
+hstu_status hstu_bf16_to_f16(const void* src, void* dst, int64_t n, void* stream);
+
 /* The keep count k(n) = min(n, floor(n^0.8)) (at least 1 for n >= 1) that
  * hstu_sl_embed applies to a raw stream of n tokens, computed on the host
  * with the same integer definition (the largest k with k^5 <= n^4), so a

@@ -47,9 +47,9 @@ def rmserr(g, r) -> float:
     return math.sqrt(float(np.mean((g - r) ** 2))) / rms
 
 
-def runner_for(w, device="cuda"):
+def runner_for(w, device="cuda", f16_weights=True):
     from hstu_sequential_transducer_layer_b200 import HSTURunner
-    return HSTURunner(hw.dims_dict(w.dims), w.weights, device)
+    return HSTURunner(hw.dims_dict(w.dims), w.weights, device, f16_weights=f16_weights)
 
 
 def run_stack(w, n_layers=None, runner=None):

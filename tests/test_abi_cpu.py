@@ -22,7 +22,7 @@ def built():
 def _declared():
     src = open(os.path.join(ROOT, "include", "hstu.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(hstu_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(hstu_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol():

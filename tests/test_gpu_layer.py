@@ -98,6 +98,19 @@ def test_bf16_stack_three_layers():
     assert e <= TOL[hw.BF16] and ed <= TOL[hw.BF16]
 
 
+def test_weights_converted_per_call_or_once_agree():
+    """The fp16 weight copies made once at load time (W1_f16 / W2_f16) and
+    the per-call conversion into the workspace give the same bits, and both
+    match the oracle."""
+    dims = hw.LayerDims(256, 2, 128, 128, 128, 128, 4, 2, 1e-6, hw.BF16)
+    w = hw.custom("f16w", [300, 129, 1, 64], dims, n_layers=3, seed=47)
+    Y1, _, _ = run_stack(w, runner=runner_for(w, f16_weights=True))
+    Y0, _, _ = run_stack(w, runner=runner_for(w, f16_weights=False))
+    np.testing.assert_array_equal(Y1, Y0)
+    ref = O.stack_fwd(w.X, w.offsets, w.timestamps, w.weights, dims)
+    assert relerr(Y1, ref) <= TOL[hw.BF16]
+
+
 def _sampled_rows_check(w, Y, users, rows_per_user=6, seed=0):
     rng = np.random.default_rng(seed)
     worst = 0.0
