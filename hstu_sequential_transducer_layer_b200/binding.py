@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 # Every symbol include/hstu.h declares.
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
             "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
-            "hstu_sl_keep_count", "hstu_bf16_to_f16",
+            "hstu_sl_keep_count", "hstu_bf16_to_f16", "hstu_retrieval_workspace_size",
+            "hstu_retrieval_topk",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
@@ -84,6 +85,10 @@ def lib() -> ctypes.CDLL:
     L.hstu_sl_keep_count.restype = i64
     L.hstu_bf16_to_f16.argtypes = [vp, vp, i64, vp]
     L.hstu_bf16_to_f16.restype = i32
+    L.hstu_retrieval_workspace_size.argtypes = [i64, i64, i32, i32, i32]
+    L.hstu_retrieval_workspace_size.restype = sz
+    L.hstu_retrieval_topk.argtypes = [i64, i64, i32, vp, vp, i64, vp, i32, vp, vp, vp, sz, vp]
+    L.hstu_retrieval_topk.restype = i32
     L.hstu_sl_embed.argtypes = [i64, i64, i64, vp, vp, vp, ctypes.c_uint64, vp, i64, vp, i64, i32,
                                 vp, vp, vp, vp, sz, vp]
     L.hstu_sl_embed.restype = i32
@@ -214,6 +219,28 @@ def hstu_bf16_to_f16(src, dst, stream=None) -> None:
     """fp16 copy of a bf16 device tensor (same shape) through the library."""
     _check(lib().hstu_bf16_to_f16(_ptr(src), _ptr(dst), int(src.numel()), _stream(stream)),
            "hstu_bf16_to_f16")
+
+
+def hstu_retrieval_workspace_size(n_users, n_items, d, K, from_rows=False) -> int:
+    n = lib().hstu_retrieval_workspace_size(n_users, n_items, d, K, 1 if from_rows else 0)
+    if n == 0:
+        raise HstuError(1, "hstu_retrieval_workspace_size")
+    return int(n)
+
+
+def hstu_retrieval_topk(H, E, K, out_scores, out_ids, workspace, user_offsets=None,
+                        n_users=None, stream=None) -> None:
+    """Top-K catalog items per user (see include/hstu.h).  H: bf16 [n_users, d]
+    user vectors, or with user_offsets the encoder output [rows, d]; E: bf16
+    [n_items, d]."""
+    U = int(n_users if n_users is not None else
+            (user_offsets.numel() - 1 if user_offsets is not None else H.shape[0]))
+    rows = int(H.shape[0]) if user_offsets is not None else 0
+    _check(lib().hstu_retrieval_topk(U, int(E.shape[0]), int(E.shape[1]), _ptr(H),
+                                     _ptr(user_offsets), rows, _ptr(E), int(K), _ptr(out_scores),
+                                     _ptr(out_ids), _ptr(workspace), _nbytes(workspace),
+                                     _stream(stream)),
+           "hstu_retrieval_topk")
 
 
 def hstu_sl_keep_count(n: int) -> int:

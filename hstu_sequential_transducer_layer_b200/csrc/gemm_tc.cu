@@ -1,7 +1,9 @@
 // gemm_tc.cu — GEMM on the 5th-generation tensor cores (tcgen05) with fused
-// epilogues, used for both projections of the HSTU layer:
+// epilogues, used for both projections of the HSTU layer and for catalog
+// scoring:
 //   f1:  G = SiLU(X W1^T + b1)         (EPI_SILU; output = [U | V | Q | K])
 //   f2:  Y = X + Z W2^T + b2           (EPI_RESID)
+//   scores: S = H E^T                  (EPI_SCORE; fp32, ragged item count)
 // ('HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか':
 // one projection f1 followed by SiLU and a split; f2 back to d_model plus
 // the residual connection.)
@@ -77,7 +79,9 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
       v[i * 8 + 2 * k + 1] = __uint_as_float(r[i * 8 + 2 * k + 1]) + bf16hi(bw[k]);
     }
   }
-  if (EPI == EPI_SILU) {
+  if (EPI == EPI_SCORE) {
+    if (col >= g.N) return false;  // a chunk past the last item: nothing to store
+  } else if (EPI == EPI_SILU) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
   } else if (g.resid_kind == RESID_F32) {  // residual chunk staged by TMA, 128-byte swizzle
@@ -104,7 +108,7 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
     }
   }
   if (__shfl_sync(0xffffffffu, valid ? 1 : 0, 0) == 0) return false;  // rows y0.. all invalid
-  const bool both = (EPI == EPI_RESID) && g.has_out32;
+  const bool both = ((EPI == EPI_RESID) && g.has_out32) || EPI == EPI_SCORE;
   if (both) {
     if (lane == 0) bulk_wait_read<0>();  // the warp's earlier stores have read the buffer
     __syncwarp();
@@ -120,7 +124,7 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
       bulk_commit();
     }
   }
-  if (g.has_out16) {
+  if (EPI != EPI_SCORE && g.has_out16) {
     // parity < 0: one 2 KB buffer (wait for the previous store to read it)
     uint8_t* buf = stage + ((both || parity < 0) ? 0 : parity * 2048);
     if (lane == 0) {
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     Mrows = m < Mrows ? m : Mrows;
   }
   if (Mrows < 0) Mrows = 0;
-  const int n_tiles = g.N / BN;
+  const int n_tiles = (g.N + BN - 1) / BN;  // the scores' last tile may be ragged
   const int m_tiles = (int)((Mrows + 127) / 128);
   const int tiles = m_tiles * n_tiles;
   const int KB = (g.K + 63) / 64;
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       const uint4* bptr = reinterpret_cast<const uint4*>(g.bias + col0);
       uint4 ba[4], bb[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ba[i] = __ldg(bptr + i);
+      for (int i = 0; i < 4; ++i) ba[i] = EPI == EPI_SCORE ? make_uint4(0, 0, 0, 0) : __ldg(bptr + i);
       if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) break;
       tc_fence_after();
       const int y0 = mt * 128 + q * 32;
@@ -334,8 +338,9 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
         if (c + 1 < CH) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            if (c & 1) ba[i] = __ldg(bptr + (c + 1) * 4 + i);
-            else bb[i] = __ldg(bptr + (c + 1) * 4 + i);
+            const uint4 bv = EPI == EPI_SCORE ? make_uint4(0, 0, 0, 0) : __ldg(bptr + (c + 1) * 4 + i);
+            if (c & 1) ba[i] = bv;
+            else bb[i] = bv;
           }
           if (c & 1) tmem_ld32(tbase + (c + 1) * 32, ra);
           else tmem_ld32(tbase + (c + 1) * 32, rb_acc);
@@ -487,6 +492,42 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   }
   if (BN == 128) return launch_one<128, 4, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
   return launch_one<64, 6, EPI_RESID>(ta, tb, to16, to32, tr, gd, grid, s);
+}
+
+cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_t ldw, int ab_f16,
+                               int64_t M_cap, int64_t N, int K, float* out, int64_t ldo,
+                               int* status, cudaStream_t s, int kernel_id) {
+  if (M_cap <= 0 || N <= 0) return cudaSuccess;
+  if (K % 64 != 0 || K <= 0 || ldo % 4 != 0 || ldo < N) return cudaErrorInvalidValue;
+  if (M_cap > (1ll << 31) - 256 || N > (1ll << 31) - 256) return cudaErrorInvalidValue;
+  constexpr int BN = 256;
+  CUtensorMap ta, tb, to32;
+  const bool f16 = ab_f16 != 0;
+  if (!encode_tmap_2d(&ta, A, (uint64_t)M_cap, (uint64_t)K, (uint64_t)lda * 2, 64, 128, f16))
+    return cudaErrorInvalidValue;
+  // rows past N read as zeros; the output map's extent is N, so stores past
+  // the last item are clipped
+  if (!encode_tmap_2d(&tb, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64, BN, f16))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d_ex(&to32, out, (uint64_t)M_cap, (uint64_t)N, (uint64_t)ldo * 4, 32, 32,
+                         CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  GemmDev gd{};
+  gd.M_cap = M_cap;
+  gd.M_dev = nullptr;
+  gd.N = (int)N;
+  gd.K = K;
+  gd.n_off = 0;
+  gd.ab_f16 = ab_f16;
+  gd.bias = nullptr;
+  gd.has_out16 = 0;
+  gd.has_out32 = 1;
+  gd.resid = nullptr;
+  gd.status = status;
+  const int64_t tiles = ((M_cap + 127) / 128) * ((N + BN - 1) / BN);
+  const int grid = (int)std::min<int64_t>(tiles, num_sms());
+  LaunchScope ls(kernel_id, s);
+  return launch_one<BN, 4, EPI_SCORE>(ta, tb, ta, to32, ta, gd, grid, s);
 }
 
 }  // namespace hstu

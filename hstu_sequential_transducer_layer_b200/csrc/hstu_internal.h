@@ -35,7 +35,11 @@ enum KernelId : int32_t {
   K_SL_OFFSETS = 16,
   K_SL_SELECT = 17,
   K_SL_GATHER = 18,
-  K_NUM_KERNELS = 19
+  K_RET_GATHER = 19,
+  K_GEMM_SCORES = 20,
+  K_TOPK_CHUNK = 21,
+  K_TOPK_MERGE = 22,
+  K_NUM_KERNELS = 23
 };
 const char* kernel_name(int id);
 
@@ -120,7 +124,7 @@ void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64
                      int32_t* t_rel, Header* hdr, cudaStream_t s);
 
 // C[M, N] = A[M, K] * W[n_off + N, K]^T with fused epilogue, bf16 tcgen05.
-enum Epilogue { EPI_SILU = 0, EPI_RESID = 1 };
+enum Epilogue { EPI_SILU = 0, EPI_RESID = 1, EPI_SCORE = 2 };
 enum ResidKind { RESID_BF16 = 0, RESID_F32 = 1, RESID_F16 = 2 };
 struct GemmCall {
   const void* A;  int64_t lda;   // [M_cap, K] row stride in elements
@@ -139,6 +143,12 @@ struct GemmCall {
   int* status;
 };
 cudaError_t launch_gemm_tc(const GemmCall& g, cudaStream_t s, int kernel_id);
+// scores[M_cap, N] (fp32, row stride ldo) = A[M_cap, K] * W[N, K]^T, no bias;
+// N may be ragged (the last 256-column tile is clipped); K % 64 == 0,
+// ldo % 4 == 0, bf16 or fp16 operands (ab_f16).
+cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_t ldw, int ab_f16,
+                               int64_t M_cap, int64_t N, int K, float* out, int64_t ldo,
+                               int* status, cudaStream_t s, int kernel_id);
 cudaError_t launch_gemm_simt_f32(const GemmCall& g, cudaStream_t s, int kernel_id);
 
 // Pointwise causal attention (SELF) or candidate-vs-history (CAND).

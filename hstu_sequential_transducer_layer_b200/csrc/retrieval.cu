@@ -1,0 +1,427 @@
+// retrieval.cu — full-catalog scoring with top-K selection on the device.
+//
+// The GenRec explainer on techistory.net (the equation s = E^T h and its
+// toy code): the user representation h is the encoder's hidden state at the
+// sequence's last position, every catalog item is scored at once by one
+// matrix product, and sorting the scores in descending order gives the
+// ranking ('NetflixのGenRec解説――LLMを生成させず推薦rankerとして使う', section
+// '全体像：LLMは入力を読み、ranking headが作品を採点する').  Here: the K highest
+// scores per user, equal scores ordered by ascending item id.
+//
+// Steps: k_ret_gather (optional) copies each user's last encoder row into
+// the workspace; the tcgen05 GEMM (EPI_SCORE) writes the fp32 scores
+// [U, M]; k_topk_chunk selects, per user and 8192-item chunk, the chunk's K
+// best items (radix select over order-preserving 32-bit keys held in shared
+// memory); k_topk_merge selects the K best of those candidates per user and
+// sorts them (bitonic sort of (key, id) pairs).
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace hstu {
+
+constexpr int kTopkChunk = 8192;
+constexpr int kTopkThreads = 256;
+constexpr int kTopkMaxK = 1024;
+constexpr int kMergeThreads = 1024;
+constexpr uint32_t kPadKey = 0xffffffffu;
+constexpr int32_t kPadId = 0x7fffffff;
+
+// Order-preserving key with the order reversed: a smaller key is a larger
+// score, so the top-K are the K smallest keys.  -0 is folded into +0 so that
+// equal scores compare equal.
+__device__ __forceinline__ uint32_t desc_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return ~asc;
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  const uint32_t asc = ~k;
+  return __uint_as_float((asc & 0x80000000u) ? (asc & 0x7fffffffu) : ~asc);
+}
+
+// Block-wide exclusive scan of one int per thread (NT threads).
+template <int NT>
+__device__ __forceinline__ int ret_block_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    before += w < warp ? s_warp[w] : 0;
+    all += s_warp[w];
+  }
+  *total = all;
+  return before + incl - v;
+}
+
+// One radix pass's digit choice (warp 0): among the 256 bins, the bin that
+// holds the `remaining`-th smallest key; writes the digit, the rank left
+// inside that bin and the bin's size.
+__device__ __forceinline__ void ret_pick_digit(const int* s_hist, int remaining, int* s_digit,
+                                               int* s_rem, int* s_cnt) {
+  const int lane = threadIdx.x & 31;
+  int h[8], loc = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    h[j] = s_hist[lane * 8 + j];
+    loc += h[j];
+  }
+  int incl = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, incl >= remaining);
+  const int owner = m ? __ffs(m) - 1 : 31;
+  if (lane == owner) {
+    int acc = incl - loc, dgt = lane * 8 + 7;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (acc + h[j] >= remaining) {
+        dgt = lane * 8 + j;
+        break;
+      }
+      acc += h[j];
+    }
+    *s_digit = dgt;
+    *s_rem = remaining - acc;
+    *s_cnt = s_hist[dgt];
+  }
+}
+
+// Radix select over n keys (read through key_at) of the k-th smallest, 8 bits
+// per pass from the top, stopping once the chosen bin holds exactly the keys
+// still to take.  On return *prefix holds the fixed high bits (bits >= *sh;
+// *sh = 32 when k == n: everything is taken) and *remaining how many keys
+// equal to the prefix on those bits are taken (the first ones in order).
+template <int NT, typename KeyAt>
+__device__ __forceinline__ void ret_radix_select(int n, int k, KeyAt key_at, int* s_hist,
+                                                 int* s_digit, int* s_rem, int* s_cnt,
+                                                 uint32_t* prefix, int* remaining, int* sh) {
+  const int tid = threadIdx.x;
+  uint32_t pre = 0;
+  int rem = k, s = 32;
+  if (k < n) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int i = tid; i < 256; i += NT) s_hist[i] = 0;
+      __syncthreads();
+      // scores crowd into few high-order digits (sign and exponent), so the
+      // lanes of a warp that hit the same bin add once, through their leader
+      for (int base = 0; base < n; base += NT) {
+        const int p = base + tid;
+        bool hit = false;
+        uint32_t bin = 0;
+        if (p < n) {
+          const uint32_t key = key_at(p);
+          hit = pass == 0 || (key >> s) == (pre >> s);
+          bin = (key >> shift) & 255u;
+        }
+        const unsigned active = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+          const unsigned peers = __match_any_sync(active, bin);
+          if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[bin], __popc(peers));
+        }
+      }
+      __syncthreads();
+      if (tid < 32) ret_pick_digit(s_hist, rem, s_digit, s_rem, s_cnt);
+      __syncthreads();
+      pre |= (uint32_t)*s_digit << shift;
+      rem = *s_rem;
+      s = shift;
+      const bool done = *s_cnt == rem;
+      __syncthreads();
+      if (done) break;
+    }
+  }
+  *prefix = pre;
+  *remaining = rem;
+  *sh = s;
+}
+
+// The user vectors: h_u = Y[offsets[u+1] - 1] (bf16), zero for an empty
+// user; offsets that are not monotone or pass the row count set the status.
+__global__ void __launch_bounds__(256)
+    k_ret_gather(const __nv_bfloat16* __restrict__ Y, int64_t rows, int d,
+                 const int64_t* __restrict__ off, int64_t U, __nv_bfloat16* __restrict__ Hg,
+                 int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t u = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); u < U;
+       u += warps) {
+    const int64_t a = off[u], b = off[u + 1];
+    const bool bad = a < 0 || b < a || b > rows;
+    if (bad && lane == 0) atomicCAS(status, HSTU_OK, HSTU_ERR_BAD_OFFSETS);
+    uint4* dst = reinterpret_cast<uint4*>(Hg + u * (int64_t)d);
+    if (!bad && b > a) {
+      const uint4* src = reinterpret_cast<const uint4*>(Y + (b - 1) * (int64_t)d);
+      for (int c = lane; c < d / 8; c += 32) dst[c] = __ldg(src + c);
+    } else {
+      for (int c = lane; c < d / 8; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// Per (chunk, user): the chunk's k = min(K, n) best items as (key, id)
+// candidates in item order, padded to K with (kPadKey, kPadId).
+__global__ void __launch_bounds__(kTopkThreads)
+    k_topk_chunk(const float* __restrict__ S, int64_t ldS, int64_t M, int K, int n_chunks,
+                 uint32_t* __restrict__ cand_key, int32_t* __restrict__ cand_id,
+                 const int* status) {
+  __shared__ uint32_t s_key[kTopkChunk];
+  __shared__ int s_hist[256];
+  __shared__ int s_digit, s_rem, s_cnt;
+  __shared__ int s_warp[kTopkThreads / 32];
+  if (*status != HSTU_OK) return;
+  const int tid = threadIdx.x;
+  const int chunk = blockIdx.x;
+  const int64_t u = blockIdx.y;
+  const int64_t m0 = (int64_t)chunk * kTopkChunk;
+  const int n = (int)min((int64_t)kTopkChunk, M - m0);
+  const int k = min(K, n);
+  const float* row = S + u * ldS + m0;  // 16-byte aligned: ldS % 4 == 0, m0 % 8192 == 0
+  for (int i = tid * 4; i < n; i += kTopkThreads * 4) {
+    if (i + 4 <= n) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + i));
+      s_key[i] = desc_key(v.x);
+      s_key[i + 1] = desc_key(v.y);
+      s_key[i + 2] = desc_key(v.z);
+      s_key[i + 3] = desc_key(v.w);
+    } else {
+      for (int j = i; j < n; ++j) s_key[j] = desc_key(__ldg(row + j));
+    }
+  }
+  __syncthreads();
+  uint32_t prefix;
+  int remaining, sh;
+  ret_radix_select<kTopkThreads>(n, k, [&](int p) { return s_key[p]; }, s_hist, &s_digit, &s_rem,
+                                 &s_cnt, &prefix, &remaining, &sh);
+  // ordered compaction: thread t owns positions 32t .. 32t+31 (read rotated
+  // by t, so a warp's lanes hit distinct banks), one packed scan
+  const uint32_t ph = sh == 32 ? 0u : prefix >> sh;
+  const int p0 = tid * 32;
+  uint32_t lt = 0, eq = 0;
+#pragma unroll 8
+  for (int j = 0; j < 32; ++j) {
+    const int jj = (j + tid) & 31;
+    const int p = p0 + jj;
+    if (p < n) {
+      if (sh == 32) {
+        lt |= 1u << jj;
+      } else {
+        const uint32_t hi = s_key[p] >> sh;
+        lt |= (uint32_t)(hi < ph) << jj;
+        eq |= (uint32_t)(hi == ph) << jj;
+      }
+    }
+  }
+  int tot;
+  const int pre = ret_block_scan<kTopkThreads>((__popc(lt) << 16) | __popc(eq), s_warp, &tot);
+  int c_lt = pre >> 16, c_eq = pre & 0xffff;
+  uint32_t* ck = cand_key + (u * n_chunks + chunk) * (int64_t)K;
+  int32_t* ci = cand_id + (u * n_chunks + chunk) * (int64_t)K;
+  for (int jj = 0; jj < 32; ++jj) {
+    const bool l = (lt >> jj) & 1u, e = (eq >> jj) & 1u;
+    if (l || (e && c_eq < remaining)) {
+      const int idx = c_lt + min(c_eq, remaining);
+      ck[idx] = s_key[p0 + jj];
+      ci[idx] = (int32_t)(m0 + p0 + jj);
+    }
+    c_lt += l;
+    c_eq += e;
+  }
+  for (int i = k + tid; i < K; i += kTopkThreads) {
+    ck[i] = kPadKey;
+    ci[i] = kPadId;
+  }
+}
+
+// Per user: the K best of its n_cand candidates (item order = id order, so
+// equal keys are taken lowest id first), sorted by (key, id).
+__global__ void __launch_bounds__(kMergeThreads)
+    k_topk_merge(const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_id,
+                 int n_cand, int K, float* __restrict__ out_scores, int64_t* __restrict__ out_ids,
+                 const int* status) {
+  __shared__ int s_hist[256];
+  __shared__ int s_digit, s_rem, s_cnt;
+  __shared__ int s_warp[kMergeThreads / 32];
+  __shared__ uint32_t s_k[kTopkMaxK];
+  __shared__ int32_t s_i[kTopkMaxK];
+  if (*status != HSTU_OK) return;
+  const int tid = threadIdx.x;
+  const int64_t u = blockIdx.x;
+  const uint32_t* keys = cand_key + u * (int64_t)n_cand;
+  const int32_t* ids = cand_id + u * (int64_t)n_cand;
+  uint32_t prefix;
+  int remaining, sh;
+  ret_radix_select<kMergeThreads>(n_cand, K, [&](int p) { return __ldg(keys + p); }, s_hist,
+                                  &s_digit, &s_rem, &s_cnt, &prefix, &remaining, &sh);
+  const uint32_t ph = sh == 32 ? 0u : prefix >> sh;
+  int run_lt = 0, run_eq = 0;
+  for (int base = 0; base < n_cand; base += kMergeThreads * 4) {
+    const int p0 = base + tid * 4;
+    unsigned lt = 0, eq = 0;
+    uint32_t kk[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int p = p0 + j;
+      kk[j] = p < n_cand ? __ldg(keys + p) : kPadKey;
+      if (p < n_cand) {
+        if (sh == 32) {
+          lt |= 1u << j;
+        } else {
+          const uint32_t hi = kk[j] >> sh;
+          lt |= (unsigned)(hi < ph) << j;
+          eq |= (unsigned)(hi == ph) << j;
+        }
+      }
+    }
+    int tot;
+    const int pre = ret_block_scan<kMergeThreads>((__popc(lt) << 16) | __popc(eq), s_warp, &tot);
+    int c_lt = run_lt + (pre >> 16), c_eq = run_eq + (pre & 0xffff);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool l = (lt >> j) & 1u, e = (eq >> j) & 1u;
+      if (l || (e && c_eq < remaining)) {
+        const int idx = c_lt + min(c_eq, remaining);
+        s_k[idx] = kk[j];
+        s_i[idx] = __ldg(ids + p0 + j);
+      }
+      c_lt += l;
+      c_eq += e;
+    }
+    run_lt += tot >> 16;
+    run_eq += tot & 0xffff;
+  }
+  // bitonic sort of the K selected pairs, padded to a power of two
+  int P = 1;
+  while (P < K) P <<= 1;
+  for (int i = K + tid; i < P; i += kMergeThreads) {
+    s_k[i] = kPadKey;
+    s_i[i] = kPadId;
+  }
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < P; i += kMergeThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const uint32_t ki = s_k[i], kj = s_k[j];
+          const int32_t ii = s_i[i], ij = s_i[j];
+          const bool gt = ki > kj || (ki == kj && ii > ij);  // (key, id) of i after j's
+          if (gt == up) {
+            s_k[i] = kj;
+            s_k[j] = ki;
+            s_i[i] = ij;
+            s_i[j] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < K; i += kMergeThreads) {
+    out_scores[u * K + i] = key_score(s_k[i]);
+    out_ids[u * K + i] = s_i[i];
+  }
+}
+
+struct RetLayout {
+  size_t hg, scores, ckey, cid, total;
+  int64_t ldS;
+  int n_chunks;
+};
+
+static bool ret_layout(int64_t U, int64_t M, int32_t d, int32_t K, bool gather, RetLayout* L) {
+  if (U < 0 || U > 65535 || M < 1 || M > (1ll << 31) - 256 || d < 64 || d % 64 != 0 || K < 1 ||
+      K > kTopkMaxK || K > M)
+    return false;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  L->ldS = (M + 63) / 64 * 64;
+  L->n_chunks = (int)((M + kTopkChunk - 1) / kTopkChunk);
+  size_t o = 256;  // status word
+  L->hg = o;
+  o += up(gather ? (size_t)U * d * 2 : 0);
+  L->scores = o;
+  o += up((size_t)U * L->ldS * 4);
+  L->ckey = o;
+  o += up((size_t)U * L->n_chunks * K * 4);
+  L->cid = o;
+  o += up((size_t)U * L->n_chunks * K * 4);
+  L->total = o;
+  return (int64_t)L->n_chunks * K <= (1ll << 30);
+}
+
+}  // namespace hstu
+
+// ---------------------------------------------------------------- C ABI
+extern "C" {
+
+size_t hstu_retrieval_workspace_size(int64_t U, int64_t M, int32_t d, int32_t K,
+                                     int32_t from_rows) {
+  hstu::RetLayout L;
+  return hstu::ret_layout(U, M, d, K, from_rows != 0, &L) ? L.total : 0;
+}
+
+hstu_status hstu_retrieval_topk(int64_t U, int64_t M, int32_t d, const void* H,
+                                const int64_t* user_offsets, int64_t total_rows, const void* E,
+                                int32_t K, float* out_scores, int64_t* out_ids, void* ws,
+                                size_t ws_bytes, void* stream_ptr) {
+  using namespace hstu;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const bool gather = user_offsets != nullptr;
+  RetLayout L;
+  if (!ret_layout(U, M, d, K, gather, &L)) return HSTU_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HSTU_ERR_WORKSPACE;
+  if (U == 0) return HSTU_OK;
+  if (!H || !E || !out_scores || !out_ids) return HSTU_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(H) & 15) || (reinterpret_cast<uintptr_t>(E) & 15))
+    return HSTU_ERR_INVALID_ARG;
+  if (gather && total_rows < 0) return HSTU_ERR_INVALID_ARG;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  const void* A = H;
+  if (gather) {
+    LaunchScope ls(K_RET_GATHER, stream);
+    const int grid = (int)std::min<int64_t>((U + 7) / 8, 4 * num_sms());
+    k_ret_gather<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(H), total_rows, d,
+                                           user_offsets, U,
+                                           reinterpret_cast<__nv_bfloat16*>(w + L.hg), status);
+    if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+    A = w + L.hg;
+  }
+  float* S = reinterpret_cast<float*>(w + L.scores);
+  if (launch_gemm_scores(A, d, E, d, 0, U, M, d, S, L.ldS, status, stream, K_GEMM_SCORES) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  uint32_t* ck = reinterpret_cast<uint32_t*>(w + L.ckey);
+  int32_t* ci = reinterpret_cast<int32_t*>(w + L.cid);
+  {
+    LaunchScope ls(K_TOPK_CHUNK, stream);
+    k_topk_chunk<<<dim3((unsigned)L.n_chunks, (unsigned)U), kTopkThreads, 0, stream>>>(
+        S, L.ldS, M, K, L.n_chunks, ck, ci, status);
+    if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  }
+  {
+    LaunchScope ls(K_TOPK_MERGE, stream);
+    k_topk_merge<<<(unsigned)U, kMergeThreads, 0, stream>>>(ck, ci, L.n_chunks * K, K, out_scores,
+                                                           out_ids, status);
+    if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  }
+  return HSTU_OK;
+}
+
+}  // extern "C"

@@ -24,7 +24,8 @@ const char* kernel_name(int id) {
       "ln_gate",    "gemm_f2_tc", "mb_plan",         "mb_gather",
       "attn_cand_tc", "score",    "gemm_f1_simt_f32", "attn_simt_f32",
       "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16", "time_buckets",
-      "sl_offsets", "sl_select", "sl_gather"};
+      "sl_offsets", "sl_select", "sl_gather", "ret_gather", "gemm_scores_tc", "topk_chunk",
+      "topk_merge"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 

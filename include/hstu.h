@@ -222,6 +222,33 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
  * (HSTU_ERR_BAD_OFFSETS: all out_offsets are 0; HSTU_ERR_BAD_IDS: that row is
  * zero), read back with hstu_read_status.  Asynchronous on `stream`. */
 size_t hstu_sl_embed_workspace_size(void);
+/* Full-catalog retrieval ('NetflixのGenRec解説――LLMを生成させず推薦rankerとして使う',
+ * section '全体像：LLMは入力を読み、ranking headが作品を採点する'; the GenRec
+ * explainer on techistory.net, s = E^T h): every one of n_items catalog
+ * items is scored against every user vector, s[u, m] = <E_m, h_u>, in fp32
+ * on the tensor cores, and the K highest scores per user are returned in
+ * descending order, equal scores ordered by ascending item id.
+ *   H             device bf16: the user vectors [n_users, d], or, when
+ *                 user_offsets is given, the encoder output [total_rows, d]
+ *                 whose row user_offsets[u+1]-1 is user u's vector (a user
+ *                 without rows scores every item 0)
+ *   user_offsets  device int64 [n_users+1] or null
+ *   E             device bf16 [n_items, d] item embeddings
+ *   out_scores    device fp32 [n_users, K]; out_ids device int64 [n_users, K]
+ *   workspace     hstu_retrieval_workspace_size(...) bytes, 256-byte aligned
+ *                 (from_rows = 1 when user_offsets will be given); it holds
+ *                 the status word and the [n_users, n_items] score matrix
+ * Requires d % 64 == 0, 1 <= K <= min(n_items, 1024), n_users <= 65535,
+ * n_items < 2^31 - 256, H and E 16-byte aligned.  Offsets that are not
+ * monotone or pass total_rows set HSTU_ERR_BAD_OFFSETS in the status word
+ * (outputs then unspecified).  Asynchronous on `stream`. */
+size_t hstu_retrieval_workspace_size(int64_t n_users, int64_t n_items, int32_t d, int32_t K,
+                                     int32_t from_rows);
+hstu_status hstu_retrieval_topk(int64_t n_users, int64_t n_items, int32_t d, const void* H,
+                                const int64_t* user_offsets, int64_t total_rows, const void* E,
+                                int32_t K, float* out_scores, int64_t* out_ids, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* Round-to-nearest conversion of n bf16 values to fp16 (device to device,
  * asynchronous on `stream`), for the optional W1_f16 / W2_f16 weight copies.
  * n must be a multiple of 8 and both pointers 16-byte aligned. */
