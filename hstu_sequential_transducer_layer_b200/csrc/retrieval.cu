@@ -117,22 +117,9 @@ __device__ __forceinline__ void ret_radix_select(int n, int k, KeyAt key_at, int
       const int shift = 24 - 8 * pass;
       for (int i = tid; i < 256; i += NT) s_hist[i] = 0;
       __syncthreads();
-      // scores crowd into few high-order digits (sign and exponent), so the
-      // lanes of a warp that hit the same bin add once, through their leader
-      for (int base = 0; base < n; base += NT) {
-        const int p = base + tid;
-        bool hit = false;
-        uint32_t bin = 0;
-        if (p < n) {
-          const uint32_t key = key_at(p);
-          hit = pass == 0 || (key >> s) == (pre >> s);
-          bin = (key >> shift) & 255u;
-        }
-        const unsigned active = __ballot_sync(0xffffffffu, hit);
-        if (hit) {
-          const unsigned peers = __match_any_sync(active, bin);
-          if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[bin], __popc(peers));
-        }
+      for (int p = tid; p < n; p += NT) {
+        const uint32_t key = key_at(p);
+        if (pass == 0 || (key >> s) == (pre >> s)) atomicAdd(&s_hist[(key >> shift) & 255u], 1);
       }
       __syncthreads();
       if (tid < 32) ret_pick_digit(s_hist, rem, s_digit, s_rem, s_cnt);
@@ -173,13 +160,59 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Ordered compaction of `count` entries (entry j's key through key_at):
+// entries whose fixed high bits are below the prefix, or equal to it and
+// among the first `remaining` such, are passed in order to emit(idx, j).
+// Each thread owns a run of consecutive entries (at most 32).
+template <int NT, typename KeyAt, typename Emit>
+__device__ __forceinline__ void ret_ordered_emit(int count, uint32_t prefix, int remaining, int sh,
+                                                 KeyAt key_at, Emit emit, int* s_warp) {
+  const int per = (count + NT - 1) / NT;  // <= 32
+  const int j0 = threadIdx.x * per;
+  const uint32_t ph = sh == 32 ? 0u : prefix >> sh;
+  uint32_t lt = 0, eq = 0;
+  for (int tt = 0; tt < per; ++tt) {
+    // runs of 32: rotated by the thread index so a warp's lanes hit distinct
+    // shared-memory banks (the bitmasks make the visiting order irrelevant)
+    const int t = per == 32 ? ((tt + (int)threadIdx.x) & 31) : tt;
+    const int j = j0 + t;
+    if (j < count) {
+      if (sh == 32) {
+        lt |= 1u << t;
+      } else {
+        const uint32_t hi = key_at(j) >> sh;
+        lt |= (uint32_t)(hi < ph) << t;
+        eq |= (uint32_t)(hi == ph) << t;
+      }
+    }
+  }
+  int tot;
+  const int pre = ret_block_scan<NT>((__popc(lt) << 16) | __popc(eq), s_warp, &tot);
+  int c_lt = pre >> 16, c_eq = pre & 0xffff;
+  for (int t = 0; t < per; ++t) {
+    const bool l = (lt >> t) & 1u, e = (eq >> t) & 1u;
+    if (l || (e && c_eq < remaining)) emit(c_lt + min(c_eq, remaining), j0 + t);
+    c_lt += l;
+    c_eq += e;
+  }
+}
+
 // Per (chunk, user): the chunk's k = min(K, n) best items as (key, id)
 // candidates in item order, padded to K with (kPadKey, kPadId).
+// The k best lie among the positions at least as good as a threshold taken
+// from a 1-in-16 sample of the chunk (its ks-th best, ks ~ 2K/16 + 8): at
+// least ks sample keys pass it, so when k or more positions pass, they hold
+// the k best.  Only those candidates (a few hundred) go through the exact
+// radix select; with fewer than k, or more than fit, every position does.
+constexpr int kSampleStride = 16;
+constexpr int kCandCap = 4096;
+
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk_chunk(const float* __restrict__ S, int64_t ldS, int64_t M, int K, int n_chunks,
                  uint32_t* __restrict__ cand_key, int32_t* __restrict__ cand_id,
                  const int* status) {
   __shared__ uint32_t s_key[kTopkChunk];
+  __shared__ uint16_t s_pos[kCandCap];
   __shared__ int s_hist[256];
   __shared__ int s_digit, s_rem, s_cnt;
   __shared__ int s_warp[kTopkThreads / 32];
@@ -205,42 +238,48 @@ __global__ void __launch_bounds__(kTopkThreads)
   __syncthreads();
   uint32_t prefix;
   int remaining, sh;
-  ret_radix_select<kTopkThreads>(n, k, [&](int p) { return s_key[p]; }, s_hist, &s_digit, &s_rem,
-                                 &s_cnt, &prefix, &remaining, &sh);
-  // ordered compaction: thread t owns positions 32t .. 32t+31 (read rotated
-  // by t, so a warp's lanes hit distinct banks), one packed scan
-  const uint32_t ph = sh == 32 ? 0u : prefix >> sh;
-  const int p0 = tid * 32;
-  uint32_t lt = 0, eq = 0;
+  // ---- candidates: positions at least as good as the sample threshold
+  int n_cand = n;  // n_cand == n: every position (no filtering)
+  const int ns = (n + kSampleStride - 1) / kSampleStride;
+  const int ks = 2 * ((K + kSampleStride - 1) / kSampleStride) + 8;
+  if (k < n && ks < ns) {
+    ret_radix_select<kTopkThreads>(ns, ks, [&](int i) { return s_key[i * kSampleStride]; },
+                                   s_hist, &s_digit, &s_rem, &s_cnt, &prefix, &remaining, &sh);
+    // every key whose fixed high bits are <= the prefix's: >= ks sample keys
+    const uint32_t thr = prefix | (uint32_t)((1ull << sh) - 1);
+    // count and place the passing positions in order (one run of 32 per thread)
+    const int p0 = tid * 32;
+    uint32_t pass = 0;
 #pragma unroll 8
-  for (int j = 0; j < 32; ++j) {
-    const int jj = (j + tid) & 31;
-    const int p = p0 + jj;
-    if (p < n) {
-      if (sh == 32) {
-        lt |= 1u << jj;
-      } else {
-        const uint32_t hi = s_key[p] >> sh;
-        lt |= (uint32_t)(hi < ph) << jj;
-        eq |= (uint32_t)(hi == ph) << jj;
-      }
+    for (int j = 0; j < 32; ++j) {
+      const int jj = (j + tid) & 31;  // rotated: a warp's lanes hit distinct banks
+      const int p = p0 + jj;
+      if (p < n && s_key[p] <= thr) pass |= 1u << jj;
     }
+    int tot;
+    const int pre = ret_block_scan<kTopkThreads>(__popc(pass), s_warp, &tot);
+    if (tot >= k && tot <= kCandCap) {
+      int idx = pre;
+      for (int jj = 0; jj < 32; ++jj)
+        if ((pass >> jj) & 1u) s_pos[idx++] = (uint16_t)(p0 + jj);
+      n_cand = tot;
+    }
+    __syncthreads();
   }
-  int tot;
-  const int pre = ret_block_scan<kTopkThreads>((__popc(lt) << 16) | __popc(eq), s_warp, &tot);
-  int c_lt = pre >> 16, c_eq = pre & 0xffff;
+  const bool filtered = n_cand < n;
+  auto cand_key_at = [&](int j) -> uint32_t { return s_key[filtered ? s_pos[j] : j]; };
+  ret_radix_select<kTopkThreads>(n_cand, k, cand_key_at, s_hist, &s_digit, &s_rem, &s_cnt,
+                                 &prefix, &remaining, &sh);
   uint32_t* ck = cand_key + (u * n_chunks + chunk) * (int64_t)K;
   int32_t* ci = cand_id + (u * n_chunks + chunk) * (int64_t)K;
-  for (int jj = 0; jj < 32; ++jj) {
-    const bool l = (lt >> jj) & 1u, e = (eq >> jj) & 1u;
-    if (l || (e && c_eq < remaining)) {
-      const int idx = c_lt + min(c_eq, remaining);
-      ck[idx] = s_key[p0 + jj];
-      ci[idx] = (int32_t)(m0 + p0 + jj);
-    }
-    c_lt += l;
-    c_eq += e;
-  }
+  ret_ordered_emit<kTopkThreads>(
+      n_cand, prefix, remaining, sh, cand_key_at,
+      [&](int idx, int j) {
+        const int p = filtered ? s_pos[j] : j;
+        ck[idx] = s_key[p];
+        ci[idx] = (int32_t)(m0 + p);
+      },
+      s_warp);
   for (int i = k + tid; i < K; i += kTopkThreads) {
     ck[i] = kPadKey;
     ci[i] = kPadId;
