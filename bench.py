@@ -12,7 +12,8 @@ way and reported in the same line under "mfalcon"; Stochastic Length sampling
 table) under "stochastic_length", and those raw streams through Stochastic
 Length, embedding and the 8-layer stack under "full_pipeline"; the stack
 output's last row per user scored against the 1M-item catalog with top-100
-selection under "retrieval".
+selection under "retrieval"; one HSTU layer against one softmax-Transformer
+layer on the long-history workload under "comparator".
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream with a 256 MB L2 flush between steps (outside the
@@ -606,6 +607,63 @@ def run_ours(args):
                "config": {"workload": "full_stack output x 1M-item catalog", "users": r_U,
                           "items": r_M, "d_model": r_d, "K": r_K}}
 
+    # ---------------- the softmax-Transformer comparator: one HSTU layer and one
+    # pre-LN Transformer layer (d_ff = 2048) on the long-history workload
+    # (16 users of 2,048-8,192 tokens, d = 512, 8 heads, head dim 64)
+    cmp_ = None
+    if not args.no_comparator:
+        wl = hw.long_history(seed=args.seed + rank)
+        rh = H.HSTURunner(hw.dims_dict(wl.dims), wl.weights, dev)
+        c_off = rh.to_device(wl.offsets, "i64")
+        c_x = rh.to_device(wl.X, "act")
+        c_ts = rh.to_device(wl.timestamps, "i64")
+        c_yh = torch.empty_like(c_x)
+        c_yt = torch.empty_like(c_x)
+        rt = H.TransformerRunner(512, 8, 2048, hw.transformer_weights(args.seed + rank, 512, 2048),
+                                 device=dev)
+
+        def time_leg(fn):
+            for _ in range(args.warmup):
+                fn()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            H.hstu_trace_enable(args.steps * 16 + 16)
+            for _ in range(args.steps):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            tr = H.hstu_trace_read()
+            H.hstu_trace_enable(0)
+            ker = {}
+            for kid, t in tr:
+                e = ker.setdefault(H.hstu_kernel_name(kid), [0, 0.0])
+                e[0] += 1
+                e[1] += t
+            return (sum(a.elapsed_time(b) for a, b in evs) / len(evs),
+                    {k: round(v[1] / v[0], 4) for k, v in ker.items()})
+        h_ms, h_k = time_leg(lambda: rh.stack(c_off, c_x, c_ts, wl.max_len, out=c_yh))
+        t_ms, t_k = time_leg(lambda: rt.layer(c_off, c_x, wl.max_len, out=c_yt))
+        if rh.status() != 0 or rt.status() != 0:
+            raise RuntimeError(f"comparator device status {rh.status()} / {rt.status()}")
+        pairs = float((wl.lengths * (wl.lengths + 1) // 2).sum())
+        attn_flops = 4.0 * 64 * 8 * pairs   # Q.K and P.V, 2 flops per multiply-add
+        sa_ms = t_k.get("tf_softmax_attn_tc", float("nan"))
+        cmp_ = {"workload": "long_history (16 users, 2048-8192 tokens, d=512, 8 heads, dh=64)",
+                "tokens": wl.T, "hstu_layer_ms": round(h_ms, 4),
+                "transformer_layer_ms": round(t_ms, 4),
+                "hstu_speedup": round(t_ms / h_ms, 3),
+                "hstu_kernels_ms": h_k, "transformer_kernels_ms": t_k,
+                "softmax_attention_tflops": round(attn_flops / (sa_ms / 1e3) / 1e12, 1),
+                "hstu_attention_tflops": round(attn_flops / (h_k.get("attn_tc", float("nan")) / 1e3)
+                                               / 1e12, 1),
+                "note": "one layer each; the Transformer layer has an FFN (4d) and no rab"}
+
     # ---------------- reduce over ranks
     tokens = float(T)
     if world > 1:
@@ -673,6 +731,7 @@ def run_ours(args):
             "stochastic_length": sl,
             "full_pipeline": pipe,
             "retrieval": ret,
+            "comparator": cmp_,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -720,6 +779,7 @@ def main():
     ap.add_argument("--no-mfalcon", action="store_true")
     ap.add_argument("--no-sl", action="store_true")
     ap.add_argument("--no-retrieval", action="store_true")
+    ap.add_argument("--no-comparator", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)

@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
             "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
             "hstu_sl_keep_count", "hstu_bf16_to_f16", "hstu_retrieval_workspace_size",
-            "hstu_retrieval_topk",
+            "hstu_retrieval_topk", "hstu_transformer_workspace_size",
+            "hstu_transformer_layer_fwd",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
@@ -51,6 +52,11 @@ class LayerWeights(ctypes.Structure):
                 ("ln_beta", ctypes.c_void_p), ("rab_pos", ctypes.c_void_p),
                 ("rab_time", ctypes.c_void_p), ("W1_f16", ctypes.c_void_p),
                 ("W2_f16", ctypes.c_void_p)]
+
+
+class TransformerWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("ln1_gamma", "ln1_beta", "W_qkv", "W_o", "ln2_gamma",
+                                               "ln2_beta", "W_1", "b_1", "W_2", "b_2")]
 
 
 _lib = None
@@ -89,6 +95,12 @@ def lib() -> ctypes.CDLL:
     L.hstu_retrieval_workspace_size.restype = sz
     L.hstu_retrieval_topk.argtypes = [i64, i64, i32, vp, vp, i64, vp, i32, vp, vp, vp, sz, vp]
     L.hstu_retrieval_topk.restype = i32
+    L.hstu_transformer_workspace_size.argtypes = [i32, i32, i32, i64, i64]
+    L.hstu_transformer_workspace_size.restype = sz
+    L.hstu_transformer_layer_fwd.argtypes = [i32, i32, i32, ctypes.c_float,
+                                             ctypes.POINTER(TransformerWeights), i64, i64, i64, vp,
+                                             vp, vp, vp, sz, vp]
+    L.hstu_transformer_layer_fwd.restype = i32
     L.hstu_sl_embed.argtypes = [i64, i64, i64, vp, vp, vp, ctypes.c_uint64, vp, i64, vp, i64, i32,
                                 vp, vp, vp, vp, sz, vp]
     L.hstu_sl_embed.restype = i32
@@ -241,6 +253,26 @@ def hstu_retrieval_topk(H, E, K, out_scores, out_ids, workspace, user_offsets=No
                                      _ptr(out_ids), _ptr(workspace), _nbytes(workspace),
                                      _stream(stream)),
            "hstu_retrieval_topk")
+
+
+def hstu_transformer_workspace_size(d_model, n_heads, d_ff, B, total_tokens) -> int:
+    n = lib().hstu_transformer_workspace_size(d_model, n_heads, d_ff, B, total_tokens)
+    if n == 0:
+        raise HstuError(1, "hstu_transformer_workspace_size")
+    return int(n)
+
+
+def hstu_transformer_layer_fwd(d_model, n_heads, d_ff, ln_eps, weights, B, total_tokens, max_len,
+                               offsets, X, out, workspace, stream=None) -> None:
+    """The softmax-Transformer comparator layer (see include/hstu.h); `weights`
+    is a TransformerWeights struct or a dict of device tensors."""
+    if not isinstance(weights, TransformerWeights):
+        weights = TransformerWeights(*[_ptr(weights[k]) for k, _ in TransformerWeights._fields_])
+    _check(lib().hstu_transformer_layer_fwd(d_model, n_heads, d_ff, float(ln_eps),
+                                            ctypes.byref(weights), B, total_tokens, max_len,
+                                            _ptr(offsets), _ptr(X), _ptr(out), _ptr(workspace),
+                                            _nbytes(workspace), _stream(stream)),
+           "hstu_transformer_layer_fwd")
 
 
 def hstu_sl_keep_count(n: int) -> int:

@@ -4,6 +4,7 @@
 //   f1:  G = SiLU(X W1^T + b1)         (EPI_SILU; output = [U | V | Q | K])
 //   f2:  Y = X + Z W2^T + b2           (EPI_RESID)
 //   scores: S = H E^T                  (EPI_SCORE; fp32, ragged item count)
+//   plain:  C = A W^T + b              (EPI_BIAS; 16-bit output)
 // ('HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか':
 // one projection f1 followed by SiLU and a split; f2 back to d_model plus
 // the residual connection.)
@@ -84,6 +85,8 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   } else if (EPI == EPI_SILU) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
+  } else if (EPI == EPI_BIAS) {
+    // bias only
   } else if (g.resid_kind == RESID_F32) {  // residual chunk staged by TMA, 128-byte swizzle
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -483,6 +486,11 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
     if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
     if (BN == 128) return launch_one<128, 6, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
     return launch_one<64, 8, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);
+  }
+  if (c.epi == EPI_BIAS) {
+    if (BN == 256) return launch_one<256, 4, EPI_BIAS>(ta, tb, to16, to32, tr, gd, grid, s);
+    if (BN == 128) return launch_one<128, 6, EPI_BIAS>(ta, tb, to16, to32, tr, gd, grid, s);
+    return launch_one<64, 8, EPI_BIAS>(ta, tb, to16, to32, tr, gd, grid, s);
   }
   // the residual buffers take one A/B stage's worth of shared memory
   if (BN == 256) {

@@ -39,7 +39,13 @@ enum KernelId : int32_t {
   K_GEMM_SCORES = 20,
   K_TOPK_CHUNK = 21,
   K_TOPK_MERGE = 22,
-  K_NUM_KERNELS = 23
+  K_TF_LN = 23,
+  K_TF_QKV = 24,
+  K_TF_ATTN = 25,
+  K_TF_OPROJ = 26,
+  K_TF_FFN1 = 27,
+  K_TF_FFN2 = 28,
+  K_NUM_KERNELS = 29
 };
 const char* kernel_name(int id);
 
@@ -124,7 +130,7 @@ void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64
                      int32_t* t_rel, Header* hdr, cudaStream_t s);
 
 // C[M, N] = A[M, K] * W[n_off + N, K]^T with fused epilogue, bf16 tcgen05.
-enum Epilogue { EPI_SILU = 0, EPI_RESID = 1, EPI_SCORE = 2 };
+enum Epilogue { EPI_SILU = 0, EPI_RESID = 1, EPI_SCORE = 2, EPI_BIAS = 3 };
 enum ResidKind { RESID_BF16 = 0, RESID_F32 = 1, RESID_F16 = 2 };
 struct GemmCall {
   const void* A;  int64_t lda;   // [M_cap, K] row stride in elements

@@ -142,3 +142,41 @@ class HSTURunner:
         def view(off, cols, dt, size):
             return ws[off:off + T * cols * size].view(dt).view(T, cols)
         return view(f1o, F, idt, es), view(oo, hdv, t.float32, 4), view(zo, hdv, idt, es)
+
+
+class TransformerRunner:
+    """Device weights and a workspace for the softmax-Transformer comparator
+    layer (hstu_transformer_layer_fwd).  Dense weights go to the device as
+    fp16, LayerNorm parameters and biases as bf16."""
+
+    DENSE = ("W_qkv", "W_o", "W_1", "W_2")
+
+    def __init__(self, d_model: int, n_heads: int, d_ff: int, weights: Dict[str, np.ndarray],
+                 ln_eps: float = 1e-6, device="cuda"):
+        import torch
+        self.torch = torch
+        self.device = torch.device(device)
+        self.d, self.h, self.ff, self.eps = int(d_model), int(n_heads), int(d_ff), float(ln_eps)
+        self.w = {}
+        for k, v in weights.items():
+            dt = torch.float16 if k in self.DENSE else torch.bfloat16
+            self.w[k] = torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(self.device, dt)
+        self._struct = _b.TransformerWeights(*[_b._ptr(self.w[k]) for k, _ in
+                                               _b.TransformerWeights._fields_])
+        self._ws = None
+
+    def layer(self, offsets, X, max_len: int, out=None, stream=None):
+        t = self.torch
+        B = offsets.numel() - 1
+        T = X.shape[0]
+        if out is None:
+            out = t.empty_like(X)
+        nb = _b.hstu_transformer_workspace_size(self.d, self.h, self.ff, B, T)
+        if self._ws is None or self._ws.numel() < nb:
+            self._ws = t.empty(nb, dtype=t.uint8, device=self.device)
+        _b.hstu_transformer_layer_fwd(self.d, self.h, self.ff, self.eps, self._struct, B, T,
+                                      max_len, offsets, X, out, self._ws, stream)
+        return out
+
+    def status(self, stream=None) -> int:
+        return _b.hstu_read_status(self._ws, stream)

@@ -439,6 +439,28 @@ def device_embedding_table(seed: int, table: int, rows: int, d: int, device):
     return torch.randn(rows, d, generator=g, device=device, dtype=torch.bfloat16)
 
 
+def round_to_f16(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest fp16 (ties to even); returns float32."""
+    return np.asarray(a, np.float32).astype(np.float16).astype(np.float32)
+
+
+def transformer_weights(seed: int, d: int, d_ff: int) -> Dict[str, np.ndarray]:
+    """Weights of the softmax-Transformer comparator layer: dense weights
+    N(0, 1/fan_in) rounded to fp16 (W_qkv [3d, d], W_o [d, d], W_1 [d_ff, d],
+    W_2 [d, d_ff]); LayerNorm gamma = 1 + N(0, 0.02), beta and biases
+    N(0, 0.02), rounded to bf16."""
+    rng = np.random.default_rng([seed, 512, d, d_ff])
+
+    def dense(o, i):
+        return round_to_f16(rng.normal(0.0, 1.0 / math.sqrt(i), size=(o, i)).astype(np.float32))
+
+    def small(n, base=0.0):
+        return round_to_bf16((base + rng.normal(0.0, 0.02, size=n)).astype(np.float32))
+    return dict(ln1_gamma=small(d, 1.0), ln1_beta=small(d), W_qkv=dense(3 * d, d),
+                W_o=dense(d, d), ln2_gamma=small(d, 1.0), ln2_beta=small(d), W_1=dense(d_ff, d),
+                b_1=small(d_ff), W_2=dense(d, d_ff), b_2=small(d))
+
+
 WORKLOADS = {
     "tiny_fp32": tiny_fp32,
     "single_layer": single_layer,

@@ -249,6 +249,39 @@ hstu_status hstu_retrieval_topk(int64_t n_users, int64_t n_items, int32_t d, con
                                 int32_t K, float* out_scores, int64_t* out_ids, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Softmax-Transformer encoder layer: the comparator of the HSTU layer on the
+ * same jagged batches ('HSTUとGenerative Recommenders', section 'Production評価の
+ * 12.4%をどう読むか': HSTU against a FlashAttention-2 Transformer at 8,192
+ * tokens, d = 512, 8 heads; attention as in the GenRec explainer on
+ * techistory.net, softmax(QK^T / sqrt(d_k)) V).  Pre-LayerNorm, causal per
+ * user:  A = LN1(X); [Q|K|V] = A W_qkv^T; ctx = per-head causal softmax
+ * attention; X1 = X + ctx W_o^T; Y = X1 + SiLU(LN2(X1) W_1^T + b_1) W_2^T + b_2.
+ * Dense weights are fp16 ([out, in] row-major: W_qkv [3d, d] with Q, K, V
+ * row blocks, W_o [d, d], W_1 [d_ff, d], W_2 [d, d_ff]); LayerNorm gamma/beta
+ * and the biases are bf16.  X and out are bf16 [T, d]; intermediates fp16.
+ * Requires d % 256 == 0, d <= 1024, head dim d/h of 64 or 128, d_ff % 256 == 0;
+ * every pointer 16-byte aligned.  Offsets are checked on the device
+ * (HSTU_ERR_BAD_OFFSETS in the status word). */
+typedef struct {
+  const void* ln1_gamma;
+  const void* ln1_beta;
+  const void* W_qkv;
+  const void* W_o;
+  const void* ln2_gamma;
+  const void* ln2_beta;
+  const void* W_1;
+  const void* b_1;
+  const void* W_2;
+  const void* b_2;
+} hstu_transformer_weights;
+size_t hstu_transformer_workspace_size(int32_t d_model, int32_t n_heads, int32_t d_ff, int64_t B,
+                                       int64_t total_tokens);
+hstu_status hstu_transformer_layer_fwd(int32_t d_model, int32_t n_heads, int32_t d_ff,
+                                       float ln_eps, const hstu_transformer_weights* weights,
+                                       int64_t B, int64_t total_tokens, int64_t max_len,
+                                       const int64_t* offsets, const void* X, void* out,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
 /* Round-to-nearest conversion of n bf16 values to fp16 (device to device,
  * asynchronous on `stream`), for the optional W1_f16 / W2_f16 weight copies.
  * n must be a multiple of 8 and both pointers 16-byte aligned. */

@@ -90,3 +90,30 @@ def layer_fwd(X, offsets, w, n_heads: int, eps: float):
         if e > s:
             Y[s:e] = user_fwd(X[s:e], w, n_heads, eps)
     return Y
+
+
+def user_rows(X, w, n_heads: int, eps: float, rows):
+    """Y at the given rows of one user only (the keys and values of every row
+    up to the last requested one are formed; the rest of the layer runs on the
+    requested rows).  Equal to user_fwd(X, ...)[rows]."""
+    X = np.asarray(X, np.float64)
+    W = {k: np.asarray(v, np.float64) for k, v in w.items()}
+    rows = np.asarray(rows, np.int64)
+    d = X.shape[1]
+    dh = d // n_heads
+    last = int(rows.max()) + 1
+    A = layer_norm(X[:last], W["ln1_gamma"], W["ln1_beta"], eps)
+    QKV = A @ W["W_qkv"].T
+    ctx = np.empty((len(rows), d))
+    for ri, i in enumerate(rows):
+        for h in range(n_heads):
+            q = QKV[i, h * dh:(h + 1) * dh]
+            k = QKV[:i + 1, d + h * dh:d + (h + 1) * dh]
+            v = QKV[:i + 1, 2 * d + h * dh:2 * d + (h + 1) * dh]
+            s = k @ q / math.sqrt(dh)
+            p = np.exp(s - s.max())
+            ctx[ri, h * dh:(h + 1) * dh] = (p / p.sum()) @ v
+    X1 = X[rows] + ctx @ W["W_o"].T
+    B = layer_norm(X1, W["ln2_gamma"], W["ln2_beta"], eps)
+    F = silu(B @ W["W_1"].T + W["b_1"])
+    return X1 + F @ W["W_2"].T + W["b_2"]

@@ -137,3 +137,13 @@ def test_planted_mistakes_are_caught():
     assert np.abs(full - good[:, :dh]).max() > 1e-3
     # Q and K swapped
     assert np.abs(TR.attention(K, Q, V, heads) - good).max() > 1e-3
+
+
+def test_rows_helper_equals_the_whole_user():
+    rng = np.random.default_rng(7)
+    d, heads = 8, 2
+    w = _weights(rng, d, heads, 16)
+    X = rng.normal(size=(20, d))
+    rows = [0, 3, 19, 7]
+    np.testing.assert_allclose(TR.user_rows(X, w, heads, 1e-6, rows),
+                               TR.user_fwd(X, w, heads, 1e-6)[rows], rtol=0, atol=1e-12)
