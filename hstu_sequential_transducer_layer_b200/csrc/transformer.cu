@@ -16,9 +16,9 @@
 // same causal work list as the HSTU attention (only tiles at or left of the
 // diagonal).  Warp 0 loads Q (lane 0, with the K tiles) and V (lane 1) by TMA
 // through 2-stage rings; warp 1 issues S = Q K^T (two TMEM buffers) and
-// O += P V (P from TMEM); warps 4-7 own one query row per thread: the whole
-// 128-column row of S is in the thread's registers, so the row maximum and sum
-// need no exchange.  Online softmax in base 2: the running maximum moves only
+// O += P V (P from TMEM); warps 4-11 hold the score rows, two threads per
+// query row (64 columns each, in registers), which exchange their row maxima
+// and sums through shared memory.  Online softmax in base 2: the running maximum moves only
 // when a tile's maximum exceeds it by more than 8 (then O is rescaled in TMEM
 // by 2^(m_old - m_new)), so P = 2^(x - m) stays below 256 and fits fp16.  At
 // the end of an item the row of O is divided by the running sum and stored.
@@ -48,9 +48,11 @@ struct SmaxCfg {
   static constexpr int NA = D / 64;
   static constexpr uint32_t Q_OFF = 0, K_OFF = 2 * TILE, V_OFF = 4 * TILE;
   static constexpr uint32_t BAR_OFF = 6 * TILE;
-  static constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;
+  static constexpr uint32_t XCH_OFF = BAR_OFF + 256;  // [2 parities][2 halves][128 rows] floats
+  static constexpr uint32_t SMEM = XCH_OFF + 2 * 2 * 128 * 4 + 1024;
   static constexpr uint32_t O_COL = 256;  // TMEM: S0 | S1 | O
-  static constexpr int THREADS = 256;     // warp 0 loads, 1 MMA, 4-7 softmax
+  // warp 0 loads, 1 MMA, 4-7 and 8-11 softmax (columns 0-63 / 64-127 of S)
+  static constexpr int THREADS = 384;
 };
 
 DEVI float ex2_approx(float x) {
@@ -84,7 +86,8 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
   uint64_t* o_done = bars + 16;   // one phase per P.V
   uint64_t* o_free = bars + 17;   // one phase per item (O read out)
   uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* xch = bars + 19;      // [4] per lane quarter: the two halves of a row met
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
   int* s_nitems = s_go + 1;
@@ -103,10 +106,11 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
       mbar_init(v_full + i, 1);
       mbar_init(v_empty + i, 1);
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 4);
+      mbar_init(p_full + i, 8);
     }
     mbar_init(o_done, 1);
-    mbar_init(o_free, 4);
+    mbar_init(o_free, 8);
+    for (int i = 0; i < 4; ++i) mbar_init(xch + i, 2);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -271,13 +275,32 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
       }
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------ softmax warps: one row each
+    // ------------------------------------------------ softmax warps: half a row each
+    // Warps 4-7 take columns 0-63 of their lane quarter's 32 rows, warps 8-11
+    // columns 64-127; the two halves of a row exchange their maxima (each
+    // tile) and sums (each item) through shared memory, meeting on the lane
+    // quarter's mbarrier (bounded waits).
     const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const float sl2 = a.scale_log2;
-    uint32_t scount = 0, pvwait = 0;
+    float* xbuf = reinterpret_cast<float*>(smem + C::XCH_OFF);  // [par][half][128]
+    uint32_t scount = 0, pvwait = 0, nx = 0;
     bool alive = true;
+    // publish v, meet the partner, return the partner's value
+    auto exchange = [&](float v) -> float {
+      const int par = nx & 1;
+      xbuf[(par * 2 + half) * 128 + r] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch + q);
+      if (!mbar_wait_warp(xch + q, par, ab, a.status)) {
+        alive = false;
+        return 0.f;
+      }
+      ++nx;
+      return xbuf[(par * 2 + (half ^ 1)) * 128 + r];
+    };
     for (int k = 0; alive; ++k) {
       const int it = snake_item(k, cta, G);
       if (it >= n_items) break;
@@ -291,35 +314,46 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld32(tmem + sb * 128 + 0 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(sr));
-        tmem_ld32(tmem + sb * 128 + 32 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-        tmem_ld32(tmem + sb * 128 + 64 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
-        tmem_ld32(tmem + sb * 128 + 96 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(sr + 96));
+        const uint32_t s_addr = tmem + sb * 128 + half * 64 + lane_base;
+        uint32_t sr[64];
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
         tmem_ld_wait();
-        const bool diag = j == (int)w.qt;
-        float mt = -INFINITY;
+        float pm = -INFINITY;
+        if (j == (int)w.qt) {  // diagonal tile: column c > row r is masked
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float x = __uint_as_float(sr[c]) * sl2;
-          if (diag && c > r) x = -INFINITY;
-          sr[c] = __float_as_uint(x);
-          mt = fmaxf(mt, x);
+          for (int c = 0; c < 64; ++c) {
+            float x = __uint_as_float(sr[c]) * sl2;
+            if (half * 64 + c > r) x = -INFINITY;
+            sr[c] = __float_as_uint(x);
+            pm = fmaxf(pm, x);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float x = __uint_as_float(sr[c]) * sl2;
+            sr[c] = __float_as_uint(x);
+            pm = fmaxf(pm, x);
+          }
         }
+        // both halves have read their S columns once they meet here, so the
+        // P writes below cannot overwrite scores the partner still needs
+        const float mt = fmaxf(pm, exchange(pm));
+        if (!alive) break;
         const bool resc = mt > m + 8.f;
         const float m_new = resc ? mt : m;
         const float alpha = resc ? ex2_approx(m - m_new) : 1.f;
         float ls = 0.f;
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 32; ++c) {
           const float p0 = ex2_approx(__uint_as_float(sr[2 * c]) - m_new);
           const float p1 = ex2_approx(__uint_as_float(sr[2 * c + 1]) - m_new);
           ls += p0 + p1;
           pk[c] = pack_f16x2_sat(p0, p1);
         }
-        // O is rescaled once the previous P.V has landed in it (tile 0's P.V
-        // overwrites O, so it needs none)
+        // this half of O is rescaled once the previous P.V has landed in it
+        // (tile 0's P.V overwrites O, so it needs none)
         if (j > 0) {
           if (!mbar_wait_warp(o_done, pvwait & 1, ab, a.status)) {
             alive = false;
@@ -329,18 +363,18 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
           if (__any_sync(0xffffffffu, resc)) {
             tc_fence_after();
 #pragma unroll
-            for (int c16 = 0; c16 < D / 16; ++c16) {
+            for (int c16 = 0; c16 < D / 32; ++c16) {
+              const uint32_t oa = tmem + C::O_COL + half * (D / 2) + c16 * 16 + lane_base;
               uint32_t o[16];
-              tmem_ld16(tmem + C::O_COL + c16 * 16 + lane_base, o);
+              tmem_ld16(oa, o);
               tmem_ld_wait();
 #pragma unroll
               for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st16(tmem + C::O_COL + c16 * 16 + lane_base, o);
+              tmem_st16(oa, o);
             }
           }
         }
-        tmem_st32(tmem + sb * 128 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        tmem_st32(tmem + sb * 128 + 32 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        tmem_st32(tmem + sb * 128 + half * 32 + lane_base, pk);
         tmem_st_wait();
         l = l * alpha + ls;
         m = m_new;
@@ -350,24 +384,27 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
         ++scount;
       }
       if (!alive) break;
-      // ---- epilogue: O / l once the item's last P.V has landed
+      // ---- epilogue: this half of O / (both halves' sums)
       if (!mbar_wait_warp(o_done, pvwait & 1, ab, a.status)) break;
       ++pvwait;
       tc_fence_after();
-      uint32_t o[D];
+      uint32_t o[D / 2];
 #pragma unroll
-      for (int c32 = 0; c32 < D / 32; ++c32)
-        tmem_ld32(tmem + C::O_COL + c32 * 32 + lane_base,
-                  *reinterpret_cast<uint32_t(*)[32]>(o + c32 * 32));
+      for (int c16 = 0; c16 < D / 32; ++c16)
+        tmem_ld16(tmem + C::O_COL + half * (D / 2) + c16 * 16 + lane_base,
+                  *reinterpret_cast<uint32_t(*)[16]>(o + c16 * 16));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_free);  // the next item's first P.V may overwrite O
+      const float lt = l + exchange(l);
+      if (!alive) break;
       if (r < rows_valid) {
-        const float inv = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(a.ctx + (int64_t)(w.q_row0 + r) * a.ldc + w.head * D);
+        const float inv = 1.f / lt;
+        uint4* dst = reinterpret_cast<uint4*>(a.ctx + (int64_t)(w.q_row0 + r) * a.ldc + w.head * D +
+                                              half * (D / 2));
 #pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
+        for (int c8 = 0; c8 < D / 16; ++c8) {
           uint4 v;
           v.x = pack_f16x2_sat(__uint_as_float(o[c8 * 8 + 0]) * inv, __uint_as_float(o[c8 * 8 + 1]) * inv);
           v.y = pack_f16x2_sat(__uint_as_float(o[c8 * 8 + 2]) * inv, __uint_as_float(o[c8 * 8 + 3]) * inv);
