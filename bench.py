@@ -642,6 +642,7 @@ def run_ours(args):
         H.hstu_trace_enable(0)
         if H.hstu_read_status(r_ws) != 0:
             raise RuntimeError(f"retrieval device status {H.hstu_read_status(r_ws)}")
+        r_fallback = H.hstu_retrieval_fallback_taken(r_ws)
         r_ms = sum(a.elapsed_time(b) for a, b in r_evs) / len(r_evs)
         r_kern = {}
         for kid, t in r_trace:
@@ -660,9 +661,10 @@ def run_ours(args):
                             "frac": round(r_bytes / (r_ms / 1e3) / 1e9 / hbm, 4),
                             "peak_source": f"hbm_gbs ({peak_src})",
                             "bytes_per_step": int(r_bytes),
-                            "note": "whole step against the catalog read once; the scores "
-                                    "matrix (4 B per user-item) is written and read back "
-                                    "between the GEMM and the top-K"},
+                            "note": "whole step against the catalog read once (the filtering "
+                                    "pass reads it once more after a 1-in-16 sample pass)"},
+               "path": ("direct (fallback: every score written)" if r_fallback else
+                        "sample threshold + filtering GEMM epilogue (no score matrix)"),
                "tflops": round(r_flops / (r_ms / 1e3) / 1e12, 1),
                "gemm_tflops": round(r_flops / (g_ms / g_n / 1e3) / 1e12, 1),
                "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / v[0], 4)}

@@ -8,7 +8,7 @@ from .binding import (  # noqa: F401
     HstuError, LayerDesc, LayerWeights, make_desc, weights_struct, weights_array,
     weights_to_device, hstu_workspace_size, hstu_layer_fwd, hstu_stack_fwd, hstu_mfalcon_rank,
     hstu_sl_embed, hstu_sl_embed_workspace_size, hstu_sl_keep_count,
-    hstu_bf16_to_f16, hstu_retrieval_workspace_size, hstu_retrieval_topk,
+    hstu_bf16_to_f16, hstu_retrieval_workspace_size, hstu_retrieval_topk, hstu_retrieval_fallback_taken,
     hstu_transformer_workspace_size, hstu_transformer_layer_fwd, TransformerWeights,
     hstu_read_status, hstu_debug_offsets, hstu_trace_enable, hstu_trace_read, hstu_kernel_name,
     hstu_launch_count, hstu_status_string, hstu_version, lib, LIB_PATH, EXPORTED,

@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
             "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
             "hstu_sl_keep_count", "hstu_bf16_to_f16", "hstu_retrieval_workspace_size",
-            "hstu_retrieval_topk", "hstu_transformer_workspace_size",
+            "hstu_retrieval_topk", "hstu_retrieval_fallback_taken",
+            "hstu_transformer_workspace_size",
             "hstu_transformer_layer_fwd",
             "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
@@ -95,6 +96,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_retrieval_workspace_size.restype = sz
     L.hstu_retrieval_topk.argtypes = [i64, i64, i32, vp, vp, i64, vp, i32, vp, vp, vp, sz, vp]
     L.hstu_retrieval_topk.restype = i32
+    L.hstu_retrieval_fallback_taken.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_int32), vp]
+    L.hstu_retrieval_fallback_taken.restype = i32
     L.hstu_transformer_workspace_size.argtypes = [i32, i32, i32, i64, i64]
     L.hstu_transformer_workspace_size.restype = sz
     L.hstu_transformer_layer_fwd.argtypes = [i32, i32, i32, ctypes.c_float,
@@ -253,6 +256,14 @@ def hstu_retrieval_topk(H, E, K, out_scores, out_ids, workspace, user_offsets=No
                                      _ptr(out_ids), _ptr(workspace), _nbytes(workspace),
                                      _stream(stream)),
            "hstu_retrieval_topk")
+
+
+def hstu_retrieval_fallback_taken(workspace, stream=None) -> bool:
+    v = ctypes.c_int32(0)
+    _check(lib().hstu_retrieval_fallback_taken(_ptr(workspace), _nbytes(workspace),
+                                               ctypes.byref(v), _stream(stream)),
+           "hstu_retrieval_fallback_taken")
+    return bool(v.value)
 
 
 def hstu_transformer_workspace_size(d_model, n_heads, d_ff, B, total_tokens) -> int:

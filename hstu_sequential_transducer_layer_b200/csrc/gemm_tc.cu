@@ -5,6 +5,8 @@
 //   f2:  Y = X + Z W2^T + b2           (EPI_RESID)
 //   scores: S = H E^T                  (EPI_SCORE; fp32, ragged item count)
 //   plain:  C = A W^T + b              (EPI_BIAS; 16-bit output)
+//   filter: (score, column) of A W^T at or above a per-row threshold, appended
+//           to per-row candidate lists (EPI_FILTER; nothing else is stored)
 // ('HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか':
 // one projection f1 followed by SiLU and a split; f2 back to d_model plus
 // the residual connection.)
@@ -37,6 +39,15 @@ struct GemmDev {
   int64_t ldr;
   int resid_kind;
   int* status;
+  const int* run_if;           // if set, the launch does nothing unless *run_if != 0
+  // EPI_FILTER: per-row threshold and candidate lists
+  const float* tau;
+  int tau_stride;
+  uint32_t* cand_key;
+  int32_t* cand_id;
+  int* cand_cnt;
+  int cand_cap;
+  int* overflow;
 };
 
 constexpr int kEpiThreads = 256;      // 8 epilogue warps
@@ -156,6 +167,26 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   return true;
 }
 
+// EPI_FILTER: this lane's row, 32 columns from `col`: scores whose key is at
+// most the row's threshold key are appended to the row's candidate list.
+DEVI void gemm_filter_chunk(const GemmDev& g, int64_t row, bool valid, int col,
+                            const uint32_t (&r)[32], uint32_t thr) {
+  if (!valid || col >= g.N) return;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t key = desc_key(__uint_as_float(r[i]));
+    if (key <= thr && col + i < g.N) {
+      const int idx = atomicAdd(g.cand_cnt + row, 1);
+      if (idx < g.cand_cap) {
+        g.cand_key[row * g.cand_cap + idx] = key;
+        g.cand_id[row * g.cand_cap + idx] = col + i;
+      } else {
+        *reinterpret_cast<volatile int*>(g.overflow) = 1;
+      }
+    }
+  }
+}
+
 template <int BN, int STAGES, int EPI, int COMPACT>
 __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -178,7 +209,8 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    *s_go = (g.status == nullptr) || (*reinterpret_cast<volatile int*>(g.status) == 0);
+    *s_go = ((g.status == nullptr) || (*reinterpret_cast<volatile int*>(g.status) == 0)) &&
+            (g.run_if == nullptr || *reinterpret_cast<volatile const int*>(g.run_if) != 0);
     ab->flag = 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
@@ -324,13 +356,15 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       const int col0 = g.n_off + nt * BN + part * (BN / 2);
       const uint4* bptr = reinterpret_cast<const uint4*>(g.bias + col0);
       uint4 ba[4], bb[4];
+      constexpr bool kNoBias = EPI == EPI_SCORE || EPI == EPI_FILTER;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ba[i] = EPI == EPI_SCORE ? make_uint4(0, 0, 0, 0) : __ldg(bptr + i);
+      for (int i = 0; i < 4; ++i) ba[i] = kNoBias ? make_uint4(0, 0, 0, 0) : __ldg(bptr + i);
       if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) break;
       tc_fence_after();
       const int y0 = mt * 128 + q * 32;
       const int64_t row = (int64_t)y0 + lane;
       const bool valid = row < Mrows;
+      const uint32_t thr = (EPI == EPI_FILTER && valid) ? desc_key(g.tau[row * g.tau_stride]) : 0u;
       const uint32_t tbase = tmem + acc * BN + part * (BN / 2) + ((uint32_t)(q * 32) << 16);
       uint32_t ra[32], rb_acc[32];
       tmem_ld32(tbase, ra);
@@ -341,7 +375,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
         if (c + 1 < CH) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint4 bv = EPI == EPI_SCORE ? make_uint4(0, 0, 0, 0) : __ldg(bptr + (c + 1) * 4 + i);
+            const uint4 bv = kNoBias ? make_uint4(0, 0, 0, 0) : __ldg(bptr + (c + 1) * 4 + i);
             if (c & 1) ba[i] = bv;
             else bb[i] = bv;
           }
@@ -357,13 +391,17 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
           rpar ^= 1;
           rsm = rbuf;
         }
-        bool stored;
-        if (c & 1)
+        bool stored = false;
+        if (EPI == EPI_FILTER) {
+          if (c & 1) gemm_filter_chunk(g, row, valid, col0 + c * 32, rb_acc, thr);
+          else gemm_filter_chunk(g, row, valid, col0 + c * 32, ra, thr);
+        } else if (c & 1) {
           stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb_acc, bb,
                                    stage, COMPACT ? -1 : (nchunk & 1), rsm);
-        else
+        } else {
           stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba,
                                    stage, COMPACT ? -1 : (nchunk & 1), rsm);
+        }
         nchunk += stored ? 1 : 0;
         if (rtma) {
           __syncwarp();  // every lane has read the residual chunk
@@ -464,7 +502,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
                            r32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
-  GemmDev gd;
+  GemmDev gd{};  // value-initialised: optional fields (run_if, filter lists) stay null
   gd.M_cap = c.M_cap;
   gd.M_dev = c.M_dev;
   gd.N = c.N;
@@ -504,7 +542,8 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
 
 cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_t ldw, int ab_f16,
                                int64_t M_cap, int64_t N, int K, float* out, int64_t ldo,
-                               int* status, cudaStream_t s, int kernel_id) {
+                               int* status, cudaStream_t s, int kernel_id, int64_t w_row_step,
+                               const int* run_if) {
   if (M_cap <= 0 || N <= 0) return cudaSuccess;
   if (K % 64 != 0 || K <= 0 || ldo % 4 != 0 || ldo < N) return cudaErrorInvalidValue;
   if (M_cap > (1ll << 31) - 256 || N > (1ll << 31) - 256) return cudaErrorInvalidValue;
@@ -514,8 +553,11 @@ cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_
   if (!encode_tmap_2d(&ta, A, (uint64_t)M_cap, (uint64_t)K, (uint64_t)lda * 2, 64, 128, f16))
     return cudaErrorInvalidValue;
   // rows past N read as zeros; the output map's extent is N, so stores past
-  // the last item are clipped
-  if (!encode_tmap_2d(&tb, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64, BN, f16))
+  // the last item are clipped.  w_row_step > 1 reads every w_row_step-th row
+  // of W (a strided sample of the items) as the N rows.
+  if (w_row_step < 1 ||
+      !encode_tmap_2d(&tb, W, (uint64_t)N, (uint64_t)K, (uint64_t)(ldw * w_row_step) * 2, 64, BN,
+                      f16))
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d_ex(&to32, out, (uint64_t)M_cap, (uint64_t)N, (uint64_t)ldo * 4, 32, 32,
                          CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -532,10 +574,44 @@ cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_
   gd.has_out32 = 1;
   gd.resid = nullptr;
   gd.status = status;
+  gd.run_if = run_if;
   const int64_t tiles = ((M_cap + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
   LaunchScope ls(kernel_id, s);
   return launch_one<BN, 4, EPI_SCORE>(ta, tb, ta, to32, ta, gd, grid, s);
+}
+
+cudaError_t launch_gemm_filter(const void* A, int64_t lda, const void* W, int64_t ldw, int ab_f16,
+                               int64_t M_cap, int64_t N, int K, const float* tau, int tau_stride,
+                               uint32_t* cand_key, int32_t* cand_id, int* cnt, int cap,
+                               int* overflow, int* status, cudaStream_t s, int kernel_id) {
+  if (M_cap <= 0 || N <= 0) return cudaSuccess;
+  if (K % 64 != 0 || K <= 0 || cap <= 0) return cudaErrorInvalidValue;
+  if (M_cap > (1ll << 31) - 256 || N > (1ll << 31) - 256) return cudaErrorInvalidValue;
+  constexpr int BN = 256;
+  CUtensorMap ta, tb;
+  const bool f16 = ab_f16 != 0;
+  if (!encode_tmap_2d(&ta, A, (uint64_t)M_cap, (uint64_t)K, (uint64_t)lda * 2, 64, 128, f16))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tb, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64, BN, f16))
+    return cudaErrorInvalidValue;
+  GemmDev gd{};
+  gd.M_cap = M_cap;
+  gd.N = (int)N;
+  gd.K = K;
+  gd.ab_f16 = ab_f16;
+  gd.status = status;
+  gd.tau = tau;
+  gd.tau_stride = tau_stride;
+  gd.cand_key = cand_key;
+  gd.cand_id = cand_id;
+  gd.cand_cnt = cnt;
+  gd.cand_cap = cap;
+  gd.overflow = overflow;
+  const int64_t tiles = ((M_cap + 127) / 128) * ((N + BN - 1) / BN);
+  const int grid = (int)std::min<int64_t>(tiles, num_sms());
+  LaunchScope ls(kernel_id, s);
+  return launch_one<BN, 4, EPI_FILTER>(ta, tb, ta, ta, ta, gd, grid, s);
 }
 
 }  // namespace hstu

@@ -45,7 +45,9 @@ enum KernelId : int32_t {
   K_TF_OPROJ = 26,
   K_TF_FFN1 = 27,
   K_TF_FFN2 = 28,
-  K_NUM_KERNELS = 29
+  K_GEMM_FILTER = 29,
+  K_FILTER_MERGE = 30,
+  K_NUM_KERNELS = 31
 };
 const char* kernel_name(int id);
 
@@ -130,7 +132,7 @@ void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64
                      int32_t* t_rel, Header* hdr, cudaStream_t s);
 
 // C[M, N] = A[M, K] * W[n_off + N, K]^T with fused epilogue, bf16 tcgen05.
-enum Epilogue { EPI_SILU = 0, EPI_RESID = 1, EPI_SCORE = 2, EPI_BIAS = 3 };
+enum Epilogue { EPI_SILU = 0, EPI_RESID = 1, EPI_SCORE = 2, EPI_BIAS = 3, EPI_FILTER = 4 };
 enum ResidKind { RESID_BF16 = 0, RESID_F32 = 1, RESID_F16 = 2 };
 struct GemmCall {
   const void* A;  int64_t lda;   // [M_cap, K] row stride in elements
@@ -154,7 +156,16 @@ cudaError_t launch_gemm_tc(const GemmCall& g, cudaStream_t s, int kernel_id);
 // ldo % 4 == 0, bf16 or fp16 operands (ab_f16).
 cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_t ldw, int ab_f16,
                                int64_t M_cap, int64_t N, int K, float* out, int64_t ldo,
-                               int* status, cudaStream_t s, int kernel_id);
+                               int* status, cudaStream_t s, int kernel_id,
+                               int64_t w_row_step = 1, const int* run_if = nullptr);
+// Scores of the same product that reach a per-row threshold, appended to
+// per-row candidate lists: row r keeps (key, column) for every score s with
+// desc_key(s) <= desc_key(tau[r * tau_stride]) (i.e. s >= tau, -0 as +0), at
+// most `cap` per row (cnt[r] counts all; beyond cap only *overflow is set).
+cudaError_t launch_gemm_filter(const void* A, int64_t lda, const void* W, int64_t ldw, int ab_f16,
+                               int64_t M_cap, int64_t N, int K, const float* tau, int tau_stride,
+                               uint32_t* cand_key, int32_t* cand_id, int* cnt, int cap,
+                               int* overflow, int* status, cudaStream_t s, int kernel_id);
 cudaError_t launch_gemm_simt_f32(const GemmCall& g, cudaStream_t s, int kernel_id);
 
 // Pointwise causal attention (SELF) or candidate-vs-history (CAND).

@@ -281,6 +281,21 @@ DEVI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
 }
 DEVI void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------- score keys
+// Order-preserving 32-bit key of an fp32 score with the order reversed (a
+// smaller key is a larger score); -0 is folded into +0 so equal scores get
+// equal keys.
+DEVI uint32_t desc_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return ~asc;
+}
+DEVI float key_score(uint32_t k) {
+  const uint32_t asc = ~k;
+  return __uint_as_float((asc & 0x80000000u) ? (asc & 0x7fffffffu) : ~asc);
+}
+
 // ---------------------------------------------------------------- math
 // SiLU(x) = x * sigmoid(x), sigmoid(x) = 0.5 + 0.5 * tanh(x / 2), one MUFU op.
 DEVI float tanh_approx(float x) {

@@ -8,12 +8,22 @@
 // '全体像：LLMは入力を読み、ranking headが作品を採点する').  Here: the K highest
 // scores per user, equal scores ordered by ascending item id.
 //
-// Steps: k_ret_gather (optional) copies each user's last encoder row into
-// the workspace; the tcgen05 GEMM (EPI_SCORE) writes the fp32 scores
-// [U, M]; k_topk_chunk selects, per user and 8192-item chunk, the chunk's K
-// best items (radix select over order-preserving 32-bit keys held in shared
-// memory); k_topk_merge selects the K best of those candidates per user and
-// sorts them (bitonic sort of (key, id) pairs).
+// Steps (catalogs of 65,536 items or more): k_ret_gather (optional) copies
+// each user's last encoder row into the workspace; the tcgen05 GEMM scores a
+// 1-in-16 strided sample of the catalog and the top-K kernels below take each
+// user's ks-th best sample score as its threshold; the GEMM then scores the
+// whole catalog with an epilogue that only appends the (key, item) pairs at
+// or above the user's threshold to a candidate list (the score matrix is
+// never written); k_filter_merge picks the K best candidates per user
+// exactly.  At least ks sample items reach the threshold, so whenever K or
+// more candidates do, they hold the K best; if a user has fewer (or more than
+// fit), a device flag makes the direct path below run instead.
+// Direct path (smaller catalogs, or that fallback): the GEMM (EPI_SCORE)
+// writes the fp32 scores [U, M]; k_topk_chunk selects, per user and
+// 8192-item chunk, the chunk's K best items (radix select over
+// order-preserving 32-bit keys held in shared memory); k_topk_merge selects
+// the K best of those candidates per user and sorts them (bitonic sort of
+// (key, id) pairs).
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
@@ -26,20 +36,6 @@ constexpr int kTopkMaxK = 1024;
 constexpr int kMergeThreads = 1024;
 constexpr uint32_t kPadKey = 0xffffffffu;
 constexpr int32_t kPadId = 0x7fffffff;
-
-// Order-preserving key with the order reversed: a smaller key is a larger
-// score, so the top-K are the K smallest keys.  -0 is folded into +0 so that
-// equal scores compare equal.
-__device__ __forceinline__ uint32_t desc_key(float f) {
-  uint32_t b = __float_as_uint(f);
-  if (b == 0x80000000u) b = 0u;
-  const uint32_t asc = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return ~asc;
-}
-__device__ __forceinline__ float key_score(uint32_t k) {
-  const uint32_t asc = ~k;
-  return __uint_as_float((asc & 0x80000000u) ? (asc & 0x7fffffffu) : ~asc);
-}
 
 // Block-wide exclusive scan of one int per thread (NT threads).
 template <int NT>
@@ -210,12 +206,13 @@ constexpr int kCandCap = 4096;
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk_chunk(const float* __restrict__ S, int64_t ldS, int64_t M, int K, int n_chunks,
                  uint32_t* __restrict__ cand_key, int32_t* __restrict__ cand_id,
-                 const int* status) {
+                 const int* status, const int* run_if) {
   __shared__ uint32_t s_key[kTopkChunk];
   __shared__ uint16_t s_pos[kCandCap];
   __shared__ int s_hist[256];
   __shared__ int s_digit, s_rem, s_cnt;
   __shared__ int s_warp[kTopkThreads / 32];
+  if (run_if && *run_if == 0) return;
   if (*status != HSTU_OK) return;
   const int tid = threadIdx.x;
   const int chunk = blockIdx.x;
@@ -286,17 +283,53 @@ __global__ void __launch_bounds__(kTopkThreads)
   }
 }
 
+// Ascending bitonic sort of n (key, id) pairs in shared memory by key, then
+// id (padded to a power of two with (kPadKey, kPadId); the arrays hold at
+// least that many entries).  Every thread of the block calls it.
+template <int NT>
+__device__ __forceinline__ void bitonic_sort_pairs(uint32_t* sk, int32_t* si, int n) {
+  const int tid = threadIdx.x;
+  int P = 1;
+  while (P < n) P <<= 1;
+  for (int i = n + tid; i < P; i += NT) {
+    sk[i] = kPadKey;
+    si[i] = kPadId;
+  }
+  __syncthreads();
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < P; i += NT) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const uint32_t ki = sk[i], kj = sk[j];
+          const int32_t ii = si[i], ij = si[j];
+          const bool gt = ki > kj || (ki == kj && ii > ij);  // (key, id) of i after j's
+          if (gt == up) {
+            sk[i] = kj;
+            sk[j] = ki;
+            si[i] = ij;
+            si[j] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // Per user: the K best of its n_cand candidates (item order = id order, so
 // equal keys are taken lowest id first), sorted by (key, id).
 __global__ void __launch_bounds__(kMergeThreads)
     k_topk_merge(const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_id,
                  int n_cand, int K, float* __restrict__ out_scores, int64_t* __restrict__ out_ids,
-                 const int* status) {
+                 const int* status, const int* run_if) {
   __shared__ int s_hist[256];
   __shared__ int s_digit, s_rem, s_cnt;
   __shared__ int s_warp[kMergeThreads / 32];
   __shared__ uint32_t s_k[kTopkMaxK];
   __shared__ int32_t s_i[kTopkMaxK];
+  if (run_if && *run_if == 0) return;
   if (*status != HSTU_OK) return;
   const int tid = threadIdx.x;
   const int64_t u = blockIdx.x;
@@ -343,44 +376,105 @@ __global__ void __launch_bounds__(kMergeThreads)
     run_lt += tot >> 16;
     run_eq += tot & 0xffff;
   }
-  // bitonic sort of the K selected pairs, padded to a power of two
-  int P = 1;
-  while (P < K) P <<= 1;
-  for (int i = K + tid; i < P; i += kMergeThreads) {
-    s_k[i] = kPadKey;
-    s_i[i] = kPadId;
-  }
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < P; i += kMergeThreads) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = (i & size) == 0;
-          const uint32_t ki = s_k[i], kj = s_k[j];
-          const int32_t ii = s_i[i], ij = s_i[j];
-          const bool gt = ki > kj || (ki == kj && ii > ij);  // (key, id) of i after j's
-          if (gt == up) {
-            s_k[i] = kj;
-            s_k[j] = ki;
-            s_i[i] = ij;
-            s_i[j] = ii;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  // sort the K selected pairs by (key, id)
+  bitonic_sort_pairs<kMergeThreads>(s_k, s_i, K);
   for (int i = tid; i < K; i += kMergeThreads) {
     out_scores[u * K + i] = key_score(s_k[i]);
     out_ids[u * K + i] = s_i[i];
   }
 }
 
+// Per user, after the filtering GEMM: the K best of the candidates that
+// reached the user's sample threshold (in no particular order), exactly: a
+// radix select of the K-th smallest key, every candidate below it on the
+// fixed high bits, and of those equal to it on those bits the best by
+// (key, id) after a sort.  Too few or too many candidates, or more equal
+// ones than fit, set *fallback (the exact unfused path then runs).
+constexpr int kEqCap = 2048;
+
+__global__ void __launch_bounds__(kMergeThreads)
+    k_filter_merge(const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_id,
+                   const int* __restrict__ cnt, int cap, int K, float* __restrict__ out_scores,
+                   int64_t* __restrict__ out_ids, int* fallback, const int* status) {
+  __shared__ int s_hist[256];
+  __shared__ int s_digit, s_rem, s_cnt;
+  __shared__ uint32_t s_k[kTopkMaxK];
+  __shared__ int32_t s_i[kTopkMaxK];
+  __shared__ uint32_t e_k[kEqCap];
+  __shared__ int32_t e_i[kEqCap];
+  __shared__ int s_nlt, s_neq;
+  if (*status != HSTU_OK) return;
+  const int tid = threadIdx.x;
+  const int64_t u = blockIdx.x;
+  const int n = cnt[u];
+  if (n < K || n > cap) {
+    if (tid == 0) atomicExch(fallback, 1);
+    return;
+  }
+  const uint32_t* keys = cand_key + u * (int64_t)cap;
+  const int32_t* ids = cand_id + u * (int64_t)cap;
+  uint32_t prefix;
+  int remaining, sh;
+  ret_radix_select<kMergeThreads>(n, K, [&](int p) { return __ldg(keys + p); }, s_hist, &s_digit,
+                                  &s_rem, &s_cnt, &prefix, &remaining, &sh);
+  if (tid == 0) {
+    s_nlt = 0;
+    s_neq = 0;
+  }
+  __syncthreads();
+  const uint32_t ph = sh == 32 ? 0u : prefix >> sh;
+  for (int p = tid; p < n; p += kMergeThreads) {
+    const uint32_t key = __ldg(keys + p);
+    const uint32_t hi = sh == 32 ? 0u : key >> sh;
+    if (sh == 32 || hi < ph) {
+      const int idx = atomicAdd(&s_nlt, 1);
+      s_k[idx] = key;
+      s_i[idx] = __ldg(ids + p);
+    } else if (hi == ph) {
+      const int idx = atomicAdd(&s_neq, 1);
+      if (idx < kEqCap) {
+        e_k[idx] = key;
+        e_i[idx] = __ldg(ids + p);
+      }
+    }
+  }
+  __syncthreads();
+  const int nlt = s_nlt, neq = s_neq;
+  if (sh != 32) {
+    if (neq > kEqCap) {  // (the sort below pads neq to a power of two <= kEqCap)
+      if (tid == 0) atomicExch(fallback, 1);
+      return;
+    }
+    bitonic_sort_pairs<kMergeThreads>(e_k, e_i, neq);
+    for (int i = tid; i < remaining; i += kMergeThreads) {
+      s_k[nlt + i] = e_k[i];
+      s_i[nlt + i] = e_i[i];
+    }
+    __syncthreads();
+  }
+  bitonic_sort_pairs<kMergeThreads>(s_k, s_i, K);
+  for (int i = tid; i < K; i += kMergeThreads) {
+    out_scores[u * K + i] = key_score(s_k[i]);
+    out_ids[u * K + i] = s_i[i];
+  }
+}
+
+// Filtering path: a 1-in-kSampleStep sample of the catalog is scored first;
+// each user's ks-th best sample score is its threshold.
+constexpr int kSampleStep = 16;
+constexpr int kFilterCap = 16384;           // candidates kept per user
+constexpr int64_t kFilterMinItems = 65536;  // smaller catalogs take the direct path
+
+static int sample_rank(int K) { return 4 * ((K + kSampleStep - 1) / kSampleStep) + 16; }
+
 struct RetLayout {
-  size_t hg, scores, ckey, cid, total;
-  int64_t ldS;
-  int n_chunks;
+  size_t hg, scores, ckey, cid;                  // direct path (and fallback)
+  size_t s_scores, s_ckey, s_cid, tau, tau_id;   // sample
+  size_t fcnt, fkey, fid;                        // filtered candidates
+  size_t total;
+  int64_t ldS, ldSs, Ms;
+  int n_chunks, n_chunks_s, ks;
+  bool filter;
 };
 
 static bool ret_layout(int64_t U, int64_t M, int32_t d, int32_t K, bool gather, RetLayout* L) {
@@ -390,7 +484,12 @@ static bool ret_layout(int64_t U, int64_t M, int32_t d, int32_t K, bool gather, 
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   L->ldS = (M + 63) / 64 * 64;
   L->n_chunks = (int)((M + kTopkChunk - 1) / kTopkChunk);
-  size_t o = 256;  // status word
+  L->Ms = (M + kSampleStep - 1) / kSampleStep;
+  L->ldSs = (L->Ms + 63) / 64 * 64;
+  L->n_chunks_s = (int)((L->Ms + kTopkChunk - 1) / kTopkChunk);
+  L->ks = sample_rank(K);
+  L->filter = M >= kFilterMinItems && L->ks <= kTopkMaxK && L->ks * 4 <= L->Ms;
+  size_t o = 256;  // status word, fallback flag
   L->hg = o;
   o += up(gather ? (size_t)U * d * 2 : 0);
   L->scores = o;
@@ -399,6 +498,23 @@ static bool ret_layout(int64_t U, int64_t M, int32_t d, int32_t K, bool gather, 
   o += up((size_t)U * L->n_chunks * K * 4);
   L->cid = o;
   o += up((size_t)U * L->n_chunks * K * 4);
+  const int ks = L->filter ? L->ks : 1;
+  L->s_scores = o;
+  o += up(L->filter ? (size_t)U * L->ldSs * 4 : 0);
+  L->s_ckey = o;
+  o += up(L->filter ? (size_t)U * L->n_chunks_s * ks * 4 : 0);
+  L->s_cid = o;
+  o += up(L->filter ? (size_t)U * L->n_chunks_s * ks * 4 : 0);
+  L->tau = o;
+  o += up(L->filter ? (size_t)U * ks * 4 : 0);
+  L->tau_id = o;
+  o += up(L->filter ? (size_t)U * ks * 8 : 0);
+  L->fcnt = o;
+  o += up(L->filter ? (size_t)U * 4 : 0);
+  L->fkey = o;
+  o += up(L->filter ? (size_t)U * kFilterCap * 4 : 0);
+  L->fid = o;
+  o += up(L->filter ? (size_t)U * kFilterCap * 4 : 0);
   L->total = o;
   return (int64_t)L->n_chunks * K <= (1ll << 30);
 }
@@ -431,7 +547,10 @@ hstu_status hstu_retrieval_topk(int64_t U, int64_t M, int32_t d, const void* H,
   if (gather && total_rows < 0) return HSTU_ERR_INVALID_ARG;
   uint8_t* w = static_cast<uint8_t*>(ws);
   int* status = reinterpret_cast<int*>(w);
-  if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  int* fallback = status + 1;
+  if (cudaMemsetAsync(w, 0, 256, stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (L.filter && cudaMemsetAsync(w + L.fcnt, 0, (size_t)U * 4, stream) != cudaSuccess)
+    return HSTU_ERR_CUDA;
   const void* A = H;
   if (gather) {
     LaunchScope ls(K_RET_GATHER, stream);
@@ -442,25 +561,76 @@ hstu_status hstu_retrieval_topk(int64_t U, int64_t M, int32_t d, const void* H,
     if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
     A = w + L.hg;
   }
-  float* S = reinterpret_cast<float*>(w + L.scores);
-  if (launch_gemm_scores(A, d, E, d, 0, U, M, d, S, L.ldS, status, stream, K_GEMM_SCORES) !=
-      cudaSuccess)
+  // the exact direct path: every score written, per-chunk top-K, merge;
+  // with run_if set it runs only if the filtering path gave up
+  auto direct = [&](const int* run_if) -> hstu_status {
+    float* S = reinterpret_cast<float*>(w + L.scores);
+    if (launch_gemm_scores(A, d, E, d, 0, U, M, d, S, L.ldS, status, stream, K_GEMM_SCORES, 1,
+                           run_if) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+    uint32_t* ck = reinterpret_cast<uint32_t*>(w + L.ckey);
+    int32_t* ci = reinterpret_cast<int32_t*>(w + L.cid);
+    {
+      LaunchScope ls(K_TOPK_CHUNK, stream);
+      k_topk_chunk<<<dim3((unsigned)L.n_chunks, (unsigned)U), kTopkThreads, 0, stream>>>(
+          S, L.ldS, M, K, L.n_chunks, ck, ci, status, run_if);
+      if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+    }
+    {
+      LaunchScope ls(K_TOPK_MERGE, stream);
+      k_topk_merge<<<(unsigned)U, kMergeThreads, 0, stream>>>(ck, ci, L.n_chunks * K, K,
+                                                             out_scores, out_ids, status, run_if);
+      if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+    }
+    return HSTU_OK;
+  };
+  if (!L.filter) return direct(nullptr);
+  // ---- threshold per user from a strided sample of the catalog
+  const int ks = L.ks;
+  float* Ss = reinterpret_cast<float*>(w + L.s_scores);
+  if (launch_gemm_scores(A, d, E, d, 0, U, L.Ms, d, Ss, L.ldSs, status, stream, K_GEMM_SCORES,
+                         kSampleStep) != cudaSuccess)
     return HSTU_ERR_CUDA;
-  uint32_t* ck = reinterpret_cast<uint32_t*>(w + L.ckey);
-  int32_t* ci = reinterpret_cast<int32_t*>(w + L.cid);
+  float* tau = reinterpret_cast<float*>(w + L.tau);
   {
+    uint32_t* sck = reinterpret_cast<uint32_t*>(w + L.s_ckey);
+    int32_t* sci = reinterpret_cast<int32_t*>(w + L.s_cid);
     LaunchScope ls(K_TOPK_CHUNK, stream);
-    k_topk_chunk<<<dim3((unsigned)L.n_chunks, (unsigned)U), kTopkThreads, 0, stream>>>(
-        S, L.ldS, M, K, L.n_chunks, ck, ci, status);
+    k_topk_chunk<<<dim3((unsigned)L.n_chunks_s, (unsigned)U), kTopkThreads, 0, stream>>>(
+        Ss, L.ldSs, L.Ms, ks, L.n_chunks_s, sck, sci, status, nullptr);
+    if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+    LaunchScope ls2(K_TOPK_MERGE, stream);
+    k_topk_merge<<<(unsigned)U, kMergeThreads, 0, stream>>>(
+        sck, sci, L.n_chunks_s * ks, ks, tau, reinterpret_cast<int64_t*>(w + L.tau_id), status,
+        nullptr);
     if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   }
+  // ---- every score at or above the user's threshold becomes a candidate
+  uint32_t* fk = reinterpret_cast<uint32_t*>(w + L.fkey);
+  int32_t* fi = reinterpret_cast<int32_t*>(w + L.fid);
+  int* fc = reinterpret_cast<int*>(w + L.fcnt);
+  if (launch_gemm_filter(A, d, E, d, 0, U, M, d, tau + (ks - 1), ks, fk, fi, fc, kFilterCap,
+                         fallback, status, stream, K_GEMM_FILTER) != cudaSuccess)
+    return HSTU_ERR_CUDA;
   {
-    LaunchScope ls(K_TOPK_MERGE, stream);
-    k_topk_merge<<<(unsigned)U, kMergeThreads, 0, stream>>>(ck, ci, L.n_chunks * K, K, out_scores,
-                                                           out_ids, status);
+    LaunchScope ls(K_FILTER_MERGE, stream);
+    k_filter_merge<<<(unsigned)U, kMergeThreads, 0, stream>>>(fk, fi, fc, kFilterCap, K, out_scores,
+                                                             out_ids, fallback, status);
     if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   }
+  return direct(fallback);
+}
+
+hstu_status hstu_retrieval_fallback_taken(const void* workspace, size_t workspace_bytes,
+                                          int32_t* taken, void* stream) {
+  if (!workspace || workspace_bytes < 256 || !taken) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(taken, static_cast<const int32_t*>(workspace) + 1, sizeof(int32_t),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return HSTU_ERR_CUDA;
   return HSTU_OK;
 }
 
 }  // extern "C"
+

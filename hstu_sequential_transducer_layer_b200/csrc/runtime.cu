@@ -26,7 +26,7 @@ const char* kernel_name(int id) {
       "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16", "time_buckets",
       "sl_offsets", "sl_select", "sl_gather", "ret_gather", "gemm_scores_tc", "topk_chunk",
       "topk_merge", "tf_ln", "tf_qkv_tc", "tf_softmax_attn_tc", "tf_oproj_tc", "tf_ffn1_tc",
-      "tf_ffn2_tc"};
+      "tf_ffn2_tc", "gemm_filter_tc", "filter_merge"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 

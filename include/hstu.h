@@ -248,6 +248,14 @@ hstu_status hstu_retrieval_topk(int64_t n_users, int64_t n_items, int32_t d, con
                                 const int64_t* user_offsets, int64_t total_rows, const void* E,
                                 int32_t K, float* out_scores, int64_t* out_ids, void* workspace,
                                 size_t workspace_bytes, void* stream);
+/* Catalogs of 65,536 items or more are first scored on a 1-in-16 strided
+ * sample to find a per-user score threshold, and the full pass keeps only
+ * the items at or above it (the score matrix is never written); a user left
+ * with fewer than K such items (or too many) makes the call fall back to
+ * scoring and selecting over every item, with the same result.  After a call
+ * (and a synchronisation of `stream`), *taken = 1 if that fallback ran. */
+hstu_status hstu_retrieval_fallback_taken(const void* workspace, size_t workspace_bytes,
+                                          int32_t* taken, void* stream);
 
 /* Softmax-Transformer encoder layer: the comparator of the HSTU layer on the
  * same jagged batches ('HSTUとGenerative Recommenders', section 'Production評価の

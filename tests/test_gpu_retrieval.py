@@ -153,11 +153,53 @@ def test_full_catalog_at_full_size():
     Ed = hw.device_embedding_table(0, 0, M, d, "cuda")
     rng = np.random.default_rng(9)
     Hh = hw.round_to_bf16(rng.standard_normal((U, d)).astype(np.float32) / 32.0)
-    st, s, i = _run(_bf16(Hh), Ed, K)
-    assert st == 0
+    st, s, i, ws = _run_ws(_bf16(Hh), Ed, K)
+    assert st == 0 and not _fallback_taken(ws)   # the filtering path decided
     users = [0, 1, 37, 64, 90, 101, 126, 127]
     Eb = Ed.view(torch.int16).cpu().numpy().view(np.uint16)
     E32 = (Eb.astype(np.uint32) << np.uint32(16)).view(np.float32)   # exact bf16 values
     del Eb
     S, A = _exact(E32, Hh[users].astype(np.float64))
     _validity(s[users], i[users], S, A, d, K)
+
+
+def _fallback_taken(ws):
+    import hstu_sequential_transducer_layer_b200 as H
+    return H.hstu_retrieval_fallback_taken(ws)
+
+
+def _run_ws(Hd, Ed, K):
+    import torch
+    import hstu_sequential_transducer_layer_b200 as H
+    U, (M, d) = Hd.shape[0], Ed.shape
+    ws = torch.empty(H.hstu_retrieval_workspace_size(U, M, d, K), dtype=torch.uint8, device="cuda")
+    s = torch.full((U, K), float("nan"), dtype=torch.float32, device="cuda")
+    i = torch.full((U, K), -1, dtype=torch.int64, device="cuda")
+    H.hstu_retrieval_topk(Hd, Ed, K, s, i, ws)
+    return H.hstu_read_status(ws), s.cpu().numpy(), i.cpu().numpy(), ws
+
+
+@pytest.mark.parametrize("U,M,K", [(7, 70000, 100), (3, 100003, 1024), (2, 65536, 1)])
+def test_filter_path_integer_inputs_exact(U, M, K):
+    """Catalogs of 65,536 items or more take the sample-threshold filtering
+    path; integer scores tie often, so the tie order is exercised too."""
+    rng = np.random.default_rng(M + K)
+    E, Hh = _ints(rng, (M, 64)), _ints(rng, (U, 64))
+    st, s, i, ws = _run_ws(_bf16(Hh), _bf16(E), K)
+    assert st == 0 and not _fallback_taken(ws)
+    rv, ri = R.retrieve(E, Hh, K)
+    np.testing.assert_array_equal(i, ri)
+    np.testing.assert_array_equal(s.astype(np.float64), rv)
+
+
+def test_fallback_when_every_score_ties():
+    # every item equal: all pass the threshold, the candidate lists overflow,
+    # the direct path runs and returns the first K ids
+    rng = np.random.default_rng(13)
+    E = np.ones((70000, 64), np.float32)
+    Hh = _ints(rng, (3, 64))
+    st, s, i, ws = _run_ws(_bf16(Hh), _bf16(E), 50)
+    assert st == 0 and _fallback_taken(ws)
+    rv, ri = R.retrieve(E, Hh, 50)
+    np.testing.assert_array_equal(i, ri)
+    np.testing.assert_array_equal(s.astype(np.float64), rv)
