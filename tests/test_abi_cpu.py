@@ -127,3 +127,60 @@ def test_host_keep_count_matches_oracle():
     got = [B.hstu_sl_keep_count(n) for n in range(0, 32768)]
     assert got == [SL.keep_count(n) for n in range(0, 32768)]
     assert B.hstu_sl_keep_count(-1) == -1 and B.hstu_sl_keep_count(32768) == -1
+
+
+def test_new_entry_points_reject_bad_arguments_before_launch():
+    """Stochastic Length, retrieval, the comparator layer and the weight
+    conversion check their arguments on the host and launch nothing when they
+    are wrong (no GPU is needed to see it)."""
+    L = B.lib()
+    n0 = H.hstu_launch_count()
+    ws, big = 0x100000, 1 << 30
+    # Stochastic Length + embedding: d % 8, max_raw_len bound, workspace, nulls, alignment
+    sl = lambda **k: L.hstu_sl_embed(
+        k.get("B", 2), k.get("R", 10), k.get("maxlen", 8), 0x1000, k.get("ids", 0x2000), 0x3000,
+        7, k.get("ctab", 0x4000), 100, 0x5000, 8, k.get("d", 64), 0x6000, 0x7000, 0x8000,
+        k.get("ws", ws), k.get("wsb", 256), None)
+    assert sl(d=12) == 1
+    assert sl(maxlen=40000) == 2
+    assert sl(ws=ws + 8) == 3 and sl(wsb=128) == 3
+    assert sl(ids=None) == 1
+    assert sl(ctab=0x4008) == 1
+    # retrieval: sizes
+    assert L.hstu_retrieval_workspace_size(4, 100, 64, 101, 0) == 0      # K > items
+    assert L.hstu_retrieval_workspace_size(4, 5000, 96, 10, 0) == 0      # d % 64
+    assert L.hstu_retrieval_workspace_size(70000, 5000, 64, 10, 0) == 0  # too many users
+    assert L.hstu_retrieval_workspace_size(4, 5000, 64, 2000, 0) == 0    # K > 1024
+    assert L.hstu_retrieval_workspace_size(4, 5000, 64, 10, 0) > 0
+    # the filtering path's buffers appear only for large catalogs
+    small = L.hstu_retrieval_workspace_size(128, 65535, 64, 100, 0)
+    large = L.hstu_retrieval_workspace_size(128, 65536, 64, 100, 0)
+    assert large > small + 128 * 16384 * 8
+    need = L.hstu_retrieval_workspace_size(4, 5000, 64, 10, 0)
+    ret = lambda **k: L.hstu_retrieval_topk(4, 5000, 64, k.get("H", 0x1000), None, 0, 0x2000,
+                                            k.get("K", 10), 0x3000, 0x4000, k.get("ws", ws),
+                                            k.get("wsb", need), None)
+    assert ret(K=0) == 1 and ret(K=5001) == 1
+    assert ret(wsb=need - 1) == 3 and ret(ws=ws + 16) == 3
+    assert ret(H=0x1008) == 1 and ret(H=None) == 1
+    taken = ctypes.c_int32(0)
+    assert L.hstu_retrieval_fallback_taken(None, 256, ctypes.byref(taken), None) == 1
+    # comparator layer: shapes it does not run
+    assert L.hstu_transformer_workspace_size(300, 4, 1024, 2, 100) == 0   # d % 256
+    assert L.hstu_transformer_workspace_size(256, 8, 1024, 2, 100) == 0   # head dim 32
+    assert L.hstu_transformer_workspace_size(256, 4, 100, 2, 100) == 0    # d_ff % 256
+    assert L.hstu_transformer_workspace_size(512, 8, 2048, 2, 100) > 0
+    tw = B.TransformerWeights(*([0x1000] * 10))
+    tneed = L.hstu_transformer_workspace_size(512, 8, 2048, 2, 100)
+    tf = lambda **k: L.hstu_transformer_layer_fwd(
+        k.get("d", 512), 8, 2048, 1e-6, ctypes.byref(k.get("w", tw)), 2, 100, 64, 0x1000,
+        k.get("X", 0x2000), 0x3000, ws, k.get("wsb", tneed), None)
+    assert tf(d=300) == 1
+    assert tf(wsb=tneed - 1) == 3
+    assert tf(w=B.TransformerWeights(*([0x1000] * 9 + [0]))) == 1
+    assert tf(X=0x2004) == 1
+    # bf16 -> fp16: length and alignment
+    assert L.hstu_bf16_to_f16(0x1000, 0x2000, 7, None) == 1
+    assert L.hstu_bf16_to_f16(0x1002, 0x2000, 8, None) == 1
+    assert L.hstu_bf16_to_f16(0x1000, 0x2000, 0, None) == 0
+    assert H.hstu_launch_count() == n0
