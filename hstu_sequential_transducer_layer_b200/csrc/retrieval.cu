@@ -540,7 +540,10 @@ hstu_status hstu_retrieval_topk(int64_t U, int64_t M, int32_t d, const void* H,
   RetLayout L;
   if (!ret_layout(U, M, d, K, gather, &L)) return HSTU_ERR_INVALID_ARG;
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HSTU_ERR_WORKSPACE;
-  if (U == 0) return HSTU_OK;
+  if (U == 0)  // nothing to score; the status word still reflects this call
+    return cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream_ptr)) == cudaSuccess
+               ? HSTU_OK
+               : HSTU_ERR_CUDA;
   if (!H || !E || !out_scores || !out_ids) return HSTU_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(H) & 15) || (reinterpret_cast<uintptr_t>(E) & 15))
     return HSTU_ERR_INVALID_ARG;

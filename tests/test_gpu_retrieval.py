@@ -203,3 +203,16 @@ def test_fallback_when_every_score_ties():
     rv, ri = R.retrieve(E, Hh, 50)
     np.testing.assert_array_equal(i, ri)
     np.testing.assert_array_equal(s.astype(np.float64), rv)
+
+
+def test_no_users():
+    import torch
+    import hstu_sequential_transducer_layer_b200 as H
+    E = _bf16(np.ones((300, 64), np.float32))
+    Hd = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    ws = torch.full((H.hstu_retrieval_workspace_size(0, 300, 64, 5),), 7, dtype=torch.uint8,
+                    device="cuda")
+    s = torch.empty((0, 5), dtype=torch.float32, device="cuda")
+    i = torch.empty((0, 5), dtype=torch.int64, device="cuda")
+    H.hstu_retrieval_topk(Hd, E, 5, s, i, ws)
+    assert H.hstu_read_status(ws) == 0   # a stale word from an earlier call would not be 0
