@@ -94,7 +94,7 @@ def mfalcon_flops(dims, n_layers, hist_lens, cands):
 class ClockSampler:
     """SM clock and clock-event reasons sampled every ~2 ms while the timed
     region runs (NVML from a thread; nvidia-smi at 100 ms if NVML is absent).
-    Samples also go to gpurun_out/clocks_rank<i>.csv."""
+    Samples also go to <HSTU_BENCH_OUT or bench_out>/clocks_rank<i>.csv."""
 
     NAMES = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
              "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
@@ -107,7 +107,8 @@ class ClockSampler:
         self.proc = None
         self.thread = None
         self.samples = []           # (sm_mhz, max_mhz, reason bitmask)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}{tag}.csv")
+        out_dir = os.environ.get("HSTU_BENCH_OUT", os.path.join(ROOT, "bench_out"))
+        self.path = os.path.join(out_dir, f"clocks_rank{gpu_index}{tag}.csv")
 
     def _nvml_handle(self):
         import pynvml

@@ -80,7 +80,7 @@ extern "C" {
 typedef enum {
   HSTU_OK = 0,
   HSTU_ERR_INVALID_ARG = 1,   /* host: null/misaligned pointer, bad size */
-  HSTU_ERR_UNSUPPORTED = 2,   /* host: shape or dtype this build does not run */
+  HSTU_ERR_UNSUPPORTED = 2,   /* host: a shape or dtype the library does not run */
   HSTU_ERR_WORKSPACE = 3,     /* host: workspace smaller than hstu_workspace_size */
   HSTU_ERR_CUDA = 4,          /* host: a CUDA runtime call failed */
   HSTU_ERR_BAD_OFFSETS = 5,   /* device: offsets not monotone, wrong total, length > max */

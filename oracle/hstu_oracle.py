@@ -46,7 +46,7 @@ def log_bucket(x, n_buckets: int, sub_bits: int) -> np.ndarray:
     """Log-linear bucket of a non-negative integer distance.
 
     The page says only that the relative bias is indexed by sequence distance
-    and by elapsed real time; the bucket rule is this build's reading: values
+    and by elapsed real time; the bucket rule is a reading made here: values
     below 2^S keep their own bucket; above, with e = floor(log2 x), the bucket
     is (e - S + 1) * 2^S + ((x >> (e - S)) - 2^S), i.e. the exponent and the
     top S mantissa bits of x; clamped to n_buckets - 1.
