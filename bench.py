@@ -774,12 +774,14 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
             "data": "synthetic (seeded; random-init weights)",
             "config": {"workload": "full_stack", "layers": w.n_layers, "d_model": w.dims.d_model,
                        "heads": w.dims.n_heads, "head_dim": w.dims.d_qk, "users_per_gpu": w.B,
                        "tokens_per_gpu": T, "max_len": w.max_len,
                        "l2": "256 MB flush between timed steps",
+                       "precision": "tensor-core operands fp16 (layer 0's f1 bf16), fp32 "
+                                    "accumulation; input and output bf16",
                        "parallelism": f"replicas x{world} (users independent, no collective)"},
             "tflops": round(step_flops / (ms / 1e3) / 1e12, 1),
             "tensor_frac": tensor_frac(step_flops / (ms / 1e3) / 1e12, peaks),
