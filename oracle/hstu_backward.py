@@ -1,4 +1,4 @@
-"""Float64 CPU oracle of the gradients of one HSTU layer (the backward pass,
+"""Float64 CPU oracle of the gradients of the HSTU layer and stack (the backward pass,
 for training).  TEST INFRASTRUCTURE ONLY: only ``tests/`` may import it; no
 kernel of the library computes a backward pass yet.
 
@@ -129,3 +129,20 @@ def layer_bwd(X, offsets, timestamps, w: Dict[str, np.ndarray], dims, dY):
     dX += dP @ W["W1"]
     g["dX"] = dX
     return g
+
+
+def stack_bwd(X, offsets, timestamps, weights, dims, dY):
+    """Gradients of sum(dY * Y) for Y = stack_fwd(X, ...) (layers applied in
+    order, each output the next layer's input): the layers' backward passes
+    in reverse order, each fed the gradient of its own output and its own
+    input.  Returns (dX, [per-layer weight gradients])."""
+    inputs = [np.asarray(X, np.float64)]
+    for w in weights[:-1]:
+        inputs.append(F.layer_fwd(inputs[-1], offsets, timestamps, w, dims))
+    grads = [None] * len(weights)
+    g_out = np.asarray(dY, np.float64)
+    for layer in range(len(weights) - 1, -1, -1):
+        g = layer_bwd(inputs[layer], offsets, timestamps, weights[layer], dims, g_out)
+        g_out = g.pop("dX")
+        grads[layer] = g
+    return g_out, grads

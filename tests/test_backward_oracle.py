@@ -109,3 +109,36 @@ def test_silu_derivative_closed_form():
     sig = 1 / (1 + np.exp(-x))
     np.testing.assert_allclose(BW.silu_grad(x), sig + x * sig * (1 - sig), rtol=1e-14, atol=1e-14)
     assert BW.silu_grad(np.array([0.0]))[0] == 0.5
+
+
+def test_stack_matches_finite_differences():
+    X, off, ts, w0, dY = _case(2)
+    w1 = {k: v * 0.9 + 0.01 for k, v in _case(3)[3].items()}
+    ws = [w0, w1]
+    dX, gs = BW.stack_bwd(X, off, ts, ws, DIMS, dY)
+
+    def obj(Xv, wl):
+        return float((dY * F.stack_fwd(Xv, off, ts, wl, DIMS)).sum())
+    eps = 1e-6
+    rng = np.random.default_rng(4)
+    # every input entry, and a random subset of each layer's parameters
+    num = np.empty_like(X)
+    for idx in np.ndindex(X.shape):
+        p, m = X.copy(), X.copy()
+        p[idx] += eps
+        m[idx] -= eps
+        num[idx] = (obj(p, ws) - obj(m, ws)) / (2 * eps)
+    assert np.abs(dX - num).max() <= 1e-6 * max(1.0, np.abs(num).max())
+    for layer in range(2):
+        for key, val in ws[layer].items():
+            for _ in range(3):
+                idx = tuple(int(rng.integers(0, n)) for n in val.shape)
+                p = [dict(wl) for wl in ws]
+                m = [dict(wl) for wl in ws]
+                p[layer][key] = val.copy()
+                m[layer][key] = val.copy()
+                p[layer][key][idx] += eps
+                m[layer][key][idx] -= eps
+                fd = (obj(X, p) - obj(X, m)) / (2 * eps)
+                got = gs[layer]["d" + key][idx]
+                assert abs(got - fd) <= 1e-6 * max(1.0, abs(fd)), (layer, key, idx, got, fd)
