@@ -653,7 +653,11 @@ def run_ours(args):
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         # algorithmic minimum: the catalog read once, the user rows and results
         r_bytes = r_M * r_d * 2 + r_U * r_d * 2 + r_U * r_K * 12
-        g_n, g_ms = r_kern.get("gemm_scores_tc", [1, float("nan")])
+        # the GEMM that scores the whole catalog: the filtering one, or on the
+        # direct path the scoring one (on the filtering path "gemm_scores_tc"
+        # is the 1-in-16 sample pass)
+        g_n, g_ms = r_kern.get("gemm_scores_tc" if r_fallback else "gemm_filter_tc",
+                               [1, float("nan")])
         r_flops = 2.0 * r_U * r_M * r_d
         ret = {"value": r_U * r_M / (r_ms / 1e3), "unit": "user-item scores/s",
                "ms_per_step": round(r_ms, 4),
