@@ -22,6 +22,16 @@ Workloads (sizes follow the pages' own workloads, see the docstring of each):
                      Length to floor(n^0.8) sampled positions; interleaved
                      content/action tokens from a 1M-id Zipf(1.1) table.
 
+Inputs of the paths around the stack:
+
+* ``full_stack_raw`` / ``raw_stream``  raw (not yet shortened) content/action
+                     streams, a 64-bit Stochastic Length seed; tables from
+                     ``embedding_table_bits`` (numpy, bf16 bit patterns) or
+                     ``device_embedding_table`` (torch's generator on the
+                     device, for the 1M x 1024 catalog).
+* ``transformer_weights``  the softmax-Transformer comparator layer's weights
+                     (dense fp16-rounded, LayerNorm and biases bf16-rounded).
+
 Every array is produced by ``numpy.random.default_rng(seed)`` in a fixed draw
 order: lengths -> timestamps -> weights -> rab -> X -> candidates -> head
 vector.  bf16 workloads round every bf16-stored tensor to bf16 here (round to
