@@ -240,15 +240,20 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
-def cpu_baseline_stack(w, budget_tokens: int):
-    """Oracle on whole users of the workload (fixed seeded sample), tokens/s."""
-    from oracle import hstu_oracle as O
+def blas_cores() -> int:
+    """Threads the oracle's BLAS calls use."""
     try:
         import threadpoolctl
         info = threadpoolctl.threadpool_info()
-        cores = max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
     except Exception:
-        cores = len(os.sched_getaffinity(0))
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline_stack(w, budget_tokens: int):
+    """Oracle on whole users of the workload (fixed seeded sample), tokens/s."""
+    from oracle import hstu_oracle as O
+    cores = blas_cores()
     order = np.random.default_rng(123).permutation(w.B)
     users, tok = [], 0
     for b in order:
@@ -320,6 +325,70 @@ def e2e_pipelined(torch, host_in, out_like, compute, steps, flush):
     return t0.elapsed_time(t1) / steps
 
 
+def time_leg(fn, args, flush, stream):
+    """Mean ms of one call of `fn` over args.steps timed calls (CUDA events on
+    `stream`, L2 flushed between calls, after args.warmup untimed ones), and
+    the library's per-kernel mean launch times from a second, traced pass."""
+    import torch
+    import hstu_sequential_transducer_layer_b200 as H
+    for _ in range(args.warmup):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    H.hstu_trace_enable(args.steps * 16 + 16)
+    for _ in range(args.steps):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    tr = H.hstu_trace_read()
+    H.hstu_trace_enable(0)
+    ker = {}
+    for kid, t in tr:
+        e = ker.setdefault(H.hstu_kernel_name(kid), [0, 0.0])
+        e[0] += 1
+        e[1] += t
+    return (sum(a.elapsed_time(b) for a, b in evs) / len(evs),
+            {k: round(v[1] / v[0], 4) for k, v in ker.items()})
+
+
+def cpu_baseline_extrapolated(w, budget_tokens: int, shortest: bool = False):
+    """The oracle on whole users of a one-layer workload (a seeded random
+    sample up to `budget_tokens`, or only the shortest user), its algorithmic
+    GFLOP/s, and the workload's tokens/s at that rate (the workload's FLOPs
+    divided by the oracle's FLOP rate): long users cost more per token, so
+    the sample's own tokens/s would not stand for the workload."""
+    from oracle import hstu_oracle as O
+    if shortest:
+        users = [int(np.argmin(w.lengths))]
+    else:
+        users, tok = [], 0
+        for b in np.random.default_rng(123).permutation(w.B):
+            users.append(int(b))
+            tok += int(w.lengths[b])
+            if tok >= budget_tokens:
+                break
+    lens = w.lengths[users]
+    t0 = time.perf_counter()
+    for b in users:
+        s, e = int(w.offsets[b]), int(w.offsets[b + 1])
+        O.stack_user(w.X[s:e], w.timestamps[s:e], w.weights, w.dims)
+    dt = time.perf_counter() - t0
+    f_sample = w.n_layers * sum(layer_flops(w.dims, lens).values())
+    f_all = w.n_layers * sum(layer_flops(w.dims, w.lengths).values())
+    rate = f_sample / dt
+    return {"value": w.T / (f_all / rate), "unit": "tokens/s", "cores": blas_cores(),
+            "kind": "oracle", "gflops": round(rate / 1e9, 3), "seconds": round(dt, 2),
+            "sample": f"{len(users)} whole user(s) ({int(lens.sum())} tokens) of the {w.name} "
+                      f"workload, numpy float64; tokens/s of the whole workload at the sample's "
+                      f"algorithmic FLOP rate"}
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -387,6 +456,17 @@ def run_ours(args):
     ms = sum(step_ms) / len(step_ms)
     if r.status() != 0:
         raise RuntimeError(f"device status {r.status()} after timing")
+    # the same steps again with no per-launch event pairs (they add a little
+    # to the headline steps above; this is the step time without them)
+    u_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    for a, b in u_evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    untraced_ms = sum(a.elapsed_time(b) for a, b in u_evs) / len(u_evs)
 
     # per-kernel device time inside the timed region
     per_kernel = {}
@@ -402,16 +482,18 @@ def run_ours(args):
         n, tot = per_kernel[dominant]
         avg_s = tot / n / 1e3
         achieved = kflops[dominant] / avg_s / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        # the timed region is a burst of well under a second at full clocks,
+        # so the denominator is the measured burst GEMM rate
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "peak_source": f"bf16_tflops_sustained ({peak_src})",
+                    "peak_source": f"bf16_tflops, burst ({peak_src})",
                     "traffic": ncu_traffic(dominant, w.name),
                     "avg_launch_ms": round(tot / n, 4),
-                    # the same achieved rate against the burst figure and the
-                    # nominal dense bf16 rate of the part (2.25 PFLOP/s)
-                    "frac_burst": round(achieved / float(peaks.get(
-                        "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 4),
+                    # the same achieved rate against the sustained figure and
+                    # the nominal dense bf16 rate of the part (2.25 PFLOP/s)
+                    "frac_sustained": round(achieved / float(peaks.get(
+                        "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])), 4),
                     "frac_nominal": round(achieved / 2250.0, 4)}
     step_flops = args_layers = w.n_layers * sum(flops.values())
     del args_layers
@@ -474,7 +556,10 @@ def run_ours(args):
         mf = {"value": C / (m_ms / 1e3), "unit": "candidates/s", "ms_per_step": round(m_ms, 4),
               "tflops": round(mflop / (m_ms / 1e3) / 1e12, 1),
               "tensor_frac": tensor_frac(mflop / (m_ms / 1e3) / 1e12, peaks),
-              "config": {"workload": "mfalcon", "users": wm.B, "candidates_per_user": wm.max_cands,
+              "config": {"workload": "mfalcon: M-FALCON ranking, 3-layer stack (d=512, 4 heads, "
+                                     "head dim 128), 32 users with 512-4096 history tokens, 1024 "
+                                     "candidates per user in microbatches of 256",
+                         "users": wm.B, "candidates_per_user": wm.max_cands,
                          "microbatch": wm.microbatch, "layers": wm.n_layers, "d_model": 512,
                          "heads": 4, "head_dim": 128, "history_tokens": wm.T}}
 
@@ -692,33 +777,10 @@ def run_ours(args):
         rt = H.TransformerRunner(512, 8, 2048, hw.transformer_weights(args.seed + rank, 512, 2048),
                                  device=dev)
 
-        def time_leg(fn):
-            for _ in range(args.warmup):
-                fn()
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-            for a, b in evs:
-                flush.zero_()
-                a.record(stream)
-                fn()
-                b.record(stream)
-            torch.cuda.synchronize()
-            H.hstu_trace_enable(args.steps * 16 + 16)
-            for _ in range(args.steps):
-                flush.zero_()
-                fn()
-            torch.cuda.synchronize()
-            tr = H.hstu_trace_read()
-            H.hstu_trace_enable(0)
-            ker = {}
-            for kid, t in tr:
-                e = ker.setdefault(H.hstu_kernel_name(kid), [0, 0.0])
-                e[0] += 1
-                e[1] += t
-            return (sum(a.elapsed_time(b) for a, b in evs) / len(evs),
-                    {k: round(v[1] / v[0], 4) for k, v in ker.items()})
-        h_ms, h_k = time_leg(lambda: rh.stack(c_off, c_x, c_ts, wl.max_len, out=c_yh))
-        t_ms, t_k = time_leg(lambda: rt.layer(c_off, c_x, wl.max_len, out=c_yt))
+        h_ms, h_k = time_leg(lambda: rh.stack(c_off, c_x, c_ts, wl.max_len, out=c_yh), args,
+                             flush, stream)
+        t_ms, t_k = time_leg(lambda: rt.layer(c_off, c_x, wl.max_len, out=c_yt), args, flush,
+                             stream)
         if rh.status() != 0 or rt.status() != 0:
             raise RuntimeError(f"comparator device status {rh.status()} / {rt.status()}")
         pairs = float((wl.lengths * (wl.lengths + 1) // 2).sum())
@@ -733,6 +795,39 @@ def run_ours(args):
                 "hstu_attention_tflops": round(attn_flops / (h_k.get("attn_tc", float("nan")) / 1e3)
                                                / 1e12, 1),
                 "note": "one layer each; the Transformer layer has an FFN (4d) and no rab"}
+
+    # ---------------- one-layer legs: the single-layer workload (64 users,
+    # lognormal lengths capped at 1024, d = 256, 4 heads, head dim 64) and the
+    # long-history workload as a layer on its own (16 users of 2,048-8,192
+    # tokens, d = 512, 8 heads, head dim 64)
+    legs = None
+    if not args.no_layer_legs:
+        legs = {}
+        for name, make, shortest in (("single_layer", hw.single_layer, False),
+                                     ("long_history", hw.long_history, True)):
+            wl = make(seed=args.seed + rank)
+            rl = H.HSTURunner(hw.dims_dict(wl.dims), wl.weights, dev)
+            l_in = (rl.to_device(wl.offsets, "i64"), rl.to_device(wl.X, "act"),
+                    rl.to_device(wl.timestamps, "i64"))
+            l_out = torch.empty_like(l_in[1])
+            l_ms, l_k = time_leg(lambda: rl.stack(l_in[0], l_in[1], l_in[2], wl.max_len,
+                                                  out=l_out), args, flush, stream)
+            if rl.status() != 0:
+                raise RuntimeError(f"{name} device status {rl.status()}")
+            lf = layer_flops(wl.dims, wl.lengths)
+            l_tf = sum(lf.values()) / (l_ms / 1e3) / 1e12
+            att = l_k.get("attn_tc")
+            legs[name] = {
+                "value": wl.T / (l_ms / 1e3), "unit": "tokens/s", "ms_per_step": round(l_ms, 4),
+                "tflops": round(l_tf, 1), "tensor_frac": tensor_frac(l_tf, peaks),
+                "attention_tflops": (round(lf["attn"] / (att / 1e3) / 1e12, 1) if att else None),
+                "kernels_ms": l_k,
+                "cpu_baseline": (None if (world > 1 or args.no_cpu_baseline) else
+                                 cpu_baseline_extrapolated(wl, args.cpu_tokens, shortest)),
+                "config": {"workload": name, "users": wl.B, "tokens": wl.T,
+                           "d_model": wl.dims.d_model, "heads": wl.dims.n_heads,
+                           "head_dim": wl.dims.d_qk, "max_len": wl.max_len}}
+            del rl, l_in, l_out
 
     # ---------------- reduce over ranks
     tokens = float(T)
@@ -763,6 +858,11 @@ def run_ours(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ret["ms_per_step"] = float(t[0])
             ret["value"] = world * ret["config"]["users"] * ret["config"]["items"] / (float(t[0]) / 1e3)
+        for leg in (legs or {}).values():
+            t = torch.tensor([leg["ms_per_step"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            leg["ms_per_step"] = float(t[0])
+            leg["value"] = world * leg["config"]["tokens"] / (float(t[0]) / 1e3)
         if sl is not None:
             t = torch.tensor([sl["ms_per_step"], rs.R, sl["config"]["kept_tokens"]],
                              dtype=torch.float64, device=dev)
@@ -775,6 +875,16 @@ def run_ours(args):
     line = None
     if rank == 0:
         cpu = None if (world > 1 or args.no_cpu_baseline) else cpu_baseline_stack(w, args.cpu_tokens)
+        if cpu is not None:
+            # the same oracle on one BLAS thread, on a smaller sample
+            try:
+                import threadpoolctl
+                with threadpoolctl.threadpool_limits(1):
+                    one = cpu_baseline_stack(w, max(1, args.cpu_tokens // 4))
+                cpu["one_thread"] = {"value": one["value"], "unit": "tokens/s", "cores": 1,
+                                     "sample": one["sample"]}
+            except Exception as exc:  # threadpoolctl absent: say so
+                cpu["one_thread"] = {"value": None, "note": f"not measured: {exc}"}
         line = {
             "metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
@@ -802,12 +912,16 @@ def run_ours(args):
                     "serial_ms_per_step": round(e2e_serial_ms, 4),
                     "serial_value": tokens / (e2e_serial_ms / 1e3)},
             "gpu_launches": int(n_launch),
+            "untraced_ms_per_step": round(untraced_ms, 4),
+            "untraced_value": tokens / (untraced_ms / 1e3),
             "clocks": clk.summary(),
-            "mfalcon": mf,
             "stochastic_length": sl,
             "full_pipeline": pipe,
             "retrieval": ret,
             "comparator": cmp_,
+            "layer_legs": legs,
+            # last key: the second half of the metric (candidates/s)
+            "mfalcon": mf,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -857,6 +971,7 @@ def main():
     ap.add_argument("--no-retrieval", action="store_true")
     ap.add_argument("--no-comparator", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layer-legs", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)
     args = ap.parse_args()

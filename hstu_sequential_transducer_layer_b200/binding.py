@@ -29,7 +29,8 @@ EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfa
             "hstu_retrieval_topk", "hstu_retrieval_fallback_taken",
             "hstu_transformer_workspace_size",
             "hstu_transformer_layer_fwd",
-            "hstu_read_status", "hstu_debug_offsets", "hstu_trace_enable", "hstu_trace_read",
+            "hstu_read_status", "hstu_debug_offsets", "hstu_debug_wait_test",
+            "hstu_trace_enable", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
 
 
@@ -112,6 +113,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_debug_offsets.argtypes = [pdesc, i64, i64, i64, ctypes.POINTER(sz),
                                      ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.hstu_debug_offsets.restype = i32
+    L.hstu_debug_wait_test.argtypes = [ctypes.c_uint32, i32]
+    L.hstu_debug_wait_test.restype = i32
     L.hstu_trace_enable.argtypes = [i32]
     L.hstu_trace_enable.restype = i32
     L.hstu_trace_read.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float), i32]
@@ -336,6 +339,11 @@ def hstu_debug_offsets(desc, B, total_tokens, max_len):
                                     ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
            "hstu_debug_offsets")
     return int(a.value), int(b.value), int(c.value)
+
+
+def hstu_debug_wait_test(wait_limit_us: int, inject_stall: int) -> None:
+    _check(lib().hstu_debug_wait_test(int(wait_limit_us), int(inject_stall)),
+           "hstu_debug_wait_test")
 
 
 def hstu_trace_enable(max_records: int) -> None:

@@ -67,6 +67,8 @@ struct AttnDev {
   int32_t* work_next;
   int32_t* work_done;
   int* status;
+  uint32_t wait_limit_us;      // bound of every in-kernel wait
+  int inject_stall;            // test hook: CTA 0 stops handing out work after two items
 };
 
 template <int D>
@@ -138,6 +140,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     *s_go = (st == 0);
     *s_nitems = *a.n_items;
     ab->flag = 0;
+    ab->limit_us = a.wait_limit_us;
     for (int i = 0; i < C::QS; ++i) {
       mbar_init(q_full + i, 1);
       mbar_init(q_empty + i, 1);
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         ++litem;
       }
       if (!ok) {  // let every load already in flight land before the CTA exits
-        AbortState tmp{0};
+        AbortState tmp{0, kWaitLimitUs};
         for (uint32_t s2 = 0; s2 < nst; ++s2)
           if ((issued >> s2) & 1u) mbar_wait(full + s2, (last_par >> s2) & 1u, &tmp, nullptr);
         for (int s2 = 0; s2 < C::QS; ++s2)
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       if (ok) flush();
       if (any) {
         tc_commit(drain);
-        AbortState tmp{0};
+        AbortState tmp{0, kWaitLimitUs};
         mbar_wait(drain, 0, &tmp, nullptr);
       }
     }
@@ -523,6 +526,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     // more than two unstarted items (a short tail at the end of the launch).
     uint32_t npub = 0;
     for (;;) {
+      // Test hook: CTA 0's fetcher stops after publishing two items, without
+      // the terminator, so every other role of this CTA waits for a third
+      // item that never comes; those bounded waits give up (HSTU_ERR_TIMEOUT)
+      // and the CTA winds down.  No load is skipped or left unwaited.
+      if (a.inject_stall && blockIdx.x == 0 && npub == 2) break;
       const int slot = npub & 1;
       bool okw = true;
       if (lane == 0) okw = mbar_wait(it_empty + slot, ((npub >> 1) & 1) ^ 1, ab, a.status);
@@ -691,12 +699,8 @@ static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tk
                                     cudaStream_t s) {
   using C = AttnCfg<D>;
   auto kfn = k_attn_tc<D, MODE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM);
+  if (e != cudaSuccess) return e;
   kfn<<<grid, C::THREADS, C::SMEM, s>>>(tq, tkv, to, ad);
   return cudaGetLastError();
 }
@@ -748,6 +752,7 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   ad.work_next = c.work_next;
   ad.work_done = c.work_done;
   ad.status = c.status;
+  take_wait_test(&ad.wait_limit_us, &ad.inject_stall);
   const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());
   LaunchScope ls(c.mode == MODE_SELF ? K_ATTN : K_ATTN_CAND, s);
   if (c.mode == MODE_SELF)

@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     *s_go = ((g.status == nullptr) || (*reinterpret_cast<volatile int*>(g.status) == 0)) &&
             (g.run_if == nullptr || *reinterpret_cast<volatile const int*>(g.run_if) != 0);
     ab->flag = 0;
+    ab->limit_us = kWaitLimitUs;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       if (!ok) {  // let every load already in flight land before the CTA exits
         for (int s = 0; s < STAGES; ++s)
           if ((issued >> s) & 1u) {
-            AbortState tmp{0};
+            AbortState tmp{0, kWaitLimitUs};
             mbar_wait(full + s, (last_par >> s) & 1u, &tmp, nullptr);
           }
       }
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       }
       if (issued_any) {
         tc_commit(drain);  // completes once every MMA issued above has finished
-        AbortState tmp{0};
+        AbortState tmp{0, kWaitLimitUs};
         mbar_wait(drain, 0, &tmp, nullptr);
       }
     }
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       if (lane == 0) mbar_arrive(tempty + acc);
     }
     if (lane == 0 && r_pending) {  // a residual load still in flight must land first
-      AbortState tmp{0};
+      AbortState tmp{0, kWaitLimitUs};
       mbar_wait(rb, rpar, &tmp, nullptr);
     }
     if (lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
@@ -449,12 +450,8 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
   using C = GemmCfg<BN, STAGES, EPI, COMPACT>;
   static_assert(C::SMEM <= 232448, "shared memory per CTA");
   auto kfn = k_gemm_tc<BN, STAGES, EPI, COMPACT>;
-  static bool attr_set = false;  // per instantiation; the attribute is per device function
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM);
+  if (e != cudaSuccess) return e;
   kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, to16, to32, tr, gd);
   return cudaGetLastError();
 }

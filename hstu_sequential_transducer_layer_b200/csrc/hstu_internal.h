@@ -63,6 +63,14 @@ struct LaunchScope {
 
 // ---------------------------------------------------------------- device info
 int num_sms();
+// Raises `fn`'s dynamic shared-memory limit to `bytes` on the current device
+// (once per kernel and device).
+cudaError_t ensure_smem_limit(const void* fn, int bytes);
+// Bound of an in-kernel wait unless a test asks for a shorter one.
+constexpr uint32_t kDefaultWaitLimitUs = 1000u * 1000u;
+// The wait bound and stall injection for the next attention launch
+// (hstu_debug_wait_test), reset to the defaults once taken.
+void take_wait_test(uint32_t* limit_us, int* inject_stall);
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).  Returns false if the driver call is unavailable/failed.
 // 2-D map of a row-major matrix with an explicit element type and swizzle.

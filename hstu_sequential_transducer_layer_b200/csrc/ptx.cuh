@@ -15,9 +15,10 @@
 
 namespace hstu {
 
-// A wait that has not completed after this many nanoseconds gives up, sets
-// the device status to HSTU_ERR_TIMEOUT and lets the kernel wind down.
-constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+// A wait that has not completed after this many microseconds (by default;
+// a kernel may set a shorter limit in its AbortState) gives up, sets the
+// device status to HSTU_ERR_TIMEOUT and lets the kernel wind down.
+constexpr uint32_t kWaitLimitUs = kDefaultWaitLimitUs;
 
 DEVI uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -59,7 +60,8 @@ DEVI bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Per-CTA failure state shared by all roles of a kernel.
 struct AbortState {
-  int flag;  // set once any wait of this CTA gave up
+  int flag;           // set once any wait of this CTA gave up
+  uint32_t limit_us;  // how long one wait may take before it gives up
 };
 
 DEVI void raise_status(int* status, int code) {
@@ -75,7 +77,7 @@ DEVI bool mbar_wait(uint64_t* bar, uint32_t parity, AbortState* ab, int* status)
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*((volatile int*)&ab->flag)) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > 1000ull * ab->limit_us) {
         *((volatile int*)&ab->flag) = 1;
         raise_status(status, HSTU_ERR_TIMEOUT);
         return false;
@@ -95,7 +97,7 @@ DEVI bool mbar_wait_warp(uint64_t* bar, uint32_t parity, AbortState* ab, int* st
       int give_up = 0;
       if (threadIdx.x % 32 == 0) {
         if (*((volatile int*)&ab->flag)) give_up = 1;
-        else if (global_timer_ns() - t0 > kWaitLimitNs) {
+        else if (global_timer_ns() - t0 > 1000ull * ab->limit_us) {
           *((volatile int*)&ab->flag) = 1;
           raise_status(status, HSTU_ERR_TIMEOUT);
           give_up = 1;

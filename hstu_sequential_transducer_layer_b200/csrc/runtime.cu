@@ -2,6 +2,8 @@
 // device queries, TMA descriptor encoding, and the workspace layout.
 #include <atomic>
 #include <mutex>
+#include <set>
+#include <utility>
 #include <vector>
 
 #include "hstu_internal.h"
@@ -44,6 +46,38 @@ LaunchScope::~LaunchScope() {
 }
 
 // ---------------------------------------------------------------- device
+// The dynamic shared-memory limit is an attribute of a kernel on one device:
+// it is raised once per (kernel, device) pair, under a lock, so the first
+// launch on a second GPU of the same process raises it there too.
+cudaError_t ensure_smem_limit(const void* fn, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_pair(fn, dev);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
+}
+
+// ---------------------------------------------------------------- wait test hook
+namespace {
+std::mutex g_wait_mu;
+uint32_t g_wait_limit_us = 0;  // 0: the default bound
+int g_inject_stall = 0;
+}  // namespace
+
+void take_wait_test(uint32_t* limit_us, int* inject_stall) {
+  std::lock_guard<std::mutex> lk(g_wait_mu);
+  *limit_us = g_wait_limit_us ? g_wait_limit_us : kDefaultWaitLimitUs;
+  *inject_stall = g_inject_stall;
+  g_wait_limit_us = 0;
+  g_inject_stall = 0;
+}
+
 int num_sms() {
   static int cached[64] = {0};
   int dev = 0;
@@ -170,6 +204,15 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
 
 // ---------------------------------------------------------------- C ABI
 extern "C" {
+
+hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall) {
+  if (inject_stall != 0 && inject_stall != 1) return HSTU_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(hstu::g_wait_mu);
+  hstu::g_wait_limit_us = wait_limit_us;
+  hstu::g_inject_stall = inject_stall;
+  return HSTU_OK;
+}
+
 
 hstu_status hstu_trace_enable(int32_t max_records) {
   using namespace hstu;

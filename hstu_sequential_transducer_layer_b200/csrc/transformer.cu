@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
     *s_go = (st == 0);
     *s_nitems = *a.n_items;
     ab->flag = 0;
+    ab->limit_us = kWaitLimitUs;
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + i, 1);
       mbar_init(q_empty + i, 1);
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
         if (!ok) break;
       }
       if (!ok) {  // let every load already in flight land before the CTA exits
-        AbortState tmp{0};
+        AbortState tmp{0, kWaitLimitUs};
         for (uint32_t s2 = 0; s2 < 2; ++s2) {
           if ((issued >> s2) & 1u) mbar_wait(full + s2, (last_par >> s2) & 1u, &tmp, nullptr);
           if ((q_issued >> s2) & 1u) mbar_wait(q_full + s2, (q_last >> s2) & 1u, &tmp, nullptr);
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(SmaxCfg<D>::THREADS, 1)
       if (ok) flush();
       if (any) {
         tc_commit(drain);
-        AbortState tmp{0};
+        AbortState tmp{0, kWaitLimitUs};
         mbar_wait(drain, 0, &tmp, nullptr);
       }
     }
@@ -527,13 +528,8 @@ template <int D>
 static cudaError_t launch_softmax_attn(const CUtensorMap& tm, const SoftmaxAttnDev& dev,
                                        cudaStream_t s) {
   using C = SmaxCfg<D>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_softmax_attn<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(k_softmax_attn<D>), C::SMEM);
+  if (e != cudaSuccess) return e;
   LaunchScope ls(K_TF_ATTN, s);
   k_softmax_attn<D><<<num_sms(), C::THREADS, C::SMEM, s>>>(tm, dev);
   return cudaGetLastError();

@@ -61,8 +61,14 @@
  *               candidate rows also keep an fp32 residual), and only the final
  *               output is rounded to bf16.  fp16 keeps 3 more mantissa bits than
  *               bf16 at the same tensor-core rate; inputs, weights and layer
- *               outputs must lie within fp16 range.  dtype HSTU_FP32: fp32 throughout (CUDA-core
- *               FMA).
+ *               outputs must lie within fp16 range (|x| <= 65504).  Weights
+ *               below 2^-14 in magnitude become fp16 subnormals (absolute
+ *               error up to 2^-25 each): against activations of order one
+ *               they stay within the bf16 bound (tested: W2 drawn from
+ *               N(0, 1e-5)); against activations in the thousands the error
+ *               they add grows with the activations and can exceed it (Q and
+ *               K rows of W1 near 1e-5 against activations of 8192 gave
+ *               2.3e-2).  dtype HSTU_FP32: fp32 throughout (CUDA-core FMA).
  *   Supported   bf16: d_qk = d_v in {64, 128}; d_model and h*d_v multiples
  *               of 64; bucket counts in [1, 4096].  fp32: d_qk, d_v <= 128
  *               and multiples of 4; d_model multiple of 4.
@@ -330,6 +336,21 @@ hstu_status hstu_trace_enable(int32_t max_records);
 int32_t hstu_trace_read(int32_t* kernel_ids, float* ms, int32_t capacity);
 const char* hstu_kernel_name(int32_t kernel_id);
 int64_t hstu_launch_count(void);
+
+/* Test hook for the failure detection of the in-kernel waits.  Every wait
+ * inside the attention kernel is bounded: after wait_limit_us microseconds
+ * (default 1 s) it gives up, the call's status word becomes HSTU_ERR_TIMEOUT,
+ * and the kernel winds down (loads in flight land, tensor memory is freed)
+ * and returns, so the context stays usable and the next call on the same
+ * workspace runs normally.  hstu_debug_wait_test sets, for the NEXT attention
+ * launch only (of any call, on any stream), the wait bound (0 = the default)
+ * and, with inject_stall = 1, makes that launch's first CTA stop handing out
+ * work after two items without telling its other roles, which then wait
+ * until the bound runs out.  It touches no memory and issues no load; the
+ * launch after that one uses the defaults again.  Not a page operation: the
+ * pages describe no failure handling.  Returns HSTU_ERR_INVALID_ARG for an
+ * inject_stall other than 0 or 1. */
+hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall);
 
 const char* hstu_status_string(hstu_status s);
 int32_t hstu_version(void);
