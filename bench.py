@@ -796,6 +796,35 @@ def run_ours(args):
                                                / 1e12, 1),
                 "note": "one layer each; the Transformer layer has an FFN (4d) and no rab"}
 
+    # ---------------- backward pass (training): hstu_stack_bwd over the same
+    # 8-layer full-stack batch, a bf16 output gradient resident in HBM
+    bwd = None
+    if not args.no_backward:
+        dYb = torch.randn(X.shape, generator=torch.Generator(device=dev).manual_seed(7),
+                          device=dev, dtype=torch.float32).to(torch.bfloat16)
+        b_dX = torch.empty_like(X)
+        b_grads = None
+
+        def bstep():
+            nonlocal b_grads
+            _, b_grads = r.stack_bwd(off, X, ts, dYb, w.max_len, dX=b_dX, grads=b_grads)
+        b_ms, b_k = time_leg(bstep, args, flush, stream)
+        if r.bwd_status() != 0:
+            raise RuntimeError(f"backward device status {r.bwd_status()}")
+        # algorithmic work of the gradients: twice the forward's products (the
+        # input-gradient and weight-gradient products of f1 and f2; dA, dV, dK
+        # and dQ against S and P.V in attention); the per-layer recompute of the
+        # forward is not counted
+        b_flops = 2.0 * step_flops
+        b_tf = b_flops / (b_ms / 1e3) / 1e12
+        bwd = {"value": T / (b_ms / 1e3), "unit": "tokens/s", "ms_per_step": round(b_ms, 4),
+               "tflops": round(b_tf, 1), "tensor_frac": tensor_frac(b_tf, peaks),
+               "kernels_ms": b_k,
+               "note": "gradients of every parameter and of the input, 8 layers; each layer's "
+                       "forward is recomputed inside the call (not counted in tflops)",
+               "config": {"workload": "full_stack backward", "layers": w.n_layers,
+                          "tokens": T}}
+
     # ---------------- one-layer legs: the single-layer workload (64 users,
     # lognormal lengths capped at 1024, d = 256, 4 heads, head dim 64) and the
     # long-history workload as a layer on its own (16 users of 2,048-8,192
@@ -858,6 +887,11 @@ def run_ours(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ret["ms_per_step"] = float(t[0])
             ret["value"] = world * ret["config"]["users"] * ret["config"]["items"] / (float(t[0]) / 1e3)
+        if bwd is not None:
+            t = torch.tensor([bwd["ms_per_step"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            bwd["ms_per_step"] = float(t[0])
+            bwd["value"] = world * T / (float(t[0]) / 1e3)
         for leg in (legs or {}).values():
             t = torch.tensor([leg["ms_per_step"]], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -920,6 +954,7 @@ def run_ours(args):
             "retrieval": ret,
             "comparator": cmp_,
             "layer_legs": legs,
+            "backward": bwd,
             # last key: the second half of the metric (candidates/s)
             "mfalcon": mf,
         }
@@ -959,6 +994,51 @@ def run_reference(args):
     return line
 
 
+def run_leg(args):
+    """One workload alone, W untimed and K timed calls, for profilers: prints
+    one small JSON line (not the bench line).  Legs: full_stack (the 8-layer
+    stack), long_history / single_layer (one layer), mfalcon (ranking),
+    backward (the 8-layer stack's backward pass)."""
+    import torch
+    import hstu_workloads as hw
+    import hstu_sequential_transducer_layer_b200 as H
+    from hstu_sequential_transducer_layer_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    make = {"full_stack": hw.full_stack, "long_history": hw.long_history,
+            "single_layer": hw.single_layer, "mfalcon": hw.mfalcon,
+            "backward": hw.full_stack}[args.leg]
+    w = make(seed=args.seed)
+    r = H.HSTURunner(hw.dims_dict(w.dims), w.weights, dev)
+    off, X, ts = r.to_device(w.offsets, "i64"), r.to_device(w.X), r.to_device(w.timestamps, "i64")
+    out = torch.empty_like(X)
+    if args.leg == "mfalcon":
+        co, cx, hv = r.to_device(w.cand_offsets, "i64"), r.to_device(w.candidates), r.to_device(w.head_vec)
+        sc = torch.empty(w.candidates.shape[0], dtype=torch.float32, device=dev)
+        fn = lambda: r.rank(off, X, ts, co, cx, None, w.microbatch, hv, w.max_len, w.max_cands,
+                            scores=sc)
+    elif args.leg == "backward":
+        dY = torch.randn(X.shape, device=dev).to(torch.bfloat16)
+        fn = lambda: r.stack_bwd(off, X, ts, dY, w.max_len)
+    else:
+        fn = lambda: r.stack(off, X, ts, w.max_len, out=out)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    st = r.bwd_status() if args.leg == "backward" else r.status()
+    print(json.dumps({"leg": args.leg, "ms_per_call": e0.elapsed_time(e1) / args.steps,
+                      "status": st}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -972,10 +1052,16 @@ def main():
     ap.add_argument("--no-comparator", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-legs", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)
+    ap.add_argument("--leg", default=None,
+                    choices=["full_stack", "long_history", "single_layer", "mfalcon", "backward"],
+                    help="run one workload alone (for profilers) instead of the bench line")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.leg:
+        run_leg(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

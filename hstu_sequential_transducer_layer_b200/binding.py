@@ -24,14 +24,17 @@ STATUS_NAMES = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTE
 
 # Every symbol include/hstu.h declares.
 EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfalcon_rank",
+            "hstu_bwd_workspace_size", "hstu_layer_bwd", "hstu_stack_bwd",
             "hstu_layer_fwd_noalloc", "hstu_sl_embed_workspace_size", "hstu_sl_embed",
             "hstu_sl_keep_count", "hstu_bf16_to_f16", "hstu_retrieval_workspace_size",
             "hstu_retrieval_topk", "hstu_retrieval_fallback_taken",
             "hstu_transformer_workspace_size",
             "hstu_transformer_layer_fwd",
-            "hstu_read_status", "hstu_debug_offsets", "hstu_debug_wait_test",
+            "hstu_read_status", "hstu_debug_offsets", "hstu_debug_keep_z",
+            "hstu_debug_wait_test",
             "hstu_trace_enable", "hstu_trace_read",
-            "hstu_kernel_name", "hstu_launch_count", "hstu_status_string", "hstu_version"]
+            "hstu_kernel_name", "hstu_launch_count", "hstu_last_error", "hstu_status_string",
+            "hstu_version"]
 
 
 class HstuError(RuntimeError):
@@ -54,6 +57,13 @@ class LayerWeights(ctypes.Structure):
                 ("ln_beta", ctypes.c_void_p), ("rab_pos", ctypes.c_void_p),
                 ("rab_time", ctypes.c_void_p), ("W1_f16", ctypes.c_void_p),
                 ("W2_f16", ctypes.c_void_p)]
+
+
+GRAD_KEYS = ("dW1", "db1", "dW2", "db2", "dln_gamma", "dln_beta", "drab_pos", "drab_time")
+
+
+class LayerGrads(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in GRAD_KEYS]
 
 
 class TransformerWeights(ctypes.Structure):
@@ -85,6 +95,13 @@ def lib() -> ctypes.CDLL:
     L.hstu_mfalcon_rank.argtypes = [pdesc, i32, pw, i64, i64, i64, vp, vp, vp, i64, i64, vp, vp,
                                     vp, i32, vp, vp, vp, sz, vp]
     L.hstu_mfalcon_rank.restype = i32
+    pg = ctypes.POINTER(LayerGrads)
+    L.hstu_bwd_workspace_size.argtypes = [pdesc, i32, i64, i64, i64]
+    L.hstu_bwd_workspace_size.restype = sz
+    L.hstu_layer_bwd.argtypes = [pdesc, pw, i64, i64, i64, vp, vp, vp, vp, vp, pg, vp, sz, vp]
+    L.hstu_layer_bwd.restype = i32
+    L.hstu_stack_bwd.argtypes = [pdesc, i32, pw, i64, i64, i64, vp, vp, vp, vp, vp, pg, vp, sz, vp]
+    L.hstu_stack_bwd.restype = i32
     L.hstu_layer_fwd_noalloc.argtypes = [pdesc, i64, i64, i64, vp, vp, pw, vp, vp, vp]
     L.hstu_layer_fwd_noalloc.restype = i32
     L.hstu_sl_embed_workspace_size.argtypes = []
@@ -113,6 +130,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_debug_offsets.argtypes = [pdesc, i64, i64, i64, ctypes.POINTER(sz),
                                      ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.hstu_debug_offsets.restype = i32
+    L.hstu_debug_keep_z.argtypes = [i32]
+    L.hstu_debug_keep_z.restype = i32
     L.hstu_debug_wait_test.argtypes = [ctypes.c_uint32, i32]
     L.hstu_debug_wait_test.restype = i32
     L.hstu_trace_enable.argtypes = [i32]
@@ -123,6 +142,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_kernel_name.restype = ctypes.c_char_p
     L.hstu_launch_count.argtypes = []
     L.hstu_launch_count.restype = i64
+    L.hstu_last_error.argtypes = []
+    L.hstu_last_error.restype = ctypes.c_char_p
     L.hstu_status_string.argtypes = [i32]
     L.hstu_status_string.restype = ctypes.c_char_p
     L.hstu_version.argtypes = []
@@ -155,6 +176,8 @@ def _nbytes(t) -> int:
 
 def _check(code: int, where: str) -> None:
     if code != 0:
+        if code == 4:  # HSTU_ERR_CUDA: name the failing runtime call
+            where = f"{where} ({lib().hstu_last_error().decode()})"
         raise HstuError(code, where)
 
 
@@ -317,6 +340,42 @@ def hstu_stack_fwd(desc, n_layers, weights, B, total_tokens, max_len, offsets, X
            "hstu_stack_fwd")
 
 
+def grads_array(gs: Sequence[Dict[str, object]]):
+    """LayerGrads array from per-layer dicts of fp32 device tensors."""
+    arr = (LayerGrads * len(gs))()
+    for i, g in enumerate(gs):
+        arr[i] = LayerGrads(*[_ptr(g[k]) for k in GRAD_KEYS])
+    return arr
+
+
+def hstu_bwd_workspace_size(desc: LayerDesc, n_layers: int, B: int, total_tokens: int,
+                            max_len: int) -> int:
+    n = int(lib().hstu_bwd_workspace_size(ctypes.byref(desc), n_layers, B, total_tokens, max_len))
+    if n == 0:
+        raise HstuError(1, "hstu_bwd_workspace_size")
+    return n
+
+
+def hstu_layer_bwd(desc, weights, B, total_tokens, max_len, offsets, X, timestamps, dY, dX,
+                   grads, workspace, stream=None) -> None:
+    w = weights if isinstance(weights, LayerWeights) else weights_struct(weights)
+    g = grads if not isinstance(grads, (list, tuple)) else grads_array(grads)
+    _check(lib().hstu_layer_bwd(ctypes.byref(desc), ctypes.byref(w), B, total_tokens, max_len,
+                                _ptr(offsets), _ptr(X), _ptr(timestamps), _ptr(dY), _ptr(dX), g,
+                                _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "hstu_layer_bwd")
+
+
+def hstu_stack_bwd(desc, n_layers, weights, B, total_tokens, max_len, offsets, X, timestamps, dY,
+                   dX, grads, workspace, stream=None) -> None:
+    arr = weights if not isinstance(weights, (list, tuple)) else weights_array(weights)
+    g = grads if not isinstance(grads, (list, tuple)) else grads_array(grads)
+    _check(lib().hstu_stack_bwd(ctypes.byref(desc), n_layers, arr, B, total_tokens, max_len,
+                                _ptr(offsets), _ptr(X), _ptr(timestamps), _ptr(dY), _ptr(dX), g,
+                                _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "hstu_stack_bwd")
+
+
 def hstu_mfalcon_rank(desc, n_layers, weights, B, total_hist, max_len, hist_offsets, history,
                       hist_timestamps, total_cands, max_cands, cand_offsets, candidates,
                       request_ts, microbatch, head_vec, scores, workspace, stream=None) -> None:
@@ -339,6 +398,10 @@ def hstu_debug_offsets(desc, B, total_tokens, max_len):
                                     ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
            "hstu_debug_offsets")
     return int(a.value), int(b.value), int(c.value)
+
+
+def hstu_debug_keep_z(on: bool) -> None:
+    _check(lib().hstu_debug_keep_z(1 if on else 0), "hstu_debug_keep_z")
 
 
 def hstu_debug_wait_test(wait_limit_us: int, inject_stall: int) -> None:

@@ -25,7 +25,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libhstu.so")
 
 SOURCES = ["runtime.cu", "api.cu", "sched.cu", "gemm_tc.cu", "attn_tc.cu", "simt_f32.cu",
-           "noalloc.cu", "sl.cu", "retrieval.cu", "transformer.cu"]
+           "noalloc.cu", "sl.cu", "retrieval.cu", "transformer.cu", "attn_bwd.cu", "bwd.cu"]
 HEADERS = [os.path.join(CSRC, "ptx.cuh"), os.path.join(CSRC, "hstu_internal.h"),
            os.path.join(INCLUDE, "hstu.h")]
 

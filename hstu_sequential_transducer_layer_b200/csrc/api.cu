@@ -171,11 +171,30 @@ cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const LayerOps& op
 // the caller's bf16 output when out16_bf16) and out32 (fp32 stream) may each
 // be null.  Each output element is read (residual) before it is written, by
 // the same warp, so a stream may be updated in place.
+// On the tensor-core path f2's A operand is LayerNorm(O) * U, built by the
+// GEMM itself from the attention's normalised O and statistics (`Z` is then
+// the normalised O, `ostats` its statistics, `f1` the layer's f1 output whose
+// first h*d_v columns are U, `z_dbg` an optional copy of Z); on the fp32 path
+// `Z` is the LayerNorm * U output.
 cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, const void* Z,
+                   const float* ostats, const void* f1, void* z_dbg,
                    const void* resid, int resid_kind, int64_t rows_cap, const int64_t* rows_dev,
                    void* out16, bool out16_bf16, float* out32) {
   GemmCall g{};
   g.A = Z;
+  if (c.bf16) {
+    g.A = nullptr;
+    g.ln_x = Z;
+    g.ln_stats = ostats;
+    g.ln_u = f1;
+    g.ld_u = c.F;
+    g.ln_gamma = w.ln_gamma;
+    g.ln_beta = w.ln_beta;
+    g.ln_eps = c.d.ln_eps;
+    g.ln_h = c.d.n_heads;
+    g.ln_dv = c.d.d_v;
+    g.z_dbg = z_dbg;
+  }
   g.lda = c.hdv;
   g.W = ops.W2;
   g.ldw = c.hdv;
@@ -251,18 +270,25 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
   a.t_rel = at<int32_t>(ws, L.t_rel);
   a.tbuckets = at<uint32_t>(ws, L.tbuckets);
   a.O = at<void>(ws, L.o);
+  a.ostats = c.bf16 ? at<float>(ws, L.ostats) : nullptr;
   e = attn(c, a);
   if (e != cudaSuccess) return e;
+  if (c.bf16)  // LayerNorm * U inside f2's operand stage
+    return run_f2(c, w, ops, at<void>(ws, L.o), at<float>(ws, L.ostats), f1,
+                  keep_z() ? at<void>(ws, L.z) : nullptr, resid, resid_kind, T, nullptr, out16,
+                  out16_bf16, out32);
   e = launch_ln_gate(c.d.dtype, at<void>(ws, L.o), f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps,
                      at<void>(ws, L.z), c.hdv, T, nullptr, c.status, c.s);
   if (e != cudaSuccess) return e;
-  return run_f2(c, w, ops, at<void>(ws, L.z), resid, resid_kind, T, nullptr, out16, out16_bf16,
-                out32);
+  return run_f2(c, w, ops, at<void>(ws, L.z), nullptr, nullptr, nullptr, resid, resid_kind, T,
+                nullptr, out16, out16_bf16, out32);
 }
 
 hstu_status finish(cudaError_t e) {
-  if (e != cudaSuccess) return HSTU_ERR_CUDA;
-  return cudaPeekAtLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  if (e == cudaSuccess) e = cudaPeekAtLastError();
+  if (e == cudaSuccess) return HSTU_OK;
+  note_cuda_error(e, "forward");
+  return HSTU_ERR_CUDA;
 }
 
 hstu_status stack_impl(const hstu_layer_desc* desc, int32_t n_layers,
@@ -447,15 +473,21 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
       a.t_rel = at<int32_t>(ws, L.t_rel);
       a.t_req_rel = t_req_rel;
       a.O = oc;
+      a.ostats = c.bf16 ? at<float>(ws, L.ostats_c) : nullptr;
       e = attn(c, a);
-      if (e != cudaSuccess) break;
-      e = launch_ln_gate(desc->dtype, oc, f1c, c.F, weights[l].ln_gamma, weights[l].ln_beta,
-                         desc->ln_eps, zc, c.hdv, R, rows_dev, c.status, c.s);
       if (e != cudaSuccess) break;
       const void* resid = first ? xb_c : (const void*)xres_c;
       void* o16 = (c.bf16 && !last) ? xh_c : nullptr;
-      e = run_f2(c, weights[l], ops, zc, resid, first ? RESID_BF16 : RESID_F32, R, rows_dev, o16,
-                 false, xres_c);
+      if (c.bf16) {  // LayerNorm * U inside f2's operand stage
+        e = run_f2(c, weights[l], ops, oc, at<float>(ws, L.ostats_c), f1c, nullptr, resid,
+                   first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);
+        continue;
+      }
+      e = launch_ln_gate(desc->dtype, oc, f1c, c.F, weights[l].ln_gamma, weights[l].ln_beta,
+                         desc->ln_eps, zc, c.hdv, R, rows_dev, c.status, c.s);
+      if (e != cudaSuccess) break;
+      e = run_f2(c, weights[l], ops, zc, nullptr, nullptr, nullptr, resid,
+                 first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);
     }
     if (e == cudaSuccess)
       e = launch_score(desc->dtype, xres_c, desc->d_model, head_vec, cand_offsets, mb_off, B, k,

@@ -26,8 +26,10 @@
 // bias, apply SiLU, mask, round to fp16 and write P back into TMEM (two
 // buffers), from where the P.V MMA reads its A operand; warps 20-23 (one per
 // lane quarter) read O at the end of an item, scale by 1/n (and, for
-// candidates, add the self term) and store fp32 through TMA bulk stores while
-// the P warps already work on the next item.  Sixteen P warps with little
+// candidates, add the self term), and store its mean and deviation per
+// (row, head) and the normalised values in fp16 through TMA bulk stores
+// (the statistics let the output projection apply LayerNorm without another
+// pass over O) while the P warps already work on the next item.  Sixteen P warps with little
 // state each hide the latency of the bias look-ups better than fewer warps
 // with more registers; every role fits in 80 registers.
 // Bias per element (causal self-attention): the position bias comes from a
@@ -62,11 +64,18 @@ struct AttnDev {
   int q_col, k_col, v_col;
   const __half* q_buf;         // for the candidate self term (fp16 f1 output)
   int64_t ld_f1;
-  float* O;                    // fp32: LayerNorm's mean subtraction would amplify rounding
+  // O of each (row, head), stored as its mean m and standard deviation s over
+  // the head's D values (fp32, [rows, h]) and the normalised values
+  // (O - m) / s in fp16 ([rows, ldo]).  LayerNorm subtracts a mean that is
+  // most of O's magnitude; normalised values keep fp16's relative precision
+  // for what remains, and the statistics give LayerNorm's row moments exactly.
+  __half* O;
   int64_t ldo;
+  float2* ostats;
   int32_t* work_next;
   int32_t* work_done;
   int* status;
+  int h;                       // heads (row stride of ostats)
   uint32_t wait_limit_us;      // bound of every in-kernel wait
   int inject_stall;            // test hook: CTA 0 stops handing out work after two items
 };
@@ -386,6 +395,41 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const float* rt_ring = reinterpret_cast<const float*>(smem + C::RT_OFF);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t scount = 0, ncon = 0;
+    uint32_t wt = 0;           // tiles this warp has started: window buffer parity
+    bool have_next = false;    // bw and window (wt & 1) already hold this item's tile 0
+    // Bias inputs of KV tile jt of item `it` into window buffer `buf` (and,
+    // causal mode, the tile's time-bucket words into bo).  Causal mode: the
+    // warp's 32 x 32 block spans the 63 distances base .. base + 62.
+    auto prep = [&](const AttnItem& it, int jt, int buf, uint32_t (&bo)[8]) {
+      float* win = win2 + buf * 64;
+      const float* Rp = a.rab_pos + (size_t)it.head * a.Np;
+      if (MODE == MODE_SELF) {
+        const uint32_t* tbw = a.tbuckets + (size_t)(it.tile0 + jt) * kBucketTileWords +
+                              (g * 8) * 128 + r;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) bo[m] = __ldg(tbw + m * 128);
+        const int base = (it.qt - jt) * 128 + q * 32 - g * 32 - 31;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int k = lane + 32 * u;
+          if (k < 63) {
+            const int dist = base + k;
+            win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
+          }
+        }
+      } else {
+        const float* Rt = a.rab_time + (size_t)it.head * a.Nt;
+        const int jc = jt * 128 + g * 32 + lane;
+        float bias = 0.f;
+        if (jc < it.n_kv) {
+          const int gap = max(a.t_req_rel[it.b] - a.t_rel[(int64_t)it.kv_row0 + jc], 0);
+          bias = __ldg(Rp + log_bucket(it.n_kv - jc, a.Sp, a.Np)) +
+                 __ldg(Rt + log_bucket(gap, a.St, a.Nt));
+        }
+        win[lane] = 0.5f * bias;
+      }
+    };
+    uint32_t bw[8], bwn[8];
     for (;;) {
       const int slot = ncon & 1;
       if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
@@ -397,47 +441,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         if (lane == 0) mbar_arrive(it_empty + slot);
         break;
       }
-      const int64_t kv0 = w.kv_row0;
       const int n_kv = w.n_kv;                   // history / sequence length
-      const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
-      const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
-      const int t_i = (MODE == MODE_SELF) ? 0 : a.t_req_rel[w.b];
-      // Bias inputs of KV tile jt into window buffer `buf` (and, causal mode,
-      // the tile's time-bucket words into bwn).  Causal mode: the warp's
-      // 32 x 32 block spans the 63 distances base .. base + 62.
-      auto prep = [&](int jt, int buf, uint32_t (&bwn)[8]) {
-        float* win = win2 + buf * 64;
-        if (MODE == MODE_SELF) {
-          const uint32_t* tbw = a.tbuckets + (size_t)(w.tile0 + jt) * kBucketTileWords +
-                                (g * 8) * 128 + r;
-#pragma unroll
-          for (int m = 0; m < 8; ++m) bwn[m] = __ldg(tbw + m * 128);
-          const int base = (w.qt - jt) * 128 + q * 32 - g * 32 - 31;
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int k = lane + 32 * u;
-            if (k < 63) {
-              const int dist = base + k;
-              win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
-            }
-          }
-        } else {
-          const int jc = jt * 128 + g * 32 + lane;
-          float bias = 0.f;
-          if (jc < n_kv) {
-            const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
-            bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
-                   __ldg(Rt + log_bucket(gap, a.St, a.Nt));
-          }
-          win[lane] = 0.5f * bias;
-        }
-      };
-      uint32_t bw[8], bwn[8];
-      if (w.nkv > 0) prep(0, 0, bw);
+      if (w.nkv > 0 && !have_next) prep(w, 0, wt & 1, bw);
+      have_next = false;
       bool alive = true;
-      for (int j = 0; j < w.nkv; ++j) {
+      for (int j = 0; j < w.nkv; ++j, ++wt) {
         __syncwarp();  // this tile's window is written; the one before it is free
-        const float* win = win2 + (j & 1) * 64;
+        const float* win = win2 + (wt & 1) * 64;
         // ---- S tile from TMEM: this warp's 32 rows x 32 columns
         const int sb = scount & 1;
         if (!mbar_wait_warp(s_full + sb, (scount >> 1) & 1, ab, a.status)) {
@@ -447,8 +457,21 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         tc_fence_after();
         uint32_t sr[32];
         tmem_ld32(tmem + sb * 128 + g * 32 + lane_base, sr);
-        // fetch the next tile's bias inputs while this tile computes
-        if (j + 1 < w.nkv) prep(j + 1, (j + 1) & 1, bwn);
+        // fetch the next tile's bias inputs while this tile computes -- at the
+        // item's last tile, those of the next item's first tile if the fetcher
+        // has published it already
+        if (j + 1 < w.nkv) {
+          prep(w, j + 1, (wt + 1) & 1, bwn);
+        } else {
+          const int ns = ncon & 1;
+          if (__all_sync(0xffffffffu, mbar_try_wait(it_full + ns, (ncon >> 1) & 1))) {
+            const AttnItem wn = ring[ns];
+            if (wn.b >= 0 && wn.nkv > 0) {
+              prep(wn, 0, (wt + 1) & 1, bwn);
+              have_next = true;
+            }
+          }
+        }
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -615,9 +638,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int ob = litem & 1;
       if (!mbar_wait_warp(o_full + ob, (litem >> 1) & 1, ab, a.status)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int c16 = 0; c16 < D / 16; ++c16) {
-        float o[16];
+      // O of this row and head, 16 columns from c16 * 16: the accumulator (or
+      // zero), plus the candidate's self term, times 1/n
+      auto load_o = [&](int c16, float (&o)[16]) {
         if (w.nkv > 0) {
           uint32_t orr[16];
           tmem_ld16(tmem + C::O_COL + ob * D + c16 * 16 + lane_base, orr);
@@ -627,11 +650,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) o[i] = 0.f;
-        }
-        if (c16 == D / 16 - 1) {  // O is fully read: the next item may accumulate
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free + ob);
         }
         if (MODE == MODE_CAND && row_ok) {
           const uint4* vp = reinterpret_cast<const uint4*>(rowp + a.v_col + w.head * D + c16 * 16);
@@ -646,28 +664,67 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             }
           }
         }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] *= inv_n;
+      };
+      // pass 1: mean and deviation of the row's D values, from sums shifted
+      // by the first value (no cancellation when the mean dominates)
+      float shift = 0.f, s1 = 0.f, s2 = 0.f;
+#pragma unroll 1
+      for (int c16 = 0; c16 < D / 16; ++c16) {
+        float o[16];
+        load_o(c16, o);
+        if (c16 == 0) shift = o[0];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float dv = o[i] - shift;
+          s1 += dv;
+          s2 = fmaf(dv, dv, s2);
+        }
+      }
+      const float mean = shift + s1 * (1.0f / D);
+      const float sd = sqrtf(fmaxf(s2 - s1 * s1 * (1.0f / D), 0.f) * (1.0f / D));
+      const float inv_sd = sd > 0.f ? 1.0f / sd : 0.f;
+      if (row_ok) a.ostats[(q0 + r) * a.h + w.head] = make_float2(mean, sd);
+      // pass 2: (O - mean) / sd in fp16, 32 columns per store -- a full
+      // 32-row block through swizzled staging and a TMA bulk store, a block
+      // at the user's ragged end row by row (the rows after it belong to the
+      // next user)
+#pragma unroll 1
+      for (int c32 = 0; c32 < D / 32; ++c32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float o[16];
+          load_o(c32 * 2 + hf, o);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[hf * 8 + i] = pack_f16x2_sat((o[2 * i] - mean) * inv_sd, (o[2 * i + 1] - mean) * inv_sd);
+        }
+        if (c32 == D / 32 - 1) {  // O is fully read: the next item may accumulate
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free + ob);
+        }
         if (full_rows) {
           uint8_t* buf = stg + (nbuf & 1) * 2048;
           if (lane == 0) bulk_wait_read<1>();  // the store two blocks back has read `buf`
           __syncwarp();
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<float4*>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
-                make_float4(o[4 * k] * inv_n, o[4 * k + 1] * inv_n, o[4 * k + 2] * inv_n,
-                            o[4 * k + 3] * inv_n);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmO, w.head * D + c16 * 16, (int)(q0 + q * 32), buf);
+            tma_store_2d(&tmO, w.head * D + c32 * 32, (int)(q0 + q * 32), buf);
             bulk_commit();
           }
           ++nbuf;
         } else if (row_ok) {
-          float4* op = reinterpret_cast<float4*>(a.O + (q0 + r) * a.ldo + w.head * D + c16 * 16);
+          uint4* op = reinterpret_cast<uint4*>(a.O + (q0 + r) * a.ldo + w.head * D + c32 * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            op[i] = make_float4(o[4 * i] * inv_n, o[4 * i + 1] * inv_n, o[4 * i + 2] * inv_n,
-                                o[4 * i + 3] * inv_n);
+          for (int k = 0; k < 4; ++k) op[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
       ++litem;
@@ -721,11 +778,12 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   } else {
     tkv = tq;
   }
-  // O: fp32 [q_rows_cap, h * d_v] with row stride ldo; 16-column x 32-row
-  // boxes (64-byte rows) for the epilogue's bulk stores.
+  // normalised O: fp16 [q_rows_cap, h * d_v] with row stride ldo; 32-column
+  // x 32-row boxes (64-byte rows) for the epilogue's bulk stores.
+  if (!c.ostats || c.ldo % 8 != 0) return cudaErrorInvalidValue;
   CUtensorMap to;
   if (!encode_tmap_2d_ex(&to, c.O, (uint64_t)c.q_rows_cap, (uint64_t)c.h * c.dv,
-                         (uint64_t)c.ldo * 4, 16, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                         (uint64_t)c.ldo * 2, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                          CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   AttnDev ad;
@@ -747,8 +805,10 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   ad.v_col = c.v_col;
   ad.q_buf = static_cast<const __half*>(c.q_buf);
   ad.ld_f1 = c.ld_f1;
-  ad.O = static_cast<float*>(c.O);
+  ad.O = static_cast<__half*>(c.O);
   ad.ldo = c.ldo;
+  ad.ostats = reinterpret_cast<float2*>(c.ostats);
+  ad.h = c.h;
   ad.work_next = c.work_next;
   ad.work_done = c.work_done;
   ad.status = c.status;

@@ -48,6 +48,21 @@ struct GemmDev {
   int* cand_cnt;
   int cand_cap;
   int* overflow;
+  // LNA: the A operand is LayerNorm(O) * U, built in shared memory
+  const __half* ln_x;          // normalised O [M, K] fp16: (O - m) / s per (row, head)
+  const float2* ln_stats;      // [M, ln_h] (m, s) per (row, head)
+  const __half* ln_u;          // U: the first K columns of the f1 output, row stride ld_u
+  int64_t ld_u;
+  const __nv_bfloat16* ln_gamma;
+  const __nv_bfloat16* ln_beta;
+  float ln_eps;
+  int ln_h, ln_dv;
+  __half* z_dbg;               // optional: Z [M, K] fp16, written by the CTAs of n-tile 0
+  // split-K: the K blocks are cut into `splits` ranges of kb_split blocks;
+  // split s stores its partial product at output rows s * split_rows + m
+  int splits, kb_split;
+  int64_t split_rows;
+  int has_pre;                 // EPI_SILU: also store the pre-activation (16-bit, tmO32)
 };
 
 constexpr int kEpiThreads = 256;      // 8 epilogue warps
@@ -55,12 +70,18 @@ constexpr uint32_t kStageBuf = 4096;  // per-warp output staging bytes (32 x 32 
 
 // COMPACT (EPI_RESID with 16-bit residual and output only): 2 KB output and
 // 2 KB residual buffers per epilogue warp, leaving room for one more A/B stage.
-template <int BN, int STAGES, int EPI, int COMPACT>
+// LNA: TMA brings the normalised attention output (as A) and U; the epilogue
+// warps turn A into LayerNorm(O) * U in place before the MMAs read it.
+template <int BN, int STAGES, int EPI, int COMPACT, int LNA = 0>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
-  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  // LNA: each stage also holds the U tile; A arrives as the normalised O and
+  // is turned into Z in place
+  static constexpr uint32_t U_BYTES = LNA ? A_BYTES : 0;
+  static constexpr uint32_t B_OFF = A_BYTES + U_BYTES;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + U_BYTES + B_BYTES;
   static constexpr uint32_t BUF = COMPACT ? 2048 : kStageBuf;         // per-warp buffers
   static constexpr uint32_t OUT_OFF = STAGES * STAGE_BYTES;             // 8 output staging buffers
   // EPI_RESID: 8 buffers that TMA fills with the next residual chunk
@@ -68,7 +89,10 @@ struct GemmCfg {
   static constexpr uint32_t BAR_OFF = RES_OFF + (EPI == EPI_RESID ? (kEpiThreads / 32) * BUF : 0);
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr int THREADS = 64 + kEpiThreads;
 };
+
+
 
 // Applies the epilogue to one 32-column chunk of this thread's row and stores
 // the warp's 32 x 32 tile: the fp32 copy through a 128-byte-swizzled buffer
@@ -94,6 +118,28 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   if (EPI == EPI_SCORE) {
     if (col >= g.N) return false;  // a chunk past the last item: nothing to store
   } else if (EPI == EPI_SILU) {
+    if (g.has_pre) {
+      // the pre-activation X W^T + b through the first 2 KB of the warp's
+      // buffer (16-bit, 64-byte swizzle), then SiLU through the second
+      if (__shfl_sync(0xffffffffu, valid ? 1 : 0, 0) == 0) return false;
+      if (lane == 0) bulk_wait_read<1>();  // the pre store before the last one has read it
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint4 o;
+        o.x = pack16(g.out_f16, v[k * 8 + 0], v[k * 8 + 1]);
+        o.y = pack16(g.out_f16, v[k * 8 + 2], v[k * 8 + 3]);
+        o.z = pack16(g.out_f16, v[k * 8 + 4], v[k * 8 + 5]);
+        o.w = pack16(g.out_f16, v[k * 8 + 6], v[k * 8 + 7]);
+        *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = o;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmO32, col, y0, stage);
+        bulk_commit();
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = silu_accurate(v[i]);
   } else if (EPI == EPI_BIAS) {
@@ -116,8 +162,14 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
       const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        v[k * 8 + 2 * m] += lo16(f16, rw[m]);
-        v[k * 8 + 2 * m + 1] += hi16(f16, rw[m]);
+        if (f16) {  // packed conversion of the pair
+          const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&rw[m]));
+          v[k * 8 + 2 * m] += p.x;
+          v[k * 8 + 2 * m + 1] += p.y;
+        } else {
+          v[k * 8 + 2 * m] += bf16lo(rw[m]);
+          v[k * 8 + 2 * m + 1] += bf16hi(rw[m]);
+        }
       }
     }
   }
@@ -139,10 +191,12 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
     }
   }
   if (EPI != EPI_SCORE && g.has_out16) {
-    // parity < 0: one 2 KB buffer (wait for the previous store to read it)
-    uint8_t* buf = stage + ((both || parity < 0) ? 0 : parity * 2048);
+    // parity < 0: one 2 KB buffer (wait for the previous store to read it);
+    // with a pre-activation store, the second 2 KB half
+    const bool pre = EPI == EPI_SILU && g.has_pre;
+    uint8_t* buf = stage + (pre ? 2048 : ((both || parity < 0) ? 0 : parity * 2048));
     if (lane == 0) {
-      if (both || parity < 0) bulk_wait_read<0>();
+      if ((both || parity < 0) && !pre) bulk_wait_read<0>();
       else bulk_wait_read<1>();
     }
     __syncwarp();
@@ -187,13 +241,15 @@ DEVI void gemm_filter_chunk(const GemmDev& g, int64_t row, bool valid, int col,
   }
 }
 
-template <int BN, int STAGES, int EPI, int COMPACT>
-__global__ void __launch_bounds__(64 + kEpiThreads, 1)
+// MAJ: bit 0 = A is MN-major (stored [K, M] row-major), bit 1 = W is
+// MN-major (stored [K, N] row-major); both arrive as 64 x 64 boxes.
+template <int BN, int STAGES, int EPI, int COMPACT, int LNA, int MAJ>
+__global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmO16,
               const __grid_constant__ CUtensorMap tmO32, const __grid_constant__ CUtensorMap tmR,
-              const GemmDev g) {
-  using C = GemmCfg<BN, STAGES, EPI, COMPACT>;
+              const __grid_constant__ CUtensorMap tmU, const GemmDev g) {
+  using C = GemmCfg<BN, STAGES, EPI, COMPACT, LNA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -203,7 +259,8 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* rbar = drain + 1;  // [8] residual chunk landed (per epilogue warp)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 8);
+  uint64_t* afull = rbar + 8;  // [STAGES] LNA: the A tile has been turned into Z
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + STAGES);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   int* s_go = reinterpret_cast<int*>(ab + 1);
 
@@ -216,6 +273,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
+      mbar_init(afull + s, kEpiThreads / 32);  // LNA: one arrival per A-building warp
     }
     mbar_init(tfull + 0, 1);
     mbar_init(tfull + 1, 1);
@@ -249,8 +307,15 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
   if (Mrows < 0) Mrows = 0;
   const int n_tiles = (g.N + BN - 1) / BN;  // the scores' last tile may be ragged
   const int m_tiles = (int)((Mrows + 127) / 128);
-  const int tiles = m_tiles * n_tiles;
+  const int mn_tiles = m_tiles * n_tiles;
+  const int tiles = mn_tiles * g.splits;
   const int KB = (g.K + 63) / 64;
+  // K blocks [kb_lo, kb_hi) of work unit t (split t / mn_tiles)
+  auto kb_range = [&](int t_, int& lo, int& hi) {
+    const int sp = t_ / mn_tiles;
+    lo = sp * g.kb_split;
+    hi = min(KB, lo + g.kb_split);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -258,16 +323,36 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       uint32_t ph = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
-        for (int kb = 0; kb < KB; ++kb) {
+        const int mn = t % mn_tiles;
+        const int mt = mn / n_tiles, nt = mn - (mn / n_tiles) * n_tiles;
+        int kb_lo, kb_hi;
+        kb_range(t, kb_lo, kb_hi);
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(empty + stage, ph ^ 1, ab, g.status)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(full + stage, C::STAGE_BYTES);
-          tma_load_2d(sa, &tmA, kb * 64, mt * 128, full + stage);
-          tma_load_2d(sa + C::A_BYTES, &tmB, kb * 64, g.n_off + nt * BN, full + stage);
+          if (LNA) {  // the normalised O (in A's place) and U; Z is formed in place
+            tma_load_2d(sa, &tmA, kb * 64, mt * 128, full + stage);
+            tma_load_2d(sa + C::A_BYTES, &tmU, kb * 64, mt * 128, full + stage);
+          } else {
+            if (MAJ & 1) {  // [K, M] source: two 64 (m) x 64 (k) boxes
+              tma_load_2d(sa, &tmA, mt * 128, kb * 64, full + stage);
+              tma_load_2d(sa + 8192, &tmA, mt * 128 + 64, kb * 64, full + stage);
+            } else {
+              tma_load_2d(sa, &tmA, kb * 64, mt * 128, full + stage);
+            }
+          }
+          if (MAJ & 2) {  // [K, N] source: BN / 64 boxes of 64 (n) x 64 (k)
+#pragma unroll
+            for (int a = 0; a < BN / 64; ++a)
+              tma_load_2d(sa + C::B_OFF + a * 8192, &tmB, g.n_off + nt * BN + a * 64, kb * 64,
+                          full + stage);
+          } else {
+            tma_load_2d(sa + C::B_OFF, &tmB, kb * 64, g.n_off + nt * BN, full + stage);
+          }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (ph << stage);
           if (++stage == STAGES) {
@@ -286,11 +371,13 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t IDESC = idesc_f16_f32(128, BN, 0, 0, g.ab_f16);
+      const uint32_t IDESC = idesc_f16_f32(128, BN, MAJ & 1, (MAJ >> 1) & 1, g.ab_f16);
       int stage = 0, local = 0;
       uint32_t ph = 0;
       bool ok = true, issued_any = false;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+        int kb_lo, kb_hi;
+        kb_range(t, kb_lo, kb_hi);
         const int acc = local & 1;
         const uint32_t aph = (local >> 1) & 1;
         if (!mbar_wait(tempty + acc, aph ^ 1, ab, g.status)) {
@@ -299,18 +386,26 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * BN;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(full + stage, ph, ab, g.status)) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
+          // LNA: A holds Z once the epilogue warps have turned it (which they do
+          // after the stage's loads landed)
+          if (!mbar_wait(LNA ? afull + stage : full + stage, ph, ab, g.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t b0 = a0 + C::A_BYTES;
+          const uint32_t b0 = a0 + C::B_OFF;
+          // K-major: the 16-wide K step is 32 bytes along a 128-byte row;
+          // MN-major: 16 rows of 128 bytes, 64-element MN chunks 8 KB apart
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma_f16_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
-                          sdesc_sw128(b0 + k * 32, 16, 1024), IDESC, (kb | k) != 0);
+            tc_mma_f16_ss(d_tmem,
+                          (MAJ & 1) ? sdesc_sw128(a0 + k * 2048, 8192, 1024)
+                                    : sdesc_sw128(a0 + k * 32, 16, 1024),
+                          (MAJ & 2) ? sdesc_sw128(b0 + k * 2048, 8192, 1024)
+                                    : sdesc_sw128(b0 + k * 32, 16, 1024),
+                          IDESC, (kb != kb_lo || k != 0) ? 1u : 0u);
           tc_commit(empty + stage);
           issued_any = true;
           if (++stage == STAGES) {
@@ -339,9 +434,10 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
     uint8_t* rbuf = smem + C::RES_OFF + (warp - 2) * C::BUF;
     uint64_t* rb = rbar + (warp - 2);
     uint32_t rpar = 0;
-    bool r_pending = false, alive = true;
-    auto r_issue = [&](int t_, int c_) {
-      const int mt_ = t_ / n_tiles, nt_ = t_ - (t_ / n_tiles) * n_tiles;
+    bool r_pending = false;
+    auto r_issue = [&](int t_, int c_) {  // (a residual is added only without split-K)
+      const int mn_ = t_ % mn_tiles;
+      const int mt_ = mn_ / n_tiles, nt_ = mn_ - (mn_ / n_tiles) * n_tiles;
       mbar_arrive_expect_tx(rb, rbytes);
       tma_load_2d(rbuf, &tmR, g.n_off + nt_ * BN + part * (BN / 2) + c_ * 32, mt_ * 128 + q * 32,
                   rb);
@@ -350,21 +446,25 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
       r_issue(blockIdx.x, 0);
       r_pending = true;
     }
-    for (int t = blockIdx.x; t < tiles && alive; t += gridDim.x, ++local) {
-      const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
+    // Drains the accumulator of tile t (this CTA's local-th) through the
+    // epilogue and frees it for the MMAs.  Returns false if a wait gave up.
+    auto epi_tile = [&](int t) -> bool {
+      const int sp = t / mn_tiles, mn = t % mn_tiles;
+      const int mt = mn / n_tiles, nt = mn - (mn / n_tiles) * n_tiles;
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
+      ++local;
       const int col0 = g.n_off + nt * BN + part * (BN / 2);
       const uint4* bptr = reinterpret_cast<const uint4*>(g.bias + col0);
       uint4 ba[4], bb[4];
       constexpr bool kNoBias = EPI == EPI_SCORE || EPI == EPI_FILTER;
 #pragma unroll
       for (int i = 0; i < 4; ++i) ba[i] = kNoBias ? make_uint4(0, 0, 0, 0) : __ldg(bptr + i);
-      if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) break;
+      if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) return false;
       tc_fence_after();
-      const int y0 = mt * 128 + q * 32;
-      const int64_t row = (int64_t)y0 + lane;
+      const int64_t row = (int64_t)mt * 128 + q * 32 + lane;
       const bool valid = row < Mrows;
+      const int y0 = (int)(sp * g.split_rows) + mt * 128 + q * 32;  // output row of lane 0
       const uint32_t thr = (EPI == EPI_FILTER && valid) ? desc_key(g.tau[row * g.tau_stride]) : 0u;
       const uint32_t tbase = tmem + acc * BN + part * (BN / 2) + ((uint32_t)(q * 32) << 16);
       uint32_t ra[32], rb_acc[32];
@@ -386,8 +486,8 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
         const uint8_t* rsm = nullptr;
         if (rtma) {
           if (!mbar_wait_warp(rb, rpar, ab, g.status)) {
-            alive = false;
-            break;
+            if (c + 1 < CH) tmem_ld_wait();
+            return false;
           }
           rpar ^= 1;
           rsm = rbuf;
@@ -422,10 +522,153 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
         }
         if (c + 1 < CH) tmem_ld_wait();
       }
-      if (!alive) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
+      return true;
+    };
+
+    if (!LNA) {
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x)
+        if (!epi_tile(t)) break;
+    } else {
+      // ---------------------------------------------- LNA: A = LayerNorm(O) * U
+      // These warps also turn the A tile of every K block into Z = ((O - mu) *
+      // rstd * gamma + beta) * U, in place in shared memory, once TMA has
+      // brought the tile of normalised O (in A's 128-byte swizzled K-major
+      // place) and the matching U tile (same layout).  O arrives normalised
+      // per (row, head): O = m + s * x, so with the row's LayerNorm moments
+      // mu, rstd, (O - mu) * rstd = a + b * x, a = (m - mu) * rstd, b = s *
+      // rstd.  Thread tw takes the 16-byte chunk c = tw & 7 of rows
+      // (tw >> 3) + 32 i, i = 0..3; the 8 threads of a row group are 8
+      // adjacent lanes.  The epilogue of tile t-1 runs once the first STAGES
+      // K blocks of tile t are turned (its accumulator is complete by then,
+      // and the MMAs have those stages to work on meanwhile).
+      const int tw = threadIdx.x - 64;
+      const int c = tw & 7;
+      const int r0 = tw >> 3;
+      const int K = g.K, H = g.ln_h;
+      int stg = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int t_prev = -1;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int mt = (t % mn_tiles) / n_tiles, nt = (t % mn_tiles) % n_tiles;
+        // the LayerNorm moments of this thread's 4 rows over all h * d_v
+        // features, from the heads' (m, s): mu = mean of m, var = mean of
+        // (s^2 + (m - mu)^2); the 8 lanes of a row group share the heads
+        float mu[4], rstd[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t row = (int64_t)mt * 128 + r0 + 32 * i;
+          const bool ok_r = row < Mrows;
+          float2 hv[4];
+          float sm = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int hh = c + 8 * j;
+            hv[j] = (ok_r && hh < H) ? __ldg(g.ln_stats + row * H + hh) : make_float2(0.f, 0.f);
+            sm += hv[j].x;
+          }
+          sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+          sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+          sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+          mu[i] = sm / (float)H;
+          float sv = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (c + 8 * j < H) {
+              const float dm = hv[j].x - mu[i];
+              sv = fmaf(hv[j].y, hv[j].y, fmaf(dm, dm, sv));
+            }
+          }
+          sv += __shfl_xor_sync(0xffffffffu, sv, 1);
+          sv += __shfl_xor_sync(0xffffffffu, sv, 2);
+          sv += __shfl_xor_sync(0xffffffffu, sv, 4);
+          rstd[i] = ok_r ? rsqrtf(sv / (float)H + g.ln_eps) : 0.f;
+        }
+        // per (row, head) statistics, gamma and beta of K block kb, fetched one
+        // block ahead of their use
+        float2 hsn[4];
+        uint4 gvn, bvn;
+        auto fetch = [&](int kb_) {
+          const int head = (kb_ * 64) / g.ln_dv;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int64_t row = (int64_t)mt * 128 + r0 + 32 * i;
+            hsn[i] = row < Mrows ? __ldg(g.ln_stats + row * H + head) : make_float2(0.f, 0.f);
+          }
+          gvn = __ldg(reinterpret_cast<const uint4*>(g.ln_gamma + kb_ * 64 + c * 8));
+          bvn = __ldg(reinterpret_cast<const uint4*>(g.ln_beta + kb_ * 64 + c * 8));
+        };
+        fetch(0);
+        for (int kb = 0; kb < KB; ++kb) {
+          const int col = kb * 64 + c * 8;
+          // the previous tile's epilogue follows this K block; the next block's
+          // fetch then waits for it (fewer registers live across the epilogue)
+          const bool epi_now = kb == (KB < STAGES ? KB : STAGES) - 1 && t_prev >= 0;
+          // The transform runs in packed fp16 (two features per instruction on
+          // the FMA pipes; fp16/fp32 conversions would saturate the XU pipe):
+          // t = a + b x, z = (t gamma + beta) u, each step rounded to fp16
+          __half2 ca[4], cb[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            ca[i] = __float2half2_rn((hsn[i].x - mu[i]) * rstd[i]);
+            cb[i] = __float2half2_rn(hsn[i].y * rstd[i]);
+          }
+          __half2 gh[4], bh[4];
+          {
+            const uint32_t gw[4] = {gvn.x, gvn.y, gvn.z, gvn.w}, bw[4] = {bvn.x, bvn.y, bvn.z, bvn.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              gh[e] = __floats2half2_rn(bf16lo(gw[e]), bf16hi(gw[e]));
+              bh[e] = __floats2half2_rn(bf16lo(bw[e]), bf16hi(bw[e]));
+            }
+          }
+          if (!epi_now && kb + 1 < KB) fetch(kb + 1);
+          // the normalised O and U of this stage have landed
+          if (!mbar_wait_warp(full + stg, ph, ab, g.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stg * C::STAGE_BYTES;
+          const uint8_t* su = sa + C::A_BYTES;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = r0 + 32 * i;
+            const uint32_t off = r * 128 + ((c ^ (r & 7)) << 4);
+            uint4 xv = *reinterpret_cast<const uint4*>(sa + off);
+            const uint4 uv = *reinterpret_cast<const uint4*>(su + off);
+            __half2* xh = reinterpret_cast<__half2*>(&xv);
+            const __half2* uh = reinterpret_cast<const __half2*>(&uv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              xh[e] = __hmul2(__hfma2(__hfma2(cb[i], xh[e], ca[i]), gh[e], bh[e]), uh[e]);
+            const uint4 zv = xv;
+            *reinterpret_cast<uint4*>(sa + off) = zv;
+            const int64_t row = (int64_t)mt * 128 + r;
+            if (g.z_dbg && nt == 0 && row < Mrows)
+              *reinterpret_cast<uint4*>(g.z_dbg + row * K + col) = zv;
+          }
+          fence_proxy_async_smem();  // the tensor cores read what these threads wrote
+          __syncwarp();
+          if (lane == 0) mbar_arrive(afull + stg);
+          if (++stg == STAGES) {
+            stg = 0;
+            ph ^= 1;
+          }
+          if (epi_now) {
+            if (!epi_tile(t_prev)) {
+              ok = false;
+              break;
+            }
+            t_prev = -1;
+            if (kb + 1 < KB) fetch(kb + 1);
+          }
+        }
+        if (ok) t_prev = t;
+      }
+      if (ok && t_prev >= 0) epi_tile(t_prev);
     }
     if (lane == 0 && r_pending) {  // a residual load still in flight must land first
       AbortState tmp{0, kWaitLimitUs};
@@ -443,16 +686,18 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
   }
 }
 
-template <int BN, int STAGES, int EPI, int COMPACT = 0>
+template <int BN, int STAGES, int EPI, int COMPACT = 0, int LNA = 0, int MAJ = 0>
 static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
                               const CUtensorMap& to16, const CUtensorMap& to32,
-                              const CUtensorMap& tr, const GemmDev& gd, int grid, cudaStream_t s) {
-  using C = GemmCfg<BN, STAGES, EPI, COMPACT>;
+                              const CUtensorMap& tr, const GemmDev& gd, int grid, cudaStream_t s,
+                              const CUtensorMap* tu_opt = nullptr) {
+  const CUtensorMap& tu = tu_opt ? *tu_opt : ta;  // LNA only: the U tiles
+  using C = GemmCfg<BN, STAGES, EPI, COMPACT, LNA>;
   static_assert(C::SMEM <= 232448, "shared memory per CTA");
-  auto kfn = k_gemm_tc<BN, STAGES, EPI, COMPACT>;
+  auto kfn = k_gemm_tc<BN, STAGES, EPI, COMPACT, LNA, MAJ>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM);
   if (e != cudaSuccess) return e;
-  kfn<<<grid, 64 + kEpiThreads, C::SMEM, s>>>(ta, tb, to16, to32, tr, gd);
+  kfn<<<grid, C::THREADS, C::SMEM, s>>>(ta, tb, to16, to32, tr, tu, gd);
   return cudaGetLastError();
 }
 
@@ -467,10 +712,23 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   else if (c.N % 128 == 0) BN = 128;
   CUtensorMap ta, tb, to16, to32, tr;
   const bool f16 = c.ab_f16 != 0;
-  if (!encode_tmap_2d(&ta, c.A, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.lda * 2, 64, 128, f16))
+  const bool lna = c.ln_x != nullptr;
+  if (lna && (c.epi != EPI_RESID || !f16 || !c.ln_stats || !c.ln_u || !c.ln_gamma ||
+              !c.ln_beta || c.ln_h <= 0 || c.ln_dv % 64 != 0 || c.ln_h * c.ln_dv != c.K ||
+              c.ld_u % 8 != 0))
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d(&tb, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K, (uint64_t)c.ldw * 2, 64,
                       (uint32_t)BN, f16))
+    return cudaErrorInvalidValue;
+  // LNA: A is the normalised O [M, K] (becomes Z in shared memory); U comes
+  // from the first K columns of ln_u
+  CUtensorMap tu;
+  if (!encode_tmap_2d(&ta, lna ? c.ln_x : c.A, (uint64_t)c.M_cap, (uint64_t)c.K,
+                      (uint64_t)(lna ? c.K : c.lda) * 2, 64, 128, f16))
+    return cudaErrorInvalidValue;
+  tu = ta;
+  if (lna && !encode_tmap_2d(&tu, c.ln_u, (uint64_t)c.M_cap, (uint64_t)c.K, (uint64_t)c.ld_u * 2,
+                             64, 128, true))
     return cudaErrorInvalidValue;
   // output maps over the whole [M_cap, ldo] matrix, 32 x 32 boxes; an unused
   // map is a copy of a valid one (never dereferenced)
@@ -484,6 +742,12 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   if (c.out32 && !encode_tmap_2d_ex(&to32, c.out32, (uint64_t)c.M_cap, (uint64_t)c.ldo,
                                     (uint64_t)c.ldo * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  // EPI_SILU's pre-activation output: a 16-bit matrix laid out like `out`
+  if (c.out_pre && (c.epi != EPI_SILU || !c.out ||
+                    !encode_tmap_2d_ex(&to32, c.out_pre, (uint64_t)c.M_cap, (uint64_t)c.ldo,
+                                       (uint64_t)c.ldo * 2, 32, 32, t16,
+                                       CU_TENSOR_MAP_SWIZZLE_64B)))
     return cudaErrorInvalidValue;
   // residual: [M_cap, n_off + N] with row stride ldr, 32 x 32 boxes (fp32 with
   // 128-byte swizzle, 16-bit with 64-byte swizzle)
@@ -514,6 +778,19 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   gd.ldr = c.ldr;
   gd.resid_kind = c.resid_kind;
   gd.status = c.status;
+  gd.ln_x = static_cast<const __half*>(c.ln_x);
+  gd.ln_stats = reinterpret_cast<const float2*>(c.ln_stats);
+  gd.ln_u = static_cast<const __half*>(c.ln_u);
+  gd.ld_u = c.ld_u;
+  gd.ln_gamma = static_cast<const __nv_bfloat16*>(c.ln_gamma);
+  gd.ln_beta = static_cast<const __nv_bfloat16*>(c.ln_beta);
+  gd.ln_eps = c.ln_eps;
+  gd.ln_h = c.ln_h;
+  gd.ln_dv = c.ln_dv;
+  gd.z_dbg = static_cast<__half*>(c.z_dbg);
+  gd.splits = 1;
+  gd.kb_split = (c.K + 63) / 64;
+  gd.has_pre = c.out_pre != nullptr && c.epi == EPI_SILU;
   const int64_t tiles = mt * (c.N / BN);
   const int grid = (int)std::min<int64_t>(tiles, sms);
   LaunchScope ls(kernel_id, s);
@@ -526,6 +803,15 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
     if (BN == 256) return launch_one<256, 4, EPI_BIAS>(ta, tb, to16, to32, tr, gd, grid, s);
     if (BN == 128) return launch_one<128, 6, EPI_BIAS>(ta, tb, to16, to32, tr, gd, grid, s);
     return launch_one<64, 8, EPI_BIAS>(ta, tb, to16, to32, tr, gd, grid, s);
+  }
+  if (lna) {  // f2 with LayerNorm * U formed in its A operand's shared memory
+    if (BN == 256) {
+      if (c.resid_kind != RESID_F32 && c.out32 == nullptr)
+        return launch_one<256, 3, EPI_RESID, 1, 1>(ta, tb, to16, to32, tr, gd, grid, s, &tu);
+      return launch_one<256, 2, EPI_RESID, 0, 1>(ta, tb, to16, to32, tr, gd, grid, s, &tu);
+    }
+    if (BN == 128) return launch_one<128, 3, EPI_RESID, 0, 1>(ta, tb, to16, to32, tr, gd, grid, s, &tu);
+    return launch_one<64, 4, EPI_RESID, 0, 1>(ta, tb, to16, to32, tr, gd, grid, s, &tu);
   }
   // the residual buffers take one A/B stage's worth of shared memory
   if (BN == 256) {
@@ -572,6 +858,8 @@ cudaError_t launch_gemm_scores(const void* A, int64_t lda, const void* W, int64_
   gd.resid = nullptr;
   gd.status = status;
   gd.run_if = run_if;
+  gd.splits = 1;
+  gd.kb_split = K / 64;
   const int64_t tiles = ((M_cap + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
   LaunchScope ls(kernel_id, s);
@@ -605,10 +893,88 @@ cudaError_t launch_gemm_filter(const void* A, int64_t lda, const void* W, int64_
   gd.cand_cnt = cnt;
   gd.cand_cap = cap;
   gd.overflow = overflow;
+  gd.splits = 1;
+  gd.kb_split = K / 64;
   const int64_t tiles = ((M_cap + 127) / 128) * ((N + BN - 1) / BN);
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
   LaunchScope ls(kernel_id, s);
   return launch_one<BN, 4, EPI_FILTER>(ta, tb, ta, ta, ta, gd, grid, s);
+}
+
+}  // namespace hstu
+
+namespace hstu {
+
+cudaError_t launch_gemm_grad(const GradGemm& c, cudaStream_t s, int kernel_id) {
+  if (c.M <= 0 || c.N <= 0 || c.K <= 0) return cudaSuccess;
+  if (c.M > (1ll << 31) - 256 || c.N > (1ll << 31) - 256 || c.K > (1ll << 31) - 256)
+    return cudaErrorInvalidValue;
+  if (c.splits < 1 || (c.resid && c.splits != 1) || c.ldo % 4 != 0) return cudaErrorInvalidValue;
+  if (c.splits > 1 && c.split_rows < ((c.M + 127) / 128) * 128) return cudaErrorInvalidValue;
+  if (!c.a_mn && c.K % 64 != 0) return cudaErrorInvalidValue;  // K-major A: whole 64-wide blocks
+  if (!c.w_mn && c.K % 64 != 0) return cudaErrorInvalidValue;
+  if (c.resid && (!c.zero_bias || c.N % 64 != 0)) return cudaErrorInvalidValue;
+  constexpr int BN = 256;
+  const bool f16 = c.ab_f16 != 0;
+  CUtensorMap ta, tb, to32, to16, tr;
+  // A: [M, K] (boxes 64 k x 128 m) or [K, M] (boxes 64 m x 64 k)
+  if (c.a_mn ? !encode_tmap_2d(&ta, c.A, (uint64_t)c.K, (uint64_t)c.M, (uint64_t)c.lda * 2, 64,
+                               64, f16)
+             : !encode_tmap_2d(&ta, c.A, (uint64_t)c.M, (uint64_t)c.K, (uint64_t)c.lda * 2, 64,
+                               128, f16))
+    return cudaErrorInvalidValue;
+  if (c.w_mn ? !encode_tmap_2d(&tb, c.W, (uint64_t)c.K, (uint64_t)c.N, (uint64_t)c.ldw * 2, 64,
+                               64, f16)
+             : !encode_tmap_2d(&tb, c.W, (uint64_t)c.N, (uint64_t)c.K, (uint64_t)c.ldw * 2, 64,
+                               BN, f16))
+    return cudaErrorInvalidValue;
+  const int64_t rows_out = c.splits > 1 ? c.splits * c.split_rows : c.M;
+  if (!encode_tmap_2d_ex(&to32, c.out, (uint64_t)rows_out, (uint64_t)c.N, (uint64_t)c.ldo * 4, 32,
+                         32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  to16 = to32;
+  tr = to32;
+  if (c.resid) {
+    if (!encode_tmap_2d_ex(&tr, c.resid, (uint64_t)c.M, (uint64_t)c.N, (uint64_t)c.ldo * 4, 32,
+                           32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    if (c.out16 && !encode_tmap_2d_ex(&to16, c.out16, (uint64_t)c.M, (uint64_t)c.N,
+                                      (uint64_t)c.ldo * 2, 32, 32,
+                                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
+  const int KB = (int)((c.K + 63) / 64);
+  const int splits = (int)std::min<int64_t>(c.splits, KB);
+  const int kb_split = (KB + splits - 1) / splits;
+  GemmDev gd{};
+  gd.M_cap = c.M;
+  gd.N = (int)c.N;
+  gd.K = (int)c.K;
+  gd.ab_f16 = c.ab_f16;
+  gd.status = c.status;
+  gd.splits = (KB + kb_split - 1) / kb_split;  // no empty split
+  if (c.splits_used) *c.splits_used = gd.splits;
+  gd.kb_split = kb_split;
+  gd.split_rows = c.split_rows;
+  const int64_t tiles = ((c.M + 127) / 128) * ((c.N + BN - 1) / BN) * gd.splits;
+  const int grid = (int)std::min<int64_t>(tiles, num_sms());
+  LaunchScope ls(kernel_id, s);
+  if (c.resid) {  // out = resid + A W^T (+ a zero bias), fp32 and optionally bf16
+    gd.bias = static_cast<const __nv_bfloat16*>(c.zero_bias);
+    gd.has_out16 = c.out16 != nullptr;
+    gd.out_f16 = 0;
+    gd.has_out32 = 1;
+    gd.resid = c.resid;
+    gd.ldr = c.ldo;
+    gd.resid_kind = RESID_F32;
+    if (!c.a_mn && c.w_mn)
+      return launch_one<256, 3, EPI_RESID, 0, 0, 2>(ta, tb, to16, to32, tr, gd, grid, s);
+    return cudaErrorInvalidValue;
+  }
+  if (c.a_mn && c.w_mn) return launch_one<256, 4, EPI_SCORE, 0, 0, 3>(ta, tb, ta, to32, ta, gd, grid, s);
+  if (c.w_mn) return launch_one<256, 4, EPI_SCORE, 0, 0, 2>(ta, tb, ta, to32, ta, gd, grid, s);
+  if (c.a_mn) return launch_one<256, 4, EPI_SCORE, 0, 0, 1>(ta, tb, ta, to32, ta, gd, grid, s);
+  return launch_one<256, 4, EPI_SCORE>(ta, tb, ta, to32, ta, gd, grid, s);
 }
 
 }  // namespace hstu

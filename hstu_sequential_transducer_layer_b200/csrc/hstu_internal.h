@@ -47,7 +47,13 @@ enum KernelId : int32_t {
   K_TF_FFN2 = 28,
   K_GEMM_FILTER = 29,
   K_FILTER_MERGE = 30,
-  K_NUM_KERNELS = 31
+  K_ATTN_BWD_DKV = 31,
+  K_ATTN_BWD_DQ = 32,
+  K_GEMM_BWD = 33,
+  K_LN_BWD = 34,
+  K_SUM_ROWS = 35,
+  K_F32_TO_F16 = 36,
+  K_NUM_KERNELS = 37
 };
 const char* kernel_name(int id);
 
@@ -63,14 +69,19 @@ struct LaunchScope {
 
 // ---------------------------------------------------------------- device info
 int num_sms();
-// Raises `fn`'s dynamic shared-memory limit to `bytes` on the current device
-// (once per kernel and device).
+// Raises `fn`'s dynamic shared-memory limit to at least `bytes` on the
+// current device (again only when a larger limit is needed).
 cudaError_t ensure_smem_limit(const void* fn, int bytes);
 // Bound of an in-kernel wait unless a test asks for a shorter one.
 constexpr uint32_t kDefaultWaitLimitUs = 1000u * 1000u;
 // The wait bound and stall injection for the next attention launch
 // (hstu_debug_wait_test), reset to the defaults once taken.
 void take_wait_test(uint32_t* limit_us, int* inject_stall);
+// Whether layer calls of the tensor-core path also write the gated Z into the
+// workspace (hstu_debug_keep_z).
+bool keep_z();
+// Records a failed CUDA runtime call for hstu_last_error (per host thread).
+void note_cuda_error(cudaError_t e, const char* where);
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda).  Returns false if the driver call is unavailable/failed.
 // 2-D map of a row-major matrix with an explicit element type and swizzle.
@@ -93,11 +104,11 @@ struct Header {           // first 256 bytes of every workspace
 };
 
 struct Layout {
-  size_t header, items, t_rel, ubase, tbuckets, f1, o, z;
+  size_t header, items, t_rel, ubase, tbuckets, f1, o, ostats, z;
   size_t xres, xh;          // residual stream: fp32 (fp32 path) / fp16, also the next f1's operand
   size_t w16;               // tensor-core path: fp16 copies of W1 (layers >= 1) and W2, per layer
   size_t f1_cache;          // M-FALCON: every layer's f1 output (its K/V) for the history
-  size_t mb_off, c_items, t_req_rel, xres_c, xb_c, xh_c, f1c, oc, zc;  // candidate microbatch
+  size_t mb_off, c_items, t_req_rel, xres_c, xb_c, xh_c, f1c, oc, ostats_c, zc;  // candidate microbatch
   size_t total;
   int64_t item_cap, cand_item_cap, mb_cap, tile_cap;
 };
@@ -157,8 +168,47 @@ struct GemmCall {
   int resid_kind;                // tensor-core EPI_RESID residual: RESID_BF16, RESID_F32, RESID_F16
   int epi;
   int* status;
+  // Tensor-core EPI_RESID only: when ln_x is set, A is not read; the kernel
+  // builds A = LayerNorm(O) * U itself from the attention output stored as
+  // (O - m) / s in fp16 (ln_x, [M, K]) with each (row, head)'s (m, s)
+  // (ln_stats, [M, ln_h] pairs), U (the first K columns of ln_u, row stride
+  // ld_u), gamma and beta (bf16 [K]); K = ln_h * ln_dv.  z_dbg (optional, fp16
+  // [M, K]) receives Z.
+  const void* ln_x;
+  const float* ln_stats;
+  const void* ln_u; int64_t ld_u;
+  const void* ln_gamma; const void* ln_beta;
+  float ln_eps;
+  int ln_h, ln_dv;
+  void* z_dbg;
+  // EPI_SILU only: also store the pre-activation A W^T + b (16-bit like `out`,
+  // same layout)
+  void* out_pre;
 };
 cudaError_t launch_gemm_tc(const GemmCall& g, cudaStream_t s, int kernel_id);
+// Products for the backward pass: out[s * split_rows + m, n] (fp32, row
+// stride ldo) = sum over the K blocks of split s of A[m, k] W[n, k], 16-bit
+// operands (fp16 if ab_f16).  a_mn: A is stored [K, M] row-major (else
+// [M, K]); w_mn: W is stored [K, N] row-major (else [N, K]).  splits > 1 cuts
+// K into that many ranges (the caller sums the partial products); M, N
+// multiples of 64 are not required (ragged edges read zeros, stores clip);
+// K rows past K_rows read zeros.  With resid (fp32, same layout as out; splits
+// = 1 only) the output is out = resid + A W^T, and out16 (bf16, optional)
+// receives a copy.
+struct GradGemm {
+  const void* A; int64_t lda; int a_mn;
+  const void* W; int64_t ldw; int w_mn;
+  int ab_f16;
+  int64_t M, N, K;
+  int splits; int64_t split_rows;
+  float* out; int64_t ldo;
+  const float* resid;
+  void* out16;
+  const void* zero_bias;   // bf16 zeros, at least N (the residual epilogue adds a bias)
+  int* status;
+  int* splits_used;        // optional: receives the number of splits launched (<= splits)
+};
+cudaError_t launch_gemm_grad(const GradGemm& g, cudaStream_t s, int kernel_id);
 // scores[M_cap, N] (fp32, row stride ldo) = A[M_cap, K] * W[N, K]^T, no bias;
 // N may be ragged (the last 256-column tile is clipped); K % 64 == 0,
 // ldo % 4 == 0, bf16 or fp16 operands (ab_f16).
@@ -194,10 +244,31 @@ struct AttnCall {
   int32_t* work_next; int32_t* work_done;  // dynamic scheduling counters (header)
   const float* rab_pos; const float* rab_time;
   int Np, Nt, Sp, St, h, dqk, dv;
-  void* O; int64_t ldo;
+  void* O; int64_t ldo;            // tensor-core path: normalised O, fp16; SIMT path: O, fp32
+  float* ostats;                   // tensor-core path: [rows, h] (mean, deviation) of each head's O
   int* status;
 };
 cudaError_t launch_attn_tc(const AttnCall& a, cudaStream_t s);
+
+// Backward pass of the causal pointwise attention (self mode): from dO
+// ([rows, h*d_v] fp16, row stride ld_do) and the f1 output (U|V|Q|K fp16,
+// [rows, F]) and its pre-activation (`pre`, same layout), writes the
+// gradients of the pre-activation's V, K and Q columns into dP ([rows, F]
+// fp16) and adds the bias-table gradients into drab_pos / drab_time (fp32;
+// the caller zeroes them).  Uses the forward's work list.
+struct AttnBwdCall {
+  const AttnItem* items; const int32_t* n_items; int64_t item_cap;
+  const void* f1; const void* pre; void* dP; int64_t ld_f1; int64_t rows;
+  const void* dO; int64_t ld_do;
+  int q_col, k_col, v_col;
+  const int32_t* t_rel;
+  const float* rab_pos; const float* rab_time;
+  float* drab_pos; float* drab_time;
+  int Np, Nt, Sp, St, h, dqk, dv;
+  int32_t* work_next; int32_t* work_done;
+  int* status;
+};
+cudaError_t launch_attn_bwd(const AttnBwdCall& c, cudaStream_t s);
 cudaError_t launch_attn_simt_f32(const AttnCall& a, cudaStream_t s);
 
 // Z = LayerNorm(O) * gamma + beta, then * U (per row over h*d_v features).

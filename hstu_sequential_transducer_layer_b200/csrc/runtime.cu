@@ -1,8 +1,9 @@
 // runtime.cu — host-side runtime of libhstu: launch counting and tracing,
 // device queries, TMA descriptor encoding, and the workspace layout.
 #include <atomic>
+#include <cstdio>
 #include <mutex>
-#include <set>
+#include <map>
 #include <utility>
 #include <vector>
 
@@ -28,7 +29,8 @@ const char* kernel_name(int id) {
       "gemm_f2_simt_f32", "attn_cand_simt_f32", "bf16_to_f16", "time_buckets",
       "sl_offsets", "sl_select", "sl_gather", "ret_gather", "gemm_scores_tc", "topk_chunk",
       "topk_merge", "tf_ln", "tf_qkv_tc", "tf_softmax_attn_tc", "tf_oproj_tc", "tf_ffn1_tc",
-      "tf_ffn2_tc", "gemm_filter_tc", "filter_merge"};
+      "tf_ffn2_tc", "gemm_filter_tc", "filter_merge", "attn_bwd_dkv_tc", "attn_bwd_dq_tc",
+      "gemm_bwd_tc", "ln_bwd", "sum_rows", "f32_to_f16"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 
@@ -47,19 +49,22 @@ LaunchScope::~LaunchScope() {
 
 // ---------------------------------------------------------------- device
 // The dynamic shared-memory limit is an attribute of a kernel on one device:
-// it is raised once per (kernel, device) pair, under a lock, so the first
-// launch on a second GPU of the same process raises it there too.
+// it is raised per (kernel, device) pair, under a lock, whenever a launch
+// needs more than was set before (so the first launch on a second GPU of the
+// same process raises it there too, and a kernel whose shared memory depends
+// on the shape gets the larger limit).
 cudaError_t ensure_smem_limit(const void* fn, int bytes) {
   static std::mutex mu;
-  static std::set<std::pair<const void*, int>> done;
+  static std::map<std::pair<const void*, int>, int> set_to;  // (kernel, device) -> limit
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(mu);
   const auto key = std::make_pair(fn, dev);
-  if (done.count(key)) return cudaSuccess;
+  const auto it = set_to.find(key);
+  if (it != set_to.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert(key);
+  if (e == cudaSuccess) set_to[key] = bytes;
   return e;
 }
 
@@ -69,6 +74,18 @@ std::mutex g_wait_mu;
 uint32_t g_wait_limit_us = 0;  // 0: the default bound
 int g_inject_stall = 0;
 }  // namespace
+
+namespace {
+std::atomic<int> g_keep_z{0};
+thread_local char g_last_error[256] = "";
+}  // namespace
+
+void note_cuda_error(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where ? where : "?",
+           cudaGetErrorString(e), (int)e);
+}
+
+bool keep_z() { return g_keep_z.load(std::memory_order_relaxed) != 0; }
 
 void take_wait_test(uint32_t* limit_us, int* inject_stall) {
   std::lock_guard<std::mutex> lk(g_wait_mu);
@@ -173,7 +190,13 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
     L->f1_cache = take((size_t)n_layers * T * F * es);
     L->f1 = L->f1_cache;
   }
-  L->o = take((size_t)T * hdv * 4);
+  // attention output: fp32 O (fp32 path), or the normalised fp16 O followed
+  // by each (row, head)'s (mean, deviation) (tensor-core path)
+  L->o = take(bf16 ? up256((size_t)T * hdv * 2) + (size_t)T * d.n_heads * 8 : (size_t)T * hdv * 4);
+  L->ostats = bf16 ? L->o + up256((size_t)T * hdv * 2) : 0;
+  // Z: the fp32 path's LayerNorm * U output; on the tensor-core path Z is
+  // formed in the output projection's shared memory and written here only
+  // when a test asks for it (hstu_debug_keep_z)
   L->z = take((size_t)T * hdv * es);
   // residual stream between layers: fp16 on the tensor-core path, fp32 otherwise
   L->xres = bf16 ? 0 : take((size_t)T * dm * 4);
@@ -191,7 +214,9 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
     L->xb_c = bf16 ? take((size_t)cap * dm * 2) : L->xres_c;
     L->xh_c = bf16 ? take((size_t)cap * dm * 2) : L->xres_c;
     L->f1c = take((size_t)cap * F * es);
-    L->oc = take((size_t)cap * hdv * 4);
+    L->oc = take(bf16 ? up256((size_t)cap * hdv * 2) + (size_t)cap * d.n_heads * 8
+                      : (size_t)cap * hdv * 4);
+    L->ostats_c = bf16 ? L->oc + up256((size_t)cap * hdv * 2) : 0;
     L->zc = take((size_t)cap * hdv * es);
   }
   (void)max_len;
@@ -204,6 +229,14 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
 
 // ---------------------------------------------------------------- C ABI
 extern "C" {
+
+const char* hstu_last_error(void) { return hstu::g_last_error; }
+
+hstu_status hstu_debug_keep_z(int32_t on) {
+  if (on != 0 && on != 1) return HSTU_ERR_INVALID_ARG;
+  hstu::g_keep_z.store(on);
+  return HSTU_OK;
+}
 
 hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall) {
   if (inject_stall != 0 && inject_stall != 1) return HSTU_ERR_INVALID_ARG;

@@ -127,21 +127,64 @@ class HSTURunner:
     def status(self, stream=None) -> int:
         return _b.hstu_read_status(self._ws, stream)
 
+    def stack_bwd(self, offsets, X, timestamps, dY, max_len: int, n_layers: Optional[int] = None,
+                  dX=None, grads=None, stream=None):
+        """hstu_stack_bwd (hstu_layer_bwd for one layer): the gradient dX of a
+        loss with respect to X given its gradient dY with respect to the
+        stack's output, and every layer's parameter gradients (fp32).
+        Returns (dX, [dict per layer])."""
+        t = self.torch
+        L = self.n_layers if n_layers is None else n_layers
+        B = offsets.numel() - 1
+        T = X.shape[0]
+        d = self.desc
+        F = 2 * d.n_heads * (d.d_v + d.d_qk)
+        hdv = d.n_heads * d.d_v
+        if dX is None:
+            dX = t.empty_like(X)
+        if grads is None:
+            shapes = dict(dW1=(F, d.d_model), db1=(F,), dW2=(d.d_model, hdv), db2=(d.d_model,),
+                          dln_gamma=(hdv,), dln_beta=(hdv,),
+                          drab_pos=(d.n_heads, d.n_pos_buckets),
+                          drab_time=(d.n_heads, d.n_time_buckets))
+            grads = [{k: t.empty(v, dtype=t.float32, device=self.device) for k, v in shapes.items()}
+                     for _ in range(L)]
+        nb = _b.hstu_bwd_workspace_size(self.desc, L, B, T, max_len)
+        if getattr(self, "_bws", None) is None or self._bws.numel() < nb:
+            self._bws = t.empty(max(nb, 256), dtype=t.uint8, device=self.device)
+        if L == 1:
+            _b.hstu_layer_bwd(self.desc, self._warr[0], B, T, max_len, offsets, X, timestamps, dY,
+                              dX, grads, self._bws, stream)
+        else:
+            _b.hstu_stack_bwd(self.desc, L, self._warr, B, T, max_len, offsets, X, timestamps, dY,
+                              dX, grads, self._bws, stream)
+        return dX, grads
+
+    def bwd_status(self, stream=None) -> int:
+        return _b.hstu_read_status(self._bws, stream)
+
     def intermediates(self, B: int, T: int, max_len: int):
-        """Views of the f1 output, O (fp32) and Z that the last layer call left
-        in the workspace.  On the tensor-core (bf16) path the f1 output and Z
-        are stored in fp16; on the fp32 path in fp32."""
+        """Views of the f1 output, the attention output and Z that the last
+        layer call left in the workspace (see hstu_debug_offsets).  fp32 path:
+        (f1, O, Z), all fp32.  Tensor-core (bf16) path: (f1 fp16, (Xn, S), Z
+        fp16) where Xn [T, h*d_v] fp16 holds (O - m) / s per (row, head) and S
+        [T, h, 2] fp32 the (m, s) pairs; Z is there only while
+        hstu_debug_keep_z(1) was in effect."""
         f1o, oo, zo = _b.hstu_debug_offsets(self.desc, B, T, max_len)
         d = self.desc
         F = 2 * d.n_heads * (d.d_v + d.d_qk)
         hdv = d.n_heads * d.d_v
         t = self.torch
-        idt, es = (t.float16, 2) if self.dtype == "bf16" else (t.float32, 4)
         ws = self._ws
 
         def view(off, cols, dt, size):
             return ws[off:off + T * cols * size].view(dt).view(T, cols)
-        return view(f1o, F, idt, es), view(oo, hdv, t.float32, 4), view(zo, hdv, idt, es)
+        if self.dtype != "bf16":
+            return view(f1o, F, t.float32, 4), view(oo, hdv, t.float32, 4), view(zo, hdv, t.float32, 4)
+        so = oo + ((T * hdv * 2 + 255) // 256) * 256
+        stats = view(so, 2 * d.n_heads, t.float32, 4).view(T, d.n_heads, 2)
+        return (view(f1o, F, t.float16, 2), (view(oo, hdv, t.float16, 2), stats),
+                view(zo, hdv, t.float16, 2))
 
 
 class TransformerRunner:

@@ -202,6 +202,62 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
                                    const hstu_layer_weights* weights, const int64_t* timestamps,
                                    void* out, void* stream);
 
+/* Backward pass (gradients, for training) of hstu_layer_fwd / hstu_stack_fwd
+ * ('HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか': the
+ * forward layer whose chain rule this is; section 'Production評価の12.4%をどう
+ * 読むか': training is where the pages report the largest gain).  Given the
+ * layers' input X and the gradient dY of a loss with respect to the stack's
+ * output, computes dX (the gradient with respect to X) and, per layer, the
+ * gradients of every parameter.  Each layer's forward is recomputed from its
+ * input inside the call (the stack's forward runs once first to obtain the
+ * layers' inputs), so nothing of a forward call has to be kept.
+ * Derivatives, per user (n = n_b) and head, written out by the chain rule:
+ *   dZ = dY W2;  dW2 = dY^T Z;  db2 = sum_rows dY
+ *   dL = dZ * U; dU = dZ * L (L = LayerNorm(O) before the gate); dgamma =
+ *   sum_rows dL * xhat; dbeta = sum_rows dL; dO = (dxh - mean(dxh) - xhat
+ *   mean(dxh xhat)) / sd with dxh = dL * gamma
+ *   dA_ij = (1/n) dO_i . V_j; dV_j = (1/n) sum_i SiLU(s_ij) dO_i;
+ *   dS_ij = dA_ij SiLU'(s_ij); dQ_i = sum_j dS_ij K_j; dK_j = sum_i dS_ij Q_i;
+ *   drab_pos[h][b] / drab_time[h][b] = sum of dS_ij over the pairs (i, j) of
+ *   bucket b
+ *   dP = [dU | dV | dQ | dK] * SiLU'(P), P = X W1^T + b1;  dW1 = dP^T X;
+ *   db1 = sum_rows dP;  dX = dY + dP W1.
+ * dtype HSTU_BF16 only (HSTU_ERR_UNSUPPORTED otherwise), with the forward's
+ * shape limits and n_time_buckets <= 256.  X and dY are bf16 [T, d] (device);
+ * dX is bf16 [T, d]; every gradient is fp32, in its parameter's layout, and
+ * is overwritten (not accumulated into).  The tensor cores take fp16
+ * operands with fp32 accumulation (as in the forward; the gradients flowing
+ * into them must lie within fp16 range); the gradient stream between layers
+ * is fp32.  The bias-table gradients are summed with atomic adds, so their
+ * last bits may differ from run to run; everything else is deterministic.
+ * grads: host array [n_layers] of device pointers.  Workspace:
+ * hstu_bwd_workspace_size() bytes, 256-byte aligned.  Asynchronous on
+ * `stream`; device-detected errors (bad offsets or timestamps, a wait that
+ * gave up) set the workspace's status word (hstu_read_status). */
+typedef struct {
+  float* dW1;        /* [F, d_model] */
+  float* db1;        /* [F] */
+  float* dW2;        /* [d_model, h*d_v] */
+  float* db2;        /* [d_model] */
+  float* dln_gamma;  /* [h*d_v] */
+  float* dln_beta;   /* [h*d_v] */
+  float* drab_pos;   /* [h, n_pos_buckets] */
+  float* drab_time;  /* [h, n_time_buckets] */
+} hstu_layer_grads;
+size_t hstu_bwd_workspace_size(const hstu_layer_desc* desc, int32_t n_layers, int64_t B,
+                               int64_t total_tokens, int64_t max_len);
+hstu_status hstu_layer_bwd(const hstu_layer_desc* desc, const hstu_layer_weights* weights,
+                           int64_t B, int64_t total_tokens, int64_t max_len,
+                           const int64_t* offsets, const void* X, const int64_t* timestamps,
+                           const void* dY, void* dX, const hstu_layer_grads* grads,
+                           void* workspace, size_t workspace_bytes, void* stream);
+hstu_status hstu_stack_bwd(const hstu_layer_desc* desc, int32_t n_layers,
+                           const hstu_layer_weights* weights, int64_t B, int64_t total_tokens,
+                           int64_t max_len, const int64_t* offsets, const void* X,
+                           const int64_t* timestamps, const void* dY, void* dX,
+                           const hstu_layer_grads* grads, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* Stochastic Length sampling and token embedding ('HSTUとGenerative
  * Recommenders', section '2. Stochastic Lengthで学習時の履歴を間引く': a long
  * history is shortened to a random subset of its positions; 4096 tokens keep
@@ -322,7 +378,14 @@ hstu_status hstu_read_status(const void* workspace, size_t workspace_bytes, void
 /* Test hook: byte offsets inside the workspace where hstu_layer_fwd (and the
  * last layer of hstu_stack_fwd) leaves its intermediates: the f1 output
  * [T, F] (U|V|Q|K after SiLU), the pre-LayerNorm attention output O [T, h*d_v]
- * (already scaled by 1/n_b) and the gated Z [T, h*d_v]. */
+ * (already scaled by 1/n_b) and the gated Z [T, h*d_v].
+ * dtype HSTU_FP32: O and Z are fp32.  dtype HSTU_BF16: the f1 output is fp16;
+ * O is stored per (row, head) as its mean m and standard deviation s over
+ * the head's d_v values and the normalised values (O - m) / s: the fp16
+ * values [T, h*d_v] at o_offset, then, at the next multiple of 256 bytes,
+ * the (m, s) pairs as fp32 [T, h, 2]; Z (fp16) is formed inside the output
+ * projection and written at z_offset only while hstu_debug_keep_z(1) is in
+ * effect. */
 hstu_status hstu_debug_offsets(const hstu_layer_desc* desc, int64_t B, int64_t total_tokens,
                                int64_t max_len, size_t* f1_offset, size_t* o_offset,
                                size_t* z_offset);
@@ -336,6 +399,13 @@ hstu_status hstu_trace_enable(int32_t max_records);
 int32_t hstu_trace_read(int32_t* kernel_ids, float* ms, int32_t capacity);
 const char* hstu_kernel_name(int32_t kernel_id);
 int64_t hstu_launch_count(void);
+
+/* Test hook: with on = 1, later layer calls on the tensor-core path also
+ * write the gated Z = LayerNorm(O) * U into the workspace (at the z offset
+ * of hstu_debug_offsets); with on = 0 (the default) Z never leaves the output
+ * projection's shared memory.  Process-wide.  Returns HSTU_ERR_INVALID_ARG
+ * for other values. */
+hstu_status hstu_debug_keep_z(int32_t on);
 
 /* Test hook for the failure detection of the in-kernel waits.  Every wait
  * inside the attention kernel is bounded: after wait_limit_us microseconds
@@ -351,6 +421,11 @@ int64_t hstu_launch_count(void);
  * pages describe no failure handling.  Returns HSTU_ERR_INVALID_ARG for an
  * inject_stall other than 0 or 1. */
 hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall);
+
+/* After an entry point returned HSTU_ERR_CUDA: the failing CUDA runtime
+ * call's error and the step it belonged to, as text (per host thread; ""
+ * if none). */
+const char* hstu_last_error(void);
 
 const char* hstu_status_string(hstu_status s);
 int32_t hstu_version(void);

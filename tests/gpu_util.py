@@ -80,3 +80,15 @@ def run_rank(w, microbatch=None, runner=None, candidates=None, cand_offsets=None
                     w.max_len, int(m.max(initial=0)))
     torch.cuda.synchronize()
     return scores.double().cpu().numpy(), r
+
+
+def decode_o(o, n_heads: int, d_v: int):
+    """The attention output O [T, h*d_v] (float64) from what the layer call
+    left in the workspace: fp32 O as is (fp32 path), or, on the tensor-core
+    path, (Xn, S) with O = m + s * Xn per (row, head)."""
+    if not isinstance(o, tuple):
+        return o.double().cpu().numpy()
+    xn, st = o
+    xn = xn.double().cpu().numpy().reshape(xn.shape[0], n_heads, d_v)
+    st = st.double().cpu().numpy()
+    return (st[:, :, :1] + st[:, :, 1:] * xn).reshape(xn.shape[0], n_heads * d_v)

@@ -30,7 +30,7 @@ import pytest
 
 import hstu_workloads as hw
 from oracle import hstu_oracle as O
-from gpu_util import TOL, relerr, rmserr, run_stack, runner_for, ulperr
+from gpu_util import TOL, decode_o, relerr, rmserr, run_stack, runner_for, ulperr
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +38,11 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def built():
     from hstu_sequential_transducer_layer_b200.build import build
+    from hstu_sequential_transducer_layer_b200 import binding as B
     build()
+    B.hstu_debug_keep_z(True)      # the layer calls of this module also write Z
+    yield
+    B.hstu_debug_keep_z(False)
 
 
 def z_checks(z, o, u, z_ref, o_ref, u_ref, gamma, beta, eps):
@@ -62,7 +66,9 @@ def z_checks(z, o, u, z_ref, o_ref, u_ref, gamma, beta, eps):
 def _check_layer(w, tol, Y, runner):
     ref, inter = O.layer_fwd(w.X, w.offsets, w.timestamps, w.weights[0], w.dims,
                              return_intermediates=True)
-    f1, o, z = (t.double().cpu().numpy() for t in runner.intermediates(w.B, w.T, w.max_len))
+    f1, o, z = runner.intermediates(w.B, w.T, w.max_len)
+    f1, z = f1.double().cpu().numpy(), z.double().cpu().numpy()
+    o = decode_o(o, w.dims.n_heads, w.dims.d_v)
     X = w.X.astype(np.float64)
     hdv = w.dims.n_heads * w.dims.d_v
     lw = w.weights[0]
