@@ -33,7 +33,8 @@ EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfa
             "hstu_read_status", "hstu_debug_offsets", "hstu_debug_keep_z",
             "hstu_debug_wait_test",
             "hstu_trace_enable", "hstu_trace_read",
-            "hstu_kernel_name", "hstu_launch_count", "hstu_last_error", "hstu_status_string",
+            "hstu_kernel_name", "hstu_launch_count", "hstu_last_error", "hstu_set_option",
+            "hstu_status_string",
             "hstu_version"]
 
 
@@ -142,6 +143,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_kernel_name.restype = ctypes.c_char_p
     L.hstu_launch_count.argtypes = []
     L.hstu_launch_count.restype = i64
+    L.hstu_set_option.argtypes = [ctypes.c_char_p, i64]
+    L.hstu_set_option.restype = i32
     L.hstu_last_error.argtypes = []
     L.hstu_last_error.restype = ctypes.c_char_p
     L.hstu_status_string.argtypes = [i32]
@@ -398,6 +401,10 @@ def hstu_debug_offsets(desc, B, total_tokens, max_len):
                                     ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
            "hstu_debug_offsets")
     return int(a.value), int(b.value), int(c.value)
+
+
+def hstu_set_option(name: str, value: int) -> None:
+    _check(lib().hstu_set_option(name.encode(), int(value)), "hstu_set_option")
 
 
 def hstu_debug_keep_z(on: bool) -> None:

@@ -171,18 +171,17 @@ cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const LayerOps& op
 // the caller's bf16 output when out16_bf16) and out32 (fp32 stream) may each
 // be null.  Each output element is read (residual) before it is written, by
 // the same warp, so a stream may be updated in place.
-// On the tensor-core path f2's A operand is LayerNorm(O) * U, built by the
-// GEMM itself from the attention's normalised O and statistics (`Z` is then
-// the normalised O, `ostats` its statistics, `f1` the layer's f1 output whose
-// first h*d_v columns are U, `z_dbg` an optional copy of Z); on the fp32 path
-// `Z` is the LayerNorm * U output.
+// With `ostats` (tensor-core path, LayerNorm * U fused): f2's A operand is
+// LayerNorm(O) * U, built by the GEMM itself from the attention's normalised
+// O (`Z`), its statistics (`ostats`) and U (the first h*d_v columns of `f1`);
+// `z_dbg` takes an optional copy of Z.  Without: `Z` is LayerNorm * U itself.
 cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, const void* Z,
                    const float* ostats, const void* f1, void* z_dbg,
                    const void* resid, int resid_kind, int64_t rows_cap, const int64_t* rows_dev,
                    void* out16, bool out16_bf16, float* out32) {
   GemmCall g{};
   g.A = Z;
-  if (c.bf16) {
+  if (c.bf16 && ostats) {  // Z formed in f2's operand stage
     g.A = nullptr;
     g.ln_x = Z;
     g.ln_stats = ostats;
@@ -273,12 +272,17 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
   a.ostats = c.bf16 ? at<float>(ws, L.ostats) : nullptr;
   e = attn(c, a);
   if (e != cudaSuccess) return e;
-  if (c.bf16)  // LayerNorm * U inside f2's operand stage
+  if (c.bf16 && ln_fusion())  // LayerNorm * U inside f2's operand stage
     return run_f2(c, w, ops, at<void>(ws, L.o), at<float>(ws, L.ostats), f1,
                   keep_z() ? at<void>(ws, L.z) : nullptr, resid, resid_kind, T, nullptr, out16,
                   out16_bf16, out32);
-  e = launch_ln_gate(c.d.dtype, at<void>(ws, L.o), f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps,
-                     at<void>(ws, L.z), c.hdv, T, nullptr, c.status, c.s);
+  if (c.bf16)  // LayerNorm * U from the normalised O, then f2 reads Z
+    e = launch_ln_gate_norm(at<void>(ws, L.o), at<float>(ws, L.ostats), f1, c.F, w.ln_gamma,
+                            w.ln_beta, c.d.ln_eps, at<void>(ws, L.z), c.hdv, c.d.n_heads,
+                            c.d.d_v, T, nullptr, c.status, c.s);
+  else
+    e = launch_ln_gate(c.d.dtype, at<void>(ws, L.o), f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps,
+                       at<void>(ws, L.z), c.hdv, T, nullptr, c.status, c.s);
   if (e != cudaSuccess) return e;
   return run_f2(c, w, ops, at<void>(ws, L.z), nullptr, nullptr, nullptr, resid, resid_kind, T,
                 nullptr, out16, out16_bf16, out32);
@@ -478,13 +482,18 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
       if (e != cudaSuccess) break;
       const void* resid = first ? xb_c : (const void*)xres_c;
       void* o16 = (c.bf16 && !last) ? xh_c : nullptr;
-      if (c.bf16) {  // LayerNorm * U inside f2's operand stage
+      if (c.bf16 && ln_fusion()) {  // LayerNorm * U inside f2's operand stage
         e = run_f2(c, weights[l], ops, oc, at<float>(ws, L.ostats_c), f1c, nullptr, resid,
                    first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);
         continue;
       }
-      e = launch_ln_gate(desc->dtype, oc, f1c, c.F, weights[l].ln_gamma, weights[l].ln_beta,
-                         desc->ln_eps, zc, c.hdv, R, rows_dev, c.status, c.s);
+      if (c.bf16)
+        e = launch_ln_gate_norm(oc, at<float>(ws, L.ostats_c), f1c, c.F, weights[l].ln_gamma,
+                                weights[l].ln_beta, desc->ln_eps, zc, c.hdv, desc->n_heads,
+                                desc->d_v, R, rows_dev, c.status, c.s);
+      else
+        e = launch_ln_gate(desc->dtype, oc, f1c, c.F, weights[l].ln_gamma, weights[l].ln_beta,
+                           desc->ln_eps, zc, c.hdv, R, rows_dev, c.status, c.s);
       if (e != cudaSuccess) break;
       e = run_f2(c, weights[l], ops, zc, nullptr, nullptr, nullptr, resid,
                  first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);

@@ -404,46 +404,55 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tmem_ld32(tmem + c0 + lane_base, sr);
           tmem_ld32(tmem + 128 + c0 + lane_base, dr);
           tmem_ld_wait();
+          // branch-free over the 32 elements: masked ones give P = dS = 0
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = tile * 128 + c0 + e;              // streamed row within the user
+            const int qi = MODE == MODE_DKV ? col : fixed_row;  // query row i
+            const int kj = MODE == MODE_DKV ? fixed_row : col;  // key row j
+            const bool ok_e = row_ok && col < n && kj <= qi;
+            const int tcol = __ldg(a.t_rel + u0 + min(col, n - 1));
+            const int ti = MODE == MODE_DKV ? tcol : t_row;
+            const int tj = MODE == MODE_DKV ? t_row : tcol;
+            const int bp = (int)log_bucket_nb(max(qi - kj, 0), a.Sp, a.Np);
+            const int bt = (int)log_bucket_nb(max(ti - tj, 0), a.St, a.Nt);
+            const float s = __uint_as_float(sr[e]) + __ldg(Rp + bp) + __ldg(Rt + bt);
+            const float sg = sigmoid_acc(s);
+            const float p = ok_e ? s * sg * inv_n : 0.f;
+            const float ds = ok_e ? __uint_as_float(dr[e]) * inv_n * sg * fmaf(s, 1.0f - sg, 1.0f)
+                                  : 0.f;
+            sr[e] = __float_as_uint(p);
+            dr[e] = __float_as_uint(ds);
+          }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float pv[2], dv2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int col = tile * 128 + c0 + e + u;          // streamed row within the user
-              const int qi = MODE == MODE_DKV ? col : fixed_row;  // query row i
-              const int kj = MODE == MODE_DKV ? fixed_row : col;  // key row j
-              const bool ok_e = row_ok && col < n && kj <= qi;
-              float p = 0.f, ds = 0.f;
-              if (ok_e) {
-                const int tcol = __ldg(a.t_rel + u0 + col);
-                const int ti = MODE == MODE_DKV ? tcol : t_row;
-                const int tj = MODE == MODE_DKV ? t_row : tcol;
-                const int bp = (int)log_bucket_nb(qi - kj, a.Sp, a.Np);
-                const int bt = (int)log_bucket_nb(max(ti - tj, 0), a.St, a.Nt);
-                const float s = __uint_as_float(sr[e + u]) + __ldg(Rp + bp) + __ldg(Rt + bt);
-                const float sg = sigmoid_acc(s);
-                p = s * sg * inv_n;
-                ds = __uint_as_float(dr[e + u]) * inv_n * sg * fmaf(s, 1.0f - sg, 1.0f);
-                if (MODE == MODE_DKV) {
-                  if (bp != cur_p) {
-                    if (cur_p >= 0) atomicAdd(dRp + cur_p, acc_p);
-                    cur_p = bp;
-                    acc_p = 0.f;
-                  }
-                  acc_p += ds;
-                  if (bt != cur_t) {
-                    if (cur_t >= 0) atomicAdd(dRt + cur_t, acc_t);
-                    cur_t = bt;
-                    acc_t = 0.f;
-                  }
-                  acc_t += ds;
-                }
+            pw[cc][e >> 1] = pack_f16x2_sat(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            sw[cc][e >> 1] = pack_f16x2_sat(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1]));
+          }
+          if (MODE == MODE_DKV) {
+            // the bias-table gradients: buckets change rarely along a row, so
+            // one atomic add per run of equal buckets
+#pragma unroll 4
+            for (int e = 0; e < 32; ++e) {
+              const int col = tile * 128 + c0 + e;
+              if (!(row_ok && col < n && fixed_row <= col)) continue;
+              const float ds = __uint_as_float(dr[e]);
+              const int bp = (int)log_bucket_nb(col - fixed_row, a.Sp, a.Np);
+              const int bt =
+                  (int)log_bucket_nb(max(__ldg(a.t_rel + u0 + col) - t_row, 0), a.St, a.Nt);
+              if (bp != cur_p) {
+                if (cur_p >= 0) atomicAdd(dRp + cur_p, acc_p);
+                cur_p = bp;
+                acc_p = 0.f;
               }
-              pv[u] = p;
-              dv2[u] = ds;
+              acc_p += ds;
+              if (bt != cur_t) {
+                if (cur_t >= 0) atomicAdd(dRt + cur_t, acc_t);
+                cur_t = bt;
+                acc_t = 0.f;
+              }
+              acc_t += ds;
             }
-            pw[cc][e >> 1] = pack_f16x2_sat(pv[0], pv[1]);
-            sw[cc][e >> 1] = pack_f16x2_sat(dv2[0], dv2[1]);
           }
         }
         if (MODE == MODE_DKV) {

@@ -467,16 +467,24 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     forward_parts(l);
     if (!ok()) break;
     GemmCall gc{};
-    gc.A = nullptr;
-    gc.ln_x = o_buf;
-    gc.ln_stats = ostats;
-    gc.ln_u = g_buf;
-    gc.ld_u = F;
-    gc.ln_gamma = W[l].ln_gamma;
-    gc.ln_beta = W[l].ln_beta;
-    gc.ln_eps = d.ln_eps;
-    gc.ln_h = h;
-    gc.ln_dv = d.d_v;
+    if (ln_fusion()) {  // LayerNorm * U inside f2's operand stage
+      gc.A = nullptr;
+      gc.ln_x = o_buf;
+      gc.ln_stats = ostats;
+      gc.ln_u = g_buf;
+      gc.ld_u = F;
+      gc.ln_gamma = W[l].ln_gamma;
+      gc.ln_beta = W[l].ln_beta;
+      gc.ln_eps = d.ln_eps;
+      gc.ln_h = h;
+      gc.ln_dv = d.d_v;
+    } else {
+      where = "LayerNorm * U (forward of the stack)";
+      e = launch_ln_gate_norm(o_buf, ostats, g_buf, F, W[l].ln_gamma, W[l].ln_beta, d.ln_eps,
+                              at<void>(ws, Lo.z), hdv, h, d.d_v, T, nullptr, status, s);
+      if (!ok()) break;
+      gc.A = at<void>(ws, Lo.z);
+    }
     gc.lda = hdv;
     gc.W = w2h(l);
     gc.ldw = hdv;

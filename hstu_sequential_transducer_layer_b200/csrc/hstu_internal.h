@@ -277,6 +277,17 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
                            int64_t rows_cap, const int64_t* rows_dev, const int* status,
                            cudaStream_t s);
 
+// Tensor-core path: Z = LayerNorm(O) * U from the attention's normalised O
+// (fp16 [rows, hdv]) and its per-(row, head) (mean, deviation) pairs.
+// hdv % 256 == 0, h <= 32.
+cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* f1, int64_t ld_f1,
+                                const void* gamma, const void* beta, float eps, void* Z, int hdv,
+                                int h, int dv, int64_t rows_cap, const int64_t* rows_dev,
+                                const int* status, cudaStream_t s);
+// Whether f2 forms LayerNorm * U in its operand stage (else a separate
+// kernel writes Z first); hstu_set_option("ln_fusion", ...).
+bool ln_fusion();
+
 // bf16 -> fp16 (round to nearest, saturating at +-65504) of up to
 // kMaxConvSegs segments in one launch; n elements each, multiples of 8.
 constexpr int kMaxConvSegs = 32;

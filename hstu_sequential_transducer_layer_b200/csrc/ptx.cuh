@@ -155,16 +155,23 @@ DEVI void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------- tcgen05
+// The warp-collective tcgen05 instructions (.sync.aligned: alloc, dealloc,
+// ld, st, wait) must be executed by all 32 lanes converged; each wrapper
+// reconverges the warp first, since callers reach them after lane-dependent
+// branches (ragged rows, lane-0 work).
 DEVI void tmem_alloc(uint32_t* slot, uint32_t ncols) {  // whole warp
+  __syncwarp();
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(slot)),
                "r"(ncols)
                : "memory");
 }
 DEVI void tmem_relinquish() {  // whole warp
+  __syncwarp();
   asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
 DEVI void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
+  __syncwarp();
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
@@ -234,6 +241,7 @@ DEVI void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32
 
 // 32 registers per thread -> 32 lanes x 32 consecutive 32-bit TMEM columns.
 DEVI void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -245,10 +253,14 @@ DEVI void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
-DEVI void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+DEVI void tmem_st_wait() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // 32 lanes x 32 consecutive 32-bit TMEM columns -> 32 registers per thread.
 DEVI void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -263,6 +275,7 @@ DEVI void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 // 32 lanes x 16 consecutive 32-bit TMEM columns -> 16 registers per thread.
 DEVI void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -273,6 +286,7 @@ DEVI void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 // 16 registers per thread -> 32 lanes x 16 consecutive 32-bit TMEM columns.
 DEVI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
@@ -281,7 +295,10 @@ DEVI void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
       "r"(r[15])
       : "memory");
 }
-DEVI void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+DEVI void tmem_ld_wait() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- score keys
 // Order-preserving 32-bit key of an fp32 score with the order reversed (a

@@ -2,6 +2,7 @@
 // device queries, TMA descriptor encoding, and the workspace layout.
 #include <atomic>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <map>
 #include <utility>
@@ -86,6 +87,12 @@ void note_cuda_error(cudaError_t e, const char* where) {
 }
 
 bool keep_z() { return g_keep_z.load(std::memory_order_relaxed) != 0; }
+
+namespace {
+std::atomic<int> g_ln_fusion{0};
+}  // namespace
+
+bool ln_fusion() { return g_ln_fusion.load(std::memory_order_relaxed) != 0; }
 
 void take_wait_test(uint32_t* limit_us, int* inject_stall) {
   std::lock_guard<std::mutex> lk(g_wait_mu);
@@ -231,6 +238,16 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
 extern "C" {
 
 const char* hstu_last_error(void) { return hstu::g_last_error; }
+
+hstu_status hstu_set_option(const char* name, int64_t value) {
+  if (!name) return HSTU_ERR_INVALID_ARG;
+  if (std::strcmp(name, "ln_fusion") == 0) {
+    if (value != 0 && value != 1) return HSTU_ERR_INVALID_ARG;
+    hstu::g_ln_fusion.store((int)value);
+    return HSTU_OK;
+  }
+  return HSTU_ERR_INVALID_ARG;
+}
 
 hstu_status hstu_debug_keep_z(int32_t on) {
   if (on != 0 && on != 1) return HSTU_ERR_INVALID_ARG;

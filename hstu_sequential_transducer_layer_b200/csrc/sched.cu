@@ -405,6 +405,80 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- LayerNorm * U from normalised O
+// Z = ((O - mu) * rstd * gamma + beta) * U, one warp per row, with O given as
+// the attention kernel stores it: per (row, head) its mean m and deviation s
+// (fp32) and the normalised values x = (O - m) / s (fp16), so (O - mu) * rstd
+// = a + b x with a = (m - mu) * rstd, b = s * rstd, and the row's moments
+// follow from the heads' (m, s): mu = mean m, var = mean (s^2 + (m - mu)^2).
+// Each lane takes 8 consecutive features per 256-feature chunk (all in one
+// head); lane hh holds head hh's statistics and broadcasts them by shuffle.
+__global__ void __launch_bounds__(256)
+    k_ln_gate_norm(const __half* __restrict__ xn, const float2* __restrict__ stats,
+                   const __half* __restrict__ f1, int64_t ld_f1,
+                   const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta,
+                   float eps, __half* __restrict__ Z, int hdv, int h, int dv, int64_t rows_cap,
+                   const int64_t* rows_dev, const int* status) {
+  if (status && *status != HSTU_OK) return;
+  int64_t rows = rows_cap;
+  if (rows_dev) rows = min(rows, *rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float2 st = lane < h ? stats[row * h + lane] : make_float2(0.f, 0.f);
+  float sm = st.x;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+  const float mu = sm / (float)h;
+  const float dm = st.x - mu;
+  float sv = lane < h ? fmaf(st.y, st.y, dm * dm) : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
+  const float rstd = rsqrtf(sv / (float)h + eps);
+  const float a_l = (st.x - mu) * rstd, b_l = st.y * rstd;  // this lane's head coefficients
+  const __half* xr = xn + row * hdv;
+  const __half* ur = f1 + row * ld_f1;
+  __half* zr = Z + row * hdv;
+  for (int k0 = lane * 8; k0 < hdv; k0 += 256) {
+    const int head = k0 / dv;
+    const float a = __shfl_sync(0xffffffffu, a_l, head);
+    const float b = __shfl_sync(0xffffffffu, b_l, head);
+    const uint4 xv = *reinterpret_cast<const uint4*>(xr + k0);
+    const uint4 uv = *reinterpret_cast<const uint4*>(ur + k0);
+    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gamma + k0));
+    const uint4 bv = __ldg(reinterpret_cast<const uint4*>(beta + k0));
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+    uint32_t zw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x2 = __half22float2(*reinterpret_cast<const __half2*>(&xw[e]));
+      const float2 u2 = __half22float2(*reinterpret_cast<const __half2*>(&uw[e]));
+      const float z0 = fmaf(fmaf(b, x2.x, a), bf16lo(gw[e]), bf16lo(bw[e])) * u2.x;
+      const float z1 = fmaf(fmaf(b, x2.y, a), bf16hi(gw[e]), bf16hi(bw[e])) * u2.y;
+      zw[e] = pack_f16x2_sat(z0, z1);
+    }
+    *reinterpret_cast<uint4*>(zr + k0) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+  }
+}
+
+cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* f1, int64_t ld_f1,
+                                const void* gamma, const void* beta, float eps, void* Z, int hdv,
+                                int h, int dv, int64_t rows_cap, const int64_t* rows_dev,
+                                const int* status, cudaStream_t s) {
+  if (rows_cap <= 0) return cudaSuccess;
+  if (h > 32 || hdv % 256 != 0 || dv % 8 != 0 || ld_f1 % 8 != 0) return cudaErrorInvalidValue;
+  LaunchScope ls(K_LN_GATE, s);
+  const int grid = (int)((rows_cap + 7) / 8);
+  k_ln_gate_norm<<<grid, 256, 0, s>>>(static_cast<const __half*>(xn),
+                                      reinterpret_cast<const float2*>(stats),
+                                      static_cast<const __half*>(f1), ld_f1,
+                                      static_cast<const __nv_bfloat16*>(gamma),
+                                      static_cast<const __nv_bfloat16*>(beta), eps,
+                                      static_cast<__half*>(Z), hdv, h, dv, rows_cap, rows_dev, status);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- bf16 -> fp16
 // One launch converts up to kMaxConvSegs segments (blockIdx.y = segment).
 __global__ void k_bf16_to_f16(ConvBatch cb) {

@@ -422,6 +422,13 @@ hstu_status hstu_debug_keep_z(int32_t on);
  * inject_stall other than 0 or 1. */
 hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall);
 
+/* Process-wide options.  "ln_fusion": 1 forms LayerNorm(O) * U inside the
+ * output projection's operand stage (Z never reaches memory), 0 (default)
+ * writes Z with a separate kernel that f2 then reads; both give the same
+ * layer within the bf16 bound.  Returns HSTU_ERR_INVALID_ARG for an unknown
+ * name or value. */
+hstu_status hstu_set_option(const char* name, int64_t value);
+
 /* After an entry point returned HSTU_ERR_CUDA: the failing CUDA runtime
  * call's error and the step it belonged to, as text (per host thread; ""
  * if none). */
