@@ -409,6 +409,7 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     peaks, peak_src = load_peaks()
+    H.hstu_set_option("ln_fusion", args.ln_fusion)
 
     # ---------------- inputs (a replica batch per rank)
     w = hw.full_stack(seed=args.seed + rank)
@@ -924,7 +925,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
             "data": "synthetic (seeded; random-init weights)",
-            "config": {"workload": "full_stack", "layers": w.n_layers, "d_model": w.dims.d_model,
+            "config": {"workload": "full_stack", "ln_fusion": args.ln_fusion,
+                       "layers": w.n_layers, "d_model": w.dims.d_model,
                        "heads": w.dims.n_heads, "head_dim": w.dims.d_qk, "users_per_gpu": w.B,
                        "tokens_per_gpu": T, "max_len": w.max_len,
                        "l2": "256 MB flush between timed steps",
@@ -1009,6 +1011,7 @@ def run_leg(args):
     make = {"full_stack": hw.full_stack, "long_history": hw.long_history,
             "single_layer": hw.single_layer, "mfalcon": hw.mfalcon,
             "backward": hw.full_stack}[args.leg]
+    H.hstu_set_option("ln_fusion", args.ln_fusion)
     w = make(seed=args.seed)
     r = H.HSTURunner(hw.dims_dict(w.dims), w.weights, dev)
     off, X, ts = r.to_device(w.offsets, "i64"), r.to_device(w.X), r.to_device(w.timestamps, "i64")
@@ -1053,6 +1056,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-legs", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--ln-fusion", type=int, default=0, choices=[0, 1],
+                    help="1: LayerNorm * U formed inside f2's operand stage; 0: a separate kernel")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)
     ap.add_argument("--leg", default=None,

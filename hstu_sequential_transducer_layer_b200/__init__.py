@@ -12,5 +12,7 @@ from .binding import (  # noqa: F401
     hstu_transformer_workspace_size, hstu_transformer_layer_fwd, TransformerWeights,
     hstu_read_status, hstu_debug_offsets, hstu_trace_enable, hstu_trace_read, hstu_kernel_name,
     hstu_launch_count, hstu_status_string, hstu_version, lib, LIB_PATH, EXPORTED,
+    LayerGrads, grads_array, hstu_bwd_workspace_size, hstu_layer_bwd, hstu_stack_bwd,
+    hstu_set_option, hstu_debug_keep_z, hstu_debug_wait_test,
 )
 from .runner import HSTURunner, TransformerRunner  # noqa: F401,E402

@@ -54,7 +54,7 @@ struct AttnBwdDev {
   const float* rab_time;
   float* drab_pos;          // MODE_DKV: [h, Np] fp32, accumulated (atomic adds)
   float* drab_time;         // MODE_DKV: [h, Nt]
-  int Np, Nt, Sp, St;
+  int Np, Nt, Sp, St, h;
   int32_t* work_next;
   int32_t* work_done;
   int* status;
@@ -67,7 +67,11 @@ struct BwdCfg {
   static constexpr uint32_t FIX_OFF = 0;            // 2 fixed tiles
   static constexpr uint32_t STR_OFF = FIX_OFF + 2 * TILE;   // RING x 2 streamed tiles
   static constexpr uint32_t PS_OFF = STR_OFF + RING * 2 * TILE;  // P^T and dS (2 x 32 KB)
-  static constexpr uint32_t BAR_OFF = PS_OFF + 2 * 32768;
+  // MODE_DKV: this CTA's bias-table gradient sums ([h][Np + Nt] fp32, when
+  // they fit), added to the global tables once at the end
+  static constexpr int BIN_FLOATS = 4096;
+  static constexpr uint32_t BIN_OFF = PS_OFF + 2 * 32768;
+  static constexpr uint32_t BAR_OFF = BIN_OFF + BIN_FLOATS * 4;
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr int EW0 = 4, NEW = 8;            // elementwise warps 4..11
   static constexpr int THREADS = 32 * (EW0 + NEW);
@@ -117,6 +121,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   int* s_nitems = s_go + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // bias-gradient bins in shared memory when every head's tables fit (shared
+  // atomics; the many CTAs of a head would otherwise all add into the same
+  // few global words near the diagonal's buckets)
+  float* bins = reinterpret_cast<float*>(smem + C::BIN_OFF);
+  const int nbin = a.h * (a.Np + a.Nt);
+  const bool use_bins = MODE == MODE_DKV && nbin <= C::BIN_FLOATS;
+  if (use_bins)
+    for (int i = threadIdx.x; i < nbin; i += blockDim.x) bins[i] = 0.f;
   if (threadIdx.x == 0) {
     const int st = a.status ? *reinterpret_cast<volatile int*>(a.status) : 0;
     *s_go = (st == 0);
@@ -382,8 +394,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int t_row = row_ok ? __ldg(a.t_rel + u0 + fixed_row) : 0;
       const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
       const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
-      float* dRp = a.drab_pos + (size_t)w.head * a.Np;
-      float* dRt = a.drab_time + (size_t)w.head * a.Nt;
+      float* dRp = use_bins ? bins + (size_t)w.head * (a.Np + a.Nt)
+                            : a.drab_pos + (size_t)w.head * a.Np;
+      float* dRt = use_bins ? bins + (size_t)w.head * (a.Np + a.Nt) + a.Np
+                            : a.drab_time + (size_t)w.head * a.Nt;
       const int nt = n_tiles_of(w);
       bool alive = true;
       for (int t = 0; t < nt; ++t, ++g) {
@@ -529,6 +543,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (use_bins) {  // this CTA's bias-gradient sums into the global tables
+    for (int i = threadIdx.x; i < nbin; i += blockDim.x) {
+      const float v = bins[i];
+      if (v != 0.f) {
+        const int hh = i / (a.Np + a.Nt), k = i - hh * (a.Np + a.Nt);
+        if (k < a.Np) atomicAdd(a.drab_pos + (size_t)hh * a.Np + k, v);
+        else atomicAdd(a.drab_time + (size_t)hh * a.Nt + (k - a.Np), v);
+      }
+    }
+  }
   if (threadIdx.x == 0) {
     // the last CTA to finish re-arms the work counter for the next launch
     __threadfence();
@@ -581,6 +605,7 @@ cudaError_t launch_attn_bwd(const AttnBwdCall& c, cudaStream_t s) {
   ad.Nt = c.Nt;
   ad.Sp = c.Sp;
   ad.St = c.St;
+  ad.h = c.h;
   ad.work_next = c.work_next;
   ad.work_done = c.work_done;
   ad.status = c.status;

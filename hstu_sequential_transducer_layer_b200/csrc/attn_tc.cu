@@ -395,41 +395,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const float* rt_ring = reinterpret_cast<const float*>(smem + C::RT_OFF);
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t scount = 0, ncon = 0;
-    uint32_t wt = 0;           // tiles this warp has started: window buffer parity
-    bool have_next = false;    // bw and window (wt & 1) already hold this item's tile 0
-    // Bias inputs of KV tile jt of item `it` into window buffer `buf` (and,
-    // causal mode, the tile's time-bucket words into bo).  Causal mode: the
-    // warp's 32 x 32 block spans the 63 distances base .. base + 62.
-    auto prep = [&](const AttnItem& it, int jt, int buf, uint32_t (&bo)[8]) {
-      float* win = win2 + buf * 64;
-      const float* Rp = a.rab_pos + (size_t)it.head * a.Np;
-      if (MODE == MODE_SELF) {
-        const uint32_t* tbw = a.tbuckets + (size_t)(it.tile0 + jt) * kBucketTileWords +
-                              (g * 8) * 128 + r;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) bo[m] = __ldg(tbw + m * 128);
-        const int base = (it.qt - jt) * 128 + q * 32 - g * 32 - 31;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int k = lane + 32 * u;
-          if (k < 63) {
-            const int dist = base + k;
-            win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
-          }
-        }
-      } else {
-        const float* Rt = a.rab_time + (size_t)it.head * a.Nt;
-        const int jc = jt * 128 + g * 32 + lane;
-        float bias = 0.f;
-        if (jc < it.n_kv) {
-          const int gap = max(a.t_req_rel[it.b] - a.t_rel[(int64_t)it.kv_row0 + jc], 0);
-          bias = __ldg(Rp + log_bucket(it.n_kv - jc, a.Sp, a.Np)) +
-                 __ldg(Rt + log_bucket(gap, a.St, a.Nt));
-        }
-        win[lane] = 0.5f * bias;
-      }
-    };
-    uint32_t bw[8], bwn[8];
     for (;;) {
       const int slot = ncon & 1;
       if (!mbar_wait_warp(it_full + slot, (ncon >> 1) & 1, ab, a.status)) break;
@@ -441,13 +406,47 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         if (lane == 0) mbar_arrive(it_empty + slot);
         break;
       }
+      const int64_t kv0 = w.kv_row0;
       const int n_kv = w.n_kv;                   // history / sequence length
-      if (w.nkv > 0 && !have_next) prep(w, 0, wt & 1, bw);
-      have_next = false;
+      const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
+      const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
+      const int t_i = (MODE == MODE_SELF) ? 0 : a.t_req_rel[w.b];
+      // Bias inputs of KV tile jt into window buffer `buf` (and, causal mode,
+      // the tile's time-bucket words into bwn).  Causal mode: the warp's
+      // 32 x 32 block spans the 63 distances base .. base + 62.
+      auto prep = [&](int jt, int buf, uint32_t (&bwn)[8]) {
+        float* win = win2 + buf * 64;
+        if (MODE == MODE_SELF) {
+          const uint32_t* tbw = a.tbuckets + (size_t)(w.tile0 + jt) * kBucketTileWords +
+                                (g * 8) * 128 + r;
+#pragma unroll
+          for (int m = 0; m < 8; ++m) bwn[m] = __ldg(tbw + m * 128);
+          const int base = (w.qt - jt) * 128 + q * 32 - g * 32 - 31;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int k = lane + 32 * u;
+            if (k < 63) {
+              const int dist = base + k;
+              win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
+            }
+          }
+        } else {
+          const int jc = jt * 128 + g * 32 + lane;
+          float bias = 0.f;
+          if (jc < n_kv) {
+            const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
+            bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
+                   __ldg(Rt + log_bucket(gap, a.St, a.Nt));
+          }
+          win[lane] = 0.5f * bias;
+        }
+      };
+      uint32_t bw[8], bwn[8];
+      if (w.nkv > 0) prep(0, 0, bw);
       bool alive = true;
-      for (int j = 0; j < w.nkv; ++j, ++wt) {
+      for (int j = 0; j < w.nkv; ++j) {
         __syncwarp();  // this tile's window is written; the one before it is free
-        const float* win = win2 + (wt & 1) * 64;
+        const float* win = win2 + (j & 1) * 64;
         // ---- S tile from TMEM: this warp's 32 rows x 32 columns
         const int sb = scount & 1;
         if (!mbar_wait_warp(s_full + sb, (scount >> 1) & 1, ab, a.status)) {
@@ -457,21 +456,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         tc_fence_after();
         uint32_t sr[32];
         tmem_ld32(tmem + sb * 128 + g * 32 + lane_base, sr);
-        // fetch the next tile's bias inputs while this tile computes -- at the
-        // item's last tile, those of the next item's first tile if the fetcher
-        // has published it already
-        if (j + 1 < w.nkv) {
-          prep(w, j + 1, (wt + 1) & 1, bwn);
-        } else {
-          const int ns = ncon & 1;
-          if (__all_sync(0xffffffffu, mbar_try_wait(it_full + ns, (ncon >> 1) & 1))) {
-            const AttnItem wn = ring[ns];
-            if (wn.b >= 0 && wn.nkv > 0) {
-              prep(wn, 0, (wt + 1) & 1, bwn);
-              have_next = true;
-            }
-          }
-        }
+        // fetch the next tile's bias inputs while this tile computes
+        if (j + 1 < w.nkv) prep(j + 1, (j + 1) & 1, bwn);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();

@@ -279,7 +279,7 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
 
 // Tensor-core path: Z = LayerNorm(O) * U from the attention's normalised O
 // (fp16 [rows, hdv]) and its per-(row, head) (mean, deviation) pairs.
-// hdv % 256 == 0, h <= 32.
+// hdv and d_v multiples of 8, h <= 32.
 cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* f1, int64_t ld_f1,
                                 const void* gamma, const void* beta, float eps, void* Z, int hdv,
                                 int h, int dv, int64_t rows_cap, const int64_t* rows_dev,

@@ -467,7 +467,7 @@ cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* 
                                 int h, int dv, int64_t rows_cap, const int64_t* rows_dev,
                                 const int* status, cudaStream_t s) {
   if (rows_cap <= 0) return cudaSuccess;
-  if (h > 32 || hdv % 256 != 0 || dv % 8 != 0 || ld_f1 % 8 != 0) return cudaErrorInvalidValue;
+  if (h > 32 || hdv % 8 != 0 || dv % 8 != 0 || ld_f1 % 8 != 0) return cudaErrorInvalidValue;
   LaunchScope ls(K_LN_GATE, s);
   const int grid = (int)((rows_cap + 7) / 8);
   k_ln_gate_norm<<<grid, 256, 0, s>>>(static_cast<const __half*>(xn),

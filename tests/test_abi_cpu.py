@@ -184,3 +184,40 @@ def test_new_entry_points_reject_bad_arguments_before_launch():
     assert L.hstu_bf16_to_f16(0x1002, 0x2000, 8, None) == 1
     assert L.hstu_bf16_to_f16(0x1000, 0x2000, 0, None) == 0
     assert H.hstu_launch_count() == n0
+
+
+def test_option_and_test_hook_arguments_checked():
+    """Process-wide options and test hooks reject what they do not know
+    (host only, nothing launched)."""
+    L = B.lib()
+    assert L.hstu_set_option(b"ln_fusion", 2) == 1
+    assert L.hstu_set_option(b"no_such_option", 0) == 1
+    assert L.hstu_set_option(None, 0) == 1
+    assert L.hstu_set_option(b"ln_fusion", 1) == 0
+    assert L.hstu_set_option(b"ln_fusion", 0) == 0
+    assert L.hstu_debug_keep_z(3) == 1
+    assert L.hstu_debug_wait_test(1000, 5) == 1
+    assert L.hstu_debug_wait_test(0, 0) == 0
+    assert L.hstu_last_error() is not None
+
+
+def test_bwd_workspace_and_argument_errors():
+    L = B.lib()
+    d = _desc()
+    a = B.hstu_bwd_workspace_size(d, 1, 4, 1000, 512)
+    b = B.hstu_bwd_workspace_size(d, 2, 4, 1000, 512)
+    assert 0 < a < b and a % 256 == 0
+    f = _desc("fp32", d=64, h=2, dqk=32, dv=32)
+    assert L.hstu_bwd_workspace_size(ctypes.byref(f), 1, 4, 100, 64) == 0   # bf16 only
+    g = B.LayerGrads(*([0x1000] * 8))
+    w = B.LayerWeights(*([0x1000] * 8))
+    code = L.hstu_layer_bwd(ctypes.byref(f), ctypes.byref(w), 4, 100, 64, 0x1000, 0x1000, 0x1000,
+                            0x1000, 0x1000, ctypes.byref(g), 0x1000, 1 << 20, None)
+    assert code == 2  # HSTU_ERR_UNSUPPORTED, nothing launched
+    code = L.hstu_layer_bwd(ctypes.byref(d), ctypes.byref(w), 4, 100, 64, 0x1000, 0x1000, 0x1000,
+                            0x1000, 0x1000, ctypes.byref(g), 0x1000, 1024, None)
+    assert code == 3  # workspace too small
+    bad = B.LayerGrads(*([0x1000] * 7 + [0]))
+    code = L.hstu_layer_bwd(ctypes.byref(d), ctypes.byref(w), 4, 100, 64, 0x1000, 0x1000, 0x1000,
+                            0x1000, 0x1000, ctypes.byref(bad), 0x1000, 1 << 40, None)
+    assert code == 1  # a null gradient pointer

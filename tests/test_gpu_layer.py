@@ -314,3 +314,28 @@ def test_residual_stream_near_fp16_limit():
     e, ed = relerr(Y, ref), rmserr(Y - X, ref - X)
     print("near-limit residual", peak, e, ed)
     assert e <= TOL[hw.BF16] and ed <= TOL[hw.BF16]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_ln_fusion_on_and_off_match_oracle(D):
+    """LayerNorm * U formed inside f2's operand stage (ln_fusion = 1) and by a
+    separate kernel (0, the default): both within the bound of the oracle on
+    a ragged 3-layer stack (and so within twice the bound of each other: the
+    fused path computes Z in packed fp16, the separate kernel in fp32)."""
+    from hstu_sequential_transducer_layer_b200 import binding as B
+    dims = hw.LayerDims(256, 2, D, D, 128, 128, 4, 2, 1e-6, hw.BF16)
+    w = hw.custom(f"lnfuse{D}", [300, 129, 1, 64, 0, 257], dims, n_layers=3, seed=95 + D)
+    ref = O.stack_fwd(w.X, w.offsets, w.timestamps, w.weights, dims)
+    X = w.X.astype(np.float64)
+    out = {}
+    try:
+        for f in (0, 1):
+            B.hstu_set_option("ln_fusion", f)
+            Y, _, _ = run_stack(w)
+            out[f] = Y
+            e, ed = relerr(Y, ref), rmserr(Y - X, ref - X)
+            print("ln_fusion", f, D, e, ed)
+            assert e <= TOL[hw.BF16] and ed <= TOL[hw.BF16], (f, e, ed)
+    finally:
+        B.hstu_set_option("ln_fusion", 0)
+    assert relerr(out[1], out[0]) <= 2 * TOL[hw.BF16]
