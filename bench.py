@@ -341,7 +341,7 @@ def time_leg(fn, args, flush, stream):
         fn()
         b.record(stream)
     torch.cuda.synchronize()
-    H.hstu_trace_enable(args.steps * 16 + 16)
+    H.hstu_trace_enable(args.steps * 256 + 256)
     for _ in range(args.steps):
         flush.zero_()
         fn()
@@ -814,15 +814,15 @@ def run_ours(args):
             raise RuntimeError(f"backward device status {r.bwd_status()}")
         # algorithmic work of the gradients: twice the forward's products (the
         # input-gradient and weight-gradient products of f1 and f2; dA, dV, dK
-        # and dQ against S and P.V in attention); the per-layer recompute of the
-        # forward is not counted
+        # and dQ against S and P.V in attention); the forward pass the call runs
+        # first is not counted
         b_flops = 2.0 * step_flops
         b_tf = b_flops / (b_ms / 1e3) / 1e12
         bwd = {"value": T / (b_ms / 1e3), "unit": "tokens/s", "ms_per_step": round(b_ms, 4),
                "tflops": round(b_tf, 1), "tensor_frac": tensor_frac(b_tf, peaks),
                "kernels_ms": b_k,
-               "note": "gradients of every parameter and of the input, 8 layers; each layer's "
-                       "forward is recomputed inside the call (not counted in tflops)",
+               "note": "gradients of every parameter and of the input, 8 layers; the stack's "
+                       "forward runs inside the call first (not counted in tflops)",
                "config": {"workload": "full_stack backward", "layers": w.n_layers,
                           "tokens": T}}
 
@@ -1035,9 +1035,24 @@ def run_leg(args):
         fn()
     e1.record()
     torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    # one more call with an event pair around every launch: per-kernel
+    # launches and device time of one call
+    H.hstu_trace_enable(8192)
+    fn()
+    torch.cuda.synchronize()
+    tr = H.hstu_trace_read()
+    H.hstu_trace_enable(0)
+    ker = {}
+    for kid, t in tr:
+        e = ker.setdefault(H.hstu_kernel_name(kid), [0, 0.0])
+        e[0] += 1
+        e[1] += t
     st = r.bwd_status() if args.leg == "backward" else r.status()
-    print(json.dumps({"leg": args.leg, "ms_per_call": e0.elapsed_time(e1) / args.steps,
-                      "status": st}), flush=True)
+    print(json.dumps({"leg": args.leg, "ms_per_call": ms, "status": st,
+                      "kernels_per_call": {k: [v[0], round(v[1], 4)] for k, v in
+                                           sorted(ker.items(), key=lambda kv: -kv[1][1])}}),
+          flush=True)
     if st != 0:
         raise SystemExit(1)
 

@@ -6,8 +6,9 @@
 // 'HSTUとGenerative Recommenders', section 'HSTUはTransformerと何が違うのか'
 // defines the forward layer; its gradients are the chain rule through it in
 // reverse order (section '長い履歴を現実の計算量へ収める4つの工夫' notes that
-// training keeps only a few activations per layer; here the backward
-// recomputes each layer's forward from the layer's input):
+// training keeps only a few activations per layer; here the call runs the
+// stack's forward once, keeping each layer's input, f1 output, f1
+// pre-activation and attention output in the workspace, then goes backward):
 //   Y = X + Z W2^T + b2      dZ = dY W2, dW2 = dY^T Z, db2 = sum dY, dX = dY + ...
 //   Z = L * U, L = LN(O) g + be
 //                            dL = dZ * U, dU = dZ * L, dg = sum dL xhat, dbe = sum dL,
@@ -27,92 +28,112 @@ namespace hstu {
 
 namespace {
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-constexpr int kLnBwdMaxPairs = 32;   // h*d_v <= 2048: 64 features per lane
 constexpr int kSumThreads = 256;
 constexpr int kGradSplits = 8;       // split-K of the weight-gradient products
-constexpr int kLnBwdBlocks = 1184;   // LayerNorm backward blocks (8 per SM)
+constexpr int kLnBwdGroups = 2368;   // LayerNorm backward row groups (partial rows of dg, dbe)
+constexpr int kLnSumSplit = 32;      // first-stage sums of those partial rows
+constexpr int kSumBlocks = 1184;     // row ranges of a column sum (8 blocks per SM)
+constexpr int kSumSplit = 32;        // first-stage sums of their partial rows
 }  // namespace
 
 // ---------------------------------------------------------------- LayerNorm * U backward
-// One warp per row.  O arrives as the attention kernel stores it, normalised
-// per (row, head): O = m + s * xn.  Per row: mu, rstd over all h*d_v features;
+// A group of G threads (G = 32, 64 or 128: one to four warps) per row, each
+// thread owning NV vectors of 8 consecutive features (vector gt + v G of the
+// row).  O arrives as the attention kernel stores it, normalised per (row,
+// head): O = m + s * xn.  Per row: mu, rstd over all h*d_v features;
 // xhat = (O - mu) rstd; L = xhat g + be; Z = L U (stored for dW2);
 // dL = dZ U; dU = dZ L, stored as dP_U = dU SiLU'(P_U) into the f1-shaped
 // gradient; dxh = dL g; dO = (dxh - mean dxh - xhat mean(dxh xhat)) rstd.
-// Column partial sums of dL xhat (dg) and dL (dbe) accumulate per warp in
-// shared memory (each lane owns its features: no atomics, a fixed order) and
-// are summed over the block's warps in warp order into one row per block.
+// The two row sums meet across the group's warps in shared memory (double-
+// buffered by row parity, one named barrier per row).  Column partial sums of
+// dL xhat (dg) and dL (dbe) stay in each thread's registers over all the rows
+// of its group (a fixed order) and are written as one partial row per group.
+template <int NV>
 __global__ void __launch_bounds__(256)
     k_ln_bwd(const float* __restrict__ dZ, const __half* __restrict__ xn,
              const float2* __restrict__ stats, const __half* __restrict__ f1,
              const __half* __restrict__ pre, int64_t ld_f1, const __nv_bfloat16* __restrict__ gamma,
              const __nv_bfloat16* __restrict__ beta, float eps, int hdv, int h, int dv,
-             int64_t rows, int64_t rows_per_block, __half* __restrict__ Z,
-             __half* __restrict__ dO, __half* __restrict__ dP, float* __restrict__ part,
-             const int* __restrict__ status) {
-  extern __shared__ float s_acc_all[];  // [warps][2][hdv]: dg, dbe partials per warp
+             int64_t rows, int G, __half* __restrict__ Z, __half* __restrict__ dO,
+             __half* __restrict__ dP, float* __restrict__ part, const int* __restrict__ status) {
+  __shared__ float2 red[2][8];  // [row parity][warp]: partial (sum dxh, sum dxh xhat)
   if (status && *status != HSTU_OK) return;
-  for (int i = threadIdx.x; i < 2 * hdv * (int)(blockDim.x / 32); i += blockDim.x) s_acc_all[i] = 0.f;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  float* s_acc = s_acc_all + (size_t)wid * 2 * hdv;
-  const int npair = hdv / 64;  // feature pairs per lane: features 2 lane + 64 j
-  const int64_t r_begin = blockIdx.x * rows_per_block;
-  const int64_t r_end = min(rows, r_begin + rows_per_block);
-  for (int64_t row = r_begin + wid; row < r_end; row += blockDim.x / 32) {
-    const float2* st = stats + row * h;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gpb = 256 / G;              // groups per block
+  const int grp = tid / G, gt = tid - grp * G;
+  const int W = G / 32, w0 = grp * W;   // warps of this group: w0 .. w0+W-1
+  const int64_t gid = (int64_t)blockIdx.x * gpb + grp;
+  const int64_t ngrp = (int64_t)gridDim.x * gpb;
+  const int nvec = hdv / 8;
+  const float inv_h = 1.0f / (float)h, inv_f = 1.0f / (float)hdv;
+  float ag[NV][8], ab[NV][8];
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ag[v][k] = ab[v][k] = 0.f;
+  int it = 0;
+  for (int64_t row = gid; row < rows; row += ngrp, ++it) {
     // row moments from the heads' (m, s): mu = mean m, var = mean (s^2 + (m - mu)^2)
-    float sm = 0.f;
-    for (int hh = lane; hh < h; hh += 32) sm += st[hh].x;
+    const float2 mine = lane < h ? stats[row * h + lane] : make_float2(0.f, 0.f);
+    float sm = mine.x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-    const float mu = sm / (float)h;
-    float sv = 0.f;
-    for (int hh = lane; hh < h; hh += 32) {
-      const float2 v = st[hh];
-      const float dm = v.x - mu;
-      sv = fmaf(v.y, v.y, fmaf(dm, dm, sv));
-    }
+    const float mu = sm * inv_h;
+    float sv = lane < h ? fmaf(mine.y, mine.y, (mine.x - mu) * (mine.x - mu)) : 0.f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
-    const float rstd = rsqrtf(sv / (float)h + eps);
-    float xh[2 * kLnBwdMaxPairs], dx[2 * kLnBwdMaxPairs];
+    const float rstd = rsqrtf(sv * inv_h + eps);
+    float xh[NV][8], dx[NV][8];
     float s_dx = 0.f, s_dxx = 0.f;
 #pragma unroll
-    for (int j = 0; j < kLnBwdMaxPairs; ++j) {
-      if (j < npair) {
-        const int k = 2 * lane + 64 * j;
-        const float2 hs = st[k / dv];
-        const __half2 xv = *reinterpret_cast<const __half2*>(xn + row * hdv + k);
-        const __half2 uv = *reinterpret_cast<const __half2*>(f1 + row * ld_f1 + k);
-        const __half2 pv = *reinterpret_cast<const __half2*>(pre + row * ld_f1 + k);
-        const float2 dz = *reinterpret_cast<const float2*>(dZ + row * hdv + k);
-        const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(gamma + k);
-        const __nv_bfloat162 bv = *reinterpret_cast<const __nv_bfloat162*>(beta + k);
-        const float x0 = (hs.x + hs.y * __low2float(xv) - mu) * rstd;
-        const float x1 = (hs.x + hs.y * __high2float(xv) - mu) * rstd;
-        const float g0 = __low2float(gv), g1 = __high2float(gv);
-        const float l0 = fmaf(x0, g0, __low2float(bv)), l1 = fmaf(x1, g1, __high2float(bv));
-        const float u0 = __low2float(uv), u1 = __high2float(uv);
-        *reinterpret_cast<__half2*>(Z + row * hdv + k) = __floats2half2_rn(l0 * u0, l1 * u1);
-        const float dl0 = dz.x * u0, dl1 = dz.y * u1;
-        // dP_U = dU * SiLU'(P_U), dU = dZ * L
-        const float p0 = __low2float(pv), p1 = __high2float(pv);
-        const float sg0 = __fdividef(1.0f, 1.0f + __expf(-p0));
-        const float sg1 = __fdividef(1.0f, 1.0f + __expf(-p1));
-        const float dp0 = dz.x * l0 * sg0 * fmaf(p0, 1.0f - sg0, 1.0f);
-        const float dp1 = dz.y * l1 * sg1 * fmaf(p1, 1.0f - sg1, 1.0f);
-        *reinterpret_cast<uint32_t*>(dP + row * ld_f1 + k) = pack_f16x2_sat(dp0, dp1);
-        s_acc[k] += dl0 * x0;
-        s_acc[k + 1] += dl1 * x1;
-        s_acc[hdv + k] += dl0;
-        s_acc[hdv + k + 1] += dl1;
-        xh[2 * j] = x0;
-        xh[2 * j + 1] = x1;
-        dx[2 * j] = dl0 * g0;
-        dx[2 * j + 1] = dl1 * g1;
-        s_dx += dx[2 * j] + dx[2 * j + 1];
-        s_dxx += dx[2 * j] * x0 + dx[2 * j + 1] * x1;
+    for (int v = 0; v < NV; ++v) {
+      const int vec = gt + v * G;
+      const int k = vec * 8;
+      const int head = min(k / dv, h - 1);
+      const float hm = __shfl_sync(0xffffffffu, mine.x, head);
+      const float hs = __shfl_sync(0xffffffffu, mine.y, head);
+      if (vec < nvec) {
+        const float a = (hm - mu) * rstd, b = hs * rstd;  // xhat = xn b + a
+        const uint4 xv = *reinterpret_cast<const uint4*>(xn + row * hdv + k);
+        const uint4 uv = *reinterpret_cast<const uint4*>(f1 + row * ld_f1 + k);
+        const uint4 pv = *reinterpret_cast<const uint4*>(pre + row * ld_f1 + k);
+        const float4 z0 = *reinterpret_cast<const float4*>(dZ + row * hdv + k);
+        const float4 z1 = *reinterpret_cast<const float4*>(dZ + row * hdv + k + 4);
+        const uint4 gv = *reinterpret_cast<const uint4*>(gamma + k);
+        const uint4 bv = *reinterpret_cast<const uint4*>(beta + k);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+        const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+        const float dz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+        uint32_t zo[4], po[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          float zz[2], pp[2];
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int e = 2 * e2 + hi;
+            const float x = fmaf(hi ? f16hi(xw[e2]) : f16lo(xw[e2]), b, a);
+            const float g = hi ? bf16hi(gw[e2]) : bf16lo(gw[e2]);
+            const float l = fmaf(x, g, hi ? bf16hi(bw[e2]) : bf16lo(bw[e2]));
+            const float u = hi ? f16hi(uw[e2]) : f16lo(uw[e2]);
+            const float p = hi ? f16hi(pw[e2]) : f16lo(pw[e2]);
+            zz[hi] = l * u;
+            const float dl = dz[e] * u;
+            // dP_U = dU * SiLU'(P_U), dU = dZ * L
+            const float sg = __fdividef(1.0f, 1.0f + __expf(-p));
+            pp[hi] = dz[e] * l * sg * fmaf(p, 1.0f - sg, 1.0f);
+            ag[v][e] = fmaf(dl, x, ag[v][e]);
+            ab[v][e] += dl;
+            xh[v][e] = x;
+            dx[v][e] = dl * g;
+            s_dx += dx[v][e];
+            s_dxx = fmaf(dx[v][e], x, s_dxx);
+          }
+          zo[e2] = pack_f16x2_sat(zz[0], zz[1]);
+          po[e2] = pack_f16x2_sat(pp[0], pp[1]);
+        }
+        *reinterpret_cast<uint4*>(Z + row * hdv + k) = make_uint4(zo[0], zo[1], zo[2], zo[3]);
+        *reinterpret_cast<uint4*>(dP + row * ld_f1 + k) = make_uint4(po[0], po[1], po[2], po[3]);
       }
     }
 #pragma unroll
@@ -120,52 +141,132 @@ __global__ void __launch_bounds__(256)
       s_dx += __shfl_xor_sync(0xffffffffu, s_dx, o);
       s_dxx += __shfl_xor_sync(0xffffffffu, s_dxx, o);
     }
-    const float m_dx = s_dx / (float)hdv, m_dxx = s_dxx / (float)hdv;
+    if (W > 1) {
+      if (lane == 0) red[it & 1][warp] = make_float2(s_dx, s_dxx);
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(G) : "memory");
+      s_dx = s_dxx = 0.f;
+      for (int ww = 0; ww < W; ++ww) {  // every thread sums in the same order
+        const float2 r2 = red[it & 1][w0 + ww];
+        s_dx += r2.x;
+        s_dxx += r2.y;
+      }
+    }
+    const float m_dx = s_dx * inv_f, m_dxx = s_dxx * inv_f;
 #pragma unroll
-    for (int j = 0; j < kLnBwdMaxPairs; ++j) {
-      if (j < npair) {
-        const int k = 2 * lane + 64 * j;
-        const float o0 = (dx[2 * j] - m_dx - xh[2 * j] * m_dxx) * rstd;
-        const float o1 = (dx[2 * j + 1] - m_dx - xh[2 * j + 1] * m_dxx) * rstd;
-        *reinterpret_cast<uint32_t*>(dO + row * hdv + k) = pack_f16x2_sat(o0, o1);
+    for (int v = 0; v < NV; ++v) {
+      const int vec = gt + v * G;
+      if (vec < nvec) {
+        uint32_t oo[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2)
+          oo[e2] = pack_f16x2_sat((dx[v][2 * e2] - m_dx - xh[v][2 * e2] * m_dxx) * rstd,
+                                  (dx[v][2 * e2 + 1] - m_dx - xh[v][2 * e2 + 1] * m_dxx) * rstd);
+        *reinterpret_cast<uint4*>(dO + row * hdv + vec * 8) = make_uint4(oo[0], oo[1], oo[2], oo[3]);
       }
     }
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 2 * hdv; i += blockDim.x) {
-    float acc = 0.f;
-    for (int wv = 0; wv < (int)(blockDim.x / 32); ++wv) acc += s_acc_all[(size_t)wv * 2 * hdv + i];
-    part[blockIdx.x * (int64_t)2 * hdv + i] = acc;
+  // this group's column partials: part[gid][0][.] = dg, part[gid][1][.] = dbe
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int vec = gt + v * G;
+    if (vec < nvec) {
+      float* pg = part + gid * 2 * hdv + vec * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        pg[e] = ag[v][e];
+        pg[hdv + e] = ab[v][e];
+      }
+    }
   }
 }
 
+// Threads per row of the LayerNorm backward for h*d_v features: one 8-feature
+// vector per thread up to four warps.
+static int ln_bwd_group(int hdv) { return std::min(128, std::max(32, (hdv / 8 + 31) / 32 * 32)); }
+
 // ---------------------------------------------------------------- reductions
-// part[blockIdx.y, n] = sum over rows [y * rows_per_block, ...) of in[r, n]
-// (fp32 or fp16 input, row stride ld).
+// part[blockIdx.x, n] = sum over rows [x * rows_per_block, ...) of in[r, n],
+// n < N (a multiple of 8; fp32 or fp16 input, row stride ld, 16-byte aligned
+// rows).  A thread sums 8 consecutive columns with 16-byte loads; when a row
+// has fewer than 256 such vectors the block's threads also split the rows
+// (row phase t / nvec) and the phases are added in a fixed order at the end.
+DEVI void load8(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+DEVI void load8(const __half* p, float (&v)[8]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = f16lo(w[k]);
+    v[2 * k + 1] = f16hi(w[k]);
+  }
+}
 template <typename T>
 __global__ void __launch_bounds__(kSumThreads)
-    k_sum_rows(const T* __restrict__ in, int64_t rows, int64_t N, int64_t ld,
-               int64_t rows_per_block, float* __restrict__ part, const int* __restrict__ status) {
+    k_sum_rows(const T* __restrict__ in, int64_t rows, int N, int64_t ld, int64_t rows_per_block,
+               float* __restrict__ part, const int* __restrict__ status) {
+  __shared__ float red[kSumThreads * 8];
   if (status && *status != HSTU_OK) return;
-  const int64_t n = blockIdx.x * (int64_t)kSumThreads + threadIdx.x;
-  if (n >= N) return;
-  const int64_t r0 = blockIdx.y * rows_per_block;
+  const int nvec = N / 8, t = threadIdx.x;
+  const int64_t r0 = blockIdx.x * rows_per_block;
   const int64_t r1 = min(rows, r0 + rows_per_block);
-  float acc = 0.f;
-  for (int64_t r = r0; r < r1; ++r) acc += (float)in[r * ld + n];
-  part[blockIdx.y * N + n] = acc;
+  float* out = part + (int64_t)blockIdx.x * N;
+  if (nvec >= kSumThreads) {
+    for (int v = t; v < nvec; v += kSumThreads) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int64_t r = r0; r < r1; ++r) {
+        float x[8];
+        load8(in + r * ld + v * 8, x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] += x[k];
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) out[v * 8 + k] = acc[k];
+    }
+    return;
+  }
+  const int RS = kSumThreads / nvec;  // row phases
+  const int v = t % nvec, rp = t / nvec;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (rp < RS) {
+#pragma unroll 4
+    for (int64_t r = r0 + rp; r < r1; r += RS) {
+      float x[8];
+      load8(in + r * ld + v * 8, x);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] += x[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) red[t * 8 + k] = acc[k];
+  __syncthreads();
+  if (t < nvec) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float sum = 0.f;
+      for (int q = 0; q < RS; ++q) sum += red[(q * nvec + t) * 8 + k];
+      out[t * 8 + k] = sum;
+    }
+  }
 }
 
-// out[x] = sum_{s < S} in[s * stride + x], x < L.
+// out[y * out_stride + x] = sum over slices s in [y * chunk, min(S, (y + 1) * chunk))
+// of in[s * stride + x], x < L, in slice order (gridDim.y = 1, chunk = S: one sum).
 __global__ void __launch_bounds__(kSumThreads)
     k_sum_slices(const float* __restrict__ in, int S, int64_t stride, int64_t L,
-                 float* __restrict__ out, const int* __restrict__ status) {
+                 float* __restrict__ out, const int* __restrict__ status, int chunk = 1 << 30,
+                 int64_t out_stride = 0) {
   if (status && *status != HSTU_OK) return;
+  const int s0 = blockIdx.y * chunk, s1 = min(S, s0 + chunk);
   for (int64_t x = blockIdx.x * (int64_t)kSumThreads + threadIdx.x; x < L;
        x += (int64_t)gridDim.x * kSumThreads) {
     float acc = 0.f;
-    for (int s = 0; s < S; ++s) acc += in[s * stride + x];
-    out[x] = acc;
+    for (int s = s0; s < s1; ++s) acc += in[s * stride + x];
+    out[blockIdx.y * out_stride + x] = acc;
   }
 }
 
@@ -212,34 +313,37 @@ cudaError_t convert(const void* src, int src_bf16, float* d32, __half* d16, int6
 
 // out[n] = sum over rows of in[r, n] (rows x N, row stride ld), via per-block
 // partials in `part` (at least 256 * N floats).
+// out[n] = sum over all rows of in[r, n] in a fixed order: kSumBlocks row
+// ranges (k_sum_rows), then kSumSplit sums of consecutive partial rows, then
+// their sum.  part holds (kSumBlocks + kSumSplit) * N floats.
 template <typename T>
 cudaError_t sum_rows(const T* in, int64_t rows, int64_t N, int64_t ld, float* part, float* out,
                      const int* status, cudaStream_t s) {
-  const int nb = (int)std::max<int64_t>(1, std::min<int64_t>(256, (rows + 127) / 128));
+  const int nb = (int)std::max<int64_t>(1, std::min<int64_t>(kSumBlocks, (rows + 15) / 16));
   const int64_t rpb = (rows + nb - 1) / nb;
-  {
-    LaunchScope ls(K_SUM_ROWS, s);
-    k_sum_rows<T><<<dim3((unsigned)((N + kSumThreads - 1) / kSumThreads), nb), kSumThreads, 0, s>>>(
-        in, rows, N, ld, rpb, part, status);
-  }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   LaunchScope ls(K_SUM_ROWS, s);
-  k_sum_slices<<<grid_for(N, kSumThreads), kSumThreads, 0, s>>>(part, nb, N, N, out, status);
+  k_sum_rows<T><<<nb, kSumThreads, 0, s>>>(in, rows, (int)N, ld, rpb, part, status);
+  float* tmp = part + (int64_t)nb * N;
+  const int chunk = (nb + kSumSplit - 1) / kSumSplit;
+  k_sum_slices<<<dim3((unsigned)grid_for(N, kSumThreads), kSumSplit), kSumThreads, 0, s>>>(
+      part, nb, N, N, tmp, status, chunk, N);
+  k_sum_slices<<<grid_for(N, kSumThreads), kSumThreads, 0, s>>>(tmp, kSumSplit, N, N, out, status);
   return cudaGetLastError();
 }
 
 struct BwdLayout {
   size_t header, items, t_rel, ubase, tbuckets;
   size_t xs;        // the layers' inputs, fp16, [n_layers][T, d]
-  size_t g, pre;    // f1 output and pre-activation, fp16 [T, F]
-  size_t o;         // normalised attention output fp16 [T, hdv] + (m, s) [T, h]
+  size_t g, pre;    // f1 output and pre-activation, fp16 [n_layers][T, F]
+  size_t o;         // normalised attention output fp16 [T, hdv] + (m, s) [T, h], per layer
+  size_t o_stride;  // bytes from one layer's o segment to the next
   size_t z, dz, dO, dP;
   size_t gy0, gy1;  // fp32 gradient streams [T, d]
   size_t gyh;       // fp16 copy of the current one
   size_t w16;       // fp16 copies of W1 and W2, per layer
   size_t part;      // partial sums
   size_t zbias;     // bf16 zeros
+  size_t rab_acc;   // fixed-point bias-table gradient sums [h][Np + Nt] (int64)
   size_t total;
   int64_t item_cap, tile_cap, part_floats;
 };
@@ -265,9 +369,10 @@ bool make_bwd_layout(const hstu_layer_desc& d, int L, int64_t B, int64_t T, int6
   o->ubase = take((size_t)(B + 1) * 8);
   o->tbuckets = take((size_t)o->tile_cap * kBucketTileWords * 4);
   o->xs = take((size_t)L * T * dm * 2);
-  o->g = take((size_t)T * F * 2);
-  o->pre = take((size_t)T * F * 2);
-  o->o = take(up256((size_t)T * hdv * 2) + (size_t)T * d.n_heads * 8);
+  o->g = take((size_t)L * T * F * 2);
+  o->pre = take((size_t)L * T * F * 2);
+  o->o_stride = up256(up256((size_t)T * hdv * 2) + (size_t)T * d.n_heads * 8);
+  o->o = take((size_t)L * o->o_stride);
   o->z = take((size_t)T * hdv * 2);
   o->dz = take((size_t)T * hdv * 4);
   o->dO = take((size_t)T * hdv * 2);
@@ -278,11 +383,12 @@ bool make_bwd_layout(const hstu_layer_desc& d, int L, int64_t B, int64_t T, int6
   o->w16 = take((size_t)L * (F * dm + dm * hdv) * 2);
   const size_t F_pad = (F + 127) / 128 * 128, d_pad = (dm + 127) / 128 * 128;
   const size_t part = std::max<size_t>({(size_t)kGradSplits * std::max(F_pad * dm, d_pad * hdv),
-                                        (size_t)kLnBwdBlocks * 2 * hdv,
-                                        (size_t)256 * std::max({F, hdv, dm})});
+                                        (size_t)(kLnBwdGroups + kLnSumSplit) * 2 * hdv,
+                                        (size_t)(kSumBlocks + kSumSplit) * std::max({F, hdv, dm})});
   o->part_floats = (int64_t)part;
   o->part = take(part * 4);
   o->zbias = take(std::max({F, hdv, dm}) * 2 + 1024);
+  o->rab_acc = take((size_t)d.n_heads * (d.n_pos_buckets + d.n_time_buckets) * 8);
   o->total = off;
   return true;
 }
@@ -398,13 +504,21 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
   };
   auto w2h = [&](int l) { return w1h(l) + (size_t)F * dm; };
   auto xs = [&](int l) { return at<__half>(ws, Lo.xs) + (size_t)l * T * dm; };
-  void* g_buf = at<void>(ws, Lo.g);
-  void* pre_buf = at<void>(ws, Lo.pre);
-  void* o_buf = at<void>(ws, Lo.o);
-  float* ostats = at<float>(ws, Lo.o + up256((size_t)T * hdv * 2));
+  // every layer's f1 output, pre-activation and attention output are kept
+  // from the forward pass for its backward (no recomputation)
+  auto g_of = [&](int l) { return at<__half>(ws, Lo.g) + (size_t)l * T * F; };
+  auto pre_of = [&](int l) { return at<__half>(ws, Lo.pre) + (size_t)l * T * F; };
+  auto o_of = [&](int l) { return at<__half>(ws, Lo.o + (size_t)l * Lo.o_stride); };
+  auto ostats_of = [&](int l) {
+    return at<float>(ws, Lo.o + (size_t)l * Lo.o_stride + up256((size_t)T * hdv * 2));
+  };
 
   // f1 (with its pre-activation) and the attention of layer l, from xs(l)
   auto forward_parts = [&](int l) {
+    void* g_buf = g_of(l);
+    void* pre_buf = pre_of(l);
+    void* o_buf = o_of(l);
+    float* ostats = ostats_of(l);
     GemmCall gc{};
     gc.A = xs(l);
     gc.lda = dm;
@@ -421,7 +535,7 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     gc.ldo = F;
     gc.epi = EPI_SILU;
     gc.status = status;
-    where = "f1 recompute";
+    where = "f1 (forward of the stack)";
     e = launch_gemm_tc(gc, s, K_GEMM_F1);
     if (!ok()) return;
     AttnCall ac{};
@@ -457,15 +571,19 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     ac.ldo = hdv;
     ac.ostats = ostats;
     ac.status = status;
-    where = "attention recompute";
+    where = "attention (forward of the stack)";
     e = launch_attn_tc(ac, s);
   };
 
-  // ---- forward through layers 0..L-2, keeping every layer's input (fp16)
+  // ---- forward through every layer, keeping each layer's input (fp16) and
+  // f1 / attention outputs; the last layer's f2 output is not needed
   e = convert(X, 1, nullptr, xs(0), (int64_t)T * dm, status, s);
-  for (int l = 0; l + 1 < L && ok(); ++l) {
+  for (int l = 0; l < L && ok(); ++l) {
     forward_parts(l);
-    if (!ok()) break;
+    if (!ok() || l == L - 1) break;
+    void* g_buf = g_of(l);
+    void* o_buf = o_of(l);
+    float* ostats = ostats_of(l);
     GemmCall gc{};
     if (ln_fusion()) {  // LayerNorm * U inside f2's operand stage
       gc.A = nullptr;
@@ -513,8 +631,10 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
   const int64_t F_pad = (F + 127) / 128 * 128, d_pad = (dm + 127) / 128 * 128;
   for (int l = L - 1; l >= 0 && ok(); --l) {
     const hstu_layer_grads& gr = grads[l];
-    forward_parts(l);
-    if (!ok()) break;
+    void* g_buf = g_of(l);
+    void* pre_buf = pre_of(l);
+    void* o_buf = o_of(l);
+    float* ostats = ostats_of(l);
     if (l < L - 1) e = convert(gy, 0, nullptr, gyh, (int64_t)T * dm, status, s);
     // dZ = dY W2
     GradGemm gg{};
@@ -535,27 +655,35 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     if (ok()) e = launch_gemm_grad(gg, s, K_GEMM_BWD);
     // LayerNorm * U backward: Z, dO, dP_U, and the dg / dbe partials
     if (ok()) {
-      // many short row ranges: each warp has few rows, so more loads are in flight
-      const int nb = (int)std::max<int64_t>(1, std::min<int64_t>(kLnBwdBlocks, (T + 31) / 32));
-      const int64_t rpb = (T + nb - 1) / nb;
+      // G threads per row, 256 / G rows at a time per block, at most
+      // kLnBwdGroups row groups (each leaves one partial row of dg, dbe)
+      const int G = ln_bwd_group(hdv), gpb = 256 / G;
+      const int nb = (int)std::max<int64_t>(
+          1, std::min<int64_t>(kLnBwdGroups / gpb, (T + gpb - 1) / gpb));
+      const int ngrp = nb * gpb;
       where = "LayerNorm backward";
       LaunchScope ls(K_LN_BWD, s);
-      const int ln_smem = 8 * 2 * hdv * 4;  // 8 warps x (dg, dbe) partials
-      e = ensure_smem_limit(reinterpret_cast<const void*>(k_ln_bwd), ln_smem);
-      if (!ok()) break;
-      k_ln_bwd<<<nb, 256, ln_smem, s>>>(
+      const bool two = hdv / 8 > G;  // two 8-feature vectors per thread (h*d_v > 1024)
+      auto kfn = two ? k_ln_bwd<2> : k_ln_bwd<1>;
+      kfn<<<nb, 256, 0, s>>>(
           at<float>(ws, Lo.dz), static_cast<const __half*>(o_buf),
           reinterpret_cast<const float2*>(ostats), static_cast<const __half*>(g_buf),
           static_cast<const __half*>(pre_buf), F, static_cast<const __nv_bfloat16*>(W[l].ln_gamma),
-          static_cast<const __nv_bfloat16*>(W[l].ln_beta), d.ln_eps, hdv, h, d.d_v, T, rpb,
+          static_cast<const __nv_bfloat16*>(W[l].ln_beta), d.ln_eps, hdv, h, d.d_v, T, G,
           at<__half>(ws, Lo.z), at<__half>(ws, Lo.dO), at<__half>(ws, Lo.dP), part, status);
       e = cudaGetLastError();
       if (ok()) {
+        // the ngrp partial rows [dg | dbe] in two stages (kLnSumSplit sums of
+        // consecutive partial rows, then their sum), each in a fixed order
         LaunchScope ls2(K_SUM_ROWS, s);
-        k_sum_slices<<<grid_for(hdv, kSumThreads), kSumThreads, 0, s>>>(part, nb, 2 * hdv, hdv,
-                                                                         gr.dln_gamma, status);
-        k_sum_slices<<<grid_for(hdv, kSumThreads), kSumThreads, 0, s>>>(part + hdv, nb, 2 * hdv,
-                                                                         hdv, gr.dln_beta, status);
+        float* tmp = part + (int64_t)ngrp * 2 * hdv;
+        const int chunk = (ngrp + kLnSumSplit - 1) / kLnSumSplit;
+        k_sum_slices<<<dim3((unsigned)grid_for(2 * hdv, kSumThreads), kLnSumSplit), kSumThreads, 0,
+                       s>>>(part, ngrp, 2 * hdv, 2 * hdv, tmp, status, chunk, 2 * hdv);
+        k_sum_slices<<<grid_for(hdv, kSumThreads), kSumThreads, 0, s>>>(tmp, kLnSumSplit, 2 * hdv,
+                                                                         hdv, gr.dln_gamma, status);
+        k_sum_slices<<<grid_for(hdv, kSumThreads), kSumThreads, 0, s>>>(
+            tmp + hdv, kLnSumSplit, 2 * hdv, hdv, gr.dln_beta, status);
         e = cudaGetLastError();
       }
     }
@@ -610,6 +738,7 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
       bc.rab_time = W[l].rab_time;
       bc.drab_pos = gr.drab_pos;
       bc.drab_time = gr.drab_time;
+      bc.rab_acc = at<unsigned long long>(ws, Lo.rab_acc);
       bc.Np = d.n_pos_buckets;
       bc.Nt = d.n_time_buckets;
       bc.Sp = d.pos_sub_bits;

@@ -263,7 +263,8 @@ struct AttnBwdCall {
   int q_col, k_col, v_col;
   const int32_t* t_rel;
   const float* rab_pos; const float* rab_time;
-  float* drab_pos; float* drab_time;
+  float* drab_pos; float* drab_time;   // written (not accumulated) from rab_acc
+  unsigned long long* rab_acc;         // workspace, h * (Np + Nt) words
   int Np, Nt, Sp, St, h, dqk, dv;
   int32_t* work_next; int32_t* work_done;
   int* status;

@@ -208,9 +208,10 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
  * 読むか': training is where the pages report the largest gain).  Given the
  * layers' input X and the gradient dY of a loss with respect to the stack's
  * output, computes dX (the gradient with respect to X) and, per layer, the
- * gradients of every parameter.  Each layer's forward is recomputed from its
- * input inside the call (the stack's forward runs once first to obtain the
- * layers' inputs), so nothing of a forward call has to be kept.
+ * gradients of every parameter.  The call runs the stack's forward itself
+ * first, keeping each layer's input, f1 output and pre-activation and
+ * attention output in the workspace (about 2 T (d + 2F + h d_v) bytes per
+ * layer), so nothing of an earlier forward call has to be kept.
  * Derivatives, per user (n = n_b) and head, written out by the chain rule:
  *   dZ = dY W2;  dW2 = dY^T Z;  db2 = sum_rows dY
  *   dL = dZ * U; dU = dZ * L (L = LayerNorm(O) before the gate); dgamma =
@@ -228,8 +229,9 @@ hstu_status hstu_layer_fwd_noalloc(const hstu_layer_desc* desc, int64_t B, int64
  * is overwritten (not accumulated into).  The tensor cores take fp16
  * operands with fp32 accumulation (as in the forward; the gradients flowing
  * into them must lie within fp16 range); the gradient stream between layers
- * is fp32.  The bias-table gradients are summed with atomic adds, so their
- * last bits may differ from run to run; everything else is deterministic.
+ * is fp32.  Every result is deterministic: the bias-table gradients are summed
+ * in 64-bit fixed point (units of 2^-32, each partial sum clamped to
+ * +-2^30), whose additions do not depend on their order, then rounded to fp32.
  * grads: host array [n_layers] of device pointers.  Workspace:
  * hstu_bwd_workspace_size() bytes, 256-byte aligned.  Asynchronous on
  * `stream`; device-detected errors (bad offsets or timestamps, a wait that
