@@ -176,7 +176,7 @@ cudaError_t run_f1(const Ctx& c, const hstu_layer_weights& w, const LayerOps& op
 // O (`Z`), its statistics (`ostats`) and U (the first h*d_v columns of `f1`);
 // `z_dbg` takes an optional copy of Z.  Without: `Z` is LayerNorm * U itself.
 cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& ops, const void* Z,
-                   const float* ostats, const void* f1, void* z_dbg,
+                   const float* ostats, uint32_t* coef, const void* f1, void* z_dbg,
                    const void* resid, int resid_kind, int64_t rows_cap, const int64_t* rows_dev,
                    void* out16, bool out16_bf16, float* out32) {
   GemmCall g{};
@@ -185,6 +185,7 @@ cudaError_t run_f2(const Ctx& c, const hstu_layer_weights& w, const LayerOps& op
     g.A = nullptr;
     g.ln_x = Z;
     g.ln_stats = ostats;
+    g.ln_coef = coef;
     g.ln_u = f1;
     g.ld_u = c.F;
     g.ln_gamma = w.ln_gamma;
@@ -273,9 +274,9 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
   e = attn(c, a);
   if (e != cudaSuccess) return e;
   if (c.bf16 && ln_fusion())  // LayerNorm * U inside f2's operand stage
-    return run_f2(c, w, ops, at<void>(ws, L.o), at<float>(ws, L.ostats), f1,
-                  keep_z() ? at<void>(ws, L.z) : nullptr, resid, resid_kind, T, nullptr, out16,
-                  out16_bf16, out32);
+    return run_f2(c, w, ops, at<void>(ws, L.o), at<float>(ws, L.ostats),
+                  at<uint32_t>(ws, L.lncoef), f1, keep_z() ? at<void>(ws, L.z) : nullptr, resid,
+                  resid_kind, T, nullptr, out16, out16_bf16, out32);
   if (c.bf16)  // LayerNorm * U from the normalised O, then f2 reads Z
     e = launch_ln_gate_norm(at<void>(ws, L.o), at<float>(ws, L.ostats), f1, c.F, w.ln_gamma,
                             w.ln_beta, c.d.ln_eps, at<void>(ws, L.z), c.hdv, c.d.n_heads,
@@ -284,8 +285,8 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
     e = launch_ln_gate(c.d.dtype, at<void>(ws, L.o), f1, c.F, w.ln_gamma, w.ln_beta, c.d.ln_eps,
                        at<void>(ws, L.z), c.hdv, T, nullptr, c.status, c.s);
   if (e != cudaSuccess) return e;
-  return run_f2(c, w, ops, at<void>(ws, L.z), nullptr, nullptr, nullptr, resid, resid_kind, T,
-                nullptr, out16, out16_bf16, out32);
+  return run_f2(c, w, ops, at<void>(ws, L.z), nullptr, nullptr, nullptr, nullptr, resid,
+                resid_kind, T, nullptr, out16, out16_bf16, out32);
 }
 
 hstu_status finish(cudaError_t e) {
@@ -483,7 +484,8 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
       const void* resid = first ? xb_c : (const void*)xres_c;
       void* o16 = (c.bf16 && !last) ? xh_c : nullptr;
       if (c.bf16 && ln_fusion()) {  // LayerNorm * U inside f2's operand stage
-        e = run_f2(c, weights[l], ops, oc, at<float>(ws, L.ostats_c), f1c, nullptr, resid,
+        e = run_f2(c, weights[l], ops, oc, at<float>(ws, L.ostats_c),
+                   at<uint32_t>(ws, L.lncoef_c), f1c, nullptr, resid,
                    first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);
         continue;
       }
@@ -495,7 +497,7 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
         e = launch_ln_gate(desc->dtype, oc, f1c, c.F, weights[l].ln_gamma, weights[l].ln_beta,
                            desc->ln_eps, zc, c.hdv, R, rows_dev, c.status, c.s);
       if (e != cudaSuccess) break;
-      e = run_f2(c, weights[l], ops, zc, nullptr, nullptr, nullptr, resid,
+      e = run_f2(c, weights[l], ops, zc, nullptr, nullptr, nullptr, nullptr, resid,
                  first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);
     }
     if (e == cudaSuccess)

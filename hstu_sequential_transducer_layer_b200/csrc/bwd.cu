@@ -344,6 +344,7 @@ struct BwdLayout {
   size_t part;      // partial sums
   size_t zbias;     // bf16 zeros
   size_t rab_acc;   // fixed-point bias-table gradient sums [h][Np + Nt] (int64)
+  size_t lncoef;    // LayerNorm coefficients per (row, head) (fused f2 of the forward)
   size_t total;
   int64_t item_cap, tile_cap, part_floats;
 };
@@ -389,6 +390,7 @@ bool make_bwd_layout(const hstu_layer_desc& d, int L, int64_t B, int64_t T, int6
   o->part = take(part * 4);
   o->zbias = take(std::max({F, hdv, dm}) * 2 + 1024);
   o->rab_acc = take((size_t)d.n_heads * (d.n_pos_buckets + d.n_time_buckets) * 8);
+  o->lncoef = take((size_t)T * d.n_heads * 4);
   o->total = off;
   return true;
 }
@@ -589,6 +591,7 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
       gc.A = nullptr;
       gc.ln_x = o_buf;
       gc.ln_stats = ostats;
+      gc.ln_coef = at<uint32_t>(ws, Lo.lncoef);
       gc.ln_u = g_buf;
       gc.ld_u = F;
       gc.ln_gamma = W[l].ln_gamma;

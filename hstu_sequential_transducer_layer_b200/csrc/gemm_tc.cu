@@ -50,7 +50,7 @@ struct GemmDev {
   int* overflow;
   // LNA: the A operand is LayerNorm(O) * U, built in shared memory
   const __half* ln_x;          // normalised O [M, K] fp16: (O - m) / s per (row, head)
-  const float2* ln_stats;      // [M, ln_h] (m, s) per (row, head)
+  const uint32_t* ln_coef;     // [M, ln_h] (a, b) fp16 pairs per (row, head)
   const __half* ln_u;          // U: the first K columns of the f1 output, row stride ld_u
   int64_t ld_u;
   const __nv_bfloat16* ln_gamma;
@@ -537,75 +537,49 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
       // rstd * gamma + beta) * U, in place in shared memory, once TMA has
       // brought the tile of normalised O (in A's 128-byte swizzled K-major
       // place) and the matching U tile (same layout).  O arrives normalised
-      // per (row, head): O = m + s * x, so with the row's LayerNorm moments
-      // mu, rstd, (O - mu) * rstd = a + b * x, a = (m - mu) * rstd, b = s *
-      // rstd.  Thread tw takes the 16-byte chunk c = tw & 7 of rows
-      // (tw >> 3) + 32 i, i = 0..3; the 8 threads of a row group are 8
-      // adjacent lanes.  The epilogue of tile t-1 runs once the first STAGES
-      // K blocks of tile t are turned (its accumulator is complete by then,
-      // and the MMAs have those stages to work on meanwhile).
+      // per (row, head): O = m + s * x, so (O - mu) * rstd = a + b * x with
+      // each (row, head)'s coefficients (a, b), computed before this launch
+      // (k_ln_coef) and fetched three K blocks ahead of their use.  Thread tw
+      // takes the 16-byte chunk c = tw & 7 of rows (tw >> 3) + 32 i, i = 0..3.
+      // The epilogue of tile t-1 runs once the first STAGES K blocks of tile t
+      // are turned (its accumulator is complete by then, and the MMAs have
+      // those stages to work on meanwhile).
       const int tw = threadIdx.x - 64;
       const int c = tw & 7;
       const int r0 = tw >> 3;
       const int K = g.K, H = g.ln_h;
+      const int kb_head = g.ln_dv / 64;  // K blocks per head
       int stg = 0;
       uint32_t ph = 0;
       bool ok = true;
       int t_prev = -1;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int mt = (t % mn_tiles) / n_tiles, nt = (t % mn_tiles) % n_tiles;
-        // the LayerNorm moments of this thread's 4 rows over all h * d_v
-        // features, from the heads' (m, s): mu = mean of m, var = mean of
-        // (s^2 + (m - mu)^2); the 8 lanes of a row group share the heads
-        float mu[4], rstd[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int64_t row = (int64_t)mt * 128 + r0 + 32 * i;
-          const bool ok_r = row < Mrows;
-          float2 hv[4];
-          float sm = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int hh = c + 8 * j;
-            hv[j] = (ok_r && hh < H) ? __ldg(g.ln_stats + row * H + hh) : make_float2(0.f, 0.f);
-            sm += hv[j].x;
-          }
-          sm += __shfl_xor_sync(0xffffffffu, sm, 1);
-          sm += __shfl_xor_sync(0xffffffffu, sm, 2);
-          sm += __shfl_xor_sync(0xffffffffu, sm, 4);
-          mu[i] = sm / (float)H;
-          float sv = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (c + 8 * j < H) {
-              const float dm = hv[j].x - mu[i];
-              sv = fmaf(hv[j].y, hv[j].y, fmaf(dm, dm, sv));
-            }
-          }
-          sv += __shfl_xor_sync(0xffffffffu, sv, 1);
-          sv += __shfl_xor_sync(0xffffffffu, sv, 2);
-          sv += __shfl_xor_sync(0xffffffffu, sv, 4);
-          rstd[i] = ok_r ? rsqrtf(sv / (float)H + g.ln_eps) : 0.f;
-        }
-        // per (row, head) statistics, gamma and beta of K block kb, fetched one
-        // block ahead of their use
-        float2 hsn[4];
-        uint4 gvn, bvn;
-        auto fetch = [&](int kb_) {
-          const int head = (kb_ * 64) / g.ln_dv;
+        // (a, b) of this thread's 4 rows for the heads of K blocks kb, kb+1,
+        // kb+2 (a three-deep register ring)
+        auto fetch_coef = [&](int kb_, uint32_t (&dst)[4]) {
+          const int head = min(kb_, KB - 1) / kb_head;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int64_t row = (int64_t)mt * 128 + r0 + 32 * i;
-            hsn[i] = row < Mrows ? __ldg(g.ln_stats + row * H + head) : make_float2(0.f, 0.f);
+            dst[i] = row < Mrows ? __ldg(g.ln_coef + row * H + head) : 0u;
           }
+        };
+        uint32_t cw0[4], cw1[4], cw2[4];
+        fetch_coef(0, cw0);
+        fetch_coef(1, cw1);
+        fetch_coef(2, cw2);
+        // gamma and beta of K block kb, fetched one block ahead of their use
+        uint4 gvn, bvn;
+        auto fetch = [&](int kb_) {
           gvn = __ldg(reinterpret_cast<const uint4*>(g.ln_gamma + kb_ * 64 + c * 8));
           bvn = __ldg(reinterpret_cast<const uint4*>(g.ln_beta + kb_ * 64 + c * 8));
         };
         fetch(0);
         for (int kb = 0; kb < KB; ++kb) {
           const int col = kb * 64 + c * 8;
-          // the previous tile's epilogue follows this K block; the next block's
-          // fetch then waits for it (fewer registers live across the epilogue)
+          // the previous tile's epilogue follows this K block; the next
+          // fetches then wait for it (fewer registers live across the epilogue)
           const bool epi_now = kb == (KB < STAGES ? KB : STAGES) - 1 && t_prev >= 0;
           // The transform runs in packed fp16 (two features per instruction on
           // the FMA pipes; fp16/fp32 conversions would saturate the XU pipe):
@@ -613,8 +587,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
           __half2 ca[4], cb[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            ca[i] = __float2half2_rn((hsn[i].x - mu[i]) * rstd[i]);
-            cb[i] = __float2half2_rn(hsn[i].y * rstd[i]);
+            const __half2 ab = *reinterpret_cast<const __half2*>(&cw0[i]);
+            ca[i] = __low2half2(ab);
+            cb[i] = __high2half2(ab);
+            cw0[i] = cw1[i];
+            cw1[i] = cw2[i];
           }
           __half2 gh[4], bh[4];
           {
@@ -625,7 +602,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
               bh[e] = __floats2half2_rn(bf16lo(bw[e]), bf16hi(bw[e]));
             }
           }
-          if (!epi_now && kb + 1 < KB) fetch(kb + 1);
+          if (!epi_now) {
+            fetch_coef(kb + 3, cw2);
+            if (kb + 1 < KB) fetch(kb + 1);
+          }
           // the normalised O and U of this stage have landed
           if (!mbar_wait_warp(full + stg, ph, ab, g.status)) {
             ok = false;
@@ -663,6 +643,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
               break;
             }
             t_prev = -1;
+            fetch_coef(kb + 3, cw2);
             if (kb + 1 < KB) fetch(kb + 1);
           }
         }
@@ -713,7 +694,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   CUtensorMap ta, tb, to16, to32, tr;
   const bool f16 = c.ab_f16 != 0;
   const bool lna = c.ln_x != nullptr;
-  if (lna && (c.epi != EPI_RESID || !f16 || !c.ln_stats || !c.ln_u || !c.ln_gamma ||
+  if (lna && (c.epi != EPI_RESID || !f16 || !c.ln_stats || !c.ln_coef || !c.ln_u || !c.ln_gamma ||
               !c.ln_beta || c.ln_h <= 0 || c.ln_dv % 64 != 0 || c.ln_h * c.ln_dv != c.K ||
               c.ld_u % 8 != 0))
     return cudaErrorInvalidValue;
@@ -779,7 +760,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   gd.resid_kind = c.resid_kind;
   gd.status = c.status;
   gd.ln_x = static_cast<const __half*>(c.ln_x);
-  gd.ln_stats = reinterpret_cast<const float2*>(c.ln_stats);
+  gd.ln_coef = c.ln_coef;
   gd.ln_u = static_cast<const __half*>(c.ln_u);
   gd.ld_u = c.ld_u;
   gd.ln_gamma = static_cast<const __nv_bfloat16*>(c.ln_gamma);
@@ -793,6 +774,11 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   gd.has_pre = c.out_pre != nullptr && c.epi == EPI_SILU;
   const int64_t tiles = mt * (c.N / BN);
   const int grid = (int)std::min<int64_t>(tiles, sms);
+  if (lna) {  // each (row, head)'s LayerNorm coefficients first
+    const cudaError_t e = launch_ln_coef(c.ln_stats, c.ln_h, c.ln_eps, c.ln_coef, c.M_cap, c.M_dev,
+                                         c.status, s);
+    if (e != cudaSuccess) return e;
+  }
   LaunchScope ls(kernel_id, s);
   if (c.epi == EPI_SILU) {
     if (BN == 256) return launch_one<256, 4, EPI_SILU>(ta, tb, to16, to32, tr, gd, grid, s);

@@ -53,7 +53,8 @@ enum KernelId : int32_t {
   K_LN_BWD = 34,
   K_SUM_ROWS = 35,
   K_F32_TO_F16 = 36,
-  K_NUM_KERNELS = 37
+  K_LN_COEF = 37,
+  K_NUM_KERNELS = 38
 };
 const char* kernel_name(int id);
 
@@ -105,6 +106,7 @@ struct Header {           // first 256 bytes of every workspace
 
 struct Layout {
   size_t header, items, t_rel, ubase, tbuckets, f1, o, ostats, z;
+  size_t lncoef, lncoef_c;  // tensor-core path: LayerNorm coefficients per (row, head)
   size_t xres, xh;          // residual stream: fp32 (fp32 path) / fp16, also the next f1's operand
   size_t w16;               // tensor-core path: fp16 copies of W1 (layers >= 1) and W2, per layer
   size_t f1_cache;          // M-FALCON: every layer's f1 output (its K/V) for the history
@@ -172,10 +174,12 @@ struct GemmCall {
   // builds A = LayerNorm(O) * U itself from the attention output stored as
   // (O - m) / s in fp16 (ln_x, [M, K]) with each (row, head)'s (m, s)
   // (ln_stats, [M, ln_h] pairs), U (the first K columns of ln_u, row stride
-  // ld_u), gamma and beta (bf16 [K]); K = ln_h * ln_dv.  z_dbg (optional, fp16
-  // [M, K]) receives Z.
+  // ld_u), gamma and beta (bf16 [K]); K = ln_h * ln_dv.  ln_coef: scratch of
+  // M * ln_h words for each (row, head)'s LayerNorm coefficients, which the
+  // launcher computes first.  z_dbg (optional, fp16 [M, K]) receives Z.
   const void* ln_x;
   const float* ln_stats;
+  uint32_t* ln_coef;
   const void* ln_u; int64_t ld_u;
   const void* ln_gamma; const void* ln_beta;
   float ln_eps;
@@ -281,6 +285,12 @@ cudaError_t launch_ln_gate(int dtype, const void* O, const void* f1, int64_t ld_
 // Tensor-core path: Z = LayerNorm(O) * U from the attention's normalised O
 // (fp16 [rows, hdv]) and its per-(row, head) (mean, deviation) pairs.
 // hdv and d_v multiples of 8, h <= 32.
+// Per (row, head) LayerNorm coefficients from the heads' (m, s): with the
+// row's moments mu, rstd over all h*d_v features, (O - mu) rstd = a + b xn for
+// the normalised O xn of that head, a = (m - mu) rstd, b = s rstd; written as
+// fp16 pairs (a in the low half) into coef [rows, h].
+cudaError_t launch_ln_coef(const float* stats, int h, float eps, uint32_t* coef, int64_t rows_cap,
+                           const int64_t* rows_dev, const int* status, cudaStream_t s);
 cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* f1, int64_t ld_f1,
                                 const void* gamma, const void* beta, float eps, void* Z, int hdv,
                                 int h, int dv, int64_t rows_cap, const int64_t* rows_dev,

@@ -31,7 +31,7 @@ const char* kernel_name(int id) {
       "sl_offsets", "sl_select", "sl_gather", "ret_gather", "gemm_scores_tc", "topk_chunk",
       "topk_merge", "tf_ln", "tf_qkv_tc", "tf_softmax_attn_tc", "tf_oproj_tc", "tf_ffn1_tc",
       "tf_ffn2_tc", "gemm_filter_tc", "filter_merge", "attn_bwd_dkv_tc", "attn_bwd_dq_tc",
-      "gemm_bwd_tc", "ln_bwd", "sum_rows", "f32_to_f16"};
+      "gemm_bwd_tc", "ln_bwd", "sum_rows", "f32_to_f16", "ln_coef"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "unknown";
 }
 
@@ -201,6 +201,8 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
   // by each (row, head)'s (mean, deviation) (tensor-core path)
   L->o = take(bf16 ? up256((size_t)T * hdv * 2) + (size_t)T * d.n_heads * 8 : (size_t)T * hdv * 4);
   L->ostats = bf16 ? L->o + up256((size_t)T * hdv * 2) : 0;
+  // LayerNorm coefficients per (row, head) for f2's operand stage
+  L->lncoef = bf16 ? take((size_t)T * d.n_heads * 4) : 0;
   // Z: the fp32 path's LayerNorm * U output; on the tensor-core path Z is
   // formed in the output projection's shared memory and written here only
   // when a test asks for it (hstu_debug_keep_z)
@@ -224,6 +226,7 @@ bool make_layout(const hstu_layer_desc& d, int n_layers, int64_t B, int64_t T, i
     L->oc = take(bf16 ? up256((size_t)cap * hdv * 2) + (size_t)cap * d.n_heads * 8
                       : (size_t)cap * hdv * 4);
     L->ostats_c = bf16 ? L->oc + up256((size_t)cap * hdv * 2) : 0;
+    L->lncoef_c = bf16 ? take((size_t)cap * d.n_heads * 4) : 0;
     L->zc = take((size_t)cap * hdv * es);
   }
   (void)max_len;

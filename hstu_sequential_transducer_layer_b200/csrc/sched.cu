@@ -479,6 +479,48 @@ cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* 
   return cudaGetLastError();
 }
 
+// One thread per row: the row's LayerNorm moments from its heads' (mean,
+// deviation) pairs, mu = mean of m, var = mean of (s^2 + (m - mu)^2), then
+// each head's coefficients a = (m - mu) rstd, b = s rstd as an fp16 pair.
+__global__ void k_ln_coef(const float2* __restrict__ stats, int h, float eps,
+                          uint32_t* __restrict__ coef, int64_t rows_cap,
+                          const int64_t* __restrict__ rows_dev, const int* __restrict__ status) {
+  if (status && *status != HSTU_OK) return;
+  int64_t rows = rows_cap;
+  if (rows_dev) rows = min(rows, *rows_dev);
+  const float inv_h = 1.0f / (float)h;
+  for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows;
+       r += (int64_t)gridDim.x * blockDim.x) {
+    const float2* st = stats + r * h;
+    float sm = 0.f;
+    for (int hh = 0; hh < h; ++hh) sm += st[hh].x;
+    const float mu = sm * inv_h;
+    float sv = 0.f;
+    for (int hh = 0; hh < h; ++hh) {
+      const float2 v = st[hh];
+      const float dm = v.x - mu;
+      sv = fmaf(v.y, v.y, fmaf(dm, dm, sv));
+    }
+    const float rstd = rsqrtf(sv * inv_h + eps);
+    for (int hh = 0; hh < h; ++hh) {
+      const float2 v = st[hh];
+      const __half2 ab = __floats2half2_rn((v.x - mu) * rstd, v.y * rstd);
+      coef[r * h + hh] = *reinterpret_cast<const uint32_t*>(&ab);
+    }
+  }
+}
+
+cudaError_t launch_ln_coef(const float* stats, int h, float eps, uint32_t* coef, int64_t rows_cap,
+                           const int64_t* rows_dev, const int* status, cudaStream_t s) {
+  if (rows_cap <= 0) return cudaSuccess;
+  if (h < 1 || h > 32 || !stats || !coef) return cudaErrorInvalidValue;
+  LaunchScope ls(K_LN_COEF, s);
+  const int grid = (int)std::min<int64_t>((rows_cap + 255) / 256, 8 * (int64_t)num_sms());
+  k_ln_coef<<<grid, 256, 0, s>>>(reinterpret_cast<const float2*>(stats), h, eps, coef, rows_cap,
+                                 rows_dev, status);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- bf16 -> fp16
 // One launch converts up to kMaxConvSegs segments (blockIdx.y = segment).
 __global__ void k_bf16_to_f16(ConvBatch cb) {
