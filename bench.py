@@ -60,6 +60,13 @@ def tensor_frac(tflops: float, peaks) -> dict:
             "of_nominal": round(tflops / 2250.0, 4)}
 
 
+def ln_mode_text(mode: int, d_model: int) -> str:
+    """Where LayerNorm * U runs for option `mode` at this layer width."""
+    inside = mode == 1 or (mode == 2 and d_model <= 512)
+    how = "inside f2's operand stage" if inside else "separate kernel, f2 reads Z"
+    return how + (" (chosen by width)" if mode == 2 else "")
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -855,6 +862,7 @@ def run_ours(args):
                 "cpu_baseline": (None if (world > 1 or args.no_cpu_baseline) else
                                  cpu_baseline_extrapolated(wl, args.cpu_tokens, shortest)),
                 "config": {"workload": name, "users": wl.B, "tokens": wl.T,
+                           "layernorm_u": ln_mode_text(args.ln_fusion, wl.dims.d_model),
                            "d_model": wl.dims.d_model, "heads": wl.dims.n_heads,
                            "head_dim": wl.dims.d_qk, "max_len": wl.max_len}}
             del rl, l_in, l_out
@@ -925,7 +933,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
             "data": "synthetic (seeded; random-init weights)",
-            "config": {"workload": "full_stack", "ln_fusion": args.ln_fusion,
+            "config": {"workload": "full_stack",
+                       "layernorm_u": ln_mode_text(args.ln_fusion, w.dims.d_model),
                        "layers": w.n_layers, "d_model": w.dims.d_model,
                        "heads": w.dims.n_heads, "head_dim": w.dims.d_qk, "users_per_gpu": w.B,
                        "tokens_per_gpu": T, "max_len": w.max_len,
@@ -1071,8 +1080,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer-legs", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--ln-fusion", type=int, default=0, choices=[0, 1],
-                    help="1: LayerNorm * U formed inside f2's operand stage; 0: a separate kernel")
+    ap.add_argument("--ln-fusion", type=int, default=2, choices=[0, 1, 2],
+                    help="1: LayerNorm * U formed inside f2's operand stage; 0: a separate "
+                         "kernel; 2: by layer width (inside f2 when d_model <= 512)")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)
     ap.add_argument("--leg", default=None,

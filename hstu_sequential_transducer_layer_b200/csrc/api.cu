@@ -273,7 +273,7 @@ cudaError_t run_layer(const Ctx& c, const hstu_layer_weights& w, const LayerOps&
   a.ostats = c.bf16 ? at<float>(ws, L.ostats) : nullptr;
   e = attn(c, a);
   if (e != cudaSuccess) return e;
-  if (c.bf16 && ln_fusion())  // LayerNorm * U inside f2's operand stage
+  if (c.bf16 && ln_fusion_for(c.d.d_model))  // LayerNorm * U inside f2's operand stage
     return run_f2(c, w, ops, at<void>(ws, L.o), at<float>(ws, L.ostats),
                   at<uint32_t>(ws, L.lncoef), f1, keep_z() ? at<void>(ws, L.z) : nullptr, resid,
                   resid_kind, T, nullptr, out16, out16_bf16, out32);
@@ -483,7 +483,7 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
       if (e != cudaSuccess) break;
       const void* resid = first ? xb_c : (const void*)xres_c;
       void* o16 = (c.bf16 && !last) ? xh_c : nullptr;
-      if (c.bf16 && ln_fusion()) {  // LayerNorm * U inside f2's operand stage
+      if (c.bf16 && ln_fusion_for(c.d.d_model)) {  // LayerNorm * U inside f2's operand stage
         e = run_f2(c, weights[l], ops, oc, at<float>(ws, L.ostats_c),
                    at<uint32_t>(ws, L.lncoef_c), f1c, nullptr, resid,
                    first ? RESID_BF16 : RESID_F32, R, rows_dev, o16, false, xres_c);

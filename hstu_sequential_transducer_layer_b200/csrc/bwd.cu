@@ -587,7 +587,7 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     void* o_buf = o_of(l);
     float* ostats = ostats_of(l);
     GemmCall gc{};
-    if (ln_fusion()) {  // LayerNorm * U inside f2's operand stage
+    if (ln_fusion_for(dm)) {  // LayerNorm * U inside f2's operand stage
       gc.A = nullptr;
       gc.ln_x = o_buf;
       gc.ln_stats = ostats;

@@ -66,6 +66,8 @@ struct GemmDev {
 };
 
 constexpr int kEpiThreads = 256;      // 8 epilogue warps
+constexpr int kLnaThreads = 128;      // LNA: 4 warps that form the A operand
+constexpr int kLnaRows = 128 / (kLnaThreads / 8);  // rows of each K block per such thread
 constexpr uint32_t kStageBuf = 4096;  // per-warp output staging bytes (32 x 32 fp32)
 
 // COMPACT (EPI_RESID with 16-bit residual and output only): 2 KB output and
@@ -89,7 +91,7 @@ struct GemmCfg {
   static constexpr uint32_t BAR_OFF = RES_OFF + (EPI == EPI_RESID ? (kEpiThreads / 32) * BUF : 0);
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static constexpr int THREADS = 64 + kEpiThreads;
+  static constexpr int THREADS = 64 + kEpiThreads + (LNA ? kLnaThreads : 0);
 };
 
 
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
-      mbar_init(afull + s, kEpiThreads / 32);  // LNA: one arrival per A-building warp
+      mbar_init(afull + s, kLnaThreads / 32);  // LNA: one arrival per A-building warp
     }
     mbar_init(tfull + 0, 1);
     mbar_init(tfull + 1, 1);
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
         mbar_wait(drain, 0, &tmp, nullptr);
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiThreads / 32) {
     const int q = warp & 3;              // TMEM lane quarter this warp may read
     const int part = (warp - 2) >> 2;    // which half of the BN columns
     constexpr int CH = BN / 64;          // 32-column chunks per warp
@@ -468,12 +470,21 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
       const uint32_t thr = (EPI == EPI_FILTER && valid) ? desc_key(g.tau[row * g.tau_stride]) : 0u;
       const uint32_t tbase = tmem + acc * BN + part * (BN / 2) + ((uint32_t)(q * 32) << 16);
       uint32_t ra[32], rb_acc[32];
+      // LNA kernels (more threads, fewer registers each) load one chunk at a
+      // time; the others load the next chunk while the current one is stored
+      constexpr bool kAhead = !LNA;
       tmem_ld32(tbase, ra);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
+        if (!kAhead && c > 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ba[i] = kNoBias ? make_uint4(0, 0, 0, 0) : __ldg(bptr + c * 4 + i);
+          tmem_ld32(tbase + c * 32, ra);
+          tmem_ld_wait();
+        }
         // the next chunk's accumulator and bias load while this chunk is stored
-        if (c + 1 < CH) {
+        if (kAhead && c + 1 < CH) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint4 bv = kNoBias ? make_uint4(0, 0, 0, 0) : __ldg(bptr + (c + 1) * 4 + i);
@@ -496,7 +507,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
         if (EPI == EPI_FILTER) {
           if (c & 1) gemm_filter_chunk(g, row, valid, col0 + c * 32, rb_acc, thr);
           else gemm_filter_chunk(g, row, valid, col0 + c * 32, ra, thr);
-        } else if (c & 1) {
+        } else if (kAhead && (c & 1)) {
           stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb_acc, bb,
                                    stage, COMPACT ? -1 : (nchunk & 1), rsm);
         } else {
@@ -520,7 +531,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
             }
           }
         }
-        if (c + 1 < CH) tmem_ld_wait();
+        if (kAhead && c + 1 < CH) tmem_ld_wait();
       }
       tc_fence_before();
       __syncwarp();
@@ -528,135 +539,108 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
       return true;
     };
 
-    if (!LNA) {
-      for (int t = blockIdx.x; t < tiles; t += gridDim.x)
-        if (!epi_tile(t)) break;
-    } else {
-      // ---------------------------------------------- LNA: A = LayerNorm(O) * U
-      // These warps also turn the A tile of every K block into Z = ((O - mu) *
-      // rstd * gamma + beta) * U, in place in shared memory, once TMA has
-      // brought the tile of normalised O (in A's 128-byte swizzled K-major
-      // place) and the matching U tile (same layout).  O arrives normalised
-      // per (row, head): O = m + s * x, so (O - mu) * rstd = a + b * x with
-      // each (row, head)'s coefficients (a, b), computed before this launch
-      // (k_ln_coef) and fetched three K blocks ahead of their use.  Thread tw
-      // takes the 16-byte chunk c = tw & 7 of rows (tw >> 3) + 32 i, i = 0..3.
-      // The epilogue of tile t-1 runs once the first STAGES K blocks of tile t
-      // are turned (its accumulator is complete by then, and the MMAs have
-      // those stages to work on meanwhile).
-      const int tw = threadIdx.x - 64;
-      const int c = tw & 7;
-      const int r0 = tw >> 3;
-      const int K = g.K, H = g.ln_h;
-      const int kb_head = g.ln_dv / 64;  // K blocks per head
-      int stg = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      int t_prev = -1;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int mt = (t % mn_tiles) / n_tiles, nt = (t % mn_tiles) % n_tiles;
-        // (a, b) of this thread's 4 rows for the heads of K blocks kb, kb+1,
-        // kb+2 (a three-deep register ring)
-        auto fetch_coef = [&](int kb_, uint32_t (&dst)[4]) {
-          const int head = min(kb_, KB - 1) / kb_head;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int64_t row = (int64_t)mt * 128 + r0 + 32 * i;
-            dst[i] = row < Mrows ? __ldg(g.ln_coef + row * H + head) : 0u;
-          }
-        };
-        uint32_t cw0[4], cw1[4], cw2[4];
-        fetch_coef(0, cw0);
-        fetch_coef(1, cw1);
-        fetch_coef(2, cw2);
-        // gamma and beta of K block kb, fetched one block ahead of their use
-        uint4 gvn, bvn;
-        auto fetch = [&](int kb_) {
-          gvn = __ldg(reinterpret_cast<const uint4*>(g.ln_gamma + kb_ * 64 + c * 8));
-          bvn = __ldg(reinterpret_cast<const uint4*>(g.ln_beta + kb_ * 64 + c * 8));
-        };
-        fetch(0);
-        for (int kb = 0; kb < KB; ++kb) {
-          const int col = kb * 64 + c * 8;
-          // the previous tile's epilogue follows this K block; the next
-          // fetches then wait for it (fewer registers live across the epilogue)
-          const bool epi_now = kb == (KB < STAGES ? KB : STAGES) - 1 && t_prev >= 0;
-          // The transform runs in packed fp16 (two features per instruction on
-          // the FMA pipes; fp16/fp32 conversions would saturate the XU pipe):
-          // t = a + b x, z = (t gamma + beta) u, each step rounded to fp16
-          __half2 ca[4], cb[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __half2 ab = *reinterpret_cast<const __half2*>(&cw0[i]);
-            ca[i] = __low2half2(ab);
-            cb[i] = __high2half2(ab);
-            cw0[i] = cw1[i];
-            cw1[i] = cw2[i];
-          }
-          __half2 gh[4], bh[4];
-          {
-            const uint32_t gw[4] = {gvn.x, gvn.y, gvn.z, gvn.w}, bw[4] = {bvn.x, bvn.y, bvn.z, bvn.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              gh[e] = __floats2half2_rn(bf16lo(gw[e]), bf16hi(gw[e]));
-              bh[e] = __floats2half2_rn(bf16lo(bw[e]), bf16hi(bw[e]));
-            }
-          }
-          if (!epi_now) {
-            fetch_coef(kb + 3, cw2);
-            if (kb + 1 < KB) fetch(kb + 1);
-          }
-          // the normalised O and U of this stage have landed
-          if (!mbar_wait_warp(full + stg, ph, ab, g.status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + stg * C::STAGE_BYTES;
-          const uint8_t* su = sa + C::A_BYTES;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = r0 + 32 * i;
-            const uint32_t off = r * 128 + ((c ^ (r & 7)) << 4);
-            uint4 xv = *reinterpret_cast<const uint4*>(sa + off);
-            const uint4 uv = *reinterpret_cast<const uint4*>(su + off);
-            __half2* xh = reinterpret_cast<__half2*>(&xv);
-            const __half2* uh = reinterpret_cast<const __half2*>(&uv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              xh[e] = __hmul2(__hfma2(__hfma2(cb[i], xh[e], ca[i]), gh[e], bh[e]), uh[e]);
-            const uint4 zv = xv;
-            *reinterpret_cast<uint4*>(sa + off) = zv;
-            const int64_t row = (int64_t)mt * 128 + r;
-            if (g.z_dbg && nt == 0 && row < Mrows)
-              *reinterpret_cast<uint4*>(g.z_dbg + row * K + col) = zv;
-          }
-          fence_proxy_async_smem();  // the tensor cores read what these threads wrote
-          __syncwarp();
-          if (lane == 0) mbar_arrive(afull + stg);
-          if (++stg == STAGES) {
-            stg = 0;
-            ph ^= 1;
-          }
-          if (epi_now) {
-            if (!epi_tile(t_prev)) {
-              ok = false;
-              break;
-            }
-            t_prev = -1;
-            fetch_coef(kb + 3, cw2);
-            if (kb + 1 < KB) fetch(kb + 1);
-          }
-        }
-        if (ok) t_prev = t;
-      }
-      if (ok && t_prev >= 0) epi_tile(t_prev);
-    }
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x)
+      if (!epi_tile(t)) break;
     if (lane == 0 && r_pending) {  // a residual load still in flight must land first
       AbortState tmp{0, kWaitLimitUs};
       mbar_wait(rb, rpar, &tmp, nullptr);
     }
     if (lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
     __syncwarp();
+  } else if (LNA) {
+    // ------------------------------------------------ LNA: A = LayerNorm(O) * U
+    // kLnaThreads / 32 warps turn the A tile of every K block into Z = ((O - mu) * rstd *
+    // gamma + beta) * U, in place in shared memory, once TMA has brought the
+    // tile of normalised O (in A's 128-byte swizzled K-major place) and the
+    // matching U tile (same layout); the MMA thread waits for their arrivals
+    // instead of TMA's.  O arrives normalised per (row, head): O = m + s * x,
+    // so (O - mu) * rstd = a + b * x with each (row, head)'s coefficients
+    // (a, b), computed before this launch (k_ln_coef) and fetched three K
+    // blocks ahead of their use.  Thread tw takes the 16-byte chunk c = tw & 7
+    // of rows (tw >> 3) + (kLnaThreads / 8) i, i < kLnaRows.  The transform runs in packed fp16
+    // (two features per instruction): t = a + b x, z = (t gamma + beta) u,
+    // each step rounded to fp16.
+    const int tw = threadIdx.x - 64 - kEpiThreads;
+    const int c = tw & 7;
+    const int r0 = tw >> 3;
+    const int K = g.K, H = g.ln_h;
+    const int kb_head = g.ln_dv / 64;  // K blocks per head
+    int stg = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      const int mt = (t % mn_tiles) / n_tiles, nt = (t % mn_tiles) % n_tiles;
+      auto fetch_coef = [&](int kb_, uint32_t (&dst)[kLnaRows]) {
+        const int head = min(kb_, KB - 1) / kb_head;
+#pragma unroll
+        for (int i = 0; i < kLnaRows; ++i) {
+          const int64_t row = (int64_t)mt * 128 + r0 + (kLnaThreads / 8) * i;
+          dst[i] = row < Mrows ? __ldg(g.ln_coef + row * H + head) : 0u;
+        }
+      };
+      uint32_t cw0[kLnaRows], cw1[kLnaRows], cw2[kLnaRows];
+      fetch_coef(0, cw0);
+      fetch_coef(1, cw1);
+      fetch_coef(2, cw2);
+      uint4 gvn = __ldg(reinterpret_cast<const uint4*>(g.ln_gamma + c * 8));
+      uint4 bvn = __ldg(reinterpret_cast<const uint4*>(g.ln_beta + c * 8));
+      for (int kb = 0; kb < KB; ++kb) {
+        const int col = kb * 64 + c * 8;
+        __half2 gh[4], bh[4];
+        {
+          const uint32_t gw[4] = {gvn.x, gvn.y, gvn.z, gvn.w}, bw[4] = {bvn.x, bvn.y, bvn.z, bvn.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            gh[e] = __floats2half2_rn(bf16lo(gw[e]), bf16hi(gw[e]));
+            bh[e] = __floats2half2_rn(bf16lo(bw[e]), bf16hi(bw[e]));
+          }
+        }
+        uint32_t cw[kLnaRows];
+#pragma unroll
+        for (int i = 0; i < kLnaRows; ++i) {
+          cw[i] = cw0[i];
+          cw0[i] = cw1[i];
+          cw1[i] = cw2[i];
+        }
+        fetch_coef(kb + 3, cw2);
+        if (kb + 1 < KB) {
+          gvn = __ldg(reinterpret_cast<const uint4*>(g.ln_gamma + col + 64));
+          bvn = __ldg(reinterpret_cast<const uint4*>(g.ln_beta + col + 64));
+        }
+        // the normalised O and U of this stage have landed
+        if (!mbar_wait_warp(full + stg, ph, ab, g.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + stg * C::STAGE_BYTES;
+        const uint8_t* su = sa + C::A_BYTES;
+#pragma unroll
+        for (int i = 0; i < kLnaRows; ++i) {
+          const int r = r0 + (kLnaThreads / 8) * i;
+          const uint32_t off = r * 128 + ((c ^ (r & 7)) << 4);
+          uint4 xv = *reinterpret_cast<const uint4*>(sa + off);
+          const uint4 uv = *reinterpret_cast<const uint4*>(su + off);
+          const __half2 ab2 = *reinterpret_cast<const __half2*>(&cw[i]);
+          const __half2 ca = __low2half2(ab2), cb = __high2half2(ab2);
+          __half2* xh = reinterpret_cast<__half2*>(&xv);
+          const __half2* uh = reinterpret_cast<const __half2*>(&uv);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            xh[e] = __hmul2(__hfma2(__hfma2(cb, xh[e], ca), gh[e], bh[e]), uh[e]);
+          *reinterpret_cast<uint4*>(sa + off) = xv;
+          const int64_t row = (int64_t)mt * 128 + r;
+          if (g.z_dbg && nt == 0 && row < Mrows)
+            *reinterpret_cast<uint4*>(g.z_dbg + row * K + col) = xv;
+        }
+        fence_proxy_async_smem();  // the tensor cores read what these threads wrote
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull + stg);
+        if (++stg == STAGES) {
+          stg = 0;
+          ph ^= 1;
+        }
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();

@@ -296,8 +296,8 @@ cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* 
                                 int h, int dv, int64_t rows_cap, const int64_t* rows_dev,
                                 const int* status, cudaStream_t s);
 // Whether f2 forms LayerNorm * U in its operand stage (else a separate
-// kernel writes Z first); hstu_set_option("ln_fusion", ...).
-bool ln_fusion();
+// kernel writes Z first) for a layer of this width; hstu_set_option("ln_fusion", ...).
+bool ln_fusion_for(int d_model);
 
 // bf16 -> fp16 (round to nearest, saturating at +-65504) of up to
 // kMaxConvSegs segments in one launch; n elements each, multiples of 8.

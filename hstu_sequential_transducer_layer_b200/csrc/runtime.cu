@@ -89,10 +89,16 @@ void note_cuda_error(cudaError_t e, const char* where) {
 bool keep_z() { return g_keep_z.load(std::memory_order_relaxed) != 0; }
 
 namespace {
-std::atomic<int> g_ln_fusion{0};
+std::atomic<int> g_ln_fusion{2};
 }  // namespace
 
-bool ln_fusion() { return g_ln_fusion.load(std::memory_order_relaxed) != 0; }
+// 2 (automatic): inside f2 when f2 has at most two 256-column output tiles
+// (d_model <= 512); with more, each A block would be formed once per tile and
+// the separate kernel is faster (measured on the 8-layer d_model = 1024 stack).
+bool ln_fusion_for(int d_model) {
+  const int m = g_ln_fusion.load(std::memory_order_relaxed);
+  return m == 1 || (m == 2 && d_model <= 512);
+}
 
 void take_wait_test(uint32_t* limit_us, int* inject_stall) {
   std::lock_guard<std::mutex> lk(g_wait_mu);
@@ -245,7 +251,7 @@ const char* hstu_last_error(void) { return hstu::g_last_error; }
 hstu_status hstu_set_option(const char* name, int64_t value) {
   if (!name) return HSTU_ERR_INVALID_ARG;
   if (std::strcmp(name, "ln_fusion") == 0) {
-    if (value != 0 && value != 1) return HSTU_ERR_INVALID_ARG;
+    if (value < 0 || value > 2) return HSTU_ERR_INVALID_ARG;
     hstu::g_ln_fusion.store((int)value);
     return HSTU_OK;
   }

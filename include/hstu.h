@@ -425,10 +425,12 @@ hstu_status hstu_debug_keep_z(int32_t on);
 hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall);
 
 /* Process-wide options.  "ln_fusion": 1 forms LayerNorm(O) * U inside the
- * output projection's operand stage (Z never reaches memory), 0 (default)
- * writes Z with a separate kernel that f2 then reads; both give the same
- * layer within the bf16 bound.  Returns HSTU_ERR_INVALID_ARG for an unknown
- * name or value. */
+ * output projection's operand stage (Z never reaches memory), 0 writes Z with
+ * a separate kernel that f2 then reads, 2 (default) chooses per layer: inside
+ * f2 when d_model <= 512 (f2 then has at most two 256-column output tiles,
+ * each of which forms Z again), the separate kernel otherwise.  All give the
+ * same layer within the bf16 bound.  Returns HSTU_ERR_INVALID_ARG for an
+ * unknown name or value. */
 hstu_status hstu_set_option(const char* name, int64_t value);
 
 /* After an entry point returned HSTU_ERR_CUDA: the failing CUDA runtime

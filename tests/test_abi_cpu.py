@@ -190,11 +190,13 @@ def test_option_and_test_hook_arguments_checked():
     """Process-wide options and test hooks reject what they do not know
     (host only, nothing launched)."""
     L = B.lib()
-    assert L.hstu_set_option(b"ln_fusion", 2) == 1
+    assert L.hstu_set_option(b"ln_fusion", 3) == 1
+    assert L.hstu_set_option(b"ln_fusion", -1) == 1
     assert L.hstu_set_option(b"no_such_option", 0) == 1
     assert L.hstu_set_option(None, 0) == 1
     assert L.hstu_set_option(b"ln_fusion", 1) == 0
     assert L.hstu_set_option(b"ln_fusion", 0) == 0
+    assert L.hstu_set_option(b"ln_fusion", 2) == 0
     assert L.hstu_debug_keep_z(3) == 1
     assert L.hstu_debug_wait_test(1000, 5) == 1
     assert L.hstu_debug_wait_test(0, 0) == 0
