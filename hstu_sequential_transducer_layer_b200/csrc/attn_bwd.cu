@@ -118,11 +118,7 @@ constexpr float kFixScale = 4294967296.0f;  // 2^32
 DEVI long long to_fix(float v) {
   return __float2ll_rn(fminf(fmaxf(v, -1073741824.0f), 1073741824.0f) * kFixScale);
 }
-DEVI float lds_f32(uint32_t addr) {
-  float v;
-  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
+
 DEVI void fix_add_shared(uint32_t lo_addr, uint32_t hi_addr, long long q) {
   const uint32_t ql = (uint32_t)q, qh = (uint32_t)((unsigned long long)q >> 32);
   uint32_t old;

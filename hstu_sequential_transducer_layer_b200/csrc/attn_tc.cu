@@ -465,15 +465,21 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const uint32_t tile = scount++;
         // ---- P = SiLU(S + bias), masked, fp16
         uint32_t pk[16];
+        // window and time table by shared-space loads: element c of this
+        // lane's row takes window entry lane + 31 - c and table entry b_c
+        const uint32_t wa = smem_u32(win) + 4u * (uint32_t)lane;
+        const uint32_t ra = smem_u32(rt);
         if (MODE == MODE_SELF) {
-          const float* wr = win + lane + 31;
           if (j == w.qt) {  // diagonal tile: causal mask j > i
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
               const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
               const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
-              float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, wr[-c]) + rt[b0]);
-              float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, wr[-c - 1]) + rt[b1]);
+              float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wa + 4u * (31 - c))) +
+                                   lds_f32(ra + 4u * b0));
+              float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f,
+                                        lds_f32(wa + 4u * (30 - c))) +
+                                   lds_f32(ra + 4u * b1));
               if (g * 32 + c > r) p0 = 0.f;
               if (g * 32 + c + 1 > r) p1 = 0.f;
               pk[c >> 1] = pack_f16x2_sat(p0, p1);
@@ -483,18 +489,22 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             for (int c = 0; c < 32; c += 2) {
               const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
               const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
-              const float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, wr[-c]) + rt[b0]);
-              const float p1 =
-                  silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, wr[-c - 1]) + rt[b1]);
+              const float p0 = silu_half(
+                  fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wa + 4u * (31 - c))) +
+                  lds_f32(ra + 4u * b0));
+              const float p1 = silu_half(
+                  fmaf(__uint_as_float(sr[c + 1]), 0.5f, lds_f32(wa + 4u * (30 - c))) +
+                  lds_f32(ra + 4u * b1));
               pk[c >> 1] = pack_f16x2_sat(p0, p1);
             }
           }
         } else {
           const int limit = n_kv - j * 128 - g * 32;
+          const uint32_t wc = smem_u32(win);
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, win[c]));
-            float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, win[c + 1]));
+            float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wc + 4u * c)));
+            float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, lds_f32(wc + 4u * (c + 1))));
             if (c >= limit) p0 = 0.f;
             if (c + 1 >= limit) p1 = 0.f;
             pk[c >> 1] = pack_f16x2_sat(p0, p1);

@@ -133,7 +133,7 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
         o.y = pack16(g.out_f16, v[k * 8 + 2], v[k * 8 + 3]);
         o.z = pack16(g.out_f16, v[k * 8 + 4], v[k * 8 + 5]);
         o.w = pack16(g.out_f16, v[k * 8 + 6], v[k * 8 + 7]);
-        *reinterpret_cast<uint4*>(stage + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = o;
+        sts_u128(smem_u32(stage) + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4), o);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -149,18 +149,17 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   } else if (g.resid_kind == RESID_F32) {  // residual chunk staged by TMA, 128-byte swizzle
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float4 rr = *reinterpret_cast<const float4*>(rsm + lane * 128 + ((k ^ (lane & 7)) << 4));
-      v[4 * k + 0] += rr.x;
-      v[4 * k + 1] += rr.y;
-      v[4 * k + 2] += rr.z;
-      v[4 * k + 3] += rr.w;
+      const uint4 rr = lds_u128(smem_u32(rsm) + lane * 128 + ((k ^ (lane & 7)) << 4));
+      v[4 * k + 0] += __uint_as_float(rr.x);
+      v[4 * k + 1] += __uint_as_float(rr.y);
+      v[4 * k + 2] += __uint_as_float(rr.z);
+      v[4 * k + 3] += __uint_as_float(rr.w);
     }
   } else {  // 16-bit residual chunk staged by TMA, 64-byte swizzle
     const int f16 = g.resid_kind == RESID_F16;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint4 rr =
-          *reinterpret_cast<const uint4*>(rsm + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4));
+      const uint4 rr = lds_u128(smem_u32(rsm) + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4));
       const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
@@ -180,11 +179,12 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
   if (both) {
     if (lane == 0) bulk_wait_read<0>();  // the warp's earlier stores have read the buffer
     __syncwarp();
-    uint8_t* rowp = stage + lane * 128;
+    const uint32_t rowp = smem_u32(stage) + lane * 128;
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      *reinterpret_cast<float4*>(rowp + ((k ^ (lane & 7)) << 4)) =
-          make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      sts_u128(rowp + ((k ^ (lane & 7)) << 4),
+               make_uint4(__float_as_uint(v[4 * k]), __float_as_uint(v[4 * k + 1]),
+                          __float_as_uint(v[4 * k + 2]), __float_as_uint(v[4 * k + 3])));
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -202,7 +202,7 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
       else bulk_wait_read<1>();
     }
     __syncwarp();
-    uint8_t* rowp = buf + lane * 64;
+    const uint32_t rowp = smem_u32(buf) + lane * 64;
     const int f16 = g.out_f16;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -211,7 +211,7 @@ DEVI bool gemm_chunk(const GemmDev& g, const CUtensorMap* tmO16, const CUtensorM
       o.y = pack16(f16, v[k * 8 + 2], v[k * 8 + 3]);
       o.z = pack16(f16, v[k * 8 + 4], v[k * 8 + 5]);
       o.w = pack16(f16, v[k * 8 + 6], v[k * 8 + 7]);
-      *reinterpret_cast<uint4*>(rowp + ((k ^ ((lane >> 1) & 3)) << 4)) = o;
+      sts_u128(rowp + ((k ^ ((lane >> 1) & 3)) << 4), o);
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -612,14 +612,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
           ok = false;
           break;
         }
-        uint8_t* sa = smem + stg * C::STAGE_BYTES;
-        const uint8_t* su = sa + C::A_BYTES;
+        const uint32_t sa = smem_u32(smem + stg * C::STAGE_BYTES);
+        const uint32_t su = sa + C::A_BYTES;
 #pragma unroll
         for (int i = 0; i < kLnaRows; ++i) {
           const int r = r0 + (kLnaThreads / 8) * i;
           const uint32_t off = r * 128 + ((c ^ (r & 7)) << 4);
-          uint4 xv = *reinterpret_cast<const uint4*>(sa + off);
-          const uint4 uv = *reinterpret_cast<const uint4*>(su + off);
+          uint4 xv = lds_u128(sa + off);
+          const uint4 uv = lds_u128(su + off);
           const __half2 ab2 = *reinterpret_cast<const __half2*>(&cw[i]);
           const __half2 ca = __low2half2(ab2), cb = __high2half2(ab2);
           __half2* xh = reinterpret_cast<__half2*>(&xv);
@@ -627,7 +627,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, STAGES, EPI, COMPACT, LNA>::THREAD
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             xh[e] = __hmul2(__hfma2(__hfma2(cb, xh[e], ca), gh[e], bh[e]), uh[e]);
-          *reinterpret_cast<uint4*>(sa + off) = xv;
+          sts_u128(sa + off, xv);
           const int64_t row = (int64_t)mt * 128 + r;
           if (g.z_dbg && nt == 0 && row < Mrows)
             *reinterpret_cast<uint4*>(g.z_dbg + row * K + col) = xv;
