@@ -114,7 +114,11 @@ typedef AttnItem RingItem;
 // y = x / 2 (score plus bias, halved); returns SiLU(x) = y + y tanh(y).
 DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
 
-template <int D, int MODE>
+// SPLIT (causal mode): a separate P loop without masks for tiles below the
+// diagonal (faster per element; for batches of short users, where every
+// other tile is a diagonal one, a single masked loop -- half the code -- is
+// faster).
+template <int D, int MODE, bool SPLIT>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
               const __grid_constant__ CUtensorMap tmO, const AttnDev a) {
@@ -470,7 +474,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const uint32_t wa = smem_u32(win) + 4u * (uint32_t)lane;
         const uint32_t ra = smem_u32(rt);
         if (MODE == MODE_SELF) {
-          if (j == w.qt) {  // diagonal tile: causal mask j > i
+          if (!SPLIT || j == w.qt) {
+            // the causal mask j > i on the diagonal tile; no column reaches
+            // the threshold on the others
+            const int lim = (j == w.qt) ? r - g * 32 : 1 << 20;
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
               const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
@@ -480,8 +487,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f,
                                         lds_f32(wa + 4u * (30 - c))) +
                                    lds_f32(ra + 4u * b1));
-              if (g * 32 + c > r) p0 = 0.f;
-              if (g * 32 + c + 1 > r) p1 = 0.f;
+              if (c > lim) p0 = 0.f;
+              if (c + 1 > lim) p1 = 0.f;
               pk[c >> 1] = pack_f16x2_sat(p0, p1);
             }
           } else {
@@ -746,12 +753,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   }
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool SPLIT = true>
 static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tkv,
                                     const CUtensorMap& to, const AttnDev& ad, int grid,
                                     cudaStream_t s) {
   using C = AttnCfg<D>;
-  auto kfn = k_attn_tc<D, MODE>;
+  auto kfn = k_attn_tc<D, MODE, SPLIT>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM);
   if (e != cudaSuccess) return e;
   kfn<<<grid, C::THREADS, C::SMEM, s>>>(tq, tkv, to, ad);
@@ -811,9 +818,16 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   take_wait_test(&ad.wait_limit_us, &ad.inject_stall);
   const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());
   LaunchScope ls(c.mode == MODE_SELF ? K_ATTN : K_ATTN_CAND, s);
-  if (c.mode == MODE_SELF)
-    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF>(tq, tkv, to, ad, grid, s)
-                       : launch_attn_inst<128, MODE_SELF>(tq, tkv, to, ad, grid, s);
+  if (c.mode == MODE_SELF) {
+    // users of 1024 rows or more on average: most tiles lie below the
+    // diagonal, so the unmasked loop pays for its code
+    const bool split = c.q_rows_cap >= 1024 * std::max<int64_t>(c.B, 1);
+    if (split)
+      return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF, true>(tq, tkv, to, ad, grid, s)
+                         : launch_attn_inst<128, MODE_SELF, true>(tq, tkv, to, ad, grid, s);
+    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF, false>(tq, tkv, to, ad, grid, s)
+                       : launch_attn_inst<128, MODE_SELF, false>(tq, tkv, to, ad, grid, s);
+  }
   return c.dqk == 64 ? launch_attn_inst<64, MODE_CAND>(tq, tkv, to, ad, grid, s)
                      : launch_attn_inst<128, MODE_CAND>(tq, tkv, to, ad, grid, s);
 }
