@@ -114,6 +114,43 @@ typedef AttnItem RingItem;
 // y = x / 2 (score plus bias, halved); returns SiLU(x) = y + y tanh(y).
 DEVI float silu_half(float y) { return fmaf(y, tanh_approx(y), y); }
 
+// A shared-memory float at base + OFF bytes (the offset in the instruction).
+template <int OFF>
+DEVI float lds_f32_at(uint32_t base) {
+  float v;
+  asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(base), "n"(OFF) : "memory");
+  return v;
+}
+
+// Causal P for columns C and C+1 of this warp's 32 x 32 block, then the next
+// pair: P = SiLU(S + position bias + time bias), zero where the column is past
+// `lim` (MASK).  wa: shared address of the lane's window entry (column c takes
+// entry 31 - c after it); ra: shared address of the head's halved time table;
+// bw: the block's bucket bytes, 4 columns per word.
+template <int C, bool MASK>
+struct PPair {
+  static DEVI void run(uint32_t (&pk)[16], const uint32_t (&sr)[32], const uint32_t (&bw)[8],
+                       uint32_t wa, uint32_t ra, int lim) {
+    const uint32_t b0 = __byte_perm(bw[C >> 2], 0u, 0x4440u | (C & 3));
+    const uint32_t b1 = __byte_perm(bw[C >> 2], 0u, 0x4440u | ((C + 1) & 3));
+    float p0 = silu_half(fmaf(__uint_as_float(sr[C]), 0.5f, lds_f32_at<4 * (31 - C)>(wa)) +
+                         lds_f32(ra + 4u * b0));
+    float p1 = silu_half(fmaf(__uint_as_float(sr[C + 1]), 0.5f, lds_f32_at<4 * (30 - C)>(wa)) +
+                         lds_f32(ra + 4u * b1));
+    if (MASK) {
+      if (C > lim) p0 = 0.f;
+      if (C + 1 > lim) p1 = 0.f;
+    }
+    pk[C >> 1] = pack_f16x2_sat(p0, p1);
+    PPair<C + 2, MASK>::run(pk, sr, bw, wa, ra, lim);
+  }
+};
+template <bool MASK>
+struct PPair<32, MASK> {
+  static DEVI void run(uint32_t (&)[16], const uint32_t (&)[32], const uint32_t (&)[8], uint32_t,
+                       uint32_t, int) {}
+};
+
 // SPLIT (causal mode): a separate P loop without masks for tiles below the
 // diagonal (faster per element; for batches of short users, where every
 // other tile is a diagonal one, a single masked loop -- half the code -- is
@@ -478,32 +515,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             // the causal mask j > i on the diagonal tile; no column reaches
             // the threshold on the others
             const int lim = (j == w.qt) ? r - g * 32 : 1 << 20;
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
-              const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
-              float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wa + 4u * (31 - c))) +
-                                   lds_f32(ra + 4u * b0));
-              float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f,
-                                        lds_f32(wa + 4u * (30 - c))) +
-                                   lds_f32(ra + 4u * b1));
-              if (c > lim) p0 = 0.f;
-              if (c + 1 > lim) p1 = 0.f;
-              pk[c >> 1] = pack_f16x2_sat(p0, p1);
-            }
+            PPair<0, true>::run(pk, sr, bw, wa, ra, lim);
           } else {
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const uint32_t b0 = __byte_perm(bw[c >> 2], 0u, 0x4440u | (c & 3));
-              const uint32_t b1 = __byte_perm(bw[c >> 2], 0u, 0x4440u | ((c + 1) & 3));
-              const float p0 = silu_half(
-                  fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wa + 4u * (31 - c))) +
-                  lds_f32(ra + 4u * b0));
-              const float p1 = silu_half(
-                  fmaf(__uint_as_float(sr[c + 1]), 0.5f, lds_f32(wa + 4u * (30 - c))) +
-                  lds_f32(ra + 4u * b1));
-              pk[c >> 1] = pack_f16x2_sat(p0, p1);
-            }
+            PPair<0, false>::run(pk, sr, bw, wa, ra, 0);
           }
         } else {
           const int limit = n_kv - j * 128 - g * 32;
@@ -641,8 +655,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int ob = litem & 1;
       if (!mbar_wait_warp(o_full + ob, (litem >> 1) & 1, ab, a.status)) break;
       tc_fence_after();
-      // O of this row and head, 16 columns from c16 * 16: the accumulator (or
-      // zero), plus the candidate's self term, times 1/n
+      // n O of this row and head, 16 columns from c16 * 16: the accumulator
+      // (or zero), plus the candidate's self term.  The 1/n of O cancels in
+      // the normalised values (O - mean) / sd and is applied to the stored
+      // mean and deviation only.
       auto load_o = [&](int c16, float (&o)[16]) {
         if (w.nkv > 0) {
           uint32_t orr[16];
@@ -667,8 +683,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             }
           }
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) o[i] *= inv_n;
       };
       // pass 1: mean and deviation of the row's D values, from sums shifted
       // by the first value (no cancellation when the mean dominates)
@@ -688,7 +702,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const float mean = shift + s1 * (1.0f / D);
       const float sd = sqrtf(fmaxf(s2 - s1 * s1 * (1.0f / D), 0.f) * (1.0f / D));
       const float inv_sd = sd > 0.f ? 1.0f / sd : 0.f;
-      if (row_ok) a.ostats[(q0 + r) * a.h + w.head] = make_float2(mean, sd);
+      const float nmean = -mean * inv_sd;  // (o - mean) / sd = o inv_sd + nmean
+      if (row_ok) a.ostats[(q0 + r) * a.h + w.head] = make_float2(mean * inv_n, sd * inv_n);
       // pass 2: (O - mean) / sd in fp16, 32 columns per store -- a full
       // 32-row block through swizzled staging and a TMA bulk store, a block
       // at the user's ragged end row by row (the rows after it belong to the
@@ -702,7 +717,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           load_o(c32 * 2 + hf, o);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            pk[hf * 8 + i] = pack_f16x2_sat((o[2 * i] - mean) * inv_sd, (o[2 * i + 1] - mean) * inv_sd);
+            pk[hf * 8 + i] = pack_f16x2_sat(fmaf(o[2 * i], inv_sd, nmean),
+                                            fmaf(o[2 * i + 1], inv_sd, nmean));
         }
         if (c32 == D / 32 - 1) {  // O is fully read: the next item may accumulate
           tc_fence_before();
