@@ -576,8 +576,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                               ? (frow0 + 31 < n && c0 + 15 < n && c0 >= frow0 + 31)
                               : (frow0 + 31 < n && c0 + 15 <= frow0);
         constexpr int HI = 4 * C::TAB_CAP;
+        // MODE_DKV runs every unit through the masked code (its bias-gradient
+        // additions make a second, unmasked copy of the loop cost more in
+        // instruction fetch than the masks cost)
         if (in_smem) {
-          if (full)
+          if (MODE == MODE_DQ && full)
             bwd_elems<MODE, false, true, HI>(sr, dr, out, c0, fixed_row, row_ok, n, tv, t_row,
                                              inv_n, bc, a.Sp, a.Np, a.St, a.Nt, cur_p, cur_t,
                                              acc_p, acc_t);

@@ -48,8 +48,10 @@ constexpr int kSumSplit = 32;        // first-stage sums of their partial rows
 // buffered by row parity, one named barrier per row).  Column partial sums of
 // dL xhat (dg) and dL (dbe) stay in each thread's registers over all the rows
 // of its group (a fixed order) and are written as one partial row per group.
+// Four blocks per SM (64 registers, a few spilled to L1): more rows in flight
+// matter more for this memory-bound kernel than the spills.
 template <int NV>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
     k_ln_bwd(const float* __restrict__ dZ, const __half* __restrict__ xn,
              const float2* __restrict__ stats, const __half* __restrict__ f1,
              const __half* __restrict__ pre, int64_t ld_f1, const __nv_bfloat16* __restrict__ gamma,
