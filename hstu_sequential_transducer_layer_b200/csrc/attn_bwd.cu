@@ -44,9 +44,8 @@
 // elementwise work and the epilogue.  Each elementwise warp writes its P^T
 // and dS^T (8 packed columns each) into the 16 TMEM columns it read S from,
 // so no warp overwrites columns another warp has yet to read.  The bias tables
-// of every head sit in shared memory (when they fit), the timestamps of a
-// unit's 16 streamed rows reach the lanes by shuffle, and elements of blocks
-// that lie wholly inside the causal region and the user skip the masks.
+// of every head sit in shared memory (when they fit) and the timestamps of a
+// unit's 16 streamed rows reach the lanes by shuffle.
 // Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -541,8 +540,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const int n = w.n_q;                       // the user's length
       const float inv_n = 1.0f / (float)max(n, 1);
       const int64_t u0 = w.kv_row0;              // the user's first row
-      const int frow0 = w.qt * 128 + q * 32;     // this warp's first fixed row
-      const int fixed_row = frow0 + lane;        // this thread's row within the user
+      const int fixed_row = w.qt * 128 + q * 32 + lane;  // this thread's row within the user
       const bool row_ok = fixed_row < n;
       const int t_row = row_ok ? __ldg(a.t_rel + u0 + fixed_row) : 0;
       BiasCtx bc;
@@ -572,22 +570,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         tmem_ld16(tmem + r * 64 + cb * 16 + lane_base, sr);
         tmem_ld16(tmem + C::DA_COL + r * 64 + cb * 16 + lane_base, dr);
         tmem_ld_wait();
-        const bool full = MODE == MODE_DKV
-                              ? (frow0 + 31 < n && c0 + 15 < n && c0 >= frow0 + 31)
-                              : (frow0 + 31 < n && c0 + 15 <= frow0);
         constexpr int HI = 4 * C::TAB_CAP;
-        // MODE_DKV runs every unit through the masked code (its bias-gradient
-        // additions make a second, unmasked copy of the loop cost more in
-        // instruction fetch than the masks cost)
+        // every unit runs through the masked code: a second, unmasked copy of
+        // the loop for the blocks inside the causal region and the user (a
+        // measured 7-12 % slower) costs more in instruction fetch than the
+        // masks cost
         if (in_smem) {
-          if (MODE == MODE_DQ && full)
-            bwd_elems<MODE, false, true, HI>(sr, dr, out, c0, fixed_row, row_ok, n, tv, t_row,
-                                             inv_n, bc, a.Sp, a.Np, a.St, a.Nt, cur_p, cur_t,
-                                             acc_p, acc_t);
-          else
-            bwd_elems<MODE, true, true, HI>(sr, dr, out, c0, fixed_row, row_ok, n, tv, t_row,
-                                            inv_n, bc, a.Sp, a.Np, a.St, a.Nt, cur_p, cur_t, acc_p,
-                                            acc_t);
+          bwd_elems<MODE, true, true, HI>(sr, dr, out, c0, fixed_row, row_ok, n, tv, t_row, inv_n,
+                                          bc, a.Sp, a.Np, a.St, a.Nt, cur_p, cur_t, acc_p, acc_t);
         } else {
           bwd_elems<MODE, true, false, HI>(sr, dr, out, c0, fixed_row, row_ok, n, tv, t_row, inv_n,
                                            bc, a.Sp, a.Np, a.St, a.Nt, cur_p, cur_t, acc_p, acc_t);
