@@ -439,12 +439,26 @@ __global__ void __launch_bounds__(256)
   const __half* xr = xn + row * hdv;
   const __half* ur = f1 + row * ld_f1;
   __half* zr = Z + row * hdv;
-  for (int k0 = lane * 8; k0 < hdv; k0 += 256) {
-    const int head = k0 / dv;
+  // every chunk's O and U loads are issued before the first is used
+  constexpr int kMaxChunks = 8;  // h * d_v <= 2048
+  uint4 xva[kMaxChunks], uva[kMaxChunks];
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    const int k0 = lane * 8 + 256 * c;
+    if (k0 < hdv) {
+      xva[c] = *reinterpret_cast<const uint4*>(xr + k0);
+      uva[c] = *reinterpret_cast<const uint4*>(ur + k0);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    const int k0 = lane * 8 + 256 * c;
+    const int head = min(k0, hdv - 1) / dv;
     const float a = __shfl_sync(0xffffffffu, a_l, head);
     const float b = __shfl_sync(0xffffffffu, b_l, head);
-    const uint4 xv = *reinterpret_cast<const uint4*>(xr + k0);
-    const uint4 uv = *reinterpret_cast<const uint4*>(ur + k0);
+    if (k0 >= hdv) continue;
+    const uint4 xv = xva[c];
+    const uint4 uv = uva[c];
     const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gamma + k0));
     const uint4 bv = __ldg(reinterpret_cast<const uint4*>(beta + k0));
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
@@ -467,7 +481,8 @@ cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* 
                                 int h, int dv, int64_t rows_cap, const int64_t* rows_dev,
                                 const int* status, cudaStream_t s) {
   if (rows_cap <= 0) return cudaSuccess;
-  if (h > 32 || hdv % 8 != 0 || dv % 8 != 0 || ld_f1 % 8 != 0) return cudaErrorInvalidValue;
+  if (h > 32 || hdv % 8 != 0 || hdv > 2048 || dv % 8 != 0 || ld_f1 % 8 != 0)
+    return cudaErrorInvalidValue;
   LaunchScope ls(K_LN_GATE, s);
   const int grid = (int)((rows_cap + 7) / 8);
   k_ln_gate_norm<<<grid, 256, 0, s>>>(static_cast<const __half*>(xn),
