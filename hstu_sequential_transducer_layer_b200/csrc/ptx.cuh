@@ -387,10 +387,12 @@ DEVI int log_bucket(int x, int S, int N) {
 }
 // log_bucket without branches (the same values; x >= 0): lanes of a warp
 // whose distances fall on both sides of 2^S do not diverge.
+// The same bucket without branches (x >= 0, S <= 20): for x >= 2^S the
+// bucket (e - S + 1) 2^S + (top S bits below x's leading one) is read off the
+// float x converted toward zero, whose exponent field is e + 127 and whose
+// mantissa's top S bits are exactly those bits: (bits >> (23 - S)) - (126 + S) 2^S.
 DEVI uint32_t log_bucket_nb(int x, int S, int N) {
-  const int e = 31 - __clz(x | 1);
-  const int sh = max(e - S, 0);
-  const int big = ((e - S + 1) << S) + ((x >> sh) - (1 << S));
+  const int big = (int)(__float_as_uint(__int2float_rz(x)) >> (23 - S)) - ((126 + S) << S);
   const int b = x < (1 << S) ? x : big;
   return (uint32_t)min(b, N - 1);
 }
