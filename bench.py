@@ -1013,7 +1013,8 @@ def run_leg(args):
     """One workload alone, W untimed and K timed calls, for profilers: prints
     one small JSON line (not the bench line).  Legs: full_stack (the 8-layer
     stack), long_history / single_layer (one layer), mfalcon (ranking),
-    backward (the 8-layer stack's backward pass)."""
+    backward (the 8-layer stack's backward pass), comparator (the
+    softmax-Transformer layer on the long-history workload)."""
     import torch
     import hstu_workloads as hw
     import hstu_sequential_transducer_layer_b200 as H
@@ -1023,7 +1024,7 @@ def run_leg(args):
     torch.cuda.set_device(dev)
     make = {"full_stack": hw.full_stack, "long_history": hw.long_history,
             "single_layer": hw.single_layer, "mfalcon": hw.mfalcon,
-            "backward": hw.full_stack}[args.leg]
+            "backward": hw.full_stack, "comparator": hw.long_history}[args.leg]
     H.hstu_set_option("ln_fusion", args.ln_fusion)
     w = make(seed=args.seed)
     r = H.HSTURunner(hw.dims_dict(w.dims), w.weights, dev)
@@ -1037,6 +1038,11 @@ def run_leg(args):
     elif args.leg == "backward":
         dY = torch.randn(X.shape, device=dev).to(torch.bfloat16)
         fn = lambda: r.stack_bwd(off, X, ts, dY, w.max_len)
+    elif args.leg == "comparator":
+        rt = H.TransformerRunner(512, 8, 2048, hw.transformer_weights(args.seed, 512, 2048),
+                                 device=dev)
+        fn = lambda: rt.layer(off, X, w.max_len, out=out)
+        r = rt
     else:
         fn = lambda: r.stack(off, X, ts, w.max_len, out=out)
     for _ in range(args.warmup):
@@ -1090,7 +1096,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=4000)
     ap.add_argument("--ref-tokens", type=int, default=600)
     ap.add_argument("--leg", default=None,
-                    choices=["full_stack", "long_history", "single_layer", "mfalcon", "backward"],
+                    choices=["full_stack", "long_history", "single_layer", "mfalcon", "backward",
+                             "comparator"],
                     help="run one workload alone (for profilers) instead of the bench line")
     args = ap.parse_args()
     if args.leg:
