@@ -452,10 +452,15 @@ def run_ours(args):
     torch.cuda.synchronize()
     untraced_ms = sum(a.elapsed_time(b) for a, b in u_evs) / len(u_evs)
 
-    # ---------------- timed region (an event pair around every launch of the
-    # library gives the per-kernel device times for the roofline)
+    # ---------------- timed region: an event pair around every launch of the
+    # dominant kernel (the f1 GEMM: 47 % of the step's device time in the ncu
+    # launch list) gives its per-launch device time for the roofline; the
+    # other kernels run without event pairs (their split comes from a
+    # separate traced pass below)
+    f1_id = next(i for i in range(64) if H.hstu_kernel_name(i) == "gemm_f1_tc")
     n_launch0 = H.hstu_launch_count()
-    H.hstu_trace_enable(args.steps * 8 * 6 + 64)
+    H.hstu_trace_only(f1_id)
+    H.hstu_trace_enable(args.steps * 8 + 64)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     if world > 1:
@@ -471,14 +476,23 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     n_launch = H.hstu_launch_count() - n_launch0
-    trace = H.hstu_trace_read()
+    f1_trace = H.hstu_trace_read()
     H.hstu_trace_enable(0)
+    H.hstu_trace_only(-1)
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = sum(step_ms) / len(step_ms)
     if r.status() != 0:
         raise RuntimeError(f"device status {r.status()} after timing")
 
-    # per-kernel device time inside the timed region
+    # per-kernel device time of every kernel, from a separate traced pass of
+    # the same steps (outside the timed region)
+    H.hstu_trace_enable(args.steps * 8 * 6 + 64)
+    for _ in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    trace = H.hstu_trace_read()
+    H.hstu_trace_enable(0)
     per_kernel = {}
     for kid, t in trace:
         nm = H.hstu_kernel_name(kid)
@@ -488,8 +502,9 @@ def run_ours(args):
     dominant = max(per_kernel.items(), key=lambda kv: kv[1][1])[0] if per_kernel else None
     kflops = {"gemm_f1_tc": flops["f1"], "gemm_f2_tc": flops["f2"], "attn_tc": flops["attn"]}
     roofline = None
-    if dominant in kflops:
-        n, tot = per_kernel[dominant]
+    if dominant == "gemm_f1_tc" and f1_trace:
+        # the dominant kernel's launches inside the timed region
+        n, tot = len(f1_trace), sum(t for _, t in f1_trace)
         avg_s = tot / n / 1e3
         achieved = kflops[dominant] / avg_s / 1e12
         # the timed region is a burst of well under a second at full clocks,
@@ -949,6 +964,8 @@ def run_ours(args):
             "tflops": round(step_flops / (ms / 1e3) / 1e12, 1),
             "tensor_frac": tensor_frac(step_flops / (ms / 1e3) / 1e12, peaks),
             "roofline": roofline,
+            # per-kernel split of the step's device time (a traced pass of the
+            # same steps after the timed region)
             "kernels": {k: {"launches": v[0], "ms": round(v[1], 3),
                             "share": round(v[1] / max(1e-9, sum(x[1] for x in per_kernel.values())), 4)}
                         for k, v in sorted(per_kernel.items(), key=lambda kv: -kv[1][1])},

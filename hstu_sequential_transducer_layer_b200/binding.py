@@ -32,7 +32,7 @@ EXPORTED = ["hstu_workspace_size", "hstu_layer_fwd", "hstu_stack_fwd", "hstu_mfa
             "hstu_transformer_layer_fwd",
             "hstu_read_status", "hstu_debug_offsets", "hstu_debug_keep_z",
             "hstu_debug_wait_test",
-            "hstu_trace_enable", "hstu_trace_read",
+            "hstu_trace_enable", "hstu_trace_only", "hstu_trace_read",
             "hstu_kernel_name", "hstu_launch_count", "hstu_last_error", "hstu_set_option",
             "hstu_status_string",
             "hstu_version"]
@@ -137,6 +137,8 @@ def lib() -> ctypes.CDLL:
     L.hstu_debug_wait_test.restype = i32
     L.hstu_trace_enable.argtypes = [i32]
     L.hstu_trace_enable.restype = i32
+    L.hstu_trace_only.argtypes = [i32]
+    L.hstu_trace_only.restype = i32
     L.hstu_trace_read.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_float), i32]
     L.hstu_trace_read.restype = i32
     L.hstu_kernel_name.argtypes = [i32]
@@ -418,6 +420,10 @@ def hstu_debug_wait_test(wait_limit_us: int, inject_stall: int) -> None:
 
 def hstu_trace_enable(max_records: int) -> None:
     _check(lib().hstu_trace_enable(max_records), "hstu_trace_enable")
+
+
+def hstu_trace_only(kernel_id: int) -> None:
+    _check(lib().hstu_trace_only(kernel_id), "hstu_trace_only")
 
 
 def hstu_trace_read(capacity: int = 1 << 16):

@@ -18,6 +18,7 @@ std::atomic<int64_t> g_launches{0};
 std::mutex g_trace_mu;
 int g_trace_cap = 0;
 int g_trace_used = 0;
+int g_trace_only = -1;  // trace only this kernel id (-1: every kernel)
 std::vector<cudaEvent_t> g_ev0, g_ev1;
 std::vector<int> g_ids;
 }  // namespace
@@ -38,7 +39,7 @@ const char* kernel_name(int id) {
 LaunchScope::LaunchScope(int kernel_id, cudaStream_t stream) : id(kernel_id), s(stream), slot(-1) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   std::lock_guard<std::mutex> lk(g_trace_mu);
-  if (g_trace_used < g_trace_cap) {
+  if (g_trace_used < g_trace_cap && (g_trace_only < 0 || g_trace_only == kernel_id)) {
     slot = g_trace_used++;
     g_ids[slot] = kernel_id;
     cudaEventRecord(g_ev0[slot], s);
@@ -292,6 +293,14 @@ hstu_status hstu_trace_enable(int32_t max_records) {
       return HSTU_ERR_CUDA;
   }
   g_trace_cap = max_records;
+  return HSTU_OK;
+}
+
+hstu_status hstu_trace_only(int32_t kernel_id) {
+  using namespace hstu;
+  if (kernel_id < -1 || kernel_id >= K_NUM_KERNELS) return HSTU_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  g_trace_only = kernel_id;
   return HSTU_OK;
 }
 

@@ -393,20 +393,24 @@ hstu_status hstu_debug_offsets(const hstu_layer_desc* desc, int64_t B, int64_t t
                                size_t* z_offset);
 
 /* Tracing.  hstu_trace_enable(n) records a CUDA event pair around each of
- * the next n kernel launches (n = 0 turns tracing off); hstu_trace_read
+ * the next n kernel launches (n = 0 turns tracing off); hstu_trace_only(id)
+ * restricts the recording to launches of one kernel id (-1, the default:
+ * every kernel; HSTU_ERR_INVALID_ARG for an unknown id); hstu_trace_read
  * synchronises and returns, per traced launch, the kernel id and the device
  * time in ms.  hstu_kernel_name maps an id to a name.  hstu_launch_count
  * counts every kernel this library has launched in this process. */
 hstu_status hstu_trace_enable(int32_t max_records);
+hstu_status hstu_trace_only(int32_t kernel_id);
 int32_t hstu_trace_read(int32_t* kernel_ids, float* ms, int32_t capacity);
 const char* hstu_kernel_name(int32_t kernel_id);
 int64_t hstu_launch_count(void);
 
 /* Test hook: with on = 1, later layer calls on the tensor-core path also
  * write the gated Z = LayerNorm(O) * U into the workspace (at the z offset
- * of hstu_debug_offsets); with on = 0 (the default) Z never leaves the output
- * projection's shared memory.  Process-wide.  Returns HSTU_ERR_INVALID_ARG
- * for other values. */
+ * of hstu_debug_offsets) when the output projection forms it in its shared
+ * memory (see the "ln_fusion" option); with on = 0 (the default) Z is in the
+ * workspace only when the separate LayerNorm * U kernel formed it.
+ * Process-wide.  Returns HSTU_ERR_INVALID_ARG for other values. */
 hstu_status hstu_debug_keep_z(int32_t on);
 
 /* Test hook for the failure detection of the in-kernel waits.  Every wait

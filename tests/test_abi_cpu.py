@@ -200,6 +200,10 @@ def test_option_and_test_hook_arguments_checked():
     assert L.hstu_debug_keep_z(3) == 1
     assert L.hstu_debug_wait_test(1000, 5) == 1
     assert L.hstu_debug_wait_test(0, 0) == 0
+    assert L.hstu_trace_only(-2) == 1
+    assert L.hstu_trace_only(100000) == 1
+    assert L.hstu_trace_only(2) == 0
+    assert L.hstu_trace_only(-1) == 0
     assert L.hstu_last_error() is not None
 
 
