@@ -317,9 +317,9 @@ hstu_status stack_impl(const hstu_layer_desc* desc, int32_t n_layers,
   launch_schedule(offsets, B, T, max_len, desc->n_heads, at<AttnItem>(ws, L.items), L.item_cap,
                   at<int64_t>(ws, L.ubase), L.tile_cap, c.hdr, c.s);
   if (T == 0) return finish(cudaSuccess);
-  launch_time_rel(offsets, B, timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
+  launch_time_rel(offsets, B, max_len, timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
   if (c.bf16)  // time buckets: computed once, shared by every head and layer
-    launch_time_buckets(offsets, B, at<int32_t>(ws, L.t_rel), at<int64_t>(ws, L.ubase),
+    launch_time_buckets(offsets, B, max_len, at<int32_t>(ws, L.t_rel), at<int64_t>(ws, L.ubase),
                         L.tile_cap, desc->time_sub_bits, desc->n_time_buckets,
                         at<uint32_t>(ws, L.tbuckets), c.hdr, c.s);
   // Between layers the residual stream is fp16 on the tensor-core path (xh: the
@@ -417,9 +417,11 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
   float* xres = at<float>(ws, L.xres);
   void* xh = at<void>(ws, L.xh);
   if (T > 0 && e == cudaSuccess) {
-    launch_time_rel(hist_offsets, B, hist_timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr, c.s);
+    launch_time_rel(hist_offsets, B, max_len, hist_timestamps, T, at<int32_t>(ws, L.t_rel), c.hdr,
+                    c.s);
     if (c.bf16 && n_layers > 1)
-      launch_time_buckets(hist_offsets, B, at<int32_t>(ws, L.t_rel), at<int64_t>(ws, L.ubase),
+      launch_time_buckets(hist_offsets, B, max_len, at<int32_t>(ws, L.t_rel),
+                          at<int64_t>(ws, L.ubase),
                           L.tile_cap, desc->time_sub_bits, desc->n_time_buckets,
                           at<uint32_t>(ws, L.tbuckets), c.hdr, c.s);
     for (int l = 0; l < n_layers && e == cudaSuccess; ++l) {

@@ -486,8 +486,8 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     if (!ok()) note_cuda_error(e, "zero gradients");
     return ok() ? HSTU_OK : HSTU_ERR_CUDA;
   }
-  launch_time_rel(offsets, B, timestamps, T, at<int32_t>(ws, Lo.t_rel), hdr, s);
-  launch_time_buckets(offsets, B, at<int32_t>(ws, Lo.t_rel), at<int64_t>(ws, Lo.ubase),
+  launch_time_rel(offsets, B, max_len, timestamps, T, at<int32_t>(ws, Lo.t_rel), hdr, s);
+  launch_time_buckets(offsets, B, max_len, at<int32_t>(ws, Lo.t_rel), at<int64_t>(ws, Lo.ubase),
                       Lo.tile_cap, d.time_sub_bits, d.n_time_buckets, at<uint32_t>(ws, Lo.tbuckets),
                       hdr, s);
   // fp16 copies of every layer's W1 and W2

@@ -145,12 +145,12 @@ void launch_schedule(const int64_t* offsets, int64_t B, int64_t T, int64_t max_l
                      AttnItem* items, int64_t item_cap, int64_t* ubase, int64_t tile_cap,
                      Header* hdr, cudaStream_t s);
 // Time-bucket tiles of every causal (q-tile, kv-tile) pair of the batch.
-void launch_time_buckets(const int64_t* offsets, int64_t B, const int32_t* t_rel,
+void launch_time_buckets(const int64_t* offsets, int64_t B, int64_t max_len, const int32_t* t_rel,
                          const int64_t* ubase, int64_t tile_cap, int St, int Nt,
                          uint32_t* tbuckets, Header* hdr, cudaStream_t s);
 // Per-row timestamp relative to the user's first one (int32), with checks.
-void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64_t T,
-                     int32_t* t_rel, Header* hdr, cudaStream_t s);
+void launch_time_rel(const int64_t* offsets, int64_t B, int64_t max_len, const int64_t* ts,
+                     int64_t T, int32_t* t_rel, Header* hdr, cudaStream_t s);
 
 // C[M, N] = A[M, K] * W[n_off + N, K]^T with fused epilogue, bf16 tcgen05.
 enum Epilogue { EPI_SILU = 0, EPI_RESID = 1, EPI_SCORE = 2, EPI_BIAS = 3, EPI_FILTER = 4 };

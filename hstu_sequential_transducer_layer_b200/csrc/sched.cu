@@ -110,17 +110,25 @@ __global__ void __launch_bounds__(kSchedThreads)
     }
     __syncthreads();
     total = s_carry;
-    for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+    // one warp per user (its lanes write the user's c * h items: head-major,
+    // q-tiles longest first), so a few long users do not serialise the writes
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+    for (int64_t b = warp; b < B; b += n_warps) {
       const int c = nq_of(b);
       if (c == 0) continue;
-      long long pos = atomicAdd(&s_cursor[c], c * h);
-      for (int hh = 0; hh < h; ++hh)
-        for (int qt = c - 1; qt >= 0; --qt, ++pos)
-          if (pos < item_cap)
-            items[pos] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, qt + 1,
-                                  (int32_t)(ubase[b] + (long long)qt * (qt + 1) / 2),
-                                  (int32_t)(off[b] + (int64_t)qt * kTile), (int32_t)off[b],
-                                  (int32_t)(off[b + 1] - off[b]), (int32_t)(off[b + 1] - off[b])};
+      long long pos = 0;
+      if (lane == 0) pos = atomicAdd(&s_cursor[c], c * h);
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      const int64_t o0 = off[b];
+      const int32_t n_b = (int32_t)(off[b + 1] - o0);
+      const long long ub = ubase[b];
+      for (int k = lane; k < c * h; k += 32) {
+        const int hh = k / c, qt = c - 1 - (k - hh * c);
+        if (pos + k < item_cap)
+          items[pos + k] = AttnItem{(int32_t)b, (int16_t)qt, (int16_t)hh, qt + 1,
+                                    (int32_t)(ub + (long long)qt * (qt + 1) / 2),
+                                    (int32_t)(o0 + (int64_t)qt * kTile), (int32_t)o0, n_b, n_b};
+      }
     }
   } else if (threadIdx.x == 0) {  // users over kMaxLevels * 128 tokens: one thread walks them
     long long pos = 0;
@@ -163,46 +171,71 @@ __device__ __forceinline__ int64_t find_user(const int64_t* off, int64_t B, int6
   return lo;
 }
 
+// Users along the grid's y dimension, each user's rows along x: no search for
+// the user of a row.
 __global__ void k_time_rel(const int64_t* __restrict__ off, int64_t B,
-                           const int64_t* __restrict__ ts, int64_t T, int32_t* __restrict__ t_rel,
+                           const int64_t* __restrict__ ts, int32_t* __restrict__ t_rel,
                            Header* hdr) {
   if (hdr->status != HSTU_OK) return;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < T;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t b = find_user(off, B, i);
-    const int64_t d = ts[i] - ts[off[b]];
-    if (d >= (1ll << 30) || d <= -(1ll << 30)) {
-      set_status(&hdr->status, HSTU_ERR_BAD_TIMESTAMPS);
-      t_rel[i] = 0;
-    } else {
-      t_rel[i] = (int32_t)d;
+  for (int64_t b = blockIdx.y; b < B; b += gridDim.y) {
+    const int64_t s0 = off[b], s1 = off[b + 1];
+    if (s1 <= s0) continue;
+    const int64_t t0 = ts[s0];
+    for (int64_t i = s0 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < s1;
+         i += (int64_t)gridDim.x * blockDim.x) {
+      const int64_t d = ts[i] - t0;
+      if (d >= (1ll << 30) || d <= -(1ll << 30)) {
+        set_status(&hdr->status, HSTU_ERR_BAD_TIMESTAMPS);
+        t_rel[i] = 0;
+      } else {
+        t_rel[i] = (int32_t)d;
+      }
     }
   }
 }
 
-void launch_time_rel(const int64_t* offsets, int64_t B, const int64_t* ts, int64_t T,
-                     int32_t* t_rel, Header* hdr, cudaStream_t s) {
-  if (T <= 0) return;
+void launch_time_rel(const int64_t* offsets, int64_t B, int64_t max_len, const int64_t* ts,
+                     int64_t T, int32_t* t_rel, Header* hdr, cudaStream_t s) {
+  if (T <= 0 || B <= 0) return;
   LaunchScope ls(K_TIME_REL, s);
-  const int grid = (int)std::min<int64_t>((T + 255) / 256, 4 * num_sms());
-  k_time_rel<<<grid, 256, 0, s>>>(offsets, B, ts, T, t_rel, hdr);
+  const dim3 grid((unsigned)std::max<int64_t>(1, std::min<int64_t>((max_len + 255) / 256, 32)),
+                  (unsigned)std::min<int64_t>(B, 65535));
+  k_time_rel<<<grid, 256, 0, s>>>(offsets, B, ts, t_rel, hdr);
 }
 
 // ---------------------------------------------------------------- time buckets
-// One block per tile (grid-stride): tile t of user b is local index
-// qt (qt + 1) / 2 + j (j <= qt).  Word (c4, r) packs the buckets of row
-// qt*128 + r against columns j*128 + 4*c4 .. +3; entries outside the causal
-// triangle or the sequence are 0 (they are masked or unused).
+// One block per tile (grid-stride over every tile of the batch, so the work is
+// even across blocks): tile t of user b is local index qt (qt + 1) / 2 + j
+// (j <= qt), b found by binary search over the users' first tiles, which each
+// block first copies into shared memory (up to kBucketUsersSmem users; beyond,
+// the search reads them from global memory).  Word (c4, r) packs the buckets
+// of row qt*128 + r against columns j*128 + 4*c4 .. +3; entries outside the
+// causal triangle or the sequence are 0 (they are masked or unused).
+constexpr int kBucketUsersSmem = 4096;
+
 __global__ void __launch_bounds__(256)
     k_time_buckets(const int64_t* __restrict__ off, int64_t B, const int32_t* __restrict__ t_rel,
                    const int64_t* __restrict__ ubase, int St, int Nt,
                    uint32_t* __restrict__ tb, const Header* hdr) {
   __shared__ __align__(16) int s_tj[kTile];
+  __shared__ int s_ub[kBucketUsersSmem + 1];  // first tile of each user (fits int: tiles < 2^31)
   if (hdr->status != HSTU_OK) return;
   const int n_tiles = hdr->n_tiles;
+  const bool ub_smem = B < kBucketUsersSmem;
+  if (ub_smem)
+    for (int64_t i = threadIdx.x; i <= B; i += blockDim.x) s_ub[i] = (int)ubase[i];
+  __syncthreads();
   for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-    const int64_t b = find_user(ubase, B, t);  // ubase[b] <= t < ubase[b+1]
-    const int64_t local = t - ubase[b];
+    // the user of tile t: ubase[b] <= t < ubase[b + 1]
+    int64_t lo = 0, hi = B;
+    while (hi - lo > 1) {
+      const int64_t mid = (lo + hi) >> 1;
+      const int64_t u = ub_smem ? (int64_t)s_ub[mid] : ubase[mid];
+      if (u <= t) lo = mid;
+      else hi = mid;
+    }
+    const int64_t b = lo;
+    const int64_t local = t - (ub_smem ? (int64_t)s_ub[b] : ubase[b]);
     int qt = (int)((sqrt(8.0 * (double)local + 1.0) - 1.0) * 0.5);
     while ((int64_t)qt * (qt + 1) / 2 > local) --qt;
     while ((int64_t)(qt + 1) * (qt + 2) / 2 <= local) ++qt;
@@ -238,10 +271,11 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-void launch_time_buckets(const int64_t* offsets, int64_t B, const int32_t* t_rel,
+void launch_time_buckets(const int64_t* offsets, int64_t B, int64_t max_len, const int32_t* t_rel,
                          const int64_t* ubase, int64_t tile_cap, int St, int Nt,
                          uint32_t* tbuckets, Header* hdr, cudaStream_t s) {
-  if (tile_cap <= 0) return;
+  (void)max_len;
+  if (tile_cap <= 0 || B <= 0) return;
   LaunchScope ls(K_TIME_BUCKETS, s);
   const int grid = (int)std::min<int64_t>(tile_cap, 8 * num_sms());
   k_time_buckets<<<grid, 256, 0, s>>>(offsets, B, t_rel, ubase, St, Nt, tbuckets, hdr);
