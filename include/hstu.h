@@ -190,7 +190,10 @@ hstu_status hstu_mfalcon_rank(const hstu_layer_desc* desc, int32_t n_layers,
  *     other argument errors are those of hstu_layer_fwd.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: after a cudaDeviceReset (which releases the module's device
+ *     memory) it is stale, so the function must not be called again in that
+ *     process.
  *   - Every call shares the one array and leaves its contents behind; each
  *     call resets what must start at zero (the status word and counters).
  *     Calls whose execution overlaps on the GPU (other streams, other host
