@@ -640,7 +640,7 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
     void* pre_buf = pre_of(l);
     void* o_buf = o_of(l);
     float* ostats = ostats_of(l);
-    if (l < L - 1) e = convert(gy, 0, nullptr, gyh, (int64_t)T * dm, status, s);
+    // (gyh, the fp16 copy of gy, was written by the layer above's dX product)
     // dZ = dY W2
     GradGemm gg{};
     gg.A = gyh;
@@ -804,7 +804,10 @@ hstu_status stack_bwd_impl(const hstu_layer_desc* desc, int32_t L, const hstu_la
       gx_.out = gx;
       gx_.ldo = dm;
       gx_.resid = gy;
-      gx_.out16 = l == 0 ? dX : nullptr;
+      // the caller's bf16 dX at layer 0; above it, the fp16 copy of this
+      // gradient stream that the next layer's products read
+      gx_.out16 = l == 0 ? dX : static_cast<void*>(gyh);
+      gx_.out16_f16 = l == 0 ? 0 : 1;
       gx_.zero_bias = at<void>(ws, Lo.zbias);
       gx_.status = status;
       e = launch_gemm_grad(gx_, s, K_GEMM_BWD);

@@ -910,7 +910,9 @@ cudaError_t launch_gemm_grad(const GradGemm& c, cudaStream_t s, int kernel_id) {
       return cudaErrorInvalidValue;
     if (c.out16 && !encode_tmap_2d_ex(&to16, c.out16, (uint64_t)c.M, (uint64_t)c.N,
                                       (uint64_t)c.ldo * 2, 32, 32,
-                                      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B))
+                                      c.out16_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                      CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
   const int KB = (int)((c.K + 63) / 64);
@@ -929,10 +931,10 @@ cudaError_t launch_gemm_grad(const GradGemm& c, cudaStream_t s, int kernel_id) {
   const int64_t tiles = ((c.M + 127) / 128) * ((c.N + BN - 1) / BN) * gd.splits;
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
   LaunchScope ls(kernel_id, s);
-  if (c.resid) {  // out = resid + A W^T (+ a zero bias), fp32 and optionally bf16
+  if (c.resid) {  // out = resid + A W^T (+ a zero bias), fp32 and optionally 16-bit
     gd.bias = static_cast<const __nv_bfloat16*>(c.zero_bias);
     gd.has_out16 = c.out16 != nullptr;
-    gd.out_f16 = 0;
+    gd.out_f16 = c.out16_f16 ? 1 : 0;
     gd.has_out32 = 1;
     gd.resid = c.resid;
     gd.ldr = c.ldo;

@@ -207,7 +207,8 @@ struct GradGemm {
   int splits; int64_t split_rows;
   float* out; int64_t ldo;
   const float* resid;
-  void* out16;
+  void* out16;             // with resid: a 16-bit copy of out, bf16 (or fp16 with out16_f16)
+  int out16_f16;
   const void* zero_bias;   // bf16 zeros, at least N (the residual epilogue adds a bias)
   int* status;
   int* splits_used;        // optional: receives the number of splits launched (<= splits)
