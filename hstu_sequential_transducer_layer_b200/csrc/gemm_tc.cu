@@ -22,6 +22,9 @@
 // tensor stores (whole lines, asynchronous).  Every wait is bounded.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <atomic>
+
 #include "ptx.cuh"
 
 namespace hstu {
@@ -666,6 +669,309 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ CTA pairs
+// The same product on clusters of two CTAs (one per SM) that share each
+// 256 x 256 output tile through the pair MMA (cta_group::2): CTA r brings rows
+// r*128.. of the A tile and W rows r*128.. of the tile's 256 into its own
+// shared memory, so each CTA streams 32 KB per K block instead of the 48 KB a
+// 128 x 256 tile of one CTA needs; rank 0 issues the MMAs (M = 256, N = 256),
+// which leave each CTA's 128 output rows x 256 columns in its own tensor
+// memory; both CTAs run the same epilogue warps on their half.
+//   rank 0: counts both CTAs' bytes on its `full` barriers (the peer's loads
+//           name them by cluster address); its MMA commits arrive on the
+//           `empty` and `tfull` barriers of both CTAs (multicast commit);
+//           both CTAs' epilogue warps arrive on rank 0's `tempty`.
+// Only the plain-bias and SiLU epilogues (16-bit output, optionally the SiLU
+// pre-activation), K-major operands.  Every wait is bounded; the two CTAs
+// leave together through a bounded exchange of arrivals.
+constexpr int kPairStages = 6;
+struct PairCfg {
+  static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // this CTA's 128 rows of A
+  static constexpr uint32_t B_BYTES = 128 * 64 * 2;  // this CTA's 128 rows of W
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t OUT_OFF = kPairStages * STAGE_BYTES;
+  static constexpr uint32_t BAR_OFF = OUT_OFF + (kEpiThreads / 32) * kStageBuf;
+  static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
+  static constexpr int THREADS = 64 + kEpiThreads;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmO16,
+                const __grid_constant__ CUtensorMap tmO32, const GemmDev g) {
+  using C = PairCfg;
+  constexpr int S = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);  // [S], rank 0's in use
+  uint64_t* empty = full + S;                                       // [S]
+  uint64_t* tfull = empty + S;                                      // [2]
+  uint64_t* tempty = tfull + 2;                                     // [2], rank 0's in use
+  uint64_t* drain = tempty + 2;
+  uint64_t* pdone = drain + 1;  // one arrival from each CTA at the end
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pdone + 1);
+  AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
+  uint32_t* s_go = reinterpret_cast<uint32_t*>(ab + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  if (threadIdx.x == 0) {
+    ab->flag = 0;
+    ab->limit_us = kWaitLimitUs;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(tfull + 0, 1);
+    mbar_init(tfull + 1, 1);
+    mbar_init(tempty + 0, 2 * (kEpiThreads / 32));
+    mbar_init(tempty + 1, 2 * (kEpiThreads / 32));
+    mbar_init(drain, 1);
+    mbar_init(pdone, 2);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised
+  // rank 0 decides for the pair, so that both CTAs take the same path
+  if (rank == 0 && threadIdx.x == 0) {
+    const uint32_t go =
+        ((g.status == nullptr) || (*reinterpret_cast<volatile int*>(g.status) == 0)) &&
+        (g.run_if == nullptr || *reinterpret_cast<volatile const int*>(g.run_if) != 0);
+    *s_go = go;
+    st_cluster_u32(mapa_shared(smem_u32(s_go), 1), go);
+  }
+  cluster_sync_all();
+  if (!*s_go) return;
+
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int64_t Mrows = g.M_cap;
+  if (g.M_dev) {
+    const int64_t m = *g.M_dev;
+    Mrows = m < Mrows ? m : Mrows;
+  }
+  if (Mrows < 0) Mrows = 0;
+  const int n_tiles = g.N / 256;
+  const int m_tiles = (int)((Mrows + 255) / 256);
+  const int tiles = m_tiles * n_tiles;
+  const int KB = g.K / 64;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = pair; t < tiles && ok; t += npairs) {
+        const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty + stage, ph ^ 1, ab, g.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(full + stage, 2 * C::STAGE_BYTES);
+          const uint32_t fb = mapa_shared(smem_u32(full + stage), 0);  // rank 0's barrier
+          tma_load_2d_pair(sa, &tmA, kb * 64, mt * 256 + (int)rank * 128, fb);
+          tma_load_2d_pair(sa + C::A_BYTES, &tmB, kb * 64, g.n_off + nt * 256 + (int)rank * 128,
+                           fb);
+          if (++stage == S) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t IDESC = idesc_f16_f32(256, 256, 0, 0, g.ab_f16);
+      int stage = 0, local = 0;
+      uint32_t ph = 0;
+      bool ok = true, issued_any = false;
+      for (int t = pair; t < tiles && ok; t += npairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait_cluster(tempty + acc, aph ^ 1, ab, g.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * 256;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full + stage, ph, ab, g.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16_ss_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
+                               sdesc_sw128(b0 + k * 32, 16, 1024), IDESC,
+                               (kb != 0 || k != 0) ? 1u : 0u);
+          tc_commit_pair(empty + stage, 0x3);
+          issued_any = true;
+          if (++stage == S) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (ok) tc_commit_pair(tfull + acc, 0x3);
+      }
+      if (issued_any) {
+        tc_commit_pair(drain, 0x1);  // every MMA issued above has finished
+        AbortState tmp{0, kWaitLimitUs};
+        mbar_wait(drain, 0, &tmp, nullptr);
+      }
+    }
+  } else {
+    const int q = warp & 3;            // TMEM lane quarter this warp may read
+    const int part = (warp - 2) >> 2;  // which 128 of the 256 columns
+    constexpr int CH = 4;              // 32-column chunks per warp
+    uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * kStageBuf;
+    int local = 0, nchunk = 0;
+    for (int t = pair; t < tiles; t += npairs) {
+      const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      ++local;
+      const int col0 = g.n_off + nt * 256 + part * 128;
+      const uint4* bptr = reinterpret_cast<const uint4*>(g.bias + col0);
+      uint4 ba[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ba[i] = __ldg(bptr + i);
+      if (!mbar_wait_warp(tfull + acc, aph, ab, g.status)) break;
+      tc_fence_after();
+      const int y0 = mt * 256 + (int)rank * 128 + q * 32;  // output row of lane 0
+      const int64_t row = (int64_t)y0 + lane;
+      const bool valid = row < Mrows;
+      const uint32_t tbase = tmem + acc * 256 + part * 128 + ((uint32_t)(q * 32) << 16);
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tbase, ra);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        // the next chunk's accumulator and bias load while this one is stored
+        if (c + 1 < CH) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 bv = __ldg(bptr + (c + 1) * 4 + i);
+            if (c & 1) ba[i] = bv;
+            else bb[i] = bv;
+          }
+          if (c & 1) tmem_ld32(tbase + (c + 1) * 32, ra);
+          else tmem_ld32(tbase + (c + 1) * 32, rb);
+        }
+        bool stored;
+        if (c & 1)
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb, bb, stage,
+                                   nchunk & 1, nullptr);
+        else
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba, stage,
+                                   nchunk & 1, nullptr);
+        nchunk += stored ? 1 : 0;
+        if (c + 1 < CH) tmem_ld_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(tempty + acc), 0));
+    }
+    if (lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
+    __syncwarp();
+  }
+  // leave together: neither CTA exits while the other may still arrive on its
+  // barriers or (rank 0's MMAs) read its shared memory
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive(pdone);
+    mbar_arrive_cluster(mapa_shared(smem_u32(pdone), rank ^ 1u));
+    AbortState tmp{0, 4 * kWaitLimitUs};
+    mbar_wait(pdone, 0, &tmp, nullptr);
+    // after a failed wait, loads already issued by either CTA may still be in
+    // flight towards this CTA's shared memory: give them time to land
+    if (g.status && *reinterpret_cast<volatile int*>(g.status) != 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 100000ull) __nanosleep(1000);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+template <int EPI>
+static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb,
+                               const CUtensorMap& to16, const CUtensorMap& to32,
+                               const GemmDev& gd, int pairs, cudaStream_t s) {
+  static_assert(PairCfg::SMEM <= 232448, "shared memory per CTA");
+  auto kfn = k_gemm_pair<EPI>;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), PairCfg::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kfn, ta, tb, to16, to32, gd);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// How many CTA pairs of the pair kernel fit on the device at once (0 if the
+// query fails): the persistent grid takes no more, so that no pair waits for
+// another to finish.
+template <int EPI>
+static int pair_capacity() {
+  static std::atomic<int> cached{-1};
+  int v = cached.load(std::memory_order_relaxed);
+  if (v >= 0) return v;
+  auto kfn = k_gemm_pair<EPI>;
+  int n = 0;
+  if (ensure_smem_limit(reinterpret_cast<const void*>(kfn), PairCfg::SMEM) == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = PairCfg::SMEM;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kfn), &cfg) !=
+        cudaSuccess)
+      n = 0;
+  }
+  (void)cudaGetLastError();
+  cached.store(n, std::memory_order_relaxed);
+  return n;
+}
+
 cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
   if (c.M_cap <= 0 || c.N <= 0) return cudaSuccess;
   if (c.N % 64 != 0 || c.K % 64 != 0) return cudaErrorInvalidValue;
@@ -762,6 +1068,21 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
     const cudaError_t e = launch_ln_coef(c.ln_stats, c.ln_h, c.ln_eps, c.ln_coef, c.M_cap, c.M_dev,
                                          c.status, s);
     if (e != cudaSuccess) return e;
+  }
+  // SiLU and plain-bias products with 256-column tiles: CTA pairs
+  if (!lna && (c.epi == EPI_SILU || c.epi == EPI_BIAS) && BN == 256 && gemm_pair_on()) {
+    const int cap = c.epi == EPI_SILU ? pair_capacity<EPI_SILU>() : pair_capacity<EPI_BIAS>();
+    if (cap > 0) {
+      CUtensorMap tb2;  // W in 128-row boxes: each CTA of a pair brings half a tile
+      if (!encode_tmap_2d(&tb2, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K,
+                          (uint64_t)c.ldw * 2, 64, 128, f16))
+        return cudaErrorInvalidValue;
+      const int64_t ptiles = ((c.M_cap + 255) / 256) * (c.N / 256);
+      const int pairs = (int)std::min<int64_t>(ptiles, cap);
+      LaunchScope ls(kernel_id, s);
+      if (c.epi == EPI_SILU) return launch_pair<EPI_SILU>(ta, tb2, to16, to32, gd, pairs, s);
+      return launch_pair<EPI_BIAS>(ta, tb2, to16, to32, gd, pairs, s);
+    }
   }
   LaunchScope ls(kernel_id, s);
   if (c.epi == EPI_SILU) {

@@ -91,7 +91,10 @@ bool keep_z() { return g_keep_z.load(std::memory_order_relaxed) != 0; }
 
 namespace {
 std::atomic<int> g_ln_fusion{2};
+std::atomic<int> g_gemm_pair{1};
 }  // namespace
+
+bool gemm_pair_on() { return g_gemm_pair.load(std::memory_order_relaxed) != 0; }
 
 // 2 (automatic): inside f2 when f2 has at most two 256-column output tiles
 // (d_model <= 512); with more, each A block would be formed once per tile and
@@ -254,6 +257,11 @@ hstu_status hstu_set_option(const char* name, int64_t value) {
   if (std::strcmp(name, "ln_fusion") == 0) {
     if (value < 0 || value > 2) return HSTU_ERR_INVALID_ARG;
     hstu::g_ln_fusion.store((int)value);
+    return HSTU_OK;
+  }
+  if (std::strcmp(name, "gemm_pair") == 0) {
+    if (value != 0 && value != 1) return HSTU_ERR_INVALID_ARG;
+    hstu::g_gemm_pair.store((int)value);
     return HSTU_OK;
   }
   return HSTU_ERR_INVALID_ARG;

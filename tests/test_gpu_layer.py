@@ -339,3 +339,31 @@ def test_ln_fusion_on_and_off_match_oracle(D):
     finally:
         B.hstu_set_option("ln_fusion", 2)
     assert relerr(out[1], out[0]) <= 2 * TOL[hw.BF16]
+
+
+def test_gemm_pair_on_and_off_match_oracle():
+    """The SiLU projection f1 on CTA pairs (256-row pair MMA, gemm_pair = 1)
+    and on single CTAs (0): both within the bound of the oracle on a ragged
+    2-layer stack whose f1 takes 256-column tiles (f1 width 2048, 4,900 rows:
+    the last 256-row tile leaves the second CTA of its pair without a valid
+    row), and identical to each other (the same fp32 accumulation order over
+    K for every output element)."""
+    from hstu_sequential_transducer_layer_b200 import binding as B
+    dims = hw.LayerDims(512, 4, 128, 128, 128, 128, 4, 2, 1e-6, hw.BF16)
+    lengths = [777, 1024, 513, 1, 900, 1685]
+    assert sum(lengths) == 4900 and dims.f1_width == 2048
+    w = hw.custom("pair", lengths, dims, n_layers=2, seed=417)
+    ref = O.stack_fwd(w.X, w.offsets, w.timestamps, w.weights, dims)
+    X = w.X.astype(np.float64)
+    out = {}
+    try:
+        for p in (0, 1):
+            B.hstu_set_option("gemm_pair", p)
+            Y, _, _ = run_stack(w)
+            out[p] = Y
+            e, ed = relerr(Y, ref), rmserr(Y - X, ref - X)
+            print("gemm_pair", p, e, ed)
+            assert e <= TOL[hw.BF16] and ed <= TOL[hw.BF16], (p, e, ed)
+    finally:
+        B.hstu_set_option("gemm_pair", 1)
+    assert np.array_equal(out[0], out[1])
