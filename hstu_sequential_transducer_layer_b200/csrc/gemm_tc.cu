@@ -1070,7 +1070,7 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
     if (e != cudaSuccess) return e;
   }
   // SiLU and plain-bias products with 256-column tiles: CTA pairs
-  if (!lna && (c.epi == EPI_SILU || c.epi == EPI_BIAS) && BN == 256 && gemm_pair_on()) {
+  if (!lna && (c.epi == EPI_SILU || c.epi == EPI_BIAS) && BN == 256 && gemm_pair_for(c.K)) {
     const int cap = c.epi == EPI_SILU ? pair_capacity<EPI_SILU>() : pair_capacity<EPI_BIAS>();
     if (cap > 0) {
       CUtensorMap tb2;  // W in 128-row boxes: each CTA of a pair brings half a tile

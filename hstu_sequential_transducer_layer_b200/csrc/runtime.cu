@@ -94,7 +94,14 @@ std::atomic<int> g_ln_fusion{2};
 std::atomic<int> g_gemm_pair{1};
 }  // namespace
 
-bool gemm_pair_on() { return g_gemm_pair.load(std::memory_order_relaxed) != 0; }
+// 1 (automatic): on pairs when K >= 1024.  With shorter K the SiLU epilogue
+// of a tile takes about as long as its MMAs, and the pair, whose MMAs wait
+// for both CTAs' epilogues, is slower than single CTAs (measured at K = 512:
+// f1 8 % slower; at K = 1024: 2-3 % faster).
+bool gemm_pair_for(int K) {
+  const int m = g_gemm_pair.load(std::memory_order_relaxed);
+  return m == 2 || (m == 1 && K >= 1024);
+}
 
 // 2 (automatic): inside f2 when f2 has at most two 256-column output tiles
 // (d_model <= 512); with more, each A block would be formed once per tile and
@@ -260,7 +267,7 @@ hstu_status hstu_set_option(const char* name, int64_t value) {
     return HSTU_OK;
   }
   if (std::strcmp(name, "gemm_pair") == 0) {
-    if (value != 0 && value != 1) return HSTU_ERR_INVALID_ARG;
+    if (value < 0 || value > 2) return HSTU_ERR_INVALID_ARG;
     hstu::g_gemm_pair.store((int)value);
     return HSTU_OK;
   }

@@ -436,8 +436,12 @@ hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall);
  * a separate kernel that f2 then reads, 2 (default) chooses per layer: inside
  * f2 when d_model <= 512 (f2 then has at most two 256-column output tiles,
  * each of which forms Z again), the separate kernel otherwise.  All give the
- * same layer within the bf16 bound.  Returns HSTU_ERR_INVALID_ARG for an
- * unknown name or value. */
+ * same layer within the bf16 bound.  "gemm_pair": where the input projection
+ * f1 (SiLU) takes 256-column output tiles, 1 (default) runs it on clusters of
+ * two CTAs sharing each 256 x 256 tile through the pair MMA when its inner
+ * dimension (d_model) is at least 1024, 2 does so at any inner dimension, 0
+ * never; all give bitwise the same result.  Returns HSTU_ERR_INVALID_ARG for
+ * an unknown name or value. */
 hstu_status hstu_set_option(const char* name, int64_t value);
 
 /* After an entry point returned HSTU_ERR_CUDA: the failing CUDA runtime

@@ -197,9 +197,10 @@ def test_option_and_test_hook_arguments_checked():
     assert L.hstu_set_option(b"ln_fusion", 1) == 0
     assert L.hstu_set_option(b"ln_fusion", 0) == 0
     assert L.hstu_set_option(b"ln_fusion", 2) == 0
-    assert L.hstu_set_option(b"gemm_pair", 2) == 1
+    assert L.hstu_set_option(b"gemm_pair", 3) == 1
     assert L.hstu_set_option(b"gemm_pair", -1) == 1
     assert L.hstu_set_option(b"gemm_pair", 0) == 0
+    assert L.hstu_set_option(b"gemm_pair", 2) == 0
     assert L.hstu_set_option(b"gemm_pair", 1) == 0
     assert L.hstu_debug_keep_z(3) == 1
     assert L.hstu_debug_wait_test(1000, 5) == 1

@@ -342,8 +342,9 @@ def test_ln_fusion_on_and_off_match_oracle(D):
 
 
 def test_gemm_pair_on_and_off_match_oracle():
-    """The SiLU projection f1 on CTA pairs (256-row pair MMA, gemm_pair = 1)
-    and on single CTAs (0): both within the bound of the oracle on a ragged
+    """The SiLU projection f1 on CTA pairs (256-row pair MMA, gemm_pair = 2,
+    which forces pairs at this K = 512) and on single CTAs (0): both within
+    the bound of the oracle on a ragged
     2-layer stack whose f1 takes 256-column tiles (f1 width 2048, 4,900 rows:
     the last 256-row tile leaves the second CTA of its pair without a valid
     row), and identical to each other (the same fp32 accumulation order over
@@ -353,6 +354,31 @@ def test_gemm_pair_on_and_off_match_oracle():
     lengths = [777, 1024, 513, 1, 900, 1685]
     assert sum(lengths) == 4900 and dims.f1_width == 2048
     w = hw.custom("pair", lengths, dims, n_layers=2, seed=417)
+    ref = O.stack_fwd(w.X, w.offsets, w.timestamps, w.weights, dims)
+    X = w.X.astype(np.float64)
+    out = {}
+    try:
+        for p in (0, 2):
+            B.hstu_set_option("gemm_pair", p)
+            Y, _, _ = run_stack(w)
+            out[p] = Y
+            e, ed = relerr(Y, ref), rmserr(Y - X, ref - X)
+            print("gemm_pair", p, e, ed)
+            assert e <= TOL[hw.BF16] and ed <= TOL[hw.BF16], (p, e, ed)
+    finally:
+        B.hstu_set_option("gemm_pair", 1)
+    assert np.array_equal(out[0], out[2])
+
+
+def test_gemm_pair_default_at_d1024_is_bitwise_single_cta():
+    """At d_model = 1024 the default (gemm_pair = 1) runs f1 on CTA pairs:
+    within the oracle's bound on a ragged layer of 2,700 rows (f1 width 4096,
+    256-column tiles) and bitwise equal to single CTAs (gemm_pair = 0)."""
+    from hstu_sequential_transducer_layer_b200 import binding as B
+    dims = hw.LayerDims(1024, 8, 128, 128, 128, 128, 4, 2, 1e-6, hw.BF16)
+    lengths = [700, 129, 1, 1024, 846]
+    assert sum(lengths) == 2700 and dims.f1_width == 4096
+    w = hw.custom("pair1024", lengths, dims, n_layers=1, seed=418)
     ref = O.stack_fwd(w.X, w.offsets, w.timestamps, w.weights, dims)
     X = w.X.astype(np.float64)
     out = {}
