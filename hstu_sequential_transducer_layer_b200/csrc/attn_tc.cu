@@ -452,6 +452,22 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const float* Rp = a.rab_pos + (size_t)w.head * a.Np;
       const float* Rt = a.rab_time + (size_t)w.head * a.Nt;
       const int t_i = (MODE == MODE_SELF) ? 0 : a.t_req_rel[w.b];
+      // Candidate mode: history time of this lane's column of KV tile jt, and
+      // the halved bias of that column from it.
+      auto cand_trel = [&](int jt) -> int {
+        const int jc = jt * 128 + g * 32 + lane;
+        return jc < n_kv ? a.t_rel[kv0 + jc] : 0;
+      };
+      auto cand_bias = [&](int jt, int trel) -> float {
+        const int jc = jt * 128 + g * 32 + lane;
+        float bias = 0.f;
+        if (jc < n_kv) {
+          const int gap = max(t_i - trel, 0);
+          bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
+                 __ldg(Rt + log_bucket(gap, a.St, a.Nt));
+        }
+        return 0.5f * bias;
+      };
       // Bias inputs of KV tile jt into window buffer `buf` (and, causal mode,
       // the tile's time-bucket words into bwn).  Causal mode: the warp's
       // 32 x 32 block spans the 63 distances base .. base + 62.
@@ -472,18 +488,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             }
           }
         } else {
-          const int jc = jt * 128 + g * 32 + lane;
-          float bias = 0.f;
-          if (jc < n_kv) {
-            const int gap = max(t_i - a.t_rel[kv0 + jc], 0);
-            bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
-                   __ldg(Rt + log_bucket(gap, a.St, a.Nt));
-          }
-          win[lane] = 0.5f * bias;
+          win[lane] = cand_bias(jt, cand_trel(jt));
         }
       };
       uint32_t bw[8], bwn[8];
       if (w.nkv > 0) prep(0, 0, bw);
+      // candidate mode: the next tile's bias is looked up while this tile
+      // computes and stored after it, from history times read a tile earlier
+      int tr_n = (MODE == MODE_CAND && w.nkv > 1) ? cand_trel(1) : 0;
       bool alive = true;
       for (int j = 0; j < w.nkv; ++j) {
         __syncwarp();  // this tile's window is written; the one before it is free
@@ -498,7 +510,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         uint32_t sr[32];
         tmem_ld32(tmem + sb * 128 + g * 32 + lane_base, sr);
         // fetch the next tile's bias inputs while this tile computes
-        if (j + 1 < w.nkv) prep(j + 1, (j + 1) & 1, bwn);
+        float nb = 0.f;
+        if (j + 1 < w.nkv) {
+          if (MODE == MODE_SELF) {
+            prep(j + 1, (j + 1) & 1, bwn);
+          } else {
+            nb = cand_bias(j + 1, tr_n);
+            if (j + 2 < w.nkv) tr_n = cand_trel(j + 2);
+          }
+        }
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -530,6 +550,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             if (c + 1 >= limit) p1 = 0.f;
             pk[c >> 1] = pack_f16x2_sat(p0, p1);
           }
+          if (j + 1 < w.nkv) win2[((j + 1) & 1) * 64 + lane] = nb;
         }
 #pragma unroll
         for (int m = 0; m < 8; ++m) bw[m] = bwn[m];
