@@ -292,10 +292,13 @@ DEVI void cluster_sync_all() {
 DEVI void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
-// Arrive on an mbarrier of either CTA of the cluster.
+// Arrive on an mbarrier of either CTA of the cluster.  CTA-scope release:
+// what the waiter needs ordered is this thread's tensor-memory reads, which
+// tcgen05.wait::ld has completed and tcgen05.fence::before_thread_sync orders
+// before the arrive; a cluster-scope release would add a memory barrier that
+// waits for all of the thread's outstanding memory operations.
 DEVI void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Bounded wait, single thread, with cluster-scope acquire (arrivals that come
 // from the peer CTA's threads).
