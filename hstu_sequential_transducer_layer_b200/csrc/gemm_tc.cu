@@ -23,7 +23,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <atomic>
+#include <map>
+#include <mutex>
 
 #include "ptx.cuh"
 
@@ -946,9 +947,13 @@ static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb,
 // another to finish.
 template <int EPI>
 static int pair_capacity() {
-  static std::atomic<int> cached{-1};
-  int v = cached.load(std::memory_order_relaxed);
-  if (v >= 0) return v;
+  static std::mutex mu;
+  static std::map<int, int> cached;  // device -> clusters
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto it = cached.find(dev);
+  if (it != cached.end()) return it->second;
   auto kfn = k_gemm_pair<EPI>;
   int n = 0;
   if (ensure_smem_limit(reinterpret_cast<const void*>(kfn), PairCfg::SMEM) == cudaSuccess) {
@@ -964,11 +969,12 @@ static int pair_capacity() {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kfn), &cfg) !=
-        cudaSuccess)
+        cudaSuccess) {
       n = 0;
+      (void)cudaGetLastError();  // the failed query's error, not a launch's
+    }
   }
-  (void)cudaGetLastError();
-  cached.store(n, std::memory_order_relaxed);
+  cached[dev] = n;
   return n;
 }
 
