@@ -254,19 +254,35 @@ __global__ void __launch_bounds__(256)
     }
     __syncthreads();
     uint32_t* dst = tb + (size_t)t * kBucketTileWords;
+    // four buckets packed into a word by byte permutes (bucket k in byte k)
+    auto pack4 = [](uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+      return __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+    };
+    if (j < qt && row_ok) {
+      // below the diagonal every column of a valid row is in the past: no mask
+#pragma unroll 4
+      for (int u = 0; u < 16; ++u) {
+        const int c4 = (threadIdx.x >> 7) + 2 * u;
+        const int4 tj = *reinterpret_cast<const int4*>(s_tj + 4 * c4);
+        dst[c4 * 128 + r] = pack4(log_bucket_nb(max(ti - tj.x, 0), St, Nt),
+                                  log_bucket_nb(max(ti - tj.y, 0), St, Nt),
+                                  log_bucket_nb(max(ti - tj.z, 0), St, Nt),
+                                  log_bucket_nb(max(ti - tj.w, 0), St, Nt));
+      }
+      continue;
+    }
 #pragma unroll 4
     for (int u = 0; u < 16; ++u) {
       const int c4 = (threadIdx.x >> 7) + 2 * u;
       const int4 tj = *reinterpret_cast<const int4*>(s_tj + 4 * c4);
       const int tjk[4] = {tj.x, tj.y, tj.z, tj.w};
-      uint32_t word = 0;
+      uint32_t bk[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int jj = j * kTile + 4 * c4 + k;
-        const uint32_t bk = log_bucket_nb(max(ti - tjk[k], 0), St, Nt);
-        word |= (row_ok && jj <= i ? bk : 0u) << (8 * k);
+        bk[k] = row_ok && jj <= i ? log_bucket_nb(max(ti - tjk[k], 0), St, Nt) : 0u;
       }
-      dst[c4 * 128 + r] = word;
+      dst[c4 * 128 + r] = pack4(bk[0], bk[1], bk[2], bk[3]);
     }
   }
 }
