@@ -102,3 +102,21 @@ def test_mfalcon_workload_sampled_users():
         err = relerr(got[cs:ce], ref[cs:ce])
         print("mfalcon user", b, lens[b], err)
         assert err <= TOL[hw.BF16]
+
+
+def test_mfalcon_workload_pairs_bitwise():
+    """The full M-FALCON workload with f1 forced onto CTA pairs
+    (gemm_pair = 2; at d_model = 512 the default keeps single CTAs): every
+    score bitwise equal to the single-CTA run.  Covers the pair kernel with a
+    device-side row count (the candidate microbatches) and the history's
+    76,827 rows."""
+    from hstu_sequential_transducer_layer_b200 import binding as B
+    w = hw.mfalcon(0)
+    out = {}
+    try:
+        for p in (0, 2):
+            B.hstu_set_option("gemm_pair", p)
+            out[p], _ = run_rank(w)
+    finally:
+        B.hstu_set_option("gemm_pair", 1)
+    assert np.array_equal(out[0], out[2])
