@@ -1111,7 +1111,9 @@ def main():
                     help="1: LayerNorm * U formed inside f2's operand stage; 0: a separate "
                          "kernel; 2: by layer width (inside f2 when d_model <= 512)")
     ap.add_argument("--cpu-tokens", type=int, default=4000)
-    ap.add_argument("--ref-tokens", type=int, default=600)
+    ap.add_argument("--ref-tokens", type=int, default=2000,
+                    help="reference arm: whole users per step, drawn like the CPU baseline's, "
+                         "until this many tokens")
     ap.add_argument("--leg", default=None,
                     choices=["full_stack", "long_history", "single_layer", "mfalcon", "backward",
                              "comparator"],
