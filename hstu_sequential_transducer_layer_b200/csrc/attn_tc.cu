@@ -102,7 +102,8 @@ struct AttnCfg {
   static_assert(QS == 2 && KS <= 4 && VS <= 4, "barrier slots");
   static_assert(SMEM <= 232448, "shared memory per CTA");
   // TMEM columns: S0 | S1 (128 each; P_j, 128 fp16 per row packed in pairs,
-  // overwrites the first 64 columns of S_j once S_j is read), then O0 | O1.
+  // is written over S_j: the P of S columns 32g .. 32g + 31 over columns
+  // 32g .. 32g + 15, which only the P warp that read them touches), then O0 | O1.
   static constexpr uint32_t O_COL = 256;
 };
 
@@ -172,7 +173,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint64_t* p_full = bars + 10;     // [2]
   uint64_t* o_full = bars + 12;     // [2]
   uint64_t* o_free = bars + 14;     // [2]
-  uint64_t* rd = bars + 21;         // [4] per lane quarter: its P warps have read S
   uint64_t* drain = bars + 16;
   uint64_t* it_full = bars + 17;    // [2] item ring
   uint64_t* it_empty = bars + 19;   // [2]
@@ -211,7 +211,6 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       mbar_init(it_full + i, 1);
       mbar_init(it_empty + i, 3 + C::PW + C::EW);  // loader lanes, MMA thread, P and O warps
     }
-    for (int i = 0; i < 4; ++i) mbar_init(rd + i, C::PW / 4);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -325,9 +324,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         tc_fence_after();
         const uint32_t p_tmem = tmem + pb * 128;
         const uint32_t v_base = smem_u32(sV + vst * C::TILE);
+        // 16 KV rows per MMA = 8 packed P columns; the P of KV columns
+        // 32g .. 32g + 31 sits at TMEM columns 32g .. 32g + 15 of the buffer
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 16 KV rows per MMA = 8 packed P columns
-          tc_mma_f16_ts(tmem + C::O_COL + ob * D, p_tmem + kk * 8,
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_f16_ts(tmem + C::O_COL + ob * D, p_tmem + (kk >> 1) * 32 + (kk & 1) * 8,
                         sdesc_sw128(v_base + kk * 2048, 16384, 1024), IDESC_O,
                         (jj > 0 || kk > 0) ? 1u : 0u);
         tc_commit(v_empty + vst);
@@ -520,10 +521,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(rd + q);  // this warp's part of S_j is in registers
-        const uint32_t tile = scount++;
+        ++scount;
         // ---- P = SiLU(S + bias), masked, fp16
         uint32_t pk[16];
         // window and time table by shared-space loads: element c of this
@@ -554,14 +552,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
 #pragma unroll
         for (int m = 0; m < 8; ++m) bw[m] = bwn[m];
-        // ---- write P over S_j: this warp's 32 rows, 32 fp16 (16 packed columns),
-        // once all four P warps of the lane quarter have read their part of S_j
-        if (!mbar_wait_warp(rd + q, tile & 1, ab, a.status)) {
-          alive = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st16(tmem + sb * 128 + g * 16 + lane_base, pk);
+        // ---- write P over the first half of this warp's own 32 columns of
+        // S_j (already in registers; no other warp reads them): 32 rows, 32
+        // fp16 as 16 packed columns
+        tmem_st16(tmem + sb * 128 + g * 32 + lane_base, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
