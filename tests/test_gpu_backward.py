@@ -116,3 +116,25 @@ def test_bwd_no_rows_gives_zero_gradients():
     assert r.bwd_status() == 0 and dX.shape == (0, 128)
     for k in GRAD_KEYS:
         assert float(grads[0][k].abs().max()) == 0.0, k
+
+
+def test_bwd_pairs_bitwise():
+    """The backward call's forward keeps f1's pre-activation next to G; with
+    f1 forced onto CTA pairs (gemm_pair = 2) on a case whose f1 takes
+    256-column tiles (f1 width 2048, 5,000 rows), every gradient and dX is
+    bitwise the single-CTA run's."""
+    from hstu_sequential_transducer_layer_b200 import binding as B
+    dims = hw.LayerDims(512, 4, 128, 128, 128, 128, 4, 2, 1e-6, hw.BF16)
+    w = hw.custom("bwdpair", [777, 1024, 513, 1, 1000, 1685], dims, n_layers=2, seed=87)
+    dY = hw.round_to_bf16(np.random.default_rng(88).standard_normal(w.X.shape).astype(np.float32))
+    out = {}
+    try:
+        for p in (0, 2):
+            B.hstu_set_option("gemm_pair", p)
+            out[p] = _run_bwd(w, dY)
+    finally:
+        B.hstu_set_option("gemm_pair", 1)
+    assert np.array_equal(out[0][0], out[2][0])
+    for layer in range(2):
+        for k in GRAD_KEYS:
+            assert np.array_equal(out[0][1][layer][k], out[2][1][layer][k]), (layer, k)
