@@ -94,3 +94,26 @@ def test_bad_offsets_set_status():
     off = torch.tensor([0, 30, 20, 50], dtype=torch.int64, device="cuda")
     r.layer(off, X, 64)
     assert r.status() == 5
+
+
+def test_pairs_bitwise():
+    """The comparator layer with its QKV (plain bias) and FFN (SiLU)
+    projections forced onto CTA pairs (gemm_pair = 2; at d = 512 the default
+    keeps single CTAs): bitwise the single-CTA result, on 7,000 ragged rows
+    (both projections take 256-column tiles)."""
+    from hstu_sequential_transducer_layer_b200 import binding as B
+    lengths = [1500, 1, 2048, 700, 2751]
+    rng = np.random.default_rng(64)
+    offsets = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    d, h, ff = 512, 8, 2048
+    X = hw.round_to_bf16(rng.standard_normal((int(offsets[-1]), d)).astype(np.float32))
+    w = hw.transformer_weights(64, d, ff)
+    out = {}
+    try:
+        for p in (0, 2):
+            B.hstu_set_option("gemm_pair", p)
+            st, out[p] = _run(X, offsets, d, h, ff, w)
+            assert st == 0
+    finally:
+        B.hstu_set_option("gemm_pair", 1)
+    assert np.array_equal(out[0], out[2])
