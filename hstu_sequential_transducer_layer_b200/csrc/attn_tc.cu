@@ -124,39 +124,38 @@ DEVI float lds_f32_at(uint32_t base) {
 }
 
 // Causal P for columns C and C+1 of this warp's 32 x 32 block, then the next
-// pair: P = SiLU(S + position bias + time bias), zero where the column is past
-// `lim` (MASK).  wa: shared address of the lane's window entry (column c takes
-// entry 31 - c after it); ra: shared address of the head's halved time table;
-// bw: the block's bucket bytes, 4 columns per word.
-template <int C, bool MASK>
+// pair: P = SiLU(S + position bias + time bias).  wa: shared address of the
+// lane's window entry (column c takes entry 31 - c after it); ra: shared
+// address of the head's halved time table; bw: the block's bucket bytes, 4
+// columns per word.  The causal mask is in the window: a future column's
+// entry is kMaskedHalfBias, for which SiLU gives exactly zero.
+template <int C>
 struct PPair {
   static DEVI void run(uint32_t (&pk)[16], const uint32_t (&sr)[32], const uint32_t (&bw)[8],
-                       uint32_t wa, uint32_t ra, int lim) {
+                       uint32_t wa, uint32_t ra) {
     const uint32_t b0 = __byte_perm(bw[C >> 2], 0u, 0x4440u | (C & 3));
     const uint32_t b1 = __byte_perm(bw[C >> 2], 0u, 0x4440u | ((C + 1) & 3));
     float p0 = silu_half(fmaf(__uint_as_float(sr[C]), 0.5f, lds_f32_at<4 * (31 - C)>(wa)) +
                          lds_f32(ra + 4u * b0));
     float p1 = silu_half(fmaf(__uint_as_float(sr[C + 1]), 0.5f, lds_f32_at<4 * (30 - C)>(wa)) +
                          lds_f32(ra + 4u * b1));
-    if (MASK) {
-      if (C > lim) p0 = 0.f;
-      if (C + 1 > lim) p1 = 0.f;
-    }
     pk[C >> 1] = pack_f16x2_sat(p0, p1);
-    PPair<C + 2, MASK>::run(pk, sr, bw, wa, ra, lim);
+    PPair<C + 2>::run(pk, sr, bw, wa, ra);
   }
 };
-template <bool MASK>
-struct PPair<32, MASK> {
+template <>
+struct PPair<32> {
   static DEVI void run(uint32_t (&)[16], const uint32_t (&)[32], const uint32_t (&)[8], uint32_t,
-                       uint32_t, int) {}
+                       uint32_t) {}
 };
 
-// SPLIT (causal mode): a separate P loop without masks for tiles below the
-// diagonal (faster per element; for batches of short users, where every
-// other tile is a diagonal one, a single masked loop -- half the code -- is
-// faster).
-template <int D, int MODE, bool SPLIT>
+// The window entry of a distance j - i > 0 (a future column): with it, y =
+// s/2 + entry + time bias is below -1e29 for any finite score, tanh.approx(y)
+// is exactly -1, and SiLU's y + y tanh(y) is exactly +0 -- the masked P,
+// with no per-element select.
+constexpr float kMaskedHalfBias = -1e30f;
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
               const __grid_constant__ CUtensorMap tmO, const AttnDev a) {
@@ -485,7 +484,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             const int k = lane + 32 * u;
             if (k < 63) {
               const int dist = base + k;
-              win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np)) : 0.f;
+              win[k] = dist >= 0 ? 0.5f * __ldg(Rp + log_bucket(dist, a.Sp, a.Np))
+                                 : kMaskedHalfBias;
             }
           }
         } else {
@@ -529,14 +529,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const uint32_t wa = smem_u32(win) + 4u * (uint32_t)lane;
         const uint32_t ra = smem_u32(rt);
         if (MODE == MODE_SELF) {
-          if (!SPLIT || j == w.qt) {
-            // the causal mask j > i on the diagonal tile; no column reaches
-            // the threshold on the others
-            const int lim = (j == w.qt) ? r - g * 32 : 1 << 20;
-            PPair<0, true>::run(pk, sr, bw, wa, ra, lim);
-          } else {
-            PPair<0, false>::run(pk, sr, bw, wa, ra, 0);
-          }
+          PPair<0>::run(pk, sr, bw, wa, ra);  // (the diagonal tile's mask is in the window)
         } else {
           const int limit = n_kv - j * 128 - g * 32;
           const uint32_t wc = smem_u32(win);
@@ -781,12 +774,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   }
 }
 
-template <int D, int MODE, bool SPLIT = true>
+template <int D, int MODE>
 static cudaError_t launch_attn_inst(const CUtensorMap& tq, const CUtensorMap& tkv,
                                     const CUtensorMap& to, const AttnDev& ad, int grid,
                                     cudaStream_t s) {
   using C = AttnCfg<D>;
-  auto kfn = k_attn_tc<D, MODE, SPLIT>;
+  auto kfn = k_attn_tc<D, MODE>;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM);
   if (e != cudaSuccess) return e;
   kfn<<<grid, C::THREADS, C::SMEM, s>>>(tq, tkv, to, ad);
@@ -846,16 +839,9 @@ cudaError_t launch_attn_tc(const AttnCall& c, cudaStream_t s) {
   take_wait_test(&ad.wait_limit_us, &ad.inject_stall);
   const int grid = (int)std::min<int64_t>(c.item_cap, num_sms());
   LaunchScope ls(c.mode == MODE_SELF ? K_ATTN : K_ATTN_CAND, s);
-  if (c.mode == MODE_SELF) {
-    // users of 1024 rows or more on average: most tiles lie below the
-    // diagonal, so the unmasked loop pays for its code
-    const bool split = c.q_rows_cap >= 1024 * std::max<int64_t>(c.B, 1);
-    if (split)
-      return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF, true>(tq, tkv, to, ad, grid, s)
-                         : launch_attn_inst<128, MODE_SELF, true>(tq, tkv, to, ad, grid, s);
-    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF, false>(tq, tkv, to, ad, grid, s)
-                       : launch_attn_inst<128, MODE_SELF, false>(tq, tkv, to, ad, grid, s);
-  }
+  if (c.mode == MODE_SELF)
+    return c.dqk == 64 ? launch_attn_inst<64, MODE_SELF>(tq, tkv, to, ad, grid, s)
+                       : launch_attn_inst<128, MODE_SELF>(tq, tkv, to, ad, grid, s);
   return c.dqk == 64 ? launch_attn_inst<64, MODE_CAND>(tq, tkv, to, ad, grid, s)
                      : launch_attn_inst<128, MODE_CAND>(tq, tkv, to, ad, grid, s);
 }
