@@ -458,15 +458,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int jc = jt * 128 + g * 32 + lane;
         return jc < n_kv ? a.t_rel[kv0 + jc] : 0;
       };
+      // A column past the history (the last tile's ragged end) gets
+      // kMaskedHalfBias: its P is exactly zero.
       auto cand_bias = [&](int jt, int trel) -> float {
         const int jc = jt * 128 + g * 32 + lane;
-        float bias = 0.f;
-        if (jc < n_kv) {
-          const int gap = max(t_i - trel, 0);
-          bias = __ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
-                 __ldg(Rt + log_bucket(gap, a.St, a.Nt));
-        }
-        return 0.5f * bias;
+        if (jc >= n_kv) return kMaskedHalfBias;
+        const int gap = max(t_i - trel, 0);
+        return 0.5f * (__ldg(Rp + log_bucket(n_kv - jc, a.Sp, a.Np)) +
+                       __ldg(Rt + log_bucket(gap, a.St, a.Nt)));
       };
       // Bias inputs of KV tile jt into window buffer `buf` (and, causal mode,
       // the tile's time-bucket words into bwn).  Causal mode: the warp's
@@ -531,14 +530,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         if (MODE == MODE_SELF) {
           PPair<0>::run(pk, sr, bw, wa, ra);  // (the diagonal tile's mask is in the window)
         } else {
-          const int limit = n_kv - j * 128 - g * 32;
+          // (columns past the history carry kMaskedHalfBias in the window)
           const uint32_t wc = smem_u32(win);
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wc + 4u * c)));
-            float p1 = silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, lds_f32(wc + 4u * (c + 1))));
-            if (c >= limit) p0 = 0.f;
-            if (c + 1 >= limit) p1 = 0.f;
+            const float p0 = silu_half(fmaf(__uint_as_float(sr[c]), 0.5f, lds_f32(wc + 4u * c)));
+            const float p1 =
+                silu_half(fmaf(__uint_as_float(sr[c + 1]), 0.5f, lds_f32(wc + 4u * (c + 1))));
             pk[c >> 1] = pack_f16x2_sat(p0, p1);
           }
           if (j + 1 < w.nkv) win2[((j + 1) & 1) * 64 + lane] = nb;
