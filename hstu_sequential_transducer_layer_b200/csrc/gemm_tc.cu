@@ -682,26 +682,34 @@ static cudaError_t launch_one(const CUtensorMap& ta, const CUtensorMap& tb,
 //           name them by cluster address); its MMA commits arrive on the
 //           `empty` and `tfull` barriers of both CTAs (multicast commit);
 //           both CTAs' epilogue warps arrive on rank 0's `tempty`.
-// Only the plain-bias and SiLU epilogues (16-bit output, optionally the SiLU
-// pre-activation), K-major operands.  Every wait is bounded; the two CTAs
-// leave together through a bounded exchange of arrivals.
+// The plain-bias and SiLU epilogues (16-bit output, optionally the SiLU
+// pre-activation) and the residual one with a 16-bit residual and output
+// only (2 KB output and residual buffers per epilogue warp; each warp's next
+// residual chunk arrives by TMA while the current one is finished);
+// K-major operands.  Every wait is bounded; the two CTAs leave together
+// through a bounded exchange of arrivals.
 constexpr int kPairStages = 6;
+template <int EPI>
 struct PairCfg {
+  static constexpr bool RES = EPI == EPI_RESID;
   static constexpr uint32_t A_BYTES = 128 * 64 * 2;  // this CTA's 128 rows of A
   static constexpr uint32_t B_BYTES = 128 * 64 * 2;  // this CTA's 128 rows of W
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t BUF = RES ? 2048 : kStageBuf;  // per epilogue warp
   static constexpr uint32_t OUT_OFF = kPairStages * STAGE_BYTES;
-  static constexpr uint32_t BAR_OFF = OUT_OFF + (kEpiThreads / 32) * kStageBuf;
+  static constexpr uint32_t RES_OFF = OUT_OFF + (kEpiThreads / 32) * BUF;
+  static constexpr uint32_t BAR_OFF = RES_OFF + (RES ? (kEpiThreads / 32) * 2048 : 0);
   static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
   static constexpr int THREADS = 64 + kEpiThreads;
 };
 
 template <int EPI>
-__global__ void __launch_bounds__(PairCfg::THREADS, 1)
+__global__ void __launch_bounds__(PairCfg<EPI>::THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmO16,
-                const __grid_constant__ CUtensorMap tmO32, const GemmDev g) {
-  using C = PairCfg;
+                const __grid_constant__ CUtensorMap tmO32,
+                const __grid_constant__ CUtensorMap tmR, const GemmDev g) {
+  using C = PairCfg<EPI>;
   constexpr int S = kPairStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -712,7 +720,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   uint64_t* tempty = tfull + 2;                                     // [2], rank 0's in use
   uint64_t* drain = tempty + 2;
   uint64_t* pdone = drain + 1;  // one arrival from each CTA at the end
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pdone + 1);
+  uint64_t* rbar = pdone + 1;   // [8] residual chunk landed (per epilogue warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 8);
   AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
   uint32_t* s_go = reinterpret_cast<uint32_t*>(ab + 1);
 
@@ -731,6 +740,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     mbar_init(tempty + 1, 2 * (kEpiThreads / 32));
     mbar_init(drain, 1);
     mbar_init(pdone, 2);
+    for (int i = 0; i < 8; ++i) mbar_init(rbar + i, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -843,9 +853,26 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     const int q = warp & 3;            // TMEM lane quarter this warp may read
     const int part = (warp - 2) >> 2;  // which 128 of the 256 columns
     constexpr int CH = 4;              // 32-column chunks per warp
-    uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * kStageBuf;
+    uint8_t* stage = smem + C::OUT_OFF + (warp - 2) * C::BUF;
     int local = 0, nchunk = 0;
-    for (int t = pair; t < tiles; t += npairs) {
+    // residual: lane 0 has TMA bring the next 32 x 32 chunk into the warp's
+    // buffer while the current one is finished
+    uint8_t* rbuf = smem + C::RES_OFF + (warp - 2) * 2048;
+    uint64_t* rb = rbar + (warp - 2);
+    uint32_t rpar = 0;
+    bool r_pending = false;
+    auto r_issue = [&](int t_, int c_) {
+      const int mt_ = t_ / n_tiles, nt_ = t_ - (t_ / n_tiles) * n_tiles;
+      mbar_arrive_expect_tx(rb, 2048u);
+      tma_load_2d(rbuf, &tmR, g.n_off + nt_ * 256 + part * 128 + c_ * 32,
+                  mt_ * 256 + (int)rank * 128 + q * 32, rb);
+    };
+    if (C::RES && lane == 0 && pair < tiles) {
+      r_issue(pair, 0);
+      r_pending = true;
+    }
+    bool alive = true;
+    for (int t = pair; t < tiles && alive; t += npairs) {
       const int mt = t / n_tiles, nt = t - (t / n_tiles) * n_tiles;
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
@@ -861,7 +888,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
       const int64_t row = (int64_t)y0 + lane;
       const bool valid = row < Mrows;
       const uint32_t tbase = tmem + acc * 256 + part * 128 + ((uint32_t)(q * 32) << 16);
-      uint32_t ra[32], rb[32];
+      uint32_t ra[32], rbv[32];
       tmem_ld32(tbase, ra);
       tmem_ld_wait();
 #pragma unroll
@@ -875,21 +902,53 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             else bb[i] = bv;
           }
           if (c & 1) tmem_ld32(tbase + (c + 1) * 32, ra);
-          else tmem_ld32(tbase + (c + 1) * 32, rb);
+          else tmem_ld32(tbase + (c + 1) * 32, rbv);
+        }
+        const uint8_t* rsm = nullptr;
+        if (C::RES) {
+          if (!mbar_wait_warp(rb, rpar, ab, g.status)) {
+            if (c + 1 < CH) tmem_ld_wait();
+            alive = false;
+            break;
+          }
+          rpar ^= 1;
+          rsm = rbuf;
         }
         bool stored;
+        const int par = C::RES ? -1 : (nchunk & 1);
         if (c & 1)
-          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rb, bb, stage,
-                                   nchunk & 1, nullptr);
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, rbv, bb,
+                                   stage, par, rsm);
         else
-          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba, stage,
-                                   nchunk & 1, nullptr);
+          stored = gemm_chunk<EPI>(g, &tmO16, &tmO32, row, valid, col0 + c * 32, y0, ra, ba,
+                                   stage, par, rsm);
         nchunk += stored ? 1 : 0;
+        if (C::RES) {
+          __syncwarp();  // every lane has read the residual chunk
+          if (lane == 0) {
+            r_pending = false;
+            int tn = t, cn = c + 1;
+            if (cn == CH) {
+              tn = t + npairs;
+              cn = 0;
+            }
+            if (tn < tiles) {
+              fence_proxy_async_smem();
+              r_issue(tn, cn);
+              r_pending = true;
+            }
+          }
+        }
         if (c + 1 < CH) tmem_ld_wait();
       }
+      if (!alive) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(tempty + acc), 0));
+    }
+    if (lane == 0 && r_pending) {  // a residual load still in flight must land first
+      AbortState tmp{0, kWaitLimitUs};
+      mbar_wait(rb, rpar, &tmp, nullptr);
     }
     if (lane == 0) bulk_wait_all();  // every store has landed before the CTA exits
     __syncwarp();
@@ -920,15 +979,17 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
 template <int EPI>
 static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb,
                                const CUtensorMap& to16, const CUtensorMap& to32,
-                               const GemmDev& gd, int pairs, cudaStream_t s) {
-  static_assert(PairCfg::SMEM <= 232448, "shared memory per CTA");
+                               const CUtensorMap& tr, const GemmDev& gd, int pairs,
+                               cudaStream_t s) {
+  using C = PairCfg<EPI>;
+  static_assert(C::SMEM <= 232448, "shared memory per CTA");
   auto kfn = k_gemm_pair<EPI>;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), PairCfg::SMEM);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = PairCfg::SMEM;
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -937,7 +998,7 @@ static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb,
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kfn, ta, tb, to16, to32, gd);
+  e = cudaLaunchKernelEx(&cfg, kfn, ta, tb, to16, to32, tr, gd);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -954,13 +1015,14 @@ static int pair_capacity() {
   std::lock_guard<std::mutex> lk(mu);
   const auto it = cached.find(dev);
   if (it != cached.end()) return it->second;
+  using C = PairCfg<EPI>;
   auto kfn = k_gemm_pair<EPI>;
   int n = 0;
-  if (ensure_smem_limit(reinterpret_cast<const void*>(kfn), PairCfg::SMEM) == cudaSuccess) {
+  if (ensure_smem_limit(reinterpret_cast<const void*>(kfn), C::SMEM) == cudaSuccess) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(2 * 74, 1, 1);
-    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = PairCfg::SMEM;
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 2;
@@ -1075,9 +1137,14 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
                                          c.status, s);
     if (e != cudaSuccess) return e;
   }
-  // SiLU and plain-bias products with 256-column tiles: CTA pairs
-  if (!lna && (c.epi == EPI_SILU || c.epi == EPI_BIAS) && BN == 256 && gemm_pair_for(c.K)) {
-    const int cap = c.epi == EPI_SILU ? pair_capacity<EPI_SILU>() : pair_capacity<EPI_BIAS>();
+  // SiLU, plain-bias and (16-bit residual and output only) residual products
+  // with 256-column tiles: CTA pairs
+  const bool pair_res = c.epi == EPI_RESID && c.resid_kind != RESID_F32 && c.out32 == nullptr;
+  if (!lna && (c.epi == EPI_SILU || c.epi == EPI_BIAS || pair_res) && BN == 256 &&
+      gemm_pair_for(c.K)) {
+    const int cap = c.epi == EPI_SILU   ? pair_capacity<EPI_SILU>()
+                    : c.epi == EPI_BIAS ? pair_capacity<EPI_BIAS>()
+                                        : pair_capacity<EPI_RESID>();
     if (cap > 0) {
       CUtensorMap tb2;  // W in 128-row boxes: each CTA of a pair brings half a tile
       if (!encode_tmap_2d(&tb2, c.W, (uint64_t)(c.n_off + c.N), (uint64_t)c.K,
@@ -1086,8 +1153,9 @@ cudaError_t launch_gemm_tc(const GemmCall& c, cudaStream_t s, int kernel_id) {
       const int64_t ptiles = ((c.M_cap + 255) / 256) * (c.N / 256);
       const int pairs = (int)std::min<int64_t>(ptiles, cap);
       LaunchScope ls(kernel_id, s);
-      if (c.epi == EPI_SILU) return launch_pair<EPI_SILU>(ta, tb2, to16, to32, gd, pairs, s);
-      return launch_pair<EPI_BIAS>(ta, tb2, to16, to32, gd, pairs, s);
+      if (c.epi == EPI_SILU) return launch_pair<EPI_SILU>(ta, tb2, to16, to32, tr, gd, pairs, s);
+      if (c.epi == EPI_BIAS) return launch_pair<EPI_BIAS>(ta, tb2, to16, to32, tr, gd, pairs, s);
+      return launch_pair<EPI_RESID>(ta, tb2, to16, to32, tr, gd, pairs, s);
     }
   }
   LaunchScope ls(kernel_id, s);
