@@ -436,11 +436,12 @@ hstu_status hstu_debug_wait_test(uint32_t wait_limit_us, int32_t inject_stall);
  * a separate kernel that f2 then reads, 2 (default) chooses per layer: inside
  * f2 when d_model <= 512 (f2 then has at most two 256-column output tiles,
  * each of which forms Z again), the separate kernel otherwise.  All give the
- * same layer within the bf16 bound.  "gemm_pair": where the input projection
- * f1 (SiLU) takes 256-column output tiles, 1 (default) runs it on clusters of
- * two CTAs sharing each 256 x 256 tile through the pair MMA when its inner
- * dimension (d_model) is at least 1024, 2 does so at any inner dimension, 0
- * never; all give bitwise the same result.  Returns HSTU_ERR_INVALID_ARG for
+ * same layer within the bf16 bound.  "gemm_pair": where a projection (f1 with
+ * SiLU, f2 with its 16-bit residual, a plain-bias product) takes 256-column
+ * output tiles, 1 (default) runs it on clusters of two CTAs sharing each
+ * 256 x 256 tile through the pair MMA when its inner dimension is at least
+ * 1024, 2 does so at any inner dimension, 0 never; all give bitwise the same
+ * result.  Returns HSTU_ERR_INVALID_ARG for
  * an unknown name or value. */
 hstu_status hstu_set_option(const char* name, int64_t value);
 
