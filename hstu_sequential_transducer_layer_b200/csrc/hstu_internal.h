@@ -299,8 +299,9 @@ cudaError_t launch_ln_gate_norm(const void* xn, const float* stats, const void* 
 // Whether f2 forms LayerNorm * U in its operand stage (else a separate
 // kernel writes Z first) for a layer of this width; hstu_set_option("ln_fusion", ...).
 bool ln_fusion_for(int d_model);
-// Whether SiLU and plain-bias products with 256-column tiles and inner
-// dimension K run on CTA pairs (the pair MMA); hstu_set_option("gemm_pair", ...).
+// Whether products with 256-column tiles and inner dimension K (SiLU, plain
+// bias, 16-bit residual) run on CTA pairs (the pair MMA);
+// hstu_set_option("gemm_pair", ...).
 bool gemm_pair_for(int K);
 
 // bf16 -> fp16 (round to nearest, saturating at +-65504) of up to

@@ -97,7 +97,7 @@ std::atomic<int> g_gemm_pair{1};
 // 1 (automatic): on pairs when K >= 1024.  With shorter K the SiLU epilogue
 // of a tile takes about as long as its MMAs, and the pair, whose MMAs wait
 // for both CTAs' epilogues, is slower than single CTAs (measured at K = 512:
-// f1 8 % slower; at K = 1024: 2-3 % faster).
+// f1 8 % slower; at K = 1024: f1 2-5 % faster, f2 15-20 %).
 bool gemm_pair_for(int K) {
   const int m = g_gemm_pair.load(std::memory_order_relaxed);
   return m == 2 || (m == 1 && K >= 1024);
